@@ -1,0 +1,483 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the CSA/HCA compressed-attention path on B200.
+
+One step = one decode token for every request of a CSA layer:
+  csla_compress_append (T=1) -> csla_indexer_scores -> csla_topk_select ->
+  csla_csa_attend.
+Workload (default): 8 requests at 131072-token context, m=4 (32768
+compressed entries each), 64 query heads, head_dim 512 (448 fp8 + 64 bf16
+RoPE dims), dc=1024 -> 16 index heads of 128, top-k 512, window 128.
+An HCA layer (4 requests at 1,048,576 tokens, m'=128) is measured after it
+and reported in the same JSON line under "hca_decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N>1 runs under torchrun: every rank serves its own 8 requests (weak scaling,
+no collective on the data path); the step time is the max over ranks.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA/HCA decode tokens/s and achieved HBM GB/s vs roofline, 1×B200"
+UNIT = "tokens/s"
+CSA = dict(B=8, L=131072, m=4, H=64, D=512, HI=16, dI=128, dc=1024, k=512, n_win=128)
+HCA = dict(B=4, L=1048576, m=128, H=64, D=512, n_win=128)
+CHUNK = 16384          # tokens per compress call while building the caches
+FLUSH_BYTES = 512 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-hca", action="store_true", help="skip the HCA layer measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--variant", type=int, default=0, help="attention variant: 0 auto, 1 saturated, 2 starved")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm = [float(r[1]) for r in self.rows if len(r) > 2 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if len(r) > 2 and r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in self.rows:
+            for i, n in enumerate(names):
+                if len(r) > 5 + i and r[5 + i].lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload build
+def build_layer(shape_kw, n_req, L0, seed, rank, device):
+    """Caches of n_req requests after appending L0 tokens each, through
+    csla_compress_append on raw streams generated on the device."""
+    import torch
+    from compressed_sparse_long_append_b200 import csla as C
+    from compressed_sparse_long_append_b200.layer import CompressParams, LayerBuffers, LayerShape
+    from csla_synth import permutation, normal
+    from csla_synth import torch_gen
+
+    sh = LayerShape(m=shape_kw["m"], D=shape_kw["D"], H=shape_kw["H"], HI=shape_kw.get("HI", 16),
+                    dI=shape_kw.get("dI", 128), dc=shape_kw.get("dc", 1024), n_win=shape_kw["n_win"])
+    L_cap = shape_kw["L"]
+    pages_per = -(-L_cap // 128)
+    n_pages = n_req * pages_per
+    lb = LayerBuffers(sh, n_req, n_pages, pages_per, device)
+    perm = permutation(seed, "pages/%d" % rank, n_pages).astype("int32").reshape(n_req, pages_per)
+    lb.block_table.copy_(torch.from_numpy(perm))
+    D, dI, m = sh.D, sh.dI, sh.m
+    g = lambda name, shp, std=1.0: torch.as_tensor(normal(seed, name, shp, std=std), dtype=torch.float32)
+    cp = CompressParams(1.0 + 0.1 * g("gamma_kv", (D,)), g("wg", (D,), 1.0 / D ** 0.5), g("gb", (m,)),
+                        g("wgi", (dI,), 1.0 / dI ** 0.5) if sh.is_csa else None,
+                        g("gbi", (m,)) if sh.is_csa else None, device)
+    for r in range(n_req):
+        slots = torch.tensor([r], dtype=torch.int32, device=device)
+        for a in range(0, L0, CHUNK):
+            b = min(L0, a + CHUNK)
+            kv = torch_gen.normal(seed, "kv/%d/%d" % (rank, r), (b - a, D), start=a * D, device=device) \
+                .to(torch.bfloat16)
+            ki = torch_gen.normal(seed, "idx/%d/%d" % (rank, r), (b - a, dI), start=a * dI, device=device) \
+                .to(torch.bfloat16) if sh.is_csa else None
+            C.csla_compress_append(lb.cfg(), lb.state(), lb.cache(), slots, 1, b - a, kv, ki, C.CSLA_BF16,
+                                   cp.struct())
+    torch.cuda.synchronize()
+    params = {"sink": g("sink", (sh.H,)).to(device), "gamma_q": (1.0 + 0.1 * g("gamma_q", (D,))).to(device)}
+    if sh.is_csa:
+        params["W_iq"] = torch_gen.normal(seed, "W_iq", (sh.HI * dI, sh.dc), device=device,
+                                          std=1.0 / sh.dc ** 0.5).to(torch.bfloat16)
+    return lb, cp, params
+
+
+def step_inputs(shape_kw, n_req, n_steps, seed, rank, device):
+    """Per-step inputs for all steps, device-resident, plus pinned host copies."""
+    import torch
+    from csla_synth import torch_gen
+    B, H, D = n_req, shape_kw["H"], shape_kw["D"]
+    out = []
+    for s in range(n_steps):
+        d = {"q": torch_gen.normal(seed, "q/%d/%d" % (rank, s), (B, H, D), device=device).to(torch.bfloat16),
+             "kv": torch_gen.normal(seed, "kvn/%d/%d" % (rank, s), (B, 1, D), device=device).to(torch.bfloat16)}
+        if shape_kw["m"] == 4:
+            d["kidx"] = torch_gen.normal(seed, "kin/%d/%d" % (rank, s), (B, 1, shape_kw["dI"]),
+                                         device=device).to(torch.bfloat16)
+            d["cq"] = torch_gen.normal(seed, "cq/%d/%d" % (rank, s), (B, shape_kw["dc"]), device=device) \
+                .to(torch.bfloat16)
+            d["head_w"] = torch_gen.normal(seed, "hw/%d/%d" % (rank, s), (B, shape_kw["HI"]), device=device) \
+                .to(torch.float32)
+        d["host"] = {k: v.cpu().pin_memory() for k, v in d.items()}
+        out.append(d)
+    return out
+
+
+class CsaStep:
+    def __init__(self, lb, cp, params, kw, variant, device):
+        import torch
+        from compressed_sparse_long_append_b200 import csla as C
+        self.C, self.lb, self.cp, self.p, self.kw, self.variant = C, lb, cp, params, kw, variant
+        B = kw["B"]
+        self.B = B
+        self.slots = torch.arange(B, dtype=torch.int32, device=device)
+        self.max_len = kw["L"]
+        self.stride = self.max_len // kw["m"]
+        self.scores = torch.zeros((B, self.stride), dtype=torch.float32, device=device)
+        self.idx = torch.zeros((B, kw["k"]), dtype=torch.int32, device=device)
+        self.out = torch.zeros((B, kw["H"], kw["D"]), dtype=torch.bfloat16, device=device)
+        cfg = lb.cfg()
+        self.wsi = C.csla_workspace_size(cfg, C.CSLA_OP_INDEXER, B, self.max_len)
+        self.wsa = C.csla_workspace_size(cfg, C.CSLA_OP_CSA_ATTEND, B, kw["k"])
+        self.ws_i = torch.zeros(self.wsi, dtype=torch.uint8, device=device)
+        self.ws_a = torch.zeros(self.wsa, dtype=torch.uint8, device=device)
+        self.cfg, self.st, self.cache, self.cps = cfg, lb.state(), lb.cache(), cp.struct()
+
+    def run(self, inp, ev=None):
+        C = self.C
+        rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
+        rec(0)
+        C.csla_compress_append(self.cfg, self.st, self.cache, self.slots, self.B, 1, inp["kv"], inp["kidx"],
+                               C.CSLA_BF16, self.cps)
+        rec(1)
+        C.csla_indexer_scores(self.cfg, self.st, self.cache, self.slots, self.B, self.max_len, inp["cq"],
+                              C.CSLA_BF16, self.p["W_iq"], C.CSLA_BF16, inp["head_w"], self.scores, self.stride,
+                              self.ws_i, self.wsi)
+        rec(2)
+        C.csla_topk_select(self.cfg, self.st, self.slots, self.B, self.max_len, self.scores, self.stride,
+                           self.kw["k"], self.idx)
+        rec(3)
+        C.csla_csa_attend(self.cfg, self.st, self.cache, self.slots, self.B, inp["q"], C.CSLA_BF16, self.idx,
+                          self.kw["k"], self.p["sink"], self.p["gamma_q"], self.out, C.CSLA_BF16, self.variant,
+                          self.ws_a, self.wsa)
+        rec(4)
+
+    def launches(self):
+        # compress, iq_project, indexer, topk, attend (+ combine when starved)
+        starved = self.variant == 2 or (self.variant == 0 and self.B < 148)
+        return 5 + (1 if starved else 0)
+
+
+class HcaStep:
+    def __init__(self, lb, cp, params, kw, variant, device):
+        import torch
+        from compressed_sparse_long_append_b200 import csla as C
+        self.C, self.lb, self.cp, self.p, self.kw, self.variant = C, lb, cp, params, kw, variant
+        B = kw["B"]
+        self.B = B
+        self.slots = torch.arange(B, dtype=torch.int32, device=device)
+        self.max_len = kw["L"]
+        self.out = torch.zeros((B, kw["H"], kw["D"]), dtype=torch.bfloat16, device=device)
+        cfg = lb.cfg()
+        self.wsa = C.csla_workspace_size(cfg, C.CSLA_OP_HCA_ATTEND, B, self.max_len)
+        self.ws_a = torch.zeros(self.wsa, dtype=torch.uint8, device=device)
+        self.cfg, self.st, self.cache, self.cps = cfg, lb.state(), lb.cache(), cp.struct()
+
+    def run(self, inp, ev=None):
+        C = self.C
+        rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
+        rec(0)
+        C.csla_compress_append(self.cfg, self.st, self.cache, self.slots, self.B, 1, inp["kv"], None,
+                               C.CSLA_BF16, self.cps)
+        rec(1)
+        C.csla_hca_attend(self.cfg, self.st, self.cache, self.slots, self.B, self.max_len, inp["q"], C.CSLA_BF16,
+                          self.p["sink"], self.p["gamma_q"], self.out, C.CSLA_BF16, self.variant, self.ws_a,
+                          self.wsa)
+        rec(2)
+
+
+def timed_steps(step, inputs, W, K, n_events, flush, e2e=False):
+    """W warm-up + K timed steps; L2 flushed before every step (outside the
+    timed events).  Returns per-step segment times (ms) [K][n_events-1] and
+    the whole-step times (ms)."""
+    import torch
+    segs, whole = [], []
+    for i in range(W + K):
+        inp = inputs[i]
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
+        if e2e:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            dev = {k: inp[k].copy_(inp["host"][k], non_blocking=True) for k in inp if k != "host"}
+            step.run(dev, ev)
+            out_h = step.out.to("cpu", non_blocking=True)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= W:
+                whole.append(e0.elapsed_time(e1))
+        else:
+            step.run(inp, ev)
+            torch.cuda.synchronize()
+            if i >= W:
+                segs.append([ev[j].elapsed_time(ev[j + 1]) for j in range(n_events - 1)])
+                whole.append(ev[0].elapsed_time(ev[-1]))
+    return segs, whole
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+def cpu_baseline(n_steps=3):
+    """fp64 oracle on one request of the CSA workload (bounded sample): the
+    oracle builds that request's cache from the seeded raw stream, then runs
+    whole decode steps (indexer -> top-k -> attention) on it."""
+    import numpy as np
+    import oracle
+    import torch
+    from csla_synth import normal, permutation
+    from csla_synth import torch_gen
+    kw = CSA
+    L, D, dI, m = kw["L"], kw["D"], kw["dI"], kw["m"]
+    seed = 1
+    gamma_kv = (1.0 + 0.1 * normal(seed, "gamma_kv", (D,))).astype(np.float32).astype(np.float64)
+    wg = normal(seed, "wg", (D,), std=1.0 / D ** 0.5).astype(np.float32).astype(np.float64)
+    gb = normal(seed, "gb", (m,)).astype(np.float32).astype(np.float64)
+    wgi = normal(seed, "wgi", (dI,), std=1.0 / dI ** 0.5).astype(np.float32).astype(np.float64)
+    gbi = normal(seed, "gbi", (m,)).astype(np.float32).astype(np.float64)
+    # raw stream of request 0, rank 0 (same generator as the GPU run), on the host
+    kv = torch_gen.normal(seed, "kv/0/0", (L, D), device="cpu").to(torch.bfloat16).double().numpy()
+    ki = torch_gen.normal(seed, "idx/0/0", (L, dI), device="cpu").to(torch.bfloat16).double().numpy()
+    epp = 128 // m
+    pages = L // 128
+    bt = permutation(seed, "cpu/pages", pages).astype(np.int32).reshape(1, pages)
+    rows = np.zeros((pages, epp, D + 64), np.uint8)
+    scales = np.zeros((pages, epp), np.float32)
+    kidx = np.zeros((pages, epp, dI), np.uint16)
+    for b in range(L // m):
+        r, s = oracle.compressed_row(kv[b * m:(b + 1) * m], wg, gb, gamma_kv, b)
+        pg = bt[0, b // epp]
+        rows[pg, b % epp], scales[pg, b % epp] = r, s
+        kidx[pg, b % epp] = oracle.index_key(ki[b * m:(b + 1) * m], wgi, gbi)
+    win = np.zeros((1, 128, D + 64), np.uint8)
+    wsc = np.zeros((1, 128), np.float32)
+    for p in range(L - 128, L):
+        win[0, p % 128], wsc[0, p % 128] = oracle.window_row(kv[p], gamma_kv, p)
+    cv = oracle.CacheView(m, D, rows, scales, bt, win, wsc, kidx, dI)
+    W = normal(seed, "W_iq_cpu", (kw["HI"] * dI, kw["dc"]), std=1.0 / kw["dc"] ** 0.5)
+    sink = normal(seed, "sink", (kw["H"],))
+    gq = 1.0 + 0.1 * normal(seed, "gamma_q", (D,))
+    times = []
+    for s in range(n_steps):
+        q = normal(seed, "cpu/q/%d" % s, (1, kw["H"], D))
+        cq = normal(seed, "cpu/cq/%d" % s, (1, kw["dc"]))
+        hw = normal(seed, "cpu/hw/%d" % s, (1, kw["HI"]))
+        t0 = time.perf_counter()
+        oracle.csa_decode(cv, [0], [L], q, gq, cq, W, hw, sink, kw["HI"], kw["k"])
+        times.append(time.perf_counter() - t0)
+    return times
+
+
+def run_reference(args):
+    t_setup = time.perf_counter()
+    times = cpu_baseline(n_steps=args.warmup + args.steps)
+    timed = times[args.warmup:]
+    per_step = sum(timed) / len(timed)
+    value = 1.0 / per_step
+    sample = "1 request of the CSA workload (context 131072, 32768 entries, k=512), fp64 oracle"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded splitmix64 / Box-Muller)",
+            "config": {"workload": "csa_decode_B8_L131072", "sample": "1 of 8 requests per step"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "setup_s": time.perf_counter() - t_setup}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from compressed_sparse_long_append_b200 import build as cbuild
+    cbuild.build()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    W, K = max(3, args.warmup), args.steps
+    seed = 1
+
+    # ---------------- CSA layer (the headline workload)
+    kw = dict(CSA)
+    L0 = kw["L"] - (W + K)
+    lb, cp, params = build_layer(kw, kw["B"], L0, seed, rank, device)
+    inputs = step_inputs(kw, kw["B"], W + K, seed, rank, device)
+    step = CsaStep(lb, cp, params, kw, args.variant, device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = ClockSampler(local)
+    clk.start()
+    segs, whole = timed_steps(step, inputs, W, K, 5, flush)
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    if world > 1:
+        dist.barrier()
+    ms_step = sum(whole) / len(whole)
+    ms_idx = sum(s[1] for s in segs) / len(segs)
+    ms_seg = [sum(s[j] for s in segs) / len(segs) for j in range(4)]
+    if world > 1:
+        t = torch.tensor([ms_step], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+
+    # e2e: host buffers, copies inside the timed region (fresh cache state)
+    lb2, cp2, params2 = build_layer(kw, kw["B"], L0, seed, rank, device)
+    step2 = CsaStep(lb2, cp2, params2, kw, args.variant, device)
+    _, whole_e2e = timed_steps(step2, inputs, W, K, 5, flush, e2e=True)
+    ms_e2e = sum(whole_e2e) / len(whole_e2e)
+    if world > 1:
+        t = torch.tensor([ms_e2e], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    h2d = sum(v.numel() * v.element_size() for k, v in inputs[0]["host"].items())
+    d2h = step2.out.numel() * step2.out.element_size()
+    del lb2, step2
+
+    # algorithmic bytes of the indexer call (dominant): keys + W_iq + scores
+    Ls = [kw["L"] - K + i for i in range(K)]    # context after each timed step's append
+    nv_mean = sum(L // kw["m"] for L in Ls) / K
+    idx_bytes = kw["B"] * nv_mean * (kw["dI"] * 2 + 4) + kw["HI"] * kw["dI"] * kw["dc"] * 2
+    peak, peak_kind = peaks()
+    achieved = idx_bytes / (ms_idx * 1e-3) / 1e9
+
+    hca = None
+    if not args.no_hca:
+        del step, lb
+        torch.cuda.empty_cache()
+        hk = dict(HCA)
+        hL0 = hk["L"] - (W + K)
+        hlb, hcp, hparams = build_layer(hk, hk["B"], hL0, seed + 1, rank, device)
+        hin = step_inputs(hk, hk["B"], W + K, seed + 1, rank, device)
+        hstep = HcaStep(hlb, hcp, hparams, hk, args.variant, device)
+        hsegs, hwhole = timed_steps(hstep, hin, W, K, 3, flush)
+        hms = sum(hwhole) / len(hwhole)
+        hms_att = sum(s[1] for s in hsegs) / len(hsegs)
+        rows = hk["L"] // hk["m"] + hk["n_win"]
+        hbytes = hk["B"] * (rows * (hk["D"] + 64 + 4) + 2 * hk["H"] * hk["D"] * 2)
+        hflops = hk["B"] * rows * hk["H"] * hk["D"] * 4
+        hca = {"workload": "hca_decode_B4_L1048576", "tokens_per_s": hk["B"] / (hms * 1e-3),
+               "ms_per_step": hms, "attend_ms": hms_att,
+               "attend_hbm_gbs": hbytes / (hms_att * 1e-3) / 1e9,
+               "attend_hbm_frac": hbytes / (hms_att * 1e-3) / 1e9 / peak,
+               "attend_tflops": hflops / (hms_att * 1e-3) / 1e12,
+               "attend_tensor_frac_sustained": hflops / (hms_att * 1e-3) / 1e12 / 1395.7}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        try:
+            ct = cpu_baseline(n_steps=3)
+            v = 1.0 / (sum(ct) / len(ct))
+            cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                   "sample": "1 request of this workload (context 131072, k=512), 3 decode steps, fp64 oracle, "
+                             "single thread"}
+        except Exception as e:  # the baseline never blocks the GPU line
+            cpu = {"value": None, "unit": UNIT, "cores": 0, "kind": "oracle", "sample": "failed: %s" % e}
+
+    if rank == 0:
+        B = kw["B"]
+        line = {
+            "metric": METRIC, "value": B * world / (ms_step * 1e-3), "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded splitmix64 / Box-Muller token streams, caches built by csla_compress_append)",
+            "config": {"workload": "csa_decode_B8_L131072", "requests_per_gpu": B, "context": kw["L"],
+                       "m": 4, "compressed_entries": kw["L"] // 4, "heads": 64, "head_dim": 512,
+                       "index_heads": 16, "index_dim": 128, "dc": 1024, "topk": 512, "window": 128,
+                       "l2": "flushed before every step (512 MiB write, outside the timed events)",
+                       "parallelism": "dp%d over requests" % world, "variant": args.variant},
+            "segments_ms": {"compress_append": ms_seg[0], "indexer_scores": ms_seg[1], "topk_select": ms_seg[2],
+                            "csa_attend": ms_seg[3]},
+            "roofline": {"bound": "hbm", "kernel": "csla_indexer_scores (iq_project + indexer)",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "peak_kind": peak_kind, "traffic": None,
+                         "algorithmic_bytes": idx_bytes},
+            "cpu_baseline": cpu,
+            "e2e": {"value": kw["B"] * world / (ms_e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": step_launches_total(K),
+            "clocks": clocks,
+            "hca_decode": hca,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def step_launches_total(K):
+    # per CSA step: compress, iq_project, indexer, topk, attend, combine
+    return 6 * K
+
+
+if __name__ == "__main__":
+    main()

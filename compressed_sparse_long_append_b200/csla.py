@@ -1,0 +1,158 @@
+"""Thin ctypes binding of libcsla (include/csla.h), same entry-point names.
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Array arguments may be torch CUDA tensors (their data_ptr is
+passed) or raw integer device addresses.  If libcsla.so is missing or cannot
+be loaded, importing this module raises: there is no fallback path.
+"""
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsla.so")
+
+CSLA_OK, CSLA_ERR_ARG, CSLA_ERR_UNSUPPORTED, CSLA_ERR_CUDA, CSLA_ERR_DEVICE = 0, 1, 2, 3, 4
+CSLA_F32, CSLA_BF16 = 0, 1
+CSLA_VARIANT_AUTO, CSLA_VARIANT_SATURATED, CSLA_VARIANT_STARVED = 0, 1, 2
+CSLA_OP_INDEXER, CSLA_OP_TOPK, CSLA_OP_CSA_ATTEND, CSLA_OP_HCA_ATTEND = 1, 2, 3, 4
+CSLA_DEVERR_PAGE, CSLA_DEVERR_INDEX, CSLA_DEVERR_LEN, CSLA_DEVERR_TIMEOUT = 1, 2, 4, 8
+CSLA_PAGE_TOKENS = 128
+
+EXPORTS = ("csla_compress_append", "csla_indexer_scores", "csla_topk_select", "csla_csa_attend",
+           "csla_hca_attend", "csla_workspace_size", "csla_device_error", "csla_strerror", "csla_version")
+
+
+class csla_cfg(ctypes.Structure):
+    _fields_ = [("m", ctypes.c_int32), ("D", ctypes.c_int32), ("d_rope", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("HI", ctypes.c_int32), ("dI", ctypes.c_int32),
+                ("dc", ctypes.c_int32), ("n_win", ctypes.c_int32), ("rope_theta", ctypes.c_float),
+                ("eps", ctypes.c_float)]
+
+
+class csla_cache(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("kidx", ctypes.c_void_p),
+                ("block_table", ctypes.c_void_p), ("bt_stride", ctypes.c_int32),
+                ("n_pages", ctypes.c_int32)]
+
+
+class csla_state(ctypes.Structure):
+    _fields_ = [("win_rows", ctypes.c_void_p), ("win_scales", ctypes.c_void_p),
+                ("tail_kv", ctypes.c_void_p), ("tail_idx", ctypes.c_void_p), ("len", ctypes.c_void_p),
+                ("n_slots", ctypes.c_int32)]
+
+
+class csla_compress_params(ctypes.Structure):
+    _fields_ = [("gamma_kv", ctypes.c_void_p), ("wg", ctypes.c_void_p), ("gb", ctypes.c_void_p),
+                ("wgi", ctypes.c_void_p), ("gbi", ctypes.c_void_p)]
+
+
+class CslaError(RuntimeError):
+    def __init__(self, fn, status, bits=0):
+        self.status, self.bits = status, bits
+        super().__init__("%s failed: %s (status %d, device bits 0x%x)"
+                         % (fn, _lib.csla_strerror(status).decode(), status, bits))
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libcsla.so not built (%s); run `python -m "
+                          "compressed_sparse_long_append_b200.build`" % LIB_PATH)
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, Z = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    sig = {
+        "csla_compress_append": [P, P, P, P, I, I, P, P, I, P, P],
+        "csla_indexer_scores": [P, P, P, P, I, I, P, I, P, I, P, P, I, P, Z, P],
+        "csla_topk_select": [P, P, P, I, I, P, I, I, P, P],
+        "csla_csa_attend": [P, P, P, P, I, P, I, P, I, P, P, P, I, I, P, Z, P],
+        "csla_hca_attend": [P, P, P, P, I, I, P, I, P, P, P, I, I, P, Z, P],
+        "csla_workspace_size": [P, I, I, I],
+        "csla_device_error": [P, ctypes.POINTER(ctypes.c_uint32)],
+        "csla_strerror": [ctypes.c_int],
+        "csla_version": [],
+    }
+    res = {"csla_workspace_size": ctypes.c_size_t, "csla_strerror": ctypes.c_char_p}
+    for name, args in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res.get(name, ctypes.c_int)
+    return L
+
+
+_lib = _load()
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _check(fn, rc):
+    if rc != CSLA_OK:
+        raise CslaError(fn, rc)
+    return rc
+
+
+def _ref(s):
+    return None if s is None else ctypes.byref(s)
+
+
+def csla_compress_append(cfg, st, cache, slots, B, T, kv_new, kidx_new, kv_dtype, params, stream=None):
+    return _check("csla_compress_append", _lib.csla_compress_append(
+        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, T, _ptr(kv_new), _ptr(kidx_new), kv_dtype,
+        _ref(params), _stream(stream)))
+
+
+def csla_indexer_scores(cfg, st, cache, slots, B, max_len, cq, cq_dtype, W_iq, w_dtype, head_w, scores,
+                        scores_stride, workspace, workspace_bytes, stream=None):
+    return _check("csla_indexer_scores", _lib.csla_indexer_scores(
+        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, max_len, _ptr(cq), cq_dtype, _ptr(W_iq), w_dtype,
+        _ptr(head_w), _ptr(scores), scores_stride, _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def csla_topk_select(cfg, st, slots, B, max_len, scores, scores_stride, k, idx, stream=None):
+    return _check("csla_topk_select", _lib.csla_topk_select(
+        _ref(cfg), _ref(st), _ptr(slots), B, max_len, _ptr(scores), scores_stride, k, _ptr(idx),
+        _stream(stream)))
+
+
+def csla_csa_attend(cfg, st, cache, slots, B, q, q_dtype, idx, k, sink, gamma_q, out, out_dtype, variant,
+                    workspace, workspace_bytes, stream=None):
+    return _check("csla_csa_attend", _lib.csla_csa_attend(
+        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, _ptr(q), q_dtype, _ptr(idx), k, _ptr(sink),
+        _ptr(gamma_q), _ptr(out), out_dtype, variant, _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def csla_hca_attend(cfg, st, cache, slots, B, max_len, q, q_dtype, sink, gamma_q, out, out_dtype, variant,
+                    workspace, workspace_bytes, stream=None):
+    return _check("csla_hca_attend", _lib.csla_hca_attend(
+        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, max_len, _ptr(q), q_dtype, _ptr(sink),
+        _ptr(gamma_q), _ptr(out), out_dtype, variant, _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def csla_workspace_size(cfg, op, B, max_len):
+    return int(_lib.csla_workspace_size(_ref(cfg), op, B, max_len))
+
+
+def csla_device_error(stream=None):
+    """Synchronise the stream; return (status, bits) of the device error word (cleared)."""
+    bits = ctypes.c_uint32(0)
+    rc = _lib.csla_device_error(_stream(stream), ctypes.byref(bits))
+    return rc, bits.value
+
+
+def csla_strerror(status):
+    return _lib.csla_strerror(status).decode()
+
+
+def csla_version():
+    return int(_lib.csla_version())

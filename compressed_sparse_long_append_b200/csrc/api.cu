@@ -1,0 +1,256 @@
+// api.cu -- the C ABI of libcsla (declared in include/csla.h): host-side
+// argument checks, TMA descriptor encoding and kernel launches.
+#include <string.h>
+
+#include "../../include/csla.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+using namespace csla;
+
+int num_sms_current() {
+    static int cached[64];
+    static bool init[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev >= 0 && dev < 64 && init[dev]) return cached[dev];
+    int n = 148;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (dev >= 0 && dev < 64) {
+        cached[dev] = n;
+        init[dev] = true;
+    }
+    return n;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor [rows][cols] (cols contiguous), box = 64 cols x box_rows, 128B swizzle.
+bool encode_bf16_2d(CUtensorMap *map, const void *ptr, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = f(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cfg(const csla_cfg *c) {
+    if (!c) return CSLA_ERR_ARG;
+    if (c->d_rope != 64 || (c->D != 128 && c->D != 512) || (c->m != 4 && c->m != 128) || c->n_win != 128)
+        return CSLA_ERR_UNSUPPORTED;
+    if (c->H < 1 || c->H > 64) return CSLA_ERR_UNSUPPORTED;
+    if (!(c->eps >= 0.f) || !(c->rope_theta > 0.f)) return CSLA_ERR_ARG;
+    return CSLA_OK;
+}
+
+int check_csa_indexer_shape(const csla_cfg *c) {
+    if (c->m != 4) return CSLA_ERR_UNSUPPORTED;
+    if (c->dI != 64 && c->dI != 128) return CSLA_ERR_UNSUPPORTED;
+    if (c->HI != 4 && c->HI != 8 && c->HI != 16) return CSLA_ERR_UNSUPPORTED;
+    if (c->dc < 8 || c->dc > 4096 || c->dc % 8) return CSLA_ERR_UNSUPPORTED;
+    return CSLA_OK;
+}
+
+int nq_of(int HI) { return (2 * HI + 15) / 16 * 16; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? CSLA_OK : CSLA_ERR_CUDA; }
+
+size_t attend_ws(const csla_cfg *c, int B, long long max_rows) {
+    const size_t per = ((size_t)c->H * c->D + 2 * (size_t)c->H) * sizeof(float);
+    return (size_t)B * attend_max_chunks(max_rows) * per;
+}
+
+}  // namespace
+
+extern "C" {
+
+int csla_version(void) { return 100; }
+
+const char *csla_strerror(int s) {
+    switch (s) {
+        case CSLA_OK: return "ok";
+        case CSLA_ERR_ARG: return "invalid argument";
+        case CSLA_ERR_UNSUPPORTED: return "unsupported shape";
+        case CSLA_ERR_CUDA: return "CUDA error";
+        case CSLA_ERR_DEVICE: return "device-side input error";
+        default: return "unknown status";
+    }
+}
+
+size_t csla_workspace_size(const csla_cfg *cfg, int32_t op, int32_t B, int32_t max_len) {
+    if (check_cfg(cfg) != CSLA_OK || B < 1 || max_len < 0) return 0;
+    switch (op) {
+        case CSLA_OP_INDEXER:
+            if (check_csa_indexer_shape(cfg) != CSLA_OK) return 0;
+            return (size_t)B * nq_of(cfg->HI) * cfg->dI * 2;
+        case CSLA_OP_TOPK: return 0;
+        case CSLA_OP_CSA_ATTEND: return attend_ws(cfg, B, (long long)max_len + cfg->n_win);
+        case CSLA_OP_HCA_ATTEND: return attend_ws(cfg, B, (long long)max_len / cfg->m + cfg->n_win);
+        default: return 0;
+    }
+}
+
+int csla_device_error(csla_stream_t stream, uint32_t *bits) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return CSLA_ERR_CUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, csla::g_dev_err, sizeof(v)) != cudaSuccess) return CSLA_ERR_CUDA;
+    if (v && cudaMemcpyToSymbol(csla::g_dev_err, &zero, sizeof(zero)) != cudaSuccess) return CSLA_ERR_CUDA;
+    if (bits) *bits = v;
+    return v ? CSLA_ERR_DEVICE : CSLA_OK;
+}
+
+int csla_compress_append(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
+                         int32_t B, int32_t T, const void *kv_new, const void *kidx_new, int32_t kv_dtype,
+                         const csla_compress_params *p, csla_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (!st || !cache || !slots || !kv_new || !p || B < 1 || T < 1 || T > 65535) return CSLA_ERR_ARG;
+    if (st->n_slots < 1 || B > 65535) return CSLA_ERR_ARG;
+    if (kv_dtype != CSLA_F32 && kv_dtype != CSLA_BF16) return CSLA_ERR_ARG;
+    if (!st->win_rows || !st->win_scales || !st->tail_kv || !st->len || !cache->rows || !cache->scales ||
+        !cache->block_table || cache->bt_stride < 1 || cache->n_pages < 1)
+        return CSLA_ERR_ARG;
+    if (!p->gamma_kv || !p->wg || !p->gb) return CSLA_ERR_ARG;
+    const bool csa = cfg->m == 4;
+    if (csa) {
+        if (cfg->dI < 1 || cfg->dI > 512 || !kidx_new || !cache->kidx || !st->tail_idx || !p->wgi || !p->gbi)
+            return CSLA_ERR_ARG;
+    }
+    CompressArgs a{};
+    a.m = cfg->m; a.D = cfg->D; a.d_rope = cfg->d_rope; a.dI = csa ? cfg->dI : 0; a.n_win = cfg->n_win;
+    a.theta = cfg->rope_theta; a.eps = cfg->eps;
+    a.slots = slots; a.B = B; a.T = T;
+    a.kv_new = kv_new; a.kidx_new = csa ? kidx_new : nullptr;
+    a.gamma_kv = p->gamma_kv; a.wg = p->wg; a.gb = p->gb; a.wgi = p->wgi; a.gbi = p->gbi;
+    a.win_rows = st->win_rows; a.win_scales = st->win_scales; a.tail_kv = st->tail_kv;
+    a.tail_idx = csa ? st->tail_idx : nullptr; a.len = st->len;
+    a.rows = cache->rows; a.scales = cache->scales; a.kidx = csa ? cache->kidx : nullptr;
+    a.block_table = cache->block_table; a.bt_stride = cache->bt_stride; a.n_pages = cache->n_pages;
+    a.n_slots = st->n_slots;
+    return cuda_status(launch_compress_append(a, kv_dtype == CSLA_BF16, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
+                        int32_t B, int32_t max_len, const void *cq, int32_t cq_dtype, const void *W_iq,
+                        int32_t w_dtype, const float *head_w, float *scores, int32_t scores_stride, void *workspace,
+                        size_t workspace_bytes, csla_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    rc = check_csa_indexer_shape(cfg);
+    if (rc) return rc;
+    if (!st || !st->len || !cache || !cache->kidx || !cache->block_table || !slots || !cq || !W_iq || !head_w ||
+        !scores || !workspace || B < 1 || max_len < 1)
+        return CSLA_ERR_ARG;
+    if ((cq_dtype != CSLA_F32 && cq_dtype != CSLA_BF16) || (w_dtype != CSLA_F32 && w_dtype != CSLA_BF16))
+        return CSLA_ERR_ARG;
+    if (scores_stride < max_len / cfg->m) return CSLA_ERR_ARG;
+    if (workspace_bytes < csla_workspace_size(cfg, CSLA_OP_INDEXER, B, max_len)) return CSLA_ERR_ARG;
+    if (!aligned16(cq) || !aligned16(W_iq) || !aligned16(cache->kidx) || !aligned16(workspace)) return CSLA_ERR_ARG;
+    const int NQ = nq_of(cfg->HI);
+    CUtensorMap kmap, qmap;
+    if (!encode_bf16_2d(&kmap, cache->kidx, (uint64_t)cfg->dI, (uint64_t)cache->n_pages * 32, 32))
+        return CSLA_ERR_CUDA;
+    if (!encode_bf16_2d(&qmap, workspace, (uint64_t)cfg->dI, (uint64_t)B * NQ, (uint32_t)NQ)) return CSLA_ERR_CUDA;
+    IndexerArgs a{};
+    a.m = cfg->m; a.HI = cfg->HI; a.dI = cfg->dI; a.dc = cfg->dc; a.NQ = NQ;
+    a.slots = slots; a.len = st->len; a.block_table = cache->block_table; a.bt_stride = cache->bt_stride;
+    a.n_pages = cache->n_pages; a.n_slots = st->n_slots; a.B = B;
+    const int nvmax = max_len / cfg->m;
+    a.tiles_per_req = (nvmax + 127) / 128;
+    if (a.tiles_per_req < 1) a.tiles_per_req = 1;
+    a.max_len = max_len;
+    a.cq = cq; a.W = W_iq; a.head_w = head_w; a.scores = scores; a.scores_stride = scores_stride;
+    a.q_ws = reinterpret_cast<uint16_t *>(workspace);
+    return cuda_status(launch_indexer(a, cq_dtype == CSLA_BF16, w_dtype == CSLA_BF16, kmap, qmap, num_sms_current(),
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *slots, int32_t B, int32_t max_len,
+                     const float *scores, int32_t scores_stride, int32_t k, int32_t *idx, csla_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (!st || !st->len || !slots || !scores || !idx || B < 1 || max_len < 0 || k < 1 || k > 2048)
+        return CSLA_ERR_ARG;
+    if (scores_stride < max_len / cfg->m) return CSLA_ERR_ARG;
+    TopkArgs a{};
+    a.scores = scores; a.stride = scores_stride; a.slots = slots; a.len = st->len;
+    a.m = cfg->m; a.k = k; a.B = B; a.max_n = max_len / cfg->m; a.idx = idx; a.n_slots = st->n_slots;
+    return cuda_status(launch_topk(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static int attend_common(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
+                         int32_t B, int32_t max_len, const void *q, int32_t q_dtype, const int32_t *idx, int32_t k,
+                         const float *sink, const float *gamma_q, void *out, int32_t out_dtype, int32_t variant,
+                         void *workspace, size_t workspace_bytes, csla_stream_t stream) {
+    if (!st || !st->len || !st->win_rows || !st->win_scales || !cache || !cache->rows || !cache->scales ||
+        !cache->block_table || !slots || !q || !sink || !gamma_q || !out || !workspace || B < 1)
+        return CSLA_ERR_ARG;
+    if ((q_dtype != CSLA_F32 && q_dtype != CSLA_BF16) || (out_dtype != CSLA_F32 && out_dtype != CSLA_BF16))
+        return CSLA_ERR_ARG;
+    if (variant < CSLA_VARIANT_AUTO || variant > CSLA_VARIANT_STARVED) return CSLA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(cache->rows) || !aligned16(st->win_rows)) return CSLA_ERR_ARG;
+    AttendArgs a{};
+    a.m = cfg->m; a.D = cfg->D; a.d_rope = cfg->d_rope; a.H = cfg->H; a.n_win = cfg->n_win;
+    a.theta = cfg->rope_theta; a.eps = cfg->eps;
+    a.slots = slots; a.len = st->len; a.B = B; a.q = q; a.idx = idx; a.k = idx ? k : 0;
+    a.sink = sink; a.gamma_q = gamma_q;
+    a.rows = cache->rows; a.scales = cache->scales; a.block_table = cache->block_table;
+    a.bt_stride = cache->bt_stride; a.n_pages = cache->n_pages; a.n_slots = st->n_slots;
+    a.win_rows = st->win_rows; a.win_scales = st->win_scales; a.out = out;
+    a.part = reinterpret_cast<float *>(workspace);
+    const long long max_rows = idx ? (long long)k + cfg->n_win : (long long)max_len / cfg->m + cfg->n_win;
+    a.max_chunks = attend_max_chunks(max_rows);
+    a.max_len = max_len;
+    if (workspace_bytes < attend_ws(cfg, B, max_rows)) return CSLA_ERR_ARG;
+    return cuda_status(launch_attend(a, q_dtype == CSLA_BF16, out_dtype == CSLA_BF16, variant, num_sms_current(),
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int csla_csa_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
+                    int32_t B, const void *q, int32_t q_dtype, const int32_t *idx, int32_t k, const float *sink,
+                    const float *gamma_q, void *out, int32_t out_dtype, int32_t variant, void *workspace,
+                    size_t workspace_bytes, csla_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (!idx || k < 1 || k > 2048) return CSLA_ERR_ARG;
+    // Without max_len the bound on the context is the int32 range.
+    return attend_common(cfg, st, cache, slots, B, 0x7FFFFFFF, q, q_dtype, idx, k, sink, gamma_q, out, out_dtype,
+                         variant, workspace, workspace_bytes, stream);
+}
+
+int csla_hca_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
+                    int32_t B, int32_t max_len, const void *q, int32_t q_dtype, const float *sink,
+                    const float *gamma_q, void *out, int32_t out_dtype, int32_t variant, void *workspace,
+                    size_t workspace_bytes, csla_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (max_len < 1) return CSLA_ERR_ARG;
+    return attend_common(cfg, st, cache, slots, B, max_len, q, q_dtype, nullptr, 0, sink, gamma_q, out, out_dtype,
+                         variant, workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,105 @@
+"""Device buffers of one CSA or HCA layer, owned by torch, described to the
+library through the csla_cache / csla_state structs.
+
+Plumbing only: this module allocates and zero-fills memory and builds the
+ctypes structs; all computation happens in libcsla's kernels.
+"""
+from dataclasses import dataclass
+
+import torch
+
+from . import csla as C
+
+
+@dataclass(frozen=True)
+class LayerShape:
+    m: int                 # 4 (CSA) or 128 (HCA)
+    D: int = 512
+    H: int = 64
+    HI: int = 16
+    dI: int = 128
+    dc: int = 1024
+    n_win: int = 128
+    d_rope: int = 64
+    theta: float = 10000.0
+    eps: float = 1e-6
+
+    @property
+    def is_csa(self):
+        return self.m == 4
+
+    @property
+    def row_bytes(self):
+        return (self.D - self.d_rope) + 2 * self.d_rope
+
+    @property
+    def epp(self):
+        return C.CSLA_PAGE_TOKENS // self.m
+
+    def cfg(self):
+        return C.csla_cfg(self.m, self.D, self.d_rope, self.H, self.HI if self.is_csa else 0,
+                          self.dI if self.is_csa else 0, self.dc if self.is_csa else 0, self.n_win,
+                          self.theta, self.eps)
+
+
+class LayerBuffers:
+    """Classical cache pages + block table + state cache for `n_slots` requests."""
+
+    def __init__(self, shape: LayerShape, n_slots: int, n_pages: int, bt_stride: int, device="cuda"):
+        s = shape
+        self.shape = s
+        self.device = torch.device(device)
+        dev = self.device
+        self.rows = torch.zeros((n_pages, s.epp, s.row_bytes), dtype=torch.uint8, device=dev)
+        self.scales = torch.zeros((n_pages, s.epp), dtype=torch.float32, device=dev)
+        self.kidx = torch.zeros((n_pages, s.epp, s.dI), dtype=torch.int16, device=dev) if s.is_csa else None
+        self.block_table = torch.full((n_slots, bt_stride), -1, dtype=torch.int32, device=dev)
+        self.win_rows = torch.zeros((n_slots, s.n_win, s.row_bytes), dtype=torch.uint8, device=dev)
+        self.win_scales = torch.zeros((n_slots, s.n_win), dtype=torch.float32, device=dev)
+        self.tail_kv = torch.zeros((n_slots, s.m, s.D), dtype=torch.float32, device=dev)
+        self.tail_idx = torch.zeros((n_slots, s.m, s.dI), dtype=torch.float32, device=dev) if s.is_csa else None
+        self.len = torch.zeros((n_slots,), dtype=torch.int32, device=dev)
+        self.n_slots, self.n_pages, self.bt_stride = n_slots, n_pages, bt_stride
+        self._cfg = s.cfg()
+
+    def cfg(self):
+        return self._cfg
+
+    def cache(self):
+        return C.csla_cache(self.rows.data_ptr(), self.scales.data_ptr(),
+                            self.kidx.data_ptr() if self.kidx is not None else None,
+                            self.block_table.data_ptr(), self.bt_stride, self.n_pages)
+
+    def state(self):
+        return C.csla_state(self.win_rows.data_ptr(), self.win_scales.data_ptr(), self.tail_kv.data_ptr(),
+                            self.tail_idx.data_ptr() if self.tail_idx is not None else None,
+                            self.len.data_ptr(), self.n_slots)
+
+    def host_view(self):
+        """Host copies of every buffer (for checks against an independent model)."""
+        out = {k: getattr(self, k).cpu().numpy() for k in
+               ("rows", "scales", "block_table", "win_rows", "win_scales", "tail_kv", "len")}
+        if self.kidx is not None:
+            out["kidx"] = self.kidx.cpu().numpy().view("uint16")
+            out["tail_idx"] = self.tail_idx.cpu().numpy()
+        return out
+
+
+class CompressParams:
+    """fp32 compressor parameters on the device."""
+
+    def __init__(self, gamma_kv, wg, gb, wgi=None, gbi=None, device="cuda"):
+        f = lambda x: None if x is None else torch.as_tensor(x, dtype=torch.float32).to(device).contiguous()
+        self.gamma_kv, self.wg, self.gb, self.wgi, self.gbi = f(gamma_kv), f(wg), f(gb), f(wgi), f(gbi)
+
+    def struct(self):
+        p = lambda t: None if t is None else t.data_ptr()
+        return C.csla_compress_params(p(self.gamma_kv), p(self.wg), p(self.gb), p(self.wgi), p(self.gbi))
+
+
+def dtype_code(t: torch.Tensor):
+    if t.dtype == torch.float32:
+        return C.CSLA_F32
+    if t.dtype == torch.bfloat16:
+        return C.CSLA_BF16
+    raise TypeError("unsupported dtype %s" % t.dtype)

@@ -1,0 +1,244 @@
+/*
+ * csla.h -- C ABI of libcsla, the B200 (sm_100a) implementation of the
+ * CSA/HCA hybrid compressed attention decode path.
+ *
+ * The operation (page title, section):
+ *   haiqwa.github.io "DeepSeek-V4" blog, §CSA：压缩稀疏注意力 and §HCA：重度压缩注意力
+ *     (every m tokens of KV become one entry; every query attends k entries);
+ *     §RMSNorm归一化 (RMSNorm on each query head and on the single KV head);
+ *     §Partial RoPE位置编码 (RoPE dims bf16, other dims fp8; sliding window);
+ *     §让注意力学会"忽略" (per-head sink logit in the softmax denominator);
+ *     §索引可见性处理 (visible compressed range computable by rule).
+ *   硅星人 article "DeepSeek V4 ... 让token大降价", §两大压缩注意力: CSA data flow
+ *     (compressor m=4, lightning indexer with dc=1024 latent and ReLU scores,
+ *     top-k 512/1024, window of 128 raw tokens, MQA), HCA (m'=128, no indexer,
+ *     no top-k), RoPE on the last 64 dims, bf16/fp8 cache, the per-request
+ *     state cache and the classical cache in blocks of lcm(4,128)=128 tokens.
+ *   QbitAI article on DeepSeek V4's batch invariance: outputs bit-identical
+ *     whatever the batch; a saturated and a starved attention kernel that
+ *     agree bit for bit.
+ *
+ * Conventions for every entry point
+ *   - All array pointers are DEVICE pointers owned by the caller (csla_cfg,
+ *     csla_cache and csla_state themselves are host structs holding device
+ *     pointers).  The library never allocates device memory; scratch comes
+ *     from the caller through `workspace` (size from csla_workspace_size).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  Host-side argument checks happen before any
+ *     launch and return an error without launching anything.
+ *   - Return value: CSLA_OK or a CSLA_ERR_* code.  Errors that only the
+ *     device can see (a page id outside the pool, an index outside the
+ *     visible range, a length above max_len) never trap: the kernel skips
+ *     the offending work, records a bit in the library's device error word
+ *     and carries on; csla_device_error() reads and clears it.
+ *   - A batch is `B` requests given by `slots` (device int32[B], distinct
+ *     state-cache slot ids).  Context length of request b after the call is
+ *     st->len[slots[b]].  `max_len` (host) is an upper bound on it, used to
+ *     size grids.
+ *
+ * Data layout (little-endian)
+ *   Cache row of one token or compressed entry, D = d_nope + d_rope dims:
+ *     bytes [0, d_nope)             E4M3 (OCP FP8 E4M3FN) codes of dims 0..d_nope-1
+ *     bytes [d_nope, d_nope+2*dr)   bf16 values of dims d_nope..D-1 (the RoPE dims)
+ *   plus one fp32 scale per row: value of dim d < d_nope = e4m3(code)*scale.
+ *   Row bytes: 576 for D=512, 192 for D=128.
+ *   Classical cache (one layer): pages of CSLA_PAGE_TOKENS=128 raw tokens,
+ *   epp = 128/m entries per page (32 for CSA, 1 for HCA):
+ *     rows   uint8 [n_pages][epp][row_bytes]
+ *     scales f32   [n_pages][epp]
+ *     kidx   bf16  [n_pages][epp][dI]         (CSA only: compressed index keys)
+ *     block_table int32 [n_slots][bt_stride]: compressed entry e of slot s is
+ *       entry e % epp of page block_table[s][e / epp].
+ *   State cache (one layer, per slot):
+ *     win_rows   uint8 [n_slots][n_win][row_bytes]  token at position p lives in
+ *     win_scales f32   [n_slots][n_win]             ring slot p % n_win
+ *     tail_kv    f32   [n_slots][m][D]       raw KV of the not yet compressed block
+ *     tail_idx   f32   [n_slots][m][dI]      raw index-key inputs (CSA only)
+ *     len        int32 [n_slots]             tokens appended so far
+ */
+#ifndef CSLA_H
+#define CSLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *csla_stream_t; /* same type as cudaStream_t */
+
+enum {
+    CSLA_OK = 0,
+    CSLA_ERR_ARG = 1,         /* null pointer, bad size, k > supported, workspace too small */
+    CSLA_ERR_UNSUPPORTED = 2, /* a shape this build has no kernel for */
+    CSLA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+    CSLA_ERR_DEVICE = 4       /* a kernel recorded a bad input (see csla_device_error) */
+};
+
+enum { CSLA_F32 = 0, CSLA_BF16 = 1 };
+
+enum { CSLA_VARIANT_AUTO = 0, CSLA_VARIANT_SATURATED = 1, CSLA_VARIANT_STARVED = 2 };
+
+enum { CSLA_OP_INDEXER = 1, CSLA_OP_TOPK = 2, CSLA_OP_CSA_ATTEND = 3, CSLA_OP_HCA_ATTEND = 4 };
+
+/* device error word bits */
+enum {
+    CSLA_DEVERR_PAGE = 1,     /* block-table entry outside [0, n_pages) */
+    CSLA_DEVERR_INDEX = 2,    /* top-k index outside [0, visible entries) */
+    CSLA_DEVERR_LEN = 4,      /* context length above max_len */
+    CSLA_DEVERR_TIMEOUT = 8   /* a bounded wait inside a kernel gave up */
+};
+
+#define CSLA_PAGE_TOKENS 128
+
+/* Layer shape.  Supported: m in {4, 128}; D in {128, 512}; d_rope = 64;
+ * 1 <= H <= 64; n_win = 128; CSA (m = 4): dI in {64, 128}, 1 <= HI <= 16,
+ * dc a multiple of 8 up to 4096, 1 <= topk <= 2048. */
+typedef struct csla_cfg {
+    int32_t m;          /* tokens per compressed entry: 4 (CSA) or 128 (HCA) */
+    int32_t D;          /* head dim; the last d_rope dims carry RoPE */
+    int32_t d_rope;     /* 64 */
+    int32_t H;          /* query heads sharing the one KV head */
+    int32_t HI;         /* lightning-indexer heads (CSA) */
+    int32_t dI;         /* index head dim (CSA) */
+    int32_t dc;         /* query latent dim fed to the indexer (CSA) */
+    int32_t n_win;      /* sliding window, 128 */
+    float rope_theta;   /* RoPE base, 10000 */
+    float eps;          /* RMSNorm epsilon, 1e-6 */
+} csla_cfg;
+
+typedef struct csla_cache {
+    uint8_t *rows;
+    float *scales;
+    uint16_t *kidx;            /* CSA only, else NULL */
+    const int32_t *block_table;
+    int32_t bt_stride;
+    int32_t n_pages;
+} csla_cache;
+
+typedef struct csla_state {
+    uint8_t *win_rows;
+    float *win_scales;
+    float *tail_kv;
+    float *tail_idx;           /* CSA only, else NULL */
+    int32_t *len;
+    int32_t n_slots;
+} csla_state;
+
+/* Compressor parameters, device f32 arrays. */
+typedef struct csla_compress_params {
+    const float *gamma_kv;     /* [D]  RMSNorm weight of the KV head */
+    const float *wg;           /* [D]  gate weight of the KV compressor */
+    const float *gb;           /* [m]  gate bias per position in the block */
+    const float *wgi;          /* [dI] gate weight of the index-key compressor (CSA) */
+    const float *gbi;          /* [m]  gate bias of the index-key compressor (CSA) */
+} csla_compress_params;
+
+/*
+ * csla_compress_append -- state-cache and classical-cache update
+ * (硅星人 §两大压缩注意力, CSA/HCA compressor and cache paragraphs; haiqwa
+ * §Partial RoPE位置编码 sliding window; §RMSNorm归一化).
+ * Appends T new tokens to each of the B requests.  For every new token at
+ * position p (p = old len + i): its window row RoPE(RMSNorm(x)*gamma_kv, p),
+ * quantised, goes to ring slot p % n_win; its raw vector joins the tail.
+ * When position p closes block b = p/m (p+1 divisible by m), the block's m raw
+ * rows are pooled with softmax weights of the scalar gate <x_i,wg> + gb[i],
+ * then RMSNorm*gamma_kv, RoPE at position b*m, quantised into compressed entry
+ * b; for CSA the index-key inputs are pooled with their own gate (wgi, gbi)
+ * and stored as bf16.  Finally len += T.
+ *   kv_new   [B][T][D]  dtype kv_dtype (CSLA_F32 or CSLA_BF16)
+ *   kidx_new [B][T][dI] dtype kv_dtype, CSA only (NULL for HCA)
+ * Requires: the block table maps every page the new tokens reach.
+ * Errors: CSLA_ERR_ARG on null/bad sizes; CSLA_ERR_UNSUPPORTED on shapes.
+ */
+int csla_compress_append(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
+                         const int32_t *slots, int32_t B, int32_t T, const void *kv_new,
+                         const void *kidx_new, int32_t kv_dtype, const csla_compress_params *p,
+                         csla_stream_t stream);
+
+/*
+ * csla_indexer_scores -- lightning indexer (硅星人 §两大压缩注意力, CSA part:
+ * the query latent dc is up-projected to HI index heads and scored with ReLU
+ * against the compressed index keys).  For request b with N_vis = len/m
+ * visible entries:
+ *   qI = W_iq . cq[b]  ([HI*dI] = [HI*dI][dc] . [dc], fp32 accumulation),
+ *   scores[b*scores_stride + s] = sum_j head_w[b][j] * max(0, <qI_j, kidx_s>)
+ * for s < N_vis (entries beyond N_vis are not written).  qI enters the tensor
+ * cores as a bf16 hi/lo pair, so scores carry fp32-level error.
+ *   cq [B][dc] (cq_dtype), W_iq [HI*dI][dc] (w_dtype), head_w [B][HI] f32,
+ *   scores f32 [B][scores_stride], scores_stride >= max_len/m.
+ * workspace: csla_workspace_size(cfg, CSLA_OP_INDEXER, B, max_len) bytes.
+ */
+int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
+                        const int32_t *slots, int32_t B, int32_t max_len, const void *cq,
+                        int32_t cq_dtype, const void *W_iq, int32_t w_dtype, const float *head_w,
+                        float *scores, int32_t scores_stride, void *workspace,
+                        size_t workspace_bytes, csla_stream_t stream);
+
+/*
+ * csla_topk_select -- top-k selector (硅星人 §两大压缩注意力, CSA part).
+ * For request b: the min(k, N_vis) entries of largest score (ties: lower
+ * index first), written to idx[b*k ..] in ascending index order, the rest of
+ * the row filled with -1.  Exact: integer radix select on the fp32 bits
+ * (-0.0 counts as +0.0).  scores as produced by csla_indexer_scores.
+ */
+int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *slots, int32_t B,
+                     int32_t max_len, const float *scores, int32_t scores_stride, int32_t k,
+                     int32_t *idx, csla_stream_t stream);
+
+/*
+ * csla_csa_attend -- core MQA of a CSA layer (硅星人 §两大压缩注意力; haiqwa
+ * §RMSNorm归一化, §Partial RoPE位置编码, §让注意力学会"忽略").
+ * For request b at position t = len-1 and head h < H:
+ *   qh = RoPE(RMSNorm(q[b][h]) * gamma_q, t)
+ *   set = compressed entries idx[b][0..k) (entries < 0 skipped), then window
+ *         tokens max(0, len-n_win) .. len-1, each row decoded as above;
+ *   s_j = <qh, x_j>/sqrt(D);  o = sum_j e^{s_j} x_j / (e^{sink[h]} + sum_j e^{s_j}).
+ * One KV head: K = V = the cached row.  Batch invariant: each request's
+ * reduction order is fixed by its own set size, identical for every variant.
+ *   q [B][H][D] (q_dtype), idx int32 [B][k], sink f32 [H], gamma_q f32 [D],
+ *   out [B][H][D] (out_dtype).
+ * variant: CSLA_VARIANT_SATURATED (one CTA walks all chunks of a request),
+ *   CSLA_VARIANT_STARVED (one CTA per chunk, then an ordered combine), or AUTO.
+ * workspace: csla_workspace_size(cfg, CSLA_OP_CSA_ATTEND, B, max_len) with
+ *   max_len here meaning k (the set size is k + n_win).
+ */
+int csla_csa_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
+                    const int32_t *slots, int32_t B, const void *q, int32_t q_dtype,
+                    const int32_t *idx, int32_t k, const float *sink, const float *gamma_q,
+                    void *out, int32_t out_dtype, int32_t variant, void *workspace,
+                    size_t workspace_bytes, csla_stream_t stream);
+
+/*
+ * csla_hca_attend -- core MQA of an HCA layer (硅星人 §两大压缩注意力, HCA part:
+ * no indexer, no top-k; every compressed entry plus the window).  As
+ * csla_csa_attend with set = all N_vis = len/m entries then the window.
+ * workspace: csla_workspace_size(cfg, CSLA_OP_HCA_ATTEND, B, max_len).
+ */
+int csla_hca_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
+                    const int32_t *slots, int32_t B, int32_t max_len, const void *q,
+                    int32_t q_dtype, const float *sink, const float *gamma_q, void *out,
+                    int32_t out_dtype, int32_t variant, void *workspace, size_t workspace_bytes,
+                    csla_stream_t stream);
+
+/* Scratch bytes an entry point needs for B requests (0 for ops with none).
+ * `max_len`: context bound (INDEXER, HCA_ATTEND) or k (CSA_ATTEND). */
+size_t csla_workspace_size(const csla_cfg *cfg, int32_t op, int32_t B, int32_t max_len);
+
+/* Synchronise `stream`, then read and clear the device error word of the
+ * current device.  Returns CSLA_OK, or CSLA_ERR_DEVICE with the CSLA_DEVERR_*
+ * bits in *bits (bits may be NULL), or CSLA_ERR_CUDA. */
+int csla_device_error(csla_stream_t stream, uint32_t *bits);
+
+/* Static text for a status code. */
+const char *csla_strerror(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int csla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSLA_H */

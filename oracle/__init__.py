@@ -319,15 +319,16 @@ def num_threads():
 
 # ---------------------------------------------------------------- expected state after appends
 def expected_append(raw_kv, raw_idx, L0, L1, m, gamma_kv, wg, gb, wgi=None, gbi=None, eps=1e-6,
-                    theta=10000.0, d_rope=64):
+                    theta=10000.0, d_rope=64, window_from=0):
     """Rows the state and classical caches must hold after tokens L0..L1-1 of a
     request are appended (raw_kv/raw_idx hold the whole token history 0..L1-1).
 
     Returns dict: window {pos: (row, scale)}, entries {b: (row, scale)},
-    keys {b: bf16 key} for every block completed by these tokens.
+    keys {b: bf16 key} for every block completed by these tokens.  Window
+    rows are produced for positions >= window_from only.
     """
     out = {"window": {}, "entries": {}, "keys": {}}
-    for p in range(L0, L1):
+    for p in range(max(L0, window_from), L1):
         out["window"][p] = window_row(raw_kv[p], gamma_kv, p, eps, theta, d_rope)
     for b in range(L0 // m, L1 // m):
         if (b + 1) * m <= L0:

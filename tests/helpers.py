@@ -42,7 +42,8 @@ def oracle_cache(w: Workload, lens, params=None, with_raw=False):
         ts = token_stream(w, s, 0, L)
         raws.append(ts)
         exp = oracle.expected_append(ts["kv"], ts.get("idx"), 0, L, w.m, p["gamma_kv"], p["wg"],
-                                     p["gb"], p.get("wgi"), p.get("gbi"), w.eps, w.theta, w.d_rope)
+                                     p["gb"], p.get("wgi"), p.get("gbi"), w.eps, w.theta, w.d_rope,
+                                     window_from=L - w.n_win)
         for pos, (r, sc) in exp["window"].items():
             if pos >= L - w.n_win:
                 win_rows[s, pos % w.n_win] = r

@@ -1,0 +1,67 @@
+"""CPU checks of the C ABI: libcsla.so loads without a GPU, exports every
+entry point include/csla.h declares, and rejects bad arguments on the host
+before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "csla.h")
+
+
+def declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(csla_[a-z_]+)\s*\(", txt)))
+
+
+def test_header_declares_the_five_calls():
+    names = declared()
+    for n in ("csla_compress_append", "csla_indexer_scores", "csla_topk_select", "csla_csa_attend",
+              "csla_hca_attend", "csla_workspace_size", "csla_device_error", "csla_strerror"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    from compressed_sparse_long_append_b200 import csla
+    lib = ctypes.CDLL(csla.LIB_PATH)
+    for n in declared():
+        assert hasattr(lib, n), n
+    assert set(csla.EXPORTS) <= set(declared())
+
+
+def _cfg(**kw):
+    from compressed_sparse_long_append_b200.layer import LayerShape
+    return LayerShape(**kw).cfg()
+
+
+def test_host_argument_checks():
+    from compressed_sparse_long_append_b200 import csla as C
+    L = C._lib
+    cfg = _cfg(m=4)
+    # null structs / pointers -> CSLA_ERR_ARG, no launch
+    assert L.csla_compress_append(ctypes.byref(cfg), None, None, None, 1, 1, None, None, 0, None, None) == C.CSLA_ERR_ARG
+    assert L.csla_topk_select(ctypes.byref(cfg), None, None, 1, 10, None, 10, 5, None, None) == C.CSLA_ERR_ARG
+    assert L.csla_hca_attend(ctypes.byref(_cfg(m=128)), None, None, None, 1, 100, None, 0, None, None, None, 0,
+                             0, None, 0, None) == C.CSLA_ERR_ARG
+    # unsupported shapes
+    for bad in (dict(m=8), dict(m=4, D=256), dict(m=4, d_rope=32), dict(m=4, H=65), dict(m=4, n_win=64)):
+        assert L.csla_topk_select(ctypes.byref(_cfg(**bad)), None, None, 1, 10, None, 10, 5, None, None) \
+            == C.CSLA_ERR_UNSUPPORTED, bad
+    assert L.csla_strerror(C.CSLA_ERR_DEVICE) == b"device-side input error"
+
+
+def test_workspace_sizes():
+    from compressed_sparse_long_append_b200 import csla as C
+    cfg = _cfg(m=4)
+    # indexer: B * NQ * dI bf16 with NQ = 2*HI rounded up to 16
+    assert C.csla_workspace_size(cfg, C.CSLA_OP_INDEXER, 8, 131072) == 8 * 32 * 128 * 2
+    assert C.csla_workspace_size(cfg, C.CSLA_OP_TOPK, 8, 131072) == 0
+    # attention: B * chunks * (H*D + 2H) floats; 512+128 rows -> 3 chunks
+    assert C.csla_workspace_size(cfg, C.CSLA_OP_CSA_ATTEND, 8, 512) == 8 * 3 * (64 * 512 + 128) * 4
+    hca = _cfg(m=128)
+    assert C.csla_workspace_size(hca, C.CSLA_OP_HCA_ATTEND, 4, 1 << 20) == 4 * 32 * (64 * 512 + 128) * 4
+    assert C.csla_workspace_size(_cfg(m=8), C.CSLA_OP_TOPK, 1, 1) == 0
