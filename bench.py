@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--no-hca", action="store_true", help="skip the HCA layer measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", type=int, default=0, help="attention variant: 0 auto, 1 saturated, 2 starved")
+    ap.add_argument("--profile", action="store_true",
+                    help="only the timed CSA steps, bracketed by cudaProfilerStart/Stop (for ncu "
+                         "--profile-from-start off); implies --no-hca --no-cpu-baseline and no e2e leg")
     return ap.parse_args()
 
 
@@ -244,7 +247,7 @@ class HcaStep:
         rec(2)
 
 
-def timed_steps(step, inputs, W, K, n_events, flush, e2e=False):
+def timed_steps(step, inputs, W, K, n_events, flush, e2e=False, profile=False):
     """W warm-up + K timed steps; L2 flushed before every step (outside the
     timed events).  Returns per-step segment times (ms) [K][n_events-1] and
     the whole-step times (ms)."""
@@ -253,6 +256,9 @@ def timed_steps(step, inputs, W, K, n_events, flush, e2e=False):
     for i in range(W + K):
         inp = inputs[i]
         flush.zero_()
+        if profile and i == W:
+            torch.cuda.synchronize()
+            torch.cuda.profiler.start()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
         if e2e:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -270,6 +276,8 @@ def timed_steps(step, inputs, W, K, n_events, flush, e2e=False):
             if i >= W:
                 segs.append([ev[j].elapsed_time(ev[j + 1]) for j in range(n_events - 1)])
                 whole.append(ev[0].elapsed_time(ev[-1]))
+    if profile:
+        torch.cuda.profiler.stop()
     return segs, whole
 
 
@@ -377,7 +385,7 @@ def main():
     torch.cuda.synchronize()
     clk = ClockSampler(local)
     clk.start()
-    segs, whole = timed_steps(step, inputs, W, K, 5, flush)
+    segs, whole = timed_steps(step, inputs, W, K, 5, flush, profile=args.profile)
     torch.cuda.synchronize()
     clocks = clk.stop()
     if world > 1:
@@ -391,17 +399,22 @@ def main():
         ms_step = float(t.item())
 
     # e2e: host buffers, copies inside the timed region (fresh cache state)
-    lb2, cp2, params2 = build_layer(kw, kw["B"], L0, seed, rank, device)
-    step2 = CsaStep(lb2, cp2, params2, kw, args.variant, device)
-    _, whole_e2e = timed_steps(step2, inputs, W, K, 5, flush, e2e=True)
-    ms_e2e = sum(whole_e2e) / len(whole_e2e)
+    if args.profile:
+        args.no_hca = args.no_cpu_baseline = True
+        ms_e2e = float("nan")
+        h2d = d2h = 0
+    else:
+        lb2, cp2, params2 = build_layer(kw, kw["B"], L0, seed, rank, device)
+        step2 = CsaStep(lb2, cp2, params2, kw, args.variant, device)
+        _, whole_e2e = timed_steps(step2, inputs, W, K, 5, flush, e2e=True)
+        ms_e2e = sum(whole_e2e) / len(whole_e2e)
+        h2d = sum(v.numel() * v.element_size() for k, v in inputs[0]["host"].items())
+        d2h = step2.out.numel() * step2.out.element_size()
+        del lb2, step2
     if world > 1:
         t = torch.tensor([ms_e2e], dtype=torch.float64, device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_e2e = float(t.item())
-    h2d = sum(v.numel() * v.element_size() for k, v in inputs[0]["host"].items())
-    d2h = step2.out.numel() * step2.out.element_size()
-    del lb2, step2
 
     # algorithmic bytes of the indexer call (dominant): keys + W_iq + scores
     Ls = [kw["L"] - K + i for i in range(K)]    # context after each timed step's append

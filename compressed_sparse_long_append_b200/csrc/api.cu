@@ -74,7 +74,7 @@ int check_csa_indexer_shape(const csla_cfg *c) {
     return CSLA_OK;
 }
 
-int nq_of(int HI) { return (2 * HI + 15) / 16 * 16; }
+int nq_of(int HI) { return (3 * HI + 15) / 16 * 16; }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? CSLA_OK : CSLA_ERR_CUDA; }
 

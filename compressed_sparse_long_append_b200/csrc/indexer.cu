@@ -8,15 +8,16 @@
 // Two kernels:
 //  1. iq_project: qI = W_iq . cq for every request, one warp per output
 //     feature, W read once per launch for the whole batch; each dot product
-//     has a fixed summation order.  qI is stored as a bf16 pair (hi, lo =
-//     bf16(qI - hi)) so the bf16 tensor-core product carries ~16 bits.
+//     has a fixed summation order.  qI is stored as three bf16 terms
+//     (hi = bf16(qI), mid = bf16(qI - hi), lo = bf16(qI - hi - mid)), so the
+//     bf16 tensor-core products carry the full fp32 value of qI.
 //  2. indexer: persistent, warp-specialised tcgen05 kernel.  A tile is 128
 //     compressed entries of one request (4 pages of 32 entries).  Warp 0
 //     streams key tiles and the request's query operand with TMA into a
 //     4-stage ring; warp 1 issues UMMA (M=128 entries, N=NQ query rows,
 //     K=dI) into one of two TMEM accumulators; warps 2-5 read the
 //     accumulator (one entry per thread) and reduce
-//       score = sum_j w_j * relu(acc[j] + acc[HI + j])
+//       score = sum_j w_j * relu((acc[j] + acc[HI + j]) + acc[2HI + j])
 //     in head order.  Every score depends only on its own entry and request.
 #include "common.cuh"
 #include "kernels.h"
@@ -67,9 +68,12 @@ __global__ void __launch_bounds__(kProjThreads) iq_project_kernel(IndexerArgs a)
         acc = warp_sum(acc);
         if (lane == 0) {
             const uint16_t hi = f32_to_bf16_bits(acc);
-            const uint16_t lo = f32_to_bf16_bits(acc - bf16_bits_to_f32(hi));
+            const float r1 = __fsub_rn(acc, bf16_bits_to_f32(hi));
+            const uint16_t mid = f32_to_bf16_bits(r1);
+            const uint16_t lo = f32_to_bf16_bits(__fsub_rn(r1, bf16_bits_to_f32(mid)));
             a.q_ws[((size_t)b * a.NQ + j) * a.dI + e] = hi;
-            a.q_ws[((size_t)b * a.NQ + a.HI + j) * a.dI + e] = lo;
+            a.q_ws[((size_t)b * a.NQ + a.HI + j) * a.dI + e] = mid;
+            a.q_ws[((size_t)b * a.NQ + 2 * a.HI + j) * a.dI + e] = lo;
         }
     }
 }
@@ -86,6 +90,12 @@ struct IdxSmem {
     static constexpr int kStageBytes = kKeyBytes + kQBytes;
     static constexpr int kBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
 };
+
+// Two accumulators of NQ columns, rounded up to a power of two >= 32.
+template <int NQ>
+constexpr uint32_t kTmemCols() {
+    return 2 * NQ <= 32 ? 32 : (2 * NQ <= 64 ? 64 : 128);
+}
 
 // Tile bookkeeping shared by the three roles (all must skip the same tiles).
 struct TileInfo {
@@ -134,7 +144,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         tma_prefetch_desc(&qmap);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_holder, (2 * NQ) < 32 ? 32 : 2 * NQ);
+        tmem_alloc(tmem_holder, kTmemCols<NQ>());
         tmem_relinquish();
     }
     tc_fence_before();
@@ -225,8 +235,18 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             if (!mbar_wait(tfull + acc, (n / 2) & 1, &abort_flag)) break;
             tc_fence_after();
             uint32_t r[NQ];
-            if constexpr (NQ == 16) tmem_ld32x16(tmem + ((uint32_t)lane_base << 16) + acc * NQ, r);
-            else tmem_ld32x32(tmem + ((uint32_t)lane_base << 16) + acc * NQ, r);
+            const uint32_t ta = tmem + ((uint32_t)lane_base << 16) + acc * NQ;
+            if constexpr (NQ == 16) {
+                tmem_ld32x16(ta, r);
+            } else if constexpr (NQ == 32) {
+                tmem_ld32x32(ta, r);
+            } else {
+                static_assert(NQ == 48, "query operand rows");
+                uint32_t (&r0)[32] = *reinterpret_cast<uint32_t (*)[32]>(r);
+                uint32_t (&r1)[16] = *reinterpret_cast<uint32_t (*)[16]>(r + 32);
+                tmem_ld32x32(ta, r0);
+                tmem_ld32x16(ta + 32, r1);
+            }
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(tempty + acc);
@@ -236,8 +256,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
                 float sc = 0.f;
 #pragma unroll
                 for (int j = 0; j < HI; ++j) {
-                    const float dot = __uint_as_float(r[j]) + __uint_as_float(r[HI + j]);
-                    sc = fmaf(__ldg(w + j), fmaxf(dot, 0.f), sc);
+                    const float dot = __fadd_rn(__fadd_rn(__uint_as_float(r[j]), __uint_as_float(r[HI + j])),
+                                                __uint_as_float(r[2 * HI + j]));
+                    sc = __fmaf_rn(__ldg(w + j), fmaxf(dot, 0.f), sc);
                 }
                 a.scores[(size_t)t.b * a.scores_stride + e] = sc;
             }
@@ -248,7 +269,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, (2 * NQ) < 32 ? 32 : 2 * NQ);
+        tmem_dealloc(tmem, kTmemCols<NQ>());
     }
 }
 
@@ -276,7 +297,7 @@ cudaError_t launch_indexer_t(const IndexerArgs &a, const CUtensorMap &kmap, cons
 
 cudaError_t launch_indexer(const IndexerArgs &a, bool cq_bf16, bool w_bf16, const CUtensorMap &kmap,
                            const CUtensorMap &qmap, int num_sms, cudaStream_t stream) {
-    if (a.NQ > 2 * a.HI) {
+    if (a.NQ > 3 * a.HI) {
         cudaError_t e = cudaMemsetAsync(a.q_ws, 0, (size_t)a.B * a.NQ * a.dI * 2, stream);
         if (e != cudaSuccess) return e;
     }
@@ -290,15 +311,15 @@ cudaError_t launch_indexer(const IndexerArgs &a, bool cq_bf16, bool w_bf16, cons
     // HI is a template parameter so the epilogue's head loop is unrolled.
     if (a.dI == 128) {
         switch (a.HI) {
-            case 16: return launch_indexer_t<128, 32, 16>(a, kmap, qmap, num_sms, stream);
-            case 8: return launch_indexer_t<128, 16, 8>(a, kmap, qmap, num_sms, stream);
+            case 16: return launch_indexer_t<128, 48, 16>(a, kmap, qmap, num_sms, stream);
+            case 8: return launch_indexer_t<128, 32, 8>(a, kmap, qmap, num_sms, stream);
             case 4: return launch_indexer_t<128, 16, 4>(a, kmap, qmap, num_sms, stream);
             default: break;
         }
     } else if (a.dI == 64) {
         switch (a.HI) {
-            case 16: return launch_indexer_t<64, 32, 16>(a, kmap, qmap, num_sms, stream);
-            case 8: return launch_indexer_t<64, 16, 8>(a, kmap, qmap, num_sms, stream);
+            case 16: return launch_indexer_t<64, 48, 16>(a, kmap, qmap, num_sms, stream);
+            case 8: return launch_indexer_t<64, 32, 8>(a, kmap, qmap, num_sms, stream);
             case 4: return launch_indexer_t<64, 16, 4>(a, kmap, qmap, num_sms, stream);
             default: break;
         }

@@ -25,8 +25,8 @@ struct CompressArgs {
 };
 cudaError_t launch_compress_append(const CompressArgs &a, bool bf16, cudaStream_t stream);
 
-// Lightning indexer.  NQ = rows of the bf16 query operand (hi heads, lo
-// heads, zero padding to a multiple of 16).
+// Lightning indexer.  NQ = rows of the bf16 query operand (hi, mid and lo
+// terms of every head, zero padding to a multiple of 16).
 struct IndexerArgs {
     int m, HI, dI, dc, NQ;
     const int32_t *slots;

@@ -93,7 +93,7 @@ enum {
 #define CSLA_PAGE_TOKENS 128
 
 /* Layer shape.  Supported: m in {4, 128}; D in {128, 512}; d_rope = 64;
- * 1 <= H <= 64; n_win = 128; CSA (m = 4): dI in {64, 128}, 1 <= HI <= 16,
+ * 1 <= H <= 64; n_win = 128; CSA (m = 4): dI in {64, 128}, HI in {4, 8, 16},
  * dc a multiple of 8 up to 4096, 1 <= topk <= 2048. */
 typedef struct csla_cfg {
     int32_t m;          /* tokens per compressed entry: 4 (CSA) or 128 (HCA) */
@@ -165,7 +165,7 @@ int csla_compress_append(const csla_cfg *cfg, const csla_state *st, const csla_c
  *   qI = W_iq . cq[b]  ([HI*dI] = [HI*dI][dc] . [dc], fp32 accumulation),
  *   scores[b*scores_stride + s] = sum_j head_w[b][j] * max(0, <qI_j, kidx_s>)
  * for s < N_vis (entries beyond N_vis are not written).  qI enters the tensor
- * cores as a bf16 hi/lo pair, so scores carry fp32-level error.
+ * cores as three bf16 terms (hi, mid, lo), so scores carry fp32-level error.
  *   cq [B][dc] (cq_dtype), W_iq [HI*dI][dc] (w_dtype), head_w [B][HI] f32,
  *   scores f32 [B][scores_stride], scores_stride >= max_len/m.
  * workspace: csla_workspace_size(cfg, CSLA_OP_INDEXER, B, max_len) bytes.

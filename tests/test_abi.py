@@ -57,8 +57,8 @@ def test_host_argument_checks():
 def test_workspace_sizes():
     from compressed_sparse_long_append_b200 import csla as C
     cfg = _cfg(m=4)
-    # indexer: B * NQ * dI bf16 with NQ = 2*HI rounded up to 16
-    assert C.csla_workspace_size(cfg, C.CSLA_OP_INDEXER, 8, 131072) == 8 * 32 * 128 * 2
+    # indexer: B * NQ * dI bf16 with NQ = 3*HI rounded up to 16
+    assert C.csla_workspace_size(cfg, C.CSLA_OP_INDEXER, 8, 131072) == 8 * 48 * 128 * 2
     assert C.csla_workspace_size(cfg, C.CSLA_OP_TOPK, 8, 131072) == 0
     # attention: B * chunks * (H*D + 2H) floats; 512+128 rows -> 3 chunks
     assert C.csla_workspace_size(cfg, C.CSLA_OP_CSA_ATTEND, 8, 512) == 8 * 3 * (64 * 512 + 128) * 4

@@ -75,7 +75,7 @@ def test_every_e4m3_code_widens_exactly():
                  _dev(np.ones(512)), [1])
     assert_no_device_error()
     want = oracle.dequantize(row, 1.0, 512)
-    got = out.cpu().numpy().astype(np.float64)
+    got = out.cpu().numpy().astype(np.float64)[0]
     for h in range(8):
         assert np.array_equal(got[h], want), np.nonzero(got[h] != want)
 

@@ -65,8 +65,9 @@ def test_indexer_matches_oracle(w, lens):
     got_all = scores.cpu().numpy()
     for s, L in enumerate(lens):
         nv = L // w.m
-        ref = oracle_scores(w, cv, s, L, si, p)
-        check_scores(got_all[s, :nv].astype(np.float64), ref)
+        if nv:
+            ref = oracle_scores(w, cv, s, L, si, p)
+            check_scores(got_all[s, :nv].astype(np.float64), ref)
         assert np.all(np.isnan(got_all[s, nv:])), "entries past the visible range were written"
 
 
