@@ -363,7 +363,11 @@ def main():
 
     import torch
     import torch.distributed as dist
-    from compressed_sparse_long_append_b200 import build as cbuild
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "csla_build", os.path.join(ROOT, "compressed_sparse_long_append_b200", "build.py"))
+    cbuild = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(cbuild)
     cbuild.build()
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)

@@ -1,6 +1,6 @@
 """Build libcsla.so (sm_100a) in-tree with nvcc.
 
-    python -m compressed_sparse_long_append_b200.build [--force]
+    python compressed_sparse_long_append_b200/build.py [--force] [--ptxas-v]
 
 The library has no torch dependency: it is plain CUDA C++ behind the C ABI
 of include/csla.h.  Kernels are compiled for sm_100a only.
