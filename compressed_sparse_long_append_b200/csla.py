@@ -19,7 +19,9 @@ CSLA_DEVERR_PAGE, CSLA_DEVERR_INDEX, CSLA_DEVERR_LEN, CSLA_DEVERR_TIMEOUT = 1, 2
 CSLA_PAGE_TOKENS = 128
 
 EXPORTS = ("csla_compress_append", "csla_indexer_scores", "csla_topk_select", "csla_csa_attend",
-           "csla_hca_attend", "csla_workspace_size", "csla_device_error", "csla_strerror", "csla_version")
+           "csla_hca_attend", "csla_workspace_size", "csla_device_error", "csla_strerror", "csla_version",
+           "csla_indexer_scores_noalloc")
+CSLA_NOALLOC_INDEXER_SCRATCH_BYTES = 786432
 
 
 class csla_cfg(ctypes.Structure):
@@ -55,8 +57,8 @@ class CslaError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError("libcsla.so not built (%s); run `python -m "
-                          "compressed_sparse_long_append_b200.build`" % LIB_PATH)
+        raise ImportError("libcsla.so not built (%s); run `python "
+                          "compressed_sparse_long_append_b200/build.py`" % LIB_PATH)
     L = ctypes.CDLL(LIB_PATH)
     P, I, Z = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     sig = {
@@ -69,6 +71,7 @@ def _load():
         "csla_device_error": [P, ctypes.POINTER(ctypes.c_uint32)],
         "csla_strerror": [ctypes.c_int],
         "csla_version": [],
+        "csla_indexer_scores_noalloc": [P, P, P, P, I, I, P, I, P, I, P, P, I, P],
     }
     res = {"csla_workspace_size": ctypes.c_size_t, "csla_strerror": ctypes.c_char_p}
     for name, args in sig.items():
@@ -117,6 +120,17 @@ def csla_indexer_scores(cfg, st, cache, slots, B, max_len, cq, cq_dtype, W_iq, w
     return _check("csla_indexer_scores", _lib.csla_indexer_scores(
         _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, max_len, _ptr(cq), cq_dtype, _ptr(W_iq), w_dtype,
         _ptr(head_w), _ptr(scores), scores_stride, _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def csla_indexer_scores_noalloc(cfg, st, cache, slots, B, max_len, cq, cq_dtype, W_iq, w_dtype, head_w,
+                                scores, scores_stride, stream=None):
+    """The indexer for callers that cannot allocate device memory: same
+    inputs and outputs as csla_indexer_scores, no workspace (the library's
+    fixed scratch array is used; see include/csla.h for the limit and the
+    rule that overlapping calls race)."""
+    return _check("csla_indexer_scores_noalloc", _lib.csla_indexer_scores_noalloc(
+        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, max_len, _ptr(cq), cq_dtype, _ptr(W_iq), w_dtype,
+        _ptr(head_w), _ptr(scores), scores_stride, _stream(stream)))
 
 
 def csla_topk_select(cfg, st, slots, B, max_len, scores, scores_stride, k, idx, stream=None):

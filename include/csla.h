@@ -222,6 +222,32 @@ int csla_hca_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache 
                     int32_t out_dtype, int32_t variant, void *workspace, size_t workspace_bytes,
                     csla_stream_t stream);
 
+/*
+ * csla_indexer_scores_noalloc -- csla_indexer_scores for callers that cannot
+ * allocate device memory.  The pages have no counterpart: this is an
+ * interface convenience, not a step of the method.
+ * Some callers cannot call cudaMalloc at all (a framework that owns and has
+ * reserved the whole memory pool, code running inside an allocator hook or
+ * a host callback, an embedding restricted to the buffers it was given).
+ * This entry point takes the same inputs and outputs as csla_indexer_scores
+ * but no workspace: its scratch is one fixed array of
+ * CSLA_NOALLOC_INDEXER_SCRATCH_BYTES inside the library, present on every
+ * GPU that loads libcsla until the process exits.  Limit: B * NQ * dI * 2
+ * bytes <= CSLA_NOALLOC_INDEXER_SCRATCH_BYTES, NQ = 3*HI rounded up to 16
+ * (64 requests at HI = 16, dI = 128); larger batches return CSLA_ERR_ARG
+ * without launching.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current); make that first
+ * call before any stream capture.  Every call shares the array: calls that
+ * overlap on the GPU race on it, calls ordered on one stream do not.  It
+ * calls no allocation routine.
+ */
+#define CSLA_NOALLOC_INDEXER_SCRATCH_BYTES 786432
+int csla_indexer_scores_noalloc(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
+                                const int32_t *slots, int32_t B, int32_t max_len, const void *cq,
+                                int32_t cq_dtype, const void *W_iq, int32_t w_dtype,
+                                const float *head_w, float *scores, int32_t scores_stride,
+                                csla_stream_t stream);
+
 /* Scratch bytes an entry point needs for B requests (0 for ops with none).
  * `max_len`: context bound (INDEXER, HCA_ATTEND) or k (CSA_ATTEND). */
 size_t csla_workspace_size(const csla_cfg *cfg, int32_t op, int32_t B, int32_t max_len);
