@@ -34,7 +34,9 @@ UNIT = "tokens/s"
 CSA = dict(B=8, L=131072, m=4, H=64, D=512, HI=16, dI=128, dc=1024, k=512, n_win=128)
 HCA = dict(B=4, L=1048576, m=128, H=64, D=512, n_win=128)
 CHUNK = 16384          # tokens per compress call while building the caches
-FLUSH_BYTES = 512 << 20
+CSA_COPIES = 4         # layer copies rotated per step: 4 x ~75 MB touched > 2 x L2
+HCA_COPIES = 14        # 14 x ~19.3 MB
+HEADROOM = 256         # cache capacity beyond the nominal context (tokens appended while timing)
 
 
 def parse():
@@ -113,9 +115,9 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ workload build
-def build_layer(shape_kw, n_req, L0, seed, rank, device):
-    """Caches of n_req requests after appending L0 tokens each, through
-    csla_compress_append on raw streams generated on the device."""
+def build_layer(shape_kw, n_req, L0s, seed, rank, device):
+    """Caches of n_req requests after appending L0s[r] tokens to request r,
+    through csla_compress_append on raw streams generated on the device."""
     import torch
     from compressed_sparse_long_append_b200 import csla as C
     from compressed_sparse_long_append_b200.layer import CompressParams, LayerBuffers, LayerShape
@@ -124,7 +126,7 @@ def build_layer(shape_kw, n_req, L0, seed, rank, device):
 
     sh = LayerShape(m=shape_kw["m"], D=shape_kw["D"], H=shape_kw["H"], HI=shape_kw.get("HI", 16),
                     dI=shape_kw.get("dI", 128), dc=shape_kw.get("dc", 1024), n_win=shape_kw["n_win"])
-    L_cap = shape_kw["L"]
+    L_cap = shape_kw["L"] + HEADROOM
     pages_per = -(-L_cap // 128)
     n_pages = n_req * pages_per
     lb = LayerBuffers(sh, n_req, n_pages, pages_per, device)
@@ -137,8 +139,8 @@ def build_layer(shape_kw, n_req, L0, seed, rank, device):
                         g("gbi", (m,)) if sh.is_csa else None, device)
     for r in range(n_req):
         slots = torch.tensor([r], dtype=torch.int32, device=device)
-        for a in range(0, L0, CHUNK):
-            b = min(L0, a + CHUNK)
+        for a in range(0, L0s[r], CHUNK):
+            b = min(L0s[r], a + CHUNK)
             kv = torch_gen.normal(seed, "kv/%d/%d" % (rank, r), (b - a, D), start=a * D, device=device) \
                 .to(torch.bfloat16)
             ki = torch_gen.normal(seed, "idx/%d/%d" % (rank, r), (b - a, dI), start=a * dI, device=device) \
@@ -175,6 +177,9 @@ def step_inputs(shape_kw, n_req, n_steps, seed, rank, device):
 
 
 class CsaStep:
+    """One CSA decode step of one layer copy as four library calls; each call
+    takes the step's input tensors x (dict of device tensors)."""
+
     def __init__(self, lb, cp, params, kw, variant, device):
         import torch
         from compressed_sparse_long_append_b200 import csla as C
@@ -182,7 +187,7 @@ class CsaStep:
         B = kw["B"]
         self.B = B
         self.slots = torch.arange(B, dtype=torch.int32, device=device)
-        self.max_len = kw["L"]
+        self.max_len = kw["L"] + HEADROOM
         self.stride = self.max_len // kw["m"]
         self.scores = torch.zeros((B, self.stride), dtype=torch.float32, device=device)
         self.idx = torch.zeros((B, kw["k"]), dtype=torch.int32, device=device)
@@ -193,33 +198,47 @@ class CsaStep:
         self.ws_i = torch.zeros(self.wsi, dtype=torch.uint8, device=device)
         self.ws_a = torch.zeros(self.wsa, dtype=torch.uint8, device=device)
         self.cfg, self.st, self.cache, self.cps = cfg, lb.state(), lb.cache(), cp.struct()
+        self.names = ["compress_append", "indexer_scores", "topk_select", "csa_attend"]
+        self.calls = [self._compress, self._indexer, self._topk, self._attend]
 
-    def run(self, inp, ev=None):
+    def _compress(self, x):
         C = self.C
-        rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
-        rec(0)
-        C.csla_compress_append(self.cfg, self.st, self.cache, self.slots, self.B, 1, inp["kv"], inp["kidx"],
+        C.csla_compress_append(self.cfg, self.st, self.cache, self.slots, self.B, 1, x["kv"], x["kidx"],
                                C.CSLA_BF16, self.cps)
-        rec(1)
-        C.csla_indexer_scores(self.cfg, self.st, self.cache, self.slots, self.B, self.max_len, inp["cq"],
-                              C.CSLA_BF16, self.p["W_iq"], C.CSLA_BF16, inp["head_w"], self.scores, self.stride,
+
+    def _indexer(self, x):
+        C = self.C
+        C.csla_indexer_scores(self.cfg, self.st, self.cache, self.slots, self.B, self.max_len, x["cq"],
+                              C.CSLA_BF16, self.p["W_iq"], C.CSLA_BF16, x["head_w"], self.scores, self.stride,
                               self.ws_i, self.wsi)
-        rec(2)
-        C.csla_topk_select(self.cfg, self.st, self.slots, self.B, self.max_len, self.scores, self.stride,
-                           self.kw["k"], self.idx)
-        rec(3)
-        C.csla_csa_attend(self.cfg, self.st, self.cache, self.slots, self.B, inp["q"], C.CSLA_BF16, self.idx,
+
+    def _topk(self, x):
+        self.C.csla_topk_select(self.cfg, self.st, self.slots, self.B, self.max_len, self.scores, self.stride,
+                                self.kw["k"], self.idx)
+
+    def _attend(self, x):
+        C = self.C
+        C.csla_csa_attend(self.cfg, self.st, self.cache, self.slots, self.B, x["q"], C.CSLA_BF16, self.idx,
                           self.kw["k"], self.p["sink"], self.p["gamma_q"], self.out, C.CSLA_BF16, self.variant,
                           self.ws_a, self.wsa)
-        rec(4)
 
     def launches(self):
-        # compress, iq_project, indexer, topk, attend (+ combine when starved)
-        starved = self.variant == 2 or (self.variant == 0 and self.B < 148)
-        return 5 + (1 if starved else 0)
+        return csa_launches(self.kw, self.variant)
+
+
+def csa_launches(kw, variant):
+    """Kernels of one CSA step: compress (pool + tail/len), iq_project +
+    indexer, topk, prep_q + attend, + combine unless the saturated variant
+    runs (forced, or automatic: one chunk per request or B >= SM count)."""
+    rows = kw["k"] + kw["n_win"]
+    chunks = -(-rows // (64 * -(-rows // 2048)))
+    saturated = variant == 1 or (variant == 0 and (kw["B"] >= 148 or chunks <= 1))
+    return 2 + 2 + 1 + 2 + (0 if saturated else 1)
 
 
 class HcaStep:
+    """One HCA decode step: compress_append then hca_attend."""
+
     def __init__(self, lb, cp, params, kw, variant, device):
         import torch
         from compressed_sparse_long_append_b200 import csla as C
@@ -227,58 +246,157 @@ class HcaStep:
         B = kw["B"]
         self.B = B
         self.slots = torch.arange(B, dtype=torch.int32, device=device)
-        self.max_len = kw["L"]
+        self.max_len = kw["L"] + HEADROOM
         self.out = torch.zeros((B, kw["H"], kw["D"]), dtype=torch.bfloat16, device=device)
         cfg = lb.cfg()
         self.wsa = C.csla_workspace_size(cfg, C.CSLA_OP_HCA_ATTEND, B, self.max_len)
         self.ws_a = torch.zeros(self.wsa, dtype=torch.uint8, device=device)
         self.cfg, self.st, self.cache, self.cps = cfg, lb.state(), lb.cache(), cp.struct()
+        self.names = ["compress_append", "hca_attend"]
+        self.calls = [self._compress, self._attend]
 
-    def run(self, inp, ev=None):
+    def _compress(self, x):
         C = self.C
-        rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
-        rec(0)
-        C.csla_compress_append(self.cfg, self.st, self.cache, self.slots, self.B, 1, inp["kv"], None,
+        C.csla_compress_append(self.cfg, self.st, self.cache, self.slots, self.B, 1, x["kv"], None,
                                C.CSLA_BF16, self.cps)
-        rec(1)
-        C.csla_hca_attend(self.cfg, self.st, self.cache, self.slots, self.B, self.max_len, inp["q"], C.CSLA_BF16,
+
+    def _attend(self, x):
+        C = self.C
+        C.csla_hca_attend(self.cfg, self.st, self.cache, self.slots, self.B, self.max_len, x["q"], C.CSLA_BF16,
                           self.p["sink"], self.p["gamma_q"], self.out, C.CSLA_BF16, self.variant, self.ws_a,
                           self.wsa)
-        rec(2)
 
 
-def timed_steps(step, inputs, W, K, n_events, flush, e2e=False, profile=False):
-    """W warm-up + K timed steps; L2 flushed before every step (outside the
-    timed events).  Returns per-step segment times (ms) [K][n_events-1] and
-    the whole-step times (ms)."""
+def clone_layer(lb, params):
+    """An independent copy of a layer's device buffers and weights (the
+    rotation below walks several such copies, like the layers of a model)."""
+    from compressed_sparse_long_append_b200.layer import LayerBuffers
+    nb = object.__new__(LayerBuffers)
+    nb.__dict__.update(lb.__dict__)
+    for k in ("rows", "scales", "kidx", "block_table", "win_rows", "win_scales", "tail_kv", "tail_idx", "len"):
+        v = getattr(lb, k)
+        setattr(nb, k, None if v is None else v.clone())
+    return nb, {k: v.clone() for k, v in params.items()}
+
+
+def make_copies(step_cls, lb, cp, params, kw, variant, device, R):
+    """R steps over R independent layer copies."""
+    steps = [step_cls(lb, cp, params, kw, variant, device)]
+    for _ in range(R - 1):
+        nb, np_ = clone_layer(lb, params)
+        steps.append(step_cls(nb, cp, np_, kw, variant, device))
+    return steps
+
+
+def capture(fn):
     import torch
-    segs, whole = [], []
-    for i in range(W + K):
-        inp = inputs[i]
-        flush.zero_()
-        if profile and i == W:
-            torch.cuda.synchronize()
-            torch.cuda.profiler.start()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def run_steps(steps, inputs, W, K, e2e=False, profile=False):
+    """W warm-up steps (direct calls), then K timed steps back to back.
+    Step i runs on layer copy i % R with inputs[i]: the R copies together
+    touch more than twice the L2 per rotation, so every step starts with its
+    caches out of L2 (no flush writes needed).  Each timed step is one CUDA
+    graph holding all of the step's library calls, captured beforehand; the
+    K replays are bracketed by one pair of events after a synchronize.
+    e2e: every step also copies its inputs from pinned host memory into the
+    device buffers the graph reads and copies its output back to pinned
+    host memory, both inside the timed region.  Returns ms per step."""
+    import torch
+    R = len(steps)
+    for i in range(W):
+        st = steps[i % R]
+        for c in st.calls:
+            c(inputs[i])
+    torch.cuda.synchronize()
+    graphs = []
+    for i in range(W, W + K):
+        st, x = steps[i % R], inputs[i]
+        graphs.append(capture(lambda: [c(x) for c in st.calls]))
+    outs = [torch.empty_like(steps[i % R].out, device="cpu").pin_memory() for i in range(W, W + K)] if e2e else None
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if profile:
+        torch.cuda.profiler.start()
+    e0.record()
+    for j, i in enumerate(range(W, W + K)):
         if e2e:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            dev = {k: inp[k].copy_(inp["host"][k], non_blocking=True) for k in inp if k != "host"}
-            step.run(dev, ev)
-            out_h = step.out.to("cpu", non_blocking=True)
-            e1.record()
-            torch.cuda.synchronize()
-            if i >= W:
-                whole.append(e0.elapsed_time(e1))
+            x = inputs[i]
+            for k, v in x["host"].items():
+                x[k].copy_(v, non_blocking=True)
+            graphs[j].replay()
+            outs[j].copy_(steps[i % R].out, non_blocking=True)
         else:
-            step.run(inp, ev)
-            torch.cuda.synchronize()
-            if i >= W:
-                segs.append([ev[j].elapsed_time(ev[j + 1]) for j in range(n_events - 1)])
-                whole.append(ev[0].elapsed_time(ev[-1]))
+            graphs[j].replay()
+    e1.record()
+    torch.cuda.synchronize()
     if profile:
         torch.cuda.profiler.stop()
-    return segs, whole
+    del graphs
+    return e0.elapsed_time(e1) / K
+
+
+def breakdown(steps, inputs, W, K):
+    """Per-call times (ms): each call of each copy captured as its own graph,
+    one event pair around each replay (includes one graph launch each, so
+    the parts add up to more than the pipelined step)."""
+    import torch
+    R = len(steps)
+    n = len(steps[0].calls)
+    graphs = [[capture(lambda c=c, x=inputs[W + r]: c(x)) for c in steps[r].calls] for r in range(R)]
+    torch.cuda.synchronize()
+    segs = []
+    for i in range(K):
+        gl = graphs[i % R]
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+        ev[0].record()
+        for j, g in enumerate(gl):
+            g.replay()
+            ev[j + 1].record()
+        torch.cuda.synchronize()
+        segs.append([ev[j].elapsed_time(ev[j + 1]) for j in range(n)])
+    del graphs
+    return [sum(x[j] for x in segs) / len(segs) for j in range(n)]
+
+
+def call_time(steps, inputs, W, K, j):
+    """Average duration (ms) of call j alone: its graphs (one per copy,
+    rotating, so the call's inputs start out of L2) replayed K times back to
+    back between one event pair.  Call j must only read the caches."""
+    import torch
+    R = len(steps)
+    graphs = [capture(lambda r=r: steps[r].calls[j](inputs[W + r])) for r in range(R)]
+    for r in range(R):
+        graphs[r].replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(K):
+        graphs[i % R].replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del graphs
+    return e0.elapsed_time(e1) / K
+
+
+def indexer_traffic():
+    """DRAM bytes per indexer launch from the committed ncu summary, if it
+    was taken on the current kernel source (else None)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)["csla_indexer_scores"]
+        h = hashlib.sha256()
+        for name in t["sources"]:
+            with open(os.path.join(ROOT, name), "rb") as f:
+                h.update(f.read())
+        return float(t["bytes_per_call"]) if h.hexdigest() == t["sha256"] else None
+    except Exception:
+        return None
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
@@ -379,75 +497,74 @@ def main():
 
     # ---------------- CSA layer (the headline workload)
     kw = dict(CSA)
-    L0 = kw["L"] - (W + K)
-    lb, cp, params = build_layer(kw, kw["B"], L0, seed, rank, device)
-    inputs = step_inputs(kw, kw["B"], W + K, seed, rank, device)
-    step = CsaStep(lb, cp, params, kw, args.variant, device)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    R, m, B = CSA_COPIES, kw["m"], kw["B"]
+    # request b starts b % m tokens short, so B/m requests close a block every step
+    before = -(-(W + K) // R)
+    L0s = [kw["L"] - before - (b % m) for b in range(B)]
+    lb, cp, params = build_layer(kw, B, L0s, seed, rank, device)
+    inputs = step_inputs(kw, B, W + K, seed, rank, device)
+    steps = make_copies(CsaStep, lb, cp, params, kw, args.variant, device, R)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clk = ClockSampler(local)
     clk.start()
-    segs, whole = timed_steps(step, inputs, W, K, 5, flush, profile=args.profile)
-    torch.cuda.synchronize()
+    ms_step = run_steps(steps, inputs, W, K, profile=args.profile)
     clocks = clk.stop()
     if world > 1:
         dist.barrier()
-    ms_step = sum(whole) / len(whole)
-    ms_idx = sum(s[1] for s in segs) / len(segs)
-    ms_seg = [sum(s[j] for s in segs) / len(segs) for j in range(4)]
-    if world > 1:
         t = torch.tensor([ms_step], dtype=torch.float64, device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_step = float(t.item())
 
-    # e2e: host buffers, copies inside the timed region (fresh cache state)
     if args.profile:
         args.no_hca = args.no_cpu_baseline = True
-        ms_e2e = float("nan")
-        h2d = d2h = 0
+        ms_e2e, h2d, d2h, seg, ms_idx = float("nan"), 0, 0, [float("nan")] * 4, float("nan")
     else:
-        lb2, cp2, params2 = build_layer(kw, kw["B"], L0, seed, rank, device)
-        step2 = CsaStep(lb2, cp2, params2, kw, args.variant, device)
-        _, whole_e2e = timed_steps(step2, inputs, W, K, 5, flush, e2e=True)
-        ms_e2e = sum(whole_e2e) / len(whole_e2e)
+        # e2e: the same steps again (contexts grow by another K/R tokens), host buffers
+        ms_e2e = run_steps(steps, inputs, W, K, e2e=True)
         h2d = sum(v.numel() * v.element_size() for k, v in inputs[0]["host"].items())
-        d2h = step2.out.numel() * step2.out.element_size()
-        del lb2, step2
+        d2h = steps[0].out.numel() * steps[0].out.element_size()
+        seg = breakdown(steps, inputs, W, K)
+        ms_idx = call_time(steps, inputs, W, K, 1)
     if world > 1:
         t = torch.tensor([ms_e2e], dtype=torch.float64, device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_e2e = float(t.item())
 
-    # algorithmic bytes of the indexer call (dominant): keys + W_iq + scores
-    Ls = [kw["L"] - K + i for i in range(K)]    # context after each timed step's append
-    nv_mean = sum(L // kw["m"] for L in Ls) / K
-    idx_bytes = kw["B"] * nv_mean * (kw["dI"] * 2 + 4) + kw["HI"] * kw["dI"] * kw["dc"] * 2
+    # algorithmic bytes of one indexer call: every visible key (dI bf16) read
+    # once, one f32 score written per key, W_iq read once
+    nv = sum(int(x) // m for st in steps for x in st.lb.len.tolist()) / R
+    idx_bytes = nv * (kw["dI"] * 2 + 4) + kw["HI"] * kw["dI"] * kw["dc"] * 2
     peak, peak_kind = peaks()
     achieved = idx_bytes / (ms_idx * 1e-3) / 1e9
 
     hca = None
     if not args.no_hca:
-        del step, lb
+        del steps, lb
         torch.cuda.empty_cache()
         hk = dict(HCA)
-        hL0 = hk["L"] - (W + K)
-        hlb, hcp, hparams = build_layer(hk, hk["B"], hL0, seed + 1, rank, device)
-        hin = step_inputs(hk, hk["B"], W + K, seed + 1, rank, device)
-        hstep = HcaStep(hlb, hcp, hparams, hk, args.variant, device)
-        hsegs, hwhole = timed_steps(hstep, hin, W, K, 3, flush)
-        hms = sum(hwhole) / len(hwhole)
-        hms_att = sum(s[1] for s in hsegs) / len(hsegs)
-        rows = hk["L"] // hk["m"] + hk["n_win"]
-        hbytes = hk["B"] * (rows * (hk["D"] + 64 + 4) + 2 * hk["H"] * hk["D"] * 2)
-        hflops = hk["B"] * rows * hk["H"] * hk["D"] * 4
-        hca = {"workload": "hca_decode_B4_L1048576", "tokens_per_s": hk["B"] / (hms * 1e-3),
+        HR, hm, hB = HCA_COPIES, hk["m"], hk["B"]
+        # requests staggered 16 tokens apart inside one block, clear of its end:
+        # with fewer than ~78 appends per copy no block closes during the run
+        # (in steady decode one closes every 128 steps per request)
+        hL0s = [hk["L"] - 127 + 16 * b for b in range(hB)]
+        closes = sum(1 for i in range(W, W + K) for b in range(hB) if (hL0s[b] + i // HR + 1) % hm == 0)
+        hlb, hcp, hparams = build_layer(hk, hB, hL0s, seed + 1, rank, device)
+        hin = step_inputs(hk, hB, W + K, seed + 1, rank, device)
+        hsteps = make_copies(HcaStep, hlb, hcp, hparams, hk, args.variant, device, HR)
+        hms = run_steps(hsteps, hin, W, K)
+        hms_att = call_time(hsteps, hin, W, K, 1)
+        rows = sum(int(x) // hm for x in hsteps[0].lb.len.tolist()) / hB + hk["n_win"]
+        hbytes = hB * (rows * (hk["D"] + 64 + 4) + 2 * hk["H"] * hk["D"] * 2)
+        hflops = hB * rows * hk["H"] * hk["D"] * 4
+        hca = {"workload": "hca_decode_B4_L1048576", "tokens_per_s": hB / (hms * 1e-3),
                "ms_per_step": hms, "attend_ms": hms_att,
                "attend_hbm_gbs": hbytes / (hms_att * 1e-3) / 1e9,
                "attend_hbm_frac": hbytes / (hms_att * 1e-3) / 1e9 / peak,
                "attend_tflops": hflops / (hms_att * 1e-3) / 1e12,
-               "attend_tensor_frac_sustained": hflops / (hms_att * 1e-3) / 1e12 / 1395.7}
+               "attend_tensor_frac_sustained": hflops / (hms_att * 1e-3) / 1e12 / 1395.7,
+               "block_closes_in_timed_steps": closes}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -461,27 +578,32 @@ def main():
             cpu = {"value": None, "unit": UNIT, "cores": 0, "kind": "oracle", "sample": "failed: %s" % e}
 
     if rank == 0:
-        B = kw["B"]
+        launches_per_step = csa_launches(kw, args.variant)
         line = {
             "metric": METRIC, "value": B * world / (ms_step * 1e-3), "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded splitmix64 / Box-Muller token streams, caches built by csla_compress_append)",
             "config": {"workload": "csa_decode_B8_L131072", "requests_per_gpu": B, "context": kw["L"],
+                       "context_stagger": "request b is b %% %d tokens shorter: %d of %d requests close a "
+                                          "block every step" % (m, B // m, B),
                        "m": 4, "compressed_entries": kw["L"] // 4, "heads": 64, "head_dim": 512,
                        "index_heads": 16, "index_dim": 128, "dc": 1024, "topk": 512, "window": 128,
-                       "l2": "flushed before every step (512 MiB write, outside the timed events)",
+                       "l2": "inputs larger than L2: %d rotating copies of the layer (caches + W_iq), "
+                             "~%d MB touched per rotation vs 126 MB L2" % (R, R * 75),
+                       "launch": "one CUDA graph per step (all four library calls), K graphs replayed back to "
+                                 "back between one event pair",
                        "parallelism": "dp%d over requests" % world, "variant": args.variant},
-            "segments_ms": {"compress_append": ms_seg[0], "indexer_scores": ms_seg[1], "topk_select": ms_seg[2],
-                            "csa_attend": ms_seg[3]},
+            "segments_ms": {"compress_append": seg[0], "indexer_scores": seg[1], "topk_select": seg[2],
+                            "csa_attend": seg[3], "note": "one graph launch per call, serialised"},
             "roofline": {"bound": "hbm", "kernel": "csla_indexer_scores (iq_project + indexer)",
                          "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                         "peak_kind": peak_kind, "traffic": None,
-                         "algorithmic_bytes": idx_bytes},
+                         "peak_kind": peak_kind, "traffic": indexer_traffic(),
+                         "algorithmic_bytes": idx_bytes, "call_ms": ms_idx},
             "cpu_baseline": cpu,
-            "e2e": {"value": kw["B"] * world / (ms_e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "e2e": {"value": B * world / (ms_e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": step_launches_total(K),
+            "gpu_launches": launches_per_step * K,
             "clocks": clocks,
             "hca_decode": hca,
         }
@@ -489,11 +611,6 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
-
-
-def step_launches_total(K):
-    # per CSA step: compress, iq_project, indexer, topk, attend, combine
-    return 6 * K
 
 
 if __name__ == "__main__":

@@ -1,6 +1,10 @@
 """Build libcsla.so (sm_100a) in-tree with nvcc.
 
     python compressed_sparse_long_append_b200/build.py [--force] [--ptxas-v]
+    python compressed_sparse_long_append_b200/build.py --timeline OUT.so
+
+The second form builds a separate library with the device timeline hooks
+compiled in (-DCSLA_TIMELINE, csla_timeline_read/clear exported).
 
 The library has no torch dependency: it is plain CUDA C++ behind the C ABI
 of include/csla.h.  Kernels are compiled for sm_100a only.
@@ -50,6 +54,15 @@ def build(force=False, verbose=False, extra=()):
     return LIB
 
 
+def build_timeline(out):
+    cmd = [NVCC, *FLAGS, "-DCSLA_TIMELINE", "-shared", "-o", out, *sources()]
+    subprocess.run(cmd, check=True)
+    return out
+
+
 if __name__ == "__main__":
+    if "--timeline" in sys.argv:
+        print(build_timeline(os.path.abspath(sys.argv[sys.argv.index("--timeline") + 1])))
+        sys.exit(0)
     extra = ["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else []
     print(build(force="--force" in sys.argv or bool(extra), verbose=True, extra=extra))

@@ -1,5 +1,6 @@
 // api.cu -- the C ABI of libcsla (declared in include/csla.h): host-side
 // argument checks, TMA descriptor encoding and kernel launches.
+#include <math.h>
 #include <string.h>
 
 #include "../../include/csla.h"
@@ -78,16 +79,45 @@ int nq_of(int HI) { return (3 * HI + 15) / 16 * 16; }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? CSLA_OK : CSLA_ERR_CUDA; }
 
+// Attention workspace: per request the 64-head Qhat image (64*D bf16), then
+// the chunk partials (H*D + 2H floats per chunk).
+size_t attend_q_bytes(const csla_cfg *c, int B) { return (size_t)B * 64 * c->D * 2; }
 size_t attend_ws(const csla_cfg *c, int B, long long max_rows) {
     const size_t per = ((size_t)c->H * c->D + 2 * (size_t)c->H) * sizeof(float);
-    return (size_t)B * attend_max_chunks(max_rows) * per;
+    return attend_q_bytes(c, B) + (size_t)B * attend_max_chunks(max_rows) * per;
 }
 
 }  // namespace
 
+#ifdef CSLA_TIMELINE
+namespace csla {
+__device__ TimelineRec g_timeline[kTimelineCap];
+__device__ unsigned int g_timeline_n = 0;
+}  // namespace csla
+#endif
+
 extern "C" {
 
 int csla_version(void) { return 100; }
+
+#ifdef CSLA_TIMELINE
+int csla_timeline_read(void *records, size_t bytes, uint32_t *count) {
+    unsigned int n = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return CSLA_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&n, csla::g_timeline_n, sizeof(n)) != cudaSuccess) return CSLA_ERR_CUDA;
+    if (n > csla::kTimelineCap) n = csla::kTimelineCap;
+    size_t want = (size_t)n * sizeof(csla::TimelineRec);
+    if (want > bytes) want = bytes / sizeof(csla::TimelineRec) * sizeof(csla::TimelineRec);
+    if (want && cudaMemcpyFromSymbol(records, csla::g_timeline, want) != cudaSuccess) return CSLA_ERR_CUDA;
+    if (count) *count = (uint32_t)(want / sizeof(csla::TimelineRec));
+    return CSLA_OK;
+}
+int csla_timeline_clear(void) {
+    unsigned int zero = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return CSLA_ERR_CUDA;
+    return cudaMemcpyToSymbol(csla::g_timeline_n, &zero, sizeof(zero)) == cudaSuccess ? CSLA_OK : CSLA_ERR_CUDA;
+}
+#endif
 
 const char *csla_strerror(int s) {
     switch (s) {
@@ -135,14 +165,18 @@ int csla_compress_append(const csla_cfg *cfg, const csla_state *st, const csla_c
         !cache->block_table || cache->bt_stride < 1 || cache->n_pages < 1)
         return CSLA_ERR_ARG;
     if (!p->gamma_kv || !p->wg || !p->gb) return CSLA_ERR_ARG;
+    if (!aligned16(st->tail_kv)) return CSLA_ERR_ARG;
     const bool csa = cfg->m == 4;
     if (csa) {
-        if (cfg->dI < 1 || cfg->dI > 512 || !kidx_new || !cache->kidx || !st->tail_idx || !p->wgi || !p->gbi)
+        if (cfg->dI < 4 || cfg->dI > 512 || cfg->dI % 4 || !kidx_new || !cache->kidx || !st->tail_idx || !p->wgi ||
+            !p->gbi)
             return CSLA_ERR_ARG;
+        if (!aligned16(st->tail_idx)) return CSLA_ERR_ARG;
     }
     CompressArgs a{};
     a.m = cfg->m; a.D = cfg->D; a.d_rope = cfg->d_rope; a.dI = csa ? cfg->dI : 0; a.n_win = cfg->n_win;
     a.theta = cfg->rope_theta; a.eps = cfg->eps;
+    a.freq = rope_freq(cfg->rope_theta, cfg->d_rope);
     a.slots = slots; a.B = B; a.T = T;
     a.kv_new = kv_new; a.kidx_new = csa ? kidx_new : nullptr;
     a.gamma_kv = p->gamma_kv; a.wg = p->wg; a.gb = p->gb; a.wgi = p->wgi; a.gbi = p->gbi;
@@ -212,16 +246,19 @@ static int attend_common(const csla_cfg *cfg, const csla_state *st, const csla_c
     if ((q_dtype != CSLA_F32 && q_dtype != CSLA_BF16) || (out_dtype != CSLA_F32 && out_dtype != CSLA_BF16))
         return CSLA_ERR_ARG;
     if (variant < CSLA_VARIANT_AUTO || variant > CSLA_VARIANT_STARVED) return CSLA_ERR_ARG;
-    if (!aligned16(q) || !aligned16(cache->rows) || !aligned16(st->win_rows)) return CSLA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(cache->rows) || !aligned16(st->win_rows) || !aligned16(workspace))
+        return CSLA_ERR_ARG;
     AttendArgs a{};
     a.m = cfg->m; a.D = cfg->D; a.d_rope = cfg->d_rope; a.H = cfg->H; a.n_win = cfg->n_win;
     a.theta = cfg->rope_theta; a.eps = cfg->eps;
+    a.freq = rope_freq(cfg->rope_theta, cfg->d_rope);
     a.slots = slots; a.len = st->len; a.B = B; a.q = q; a.idx = idx; a.k = idx ? k : 0;
     a.sink = sink; a.gamma_q = gamma_q;
     a.rows = cache->rows; a.scales = cache->scales; a.block_table = cache->block_table;
     a.bt_stride = cache->bt_stride; a.n_pages = cache->n_pages; a.n_slots = st->n_slots;
     a.win_rows = st->win_rows; a.win_scales = st->win_scales; a.out = out;
-    a.part = reinterpret_cast<float *>(workspace);
+    a.qimg = reinterpret_cast<uint8_t *>(workspace);
+    a.part = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + attend_q_bytes(cfg, B));
     const long long max_rows = idx ? (long long)k + cfg->n_win : (long long)max_len / cfg->m + cfg->n_win;
     a.max_chunks = attend_max_chunks(max_rows);
     a.max_len = max_len;

@@ -11,33 +11,44 @@
 // Canonical reduction.  A request's attention set (n rows: compressed
 // entries, then window tokens, in that order) is cut into chunks of
 // attend_chunk_rows(n) rows -- a function of n alone.  Each chunk yields a
-// partial (running max m, sum l, unnormalised O) computed by chunk_pass();
-// the partials are folded left to right, starting from the sink, by
-// fold_store().  The saturated kernel walks all chunks of a request in one
-// CTA and folds at the end; the starved kernel gives every chunk its own CTA
-// and a combine kernel folds.  Both run the same two functions on the same
-// data, so their outputs are identical bit for bit, and nothing depends on
-// which other requests share the launch.
+// partial (running max m, sum l, unnormalised O); fold_weights()/fold_dim()
+// combine them with the sink in chunk order.  The saturated kernel walks
+// all chunks of a request in one CTA and folds at the end; the starved kernel
+// gives every chunk its own CTA and a combine kernel folds.  Both run the
+// same code on the same data, so their outputs are identical bit for bit,
+// and nothing depends on which other requests share the launch.
 //
-// Per 64-row tile of a chunk (one CTA = 128 threads, warp 0 lane 0 issues UMMA):
-//   X  [64 rows x D] bf16 in smem (fp8 codes widened exactly, bf16 RoPE dims)
-//   S  = Qhat . X^T      tcgen05 M=64 (heads) N=64 (rows), nope and RoPE dims
-//                        into separate TMEM accumulators: s = scale*S_nope + S_rope
-//   P  = 2^(s - m)       one thread per head; P_nope = P*scale, P_rope = P (bf16)
-//   O^T += X^T . P^T     tcgen05 M=128 (dims) N=64 (heads), accumulated in TMEM
-// Lazy rescale: the running max moves only when a tile's max exceeds it by
-// more than 8 (log2 units); then O^T columns and l are rescaled in place.
+// One CTA = three roles over a stream of 64-row tiles:
+//   warps 4-7 (loader)  compute row addresses for a chunk, gather the raw
+//                       cache rows of tile t+1 into registers while tile t is
+//                       in flight, widen fp8 codes to bf16 (exact) into the
+//                       SW128 K-major X tile (double-buffered);
+//   warp 8 (MMA)        S = Qhat . X^T   tcgen05 M=64 (heads) N=64 (rows),
+//                                        nope and RoPE dims in separate TMEM
+//                                        accumulators: s = scale*S_nope + S_rope
+//                       O^T += X^T . P^T tcgen05 M=128 (dims) N=64 (heads);
+//   warps 0-3 (softmax) bulk-copy the request's Qhat image (prep_q_kernel:
+//                       RoPE(RMSNorm(q)*gamma_q, t)) into smem; per tile read S, P = 2^(s - m) (lanes 0-15 of each warp own one
+//                       head), P_nope = bf16(P*scale), P_rope = bf16(P); lazy
+//                       rescale of O^T when a head's max grows by more than 8
+//                       (log2 units); at chunk end read O^T out as the partial.
+// mbarriers hand tiles between roles; every wait is bounded.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace csla {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kSoftWarps = 4, kLoadWarps = 4;
+constexpr int kThreads = 32 * (kSoftWarps + kLoadWarps + 1);   // 288
+constexpr int kLoadThreads = 32 * kLoadWarps;
+constexpr int kMmaWarp = kSoftWarps + kLoadWarps;               // warp 8
 constexpr int kHP = 64;          // heads padded to the UMMA M of the S product
 constexpr int kTile = 64;        // rows per tile
+constexpr int kRowInfo = 512;    // row addresses held at once by the loader
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThresh = 8.0f;
+constexpr int kBarLoad = 1;   // named barrier of the loader warps (0 = __syncthreads)
 
 template <int D>
 struct Cfg {
@@ -52,6 +63,9 @@ struct Cfg {
     static constexpr int kQKB = kHP * 128;             // one K block of Qhat
     static constexpr int kQBytes = kKB * kQKB;
     static constexpr int kPBytes = kHP * kTile * 2;
+    static constexpr int kTasks = kTile * kCH;         // 16-byte loads per tile
+    static constexpr int kTPT = kTasks / kLoadThreads; // loads per loader thread
+    static_assert(kTasks % kLoadThreads == 0, "tile split");
     // TMEM columns
     static constexpr int kColSN = 0, kColSR = 64, kColO = 128;
     static constexpr int kColOR = 128 + 64 * kMB;
@@ -63,20 +77,23 @@ struct Cfg {
     static constexpr int kOffPn = kOffX1 + kXBytes;
     static constexpr int kOffPr = kOffPn + kPBytes;
     static constexpr int kOffMisc = kOffPr + kPBytes;
-    static constexpr int kSmemBytes = kOffMisc + 4096 + 1024;
 };
 
 struct Misc {
-    const uint8_t *rowptr[kTile];
-    float rscale[kTile];
-    int rvalid[kTile];
-    float fac[kHP];
-    float cs[32][2];
-    uint64_t bar_s, bar_o;
+    const uint8_t *rowptr[kRowInfo];   // loader-private: sources of the current row group
+    float rowscale[kRowInfo];
+    float tscale[2][kTile];            // per X buffer: fp8 scale of each row (0 = masked)
+    int tvalid[2][kTile];
+    float fac[2][kHP];                 // per tile parity: O^T column factors (1 = none)
+    uint64_t x_full[2], x_empty[2], s_full, s_free, p_full, pv_done, o_free, q_ready, fac_ready;
     uint32_t tmem;
-    int any_rescale;
     int abort;
 };
+
+template <int D>
+constexpr int smem_bytes() {
+    return Cfg<D>::kOffMisc + (int)sizeof(Misc) + 1024;
+}
 
 // Request-level facts both variants derive the same way.
 struct Req {
@@ -107,6 +124,10 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
     return v;
 }
 
+__device__ __forceinline__ void named_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 // Byte offset of 8-element group g (dims 8g..8g+7) of row r in a SW128
 // K-major tile whose K blocks are `kb_bytes` apart.
 __device__ __forceinline__ uint32_t sw128_off(int r, int g, int kb_bytes) {
@@ -117,86 +138,108 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return (uint32_t)f32_to_bf16_bits(lo) | ((uint32_t)f32_to_bf16_bits(hi) << 16);
 }
 
-// qhat = RoPE(RMSNorm(q_h) * gamma_q, t) for the 64 (padded) heads -> smem.
+// ---------------------------------------------------------------- query preparation
+// qhat = RoPE(RMSNorm(q_h) * gamma_q, t) for the 64 (padded) heads of request
+// b, written as the bf16 SW128 K-major shared-memory image the attention
+// kernel copies in with bulk copies.  grid (B, 8), one warp per head.
 template <int D>
-__device__ void prepare_q(const AttendArgs &a, int b, long long t, bool q_bf16, uint8_t *qs, Misc *ms) {
+__global__ void __launch_bounds__(256) prep_q_kernel(AttendArgs a, int q_bf16) {
+    CSLA_TL_SCOPE(kTlPrepQ);
+    using C = Cfg<D>;
+    __shared__ float cs[32][2];
+    pdl_trigger();
+    const int b = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x < 32) {
-        float c, s;
-        rope_cos_sin(t, threadIdx.x, 64, a.theta, &c, &s);
-        ms->cs[threadIdx.x][0] = c;
-        ms->cs[threadIdx.x][1] = s;
-    }
-    __syncthreads();
+    const int h = blockIdx.y * 8 + warp;
+    const int slot = __ldg(a.slots + b);
+    const bool slot_ok = slot >= 0 && slot < a.n_slots;
     constexpr int NG = D / 8;                   // 8-dim groups per head
     constexpr int GPL = (NG + 31) / 32;         // groups per lane
-    for (int h = warp; h < kHP; h += 4) {
-        float x[GPL][8];
-        float ss = 0.f;
+    // ---- before the wait: RMSNorm(q) * gamma_q in registers (q and gamma
+    // are inputs of the call)
+    float y[GPL][8];
+    float ss = 0.f;
 #pragma unroll
-        for (int i = 0; i < GPL; ++i) {
-            const int g = lane + 32 * i;
+    for (int i = 0; i < GPL; ++i) {
+        const int g = lane + 32 * i;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[i][e] = 0.f;
-            if (g < NG && h < a.H) {
-                const size_t off = ((size_t)b * a.H + h) * D + (size_t)g * 8;
-                if (q_bf16) {
-                    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
-                        reinterpret_cast<const __nv_bfloat16 *>(a.q) + off));
-                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        for (int e = 0; e < 8; ++e) y[i][e] = 0.f;
+        if (g < NG && h < a.H) {
+            const size_t off = ((size_t)b * a.H + h) * D + (size_t)g * 8;
+            if (q_bf16) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
+                    reinterpret_cast<const __nv_bfloat16 *>(a.q) + off));
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        x[i][2 * e] = bf16_bits_to_f32(w[e] & 0xFFFFu);
-                        x[i][2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
-                    }
-                } else {
-                    const float4 *p = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(a.q) + off);
-                    const float4 u0 = __ldg(p), u1 = __ldg(p + 1);
-                    x[i][0] = u0.x; x[i][1] = u0.y; x[i][2] = u0.z; x[i][3] = u0.w;
-                    x[i][4] = u1.x; x[i][5] = u1.y; x[i][6] = u1.z; x[i][7] = u1.w;
+                for (int e = 0; e < 4; ++e) {
+                    y[i][2 * e] = bf16_bits_to_f32(w[e] & 0xFFFFu);
+                    y[i][2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
                 }
+            } else {
+                const float4 *p = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(a.q) + off);
+                const float4 u0 = __ldg(p), u1 = __ldg(p + 1);
+                y[i][0] = u0.x; y[i][1] = u0.y; y[i][2] = u0.z; y[i][3] = u0.w;
+                y[i][4] = u1.x; y[i][5] = u1.y; y[i][6] = u1.z; y[i][7] = u1.w;
             }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) ss = __fmaf_rn(x[i][e], x[i][e], ss);
         }
-        ss = warp_sum(ss);
-        const float r = 1.0f / sqrtf(__fdiv_rn(ss, (float)D) + a.eps);
 #pragma unroll
-        for (int i = 0; i < GPL; ++i) {
-            const int g = lane + 32 * i;
-            if (g >= NG) continue;
-            float y[8];
+        for (int e = 0; e < 8; ++e) ss = __fmaf_rn(y[i][e], y[i][e], ss);
+    }
+    ss = warp_sum(ss);
+    const float r = 1.0f / sqrtf(__fdiv_rn(ss, (float)D) + a.eps);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(__fmul_rn(x[i][e], r), __ldg(a.gamma_q + g * 8 + e));
-            if (g * 8 >= D - 64) {
+    for (int i = 0; i < GPL; ++i) {
+        const int g = lane + 32 * i;
+        if (g >= NG) continue;
 #pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    const int pi = (g * 8 + e - (D - 64)) >> 1;
-                    const float c = ms->cs[pi][0], s = ms->cs[pi][1];
-                    const float y0 = y[e], y1 = y[e + 1];
-                    y[e] = __fsub_rn(__fmul_rn(y0, c), __fmul_rn(y1, s));
-                    y[e + 1] = __fadd_rn(__fmul_rn(y0, s), __fmul_rn(y1, c));
-                }
+        for (int e = 0; e < 8; ++e) y[i][e] = __fmul_rn(__fmul_rn(y[i][e], r), __ldg(a.gamma_q + g * 8 + e));
+    }
+    pdl_wait();
+    CSLA_TL_WAITED();
+
+    // ---- the query position is len - 1
+    const int L = slot_ok ? a.len[slot] : 0;
+    if (!slot_ok || L < 1 || L > a.max_len) return;   // the attention kernel reports it
+    if (threadIdx.x < 32) {
+        float c, sn;
+        rope_cos_sin((long long)L - 1, a.freq.inv[threadIdx.x], &c, &sn);
+        cs[threadIdx.x][0] = c;
+        cs[threadIdx.x][1] = sn;
+    }
+    __syncthreads();
+    uint8_t *img = a.qimg + (size_t)b * C::kQBytes;
+#pragma unroll
+    for (int i = 0; i < GPL; ++i) {
+        const int g = lane + 32 * i;
+        if (g >= NG) continue;
+        if (g * 8 >= D - 64) {
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+                const int pi = (g * 8 + e - (D - 64)) >> 1;
+                const float c = cs[pi][0], sn = cs[pi][1];
+                const float y0 = y[i][e], y1 = y[i][e + 1];
+                y[i][e] = __fsub_rn(__fmul_rn(y0, c), __fmul_rn(y1, sn));
+                y[i][e + 1] = __fadd_rn(__fmul_rn(y0, sn), __fmul_rn(y1, c));
             }
-            uint4 o;
-            o.x = pack_bf16x2(y[0], y[1]);
-            o.y = pack_bf16x2(y[2], y[3]);
-            o.z = pack_bf16x2(y[4], y[5]);
-            o.w = pack_bf16x2(y[6], y[7]);
-            *reinterpret_cast<uint4 *>(qs + sw128_off(h, g, Cfg<D>::kQKB)) = o;
         }
+        uint4 o;
+        o.x = pack_bf16x2(y[i][0], y[i][1]);
+        o.y = pack_bf16x2(y[i][2], y[i][3]);
+        o.z = pack_bf16x2(y[i][4], y[i][5]);
+        o.w = pack_bf16x2(y[i][6], y[i][7]);
+        *reinterpret_cast<uint4 *>(img + sw128_off(h, g, C::kQKB)) = o;
     }
 }
 
-// Sources of the tile's rows [r0, r0+64) restricted to [lo, hi).
-__device__ void tile_sources(const AttendArgs &a, int b, const Req &rq, int r0, int hi, int rb, Misc *ms) {
-    const int t = threadIdx.x;
-    if (t >= kTile) return;
-    const int r = r0 + t;
-    const uint8_t *p = nullptr;
-    float sc = 0.f;
-    int ok = 0;
-    if (r < hi) {
+// ---------------------------------------------------------------- loader role helpers
+// Sources of rows [r0, r0 + cnt) of the request's set (cnt <= kRowInfo):
+// ms->rowptr / rowscale, null pointer = masked row.  Loader threads only.
+__device__ void row_sources(const AttendArgs &a, int b, const Req &rq, int r0, int cnt, int rb, Misc *ms) {
+    const int lt = threadIdx.x - 32 * kSoftWarps;
+    for (int i = lt; i < cnt; i += kLoadThreads) {
+        const int r = r0 + i;
+        const uint8_t *p = nullptr;
+        float sc = 0.f;
         if (r < rq.n_cmp) {
             const int e = a.idx ? __ldg(a.idx + (size_t)b * a.k + r) : r;
             if (e >= 0) {
@@ -212,104 +255,125 @@ __device__ void tile_sources(const AttendArgs &a, int b, const Req &rq, int r0, 
                         const size_t ent = (size_t)pg * epp + (size_t)(e % epp);
                         p = a.rows + ent * rb;
                         sc = __ldg(a.scales + ent);
-                        ok = 1;
                     }
                 }
             }
-        } else {
+        } else if (r < rq.n_rows) {
             const int w = r - rq.n_cmp;
             const int pos = rq.L - rq.win_len + w;
             const size_t ring = (size_t)rq.slot * a.n_win + (size_t)(pos % a.n_win);
             p = a.win_rows + ring * rb;
             sc = __ldg(a.win_scales + ring);
-            ok = 1;
         }
+        ms->rowptr[i] = p;
+        ms->rowscale[i] = sc;
     }
-    ms->rowptr[t] = p;
-    ms->rscale[t] = sc;
-    ms->rvalid[t] = ok;
 }
 
-// Widen the tile's cache rows into the bf16 SW128 K-major X tile.
+// Widen one 16-byte chunk of a cache row into the bf16 X tile.
 template <int D>
-__device__ void load_tile(uint8_t *xs, const Misc *ms) {
+__device__ __forceinline__ void store_chunk(uint8_t *xs, int r, int c, const uint4 v) {
     using C = Cfg<D>;
-    constexpr int kTasks = kTile * C::kCH;
-    constexpr int kU = 6;
-    static_assert(kTasks % (kThreads * kU) == 0 || kTasks < kThreads * kU, "task split");
-    for (int base = 0; base < kTasks; base += kThreads * kU) {
-        uint4 v[kU];
-        int rr[kU], cc[kU];
+    if (c < C::kNopeCH) {
+        const int g0 = c * 2;   // 16 codes = two 8-dim groups
+        uint4 lo, hi;
+        lo.x = e4m3x2_to_bf16x2(v.x & 0xFFFFu);
+        lo.y = e4m3x2_to_bf16x2(v.x >> 16);
+        lo.z = e4m3x2_to_bf16x2(v.y & 0xFFFFu);
+        lo.w = e4m3x2_to_bf16x2(v.y >> 16);
+        hi.x = e4m3x2_to_bf16x2(v.z & 0xFFFFu);
+        hi.y = e4m3x2_to_bf16x2(v.z >> 16);
+        hi.z = e4m3x2_to_bf16x2(v.w & 0xFFFFu);
+        hi.w = e4m3x2_to_bf16x2(v.w >> 16);
+        *reinterpret_cast<uint4 *>(xs + sw128_off(r, g0, C::kKBBytes)) = lo;
+        *reinterpret_cast<uint4 *>(xs + sw128_off(r, g0 + 1, C::kKBBytes)) = hi;
+    } else {
+        const int g = (D - 64) / 8 + (c - C::kNopeCH);
+        *reinterpret_cast<uint4 *>(xs + sw128_off(r, g, C::kKBBytes)) = v;
+    }
+}
+
+// The chunk range a CTA works on, and where chunk c's partial lives.
+struct Span {
+    int c0, c1;
+};
+
+__device__ __forceinline__ float *partial_ptr(const AttendArgs &a, int b, int c, int D) {
+    const size_t stride = (size_t)a.H * D + 2 * (size_t)a.H;
+    return a.part + ((size_t)b * a.max_chunks + c) * stride;
+}
+
+// ---------------------------------------------------------------- the three roles
+template <int D>
+__device__ void loader_role(const AttendArgs &a, int b, const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
+    using C = Cfg<D>;
+    const int lt = threadIdx.x - 32 * kSoftWarps;
+    int g = 0;   // tile counter across the CTA's chunks
+    // Loop bounds are uniform over the loader warps and nothing below leaves
+    // a loop early, so every loader thread reaches every named barrier.
+    for (int c = sp.c0; c < sp.c1; ++c) {
+        const int lo = c * rq.chunk;
+        const int hi = min(rq.n_rows, lo + rq.chunk);
+        for (int grp = lo; grp < hi; grp += kRowInfo) {
+            const int cnt = min(kRowInfo, hi - grp);
+            named_sync(kBarLoad, kLoadThreads);          // previous group fully consumed
+            row_sources(a, b, rq, grp, cnt, C::kRB, ms);
+            named_sync(kBarLoad, kLoadThreads);
+            if (lt == 0 && grp == lo) CSLA_TL_MARK(0);
+            for (int t0 = 0; t0 < cnt; t0 += kTile, ++g) {
+                if (ms->abort) continue;
+                const int buf = g & 1;
+                // gather the tile's raw rows into registers first ...
+                uint4 v[C::kTPT];
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            const int id = base + u * kThreads + threadIdx.x;
-            rr[u] = id / C::kCH;
-            cc[u] = id % C::kCH;
-            v[u] = make_uint4(0u, 0u, 0u, 0u);
-            if (id < kTasks && ms->rvalid[rr[u]]) v[u] = ld_nc_v4(ms->rowptr[rr[u]] + cc[u] * 16);
-        }
+                for (int u = 0; u < C::kTPT; ++u) {
+                    const int id = u * kLoadThreads + lt;
+                    const int r = id / C::kCH, ch = id % C::kCH;
+                    const uint8_t *p = (t0 + r < cnt) ? ms->rowptr[t0 + r] : nullptr;
+                    v[u] = p ? ld_nc_v4(p + ch * 16) : make_uint4(0u, 0u, 0u, 0u);
+                }
+                if (lt == 0 && g == 0) CSLA_TL_MARK(6);
+                // ... then wait until PV of the tile that last used this buffer is done
+                if (g >= 2 && !mbar_wait(&ms->x_empty[buf], ((g >> 1) - 1) & 1, &ms->abort)) continue;
+                uint8_t *xs = smem + (buf ? C::kOffX1 : C::kOffX0);
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            const int id = base + u * kThreads + threadIdx.x;
-            if (id >= kTasks) continue;
-            const int r = rr[u], c = cc[u];
-            if (c < C::kNopeCH) {
-                const int g0 = c * 2;   // 16 codes = two 8-dim groups
-                uint4 lo, hi;
-                lo.x = e4m3x2_to_bf16x2(v[u].x & 0xFFFFu);
-                lo.y = e4m3x2_to_bf16x2(v[u].x >> 16);
-                lo.z = e4m3x2_to_bf16x2(v[u].y & 0xFFFFu);
-                lo.w = e4m3x2_to_bf16x2(v[u].y >> 16);
-                hi.x = e4m3x2_to_bf16x2(v[u].z & 0xFFFFu);
-                hi.y = e4m3x2_to_bf16x2(v[u].z >> 16);
-                hi.z = e4m3x2_to_bf16x2(v[u].w & 0xFFFFu);
-                hi.w = e4m3x2_to_bf16x2(v[u].w >> 16);
-                *reinterpret_cast<uint4 *>(xs + sw128_off(r, g0, C::kKBBytes)) = lo;
-                *reinterpret_cast<uint4 *>(xs + sw128_off(r, g0 + 1, C::kKBBytes)) = hi;
-            } else {
-                const int g = (D - 64) / 8 + (c - C::kNopeCH);
-                *reinterpret_cast<uint4 *>(xs + sw128_off(r, g, C::kKBBytes)) = v[u];
+                for (int u = 0; u < C::kTPT; ++u) {
+                    const int id = u * kLoadThreads + lt;
+                    store_chunk<D>(xs, id / C::kCH, id % C::kCH, v[u]);
+                }
+                if (lt < kTile) {
+                    const bool ok = (t0 + lt < cnt) && ms->rowptr[t0 + lt] != nullptr;
+                    ms->tscale[buf][lt] = ok ? ms->rowscale[t0 + lt] : 0.f;
+                    ms->tvalid[buf][lt] = ok ? 1 : 0;
+                }
+                fence_proxy_async_smem();
+                if (lt == 0 && g == 0) CSLA_TL_MARK(4);
+                mbar_arrive(&ms->x_full[buf]);
             }
         }
     }
 }
 
-struct HeadState {
-    float m, l;
-};
-
-// One chunk of request b: rows [lo, hi) of its attention set.  Writes the
-// chunk partial (O [H][D], m [H], l [H]) to `part`.  Ends with every thread
-// past a __syncthreads and no UMMA in flight.
 template <int D>
-__device__ void chunk_pass(const AttendArgs &a, int b, const Req &rq, int lo, int hi, uint8_t *smem, Misc *ms,
-                           uint32_t &ph_s, uint32_t &ph_o, float *part) {
+__device__ void mma_role(const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
     using C = Cfg<D>;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    const int h = 16 * warp + lane;       // head owned by lanes 0..15 (M=64 TMEM layout)
-    const bool head_thread = lane < 16;
-    const float cscale = kLog2e / sqrtf((float)D);
     constexpr uint32_t kIdescS = idesc_bf16(64, 64, false, false);
     constexpr uint32_t kIdescO = idesc_bf16(128, 64, true, false);
-    uint8_t *qs = smem + C::kOffQ;
-    uint8_t *pn = smem + C::kOffPn;
-    uint8_t *pr = smem + C::kOffPr;
     const uint32_t tmem = ms->tmem;
-    HeadState hs{-INFINITY, 0.f};
-    int buf = 0;
-
-    for (int r0 = lo, ti = 0; r0 < hi; r0 += kTile, ++ti, buf ^= 1) {
-        uint8_t *xs = smem + (buf ? C::kOffX1 : C::kOffX0);
-        tile_sources(a, b, rq, r0, hi, C::kRB, ms);
-        __syncthreads();
-        load_tile<D>(xs, ms);
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (threadIdx.x == 0) {
+    const uint32_t q0 = smem_u32(smem + C::kOffQ);
+    const uint32_t p0n = smem_u32(smem + C::kOffPn), p0r = smem_u32(smem + C::kOffPr);
+    if (!mbar_wait(&ms->q_ready, 0, &ms->abort)) return;
+    CSLA_TL_MARK(5);
+    int g = 0;
+    for (int c = sp.c0; c < sp.c1; ++c) {
+        const int lo = c * rq.chunk;
+        const int hi = min(rq.n_rows, lo + rq.chunk);
+        for (int r0 = lo, ti = 0; r0 < hi; r0 += kTile, ++ti, ++g) {
+            const int buf = g & 1;
+            if (!mbar_wait(&ms->x_full[buf], (g >> 1) & 1, &ms->abort)) return;
+            if (g > 0 && !mbar_wait(&ms->s_free, (g - 1) & 1, &ms->abort)) return;
             tc_fence_after();
-            const uint32_t q0 = smem_u32(qs), x0 = smem_u32(xs);
+            const uint32_t x0 = smem_u32(smem + (buf ? C::kOffX1 : C::kOffX0));
 #pragma unroll
             for (int kb = 0; kb < C::kKBN; ++kb)
 #pragma unroll
@@ -320,165 +384,217 @@ __device__ void chunk_pass(const AttendArgs &a, int b, const Req &rq, int lo, in
             for (int ks = 0; ks < 4; ++ks)
                 umma_bf16(tmem + C::kColSR, sdesc(q0 + C::kKBN * C::kQKB + ks * 32, 16, 1024),
                           sdesc(x0 + C::kKBN * C::kKBBytes + ks * 32, 16, 1024), kIdescS, ks ? 1u : 0u);
-            umma_commit(&ms->bar_s);
-        }
-        mbar_wait(&ms->bar_s, ph_s, &ms->abort);
-        ph_s ^= 1;
-        tc_fence_after();
-
-        // ---- scores of this tile: lanes 0..15 hold head rows
-        float s[kTile];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            uint32_t rn[32], rrp[32];
-            tmem_ld32x32(tmem + lane_base + C::kColSN + 32 * half, rn);
-            tmem_ld32x32(tmem + lane_base + C::kColSR + 32 * half, rrp);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int jj = 32 * half + j;
-                const float v = __fmul_rn(__fmaf_rn(ms->rscale[jj], __uint_as_float(rn[j]), __uint_as_float(rrp[j])),
-                                          cscale);
-                s[jj] = ms->rvalid[jj] ? v : -INFINITY;
-            }
-        }
-        float mt = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < kTile; ++j) mt = fmaxf(mt, s[j]);
-
-        // PV of the previous tile must be done before P and O^T are touched.
-        if (ti > 0) {
-            mbar_wait(&ms->bar_o, ph_o, &ms->abort);
-            ph_o ^= 1;
+            umma_commit(&ms->s_full);
+            if (!mbar_wait(&ms->p_full, g & 1, &ms->abort)) return;
+            if (ti == 0 && c > sp.c0 && !mbar_wait(&ms->o_free, (c - sp.c0 - 1) & 1, &ms->abort)) return;
             tc_fence_after();
-        }
-        if (threadIdx.x == 0) ms->any_rescale = 0;
-        __syncthreads();
-        float f = 1.f;
-        if (head_thread) {
-            float mnew = hs.m;
-            if (ti == 0) {
-                mnew = mt;
-            } else if (mt > hs.m + kRescaleThresh || (hs.m == -INFINITY && mt > -INFINITY)) {
-                mnew = mt;
-                f = exp2f(__fsub_rn(hs.m, mnew));
-            }
-            const float muse = mnew == -INFINITY ? 0.f : mnew;
-            float lsum = 0.f;
-#pragma unroll
-            for (int c8 = 0; c8 < kTile / 8; ++c8) {
-                float p[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    p[e] = exp2f(__fsub_rn(s[c8 * 8 + e], muse));
-                    lsum = __fadd_rn(lsum, p[e]);
-                }
-                uint4 un, ur;
-                un.x = pack_bf16x2(__fmul_rn(p[0], ms->rscale[c8 * 8 + 0]), __fmul_rn(p[1], ms->rscale[c8 * 8 + 1]));
-                un.y = pack_bf16x2(__fmul_rn(p[2], ms->rscale[c8 * 8 + 2]), __fmul_rn(p[3], ms->rscale[c8 * 8 + 3]));
-                un.z = pack_bf16x2(__fmul_rn(p[4], ms->rscale[c8 * 8 + 4]), __fmul_rn(p[5], ms->rscale[c8 * 8 + 5]));
-                un.w = pack_bf16x2(__fmul_rn(p[6], ms->rscale[c8 * 8 + 6]), __fmul_rn(p[7], ms->rscale[c8 * 8 + 7]));
-                ur.x = pack_bf16x2(p[0], p[1]);
-                ur.y = pack_bf16x2(p[2], p[3]);
-                ur.z = pack_bf16x2(p[4], p[5]);
-                ur.w = pack_bf16x2(p[6], p[7]);
-                const uint32_t off = (uint32_t)((h >> 3) * 1024 + (h & 7) * 128 + ((c8 ^ (h & 7)) << 4));
-                *reinterpret_cast<uint4 *>(pn + off) = un;
-                *reinterpret_cast<uint4 *>(pr + off) = ur;
-            }
-            hs.l = (ti == 0) ? lsum : __fadd_rn(__fmul_rn(hs.l, f), lsum);
-            hs.m = mnew;
-            ms->fac[h] = f;
-            if (ti > 0 && f != 1.f) ms->any_rescale = 1;
-        }
-        __syncthreads();
-        if (ms->any_rescale) {
-            // O^T columns are heads: every thread scales its own dim lane.
-#pragma unroll 1
-            for (int blk = 0; blk <= C::kMB; ++blk) {
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t v[32];
-                    const uint32_t addr = tmem + lane_base + C::kColO + 64 * blk + 32 * half;
-                    tmem_ld32x32(addr, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        v[j] = __float_as_uint(__fmul_rn(__uint_as_float(v[j]), ms->fac[32 * half + j]));
-                    tmem_st32x32(addr, v);
-                }
-            }
-            tmem_wait_st();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            tc_fence_after();
-            const uint32_t x0 = smem_u32(xs), p0n = smem_u32(pn), p0r = smem_u32(pr);
 #pragma unroll
             for (int mb = 0; mb < C::kMB; ++mb)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    umma_bf16(tmem + C::kColO + 64 * mb, sdesc(x0 + 2 * mb * C::kKBBytes + 2 * ks * 1024, C::kKBBytes, 1024),
+                    umma_bf16(tmem + C::kColO + 64 * mb,
+                              sdesc(x0 + 2 * mb * C::kKBBytes + 2 * ks * 1024, C::kKBBytes, 1024),
                               sdesc(p0n + ks * 32, 16, 1024), kIdescO, (ti > 0 || ks > 0) ? 1u : 0u);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                umma_bf16(tmem + C::kColOR, sdesc(x0 + 2 * (C::kMB - 1) * C::kKBBytes + 2 * ks * 1024, C::kKBBytes, 1024),
+                umma_bf16(tmem + C::kColOR,
+                          sdesc(x0 + 2 * (C::kMB - 1) * C::kKBBytes + 2 * ks * 1024, C::kKBBytes, 1024),
                           sdesc(p0r + ks * 32, 16, 1024), kIdescO, (ti > 0 || ks > 0) ? 1u : 0u);
-            umma_commit(&ms->bar_o);
+            umma_commit(&ms->x_empty[buf]);
+            umma_commit(&ms->pv_done);
         }
     }
-    // drain the last PV, then read O^T out of TMEM
-    mbar_wait(&ms->bar_o, ph_o, &ms->abort);
-    ph_o ^= 1;
-    tc_fence_after();
-    const size_t HD = (size_t)a.H * D;
-#pragma unroll 1
-    for (int blk = 0; blk <= C::kMB; ++blk) {
-        const bool rope_blk = blk == C::kMB;
-        const int dim = (rope_blk ? (D - 128) : 128 * blk) + 32 * warp + lane;
-        const bool write = rope_blk ? (dim >= D - 64) : (dim < D - 64);
+}
+
+template <int D>
+__device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
+    using C = Cfg<D>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    const int h = 16 * warp + lane;       // head owned by lanes 0..15 (M=64 TMEM layout)
+    const bool head_thread = lane < 16;
+    const float cscale = kLog2e / sqrtf((float)D);
+    const uint32_t tmem = ms->tmem;
+    uint8_t *pn = smem + C::kOffPn;
+    uint8_t *pr = smem + C::kOffPr;
+
+    if (threadIdx.x == 0) {
+        // the request's Qhat image, written by prep_q_kernel
+        const uint8_t *src = a.qimg + (size_t)b * C::kQBytes;
+        mbar_arrive_expect_tx(&ms->q_ready, (uint32_t)C::kQBytes);
+        for (int off = 0; off < C::kQBytes; off += 16384)
+            bulk_load(smem + C::kOffQ + off, src + off, (uint32_t)min(16384, C::kQBytes - off), &ms->q_ready);
+    }
+
+    int g = 0;
+    for (int c = sp.c0; c < sp.c1; ++c) {
+        const int lo = c * rq.chunk;
+        const int hi = min(rq.n_rows, lo + rq.chunk);
+        float m_run = -INFINITY, l_run = 0.f;
+        for (int r0 = lo, ti = 0; r0 < hi; r0 += kTile, ++ti, ++g) {
+            const int buf = g & 1;
+            if (!mbar_wait(&ms->x_full[buf], (g >> 1) & 1, &ms->abort)) return;
+            if (!mbar_wait(&ms->s_full, g & 1, &ms->abort)) return;
+            if (threadIdx.x == 0 && g == 0) CSLA_TL_MARK(1);
+            tc_fence_after();
+            float s[kTile];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            uint32_t v[32];
-            tmem_ld32x32(tmem + lane_base + C::kColO + 64 * blk + 32 * half, v);
-            tmem_wait_ld();
-            if (write) {
+            for (int half = 0; half < 2; ++half) {
+                uint32_t rn[32], rr[32];
+                tmem_ld32x32(tmem + lane_base + C::kColSN + 32 * half, rn);
+                tmem_ld32x32(tmem + lane_base + C::kColSR + 32 * half, rr);
+                tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const int hh = 32 * half + j;
-                    if (hh < a.H) part[(size_t)hh * D + dim] = __uint_as_float(v[j]);
+                    const int jj = 32 * half + j;
+                    const float v = __fmul_rn(
+                        __fmaf_rn(ms->tscale[buf][jj], __uint_as_float(rn[j]), __uint_as_float(rr[j])), cscale);
+                    s[jj] = ms->tvalid[buf][jj] ? v : -INFINITY;
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&ms->s_free);        // S may be overwritten by the next tile's MMA
+            float mt = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < kTile; ++j) mt = fmaxf(mt, s[j]);
+            // PV of the previous tile must be done before P and O^T are touched.
+            if (g > 0 && !mbar_wait(&ms->pv_done, (g - 1) & 1, &ms->abort)) return;
+            tc_fence_after();
+            float f = 1.f;
+            if (head_thread) {
+                float mnew = m_run;
+                if (ti == 0) {
+                    mnew = mt;
+                } else if (mt > m_run + kRescaleThresh || (m_run == -INFINITY && mt > -INFINITY)) {
+                    mnew = mt;
+                    f = exp2f(__fsub_rn(m_run, mnew));
+                }
+                const float muse = mnew == -INFINITY ? 0.f : mnew;
+                float lsum = 0.f;
+#pragma unroll
+                for (int c8 = 0; c8 < kTile / 8; ++c8) {
+                    float p[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        p[e] = exp2f(__fsub_rn(s[c8 * 8 + e], muse));
+                        lsum = __fadd_rn(lsum, p[e]);
+                    }
+                    const float *sc = &ms->tscale[buf][c8 * 8];
+                    uint4 un, ur;
+                    un.x = pack_bf16x2(__fmul_rn(p[0], sc[0]), __fmul_rn(p[1], sc[1]));
+                    un.y = pack_bf16x2(__fmul_rn(p[2], sc[2]), __fmul_rn(p[3], sc[3]));
+                    un.z = pack_bf16x2(__fmul_rn(p[4], sc[4]), __fmul_rn(p[5], sc[5]));
+                    un.w = pack_bf16x2(__fmul_rn(p[6], sc[6]), __fmul_rn(p[7], sc[7]));
+                    ur.x = pack_bf16x2(p[0], p[1]);
+                    ur.y = pack_bf16x2(p[2], p[3]);
+                    ur.z = pack_bf16x2(p[4], p[5]);
+                    ur.w = pack_bf16x2(p[6], p[7]);
+                    const uint32_t off = (uint32_t)((h >> 3) * 1024 + (h & 7) * 128 + ((c8 ^ (h & 7)) << 4));
+                    *reinterpret_cast<uint4 *>(pn + off) = un;
+                    *reinterpret_cast<uint4 *>(pr + off) = ur;
+                }
+                l_run = (ti == 0) ? lsum : __fadd_rn(__fmul_rn(l_run, f), lsum);
+                m_run = mnew;
+                ms->fac[g & 1][h] = f;
+            }
+            // every head's factor is needed by every thread (each owns one O^T row)
+            mbar_arrive(&ms->fac_ready);
+            if (!mbar_wait(&ms->fac_ready, g & 1, &ms->abort)) return;
+            bool any_rescale = false;
+#pragma unroll 8
+            for (int j = 0; j < kHP; ++j) any_rescale |= ms->fac[g & 1][j] != 1.f;
+            if (any_rescale) {
+                // O^T columns are heads: every thread scales its own dim lane.
+#pragma unroll 1
+                for (int blk = 0; blk <= C::kMB; ++blk) {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t v[32];
+                        const uint32_t addr = tmem + lane_base + C::kColO + 64 * blk + 32 * half;
+                        tmem_ld32x32(addr, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            v[j] = __float_as_uint(__fmul_rn(__uint_as_float(v[j]), ms->fac[g & 1][32 * half + j]));
+                        tmem_st32x32(addr, v);
+                    }
+                }
+                tmem_wait_st();
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&ms->p_full);
+        }
+        // chunk done: drain its last PV and read O^T out as the partial
+        if (!mbar_wait(&ms->pv_done, (g - 1) & 1, &ms->abort)) return;
+        if (threadIdx.x == 0) CSLA_TL_MARK(2);
+        tc_fence_after();
+        float *part = partial_ptr(a, b, c, D);
+        const size_t HD = (size_t)a.H * D;
+#pragma unroll 1
+        for (int blk = 0; blk <= C::kMB; ++blk) {
+            const bool rope_blk = blk == C::kMB;
+            const int dim = (rope_blk ? (D - 128) : 128 * blk) + 32 * warp + lane;
+            const bool write = rope_blk ? (dim >= D - 64) : (dim < D - 64);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t v[32];
+                tmem_ld32x32(tmem + lane_base + C::kColO + 64 * blk + 32 * half, v);
+                tmem_wait_ld();
+                if (write) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int hh = 32 * half + j;
+                        if (hh < a.H) part[(size_t)hh * D + dim] = __uint_as_float(v[j]);
+                    }
                 }
             }
         }
+        if (head_thread && h < a.H) {
+            part[HD + h] = m_run;
+            part[HD + a.H + h] = l_run;
+        }
+        if (threadIdx.x == 0) CSLA_TL_MARK(3);
+        tc_fence_before();
+        mbar_arrive(&ms->o_free);
     }
-    if (head_thread && h < a.H) {
-        part[HD + h] = hs.m;
-        part[HD + a.H + h] = hs.l;
-    }
-    tc_fence_before();
-    __syncthreads();
 }
 
-// Ordered fold of the chunk partials of request b, head h, dim d (sink first).
-__device__ __forceinline__ float fold_one(const AttendArgs &a, int b, int n_chunks, int h, int d, int D,
-                                          float *l_out) {
+// Fold of the chunk partials of request b, head h (sink first):
+//   M = max(sink*log2e, m_0 .. m_{n-1})                (exact, order-free)
+//   w_c = 2^(m_c - M);  l = 2^(sink*log2e - M) + sum_c l_c w_c;  o_d = sum_c O_c[d] w_c
+// with both sums taken in chunk order; out = o / l.  The saturated and the
+// starved kernels both use these two functions.
+// fold_weights is warp-collective (lane c loads chunk c, n_chunks <= 32);
+// on return every lane holds w_c of its own chunk c in *w_lane and l in *l_out.
+__device__ __forceinline__ void fold_weights(const AttendArgs &a, int b, int n_chunks, int h, int D, float *w_lane,
+                                             float *l_out) {
     const size_t stride = (size_t)a.H * D + 2 * (size_t)a.H;
-    const float *p = a.part + (size_t)b * a.max_chunks * stride;
-    float m = __fmul_rn(__ldg(a.sink + h), kLog2e);
-    float l = 1.f, o = 0.f;
-    for (int c = 0; c < n_chunks; ++c, p += stride) {
-        const float mc = p[(size_t)a.H * D + h];
-        const float lc = p[(size_t)a.H * D + a.H + h];
-        const float mn = fmaxf(m, mc);
-        const float fa = exp2f(__fsub_rn(m, mn));
-        const float fb = exp2f(__fsub_rn(mc, mn));
-        l = __fmaf_rn(l, fa, __fmul_rn(lc, fb));
-        o = __fmaf_rn(o, fa, __fmul_rn(p[(size_t)h * D + d], fb));
-        m = mn;
-    }
+    const float *p = a.part + (size_t)b * a.max_chunks * stride + (size_t)a.H * D;
+    const int lane = threadIdx.x & 31;
+    const float z = __fmul_rn(__ldg(a.sink + h), kLog2e);
+    const float mc = lane < n_chunks ? p[lane * stride + h] : -INFINITY;
+    const float lc = lane < n_chunks ? p[lane * stride + a.H + h] : 0.f;
+    const float M = fmaxf(z, warp_max(mc));
+    const float wc = lane < n_chunks ? exp2f(__fsub_rn(mc, M)) : 0.f;
+    float l = exp2f(__fsub_rn(z, M));
+    for (int c = 0; c < n_chunks; ++c)
+        l = __fmaf_rn(__shfl_sync(0xffffffffu, lc, c), __shfl_sync(0xffffffffu, wc, c), l);
+    *w_lane = wc;
     *l_out = l;
+}
+// o_d = sum_c O_c[d] w_c in chunk order, w[] the per-chunk weights.
+__device__ __forceinline__ float fold_dim(const AttendArgs &a, int b, int n_chunks, int h, int d, int D,
+                                          const float *w, float l) {
+    const size_t stride = (size_t)a.H * D + 2 * (size_t)a.H;
+    const float *p = a.part + (size_t)b * a.max_chunks * stride + (size_t)h * D + d;
+    float v[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] = c < n_chunks ? p[c * stride] : 0.f;
+    float o = 0.f;
+#pragma unroll
+    for (int c = 0; c < 32; ++c)
+        if (c < n_chunks) o = __fmaf_rn(v[c], w[c], o);
     return __fdiv_rn(o, l);
 }
 
@@ -488,104 +604,128 @@ __device__ __forceinline__ void store_out(const AttendArgs &a, bool out_bf16, si
 }
 
 template <int D, bool kSaturated>
-__global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int q_bf16, int out_bf16) {
+__global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int out_bf16) {
+    CSLA_TL_SCOPE(kTlAttend);
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     Misc *ms = reinterpret_cast<Misc *>(smem + C::kOffMisc);
-
     const int b = kSaturated ? blockIdx.x : blockIdx.y;
-    const Req rq = request(a, b);
-    if (!rq.ok) {
-        if (threadIdx.x == 0 && (kSaturated || blockIdx.x == 0)) set_dev_err(CSLA_DEVERR_LEN);
-        return;
-    }
-    if (!kSaturated && (int)blockIdx.x >= rq.n_chunks) return;
+    const int warp = threadIdx.x >> 5;
 
+    // ---- before the wait: barriers and TMEM
     if (threadIdx.x == 0) {
-        mbar_init(&ms->bar_s, 1);
-        mbar_init(&ms->bar_o, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ms->x_full[i], kLoadThreads);
+            mbar_init(&ms->x_empty[i], 1);
+        }
+        mbar_init(&ms->s_full, 1);
+        mbar_init(&ms->s_free, 32 * kSoftWarps);
+        mbar_init(&ms->p_full, 32 * kSoftWarps);
+        mbar_init(&ms->pv_done, 1);
+        mbar_init(&ms->o_free, 32 * kSoftWarps);
+        mbar_init(&ms->q_ready, 1);
+        mbar_init(&ms->fac_ready, 32 * kSoftWarps);
         ms->abort = 0;
         fence_mbar_init();
     }
-    if (threadIdx.x < 32) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&ms->tmem, C::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_trigger();   // after the TMEM allocation (see the indexer kernel)
+    pdl_wait();
+    CSLA_TL_WAITED();
 
-    prepare_q<D>(a, b, (long long)rq.L - 1, q_bf16 != 0, smem + C::kOffQ, ms);
-    fence_proxy_async_smem();
-    __syncthreads();
-
-    uint32_t ph_s = 0, ph_o = 0;
-    const size_t stride = (size_t)a.H * D + 2 * (size_t)a.H;
-    const int c0 = kSaturated ? 0 : (int)blockIdx.x;
-    const int c1 = kSaturated ? rq.n_chunks : c0 + 1;
-    for (int c = c0; c < c1; ++c) {
-        const int lo = c * rq.chunk;
-        const int hi = min(rq.n_rows, lo + rq.chunk);
-        float *part = a.part + ((size_t)b * a.max_chunks + c) * stride;
-        chunk_pass<D>(a, b, rq, lo, hi, smem, ms, ph_s, ph_o, part);
+    const Req rq = request(a, b);
+    if (!rq.ok && threadIdx.x == 0 && (kSaturated || blockIdx.x == 0)) set_dev_err(CSLA_DEVERR_LEN);
+    const bool run = rq.ok && (kSaturated || (int)blockIdx.x < rq.n_chunks);
+    const Span sp = kSaturated ? Span{0, rq.n_chunks} : Span{(int)blockIdx.x, (int)blockIdx.x + 1};
+    if (!run) {
+        // nothing to do: fall through to the teardown
+    } else if (warp < kSoftWarps) {
+        softmax_role<D>(a, b, rq, sp, smem, ms);
+    } else if (warp < kSoftWarps + kLoadWarps) {
+        loader_role<D>(a, b, rq, sp, smem, ms);
+    } else if ((threadIdx.x & 31) == 0) {
+        mma_role<D>(rq, sp, smem, ms);
     }
-    if (threadIdx.x < 32) {
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(ms->tmem, C::kTmemCols);
     }
+    if (!run) return;
     if (kSaturated) {
-        __syncthreads();   // partials written by this CTA are visible to it
-        for (int i = threadIdx.x; i < a.H * D; i += kThreads) {
-            const int hh = i / D, d = i % D;
-            float l;
-            const float v = fold_one(a, b, rq.n_chunks, hh, d, D, &l);
-            store_out(a, out_bf16 != 0, ((size_t)b * a.H + hh) * D + d, v);
+        // partials written by this CTA are visible to it after the barrier above
+        __shared__ float wts[kThreads / 32][32];   // per warp: chunk weights
+        const int lane = threadIdx.x & 31;
+        for (int hh = warp; hh < a.H; hh += kThreads / 32) {
+            float wl, l;
+            fold_weights(a, b, rq.n_chunks, hh, D, &wl, &l);
+            wts[warp][lane] = wl;
+            __syncwarp();
+            for (int d = lane; d < D; d += 32)
+                store_out(a, out_bf16 != 0, ((size_t)b * a.H + hh) * D + d,
+                          fold_dim(a, b, rq.n_chunks, hh, d, D, wts[warp], l));
+            __syncwarp();
         }
     }
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads) combine_kernel(AttendArgs a, int out_bf16) {
+__global__ void __launch_bounds__(128) combine_kernel(AttendArgs a, int out_bf16) {
+    CSLA_TL_SCOPE(kTlCombine);
+    __shared__ float wts[33];
+    pdl_trigger();
+    pdl_wait();
+    CSLA_TL_WAITED();
     const int h = blockIdx.x, b = blockIdx.y;
     const Req rq = request(a, b);
     if (!rq.ok) return;
-    for (int d = threadIdx.x; d < D; d += kThreads) {
-        float l;
-        const float v = fold_one(a, b, rq.n_chunks, h, d, D, &l);
-        store_out(a, out_bf16 != 0, ((size_t)b * a.H + h) * D + d, v);
+    if (threadIdx.x < 32) {
+        float wl, l;
+        fold_weights(a, b, rq.n_chunks, h, D, &wl, &l);
+        wts[threadIdx.x] = wl;
+        if (threadIdx.x == 0) wts[32] = l;
     }
+    __syncthreads();
+    for (int d = threadIdx.x; d < D; d += 128)
+        store_out(a, out_bf16 != 0, ((size_t)b * a.H + h) * D + d, fold_dim(a, b, rq.n_chunks, h, d, D, wts, wts[32]));
 }
 
 template <int D>
 cudaError_t launch_attend_t(const AttendArgs &a, bool q_bf16, bool out_bf16, int variant, int num_sms,
                             cudaStream_t stream) {
-    using C = Cfg<D>;
+    constexpr int kSmem = smem_bytes<D>();
+    static_assert(kSmem <= 232448, "shared memory budget");
     static int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
         cudaError_t e = cudaFuncSetAttribute(attend_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::kSmemBytes);
+                                             kSmem);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(attend_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::kSmemBytes);
+        e = cudaFuncSetAttribute(attend_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
+    cudaError_t pe = launch_pdl(prep_q_kernel<D>, dim3(a.B, 8), dim3(256), 0, stream, a, (int)q_bf16);
+    if (pe != cudaSuccess) return pe;
     bool saturated;
     if (variant == CSLA_VARIANT_SATURATED) saturated = true;
     else if (variant == CSLA_VARIANT_STARVED) saturated = false;
     else saturated = a.B >= num_sms || a.max_chunks <= 1;
-    if (saturated) {
-        attend_kernel<D, true><<<a.B, kThreads, C::kSmemBytes, stream>>>(a, q_bf16, out_bf16);
-        return cudaGetLastError();
-    }
-    attend_kernel<D, false><<<dim3(a.max_chunks, a.B), kThreads, C::kSmemBytes, stream>>>(a, q_bf16, out_bf16);
-    cudaError_t e = cudaGetLastError();
+    if (saturated)
+        return launch_pdl(attend_kernel<D, true>, dim3(a.B), dim3(kThreads), kSmem, stream, a, (int)out_bf16);
+    cudaError_t e =
+        launch_pdl(attend_kernel<D, false>, dim3(a.max_chunks, a.B), dim3(kThreads), kSmem, stream, a, (int)out_bf16);
     if (e != cudaSuccess) return e;
-    combine_kernel<D><<<dim3(a.H, a.B), kThreads, 0, stream>>>(a, out_bf16);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel<D>, dim3(a.H, a.B), dim3(128), 0, stream, a, (int)out_bf16);
 }
 
 }  // namespace

@@ -11,6 +11,7 @@
 #include <stdint.h>
 
 #include "../../include/csla.h"
+#include "kernels.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
 #error "libcsla kernels target sm_100a only"
@@ -47,6 +48,87 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two_codes) {
     v = __hmul2(v, k);                                  // 0x7B80 = 2^120
     return *reinterpret_cast<uint32_t *>(&v);
 }
+
+// ------------------------------------------------------------ programmatic dependent launch
+// Every libcsla kernel is launched with programmatic stream serialization
+// (programmatic dependent launch) and calls pdl_trigger() first (kernels that
+// allocate TMEM: right after the allocation), so the next kernel on the
+// stream can be scheduled while it runs.  pdl_wait() blocks
+// until the preceding kernel has completed and its writes are visible; a
+// kernel calls it before it reads anything produced on the stream or writes
+// global memory (the device error word aside).  Before the wait a kernel
+// only reads its call's read-only inputs (activations, weights, slot lists,
+// block tables) into registers, shared memory or TMEM, and sets up barriers
+// and TMEM.  Every launch has at least one CTA that waits before exiting, so
+// kernel completion stays ordered along the stream.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ------------------------------------------------------------ device timeline
+// Built with -DCSLA_TIMELINE only (see build.py --timeline): thread 0 of
+// every CTA records its kernel id, CTA index and global-timer stamps (start,
+// grid-dependency wait passed, exit, and up to eight marks a kernel sets at
+// points of interest) into g_timeline, read back with csla_timeline_read().  In normal builds the hooks compile to nothing.
+enum TimelineKernel : uint32_t {
+    kTlCompress = 1, kTlTailUpdate, kTlIqProject, kTlIqProjectWide, kTlIndexer, kTlTopk, kTlPrepQ, kTlAttend,
+    kTlCombine
+};
+#ifdef CSLA_TIMELINE
+constexpr int kTimelineMarks = 8;
+struct TimelineRec {
+    uint32_t kernel, cta;
+    unsigned long long t0, t1, t2, m[kTimelineMarks];
+    unsigned long long clk0, clk2;   // SM cycle counter at start and exit
+};
+constexpr unsigned kTimelineCap = 1u << 16;
+extern __device__ TimelineRec g_timeline[kTimelineCap];
+extern __device__ unsigned int g_timeline_n;
+__device__ __forceinline__ unsigned long long timeline_now() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+static __shared__ unsigned long long tl_marks[kTimelineMarks];   // per CTA; any thread may set a mark
+__device__ __forceinline__ void timeline_mark(int i) { tl_marks[i] = timeline_now(); }
+__device__ __forceinline__ unsigned long long timeline_clock() {
+    unsigned long long c;
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(c));
+    return c;
+}
+struct TimelineScope {
+    uint32_t k;
+    unsigned long long t0, t1, c0;
+    __device__ explicit TimelineScope(uint32_t kernel) : k(kernel), t0(timeline_now()), t1(0), c0(timeline_clock()) {
+        if (threadIdx.x == 0)
+            for (int i = 0; i < kTimelineMarks; ++i) tl_marks[i] = 0;
+    }
+    __device__ void waited() { t1 = timeline_now(); }
+    __device__ ~TimelineScope() {
+        if (threadIdx.x == 0) {
+            const unsigned i = atomicAdd(&g_timeline_n, 1u);
+            const uint32_t cta = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+            if (i < kTimelineCap) {
+                TimelineRec r{k, cta, t0, t1, timeline_now(), {}, c0, timeline_clock()};
+                for (int j = 0; j < kTimelineMarks; ++j) r.m[j] = tl_marks[j];
+                g_timeline[i] = r;
+            }
+        }
+    }
+};
+#define CSLA_TL_SCOPE(kernel) ::csla::TimelineScope csla_tl_scope_(kernel)
+#define CSLA_TL_WAITED() csla_tl_scope_.waited()
+#define CSLA_TL_MARK(i) ::csla::timeline_mark(i)
+#else
+#define CSLA_TL_SCOPE(kernel) \
+    do {                      \
+    } while (0)
+#define CSLA_TL_WAITED() \
+    do {                 \
+    } while (0)
+#define CSLA_TL_MARK(i) \
+    do {                \
+    } while (0)
+#endif
 
 // ------------------------------------------------------------ smem / sync
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -114,6 +196,14 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
@@ -235,16 +325,19 @@ __device__ __forceinline__ float block_max(float v, float *red) {
     return s;
 }
 
-// RoPE angle of pair i at position pos: pos * theta^(-2i/d_rope), reduced and
-// evaluated in double so that positions near 2^20 keep full fp32 accuracy.
-__device__ __forceinline__ void rope_cos_sin(long long pos, int i, int d_rope, float theta, float *c,
-                                             float *s) {
-    double inv = pow((double)theta, -(2.0 * (double)i) / (double)d_rope);
-    double ang = (double)pos * inv;
-    double sd, cd;
-    sincos(ang, &sd, &cd);
-    *c = (float)cd;
-    *s = (float)sd;
+// cos and sin of pos * inv_freq.  The angle (up to ~2^21 rad) is reduced to
+// [-pi, pi] first (Cody-Waite style: 2*pi split into a double pair, the
+// product k*2pi removed with fused multiply-adds), then evaluated with the
+// fp32 sincosf; the reduction keeps the fp32 result accurate for every
+// position a 2^20-token context reaches.
+__device__ __forceinline__ void rope_cos_sin(long long pos, double inv_freq, float *c, float *s) {
+    const double kTwoPiHi = 6.283185307179586232;     // double nearest to 2*pi
+    const double kTwoPiLo = 2.4492935982947064e-16;   // 2*pi - kTwoPiHi
+    const double ang = (double)pos * inv_freq;
+    const double k = rint(ang * 0.15915494309189535);  // 1 / (2*pi)
+    double r = fma(-k, kTwoPiHi, ang);
+    r = fma(-k, kTwoPiLo, r);
+    sincosf((float)r, s, c);
 }
 
 }  // namespace csla

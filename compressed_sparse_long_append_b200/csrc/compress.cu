@@ -1,14 +1,19 @@
 // compress.cu -- state-cache / classical-cache update (csla_compress_append).
 //
-// One CTA per new token (blockIdx.x = token i of the call, blockIdx.y =
-// request b).  The CTA writes the token's sliding-window row and, when the
-// token closes a block of m positions, pools that block into one compressed
-// entry (plus, for CSA, one compressed index key).
 //   硅星人 "DeepSeek V4 ... 让token大降价" §两大压缩注意力: token-level compressor
 //   (m = 4 for CSA, m' = 128 for HCA), window of 128 raw tokens, RoPE on the
 //   last 64 dims, bf16 RoPE dims + fp8 other dims, state cache holding the
 //   window and the tail, classical cache in blocks of 128 tokens.
 //   haiqwa "DeepSeek-V4" §RMSNorm归一化: RMSNorm on the compressed KV head.
+//
+// One launch, grid (T + NB, B, J): for request b,
+//   x <  T : new token x -> its sliding-window row (if it stays in the ring)
+//            and, for single-token calls, its raw row into the tail;
+//   x >= T : the (x-T)-th block this call completes -> z = 0: the pooled KV
+//            entry (gate softmax, weighted sum, RMSNorm, RoPE at the block's
+//            first position, quantisation), z = 1 (CSA): the index key.
+// A second small launch stores the raw rows of multi-token calls' open block
+// in the tail (after every pooling CTA has read the old tail) and sets len.
 // All arithmetic is fp32 with fixed-order reductions; the quantised codes
 // are taken with the hardware's round-to-nearest-even conversions.
 #include "common.cuh"
@@ -20,7 +25,7 @@ __device__ unsigned int g_dev_err = 0;
 
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
 template <typename T>
@@ -33,52 +38,127 @@ __device__ __forceinline__ float load_act<__nv_bfloat16>(const __nv_bfloat16 *p,
 }
 
 // RMSNorm(v) * gamma, partial RoPE at `pos`, quantise into one cache row.
-// v: smem [D] (overwritten), red: smem scratch.
-__device__ void norm_rope_quantise(float *v, const CompressArgs &a, long long pos, uint8_t *row,
+// v, gam: smem [D] (v overwritten); red: smem scratch.  The rotation angles
+// are taken first so their latency overlaps the reductions.
+__device__ void norm_rope_quantise(float *v, const float *gam, const CompressArgs &a, long long pos, uint8_t *row,
                                    float *scale_out, float *red) {
     const int D = a.D, dr = a.d_rope, dn = D - dr;
+    float c = 1.f, s = 0.f;
+    if (threadIdx.x < dr / 2) rope_cos_sin(pos, a.freq.inv[threadIdx.x], &c, &s);
     float ss = 0.f;
-    for (int d = threadIdx.x; d < D; d += kThreads) ss += v[d] * v[d];
+    for (int d = threadIdx.x; d < D; d += kThreads) ss = __fmaf_rn(v[d], v[d], ss);
     ss = block_sum<kWarps>(ss, red);
-    const float r = 1.0f / sqrtf(ss / (float)D + a.eps);
-    for (int d = threadIdx.x; d < D; d += kThreads) v[d] = v[d] * r * __ldg(a.gamma_kv + d);
+    const float r = 1.0f / sqrtf(__fdiv_rn(ss, (float)D) + a.eps);
+    for (int d = threadIdx.x; d < D; d += kThreads) v[d] = __fmul_rn(__fmul_rn(v[d], r), gam[d]);
     __syncthreads();
     if (threadIdx.x < dr / 2) {
         const int i = threadIdx.x;
-        float c, s;
-        rope_cos_sin(pos, i, dr, a.theta, &c, &s);
         const float x0 = v[dn + 2 * i], x1 = v[dn + 2 * i + 1];
-        v[dn + 2 * i] = x0 * c - x1 * s;
-        v[dn + 2 * i + 1] = x0 * s + x1 * c;
+        v[dn + 2 * i] = __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, s));
+        v[dn + 2 * i + 1] = __fadd_rn(__fmul_rn(x0, s), __fmul_rn(x1, c));
     }
     __syncthreads();
     float amax = 0.f;
     for (int d = threadIdx.x; d < dn; d += kThreads) amax = fmaxf(amax, fabsf(v[d]));
     amax = block_max<kWarps>(amax, red);
-    const float scale = amax > 0.f ? amax / 448.0f : 1.0f;
-    for (int d = threadIdx.x; d < dn; d += kThreads) row[d] = f32_to_e4m3(v[d] / scale);
+    const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    for (int d = threadIdx.x; d < dn; d += kThreads) row[d] = f32_to_e4m3(__fdiv_rn(v[d], scale));
     uint16_t *rope = reinterpret_cast<uint16_t *>(row + dn);
     for (int d = threadIdx.x; d < dr; d += kThreads) rope[d] = f32_to_bf16_bits(v[dn + d]);
     if (threadIdx.x == 0) *scale_out = scale;
 }
 
-// Softmax weights of the block's scalar gates g_i = <x_i, w> + bias[i]
-// into alpha[0..m).  Row i of the block comes from row_ptr(i).
-template <typename T, typename RowFn>
-__device__ void block_gate(RowFn row_ptr, int m, int width, const float *w, const float *bias, float *alpha,
-                           float *red) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int i = warp; i < m; i += kWarps) {
-        const T *x = nullptr;
-        const float *xf = nullptr;
-        row_ptr(i, &x, &xf);
-        float acc = 0.f;
-        for (int d = lane; d < width; d += 32) {
-            const float xv = xf ? xf[d] : load_act<T>(x, d);
-            acc += xv * __ldg(w + d);
+// Four consecutive activations (16-byte or 8-byte vector load when `vec`).
+template <typename T>
+__device__ __forceinline__ float4 load4(const T *p, size_t o, bool vec);
+template <>
+__device__ __forceinline__ float4 load4<float>(const float *p, size_t o, bool vec) {
+    if (vec) return __ldg(reinterpret_cast<const float4 *>(p + o));
+    return make_float4(__ldg(p + o), __ldg(p + o + 1), __ldg(p + o + 2), __ldg(p + o + 3));
+}
+template <>
+__device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16 *p, size_t o, bool vec) {
+    if (vec) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p + o));
+        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+        return make_float4(lo.x, lo.y, hi.x, hi.y);
+    }
+    return make_float4(__bfloat162float(p[o]), __bfloat162float(p[o + 1]), __bfloat162float(p[o + 2]),
+                       __bfloat162float(p[o + 3]));
+}
+
+// One block of m rows (width floats each, width % 4 == 0, width <= 512):
+// rows 0..n_tail-1 are the tail's rows, the others rows of `fresh`.
+template <typename T>
+struct BlockRows {
+    const float *tail;
+    const T *fresh;
+    int n_tail, width;
+    bool vec;
+    __device__ __forceinline__ float4 get(int i, int c4) const {
+        if (i < n_tail) return *reinterpret_cast<const float4 *>(tail + (size_t)i * width + 4 * c4);
+        return load4<T>(fresh, (size_t)(i - n_tail) * width + 4 * c4, vec);
+    }
+};
+
+constexpr int kMaxIdxPerThread = 2;   // index-key inputs (dI <= 512) per thread
+constexpr int kStageRows = 32;    // block rows staged in shared memory at a time
+constexpr int kStageBatch = 16;   // float4 loads a thread keeps in flight while staging
+
+// Rows c0 .. c0+R-1 of the block into xs[R][width] (shared memory); all of a
+// thread's loads of a batch are issued before any store.
+template <typename T>
+__device__ __forceinline__ void stage_rows(const BlockRows<T> &x, int c0, int R, float *xs) {
+    const int nq = x.width >> 2, total = R * nq;
+    for (int i0 = 0; i0 < total; i0 += kThreads * kStageBatch) {
+        float4 v[kStageBatch];
+#pragma unroll
+        for (int u = 0; u < kStageBatch; ++u) {
+            const int idx = i0 + u * kThreads + threadIdx.x;
+            if (idx < total) v[u] = x.get(c0 + idx / nq, idx % nq);
         }
-        acc = warp_sum(acc);
-        if (lane == 0) alpha[i] = acc + __ldg(bias + i);
+#pragma unroll
+        for (int u = 0; u < kStageBatch; ++u) {
+            const int idx = i0 + u * kThreads + threadIdx.x;
+            if (idx < total) reinterpret_cast<float4 *>(xs)[idx] = v[u];
+        }
+    }
+}
+
+// Pool the block with softmax weights of the scalar gates g_i = <x_i, w> +
+// bias_i.  On entry alpha[i] = bias_i and wsm = w (smem); the pooled row
+// (width floats) goes to out (smem).  The rows pass through shared memory
+// (xs) kStageRows at a time; a block of at most kStageRows rows is staged
+// once for both passes.  Gates: one warp per row, lane l sums columns
+// 4(l + 32j) .. +3 in order of j, then a butterfly over the lanes.  Pooled
+// sum: G = 256 / (width / 4) row groups; group g sums rows g, g + G, ... in
+// order, and the groups are added in order.
+template <typename T>
+__device__ void pool_block(const BlockRows<T> &x, int m, const float *wsm, float *alpha, float *part, float *xs,
+                           float *out, float *red) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int width = x.width, nq = width >> 2;
+    const float4 *xs4 = reinterpret_cast<const float4 *>(xs);
+    const float4 *w4 = reinterpret_cast<const float4 *>(wsm);
+    const bool staged_once = m <= kStageRows;
+    for (int c0 = 0; c0 < m; c0 += kStageRows) {
+        const int R = min(kStageRows, m - c0);
+        __syncthreads();   // the previous chunk is consumed
+        stage_rows(x, c0, R, xs);
+        __syncthreads();
+        for (int r = warp; r < R; r += kWarps) {
+            float acc = 0.f;
+            for (int c4 = lane; c4 < nq; c4 += 32) {
+                const float4 xv = xs4[r * nq + c4], wv = w4[c4];
+                acc = __fmaf_rn(xv.x, wv.x, acc);
+                acc = __fmaf_rn(xv.y, wv.y, acc);
+                acc = __fmaf_rn(xv.z, wv.z, acc);
+                acc = __fmaf_rn(xv.w, wv.w, acc);
+            }
+            acc = warp_sum(acc);
+            if (lane == 0) alpha[c0 + r] = __fadd_rn(acc, alpha[c0 + r]);
+        }
     }
     __syncthreads();
     float gmax = -INFINITY;
@@ -86,140 +166,187 @@ __device__ void block_gate(RowFn row_ptr, int m, int width, const float *w, cons
     gmax = block_max<kWarps>(gmax, red);
     float e = 0.f;
     for (int i = threadIdx.x; i < m; i += kThreads) {
-        const float ev = expf(alpha[i] - gmax);
+        const float ev = expf(__fsub_rn(alpha[i], gmax));
         alpha[i] = ev;
-        e += ev;
+        e = __fadd_rn(e, ev);
     }
     const float z = block_sum<kWarps>(e, red);   // ends with __syncthreads
-    for (int i = threadIdx.x; i < m; i += kThreads) alpha[i] = alpha[i] / z;
+    for (int i = threadIdx.x; i < m; i += kThreads) alpha[i] = __fdiv_rn(alpha[i], z);
+    __syncthreads();
+    const int G = kThreads / nq;   // nq <= 128, so G >= 2
+    const int g = threadIdx.x / nq, c4 = threadIdx.x % nq;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = 0; c0 < m; c0 += kStageRows) {
+        const int R = min(kStageRows, m - c0);
+        if (!staged_once) {
+            __syncthreads();
+            stage_rows(x, c0, R, xs);
+            __syncthreads();
+        }
+        if (g < G) {
+            for (int r = g; r < R; r += G) {
+                const float al = alpha[c0 + r];
+                const float4 xv = xs4[r * nq + c4];
+                acc.x = __fmaf_rn(al, xv.x, acc.x);
+                acc.y = __fmaf_rn(al, xv.y, acc.y);
+                acc.z = __fmaf_rn(al, xv.z, acc.z);
+                acc.w = __fmaf_rn(al, xv.w, acc.w);
+            }
+        }
+    }
+    if (g < G) reinterpret_cast<float4 *>(part)[g * nq + c4] = acc;
+    __syncthreads();
+    for (int d = threadIdx.x; d < width; d += kThreads) {
+        float t = part[d];
+        for (int q = 1; q < G; ++q) t = __fadd_rn(t, part[q * width + d]);
+        out[d] = t;
+    }
     __syncthreads();
 }
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs a) {
-    extern __shared__ float sm[];
-    float *v = sm;                       // [D]
-    float *alpha = sm + a.D;             // [m]
-    float *red = alpha + a.m;            // [32]
+    CSLA_TL_SCOPE(kTlCompress);
+    extern __shared__ __align__(16) float sm[];
+    const int D = a.D, m = a.m;
+    const int W = D > a.dI ? D : a.dI;  // widest row pooled (KV or index key)
+    float *v = sm;                      // [W]
+    float *gam = v + W;                 // [D]   gamma_kv
+    float *wsm = gam + D;               // [W]   gate weight (wg, or wgi for index keys)
+    float *alpha = wsm + W;             // [m]   gate bias, then weights
+    float *part = alpha + m;            // [4 * kThreads]
+    float *red = part + 4 * kThreads;   // [32]
+    float *xs = red + 32;               // [min(m, kStageRows)][W]  staged block rows
     __shared__ int s_old_len;
-
-    const int tok = blockIdx.x, b = blockIdx.y;
-    const int slot = a.slots[b];
+    pdl_trigger();
+    const int x = blockIdx.x, b = blockIdx.y, z = blockIdx.z;
+    const bool token = x < a.T;
+    if (token && z != 0) return;
+    if (!token && z == 1 && a.kidx == nullptr) return;
+    const int slot = __ldg(a.slots + b);
     if (slot < 0 || slot >= a.n_slots) {
-        if (threadIdx.x == 0 && tok == 0) set_dev_err(CSLA_DEVERR_INDEX);
+        if (threadIdx.x == 0 && x == 0 && z == 0) set_dev_err(CSLA_DEVERR_INDEX);
         return;
     }
+    // ---- before the wait: only this call's read-only inputs (weights and
+    // the new rows), into shared memory and registers
+    const bool in_window = token && x >= a.T - a.n_win;   // token stays in the ring
+    float kreg[kMaxIdxPerThread];
+    if (z == 0)
+        for (int d = threadIdx.x; d < D; d += kThreads) gam[d] = __ldg(a.gamma_kv + d);
+    if (token) {
+        const T *kv = reinterpret_cast<const T *>(a.kv_new) + ((size_t)b * a.T + x) * D;
+        if (a.T == 1 || in_window)
+            for (int d = threadIdx.x; d < D; d += kThreads) v[d] = load_act<T>(kv, d);
+        if (a.T == 1 && a.kidx != nullptr) {
+            const T *ki = reinterpret_cast<const T *>(a.kidx_new) + (size_t)b * a.dI;
+#pragma unroll
+            for (int u = 0; u < kMaxIdxPerThread; ++u) {
+                const int e = threadIdx.x + u * kThreads;
+                kreg[u] = e < a.dI ? load_act<T>(ki, e) : 0.f;
+            }
+        }
+    } else {
+        const int width = z == 0 ? D : a.dI;
+        const float *w = z == 0 ? a.wg : a.wgi;
+        const float *gb = z == 0 ? a.gb : a.gbi;
+        for (int d = threadIdx.x; d < width; d += kThreads) wsm[d] = __ldg(w + d);
+        for (int i = threadIdx.x; i < m; i += kThreads) alpha[i] = __ldg(gb + i);
+    }
+    pdl_wait();
+    CSLA_TL_WAITED();
+
     if (threadIdx.x == 0) s_old_len = a.len[slot];
     __syncthreads();
+    CSLA_TL_MARK(0);
     const long long L0 = s_old_len;
-    const long long pos = L0 + tok;
     const long long L1 = L0 + a.T;
-    const int D = a.D, m = a.m;
     const int rb = (D - a.d_rope) + 2 * a.d_rope;
-    const T *kv = reinterpret_cast<const T *>(a.kv_new) + ((size_t)b * a.T + tok) * D;
 
-    // 1. sliding-window row of this token (only tokens that stay in the ring)
-    if (pos >= L1 - a.n_win) {
-        for (int d = threadIdx.x; d < D; d += kThreads) v[d] = load_act<T>(kv, d);
-        __syncthreads();
-        const size_t ring = (size_t)slot * a.n_win + (size_t)(pos % a.n_win);
-        norm_rope_quantise(v, a, pos, a.win_rows + ring * rb, a.win_scales + ring, red);
-        __syncthreads();
-    }
-
-    // 2. block closed by this token -> one compressed entry (+ index key)
-    if ((pos + 1) % m == 0) {
-        const long long bk = pos / m;
-        const long long p0 = bk * m;
-        const int epp = CSLA_PAGE_TOKENS / m;
-        const long long col = bk / epp;
-        const int page = col < a.bt_stride ? a.block_table[(size_t)slot * a.bt_stride + (size_t)col] : -1;
-        const bool page_ok = page >= 0 && page < a.n_pages;
-        if (!page_ok && threadIdx.x == 0) set_dev_err(CSLA_DEVERR_PAGE);
-        const T *kv_b = reinterpret_cast<const T *>(a.kv_new) + (size_t)b * a.T * D;
-        const float *tail = a.tail_kv + (size_t)slot * m * D;
-        auto row_kv = [&](int i, const T **x, const float **xf) {
-            const long long p = p0 + i;
-            if (p < L0) *xf = tail + (size_t)(p % m) * D;
-            else *x = kv_b + (size_t)(p - L0) * D;
-        };
-        block_gate<T>(row_kv, m, D, a.wg, a.gb, alpha, red);
-        for (int d = threadIdx.x; d < D; d += kThreads) {
-            float c = 0.f;
-            for (int i = 0; i < m; ++i) {
-                const T *x = nullptr;
-                const float *xf = nullptr;
-                row_kv(i, &x, &xf);
-                c += alpha[i] * (xf ? xf[d] : load_act<T>(x, d));
-            }
-            v[d] = c;
-        }
-        __syncthreads();
-        if (page_ok) {
-            const size_t e = (size_t)page * epp + (size_t)(bk % epp);
-            norm_rope_quantise(v, a, p0, a.rows + e * rb, a.scales + e, red);
-        }
-        __syncthreads();
-        if (a.kidx != nullptr) {   // CSA: compressed index key
-            const int dI = a.dI;
-            const T *ki_b = reinterpret_cast<const T *>(a.kidx_new) + (size_t)b * a.T * dI;
-            const float *tail_i = a.tail_idx + (size_t)slot * m * dI;
-            auto row_ix = [&](int i, const T **x, const float **xf) {
-                const long long p = p0 + i;
-                if (p < L0) *xf = tail_i + (size_t)(p % m) * dI;
-                else *x = ki_b + (size_t)(p - L0) * dI;
-            };
-            block_gate<T>(row_ix, m, dI, a.wgi, a.gbi, alpha, red);
-            for (int e = threadIdx.x; e < dI; e += kThreads) {
-                float c = 0.f;
-                for (int i = 0; i < m; ++i) {
-                    const T *x = nullptr;
-                    const float *xf = nullptr;
-                    row_ix(i, &x, &xf);
-                    c += alpha[i] * (xf ? xf[e] : load_act<T>(x, e));
+    if (token) {
+        // ---- token x: window row (+ tail row for single-token calls)
+        const long long pos = L0 + x;
+        if (a.T == 1) {
+            // the pooled block never reads this slot: it takes the new row from kv_new
+            const int ts = (int)(pos % m);
+            for (int d = threadIdx.x; d < D; d += kThreads) a.tail_kv[((size_t)slot * m + ts) * D + d] = v[d];
+            if (a.kidx != nullptr) {
+#pragma unroll
+                for (int u = 0; u < kMaxIdxPerThread; ++u) {
+                    const int e = threadIdx.x + u * kThreads;
+                    if (e < a.dI) a.tail_idx[((size_t)slot * m + ts) * a.dI + e] = kreg[u];
                 }
-                if (page_ok)
-                    a.kidx[((size_t)page * epp + (size_t)(bk % epp)) * dI + e] = f32_to_bf16_bits(c);
             }
         }
-        __syncthreads();
+        CSLA_TL_MARK(1);
+        if (!in_window) return;
+        const size_t ring = (size_t)slot * a.n_win + (size_t)(pos % a.n_win);
+        norm_rope_quantise(v, gam, a, pos, a.win_rows + ring * rb, a.win_scales + ring, red);
+        CSLA_TL_MARK(2);
+        return;
     }
-
-    // 3. single-token calls: push the raw row into the tail and bump len here
-    //    (the block read above finished before this overwrite).
-    if (a.T == 1) {
-        const int ts = (int)(pos % m);
-        for (int d = threadIdx.x; d < D; d += kThreads)
-            a.tail_kv[((size_t)slot * m + ts) * D + d] = load_act<T>(kv, d);
-        if (a.kidx != nullptr) {
-            const T *ki = reinterpret_cast<const T *>(a.kidx_new) + (size_t)b * a.dI;
-            for (int e = threadIdx.x; e < a.dI; e += kThreads)
-                a.tail_idx[((size_t)slot * m + ts) * a.dI + e] = load_act<T>(ki, e);
-        }
-        if (threadIdx.x == 0) a.len[slot] = (int32_t)L1;
+    // ---- the (x - T)-th block completed by this call
+    const long long bk = L0 / m + (x - a.T);
+    if ((bk + 1) * m > L1) return;                     // no such block in this call
+    const long long p0 = bk * m;
+    const int epp = CSLA_PAGE_TOKENS / m;
+    const long long col = bk / epp;
+    const int page = col < a.bt_stride ? a.block_table[(size_t)slot * a.bt_stride + (size_t)col] : -1;
+    if (page < 0 || page >= a.n_pages) {
+        if (threadIdx.x == 0) set_dev_err(CSLA_DEVERR_PAGE);
+        return;
+    }
+    const size_t ent = (size_t)page * epp + (size_t)(bk % epp);
+    const long long nt = L0 - p0;
+    const int n_tail = nt <= 0 ? 0 : (int)(nt < m ? nt : m);
+    const size_t f0 = (size_t)(p0 + n_tail - L0);      // kv_new row of the block's first fresh row
+    const uintptr_t vec_mask = sizeof(T) == 4 ? 15u : 7u;
+    if (z == 0) {
+        const T *fresh = reinterpret_cast<const T *>(a.kv_new) + ((size_t)b * a.T + f0) * D;
+        const BlockRows<T> rows{a.tail_kv + (size_t)slot * m * D, fresh, n_tail, D,
+                                (reinterpret_cast<uintptr_t>(a.kv_new) & vec_mask) == 0};
+        pool_block<T>(rows, m, wsm, alpha, part, xs, v, red);
+        CSLA_TL_MARK(1);
+        norm_rope_quantise(v, gam, a, p0, a.rows + ent * rb, a.scales + ent, red);
+        CSLA_TL_MARK(2);
+    } else {
+        const int dI = a.dI;
+        const T *fresh = reinterpret_cast<const T *>(a.kidx_new) + ((size_t)b * a.T + f0) * dI;
+        const BlockRows<T> rows{a.tail_idx + (size_t)slot * m * dI, fresh, n_tail, dI,
+                                (reinterpret_cast<uintptr_t>(a.kidx_new) & vec_mask) == 0};
+        pool_block<T>(rows, m, wsm, alpha, part, xs, v, red);
+        CSLA_TL_MARK(1);
+        for (int e = threadIdx.x; e < dI; e += kThreads) a.kidx[ent * dI + e] = f32_to_bf16_bits(v[e]);
+        CSLA_TL_MARK(2);
     }
 }
 
-// Multi-token calls: after every block read the old tail, store the raw rows
-// of the still-open last block and set len.  grid = B.
+// After the pooling: raw rows of the still-open last block of multi-token
+// calls go to the tail; len advances.  grid = B.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) tail_update_kernel(CompressArgs a) {
+    CSLA_TL_SCOPE(kTlTailUpdate);
+    pdl_trigger();
     const int b = blockIdx.x;
-    const int slot = a.slots[b];
+    const int slot = __ldg(a.slots + b);
+    pdl_wait();
+    CSLA_TL_WAITED();
     if (slot < 0 || slot >= a.n_slots) return;
     const long long L0 = a.len[slot];
     const long long L1 = L0 + a.T;
     const int m = a.m, D = a.D;
-    long long start = (L1 / m) * m;
-    if (start < L0) start = L0;
-    for (long long p = start; p < L1; ++p) {
-        const T *kv = reinterpret_cast<const T *>(a.kv_new) + ((size_t)b * a.T + (size_t)(p - L0)) * D;
-        for (int d = threadIdx.x; d < D; d += kThreads)
-            a.tail_kv[((size_t)slot * m + (size_t)(p % m)) * D + d] = load_act<T>(kv, d);
-        if (a.kidx != nullptr) {
-            const T *ki = reinterpret_cast<const T *>(a.kidx_new) + ((size_t)b * a.T + (size_t)(p - L0)) * a.dI;
-            for (int e = threadIdx.x; e < a.dI; e += kThreads)
-                a.tail_idx[((size_t)slot * m + (size_t)(p % m)) * a.dI + e] = load_act<T>(ki, e);
+    if (a.T > 1) {
+        long long start = (L1 / m) * m;
+        if (start < L0) start = L0;
+        for (long long p = start; p < L1; ++p) {
+            const T *kv = reinterpret_cast<const T *>(a.kv_new) + ((size_t)b * a.T + (size_t)(p - L0)) * D;
+            for (int d = threadIdx.x; d < D; d += kThreads)
+                a.tail_kv[((size_t)slot * m + (size_t)(p % m)) * D + d] = load_act<T>(kv, d);
+            if (a.kidx != nullptr) {
+                const T *ki = reinterpret_cast<const T *>(a.kidx_new) + ((size_t)b * a.T + (size_t)(p - L0)) * a.dI;
+                for (int e = threadIdx.x; e < a.dI; e += kThreads)
+                    a.tail_idx[((size_t)slot * m + (size_t)(p % m)) * a.dI + e] = load_act<T>(ki, e);
+            }
         }
     }
     __syncthreads();
@@ -229,15 +356,30 @@ __global__ void __launch_bounds__(kThreads) tail_update_kernel(CompressArgs a) {
 }  // namespace
 
 cudaError_t launch_compress_append(const CompressArgs &a, bool bf16, cudaStream_t stream) {
-    const size_t smem = ((size_t)a.D + (size_t)a.m + 32) * sizeof(float);
-    dim3 grid(a.T, a.B);
-    if (bf16) compress_append_kernel<__nv_bfloat16><<<grid, kThreads, smem, stream>>>(a);
-    else compress_append_kernel<float><<<grid, kThreads, smem, stream>>>(a);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess || a.T == 1) return e;
-    if (bf16) tail_update_kernel<__nv_bfloat16><<<a.B, kThreads, 0, stream>>>(a);
-    else tail_update_kernel<float><<<a.B, kThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+    const int nb = a.T / a.m + 1;   // blocks one call can complete
+    const size_t W = (size_t)(a.D > a.dI ? a.D : a.dI);
+    const size_t R = (size_t)(a.m < kStageRows ? a.m : kStageRows);
+    const size_t smem = (2 * W + (size_t)a.D + (size_t)a.m + 4 * kThreads + 32 + R * W) * sizeof(float);
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        // largest case: W = 512, m = 128
+        const int most = (int)((2 * 512 + 512 + 128 + 4 * kThreads + 32 + kStageRows * 512) * sizeof(float));
+        cudaError_t e = cudaFuncSetAttribute(compress_append_kernel<float>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(compress_append_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 most);
+        if (e != cudaSuccess) return e;
+        configured_dev = dev;
+    }
+    const dim3 grid(a.T + nb, a.B, a.kidx ? 2 : 1);
+    cudaError_t e = bf16 ? launch_pdl(compress_append_kernel<__nv_bfloat16>, grid, dim3(kThreads), smem, stream, a)
+                         : launch_pdl(compress_append_kernel<float>, grid, dim3(kThreads), smem, stream, a);
+    if (e != cudaSuccess) return e;
+    return bf16 ? launch_pdl(tail_update_kernel<__nv_bfloat16>, dim3(a.B), dim3(kThreads), 0, stream, a)
+                : launch_pdl(tail_update_kernel<float>, dim3(a.B), dim3(kThreads), 0, stream, a);
 }
 
 }  // namespace csla

@@ -11,10 +11,11 @@
 //     has a fixed summation order.  qI is stored as three bf16 terms
 //     (hi = bf16(qI), mid = bf16(qI - hi), lo = bf16(qI - hi - mid)), so the
 //     bf16 tensor-core products carry the full fp32 value of qI.
-//  2. indexer: persistent, warp-specialised tcgen05 kernel.  A tile is 128
-//     compressed entries of one request (4 pages of 32 entries).  Warp 0
-//     streams key tiles and the request's query operand with TMA into a
-//     4-stage ring; warp 1 issues UMMA (M=128 entries, N=NQ query rows,
+//  2. indexer: warp-specialised tcgen05 kernel; a CTA owns 8 consecutive
+//     tiles of one request, a tile being 128 compressed entries (4 pages of
+//     32).  Warp 0 loads the request's query operand once and streams key
+//     tiles with TMA into a 3-stage ring (page ids fetched up front, one
+//     lane per page); warp 1 issues UMMA (M=128 entries, N=NQ query rows,
 //     K=dI) into one of two TMEM accumulators; warps 2-5 read the
 //     accumulator (one entry per thread) and reduce
 //       score = sum_j w_j * relu((acc[j] + acc[HI + j]) + acc[2HI + j])
@@ -47,8 +48,108 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *p, flo
     }
 }
 
+constexpr int kProjWarps = kProjThreads / 32;   // output features per CTA
+constexpr int kProjChunkB = 8;                   // requests' cq rows staged in shared memory at a time
+constexpr int kProjKeepB = 128;                  // requests whose results are held before the wait
+
+// One warp per output feature r; lane l covers 8-element chunks l, l+32, ...
+// of the dc inputs.  The W row is read once into registers; the cq rows are
+// staged in shared memory kProjChunkB requests at a time.  The products are
+// formed before the grid-dependency wait (W and cq are inputs of the call)
+// and held in shared memory; the stores into the workspace follow the wait.
 template <typename TC, typename TW>
-__global__ void __launch_bounds__(kProjThreads) iq_project_kernel(IndexerArgs a) {
+__global__ void __launch_bounds__(kProjThreads, 2) iq_project_kernel(IndexerArgs a) {
+    CSLA_TL_SCOPE(kTlIqProject);
+    constexpr int kMaxCh = 4;   // dc <= 32 * 8 * kMaxCh = 1024 on this path
+    __shared__ __align__(16) float cs[kProjChunkB][1024];
+    __shared__ uint16_t res[kProjKeepB][kProjWarps][3];
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r0 = blockIdx.x * kProjWarps;
+    const int r = r0 + warp;
+    const bool active = r < a.HI * a.dI;
+    const TW *w = reinterpret_cast<const TW *>(a.W) + (size_t)(active ? r : 0) * a.dc;
+    const int nch = a.dc / 8;
+    float wv[kMaxCh][8];
+#pragma unroll
+    for (int q = 0; q < kMaxCh; ++q) {
+        const int ch = lane + 32 * q;
+        if (active && ch < nch) load8<TW>(w + ch * 8, wv[q]);
+        else
+#pragma unroll
+            for (int i = 0; i < 8; ++i) wv[q][i] = 0.f;
+    }
+    bool waited = false;
+    int held0 = 0;   // first request whose results sit in res
+    for (int b0 = 0; b0 < a.B; b0 += kProjChunkB) {
+        const int nb = min(kProjChunkB, a.B - b0);
+        __syncthreads();   // the previous chunk's cq rows are consumed
+        for (int i = threadIdx.x; i < nb * nch; i += kProjThreads) {
+            const int u = i / nch, ch = i % nch;
+            float t[8];
+            load8<TC>(reinterpret_cast<const TC *>(a.cq) + (size_t)(b0 + u) * a.dc + ch * 8, t);
+            float4 *dst = reinterpret_cast<float4 *>(&cs[u][ch * 8]);
+            dst[0] = make_float4(t[0], t[1], t[2], t[3]);
+            dst[1] = make_float4(t[4], t[5], t[6], t[7]);
+        }
+        __syncthreads();
+        if (active) {
+            for (int u = 0; u < nb; ++u) {
+                float acc = 0.f;
+#pragma unroll
+                for (int q = 0; q < kMaxCh; ++q) {
+                    const int ch = lane + 32 * q;
+                    if (ch < nch) {
+                        const float4 c0 = reinterpret_cast<const float4 *>(&cs[u][ch * 8])[0];
+                        const float4 c1 = reinterpret_cast<const float4 *>(&cs[u][ch * 8])[1];
+                        const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) acc = __fmaf_rn(wv[q][i], cv[i], acc);
+                    }
+                }
+                acc = warp_sum(acc);
+                if (lane == 0) {
+                    const uint16_t hi = f32_to_bf16_bits(acc);
+                    const float r1 = __fsub_rn(acc, bf16_bits_to_f32(hi));
+                    const uint16_t mid = f32_to_bf16_bits(r1);
+                    const uint16_t lo = f32_to_bf16_bits(__fsub_rn(r1, bf16_bits_to_f32(mid)));
+                    uint16_t *o = res[(b0 + u) - held0][warp];
+                    o[0] = hi;
+                    o[1] = mid;
+                    o[2] = lo;
+                }
+            }
+        }
+        const int held = b0 + nb - held0;
+        if (held == kProjKeepB || b0 + nb == a.B) {
+            __syncthreads();
+            if (!waited) {
+                pdl_wait();
+                CSLA_TL_WAITED();
+                waited = true;
+            }
+            const int nf = min(kProjWarps, a.HI * a.dI - r0);
+            for (int i = threadIdx.x; i < held * nf * 3; i += kProjThreads) {
+                const int f = i % nf, t = (i / nf) % 3, bb = i / (3 * nf);
+                const int rr = r0 + f, j = rr / a.dI, e = rr % a.dI;
+                a.q_ws[((size_t)(held0 + bb) * a.NQ + t * a.HI + j) * a.dI + e] = res[bb][f][t];
+            }
+            held0 = b0 + nb;
+        }
+    }
+    if (!waited) {
+        pdl_wait();
+        CSLA_TL_WAITED();
+    }
+}
+
+// Same product for latents wider than 1024 (W row re-read per request).
+template <typename TC, typename TW>
+__global__ void __launch_bounds__(kProjThreads) iq_project_wide_kernel(IndexerArgs a) {
+    CSLA_TL_SCOPE(kTlIqProjectWide);
+    pdl_trigger();
+    pdl_wait();
+    CSLA_TL_WAITED();
     const int r = blockIdx.x * (kProjThreads / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (r >= a.HI * a.dI) return;
@@ -63,7 +164,7 @@ __global__ void __launch_bounds__(kProjThreads) iq_project_kernel(IndexerArgs a)
             load8<TW>(w + ch * 8, wv);
             load8<TC>(c + ch * 8, cv);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc = fmaf(wv[i], cv[i], acc);
+            for (int i = 0; i < 8; ++i) acc = __fmaf_rn(wv[i], cv[i], acc);
         }
         acc = warp_sum(acc);
         if (lane == 0) {
@@ -78,17 +179,17 @@ __global__ void __launch_bounds__(kProjThreads) iq_project_kernel(IndexerArgs a)
     }
 }
 
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kTileE = 128;          // entries per tile
 constexpr int kPageE = 32;           // CSA entries per 128-token page
+constexpr int kTPC = 8;              // tiles per CTA (consecutive, one request)
 constexpr int kIdxThreads = 192;     // warp 0: TMA, warp 1: MMA, warps 2..5: epilogue
 
 template <int DI, int NQ>
 struct IdxSmem {
     static constexpr int kKeyBytes = kTileE * DI * 2;
     static constexpr int kQBytes = NQ * DI * 2;
-    static constexpr int kStageBytes = kKeyBytes + kQBytes;
-    static constexpr int kBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+    static constexpr int kBytes = kStages * kKeyBytes + kQBytes + 1024 /*align*/ + 512 /*barriers, pages*/;
 };
 
 // Two accumulators of NQ columns, rounded up to a power of two >= 32.
@@ -97,38 +198,31 @@ constexpr uint32_t kTmemCols() {
     return 2 * NQ <= 32 ? 32 : (2 * NQ <= 64 ? 64 : 128);
 }
 
-// Tile bookkeeping shared by the three roles (all must skip the same tiles).
-struct TileInfo {
-    int b, tt, slot, nv;
-    bool live;
-};
-__device__ __forceinline__ TileInfo tile_info(const IndexerArgs &a, int tile) {
-    TileInfo t;
-    t.b = tile / a.tiles_per_req;
-    t.tt = tile % a.tiles_per_req;
-    t.slot = __ldg(a.slots + t.b);
-    const bool slot_ok = t.slot >= 0 && t.slot < a.n_slots;
-    const int L = slot_ok ? __ldg(a.len + t.slot) : 0;
-    t.nv = (slot_ok && L <= a.max_len) ? L / a.m : 0;
-    t.live = t.tt * kTileE < t.nv;
-    return t;
-}
-
+// CTA (blockIdx.x, blockIdx.y = request b) scores tiles
+// [blockIdx.x*kTPC, blockIdx.x*kTPC + kTPC) of request b (128 entries each).
 template <int DI, int NQ, int HI>
-__global__ void __launch_bounds__(kIdxThreads, 1)
+__global__ void __launch_bounds__(kIdxThreads)
     indexer_kernel(IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap qmap) {
+    CSLA_TL_SCOPE(kTlIndexer);
     using S = IdxSmem<DI, NQ>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(base + kStages * S::kStageBytes);
+    uint8_t *qbuf = base + kStages * S::kKeyBytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(qbuf + S::kQBytes);
     uint64_t *full = bars, *empty = bars + kStages, *tfull = bars + 2 * kStages, *tempty = tfull + 2;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tempty + 2);
+    uint64_t *qfull = tempty + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(qfull + 1);
+    int *pages = reinterpret_cast<int *>(tmem_holder + 1);      // [kTPC * 4]
     __shared__ volatile int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int total = a.B * a.tiles_per_req;
+    const int b = blockIdx.y;
+    const int slot = __ldg(a.slots + b);
+    const bool slot_ok = slot >= 0 && slot < a.n_slots;
+    const int t_begin = blockIdx.x * kTPC;
 
+    // ---- before the wait: barriers, TMEM, page ids, head weights
     if (threadIdx.x == 0) {
         abort_flag = 0;
         for (int s = 0; s < kStages; ++s) {
@@ -139,98 +233,116 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             mbar_init(tfull + i, 1);
             mbar_init(tempty + i, 128);
         }
+        mbar_init(qfull, 1);
         fence_mbar_init();
-        tma_prefetch_desc(&kmap);
-        tma_prefetch_desc(&qmap);
+    }
+    int pg = -1;   // warp 0: page id of this CTA's page `lane`
+    if (warp == 0) {
+        const int col = (t_begin * kTileE + lane * kPageE) / kPageE;
+        if (slot_ok && lane < kTPC * 4 && col < a.bt_stride)
+            pg = __ldg(a.block_table + (size_t)slot * a.bt_stride + col);
+        if (lane == 0) {
+            tma_prefetch_desc(&kmap);
+            tma_prefetch_desc(&qmap);
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_holder, kTmemCols<NQ>());
         tmem_relinquish();
     }
+    float wj[HI];
+    if (warp >= 2) {
+        const float *w = a.head_w + (size_t)b * HI;
+#pragma unroll
+        for (int j = 0; j < HI; ++j) wj[j] = __ldg(w + j);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    // the next kernel may start only once this CTA holds its TMEM: a later
+    // kernel's CTA allocating first and then waiting on this grid could
+    // otherwise keep this CTA from ever getting its columns
+    pdl_trigger();
+    pdl_wait();
+    CSLA_TL_WAITED();
 
-    if (warp == 0) {
+    const int L = slot_ok ? a.len[slot] : 0;
+    const bool ok = slot_ok && L <= a.max_len;
+    if (!ok && threadIdx.x == 0 && blockIdx.x == 0) set_dev_err(slot_ok ? CSLA_DEVERR_LEN : CSLA_DEVERR_INDEX);
+    const int nv = ok ? L / a.m : 0;
+    const int n_tiles = ok ? min(kTPC, (nv + kTileE - 1) / kTileE - t_begin) : 0;
+    if (warp == 0 && lane < kTPC * 4) {
+        const int e0 = t_begin * kTileE + lane * kPageE;
+        if (e0 < nv && (pg < 0 || pg >= a.n_pages)) {
+            set_dev_err(CSLA_DEVERR_PAGE);
+            pg = -1;
+        }
+        pages[lane] = e0 < nv ? pg : -1;
+    }
+    __syncwarp();
+
+    if (n_tiles <= 0) {
+        // nothing to score: fall through to the teardown
+    } else if (warp == 0) {
         if (lane == 0) {
+            mbar_arrive_expect_tx(qfull, (uint32_t)S::kQBytes);
+#pragma unroll
+            for (int h = 0; h < DI / 64; ++h) tma_load_2d(qbuf + h * NQ * 128, &qmap, h * 64, b * NQ, qfull);
             int n = 0;
-            for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
-                const TileInfo t = tile_info(a, tile);
-                if (!t.live) continue;
+            for (int t = 0; t < n_tiles; ++t, ++n) {
                 const int s = n % kStages;
                 if (n >= kStages && !mbar_wait(empty + s, ((n / kStages) - 1) & 1, &abort_flag)) break;
-                uint8_t *kb = base + s * S::kStageBytes;
-                uint8_t *qb = kb + S::kKeyBytes;
-                int pages[4];
+                uint8_t *kb = base + s * S::kKeyBytes;
                 int np = 0;
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const int e0 = t.tt * kTileE + p * kPageE;
-                    pages[p] = -1;
-                    if (e0 < t.nv) {
-                        const int col = e0 / kPageE;
-                        const int pg = col < a.bt_stride ? __ldg(a.block_table + (size_t)t.slot * a.bt_stride + col) : -1;
-                        if (pg >= 0 && pg < a.n_pages) {
-                            pages[p] = pg;
-                            ++np;
-                        } else {
-                            set_dev_err(CSLA_DEVERR_PAGE);
-                        }
-                    }
-                }
-                mbar_arrive_expect_tx(full + s, (uint32_t)(S::kQBytes + np * kPageE * DI * 2));
-#pragma unroll
-                for (int h = 0; h < DI / 64; ++h)
-                    tma_load_2d(qb + h * NQ * 128, &qmap, h * 64, t.b * NQ, full + s);
+                for (int p = 0; p < 4; ++p) np += pages[t * 4 + p] >= 0;
+                mbar_arrive_expect_tx(full + s, (uint32_t)(np * kPageE * DI * 2));
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
-                    if (pages[p] < 0) continue;
+                    const int pg = pages[t * 4 + p];
+                    if (pg < 0) continue;
 #pragma unroll
                     for (int h = 0; h < DI / 64; ++h)
-                        tma_load_2d(kb + h * (kTileE * 128) + p * (kPageE * 128), &kmap, h * 64,
-                                    pages[p] * kPageE, full + s);
+                        tma_load_2d(kb + h * (kTileE * 128) + p * (kPageE * 128), &kmap, h * 64, pg * kPageE,
+                                    full + s);
                 }
-                ++n;
             }
             // every issued copy must land before the CTA may exit
             for (int i = (n > kStages ? n - kStages : 0); i < n; ++i)
                 mbar_wait(full + (i % kStages), (i / kStages) & 1, nullptr);
+            mbar_wait(qfull, 0, nullptr);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16(128, NQ, false, false);
             int n = 0;
-            for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
-                const TileInfo t = tile_info(a, tile);
-                if (!t.live) continue;
-                const int s = n % kStages;
-                const int acc = n & 1;
-                if (!mbar_wait(full + s, (n / kStages) & 1, &abort_flag)) break;
-                if (n >= 2 && !mbar_wait(tempty + acc, ((n / 2) - 1) & 1, &abort_flag)) break;
-                tc_fence_after();
-                const uint32_t kb = smem_u32(base + s * S::kStageBytes);
-                const uint32_t qb = kb + S::kKeyBytes;
+            if (mbar_wait(qfull, 0, &abort_flag)) {
+                const uint32_t qb = smem_u32(qbuf);
+                for (int t = 0; t < n_tiles; ++t, ++n) {
+                    const int s = n % kStages;
+                    const int acc = n & 1;
+                    if (!mbar_wait(full + s, (n / kStages) & 1, &abort_flag)) break;
+                    if (n >= 2 && !mbar_wait(tempty + acc, ((n / 2) - 1) & 1, &abort_flag)) break;
+                    tc_fence_after();
+                    const uint32_t kb = smem_u32(base + s * S::kKeyBytes);
 #pragma unroll
-                for (int k = 0; k < DI / 16; ++k) {
-                    const uint32_t half = k / 4, ko = (k % 4) * 32;
-                    const uint64_t ad = sdesc(kb + half * (kTileE * 128) + ko, 16, 1024);
-                    const uint64_t bd = sdesc(qb + half * (NQ * 128) + ko, 16, 1024);
-                    umma_bf16(tmem + acc * NQ, ad, bd, idesc, k > 0 ? 1u : 0u);
+                    for (int k = 0; k < DI / 16; ++k) {
+                        const uint32_t half = k / 4, ko = (k % 4) * 32;
+                        const uint64_t ad = sdesc(kb + half * (kTileE * 128) + ko, 16, 1024);
+                        const uint64_t bd = sdesc(qb + half * (NQ * 128) + ko, 16, 1024);
+                        umma_bf16(tmem + acc * NQ, ad, bd, idesc, k > 0 ? 1u : 0u);
+                    }
+                    umma_commit(empty + s);
+                    umma_commit(tfull + acc);
                 }
-                umma_commit(empty + s);
-                umma_commit(tfull + acc);
-                ++n;
             }
             if (n > 0) mbar_wait(tfull + ((n - 1) & 1), ((n - 1) / 2) & 1, nullptr);
         }
     } else {
         const int lane_base = 32 * (warp & 3);
         const int row = lane_base + lane;
-        int n = 0;
-        for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
-            const TileInfo t = tile_info(a, tile);
-            if (!t.live) continue;
+        for (int t = 0, n = 0; t < n_tiles; ++t, ++n) {
             const int acc = n & 1;
             if (!mbar_wait(tfull + acc, (n / 2) & 1, &abort_flag)) break;
             tc_fence_after();
@@ -250,19 +362,17 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(tempty + acc);
-            const int e = t.tt * kTileE + row;
-            if (e < t.nv) {
-                const float *w = a.head_w + (size_t)t.b * HI;
+            const int e = (t_begin + t) * kTileE + row;
+            if (e < nv) {
                 float sc = 0.f;
 #pragma unroll
                 for (int j = 0; j < HI; ++j) {
                     const float dot = __fadd_rn(__fadd_rn(__uint_as_float(r[j]), __uint_as_float(r[HI + j])),
                                                 __uint_as_float(r[2 * HI + j]));
-                    sc = __fmaf_rn(__ldg(w + j), fmaxf(dot, 0.f), sc);
+                    sc = __fmaf_rn(wj[j], fmaxf(dot, 0.f), sc);
                 }
-                a.scores[(size_t)t.b * a.scores_stride + e] = sc;
+                a.scores[(size_t)b * a.scores_stride + e] = sc;
             }
-            ++n;
         }
     }
     tc_fence_before();
@@ -286,11 +396,10 @@ cudaError_t launch_indexer_t(const IndexerArgs &a, const CUtensorMap &kmap, cons
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
-    const int total = a.B * a.tiles_per_req;
-    int grid = total < num_sms ? total : num_sms;
-    if (grid < 1) grid = 1;
-    indexer_kernel<DI, NQ, HI><<<grid, kIdxThreads, S::kBytes, stream>>>(a, kmap, qmap);
-    return cudaGetLastError();
+    (void)num_sms;
+    const int groups = (a.tiles_per_req + kTPC - 1) / kTPC;
+    return launch_pdl(indexer_kernel<DI, NQ, HI>, dim3(groups, a.B), dim3(kIdxThreads), S::kBytes, stream, a, kmap,
+                      qmap);
 }
 
 }  // namespace
@@ -302,11 +411,19 @@ cudaError_t launch_indexer(const IndexerArgs &a, bool cq_bf16, bool w_bf16, cons
         if (e != cudaSuccess) return e;
     }
     const int pblocks = (a.HI * a.dI + kProjThreads / 32 - 1) / (kProjThreads / 32);
-    if (cq_bf16 && w_bf16) iq_project_kernel<__nv_bfloat16, __nv_bfloat16><<<pblocks, kProjThreads, 0, stream>>>(a);
-    else if (cq_bf16) iq_project_kernel<__nv_bfloat16, float><<<pblocks, kProjThreads, 0, stream>>>(a);
-    else if (w_bf16) iq_project_kernel<float, __nv_bfloat16><<<pblocks, kProjThreads, 0, stream>>>(a);
-    else iq_project_kernel<float, float><<<pblocks, kProjThreads, 0, stream>>>(a);
-    cudaError_t e = cudaGetLastError();
+    const dim3 pg(pblocks), pb(kProjThreads);
+    cudaError_t e;
+    if (a.dc <= 1024) {
+        if (cq_bf16 && w_bf16) e = launch_pdl(iq_project_kernel<__nv_bfloat16, __nv_bfloat16>, pg, pb, 0, stream, a);
+        else if (cq_bf16) e = launch_pdl(iq_project_kernel<__nv_bfloat16, float>, pg, pb, 0, stream, a);
+        else if (w_bf16) e = launch_pdl(iq_project_kernel<float, __nv_bfloat16>, pg, pb, 0, stream, a);
+        else e = launch_pdl(iq_project_kernel<float, float>, pg, pb, 0, stream, a);
+    } else {
+        if (cq_bf16 && w_bf16) e = launch_pdl(iq_project_wide_kernel<__nv_bfloat16, __nv_bfloat16>, pg, pb, 0, stream, a);
+        else if (cq_bf16) e = launch_pdl(iq_project_wide_kernel<__nv_bfloat16, float>, pg, pb, 0, stream, a);
+        else if (w_bf16) e = launch_pdl(iq_project_wide_kernel<float, __nv_bfloat16>, pg, pb, 0, stream, a);
+        else e = launch_pdl(iq_project_wide_kernel<float, float>, pg, pb, 0, stream, a);
+    }
     if (e != cudaSuccess) return e;
     // HI is a template parameter so the epilogue's head loop is unrolled.
     if (a.dI == 128) {

@@ -5,11 +5,43 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace csla {
+
+// RoPE inverse frequencies theta^(-2i/d_rope), i < d_rope/2, computed on the
+// host in double and passed to the kernels.
+struct RopeFreq {
+    double inv[32];
+};
+
+inline RopeFreq rope_freq(float theta, int d_rope) {
+    RopeFreq f{};
+    for (int i = 0; i < d_rope / 2 && i < 32; ++i) f.inv[i] = pow((double)theta, -(2.0 * i) / (double)d_rope);
+    return f;
+}
+
+// Launch with programmatic stream serialization (see pdl_wait in common.cuh).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args &&...args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 struct CompressArgs {
     int m, D, d_rope, dI, n_win;
     float theta, eps;
+    RopeFreq freq;
     const int32_t *slots;
     int B, T;
     const void *kv_new, *kidx_new;
@@ -58,6 +90,7 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream);
 struct AttendArgs {
     int m, D, d_rope, H, n_win;
     float theta, eps;
+    RopeFreq freq;
     const int32_t *slots;
     const int32_t *len;
     int B;
@@ -72,18 +105,20 @@ struct AttendArgs {
     const uint8_t *win_rows;
     const float *win_scales;
     void *out;
-    float *part;          // chunk partials workspace
+    uint8_t *qimg;        // workspace: per request, Qhat as the kernel's shared-memory image
+    float *part;          // workspace: chunk partials
     int max_chunks;
     int max_len;
 };
 cudaError_t launch_attend(const AttendArgs &a, bool q_bf16, bool out_bf16, int variant, int num_sms,
                           cudaStream_t stream);
 
-// Canonical chunk length for a set of n rows (a function of n only).
+// Canonical chunk length for a set of n rows (a function of n only):
+// 64 * ceil(n / 2048) rows, so a request never has more than 32 chunks.
 __host__ __device__ inline int attend_chunk_rows(long long n) {
-    long long c = (n + 8191) / 8192;
+    long long c = (n + 2047) / 2048;
     if (c < 1) c = 1;
-    return (int)(256 * c);
+    return (int)(64 * c);
 }
 __host__ __device__ inline int attend_num_chunks(long long n) {
     const int c = attend_chunk_rows(n);
@@ -91,7 +126,7 @@ __host__ __device__ inline int attend_num_chunks(long long n) {
 }
 // Largest chunk count over all set sizes <= n (never above 32).
 __host__ __device__ inline int attend_max_chunks(long long n) {
-    const long long c = (n + 255) / 256;
+    const long long c = (n + 63) / 64;
     return (int)(c < 1 ? 1 : (c > 32 ? 32 : c));
 }
 

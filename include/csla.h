@@ -149,8 +149,14 @@ typedef struct csla_compress_params {
  * and stored as bf16.  Finally len += T.
  *   kv_new   [B][T][D]  dtype kv_dtype (CSLA_F32 or CSLA_BF16)
  *   kidx_new [B][T][dI] dtype kv_dtype, CSA only (NULL for HCA)
- * Requires: the block table maps every page the new tokens reach.
- * Errors: CSLA_ERR_ARG on null/bad sizes; CSLA_ERR_UNSUPPORTED on shapes.
+ * Requires: the block table maps every page the new tokens reach;
+ * st->tail_kv and st->tail_idx 16-byte aligned; CSA: dI a multiple of 4,
+ * 4 <= dI <= 512.  kv_new / kidx_new need no alignment (aligned inputs take
+ * vector loads).  gamma_kv, wg, gb, wgi, gbi are read before the kernel
+ * waits on the grid launched before it on the stream (programmatic
+ * dependent launch); write them no later than the kernel before that one.
+ * Errors: CSLA_ERR_ARG on null/bad sizes or misaligned tails;
+ * CSLA_ERR_UNSUPPORTED on shapes.
  */
 int csla_compress_append(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
                          const int32_t *slots, int32_t B, int32_t T, const void *kv_new,
@@ -262,6 +268,27 @@ const char *csla_strerror(int status);
 
 /* Library version as major*10000 + minor*100 + patch. */
 int csla_version(void);
+
+/*
+ * Device timeline (libraries built with -DCSLA_TIMELINE only, e.g.
+ * `build.py --timeline OUT.so`; absent from normal builds).  Thread 0 of
+ * every CTA of every library kernel appends one record
+ *   { uint32 kernel id, uint32 linear CTA index, uint64 t_start,
+ *     uint64 t_waited (0 if the CTA exited before its grid-dependency wait),
+ *     uint64 t_exit, uint64 marks[8] (kernel-specific points, 0 if unset),
+ *     uint64 clock_start, uint64 clock_exit (SM cycle counter) }
+ *   (global-timer nanoseconds, 112 bytes)
+ * to a device buffer of 65536 records.  csla_timeline_read synchronises the
+ * device and copies up to `bytes` of records to host memory `records`,
+ * storing how many in *count; csla_timeline_clear synchronises and empties
+ * the buffer.  Kernel ids: 1 compress, 2 tail update, 3 index-query
+ * projection, 4 wide projection, 5 indexer, 6 top-k, 7 query preparation,
+ * 8 attention, 9 chunk combine.
+ */
+#ifdef CSLA_TIMELINE
+int csla_timeline_read(void *records, size_t bytes, uint32_t *count);
+int csla_timeline_clear(void);
+#endif
 
 #ifdef __cplusplus
 }

@@ -12,10 +12,23 @@ from conftest import ROOT
 HEADER = os.path.join(ROOT, "include", "csla.h")
 
 
-def declared():
+def declared(timeline=False):
+    """Entry points the header declares for a normal build (the device
+    timeline readers exist only in builds with -DCSLA_TIMELINE)."""
     txt = open(HEADER).read()
     txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    if not timeline:
+        txt = re.sub(r"#ifdef CSLA_TIMELINE.*?#endif", "", txt, flags=re.S)
     return sorted(set(re.findall(r"\b(csla_[a-z_]+)\s*\(", txt)))
+
+
+def test_timeline_readers_are_build_variant_only():
+    from compressed_sparse_long_append_b200 import csla
+    lib = ctypes.CDLL(csla.LIB_PATH)
+    extra = set(declared(timeline=True)) - set(declared())
+    assert extra == {"csla_timeline_read", "csla_timeline_clear"}
+    for n in extra:
+        assert not hasattr(lib, n), n
 
 
 def test_header_declares_the_five_calls():
@@ -60,8 +73,9 @@ def test_workspace_sizes():
     # indexer: B * NQ * dI bf16 with NQ = 3*HI rounded up to 16
     assert C.csla_workspace_size(cfg, C.CSLA_OP_INDEXER, 8, 131072) == 8 * 48 * 128 * 2
     assert C.csla_workspace_size(cfg, C.CSLA_OP_TOPK, 8, 131072) == 0
-    # attention: B * chunks * (H*D + 2H) floats; 512+128 rows -> 3 chunks
-    assert C.csla_workspace_size(cfg, C.CSLA_OP_CSA_ATTEND, 8, 512) == 8 * 3 * (64 * 512 + 128) * 4
+    # attention: B * 64 * D bf16 (query image) + B * chunks * (H*D + 2H) floats;
+    # 512+128 rows -> 10 chunks of 64
+    assert C.csla_workspace_size(cfg, C.CSLA_OP_CSA_ATTEND, 8, 512) == 8 * 64 * 512 * 2 + 8 * 10 * (64 * 512 + 128) * 4
     hca = _cfg(m=128)
-    assert C.csla_workspace_size(hca, C.CSLA_OP_HCA_ATTEND, 4, 1 << 20) == 4 * 32 * (64 * 512 + 128) * 4
+    assert C.csla_workspace_size(hca, C.CSLA_OP_HCA_ATTEND, 4, 1 << 20) == 4 * 64 * 512 * 2 + 4 * 32 * (64 * 512 + 128) * 4
     assert C.csla_workspace_size(_cfg(m=8), C.CSLA_OP_TOPK, 1, 1) == 0

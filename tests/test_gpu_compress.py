@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from csla_synth.workloads import CSA_DECODE, CSA_TINY, HCA_DECODE, layer_params, token_stream
-from gpu_helpers import assert_no_device_error, build_layer, compare_rows
+from gpu_helpers import assert_bf16_close, assert_no_device_error, build_layer, compare_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -37,9 +37,11 @@ def _check_layer(w, lb, p, lens):
             tolerated += compare_rows(h["rows"][pg, b % epp], h["scales"][pg, b % epp], y, w.D, w.d_rope)
             checked += 1
             if w.is_csa:
-                ref = oracle.index_key(ts["idx"][b * w.m:(b + 1) * w.m], p["wgi"], p["gbi"])
+                xi = ts["idx"][b * w.m:(b + 1) * w.m]
+                ref = oracle.index_key(xi, p["wgi"], p["gbi"])
                 got = h["kidx"][pg, b % epp]
-                assert np.all(np.abs(got.astype(np.int64) - ref.astype(np.int64)) <= 1), b
+                # fp32 gates and pooled sum: error well under 1e-5 of the largest input
+                assert_bf16_close(got, ref, 1e-5 * float(np.max(np.abs(xi))))
         # tail: raw rows of the open block, exact fp32 copies
         for pos in range((L // w.m) * w.m, L):
             assert np.array_equal(h["tail_kv"][s, pos % w.m], ts["kv"][pos].astype(np.float32))
