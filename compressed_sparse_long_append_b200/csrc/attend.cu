@@ -319,7 +319,7 @@ __device__ void loader_role(const AttendArgs &a, int b, const Req &rq, Span sp, 
             named_sync(kBarLoad, kLoadThreads);          // previous group fully consumed
             row_sources(a, b, rq, grp, cnt, C::kRB, ms);
             named_sync(kBarLoad, kLoadThreads);
-            if (lt == 0 && grp == lo) CSLA_TL_MARK(0);
+            if (lt == 0 && grp == lo) CSLA_TL_MARK_ANY(0);
             for (int t0 = 0; t0 < cnt; t0 += kTile, ++g) {
                 if (ms->abort) continue;
                 const int buf = g & 1;
@@ -332,7 +332,7 @@ __device__ void loader_role(const AttendArgs &a, int b, const Req &rq, Span sp, 
                     const uint8_t *p = (t0 + r < cnt) ? ms->rowptr[t0 + r] : nullptr;
                     v[u] = p ? ld_nc_v4(p + ch * 16) : make_uint4(0u, 0u, 0u, 0u);
                 }
-                if (lt == 0 && g == 0) CSLA_TL_MARK(6);
+                if (lt == 0 && g == 0) CSLA_TL_MARK_ANY(6);
                 // ... then wait until PV of the tile that last used this buffer is done
                 if (g >= 2 && !mbar_wait(&ms->x_empty[buf], ((g >> 1) - 1) & 1, &ms->abort)) continue;
                 uint8_t *xs = smem + (buf ? C::kOffX1 : C::kOffX0);
@@ -347,7 +347,7 @@ __device__ void loader_role(const AttendArgs &a, int b, const Req &rq, Span sp, 
                     ms->tvalid[buf][lt] = ok ? 1 : 0;
                 }
                 fence_proxy_async_smem();
-                if (lt == 0 && g == 0) CSLA_TL_MARK(4);
+                if (lt == 0 && g == 0) CSLA_TL_MARK_ANY(4);
                 mbar_arrive(&ms->x_full[buf]);
             }
         }
@@ -363,7 +363,7 @@ __device__ void mma_role(const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
     const uint32_t q0 = smem_u32(smem + C::kOffQ);
     const uint32_t p0n = smem_u32(smem + C::kOffPn), p0r = smem_u32(smem + C::kOffPr);
     if (!mbar_wait(&ms->q_ready, 0, &ms->abort)) return;
-    CSLA_TL_MARK(5);
+    CSLA_TL_MARK_ANY(5);
     int g = 0;
     for (int c = sp.c0; c < sp.c1; ++c) {
         const int lo = c * rq.chunk;

@@ -117,7 +117,11 @@ struct TimelineScope {
 };
 #define CSLA_TL_SCOPE(kernel) ::csla::TimelineScope csla_tl_scope_(kernel)
 #define CSLA_TL_WAITED() csla_tl_scope_.waited()
-#define CSLA_TL_MARK(i) ::csla::timeline_mark(i)
+#define CSLA_TL_MARK(i)                            \
+    do {                                           \
+        if (threadIdx.x == 0) ::csla::timeline_mark(i); \
+    } while (0)
+#define CSLA_TL_MARK_ANY(i) ::csla::timeline_mark(i)
 #else
 #define CSLA_TL_SCOPE(kernel) \
     do {                      \
@@ -127,6 +131,9 @@ struct TimelineScope {
     } while (0)
 #define CSLA_TL_MARK(i) \
     do {                \
+    } while (0)
+#define CSLA_TL_MARK_ANY(i) \
+    do {                    \
     } while (0)
 #endif
 

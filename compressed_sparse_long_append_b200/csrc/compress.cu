@@ -147,6 +147,7 @@ __device__ void pool_block(const BlockRows<T> &x, int m, const float *wsm, float
         __syncthreads();   // the previous chunk is consumed
         stage_rows(x, c0, R, xs);
         __syncthreads();
+        if (c0 == 0) CSLA_TL_MARK(3);
         for (int r = warp; r < R; r += kWarps) {
             float acc = 0.f;
             for (int c4 = lane; c4 < nq; c4 += 32) {
@@ -161,6 +162,7 @@ __device__ void pool_block(const BlockRows<T> &x, int m, const float *wsm, float
         }
     }
     __syncthreads();
+    CSLA_TL_MARK(4);
     float gmax = -INFINITY;
     for (int i = threadIdx.x; i < m; i += kThreads) gmax = fmaxf(gmax, alpha[i]);
     gmax = block_max<kWarps>(gmax, red);
@@ -173,6 +175,7 @@ __device__ void pool_block(const BlockRows<T> &x, int m, const float *wsm, float
     const float z = block_sum<kWarps>(e, red);   // ends with __syncthreads
     for (int i = threadIdx.x; i < m; i += kThreads) alpha[i] = __fdiv_rn(alpha[i], z);
     __syncthreads();
+    CSLA_TL_MARK(5);
     const int G = kThreads / nq;   // nq <= 128, so G >= 2
     const int g = threadIdx.x / nq, c4 = threadIdx.x % nq;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -196,6 +199,7 @@ __device__ void pool_block(const BlockRows<T> &x, int m, const float *wsm, float
     }
     if (g < G) reinterpret_cast<float4 *>(part)[g * nq + c4] = acc;
     __syncthreads();
+    CSLA_TL_MARK(6);
     for (int d = threadIdx.x; d < width; d += kThreads) {
         float t = part[d];
         for (int q = 1; q < G; ++q) t = __fadd_rn(t, part[q * width + d]);

@@ -213,6 +213,341 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
     CSLA_TL_MARK(6);
 }
 
+// ---------------------------------------------------------------- register variant
+// For n <= kRegMax, one CTA of 512 threads.  Warp w owns the contiguous
+// range [w*seg, (w+1)*seg), seg = ceil(n / 16); lane l holds the scores
+// w*seg + 32j + l (j < kPer) in registers, so a warp's ballots walk its
+// range in index order.
+//  1. Threshold t0 from a sample (no shared-memory pass): every warp sorts
+//     32 keys spread over its range, one per lane (bitonic, shuffles), and
+//     takes its rw-th largest; t0 is the smallest of these over the warps,
+//     so at least 16*rw of the 512 sample keys are >= t0: rw = ceil(48k/n)
+//     puts about 1.5k or more keys >= t0 in expectation.
+//  2. One sweep converts the scores to keys and compacts the keys >= t0
+//     (with their indices) into per-warp regions of shared memory, in index
+//     order.  When every region fits and there are at least k of them, the
+//     exact k-th largest key T is found among the candidates alone (every
+//     key >= T is one of them) and the output is taken from the regions.
+//  3. Otherwise (rare) T is found among all keys and the output is taken
+//     from the registers.  Either way the output holds the keys > T and the
+//     lowest-index keys == T, ascending.
+// The radix selects use 11/11/10-bit digits and one shared histogram.
+constexpr int kRThreads = 512;
+constexpr int kRWarps = kRThreads / 32;
+constexpr int kPer = 72;                          // scores per thread
+constexpr int kRegMax = kPer * kRThreads;         // 36864
+constexpr int kRegion = 512;                      // candidates per warp
+
+// The float whose key is `key` (inverse of score_key; key 0 -> padding NaN).
+__device__ __forceinline__ float key_value(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+struct RegShared {
+    int hist[kBins];
+    uint32_t ckey[kRWarps][kRegion];
+    int cidx[kRWarps][kRegion];
+    int cnt[kRWarps];
+    uint32_t tw[kRWarps];
+    int warp_a[kRWarps], warp_b[kRWarps];
+    int sel_bin, sel_krem;
+    uint32_t small[32];
+    int small_n;
+    uint32_t small_t;
+};
+
+// Exclusive prefix over the kRWarps per-warp values v[] for warp `warp`,
+// and their total.  Every thread calls it after a barrier that published v[].
+__device__ __forceinline__ int warp_prefix(const int *v, int warp, int *total) {
+    const int lane = threadIdx.x & 31;
+    const int x = lane < kRWarps ? v[lane] : 0;
+    int incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    *total = __shfl_sync(0xffffffffu, incl, 31);
+    return __shfl_sync(0xffffffffu, incl - x, warp);
+}
+
+// Radix select: the key of rank `rank` (1 = largest) among the non-zero keys
+// that each thread passes to the callback given to each(), all of which
+// share their top 32 - bits bits with `prefix`; *krem_out = how many keys
+// equal to the result are within that rank.  Digits of up to 11 bits, from
+// the top of the `bits` low bits down.
+template <typename Each>
+__device__ uint32_t radix_select(RegShared &sh, const Each &each, int rank, uint32_t prefix, int bits,
+                                 int *krem_out) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t pmask = bits >= 32 ? 0u : ~((1u << bits) - 1u);
+    prefix &= pmask;
+    int krem = rank;
+#pragma unroll 1
+    for (int left = bits; left > 0;) {
+        const int width = left > 11 ? 11 : left;
+        const int shb = left - width;
+        const int nb = 1 << width;
+        left = shb;
+        for (int i = threadIdx.x; i < kBins; i += kRThreads) sh.hist[i] = 0;
+        __syncthreads();
+        each([&](uint32_t key) {
+            if (key != 0u && (key & pmask) == prefix) atomicAdd(&sh.hist[(key >> shb) & (uint32_t)(nb - 1)], 1);
+        });
+        __syncthreads();
+        // thread t covers bins nb-1-t*per .. (highest first); per = 0 for t beyond nb
+        const int per = (nb + kRThreads - 1) / kRThreads;
+        int c = 0;
+        for (int q = 0; q < per; ++q) {
+            const int bin = nb - 1 - (threadIdx.x * per + q);
+            if (bin >= 0) c += sh.hist[bin];
+        }
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        if (lane == 31) sh.warp_a[warp] = incl;
+        __syncthreads();
+        int total;
+        const int before = warp_prefix(sh.warp_a, warp, &total);
+        const int excl = before + incl - c;
+        if (excl < krem && krem <= excl + c) {
+            int run = excl;
+            for (int q = 0; q < per; ++q) {
+                const int bin = nb - 1 - (threadIdx.x * per + q);
+                const int h = bin >= 0 ? sh.hist[bin] : 0;
+                if (run + h >= krem) {
+                    sh.sel_bin = bin;
+                    sh.sel_krem = krem - run;
+                    break;
+                }
+                run += h;
+            }
+        }
+        __syncthreads();
+        const int sel = sh.sel_bin;
+        prefix |= (uint32_t)sel << shb;
+        pmask |= (uint32_t)(nb - 1) << shb;
+        krem = sh.sel_krem;
+        if (left > 0 && sh.hist[sel] <= 32) {
+            // at most 32 keys left in the bin: gather them and let one warp
+            // sort them (bitonic, descending) instead of further passes
+            if (threadIdx.x == 0) sh.small_n = 0;
+            __syncthreads();
+            each([&](uint32_t key) {
+                if (key != 0u && (key & pmask) == prefix) sh.small[atomicAdd(&sh.small_n, 1)] = key;
+            });
+            __syncthreads();
+            if (warp == 0) {
+                uint32_t v = lane < sh.small_n ? sh.small[lane] : 0u;
+#pragma unroll
+                for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+                    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                        const uint32_t o = __shfl_xor_sync(0xffffffffu, v, stride);
+                        const bool desc = (lane & size) == 0 || size == 32;
+                        const bool lower = (lane & stride) == 0;
+                        v = (lower == desc) ? max(v, o) : min(v, o);
+                    }
+                }
+                const uint32_t t = __shfl_sync(0xffffffffu, v, krem - 1);
+                // keys == t among the first krem of the sorted bin
+                const int eqn = __popc(__ballot_sync(0xffffffffu, lane < krem && v == t));
+                if (lane == 0) {
+                    sh.small_t = t;
+                    sh.sel_krem = eqn;
+                }
+            }
+            __syncthreads();
+            *krem_out = sh.sel_krem;
+            return sh.small_t;
+        }
+    }
+    *krem_out = krem;
+    return prefix;
+}
+
+__global__ void __launch_bounds__(kRThreads, 1) topk_reg_kernel(TopkArgs a) {
+    CSLA_TL_SCOPE(kTlTopk);
+    extern __shared__ __align__(16) uint8_t dyn_raw[];
+    RegShared &sh = *reinterpret_cast<RegShared *>(dyn_raw);
+    pdl_trigger();
+    const int b = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int slot = __ldg(a.slots + b);
+    const bool slot_ok = slot >= 0 && slot < a.n_slots;
+    pdl_wait();
+    CSLA_TL_WAITED();
+    const int L = slot_ok ? a.len[slot] : 0;
+    int n = L / a.m;
+    if (!slot_ok || L > a.max_n * a.m) {
+        if (threadIdx.x == 0) set_dev_err(CSLA_DEVERR_LEN);
+        n = 0;
+    }
+    const int k = a.k;
+    int32_t *out = a.idx + (size_t)b * k;
+    if (n <= k) {
+        for (int j = threadIdx.x; j < k; j += kRThreads) out[j] = j < n ? j : -1;
+        return;
+    }
+    const float *sc = a.scores + (size_t)b * a.stride;
+    const int seg = (n + kRWarps - 1) / kRWarps;
+    const int base = warp * seg;
+    float f[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int r = 32 * j + lane, i = base + r;
+        f[j] = (r < seg && i < n) ? sc[i] : __int_as_float(-1);   // the NaN whose key is 0: padding
+    }
+    CSLA_TL_MARK(0);
+
+    // ---- 1. threshold: per-warp sorted sample, smallest rw-th largest over warps
+    // lane l samples row js = l * rows / 32 of the warp's range (rows = ceil(seg / 32))
+    const int js = (lane * ((seg + 31) >> 5)) >> 5;
+    uint32_t smp = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j)
+        if (j == js) smp = score_key(f[j]);
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const uint32_t o = __shfl_xor_sync(0xffffffffu, smp, stride);
+            const bool desc = (lane & size) == 0 || size == 32;
+            const bool lower = (lane & stride) == 0;
+            smp = (lower == desc) ? max(smp, o) : min(smp, o);
+        }
+    }
+    // each warp keeps >= rw samples >= t0, so in expectation >= rw * n / 32 keys are >= t0
+    const int rw = min(32, (int)((48LL * k + n - 1) / n));
+    const uint32_t s_w = __shfl_sync(0xffffffffu, smp, rw - 1);
+    if (lane == 0) sh.tw[warp] = s_w;
+    __syncthreads();
+    uint32_t t0 = lane < kRWarps ? sh.tw[lane] : 0xFFFFFFFFu;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t0 = min(t0, __shfl_xor_sync(0xffffffffu, t0, o));
+    CSLA_TL_MARK(1);
+
+    // ---- 2. candidates: scores >= the value of t0 (padding, a NaN, never
+    // qualifies; t0 = 0 admits every real score) into this warp's region
+    const float f0 = t0 == 0u ? -INFINITY : key_value(t0);
+    int pos = 0;
+    uint32_t cmax = 0;
+    const unsigned below = (1u << lane) - 1u;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const bool q = f[j] >= f0;
+        const unsigned mq = __ballot_sync(0xffffffffu, q);
+        const int at = pos + __popc(mq & below);
+        if (q && at < kRegion) {
+            const uint32_t key = score_key(f[j]);
+            sh.ckey[warp][at] = key;
+            sh.cidx[warp][at] = base + 32 * j + lane;
+            cmax = max(cmax, key);
+        }
+        pos += __popc(mq);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+    if (lane == 0) {
+        sh.cnt[warp] = pos;
+        sh.tw[warp] = cmax;
+    }
+    __syncthreads();
+    int n_ge;
+    warp_prefix(sh.cnt, warp, &n_ge);
+    bool fits = true;
+#pragma unroll
+    for (int w = 0; w < kRWarps; ++w) fits &= sh.cnt[w] <= kRegion;
+    CSLA_TL_MARK(2);
+
+    int krem;
+    if (fits && n_ge >= k) {
+        const int my_n = sh.cnt[warp];
+        // every candidate lies in [t0, kmax]: they share the top clz(t0 ^ kmax) bits
+        uint32_t kmax = lane < kRWarps ? sh.tw[lane] : 0u;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+        const int bits = 32 - __clz(t0 ^ kmax);
+        const uint32_t T = radix_select(sh, [&](auto fn) {
+            for (int i = lane; i < my_n; i += 32) fn(sh.ckey[warp][i]);
+        }, k, kmax, bits, &krem);
+        CSLA_TL_MARK(3);
+        // ---- 3. output from the regions (index order within and across warps)
+        int gt = 0, eq = 0;
+        for (int i = lane; i < my_n; i += 32) {
+            const uint32_t key = sh.ckey[warp][i];
+            gt += key > T;
+            eq += key == T;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            gt += __shfl_xor_sync(0xffffffffu, gt, o);
+            eq += __shfl_xor_sync(0xffffffffu, eq, o);
+        }
+        if (lane == 0) {
+            sh.warp_a[warp] = gt;
+            sh.warp_b[warp] = eq;
+        }
+        __syncthreads();
+        int tot;
+        const int gt_before = warp_prefix(sh.warp_a, warp, &tot);
+        const int eq_before = warp_prefix(sh.warp_b, warp, &tot);
+        int opos = gt_before + min(eq_before, krem);
+        int eq_seen = eq_before;
+        for (int i0 = 0; i0 < my_n; i0 += 32) {
+            const int i = i0 + lane;
+            const uint32_t key = i < my_n ? sh.ckey[warp][i] : 0u;
+            const bool is_gt = i < my_n && key > T;
+            const bool is_eq = i < my_n && key == T;
+            const unsigned meq = __ballot_sync(0xffffffffu, is_eq);
+            const bool take_eq = is_eq && (eq_seen + __popc(meq & below)) < krem;
+            const unsigned mtake = __ballot_sync(0xffffffffu, is_gt || take_eq);
+            if (is_gt || take_eq) out[opos + __popc(mtake & below)] = sh.cidx[warp][i];
+            opos += __popc(mtake);
+            eq_seen += __popc(meq);
+        }
+    } else {
+        const uint32_t T = radix_select(sh, [&](auto fn) {
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) fn(score_key(f[j]));
+        }, k, 0u, 32, &krem);
+        CSLA_TL_MARK(3);
+        int gt = 0, eq = 0;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const uint32_t key = score_key(f[j]);
+            gt += __popc(__ballot_sync(0xffffffffu, key > T));
+            eq += __popc(__ballot_sync(0xffffffffu, key == T));
+        }
+        if (lane == 0) {
+            sh.warp_a[warp] = gt;
+            sh.warp_b[warp] = eq;
+        }
+        __syncthreads();
+        int tot;
+        const int gt_before = warp_prefix(sh.warp_a, warp, &tot);
+        const int eq_before = warp_prefix(sh.warp_b, warp, &tot);
+        int opos = gt_before + min(eq_before, krem);
+        int eq_seen = eq_before;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const uint32_t key = score_key(f[j]);
+            const bool is_gt = key > T;
+            const bool is_eq = key == T;
+            const unsigned meq = __ballot_sync(0xffffffffu, is_eq);
+            const bool take_eq = is_eq && (eq_seen + __popc(meq & below)) < krem;
+            const unsigned mtake = __ballot_sync(0xffffffffu, is_gt || take_eq);
+            if (is_gt || take_eq) out[opos + __popc(mtake & below)] = base + 32 * j + lane;
+            opos += __popc(mtake);
+            eq_seen += __popc(meq);
+        }
+    }
+    CSLA_TL_MARK(4);
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
@@ -225,8 +560,12 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kHistBytes);
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(topk_reg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RegShared));
+        if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
+    if (a.max_n <= kRegMax)
+        return launch_pdl(topk_reg_kernel, dim3(a.B), dim3(kRThreads), sizeof(RegShared), stream, a);
     if (a.max_n <= kSmemKeysMax) {
         const size_t smem = kHistBytes + (size_t)(a.max_n > 0 ? a.max_n : 1) * sizeof(uint32_t);
         return launch_pdl(topk_kernel<true>, dim3(a.B), dim3(kThreads), smem, stream, a);
