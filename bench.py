@@ -228,12 +228,12 @@ class CsaStep:
 
 def csa_launches(kw, variant):
     """Kernels of one CSA step: compress (pool + tail/len), iq_project +
-    indexer, topk, prep_q + attend, + combine unless the saturated variant
-    runs (forced, or automatic: one chunk per request or B >= SM count)."""
+    indexer, topk, attend, + combine unless the saturated variant runs
+    (forced, or automatic: one chunk per request or B >= SM count)."""
     rows = kw["k"] + kw["n_win"]
     chunks = -(-rows // (64 * -(-rows // 2048)))
     saturated = variant == 1 or (variant == 0 and (kw["B"] >= 148 or chunks <= 1))
-    return 2 + 2 + 1 + 2 + (0 if saturated else 1)
+    return 2 + 2 + 1 + 1 + (0 if saturated else 1)
 
 
 class HcaStep:

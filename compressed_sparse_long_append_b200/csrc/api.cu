@@ -79,12 +79,10 @@ int nq_of(int HI) { return (3 * HI + 15) / 16 * 16; }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? CSLA_OK : CSLA_ERR_CUDA; }
 
-// Attention workspace: per request the 64-head Qhat image (64*D bf16), then
-// the chunk partials (H*D + 2H floats per chunk).
-size_t attend_q_bytes(const csla_cfg *c, int B) { return (size_t)B * 64 * c->D * 2; }
+// Attention workspace: the chunk partials (H*D + 2H floats per chunk).
 size_t attend_ws(const csla_cfg *c, int B, long long max_rows) {
     const size_t per = ((size_t)c->H * c->D + 2 * (size_t)c->H) * sizeof(float);
-    return attend_q_bytes(c, B) + (size_t)B * attend_max_chunks(max_rows) * per;
+    return (size_t)B * attend_max_chunks(max_rows) * per;
 }
 
 }  // namespace
@@ -257,8 +255,7 @@ static int attend_common(const csla_cfg *cfg, const csla_state *st, const csla_c
     a.rows = cache->rows; a.scales = cache->scales; a.block_table = cache->block_table;
     a.bt_stride = cache->bt_stride; a.n_pages = cache->n_pages; a.n_slots = st->n_slots;
     a.win_rows = st->win_rows; a.win_scales = st->win_scales; a.out = out;
-    a.qimg = reinterpret_cast<uint8_t *>(workspace);
-    a.part = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + attend_q_bytes(cfg, B));
+    a.part = reinterpret_cast<float *>(workspace);
     const long long max_rows = idx ? (long long)k + cfg->n_win : (long long)max_len / cfg->m + cfg->n_win;
     a.max_chunks = attend_max_chunks(max_rows);
     a.max_len = max_len;

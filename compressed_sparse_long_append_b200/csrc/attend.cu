@@ -19,17 +19,21 @@
 // and nothing depends on which other requests share the launch.
 //
 // One CTA = three roles over a stream of 64-row tiles:
-//   warps 4-7 (loader)  compute row addresses for a chunk, gather the raw
-//                       cache rows of tile t+1 into registers while tile t is
-//                       in flight, widen fp8 codes to bf16 (exact) into the
-//                       SW128 K-major X tile (double-buffered);
+//   warps 4-7 (loader)  resolve the 64 row addresses of a tile (one thread
+//                       per row) and fetch the raw cache rows with 1-D bulk
+//                       copies into one of two staging buffers (tiles t+1 and
+//                       t+2 are in flight while tile t is converted); widen
+//                       fp8 codes to bf16 (exact) into the SW128 K-major X
+//                       tile once the previous tile's PV product is done;
 //   warp 8 (MMA)        S = Qhat . X^T   tcgen05 M=64 (heads) N=64 (rows),
 //                                        nope and RoPE dims in separate TMEM
 //                                        accumulators: s = scale*S_nope + S_rope
 //                       O^T += X^T . P^T tcgen05 M=128 (dims) N=64 (heads);
-//   warps 0-3 (softmax) bulk-copy the request's Qhat image (prep_q_kernel:
-//                       RoPE(RMSNorm(q)*gamma_q, t)) into smem; per tile read S, P = 2^(s - m) (lanes 0-15 of each warp own one
-//                       head), P_nope = bf16(P*scale), P_rope = bf16(P); lazy
+//   warps 0-3 (softmax) build Qhat = RoPE(RMSNorm(q)*gamma_q, t) in smem
+//                       (the norm before the grid-dependency wait, the
+//                       rotation after it); per tile read S, P = 2^(s - m)
+//                       (lanes 0-15 of each warp own one head),
+//                       P_nope = bf16(P*scale), P_rope = bf16(P); lazy
 //                       rescale of O^T when a head's max grows by more than 8
 //                       (log2 units); at chunk end read O^T out as the partial.
 // mbarriers hand tiles between roles; every wait is bounded.
@@ -45,7 +49,6 @@ constexpr int kLoadThreads = 32 * kLoadWarps;
 constexpr int kMmaWarp = kSoftWarps + kLoadWarps;               // warp 8
 constexpr int kHP = 64;          // heads padded to the UMMA M of the S product
 constexpr int kTile = 64;        // rows per tile
-constexpr int kRowInfo = 512;    // row addresses held at once by the loader
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThresh = 8.0f;
 constexpr int kBarLoad = 1;   // named barrier of the loader warps (0 = __syncthreads)
@@ -63,29 +66,32 @@ struct Cfg {
     static constexpr int kQKB = kHP * 128;             // one K block of Qhat
     static constexpr int kQBytes = kKB * kQKB;
     static constexpr int kPBytes = kHP * kTile * 2;
-    static constexpr int kTasks = kTile * kCH;         // 16-byte loads per tile
-    static constexpr int kTPT = kTasks / kLoadThreads; // loads per loader thread
+    static constexpr int kTasks = kTile * kCH;         // 16-byte chunks per tile
+    static constexpr int kTPT = kTasks / kLoadThreads; // chunks widened per loader thread
     static_assert(kTasks % kLoadThreads == 0, "tile split");
+    static constexpr int kRawBytes = kTile * kRB;      // one staged tile of raw rows
     // TMEM columns
     static constexpr int kColSN = 0, kColSR = 64, kColO = 128;
     static constexpr int kColOR = 128 + 64 * kMB;
     static constexpr int kTmemCols = (kColOR + 64) <= 256 ? 256 : 512;
     // smem offsets (from a 1024-aligned base)
     static constexpr int kOffQ = 0;
-    static constexpr int kOffX0 = kOffQ + kQBytes;
-    static constexpr int kOffX1 = kOffX0 + kXBytes;
-    static constexpr int kOffPn = kOffX1 + kXBytes;
+    static constexpr int kOffX = kOffQ + kQBytes;
+    static constexpr int kOffRaw0 = kOffX + kXBytes;
+    static constexpr int kOffRaw1 = kOffRaw0 + kRawBytes;
+    static constexpr int kOffPn = kOffRaw1 + kRawBytes;
     static constexpr int kOffPr = kOffPn + kPBytes;
     static constexpr int kOffMisc = kOffPr + kPBytes;
 };
 
 struct Misc {
-    const uint8_t *rowptr[kRowInfo];   // loader-private: sources of the current row group
-    float rowscale[kRowInfo];
-    float tscale[2][kTile];            // per X buffer: fp8 scale of each row (0 = masked)
+    float rawscale[2][kTile];          // loader-private, per staging buffer: fp8 scale of each row
+    int rawvalid[2][kTile];
+    float tscale[2][kTile];            // per tile parity: fp8 scale of each row (0 = masked)
     int tvalid[2][kTile];
     float fac[2][kHP];                 // per tile parity: O^T column factors (1 = none)
-    uint64_t x_full[2], x_empty[2], s_full, s_free, p_full, pv_done, o_free, q_ready, fac_ready;
+    uint64_t raw_full[2], x_full[2], x_empty[2], s_full, s_free, p_full, pv_done, o_free, q_ready, fac_ready;
+    int go[2];                         // loader: keep fetching (per tile parity)
     uint32_t tmem;
     int abort;
 };
@@ -139,135 +145,155 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // ---------------------------------------------------------------- query preparation
-// qhat = RoPE(RMSNorm(q_h) * gamma_q, t) for the 64 (padded) heads of request
-// b, written as the bf16 SW128 K-major shared-memory image the attention
-// kernel copies in with bulk copies.  grid (B, 8), one warp per head.
+// Qhat = RoPE(RMSNorm(q_h) * gamma_q, t) for the 64 (padded) heads of the
+// request, built in shared memory by the softmax warps in two steps.
+// Before the grid-dependency wait (q and gamma_q are inputs of the call):
+// warp w normalises heads 16w .. 16w+15, lane l owning dims l*D/32 ..; the
+// non-RoPE dims go to the SW128 K-major Qhat image as bf16, the RoPE dims
+// stay fp32 in the P area (64 heads x 64 dims x 4 B, unused until the first
+// tile's softmax).  After the wait, when the position t = len - 1 is known,
+// lane i rotates pair i of its warp's 16 heads and writes them as bf16.
 template <int D>
-__global__ void __launch_bounds__(256) prep_q_kernel(AttendArgs a, int q_bf16) {
-    CSLA_TL_SCOPE(kTlPrepQ);
+__device__ void build_q_normed(const AttendArgs &a, int b, uint8_t *smem, int q_bf16) {
     using C = Cfg<D>;
-    __shared__ float cs[32][2];
-    pdl_trigger();
-    const int b = blockIdx.x;
+    constexpr int DPL = D / 32;              // dims per lane (16 or 4)
+    constexpr int kBatch = 4;                // heads whose loads are in flight together
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.y * 8 + warp;
-    const int slot = __ldg(a.slots + b);
-    const bool slot_ok = slot >= 0 && slot < a.n_slots;
-    constexpr int NG = D / 8;                   // 8-dim groups per head
-    constexpr int GPL = (NG + 31) / 32;         // groups per lane
-    // ---- before the wait: RMSNorm(q) * gamma_q in registers (q and gamma
-    // are inputs of the call)
-    float y[GPL][8];
-    float ss = 0.f;
+    float *ropef = reinterpret_cast<float *>(smem + C::kOffPn);   // [64 heads][64 dims]
+    const int d0 = lane * DPL;
+    float gam[DPL];
 #pragma unroll
-    for (int i = 0; i < GPL; ++i) {
-        const int g = lane + 32 * i;
+    for (int e = 0; e < DPL; ++e) gam[e] = __ldg(a.gamma_q + d0 + e);
+    for (int h0 = 16 * warp; h0 < 16 * warp + 16; h0 += kBatch) {
+        float x[kBatch][DPL];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) y[i][e] = 0.f;
-        if (g < NG && h < a.H) {
-            const size_t off = ((size_t)b * a.H + h) * D + (size_t)g * 8;
-            if (q_bf16) {
-                const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
-                    reinterpret_cast<const __nv_bfloat16 *>(a.q) + off));
-                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        for (int u = 0; u < kBatch; ++u) {
+            const int h = h0 + u;
+            const size_t off = ((size_t)b * a.H + h) * D + d0;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    y[i][2 * e] = bf16_bits_to_f32(w[e] & 0xFFFFu);
-                    y[i][2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
-                }
-            } else {
-                const float4 *p = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(a.q) + off);
-                const float4 u0 = __ldg(p), u1 = __ldg(p + 1);
-                y[i][0] = u0.x; y[i][1] = u0.y; y[i][2] = u0.z; y[i][3] = u0.w;
-                y[i][4] = u1.x; y[i][5] = u1.y; y[i][6] = u1.z; y[i][7] = u1.w;
-            }
-        }
+            for (int e0 = 0; e0 < DPL; e0 += 8 > DPL ? DPL : 8) {
+                if (h >= a.H) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ss = __fmaf_rn(y[i][e], y[i][e], ss);
-    }
-    ss = warp_sum(ss);
-    const float r = 1.0f / sqrtf(__fdiv_rn(ss, (float)D) + a.eps);
+                    for (int e = 0; e < (8 > DPL ? DPL : 8); ++e) x[u][e0 + e] = 0.f;
+                } else if (q_bf16) {
+                    if constexpr (DPL >= 8) {
+                        const uint4 w4 = __ldg(reinterpret_cast<const uint4 *>(
+                            reinterpret_cast<const __nv_bfloat16 *>(a.q) + off + e0));
+                        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-    for (int i = 0; i < GPL; ++i) {
-        const int g = lane + 32 * i;
-        if (g >= NG) continue;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[i][e] = __fmul_rn(__fmul_rn(y[i][e], r), __ldg(a.gamma_q + g * 8 + e));
-    }
-    pdl_wait();
-    CSLA_TL_WAITED();
-
-    // ---- the query position is len - 1
-    const int L = slot_ok ? a.len[slot] : 0;
-    if (!slot_ok || L < 1 || L > a.max_len) return;   // the attention kernel reports it
-    if (threadIdx.x < 32) {
-        float c, sn;
-        rope_cos_sin((long long)L - 1, a.freq.inv[threadIdx.x], &c, &sn);
-        cs[threadIdx.x][0] = c;
-        cs[threadIdx.x][1] = sn;
-    }
-    __syncthreads();
-    uint8_t *img = a.qimg + (size_t)b * C::kQBytes;
-#pragma unroll
-    for (int i = 0; i < GPL; ++i) {
-        const int g = lane + 32 * i;
-        if (g >= NG) continue;
-        if (g * 8 >= D - 64) {
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-                const int pi = (g * 8 + e - (D - 64)) >> 1;
-                const float c = cs[pi][0], sn = cs[pi][1];
-                const float y0 = y[i][e], y1 = y[i][e + 1];
-                y[i][e] = __fsub_rn(__fmul_rn(y0, c), __fmul_rn(y1, sn));
-                y[i][e + 1] = __fadd_rn(__fmul_rn(y0, sn), __fmul_rn(y1, c));
-            }
-        }
-        uint4 o;
-        o.x = pack_bf16x2(y[i][0], y[i][1]);
-        o.y = pack_bf16x2(y[i][2], y[i][3]);
-        o.z = pack_bf16x2(y[i][4], y[i][5]);
-        o.w = pack_bf16x2(y[i][6], y[i][7]);
-        *reinterpret_cast<uint4 *>(img + sw128_off(h, g, C::kQKB)) = o;
-    }
-}
-
-// ---------------------------------------------------------------- loader role helpers
-// Sources of rows [r0, r0 + cnt) of the request's set (cnt <= kRowInfo):
-// ms->rowptr / rowscale, null pointer = masked row.  Loader threads only.
-__device__ void row_sources(const AttendArgs &a, int b, const Req &rq, int r0, int cnt, int rb, Misc *ms) {
-    const int lt = threadIdx.x - 32 * kSoftWarps;
-    for (int i = lt; i < cnt; i += kLoadThreads) {
-        const int r = r0 + i;
-        const uint8_t *p = nullptr;
-        float sc = 0.f;
-        if (r < rq.n_cmp) {
-            const int e = a.idx ? __ldg(a.idx + (size_t)b * a.k + r) : r;
-            if (e >= 0) {
-                if (e >= rq.nv) {
-                    set_dev_err(CSLA_DEVERR_INDEX);
-                } else {
-                    const int epp = CSLA_PAGE_TOKENS / a.m;
-                    const int col = e / epp;
-                    const int pg = col < a.bt_stride ? __ldg(a.block_table + (size_t)rq.slot * a.bt_stride + col) : -1;
-                    if (pg < 0 || pg >= a.n_pages) {
-                        set_dev_err(CSLA_DEVERR_PAGE);
+                        for (int e = 0; e < 4; ++e) {
+                            x[u][e0 + 2 * e] = bf16_bits_to_f32(w[e] & 0xFFFFu);
+                            x[u][e0 + 2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
+                        }
                     } else {
-                        const size_t ent = (size_t)pg * epp + (size_t)(e % epp);
-                        p = a.rows + ent * rb;
-                        sc = __ldg(a.scales + ent);
+                        const uint2 w2 = __ldg(reinterpret_cast<const uint2 *>(
+                            reinterpret_cast<const __nv_bfloat16 *>(a.q) + off + e0));
+                        x[u][e0] = bf16_bits_to_f32(w2.x & 0xFFFFu);
+                        x[u][e0 + 1] = bf16_bits_to_f32(w2.x >> 16);
+                        x[u][e0 + 2] = bf16_bits_to_f32(w2.y & 0xFFFFu);
+                        x[u][e0 + 3] = bf16_bits_to_f32(w2.y >> 16);
+                    }
+                } else {
+                    const float4 *p4 = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(a.q) + off + e0);
+#pragma unroll
+                    for (int e = 0; e < (8 > DPL ? DPL : 8); e += 4) {
+                        const float4 f4 = __ldg(p4 + e / 4);
+                        x[u][e0 + e] = f4.x;
+                        x[u][e0 + e + 1] = f4.y;
+                        x[u][e0 + e + 2] = f4.z;
+                        x[u][e0 + e + 3] = f4.w;
                     }
                 }
             }
-        } else if (r < rq.n_rows) {
-            const int w = r - rq.n_cmp;
-            const int pos = rq.L - rq.win_len + w;
-            const size_t ring = (size_t)rq.slot * a.n_win + (size_t)(pos % a.n_win);
-            p = a.win_rows + ring * rb;
-            sc = __ldg(a.win_scales + ring);
         }
-        ms->rowptr[i] = p;
-        ms->rowscale[i] = sc;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int h = h0 + u;
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) ss = __fmaf_rn(x[u][e], x[u][e], ss);
+            ss = warp_sum(ss);
+            const float r = 1.0f / sqrtf(__fdiv_rn(ss, (float)D) + a.eps);
+            float y[DPL];   // padding heads (h >= H) are zero
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) y[e] = h < a.H ? __fmul_rn(__fmul_rn(x[u][e], r), gam[e]) : 0.f;
+            if (d0 >= D - 64) {
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) ropef[h * 64 + (d0 - (D - 64)) + e] = y[e];
+            } else {
+#pragma unroll
+                for (int e0 = 0; e0 < DPL; e0 += 8 > DPL ? DPL : 8) {
+                    const int d = d0 + e0;
+                    if constexpr (DPL >= 8) {
+                        uint4 o;
+                        o.x = pack_bf16x2(y[e0], y[e0 + 1]);
+                        o.y = pack_bf16x2(y[e0 + 2], y[e0 + 3]);
+                        o.z = pack_bf16x2(y[e0 + 4], y[e0 + 5]);
+                        o.w = pack_bf16x2(y[e0 + 6], y[e0 + 7]);
+                        *reinterpret_cast<uint4 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB)) = o;
+                    } else {
+                        uint2 o;
+                        o.x = pack_bf16x2(y[e0], y[e0 + 1]);
+                        o.y = pack_bf16x2(y[e0 + 2], y[e0 + 3]);
+                        *reinterpret_cast<uint2 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB) + (d & 7) * 2) = o;
+                    }
+                }
+            }
+        }
     }
+}
+
+// After the wait: rotate the RoPE dims by position t and publish Qhat.
+template <int D>
+__device__ void build_q_rope(const AttendArgs &a, long long t, uint8_t *smem, Misc *ms) {
+    using C = Cfg<D>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float *ropef = reinterpret_cast<const float *>(smem + C::kOffPn);
+    float c, sn;
+    rope_cos_sin(t, a.freq.inv[lane], &c, &sn);
+    const int dim = (D - 64) + 2 * lane;
+    for (int h = 16 * warp; h < 16 * warp + 16; ++h) {
+        const float y0 = ropef[h * 64 + 2 * lane], y1 = ropef[h * 64 + 2 * lane + 1];
+        const float r0 = __fsub_rn(__fmul_rn(y0, c), __fmul_rn(y1, sn));
+        const float r1 = __fadd_rn(__fmul_rn(y0, sn), __fmul_rn(y1, c));
+        *reinterpret_cast<uint32_t *>(smem + C::kOffQ + sw128_off(h, dim >> 3, C::kQKB) + (dim & 7) * 2) =
+            pack_bf16x2(r0, r1);
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(&ms->q_ready);
+}
+
+// ---------------------------------------------------------------- loader role helpers
+// Source row (nullptr = masked) and fp8 scale of row r of the request's set.
+__device__ __forceinline__ const uint8_t *row_source(const AttendArgs &a, int b, const Req &rq, int r, int rb,
+                                                     float *scale) {
+    *scale = 0.f;
+    if (r < rq.n_cmp) {
+        const int e = a.idx ? __ldg(a.idx + (size_t)b * a.k + r) : r;
+        if (e < 0) return nullptr;
+        if (e >= rq.nv) {
+            set_dev_err(CSLA_DEVERR_INDEX);
+            return nullptr;
+        }
+        const int epp = CSLA_PAGE_TOKENS / a.m;
+        const int col = e / epp;
+        const int pg = col < a.bt_stride ? __ldg(a.block_table + (size_t)rq.slot * a.bt_stride + col) : -1;
+        if (pg < 0 || pg >= a.n_pages) {
+            set_dev_err(CSLA_DEVERR_PAGE);
+            return nullptr;
+        }
+        const size_t ent = (size_t)pg * epp + (size_t)(e % epp);
+        *scale = __ldg(a.scales + ent);
+        return a.rows + ent * rb;
+    }
+    if (r < rq.n_rows) {
+        const int w = r - rq.n_cmp;
+        const int pos = rq.L - rq.win_len + w;
+        const size_t ring = (size_t)rq.slot * a.n_win + (size_t)(pos % a.n_win);
+        *scale = __ldg(a.win_scales + ring);
+        return a.win_rows + ring * rb;
+    }
+    return nullptr;
 }
 
 // Widen one 16-byte chunk of a cache row into the bf16 X tile.
@@ -308,50 +334,68 @@ template <int D>
 __device__ void loader_role(const AttendArgs &a, int b, const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
     using C = Cfg<D>;
     const int lt = threadIdx.x - 32 * kSoftWarps;
-    int g = 0;   // tile counter across the CTA's chunks
-    // Loop bounds are uniform over the loader warps and nothing below leaves
-    // a loop early, so every loader thread reaches every named barrier.
-    for (int c = sp.c0; c < sp.c1; ++c) {
-        const int lo = c * rq.chunk;
-        const int hi = min(rq.n_rows, lo + rq.chunk);
-        for (int grp = lo; grp < hi; grp += kRowInfo) {
-            const int cnt = min(kRowInfo, hi - grp);
-            named_sync(kBarLoad, kLoadThreads);          // previous group fully consumed
-            row_sources(a, b, rq, grp, cnt, C::kRB, ms);
-            named_sync(kBarLoad, kLoadThreads);
-            if (lt == 0 && grp == lo) CSLA_TL_MARK_ANY(0);
-            for (int t0 = 0; t0 < cnt; t0 += kTile, ++g) {
-                if (ms->abort) continue;
-                const int buf = g & 1;
-                // gather the tile's raw rows into registers first ...
-                uint4 v[C::kTPT];
-#pragma unroll
-                for (int u = 0; u < C::kTPT; ++u) {
-                    const int id = u * kLoadThreads + lt;
-                    const int r = id / C::kCH, ch = id % C::kCH;
-                    const uint8_t *p = (t0 + r < cnt) ? ms->rowptr[t0 + r] : nullptr;
-                    v[u] = p ? ld_nc_v4(p + ch * 16) : make_uint4(0u, 0u, 0u, 0u);
-                }
-                if (lt == 0 && g == 0) CSLA_TL_MARK_ANY(6);
-                // ... then wait until PV of the tile that last used this buffer is done
-                if (g >= 2 && !mbar_wait(&ms->x_empty[buf], ((g >> 1) - 1) & 1, &ms->abort)) continue;
-                uint8_t *xs = smem + (buf ? C::kOffX1 : C::kOffX0);
-#pragma unroll
-                for (int u = 0; u < C::kTPT; ++u) {
-                    const int id = u * kLoadThreads + lt;
-                    store_chunk<D>(xs, id / C::kCH, id % C::kCH, v[u]);
-                }
-                if (lt < kTile) {
-                    const bool ok = (t0 + lt < cnt) && ms->rowptr[t0 + lt] != nullptr;
-                    ms->tscale[buf][lt] = ok ? ms->rowscale[t0 + lt] : 0.f;
-                    ms->tvalid[buf][lt] = ok ? 1 : 0;
-                }
-                fence_proxy_async_smem();
-                if (lt == 0 && g == 0) CSLA_TL_MARK_ANY(4);
-                mbar_arrive(&ms->x_full[buf]);
+    // the span's rows, in 64-row tiles (chunk boundaries are tile boundaries)
+    const int r_begin = sp.c0 * rq.chunk;
+    const int r_end = min(rq.n_rows, sp.c1 * rq.chunk);
+    const int n_tiles = (r_end - r_begin + kTile - 1) / kTile;
+    // Bulk-copy tile t's rows into staging buffer t & 1.  Every thread that
+    // issues a copy first adds its bytes to the buffer's transaction count;
+    // one arrival after the loader barrier closes the phase's bookkeeping.
+    // Called uniformly by all loader threads (each reaches the barrier).
+    auto issue = [&](int t) {
+        const int buf = t & 1;
+        if (lt < kTile) {
+            float sc;
+            const int r = r_begin + t * kTile + lt;
+            const uint8_t *p = r < r_end ? row_source(a, b, rq, r, C::kRB, &sc) : nullptr;
+            if (p) {
+                mbar_expect_tx(&ms->raw_full[buf], (uint32_t)C::kRB);
+                bulk_load(smem + (buf ? C::kOffRaw1 : C::kOffRaw0) + lt * C::kRB, p, (uint32_t)C::kRB,
+                          &ms->raw_full[buf]);
             }
+            ms->rawscale[buf][lt] = p ? sc : 0.f;   // the scale load completes while the copy runs
+            ms->rawvalid[buf][lt] = p ? 1 : 0;
         }
+        named_sync(kBarLoad, kLoadThreads);
+        if (lt == 0) mbar_arrive(&ms->raw_full[buf]);
+    };
+    int issued = 0, first_fail = n_tiles;
+    if (n_tiles > 0) issue(issued++);
+    if (n_tiles > 1) issue(issued++);
+    CSLA_TL_MARK_ANY(6);
+    for (int t = 0; t < n_tiles; ++t) {
+        const int buf = t & 1;
+        // the staged rows, and the X tile free again (PV of the previous tile done)
+        bool ok = t < issued && mbar_wait(&ms->raw_full[buf], (t >> 1) & 1, &ms->abort);
+        if (!ok && t < first_fail) first_fail = t;
+        if (ok && t > 0) ok = mbar_wait(&ms->x_empty[(t - 1) & 1], ((t - 1) >> 1) & 1, &ms->abort);
+        if (ok) {
+            const uint8_t *raw = smem + (buf ? C::kOffRaw1 : C::kOffRaw0);
+            uint8_t *xs = smem + C::kOffX;
+#pragma unroll 6
+            for (int u = 0; u < C::kTPT; ++u) {
+                const int id = u * kLoadThreads + lt;
+                const int r = id / C::kCH, ch = id % C::kCH;
+                const uint4 v = ms->rawvalid[buf][r] ? *reinterpret_cast<const uint4 *>(raw + r * C::kRB + ch * 16)
+                                                     : make_uint4(0u, 0u, 0u, 0u);
+                store_chunk<D>(xs, r, ch, v);
+            }
+            if (lt < kTile) {
+                ms->tscale[buf][lt] = ms->rawscale[buf][lt];
+                ms->tvalid[buf][lt] = ms->rawvalid[buf][lt];
+            }
+            fence_proxy_async_smem();
+            if (lt == 0 && t == 0) CSLA_TL_MARK_ANY(4);
+        }
+        mbar_arrive(&ms->x_full[buf]);
+        // staging buffer `buf` is consumed: fetch tile t + 2 into it, unless
+        // the CTA is aborting (one decision for all loader threads)
+        if (lt == 0) ms->go[t & 1] = ms->abort ? 0 : 1;
+        named_sync(kBarLoad, kLoadThreads);
+        if (t + 2 < n_tiles && ms->go[t & 1]) issue(issued++);
     }
+    // copies still in flight after an abort must land before the CTA exits
+    for (int t = first_fail; t < issued; ++t) mbar_wait(&ms->raw_full[t & 1], (t >> 1) & 1, nullptr);
 }
 
 template <int D>
@@ -373,7 +417,7 @@ __device__ void mma_role(const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
             if (!mbar_wait(&ms->x_full[buf], (g >> 1) & 1, &ms->abort)) return;
             if (g > 0 && !mbar_wait(&ms->s_free, (g - 1) & 1, &ms->abort)) return;
             tc_fence_after();
-            const uint32_t x0 = smem_u32(smem + (buf ? C::kOffX1 : C::kOffX0));
+            const uint32_t x0 = smem_u32(smem + C::kOffX);
 #pragma unroll
             for (int kb = 0; kb < C::kKBN; ++kb)
 #pragma unroll
@@ -418,13 +462,7 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
     uint8_t *pn = smem + C::kOffPn;
     uint8_t *pr = smem + C::kOffPr;
 
-    if (threadIdx.x == 0) {
-        // the request's Qhat image, written by prep_q_kernel
-        const uint8_t *src = a.qimg + (size_t)b * C::kQBytes;
-        mbar_arrive_expect_tx(&ms->q_ready, (uint32_t)C::kQBytes);
-        for (int off = 0; off < C::kQBytes; off += 16384)
-            bulk_load(smem + C::kOffQ + off, src + off, (uint32_t)min(16384, C::kQBytes - off), &ms->q_ready);
-    }
+    build_q_rope<D>(a, (long long)rq.L - 1, smem, ms);
 
     int g = 0;
     for (int c = sp.c0; c < sp.c1; ++c) {
@@ -604,7 +642,7 @@ __device__ __forceinline__ void store_out(const AttendArgs &a, bool out_bf16, si
 }
 
 template <int D, bool kSaturated>
-__global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int out_bf16) {
+__global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int q_bf16, int out_bf16) {
     CSLA_TL_SCOPE(kTlAttend);
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -616,6 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int o
     // ---- before the wait: barriers and TMEM
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
+            mbar_init(&ms->raw_full[i], 1);
             mbar_init(&ms->x_full[i], kLoadThreads);
             mbar_init(&ms->x_empty[i], 1);
         }
@@ -624,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int o
         mbar_init(&ms->p_full, 32 * kSoftWarps);
         mbar_init(&ms->pv_done, 1);
         mbar_init(&ms->o_free, 32 * kSoftWarps);
-        mbar_init(&ms->q_ready, 1);
+        mbar_init(&ms->q_ready, 32 * kSoftWarps);
         mbar_init(&ms->fac_ready, 32 * kSoftWarps);
         ms->abort = 0;
         fence_mbar_init();
@@ -637,6 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int o
     __syncthreads();
     tc_fence_after();
     pdl_trigger();   // after the TMEM allocation (see the indexer kernel)
+    if (warp < kSoftWarps) build_q_normed<D>(a, b, smem, q_bf16);
     pdl_wait();
     CSLA_TL_WAITED();
 
@@ -677,25 +717,45 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int o
     }
 }
 
-template <int D>
+// One CTA of 128 threads per (head, request); thread t folds dims t, t+128,
+// ... (D/128 of them).  All of a thread's partial loads are issued before
+// the chunk weights are known (warp 0 forms them meanwhile); each dim is
+// then folded in chunk order exactly like fold_dim().  kMaxC bounds the
+// chunk count (it sizes the register array).
+template <int D, int kMaxC>
 __global__ void __launch_bounds__(128) combine_kernel(AttendArgs a, int out_bf16) {
     CSLA_TL_SCOPE(kTlCombine);
+    constexpr int kDPT = D / 128;   // dims per thread
     __shared__ float wts[33];
     pdl_trigger();
+    const int h = blockIdx.x, b = blockIdx.y;
     pdl_wait();
     CSLA_TL_WAITED();
-    const int h = blockIdx.x, b = blockIdx.y;
     const Req rq = request(a, b);
     if (!rq.ok) return;
+    const int n_chunks = rq.n_chunks;
+    const size_t stride = (size_t)a.H * D + 2 * (size_t)a.H;
+    const float *p = a.part + (size_t)b * a.max_chunks * stride + (size_t)h * D + threadIdx.x;
+    float v[kDPT][kMaxC];
+#pragma unroll
+    for (int c = 0; c < kMaxC; ++c)
+#pragma unroll
+        for (int j = 0; j < kDPT; ++j) v[j][c] = c < n_chunks ? p[c * stride + 128 * j] : 0.f;
     if (threadIdx.x < 32) {
         float wl, l;
-        fold_weights(a, b, rq.n_chunks, h, D, &wl, &l);
+        fold_weights(a, b, n_chunks, h, D, &wl, &l);
         wts[threadIdx.x] = wl;
         if (threadIdx.x == 0) wts[32] = l;
     }
     __syncthreads();
-    for (int d = threadIdx.x; d < D; d += 128)
-        store_out(a, out_bf16 != 0, ((size_t)b * a.H + h) * D + d, fold_dim(a, b, rq.n_chunks, h, d, D, wts, wts[32]));
+#pragma unroll
+    for (int j = 0; j < kDPT; ++j) {
+        float o = 0.f;
+#pragma unroll
+        for (int c = 0; c < kMaxC; ++c)
+            if (c < n_chunks) o = __fmaf_rn(v[j][c], wts[c], o);
+        store_out(a, out_bf16 != 0, ((size_t)b * a.H + h) * D + threadIdx.x + 128 * j, __fdiv_rn(o, wts[32]));
+    }
 }
 
 template <int D>
@@ -714,18 +774,20 @@ cudaError_t launch_attend_t(const AttendArgs &a, bool q_bf16, bool out_bf16, int
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
-    cudaError_t pe = launch_pdl(prep_q_kernel<D>, dim3(a.B, 8), dim3(256), 0, stream, a, (int)q_bf16);
-    if (pe != cudaSuccess) return pe;
     bool saturated;
     if (variant == CSLA_VARIANT_SATURATED) saturated = true;
     else if (variant == CSLA_VARIANT_STARVED) saturated = false;
     else saturated = a.B >= num_sms || a.max_chunks <= 1;
     if (saturated)
-        return launch_pdl(attend_kernel<D, true>, dim3(a.B), dim3(kThreads), kSmem, stream, a, (int)out_bf16);
+        return launch_pdl(attend_kernel<D, true>, dim3(a.B), dim3(kThreads), kSmem, stream, a, (int)q_bf16,
+                          (int)out_bf16);
     cudaError_t e =
-        launch_pdl(attend_kernel<D, false>, dim3(a.max_chunks, a.B), dim3(kThreads), kSmem, stream, a, (int)out_bf16);
+        launch_pdl(attend_kernel<D, false>, dim3(a.max_chunks, a.B), dim3(kThreads), kSmem, stream, a, (int)q_bf16,
+                   (int)out_bf16);
     if (e != cudaSuccess) return e;
-    return launch_pdl(combine_kernel<D>, dim3(a.H, a.B), dim3(128), 0, stream, a, (int)out_bf16);
+    if (a.max_chunks <= 16)
+        return launch_pdl(combine_kernel<D, 16>, dim3(a.H, a.B), dim3(128), 0, stream, a, (int)out_bf16);
+    return launch_pdl(combine_kernel<D, 32>, dim3(a.H, a.B), dim3(128), 0, stream, a, (int)out_bf16);
 }
 
 }  // namespace

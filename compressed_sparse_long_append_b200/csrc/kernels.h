@@ -105,7 +105,6 @@ struct AttendArgs {
     const uint8_t *win_rows;
     const float *win_scales;
     void *out;
-    uint8_t *qimg;        // workspace: per request, Qhat as the kernel's shared-memory image
     float *part;          // workspace: chunk partials
     int max_chunks;
     int max_len;

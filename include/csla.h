@@ -282,7 +282,7 @@ int csla_version(void);
  * device and copies up to `bytes` of records to host memory `records`,
  * storing how many in *count; csla_timeline_clear synchronises and empties
  * the buffer.  Kernel ids: 1 compress, 2 tail update, 3 index-query
- * projection, 4 wide projection, 5 indexer, 6 top-k, 7 query preparation,
+ * projection, 4 wide projection, 5 indexer, 6 top-k, (7 unused),
  * 8 attention, 9 chunk combine.
  */
 #ifdef CSLA_TIMELINE

@@ -73,9 +73,9 @@ def test_workspace_sizes():
     # indexer: B * NQ * dI bf16 with NQ = 3*HI rounded up to 16
     assert C.csla_workspace_size(cfg, C.CSLA_OP_INDEXER, 8, 131072) == 8 * 48 * 128 * 2
     assert C.csla_workspace_size(cfg, C.CSLA_OP_TOPK, 8, 131072) == 0
-    # attention: B * 64 * D bf16 (query image) + B * chunks * (H*D + 2H) floats;
+    # attention: B * chunks * (H*D + 2H) floats (chunk partials);
     # 512+128 rows -> 10 chunks of 64
-    assert C.csla_workspace_size(cfg, C.CSLA_OP_CSA_ATTEND, 8, 512) == 8 * 64 * 512 * 2 + 8 * 10 * (64 * 512 + 128) * 4
+    assert C.csla_workspace_size(cfg, C.CSLA_OP_CSA_ATTEND, 8, 512) == 8 * 10 * (64 * 512 + 128) * 4
     hca = _cfg(m=128)
-    assert C.csla_workspace_size(hca, C.CSLA_OP_HCA_ATTEND, 4, 1 << 20) == 4 * 64 * 512 * 2 + 4 * 32 * (64 * 512 + 128) * 4
+    assert C.csla_workspace_size(hca, C.CSLA_OP_HCA_ATTEND, 4, 1 << 20) == 4 * 32 * (64 * 512 + 128) * 4
     assert C.csla_workspace_size(_cfg(m=8), C.CSLA_OP_TOPK, 1, 1) == 0
