@@ -364,22 +364,22 @@ def breakdown(steps, inputs, W, K):
 
 
 def call_time(steps, inputs, W, K, j):
-    """Average duration (ms) of call j alone: its graphs (one per copy,
-    rotating, so the call's inputs start out of L2) replayed K times back to
-    back between one event pair.  Call j must only read the caches."""
+    """Average duration (ms) of call j alone: K calls on the R copies in turn
+    (so each call's inputs start out of L2), captured as one CUDA graph so
+    the calls follow each other like kernels in a step (launch overlap as in
+    the step), one event pair around the replay.  Call j must only read the
+    caches."""
     import torch
     R = len(steps)
-    graphs = [capture(lambda r=r: steps[r].calls[j](inputs[W + r])) for r in range(R)]
-    for r in range(R):
-        graphs[r].replay()
+    g = capture(lambda: [steps[i % R].calls[j](inputs[W + i % R]) for i in range(K)])
+    g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for i in range(K):
-        graphs[i % R].replay()
+    g.replay()
     e1.record()
     torch.cuda.synchronize()
-    del graphs
+    del g
     return e0.elapsed_time(e1) / K
 
 

@@ -23,8 +23,9 @@
 //                       per row) and fetch the raw cache rows with 1-D bulk
 //                       copies into one of two staging buffers (tiles t+1 and
 //                       t+2 are in flight while tile t is converted); widen
-//                       fp8 codes to bf16 (exact) into the SW128 K-major X
-//                       tile once the previous tile's PV product is done;
+//                       fp8 codes to f16 (exact; the RoPE dims stay bf16)
+//                       into the SW128 K-major X tile once the previous
+//                       tile's PV product is done;
 //   warp 8 (MMA)        S = Qhat . X^T   tcgen05 M=64 (heads) N=64 (rows),
 //                                        nope and RoPE dims in separate TMEM
 //                                        accumulators: s = scale*S_nope + S_rope
@@ -33,7 +34,7 @@
 //                       (the norm before the grid-dependency wait, the
 //                       rotation after it); per tile read S, P = 2^(s - m)
 //                       (lanes 0-15 of each warp own one head),
-//                       P_nope = bf16(P*scale), P_rope = bf16(P); lazy
+//                       P_nope = f16(P*scale), P_rope = bf16(P); lazy
 //                       rescale of O^T when a head's max grows by more than 8
 //                       (log2 units); at chunk end read O^T out as the partial.
 // mbarriers hand tiles between roles; every wait is bounded.
@@ -91,6 +92,7 @@ struct Misc {
     int tvalid[2][kTile];
     float fac[2][kHP];                 // per tile parity: O^T column factors (1 = none)
     uint64_t raw_full[2], x_full[2], x_empty[2], s_full, s_free, p_full, pv_done, o_free, q_ready, fac_ready;
+    uint64_t kb_full[8];               // per K block of X: widened (one phase per tile)
     int go[2];                         // loader: keep fetching (per tile parity)
     uint32_t tmem;
     int abort;
@@ -143,13 +145,17 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int g, int kb_bytes) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return (uint32_t)f32_to_bf16_bits(lo) | ((uint32_t)f32_to_bf16_bits(hi) << 16);
 }
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
 
 // ---------------------------------------------------------------- query preparation
 // Qhat = RoPE(RMSNorm(q_h) * gamma_q, t) for the 64 (padded) heads of the
 // request, built in shared memory by the softmax warps in two steps.
 // Before the grid-dependency wait (q and gamma_q are inputs of the call):
 // warp w normalises heads 16w .. 16w+15, lane l owning dims l*D/32 ..; the
-// non-RoPE dims go to the SW128 K-major Qhat image as bf16, the RoPE dims
+// non-RoPE dims go to the SW128 K-major Qhat image as f16, the RoPE dims
 // stay fp32 in the P area (64 heads x 64 dims x 4 B, unused until the first
 // tile's softmax).  After the wait, when the position t = len - 1 is known,
 // lane i rotates pair i of its warp's 16 heads and writes them as bf16.
@@ -226,15 +232,15 @@ __device__ void build_q_normed(const AttendArgs &a, int b, uint8_t *smem, int q_
                     const int d = d0 + e0;
                     if constexpr (DPL >= 8) {
                         uint4 o;
-                        o.x = pack_bf16x2(y[e0], y[e0 + 1]);
-                        o.y = pack_bf16x2(y[e0 + 2], y[e0 + 3]);
-                        o.z = pack_bf16x2(y[e0 + 4], y[e0 + 5]);
-                        o.w = pack_bf16x2(y[e0 + 6], y[e0 + 7]);
+                        o.x = pack_f16x2(y[e0], y[e0 + 1]);
+                        o.y = pack_f16x2(y[e0 + 2], y[e0 + 3]);
+                        o.z = pack_f16x2(y[e0 + 4], y[e0 + 5]);
+                        o.w = pack_f16x2(y[e0 + 6], y[e0 + 7]);
                         *reinterpret_cast<uint4 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB)) = o;
                     } else {
                         uint2 o;
-                        o.x = pack_bf16x2(y[e0], y[e0 + 1]);
-                        o.y = pack_bf16x2(y[e0 + 2], y[e0 + 3]);
+                        o.x = pack_f16x2(y[e0], y[e0 + 1]);
+                        o.y = pack_f16x2(y[e0 + 2], y[e0 + 3]);
                         *reinterpret_cast<uint2 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB) + (d & 7) * 2) = o;
                     }
                 }
@@ -296,21 +302,22 @@ __device__ __forceinline__ const uint8_t *row_source(const AttendArgs &a, int b,
     return nullptr;
 }
 
-// Widen one 16-byte chunk of a cache row into the bf16 X tile.
+// Widen one 16-byte chunk of a cache row into the X tile: fp8 codes become
+// f16 (exact), the RoPE dims stay bf16.
 template <int D>
 __device__ __forceinline__ void store_chunk(uint8_t *xs, int r, int c, const uint4 v) {
     using C = Cfg<D>;
     if (c < C::kNopeCH) {
         const int g0 = c * 2;   // 16 codes = two 8-dim groups
         uint4 lo, hi;
-        lo.x = e4m3x2_to_bf16x2(v.x & 0xFFFFu);
-        lo.y = e4m3x2_to_bf16x2(v.x >> 16);
-        lo.z = e4m3x2_to_bf16x2(v.y & 0xFFFFu);
-        lo.w = e4m3x2_to_bf16x2(v.y >> 16);
-        hi.x = e4m3x2_to_bf16x2(v.z & 0xFFFFu);
-        hi.y = e4m3x2_to_bf16x2(v.z >> 16);
-        hi.z = e4m3x2_to_bf16x2(v.w & 0xFFFFu);
-        hi.w = e4m3x2_to_bf16x2(v.w >> 16);
+        lo.x = e4m3x2_to_f16x2(v.x & 0xFFFFu);
+        lo.y = e4m3x2_to_f16x2(v.x >> 16);
+        lo.z = e4m3x2_to_f16x2(v.y & 0xFFFFu);
+        lo.w = e4m3x2_to_f16x2(v.y >> 16);
+        hi.x = e4m3x2_to_f16x2(v.z & 0xFFFFu);
+        hi.y = e4m3x2_to_f16x2(v.z >> 16);
+        hi.z = e4m3x2_to_f16x2(v.w & 0xFFFFu);
+        hi.w = e4m3x2_to_f16x2(v.w >> 16);
         *reinterpret_cast<uint4 *>(xs + sw128_off(r, g0, C::kKBBytes)) = lo;
         *reinterpret_cast<uint4 *>(xs + sw128_off(r, g0 + 1, C::kKBBytes)) = hi;
     } else {
@@ -324,9 +331,10 @@ struct Span {
     int c0, c1;
 };
 
+// Chunk partial record: O[H][D], then m[H] and l[H], all f32.
+__device__ __forceinline__ size_t partial_floats(int H, int D) { return (size_t)H * D + 2 * (size_t)H; }
 __device__ __forceinline__ float *partial_ptr(const AttendArgs &a, int b, int c, int D) {
-    const size_t stride = (size_t)a.H * D + 2 * (size_t)a.H;
-    return a.part + ((size_t)b * a.max_chunks + c) * stride;
+    return a.part + ((size_t)b * a.max_chunks + c) * partial_floats(a.H, D);
 }
 
 // ---------------------------------------------------------------- the three roles
@@ -367,24 +375,37 @@ __device__ void loader_role(const AttendArgs &a, int b, const Req &rq, Span sp, 
         const int buf = t & 1;
         // the staged rows, and the X tile free again (PV of the previous tile done)
         bool ok = t < issued && mbar_wait(&ms->raw_full[buf], (t >> 1) & 1, &ms->abort);
+        if (lt == 0 && t == 0) CSLA_TL_MARK_ANY(7);
         if (!ok && t < first_fail) first_fail = t;
         if (ok && t > 0) ok = mbar_wait(&ms->x_empty[(t - 1) & 1], ((t - 1) >> 1) & 1, &ms->abort);
-        if (ok) {
-            const uint8_t *raw = smem + (buf ? C::kOffRaw1 : C::kOffRaw0);
-            uint8_t *xs = smem + C::kOffX;
-#pragma unroll 6
-            for (int u = 0; u < C::kTPT; ++u) {
-                const int id = u * kLoadThreads + lt;
-                const int r = id / C::kCH, ch = id % C::kCH;
-                const uint4 v = ms->rawvalid[buf][r] ? *reinterpret_cast<const uint4 *>(raw + r * C::kRB + ch * 16)
-                                                     : make_uint4(0u, 0u, 0u, 0u);
-                store_chunk<D>(xs, r, ch, v);
+        const uint8_t *raw = smem + (buf ? C::kOffRaw1 : C::kOffRaw0);
+        uint8_t *xs = smem + C::kOffX;
+        // widen K block by K block; the MMA warp starts on a block as soon
+        // as every loader thread has arrived on its barrier
+#pragma unroll 1
+        for (int kb = 0; kb < C::kKB; ++kb) {
+            if (ok) {
+                // source chunks of this block: 4 fp8 chunks per row (nope) or
+                // 8 bf16 chunks per row (RoPE block)
+                const int cpr = kb < C::kKBN ? 4 : 8;
+                const int ch0 = kb < C::kKBN ? 4 * kb : C::kNopeCH;
+#pragma unroll 4
+                for (int id = lt; id < kTile * cpr; id += kLoadThreads) {
+                    const int r = id / cpr, ch = ch0 + id % cpr;
+                    const uint4 v = ms->rawvalid[buf][r]
+                                        ? *reinterpret_cast<const uint4 *>(raw + r * C::kRB + ch * 16)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+                    store_chunk<D>(xs, r, ch, v);
+                }
+                fence_proxy_async_smem();
             }
+            mbar_arrive(&ms->kb_full[kb]);
+        }
+        if (ok) {
             if (lt < kTile) {
                 ms->tscale[buf][lt] = ms->rawscale[buf][lt];
                 ms->tvalid[buf][lt] = ms->rawvalid[buf][lt];
             }
-            fence_proxy_async_smem();
             if (lt == 0 && t == 0) CSLA_TL_MARK_ANY(4);
         }
         mbar_arrive(&ms->x_full[buf]);
@@ -401,8 +422,14 @@ __device__ void loader_role(const AttendArgs &a, int b, const Req &rq, Span sp, 
 template <int D>
 __device__ void mma_role(const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
     using C = Cfg<D>;
-    constexpr uint32_t kIdescS = idesc_bf16(64, 64, false, false);
-    constexpr uint32_t kIdescO = idesc_bf16(128, 64, true, false);
+    // f16 operands for the fp8-coded dims, bf16 for the RoPE dims.  The PV
+    // blocks are 128 dims tall, so the last non-RoPE block also spans the
+    // RoPE dims (and the RoPE block the last 64 non-RoPE dims) read as the
+    // other type: those O^T rows are never read out.
+    constexpr uint32_t kIdescSN = idesc_f16(64, 64, false, false);
+    constexpr uint32_t kIdescSR = idesc_bf16(64, 64, false, false);
+    constexpr uint32_t kIdescON = idesc_f16(128, 64, true, false);
+    constexpr uint32_t kIdescOR = idesc_bf16(128, 64, true, false);
     const uint32_t tmem = ms->tmem;
     const uint32_t q0 = smem_u32(smem + C::kOffQ);
     const uint32_t p0n = smem_u32(smem + C::kOffPn), p0r = smem_u32(smem + C::kOffPr);
@@ -414,20 +441,24 @@ __device__ void mma_role(const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
         const int hi = min(rq.n_rows, lo + rq.chunk);
         for (int r0 = lo, ti = 0; r0 < hi; r0 += kTile, ++ti, ++g) {
             const int buf = g & 1;
-            if (!mbar_wait(&ms->x_full[buf], (g >> 1) & 1, &ms->abort)) return;
             if (g > 0 && !mbar_wait(&ms->s_free, (g - 1) & 1, &ms->abort)) return;
-            tc_fence_after();
             const uint32_t x0 = smem_u32(smem + C::kOffX);
-#pragma unroll
-            for (int kb = 0; kb < C::kKBN; ++kb)
+#pragma unroll 1
+            for (int kb = 0; kb < C::kKBN; ++kb) {
+                if (!mbar_wait(&ms->kb_full[kb], g & 1, &ms->abort)) return;
+                tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    umma_bf16(tmem + C::kColSN, sdesc(q0 + kb * C::kQKB + ks * 32, 16, 1024),
-                              sdesc(x0 + kb * C::kKBBytes + ks * 32, 16, 1024), kIdescS, (kb | ks) ? 1u : 0u);
+                    umma_kind_f16(tmem + C::kColSN, sdesc(q0 + kb * C::kQKB + ks * 32, 16, 1024),
+                                  sdesc(x0 + kb * C::kKBBytes + ks * 32, 16, 1024), kIdescSN, (kb | ks) ? 1u : 0u);
+            }
+            if (!mbar_wait(&ms->kb_full[C::kKBN], g & 1, &ms->abort)) return;
+            tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                umma_bf16(tmem + C::kColSR, sdesc(q0 + C::kKBN * C::kQKB + ks * 32, 16, 1024),
-                          sdesc(x0 + C::kKBN * C::kKBBytes + ks * 32, 16, 1024), kIdescS, ks ? 1u : 0u);
+                umma_kind_f16(tmem + C::kColSR, sdesc(q0 + C::kKBN * C::kQKB + ks * 32, 16, 1024),
+                              sdesc(x0 + C::kKBN * C::kKBBytes + ks * 32, 16, 1024), kIdescSR, ks ? 1u : 0u);
+            if (g == 0) CSLA_TL_MARK_ANY(0);
             umma_commit(&ms->s_full);
             if (!mbar_wait(&ms->p_full, g & 1, &ms->abort)) return;
             if (ti == 0 && c > sp.c0 && !mbar_wait(&ms->o_free, (c - sp.c0 - 1) & 1, &ms->abort)) return;
@@ -436,14 +467,14 @@ __device__ void mma_role(const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
             for (int mb = 0; mb < C::kMB; ++mb)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    umma_bf16(tmem + C::kColO + 64 * mb,
+                    umma_kind_f16(tmem + C::kColO + 64 * mb,
                               sdesc(x0 + 2 * mb * C::kKBBytes + 2 * ks * 1024, C::kKBBytes, 1024),
-                              sdesc(p0n + ks * 32, 16, 1024), kIdescO, (ti > 0 || ks > 0) ? 1u : 0u);
+                              sdesc(p0n + ks * 32, 16, 1024), kIdescON, (ti > 0 || ks > 0) ? 1u : 0u);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                umma_bf16(tmem + C::kColOR,
+                umma_kind_f16(tmem + C::kColOR,
                           sdesc(x0 + 2 * (C::kMB - 1) * C::kKBBytes + 2 * ks * 1024, C::kKBBytes, 1024),
-                          sdesc(p0r + ks * 32, 16, 1024), kIdescO, (ti > 0 || ks > 0) ? 1u : 0u);
+                          sdesc(p0r + ks * 32, 16, 1024), kIdescOR, (ti > 0 || ks > 0) ? 1u : 0u);
             umma_commit(&ms->x_empty[buf]);
             umma_commit(&ms->pv_done);
         }
@@ -464,7 +495,7 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
 
     build_q_rope<D>(a, (long long)rq.L - 1, smem, ms);
 
-    int g = 0;
+    int g = 0, nfac = 0;
     for (int c = sp.c0; c < sp.c1; ++c) {
         const int lo = c * rq.chunk;
         const int hi = min(rq.n_rows, lo + rq.chunk);
@@ -519,10 +550,10 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
                     }
                     const float *sc = &ms->tscale[buf][c8 * 8];
                     uint4 un, ur;
-                    un.x = pack_bf16x2(__fmul_rn(p[0], sc[0]), __fmul_rn(p[1], sc[1]));
-                    un.y = pack_bf16x2(__fmul_rn(p[2], sc[2]), __fmul_rn(p[3], sc[3]));
-                    un.z = pack_bf16x2(__fmul_rn(p[4], sc[4]), __fmul_rn(p[5], sc[5]));
-                    un.w = pack_bf16x2(__fmul_rn(p[6], sc[6]), __fmul_rn(p[7], sc[7]));
+                    un.x = pack_f16x2(__fmul_rn(p[0], sc[0]), __fmul_rn(p[1], sc[1]));
+                    un.y = pack_f16x2(__fmul_rn(p[2], sc[2]), __fmul_rn(p[3], sc[3]));
+                    un.z = pack_f16x2(__fmul_rn(p[4], sc[4]), __fmul_rn(p[5], sc[5]));
+                    un.w = pack_f16x2(__fmul_rn(p[6], sc[6]), __fmul_rn(p[7], sc[7]));
                     ur.x = pack_bf16x2(p[0], p[1]);
                     ur.y = pack_bf16x2(p[2], p[3]);
                     ur.z = pack_bf16x2(p[4], p[5]);
@@ -535,12 +566,16 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
                 m_run = mnew;
                 ms->fac[g & 1][h] = f;
             }
-            // every head's factor is needed by every thread (each owns one O^T row)
-            mbar_arrive(&ms->fac_ready);
-            if (!mbar_wait(&ms->fac_ready, g & 1, &ms->abort)) return;
+            // every head's factor is needed by every thread (each owns one O^T
+            // row); a chunk's first tile has none (every factor is 1)
             bool any_rescale = false;
+            if (ti > 0) {
+                mbar_arrive(&ms->fac_ready);
+                if (!mbar_wait(&ms->fac_ready, nfac & 1, &ms->abort)) return;
+                ++nfac;
 #pragma unroll 8
-            for (int j = 0; j < kHP; ++j) any_rescale |= ms->fac[g & 1][j] != 1.f;
+                for (int j = 0; j < kHP; ++j) any_rescale |= ms->fac[g & 1][j] != 1.f;
+            }
             if (any_rescale) {
                 // O^T columns are heads: every thread scales its own dim lane.
 #pragma unroll 1
@@ -568,7 +603,7 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
         if (threadIdx.x == 0) CSLA_TL_MARK(2);
         tc_fence_after();
         float *part = partial_ptr(a, b, c, D);
-        const size_t HD = (size_t)a.H * D;
+        float *ml = part + (size_t)a.H * D;
 #pragma unroll 1
         for (int blk = 0; blk <= C::kMB; ++blk) {
             const bool rope_blk = blk == C::kMB;
@@ -589,8 +624,8 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
             }
         }
         if (head_thread && h < a.H) {
-            part[HD + h] = m_run;
-            part[HD + a.H + h] = l_run;
+            ml[h] = m_run;
+            ml[a.H + h] = l_run;
         }
         if (threadIdx.x == 0) CSLA_TL_MARK(3);
         tc_fence_before();
@@ -602,12 +637,12 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
 //   M = max(sink*log2e, m_0 .. m_{n-1})                (exact, order-free)
 //   w_c = 2^(m_c - M);  l = 2^(sink*log2e - M) + sum_c l_c w_c;  o_d = sum_c O_c[d] w_c
 // with both sums taken in chunk order; out = o / l.  The saturated and the
-// starved kernels both use these two functions.
+// starved kernels both use these functions.
 // fold_weights is warp-collective (lane c loads chunk c, n_chunks <= 32);
 // on return every lane holds w_c of its own chunk c in *w_lane and l in *l_out.
 __device__ __forceinline__ void fold_weights(const AttendArgs &a, int b, int n_chunks, int h, int D, float *w_lane,
                                              float *l_out) {
-    const size_t stride = (size_t)a.H * D + 2 * (size_t)a.H;
+    const size_t stride = partial_floats(a.H, D);
     const float *p = a.part + (size_t)b * a.max_chunks * stride + (size_t)a.H * D;
     const int lane = threadIdx.x & 31;
     const float z = __fmul_rn(__ldg(a.sink + h), kLog2e);
@@ -621,14 +656,16 @@ __device__ __forceinline__ void fold_weights(const AttendArgs &a, int b, int n_c
     *w_lane = wc;
     *l_out = l;
 }
+// O_c[d] of head h, chunk c.
+__device__ __forceinline__ float partial_o(const AttendArgs &a, int b, int c, int h, int d, int D) {
+    return partial_ptr(a, b, c, D)[(size_t)h * D + d];
+}
 // o_d = sum_c O_c[d] w_c in chunk order, w[] the per-chunk weights.
 __device__ __forceinline__ float fold_dim(const AttendArgs &a, int b, int n_chunks, int h, int d, int D,
                                           const float *w, float l) {
-    const size_t stride = (size_t)a.H * D + 2 * (size_t)a.H;
-    const float *p = a.part + (size_t)b * a.max_chunks * stride + (size_t)h * D + d;
     float v[32];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) v[c] = c < n_chunks ? p[c * stride] : 0.f;
+    for (int c = 0; c < 32; ++c) v[c] = c < n_chunks ? partial_o(a, b, c, h, d, D) : 0.f;
     float o = 0.f;
 #pragma unroll
     for (int c = 0; c < 32; ++c)
@@ -658,6 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int q
             mbar_init(&ms->x_full[i], kLoadThreads);
             mbar_init(&ms->x_empty[i], 1);
         }
+        for (int i = 0; i < C::kKB; ++i) mbar_init(&ms->kb_full[i], kLoadThreads);
         mbar_init(&ms->s_full, 1);
         mbar_init(&ms->s_free, 32 * kSoftWarps);
         mbar_init(&ms->p_full, 32 * kSoftWarps);
@@ -734,13 +772,12 @@ __global__ void __launch_bounds__(128) combine_kernel(AttendArgs a, int out_bf16
     const Req rq = request(a, b);
     if (!rq.ok) return;
     const int n_chunks = rq.n_chunks;
-    const size_t stride = (size_t)a.H * D + 2 * (size_t)a.H;
-    const float *p = a.part + (size_t)b * a.max_chunks * stride + (size_t)h * D + threadIdx.x;
     float v[kDPT][kMaxC];
 #pragma unroll
     for (int c = 0; c < kMaxC; ++c)
 #pragma unroll
-        for (int j = 0; j < kDPT; ++j) v[j][c] = c < n_chunks ? p[c * stride + 128 * j] : 0.f;
+        for (int j = 0; j < kDPT; ++j)
+            v[j][c] = c < n_chunks ? partial_o(a, b, c, h, threadIdx.x + 128 * j, D) : 0.f;
     if (threadIdx.x < 32) {
         float wl, l;
         fold_weights(a, b, n_chunks, h, D, &wl, &l);

@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(kIdxThreads)
                         const uint32_t half = k / 4, ko = (k % 4) * 32;
                         const uint64_t ad = sdesc(kb + half * (kTileE * 128) + ko, 16, 1024);
                         const uint64_t bd = sdesc(qb + half * (NQ * 128) + ko, 16, 1024);
-                        umma_bf16(tmem + acc * NQ, ad, bd, idesc, k > 0 ? 1u : 0u);
+                        umma_kind_f16(tmem + acc * NQ, ad, bd, idesc, k > 0 ? 1u : 0u);
                     }
                     umma_commit(empty + s);
                     umma_commit(tfull + acc);

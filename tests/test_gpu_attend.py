@@ -17,7 +17,7 @@ from helpers import oracle_cache
 pytestmark = pytest.mark.gpu
 
 MAX_ABS = 1e-2        # the contract's bound for O(1) outputs
-REL_RMS = 2e-2        # derived bound: error / RMS(output) (bf16 q and P operands)
+REL_RMS = 2e-2        # derived bound: error / RMS(output) (f16/bf16 q and P operands)
 
 
 def attend(w, lb, q, sink, gamma_q, lens, idx=None, variant=C.CSLA_VARIANT_AUTO, slots=None,
