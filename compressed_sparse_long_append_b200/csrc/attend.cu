@@ -174,14 +174,12 @@ __device__ void build_q_normed(const AttendArgs &a, int b, uint8_t *smem, int q_
         float x[kBatch][DPL];
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
-            const int h = h0 + u;
+            // padding heads (h >= H) load head H-1 (in bounds); their values are zeroed below
+            const int h = min(h0 + u, a.H - 1);
             const size_t off = ((size_t)b * a.H + h) * D + d0;
 #pragma unroll
             for (int e0 = 0; e0 < DPL; e0 += 8 > DPL ? DPL : 8) {
-                if (h >= a.H) {
-#pragma unroll
-                    for (int e = 0; e < (8 > DPL ? DPL : 8); ++e) x[u][e0 + e] = 0.f;
-                } else if (q_bf16) {
+                if (q_bf16) {
                     if constexpr (DPL >= 8) {
                         const uint4 w4 = __ldg(reinterpret_cast<const uint4 *>(
                             reinterpret_cast<const __nv_bfloat16 *>(a.q) + off + e0));
@@ -665,7 +663,7 @@ __device__ __forceinline__ float fold_dim(const AttendArgs &a, int b, int n_chun
                                           const float *w, float l) {
     float v[32];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) v[c] = c < n_chunks ? partial_o(a, b, c, h, d, D) : 0.f;
+    for (int c = 0; c < 32; ++c) v[c] = partial_o(a, b, min(c, n_chunks - 1), h, d, D);
     float o = 0.f;
 #pragma unroll
     for (int c = 0; c < 32; ++c)
@@ -772,12 +770,12 @@ __global__ void __launch_bounds__(128) combine_kernel(AttendArgs a, int out_bf16
     const Req rq = request(a, b);
     if (!rq.ok) return;
     const int n_chunks = rq.n_chunks;
+    // unconditional loads (chunks past the last reread the last one; unused)
     float v[kDPT][kMaxC];
 #pragma unroll
     for (int c = 0; c < kMaxC; ++c)
 #pragma unroll
-        for (int j = 0; j < kDPT; ++j)
-            v[j][c] = c < n_chunks ? partial_o(a, b, c, h, threadIdx.x + 128 * j, D) : 0.f;
+        for (int j = 0; j < kDPT; ++j) v[j][c] = partial_o(a, b, min(c, n_chunks - 1), h, threadIdx.x + 128 * j, D);
     if (threadIdx.x < 32) {
         float wl, l;
         fold_weights(a, b, n_chunks, h, D, &wl, &l);

@@ -104,26 +104,14 @@ struct BlockRows {
 
 constexpr int kMaxIdxPerThread = 2;   // index-key inputs (dI <= 512) per thread
 constexpr int kStageRows = 32;    // block rows staged in shared memory at a time
-constexpr int kStageBatch = 16;   // float4 loads a thread keeps in flight while staging
 
-// Rows c0 .. c0+R-1 of the block into xs[R][width] (shared memory); all of a
-// thread's loads of a batch are issued before any store.
+// Rows c0 .. c0+R-1 of the block into xs[R][width] (shared memory), one
+// float4 per thread and iteration.
 template <typename T>
 __device__ __forceinline__ void stage_rows(const BlockRows<T> &x, int c0, int R, float *xs) {
     const int nq = x.width >> 2, total = R * nq;
-    for (int i0 = 0; i0 < total; i0 += kThreads * kStageBatch) {
-        float4 v[kStageBatch];
-#pragma unroll
-        for (int u = 0; u < kStageBatch; ++u) {
-            const int idx = i0 + u * kThreads + threadIdx.x;
-            if (idx < total) v[u] = x.get(c0 + idx / nq, idx % nq);
-        }
-#pragma unroll
-        for (int u = 0; u < kStageBatch; ++u) {
-            const int idx = i0 + u * kThreads + threadIdx.x;
-            if (idx < total) reinterpret_cast<float4 *>(xs)[idx] = v[u];
-        }
-    }
+    for (int idx = threadIdx.x; idx < total; idx += kThreads)
+        reinterpret_cast<float4 *>(xs)[idx] = x.get(c0 + idx / nq, idx % nq);
 }
 
 // Pool the block with softmax weights of the scalar gates g_i = <x_i, w> +
