@@ -296,6 +296,18 @@ def capture(fn):
     return g
 
 
+def dp_max(value, world, device):
+    """Max over the ranks of a per-rank time (ms): the step time of the
+    data-parallel job is its slowest rank.  world == 1 returns value."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_steps(steps, inputs, W, K, e2e=False, profile=False):
     """W warm-up steps (direct calls), then K timed steps back to back.
     Step i runs on layer copy i % R with inputs[i]: the R copies together
@@ -513,9 +525,7 @@ def main():
     clocks = clk.stop()
     if world > 1:
         dist.barrier()
-        t = torch.tensor([ms_step], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = dp_max(ms_step, world, device)
 
     if args.profile:
         args.no_hca = args.no_cpu_baseline = True
@@ -527,10 +537,7 @@ def main():
         d2h = steps[0].out.numel() * steps[0].out.element_size()
         seg = breakdown(steps, inputs, W, K)
         ms_idx = call_time(steps, inputs, W, K, 1)
-    if world > 1:
-        t = torch.tensor([ms_e2e], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = dp_max(ms_e2e, world, device)
 
     # algorithmic bytes of one indexer call: every visible key (dI bf16) read
     # once, one f32 score written per key, W_iq read once

@@ -277,14 +277,18 @@ void csla_orc_index_scores(const double *qI, const double *w, int HI, int dI, co
 /* Top-k selector ([silicon] §CSA: picks the 512 (Pro: 1024) most relevant
  * compressed blocks).  Reading: total order (score descending, index
  * ascending); take min(k, n); return them in ascending index order; pad -1. */
-static const double *g_sort_scores;
+/* Sort key: the score travels with its index, so the comparator needs no
+ * shared state (requests are sorted concurrently under OpenMP). */
+typedef struct {
+    double score;
+    int32_t index;
+} orc_ranked;
 static int cmp_rank(const void *pa, const void *pb)
 {
-    int32_t a = *(const int32_t *)pa, b = *(const int32_t *)pb;
-    double sa = g_sort_scores[a], sb = g_sort_scores[b];
-    if (sa > sb) return -1;
-    if (sa < sb) return 1;
-    return (a < b) ? -1 : (a > b);
+    const orc_ranked *a = (const orc_ranked *)pa, *b = (const orc_ranked *)pb;
+    if (a->score > b->score) return -1;
+    if (a->score < b->score) return 1;
+    return (a->index < b->index) ? -1 : (a->index > b->index);
 }
 static int cmp_int(const void *pa, const void *pb)
 {
@@ -294,13 +298,18 @@ static int cmp_int(const void *pa, const void *pb)
 void csla_orc_topk(const double *scores, int n, int k, int32_t *idx)
 {
     int i, take = n < k ? n : k;
-    int32_t *order = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n > 0 ? n : 1));
-    for (i = 0; i < n; ++i) order[i] = i;
-    g_sort_scores = scores;
-    qsort(order, (size_t)n, sizeof(int32_t), cmp_rank);
-    qsort(order, (size_t)take, sizeof(int32_t), cmp_int);
-    for (i = 0; i < k; ++i) idx[i] = (i < take) ? order[i] : -1;
+    orc_ranked *order = (orc_ranked *)malloc(sizeof(orc_ranked) * (size_t)(n > 0 ? n : 1));
+    int32_t *picked = (int32_t *)malloc(sizeof(int32_t) * (size_t)(take > 0 ? take : 1));
+    for (i = 0; i < n; ++i) {
+        order[i].score = scores[i];
+        order[i].index = i;
+    }
+    qsort(order, (size_t)n, sizeof(orc_ranked), cmp_rank);
+    for (i = 0; i < take; ++i) picked[i] = order[i].index;
+    qsort(picked, (size_t)take, sizeof(int32_t), cmp_int);
+    for (i = 0; i < k; ++i) idx[i] = (i < take) ? picked[i] : -1;
     free(order);
+    free(picked);
 }
 
 /* Core MQA with sink ([silicon] §CSA: top-k entries concatenated with the 128

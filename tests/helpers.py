@@ -24,9 +24,10 @@ def block_table(w: Workload, lens, n_slots, seed_name="bt"):
     return bt, max(total, 1)
 
 
-def oracle_cache(w: Workload, lens, params=None, with_raw=False):
-    """Expected cache of len(lens) requests (slot i = request i) after their
-    whole token streams 0..L_i-1 were appended, computed by the oracle."""
+def oracle_cache(w: Workload, lens, params=None, with_raw=False, stream_ids=None):
+    """Expected cache of len(lens) requests (slot i = request i, whose token
+    stream is stream_ids[i], default i) after their whole token streams
+    0..L_i-1 were appended, computed by the oracle."""
     p = params or layer_params(w)
     n_slots = len(lens)
     bt, n_pages = block_table(w, lens, n_slots)
@@ -39,7 +40,7 @@ def oracle_cache(w: Workload, lens, params=None, with_raw=False):
     win_scales = np.zeros((n_slots, w.n_win), np.float32)
     raws = []
     for s, L in enumerate(lens):
-        ts = token_stream(w, s, 0, L)
+        ts = token_stream(w, s if stream_ids is None else stream_ids[s], 0, L)
         raws.append(ts)
         exp = oracle.expected_append(ts["kv"], ts.get("idx"), 0, L, w.m, p["gamma_kv"], p["wg"],
                                      p["gb"], p.get("wgi"), p.get("gbi"), w.eps, w.theta, w.d_rope,
