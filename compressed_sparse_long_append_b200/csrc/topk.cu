@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
     CSLA_TL_WAITED();
     const int L = slot_ok ? a.len[slot] : 0;
     int n = L / a.m;
-    if (!slot_ok || L > a.max_n * a.m) {
+    if (!slot_ok || L / a.m > a.max_n) {
         if (threadIdx.x == 0) set_dev_err(CSLA_DEVERR_LEN);
         n = 0;
     }
@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kRThreads, 1) topk_reg_kernel(TopkArgs a) {
     CSLA_TL_WAITED();
     const int L = slot_ok ? a.len[slot] : 0;
     int n = L / a.m;
-    if (!slot_ok || L > a.max_n * a.m) {
+    if (!slot_ok || L / a.m > a.max_n) {
         if (threadIdx.x == 0) set_dev_err(CSLA_DEVERR_LEN);
         n = 0;
     }
