@@ -16,8 +16,12 @@
 // owns a contiguous range, per-warp counts give its first slot and ballots
 // place the picks, so indices come out ascending.  All counts are integers:
 // the selection is exact and independent of thread timing and batch.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
+
+namespace cg = cooperative_groups;
 
 namespace csla {
 namespace {
@@ -271,6 +275,44 @@ __device__ __forceinline__ int warp_prefix(const int *v, int warp, int *total) {
     return __shfl_sync(0xffffffffu, incl - x, warp);
 }
 
+// The bin of sh.hist[0..nb) holding the krem-th largest key (counted from
+// the top): sh.sel_bin, and the rank within it: sh.sel_krem.  All threads.
+__device__ void pick_bin_r(RegShared &sh, int nb, int krem) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // thread t covers bins nb-1-t*per .. (highest first); per = 0 for t beyond nb
+    const int per = (nb + kRThreads - 1) / kRThreads;
+    int c = 0;
+    for (int q = 0; q < per; ++q) {
+        const int bin = nb - 1 - (threadIdx.x * per + q);
+        if (bin >= 0) c += sh.hist[bin];
+    }
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) sh.warp_a[warp] = incl;
+    __syncthreads();
+    int total;
+    const int before = warp_prefix(sh.warp_a, warp, &total);
+    const int excl = before + incl - c;
+    if (excl < krem && krem <= excl + c) {
+        int run = excl;
+        for (int q = 0; q < per; ++q) {
+            const int bin = nb - 1 - (threadIdx.x * per + q);
+            const int h = bin >= 0 ? sh.hist[bin] : 0;
+            if (run + h >= krem) {
+                sh.sel_bin = bin;
+                sh.sel_krem = krem - run;
+                break;
+            }
+            run += h;
+        }
+    }
+    __syncthreads();
+}
+
 // Radix select: the key of rank `rank` (1 = largest) among the non-zero keys
 // that each thread passes to the callback given to each(), all of which
 // share their top 32 - bits bits with `prefix`; *krem_out = how many keys
@@ -295,38 +337,7 @@ __device__ uint32_t radix_select(RegShared &sh, const Each &each, int rank, uint
             if (key != 0u && (key & pmask) == prefix) atomicAdd(&sh.hist[(key >> shb) & (uint32_t)(nb - 1)], 1);
         });
         __syncthreads();
-        // thread t covers bins nb-1-t*per .. (highest first); per = 0 for t beyond nb
-        const int per = (nb + kRThreads - 1) / kRThreads;
-        int c = 0;
-        for (int q = 0; q < per; ++q) {
-            const int bin = nb - 1 - (threadIdx.x * per + q);
-            if (bin >= 0) c += sh.hist[bin];
-        }
-        int incl = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += t;
-        }
-        if (lane == 31) sh.warp_a[warp] = incl;
-        __syncthreads();
-        int total;
-        const int before = warp_prefix(sh.warp_a, warp, &total);
-        const int excl = before + incl - c;
-        if (excl < krem && krem <= excl + c) {
-            int run = excl;
-            for (int q = 0; q < per; ++q) {
-                const int bin = nb - 1 - (threadIdx.x * per + q);
-                const int h = bin >= 0 ? sh.hist[bin] : 0;
-                if (run + h >= krem) {
-                    sh.sel_bin = bin;
-                    sh.sel_krem = krem - run;
-                    break;
-                }
-                run += h;
-            }
-        }
-        __syncthreads();
+        pick_bin_r(sh, nb, krem);
         const int sel = sh.sel_bin;
         prefix |= (uint32_t)sel << shb;
         pmask |= (uint32_t)(nb - 1) << shb;
@@ -548,6 +559,302 @@ __global__ void __launch_bounds__(kRThreads, 1) topk_reg_kernel(TopkArgs a) {
     CSLA_TL_MARK(4);
 }
 
+// ---------------------------------------------------------------- cluster variant
+// For n <= kRegMax: one cluster of kG = 4 CTAs (512 threads each) per
+// request; CTA c owns the c-th quarter of the scores, warp w of it a
+// contiguous range, lane l the scores 32j + l of that range (18 rows) in
+// registers.  The steps of the register variant, spread over the cluster:
+//  1. every warp sorts a 32-key sample of its range and publishes its
+//     2nd-largest key; after a cluster barrier every CTA reads all 64 and
+//     takes the j-th largest as the threshold t0 (j = ceil(2048k/n), at
+//     most 64), so that about 2k keys or more lie above it;
+//  2. each warp compacts its scores >= t0 into its own region (index
+//     order) and publishes the count; after a cluster barrier every CTA
+//     reads the 64 counts, and when every region fitted and there are at
+//     least k candidates, copies its regions into CTA 0's shared memory at
+//     their exclusive-prefix offsets (so CTA 0 holds all candidates in
+//     index order);
+//  3. after a third barrier CTA 0 finds the exact k-th key among the
+//     candidates and writes the output, as the register variant does.
+// Otherwise (rare: heavy ties, or a sample far off) all four CTAs run the
+// radix select over every key with their four histograms summed through
+// distributed shared memory, and each writes its own picks.
+constexpr int kG = 4;
+constexpr int kCPer = kPer / kG;                  // 18 scores per thread
+constexpr int kOwn = 128;                         // candidates per warp region
+
+struct ClShared {
+    RegShared reg;                                // CTA 0: gathered candidates and select scratch
+    uint32_t okey[kRWarps][kOwn];
+    int oidx[kRWarps][kOwn];
+    int ocnt[kRWarps];
+    uint32_t tw[kRWarps], wmax[kRWarps];
+    int hist[kBins];                              // fallback: this CTA's histogram
+    int fgt[kRWarps], feq[kRWarps];               // fallback: per-warp output counts
+};
+
+__global__ void __cluster_dims__(kG, 1, 1) __launch_bounds__(kRThreads, 1) topk_cluster_kernel(TopkArgs a) {
+    CSLA_TL_SCOPE(kTlTopk);
+    extern __shared__ __align__(16) uint8_t dyn_cl[];
+    ClShared &sh = *reinterpret_cast<ClShared *>(dyn_cl);
+    pdl_trigger();
+    cg::cluster_group cl = cg::this_cluster();
+    const int cr = (int)cl.block_rank();
+    const int b = blockIdx.x / kG;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const unsigned below = (1u << lane) - 1u;
+    const int slot = __ldg(a.slots + b);
+    const bool slot_ok = slot >= 0 && slot < a.n_slots;
+    pdl_wait();
+    CSLA_TL_WAITED();
+    const int L = slot_ok ? a.len[slot] : 0;
+    int n = L / a.m;
+    if (!slot_ok || L / a.m > a.max_n) {
+        if (threadIdx.x == 0 && cr == 0) set_dev_err(CSLA_DEVERR_LEN);
+        n = 0;
+    }
+    const int k = a.k;
+    int32_t *out = a.idx + (size_t)b * k;
+    if (n <= k) {   // the same decision in every CTA of the cluster
+        if (cr == 0)
+            for (int j = threadIdx.x; j < k; j += kRThreads) out[j] = j < n ? j : -1;
+        return;
+    }
+    const float *sc = a.scores + (size_t)b * a.stride;
+    const int segc = (n + kG - 1) / kG;
+    const int c0 = min(n, cr * segc), cn = min(n, c0 + segc) - c0;
+    const int seg = (cn + kRWarps - 1) / kRWarps;
+    const int wlo = warp * seg;                   // the warp's range, relative to c0
+    const int base = c0 + wlo;
+    float f[kCPer];
+#pragma unroll
+    for (int j = 0; j < kCPer; ++j) {
+        const int r = 32 * j + lane;
+        f[j] = (r < seg && wlo + r < cn) ? sc[base + r] : __int_as_float(-1);   // the NaN whose key is 0
+    }
+    CSLA_TL_MARK(0);
+
+    // ---- 1. threshold: per-warp sorted sample, smallest rw-th largest over the cluster
+    const int js = (lane * ((seg + 31) >> 5)) >> 5;
+    uint32_t smp = 0;
+#pragma unroll
+    for (int j = 0; j < kCPer; ++j)
+        if (j == js) smp = score_key(f[j]);
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const uint32_t o = __shfl_xor_sync(0xffffffffu, smp, stride);
+            const bool desc = (lane & size) == 0 || size == 32;
+            const bool lower = (lane & stride) == 0;
+            smp = (lower == desc) ? max(smp, o) : min(smp, o);
+        }
+    }
+    // each warp publishes its 2nd-largest sample key; t0 = the j-th largest of
+    // the 64 published keys, so that >= 2j samples (1 per n/2048 keys) are
+    // >= t0: j = ceil(k * 2048 / n) puts about 2k keys or more above t0
+    const uint32_t s_w = __shfl_sync(0xffffffffu, smp, 1);
+    if (lane == 0) sh.tw[warp] = s_w;
+    cl.sync();
+    const int jth = min(2 * kRWarps * kG, max(1, (int)((2048LL * k + n - 1) / n)));
+    const uint32_t v0 = cl.map_shared_rank(sh.tw, lane / kRWarps)[lane % kRWarps];
+    const uint32_t v1 = cl.map_shared_rank(sh.tw, 2 + lane / kRWarps)[lane % kRWarps];
+    // rank of each value (larger first, ties by position) among the 64
+    int r0 = 0, r1 = 0;
+#pragma unroll 8
+    for (int q = 0; q < 32; ++q) {
+        const uint32_t w0 = __shfl_sync(0xffffffffu, v0, q), w1 = __shfl_sync(0xffffffffu, v1, q);
+        r0 += (w0 > v0 || (w0 == v0 && q < lane)) + (w1 > v0);
+        r1 += (w0 > v1 || w0 == v1) + (w1 > v1 || (w1 == v1 && q < lane));
+    }
+    const unsigned h0 = __ballot_sync(0xffffffffu, r0 == jth - 1), h1 = __ballot_sync(0xffffffffu, r1 == jth - 1);
+    const uint32_t t0 = h0 ? __shfl_sync(0xffffffffu, v0, __ffs(h0) - 1) : __shfl_sync(0xffffffffu, v1, __ffs(h1) - 1);
+    CSLA_TL_MARK(1);
+
+    // ---- 2. this warp's candidates (scores >= the value of t0) into its region
+    const float f0 = t0 == 0u ? -INFINITY : key_value(t0);
+    int pos = 0;
+    uint32_t cmax = 0;
+#pragma unroll
+    for (int j = 0; j < kCPer; ++j) {
+        const bool q = f[j] >= f0;
+        const unsigned mq = __ballot_sync(0xffffffffu, q);
+        const int at = pos + __popc(mq & below);
+        if (q && at < kOwn) {
+            const uint32_t key = score_key(f[j]);
+            sh.okey[warp][at] = key;
+            sh.oidx[warp][at] = base + 32 * j + lane;
+            cmax = max(cmax, key);
+        }
+        pos += __popc(mq);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+    if (lane == 0) {
+        sh.ocnt[warp] = pos;
+        sh.wmax[warp] = cmax;
+    }
+    cl.sync();
+    // the 64 counts in (CTA, warp) order: lane l holds entries l and 32 + l
+    const int *rc0 = cl.map_shared_rank(sh.ocnt, lane / kRWarps);
+    const int *rc1 = cl.map_shared_rank(sh.ocnt, 2 + lane / kRWarps);
+    const int n0 = rc0[lane % kRWarps], n1 = rc1[lane % kRWarps];
+    uint32_t kmax = max(cl.map_shared_rank(sh.wmax, lane / kRWarps)[lane % kRWarps],
+                        cl.map_shared_rank(sh.wmax, 2 + lane / kRWarps)[lane % kRWarps]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    const bool fits = __all_sync(0xffffffffu, n0 <= kOwn && n1 <= kOwn);
+    int i0 = n0, i1 = n1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, i0, o);
+        const int u = __shfl_up_sync(0xffffffffu, i1, o);
+        if (lane >= o) {
+            i0 += t;
+            i1 += u;
+        }
+    }
+    const int tot0 = __shfl_sync(0xffffffffu, i0, 31);
+    const int n_ge = tot0 + __shfl_sync(0xffffffffu, i1, 31);
+    const int e = cr * kRWarps + warp;            // this warp's entry in (CTA, warp) order
+    const int off = e < 32 ? __shfl_sync(0xffffffffu, i0 - n0, e)
+                           : tot0 + __shfl_sync(0xffffffffu, i1 - n1, e - 32);
+    const bool fast = fits && n_ge >= k;
+    if (fast) {
+        uint32_t *gk = cl.map_shared_rank(&sh.reg.ckey[0][0], 0);
+        int *gi = cl.map_shared_rank(&sh.reg.cidx[0][0], 0);
+        const int my = sh.ocnt[warp];
+        for (int i = lane; i < my; i += 32) {
+            gk[off + i] = sh.okey[warp][i];
+            gi[off + i] = sh.oidx[warp][i];
+        }
+    }
+    cl.sync();
+    CSLA_TL_MARK(2);
+
+    if (fast) {
+        if (cr != 0) return;
+        // ---- 3. CTA 0: warp w takes the flat candidates [512w, 512w + 512)
+        RegShared &rs = sh.reg;
+        const int my_n = min(kRegion, max(0, n_ge - warp * kRegion));
+        int krem;
+        const int bits = 32 - __clz(t0 ^ kmax);
+        const uint32_t T = radix_select(rs, [&](auto fn) {
+            for (int i = lane; i < my_n; i += 32) fn(rs.ckey[warp][i]);
+        }, k, kmax, bits, &krem);
+        CSLA_TL_MARK(3);
+        int gt = 0, eq = 0;
+        for (int i = lane; i < my_n; i += 32) {
+            const uint32_t key = rs.ckey[warp][i];
+            gt += key > T;
+            eq += key == T;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            gt += __shfl_xor_sync(0xffffffffu, gt, o);
+            eq += __shfl_xor_sync(0xffffffffu, eq, o);
+        }
+        if (lane == 0) {
+            rs.warp_a[warp] = gt;
+            rs.warp_b[warp] = eq;
+        }
+        __syncthreads();
+        int tot;
+        const int gt_before = warp_prefix(rs.warp_a, warp, &tot);
+        const int eq_before = warp_prefix(rs.warp_b, warp, &tot);
+        int opos = gt_before + min(eq_before, krem);
+        int eq_seen = eq_before;
+        for (int i0 = 0; i0 < my_n; i0 += 32) {
+            const int i = i0 + lane;
+            const uint32_t key = i < my_n ? rs.ckey[warp][i] : 0u;
+            const bool is_gt = i < my_n && key > T;
+            const bool is_eq = i < my_n && key == T;
+            const unsigned meq = __ballot_sync(0xffffffffu, is_eq);
+            const bool take_eq = is_eq && (eq_seen + __popc(meq & below)) < krem;
+            const unsigned mtake = __ballot_sync(0xffffffffu, is_gt || take_eq);
+            if (is_gt || take_eq) out[opos + __popc(mtake & below)] = rs.cidx[warp][i];
+            opos += __popc(mtake);
+            eq_seen += __popc(meq);
+        }
+        CSLA_TL_MARK(4);
+        return;
+    }
+
+    // ---- fallback: radix select over every key, histograms summed across the cluster
+    RegShared &rs = sh.reg;
+    uint32_t prefix = 0, pmask = 0;
+    int krem = k;
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shb = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const int nb = pass == 2 ? 1024 : 2048;
+        for (int i = threadIdx.x; i < kBins; i += kRThreads) sh.hist[i] = 0;
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < kCPer; ++j) {
+            const uint32_t key = score_key(f[j]);
+            if (key != 0u && (key & pmask) == prefix) atomicAdd(&sh.hist[(key >> shb) & (uint32_t)(nb - 1)], 1);
+        }
+        cl.sync();
+        for (int i = threadIdx.x; i < nb; i += kRThreads) {
+            int t = 0;
+#pragma unroll
+            for (int q = 0; q < kG; ++q) t += cl.map_shared_rank(sh.hist, q)[i];
+            rs.hist[i] = t;
+        }
+        __syncthreads();
+        pick_bin_r(rs, nb, krem);
+        prefix |= (uint32_t)rs.sel_bin << shb;
+        pmask |= (uint32_t)(nb - 1) << shb;
+        krem = rs.sel_krem;
+        cl.sync();   // every CTA has read every histogram before the next pass clears them
+    }
+    const uint32_t T = prefix;
+    int gt = 0, eq = 0;
+#pragma unroll
+    for (int j = 0; j < kCPer; ++j) {
+        const uint32_t key = score_key(f[j]);
+        gt += __popc(__ballot_sync(0xffffffffu, key > T));
+        eq += __popc(__ballot_sync(0xffffffffu, key == T));
+    }
+    if (lane == 0) {
+        sh.fgt[warp] = gt;
+        sh.feq[warp] = eq;
+    }
+    cl.sync();
+    // keys before this warp: the lower CTAs' warps, then this CTA's lower warps
+    int gt_before = 0, eq_before = 0;
+    for (int q = 0; q < cr; ++q) {
+        const int *rg = cl.map_shared_rank(sh.fgt, q), *re = cl.map_shared_rank(sh.feq, q);
+        gt_before += lane < kRWarps ? rg[lane] : 0;
+        eq_before += lane < kRWarps ? re[lane] : 0;
+    }
+    if (lane < kRWarps && lane < warp) {
+        gt_before += sh.fgt[lane];
+        eq_before += sh.feq[lane];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        gt_before += __shfl_xor_sync(0xffffffffu, gt_before, o);
+        eq_before += __shfl_xor_sync(0xffffffffu, eq_before, o);
+    }
+    int opos = gt_before + min(eq_before, krem);
+    int eq_seen = eq_before;
+#pragma unroll
+    for (int j = 0; j < kCPer; ++j) {
+        const uint32_t key = score_key(f[j]);
+        const bool is_gt = key > T;
+        const bool is_eq = key == T;
+        const unsigned meq = __ballot_sync(0xffffffffu, is_eq);
+        const bool take_eq = is_eq && (eq_seen + __popc(meq & below)) < krem;
+        const unsigned mtake = __ballot_sync(0xffffffffu, is_gt || take_eq);
+        if (is_gt || take_eq) out[opos + __popc(mtake & below)] = base + 32 * j + lane;
+        opos += __popc(mtake);
+        eq_seen += __popc(meq);
+    }
+    cl.sync();   // no CTA leaves while another may still read its counts
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
@@ -562,10 +869,13 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(topk_reg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RegShared));
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(ClShared));
+        if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
     if (a.max_n <= kRegMax)
-        return launch_pdl(topk_reg_kernel, dim3(a.B), dim3(kRThreads), sizeof(RegShared), stream, a);
+        return launch_pdl(topk_cluster_kernel, dim3(a.B * kG), dim3(kRThreads), sizeof(ClShared), stream, a);
     if (a.max_n <= kSmemKeysMax) {
         const size_t smem = kHistBytes + (size_t)(a.max_n > 0 ? a.max_n : 1) * sizeof(uint32_t);
         return launch_pdl(topk_kernel<true>, dim3(a.B), dim3(kThreads), smem, stream, a);
