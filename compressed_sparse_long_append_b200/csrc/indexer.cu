@@ -323,6 +323,8 @@ __global__ void __launch_bounds__(kIdxThreads)
                     const int s = n % kStages;
                     const int acc = n & 1;
                     if (!mbar_wait(full + s, (n / kStages) & 1, &abort_flag)) break;
+                    if (t == 0) CSLA_TL_MARK_ANY(0);
+                    if (t == kTPC - 1) CSLA_TL_MARK_ANY(1);
                     if (n >= 2 && !mbar_wait(tempty + acc, ((n / 2) - 1) & 1, &abort_flag)) break;
                     tc_fence_after();
                     const uint32_t kb = smem_u32(base + s * S::kKeyBytes);
@@ -362,6 +364,8 @@ __global__ void __launch_bounds__(kIdxThreads)
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(tempty + acc);
+            if (threadIdx.x == 64 && t == 0) CSLA_TL_MARK_ANY(2);
+            if (threadIdx.x == 64 && t == kTPC - 1) CSLA_TL_MARK_ANY(3);
             const int e = (t_begin + t) * kTileE + row;
             if (e < nv) {
                 float sc = 0.f;
