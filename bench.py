@@ -8,7 +8,9 @@ Workload (default): 8 requests at 131072-token context, m=4 (32768
 compressed entries each), 64 query heads, head_dim 512 (448 fp8 + 64 bf16
 RoPE dims), dc=1024 -> 16 index heads of 128, top-k 512, window 128.
 An HCA layer (4 requests at 1,048,576 tokens, m'=128) is measured after it
-and reported in the same JSON line under "hca_decode".
+and reported in the same JSON line under "hca_decode", then a CSA prefill
+chunk (4096 new tokens and their queries after a 262144-token prefix, top-k
+1024) under "csa_prefill".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -37,6 +39,8 @@ CHUNK = 16384          # tokens per compress call while building the caches
 CSA_COPIES = 4         # layer copies rotated per step: 4 x ~75 MB touched > 2 x L2
 HCA_COPIES = 14        # 14 x ~19.3 MB
 HEADROOM = 256         # cache capacity beyond the nominal context (tokens appended while timing)
+PREFILL = dict(T=4096, L0=262144, m=4, H=64, D=512, HI=16, dI=128, dc=1024, k=1024, n_win=128)
+NW = 127               # window rows from before a prefill chunk that its first query needs
 
 
 def parse():
@@ -46,12 +50,23 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-hca", action="store_true", help="skip the HCA layer measurement")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the CSA prefill-chunk measurement")
+    ap.add_argument("--prefill-only", action="store_true", help="only the CSA prefill-chunk measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", type=int, default=0, help="attention variant: 0 auto, 1 saturated, 2 starved")
     ap.add_argument("--profile", action="store_true",
                     help="only the timed CSA steps, bracketed by cudaProfilerStart/Stop (for ncu "
                          "--profile-from-start off); implies --no-hca --no-cpu-baseline and no e2e leg")
     return ap.parse_args()
+
+
+def tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops_sustained"]), "measured (sustained)"
+    except Exception:
+        return 1400.0, "fallback (sustained)"
 
 
 def peaks():
@@ -265,6 +280,147 @@ class HcaStep:
         C.csla_hca_attend(self.cfg, self.st, self.cache, self.slots, self.B, self.max_len, x["q"], C.CSLA_BF16,
                           self.p["sink"], self.p["gamma_q"], self.out, C.CSLA_BF16, self.variant, self.ws_a,
                           self.wsa)
+
+
+class PrefillStep:
+    """One CSA prefill chunk of one request: the ring snapshot of the NW
+    positions before the chunk, the chunk's append (T tokens, every token's
+    window row kept), then the T queries (query i at position L0+i) through
+    the indexer, top-k and attention with per-row visible lengths and the
+    window rows from the chunk buffer.  A last pair of device copies puts the
+    request's length and ring back to their pre-chunk state, so that every
+    step does the same work (the appended entries are rewritten with the same
+    bytes)."""
+
+    def __init__(self, lb, cp, params, kw, variant, device):
+        import torch
+        from compressed_sparse_long_append_b200 import csla as C
+        self.C, self.lb, self.cp, self.p, self.kw, self.variant = C, lb, cp, params, kw, variant
+        T, L0, k = kw["T"], kw["L0"], kw["k"]
+        L1 = L0 + T
+        self.T, self.max_len, self.stride = T, L1, L1 // kw["m"]
+        rb = (kw["D"] - 64) + 2 * 64
+        self.slot = torch.zeros(1, dtype=torch.int32, device=device)
+        self.rows_slots = torch.zeros(T, dtype=torch.int32, device=device)
+        self.buf = torch.zeros((NW + T, rb), dtype=torch.uint8, device=device)
+        self.bufsc = torch.zeros(NW + T, dtype=torch.float32, device=device)
+        self.q_len = torch.arange(L0 + 1, L1 + 1, dtype=torch.int32, device=device)
+        self.base = torch.full((T,), NW - L0, dtype=torch.int32, device=device)
+        self.qs_rows = C.queries(self.q_len)
+        self.qs_att = C.queries(self.q_len, self.buf, self.bufsc, self.base, NW + T)
+        self.tok = C.token_rows(self.buf, self.bufsc, NW + T, NW)
+        self.scores = torch.zeros((T, self.stride), dtype=torch.float32, device=device)
+        self.idx = torch.zeros((T, k), dtype=torch.int32, device=device)
+        self.out = torch.zeros((T, kw["H"], kw["D"]), dtype=torch.bfloat16, device=device)
+        cfg = lb.cfg()
+        self.wsi = C.csla_workspace_size(cfg, C.CSLA_OP_INDEXER, T, self.max_len)
+        self.wsa = C.csla_workspace_size(cfg, C.CSLA_OP_CSA_ATTEND, T, k)
+        self.ws_i = torch.zeros(self.wsi, dtype=torch.uint8, device=device)
+        self.ws_a = torch.zeros(self.wsa, dtype=torch.uint8, device=device)
+        self.len0, self.win0, self.wsc0 = lb.len.clone(), lb.win_rows.clone(), lb.win_scales.clone()
+        self.cfg, self.st, self.cache, self.cps = cfg, lb.state(), lb.cache(), cp.struct()
+        self.names = ["window_rows", "compress_append", "indexer_scores", "topk_select", "csa_attend", "rewind"]
+        self.calls = [self._snapshot, self._compress, self._indexer, self._topk, self._attend, self._rewind]
+
+    def _snapshot(self, x):
+        self.C.csla_window_rows(self.cfg, self.st, self.slot, 1, NW, self.buf, self.bufsc, NW + self.T)
+
+    def _compress(self, x):
+        C = self.C
+        C.csla_compress_append(self.cfg, self.st, self.cache, self.slot, 1, self.T, x["kv"], x["kidx"],
+                               C.CSLA_BF16, self.cps, tok=self.tok)
+
+    def _indexer(self, x):
+        C = self.C
+        C.csla_indexer_scores(self.cfg, self.st, self.cache, self.rows_slots, self.T, self.max_len, x["cq"],
+                              C.CSLA_BF16, self.p["W_iq"], C.CSLA_BF16, x["head_w"], self.scores, self.stride,
+                              self.ws_i, self.wsi, qs=self.qs_rows)
+
+    def _topk(self, x):
+        self.C.csla_topk_select(self.cfg, self.st, self.rows_slots, self.T, self.max_len, self.scores, self.stride,
+                                self.kw["k"], self.idx, qs=self.qs_rows)
+
+    def _attend(self, x):
+        C = self.C
+        C.csla_csa_attend(self.cfg, self.st, self.cache, self.rows_slots, self.T, x["q"], C.CSLA_BF16, self.idx,
+                          self.kw["k"], self.p["sink"], self.p["gamma_q"], self.out, C.CSLA_BF16, self.variant,
+                          self.ws_a, self.wsa, qs=self.qs_att)
+
+    def _rewind(self, x):
+        self.lb.len.copy_(self.len0)
+        self.lb.win_rows.copy_(self.win0)
+        self.lb.win_scales.copy_(self.wsc0)
+
+    def flops(self):
+        """Algorithmic tensor FLOPs of the chunk's queries: indexer
+        2*HI*dI per visible entry per query; attention 4*H*D per set row
+        (q.k and p.v) per query."""
+        kw = self.kw
+        L = [kw["L0"] + 1 + i for i in range(self.T)]
+        fi = sum(2 * kw["HI"] * kw["dI"] * (x // kw["m"]) for x in L)
+        fa = sum(4 * kw["H"] * kw["D"] * (min(kw["k"], x // kw["m"]) + min(kw["n_win"], x)) for x in L)
+        return fi, fa
+
+
+def prefill_leg(W, K, seed, rank, world, device, variant):
+    """Times the prefill chunk: one CUDA graph of the whole step (five library
+    calls and the rewind copies) replayed K times between one event pair."""
+    import torch
+    from csla_synth import torch_gen
+    kw = dict(PREFILL)
+    T, L0 = kw["T"], kw["L0"]
+    lb, cp, params = build_layer(dict(kw, B=1, L=L0 + T), 1, [L0], seed, rank, device)
+    x = {"q": torch_gen.normal(seed, "pq/%d" % rank, (T, kw["H"], kw["D"]), device=device).to(torch.bfloat16),
+         "kv": torch_gen.normal(seed, "kv/%d/0" % rank, (T, kw["D"]), start=L0 * kw["D"], device=device)
+         .to(torch.bfloat16),
+         "kidx": torch_gen.normal(seed, "idx/%d/0" % rank, (T, kw["dI"]), start=L0 * kw["dI"], device=device)
+         .to(torch.bfloat16),
+         "cq": torch_gen.normal(seed, "pcq/%d" % rank, (T, kw["dc"]), device=device).to(torch.bfloat16),
+         "head_w": torch_gen.normal(seed, "phw/%d" % rank, (T, kw["HI"]), device=device).to(torch.float32)}
+    st = PrefillStep(lb, cp, params, kw, variant, device)
+    for _ in range(W):
+        for c in st.calls:
+            c(x)
+    torch.cuda.synchronize()
+    g = capture(lambda: [c(x) for c in st.calls])
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = dp_max(e0.elapsed_time(e1) / K, world, device)
+    del g
+    # per-call times: each call its own graph, one event pair around each replay
+    gs = [capture(lambda c=c: c(x)) for c in st.calls]
+    seg = [0.0] * len(gs)
+    for _ in range(max(1, K // 2)):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(gs) + 1)]
+        ev[0].record()
+        for j, gg in enumerate(gs):
+            gg.replay()
+            ev[j + 1].record()
+        torch.cuda.synchronize()
+        for j in range(len(gs)):
+            seg[j] += ev[j].elapsed_time(ev[j + 1]) / max(1, K // 2)
+    del gs
+    fi, fa = st.flops()
+    tpk, tkind = tensor_peak()
+    tf = (fi + fa) / (ms * 1e-3) / 1e12
+    out = {"workload": "csa_prefill_T4096_L262144", "tokens_per_s": T * world / (ms * 1e-3), "ms_per_chunk": ms,
+           "queries": T, "prefix": L0, "topk": kw["k"],
+           "segments_ms": dict(zip(st.names, seg)),
+           "algorithmic_tflop": (fi + fa) / 1e12, "indexer_tflop": fi / 1e12, "attend_tflop": fa / 1e12,
+           "tensor_tflops": tf, "tensor_peak": tpk, "tensor_peak_kind": tkind, "tensor_frac": tf / tpk,
+           "indexer_tensor_frac": fi / (seg[2] * 1e-3) / 1e12 / tpk,
+           "attend_tensor_frac": fa / (seg[4] * 1e-3) / 1e12 / tpk,
+           "l2": "inputs larger than L2 (q 268 MB, fp32 scores 1.09 GB per chunk)",
+           "launch": "one CUDA graph per chunk, K replays between one event pair"}
+    del st, lb
+    torch.cuda.empty_cache()
+    return out
 
 
 def clone_layer(lb, params):
@@ -506,6 +662,14 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
     W, K = max(3, args.warmup), args.steps
     seed = 1
+    if args.prefill_only:
+        pre = prefill_leg(W, K, seed + 2, rank, world, device, args.variant)
+        if rank == 0:
+            print(json.dumps({"csa_prefill": pre}), flush=True)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
 
     # ---------------- CSA layer (the headline workload)
     kw = dict(CSA)
@@ -572,6 +736,15 @@ def main():
                "attend_tflops": hflops / (hms_att * 1e-3) / 1e12,
                "attend_tensor_frac_sustained": hflops / (hms_att * 1e-3) / 1e12 / 1395.7,
                "block_closes_in_timed_steps": closes}
+        del hsteps, hlb, hin
+        torch.cuda.empty_cache()
+
+    pre = None
+    if not args.no_prefill and not args.profile:
+        if args.no_hca:
+            del steps, lb
+            torch.cuda.empty_cache()
+        pre = prefill_leg(W, K, seed + 2, rank, world, device, args.variant)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -613,6 +786,7 @@ def main():
             "gpu_launches": launches_per_step * K,
             "clocks": clocks,
             "hca_decode": hca,
+            "csa_prefill": pre,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

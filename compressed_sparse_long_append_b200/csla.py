@@ -20,7 +20,7 @@ CSLA_PAGE_TOKENS = 128
 
 EXPORTS = ("csla_compress_append", "csla_indexer_scores", "csla_topk_select", "csla_csa_attend",
            "csla_hca_attend", "csla_workspace_size", "csla_device_error", "csla_strerror", "csla_version",
-           "csla_indexer_scores_noalloc")
+           "csla_indexer_scores_noalloc", "csla_window_rows")
 CSLA_NOALLOC_INDEXER_SCRATCH_BYTES = 786432
 
 
@@ -48,6 +48,32 @@ class csla_compress_params(ctypes.Structure):
                 ("wgi", ctypes.c_void_p), ("gbi", ctypes.c_void_p)]
 
 
+class csla_queries(ctypes.Structure):
+    """Query rows other than each request's latest token (see include/csla.h)."""
+    _fields_ = [("q_len", ctypes.c_void_p), ("win_rows", ctypes.c_void_p), ("win_scales", ctypes.c_void_p),
+                ("win_base", ctypes.c_void_p), ("n_win_rows", ctypes.c_int32)]
+
+
+class csla_token_rows(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("stride", ctypes.c_int32),
+                ("offset", ctypes.c_int32)]
+
+
+def queries(q_len, win_rows=None, win_scales=None, win_base=None, n_win_rows=0):
+    """csla_queries from tensors (or device addresses); the struct keeps the
+    tensors alive for as long as it lives."""
+    q = csla_queries(_ptr(q_len), _ptr(win_rows), _ptr(win_scales), _ptr(win_base), int(n_win_rows))
+    q._keep = (q_len, win_rows, win_scales, win_base)
+    return q
+
+
+def token_rows(rows, scales, stride, offset=0):
+    """csla_token_rows from tensors (or device addresses), kept alive by the struct."""
+    t = csla_token_rows(_ptr(rows), _ptr(scales), int(stride), int(offset))
+    t._keep = (rows, scales)
+    return t
+
+
 class CslaError(RuntimeError):
     def __init__(self, fn, status, bits=0):
         self.status, self.bits = status, bits
@@ -62,16 +88,17 @@ def _load():
     L = ctypes.CDLL(LIB_PATH)
     P, I, Z = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     sig = {
-        "csla_compress_append": [P, P, P, P, I, I, P, P, I, P, P],
-        "csla_indexer_scores": [P, P, P, P, I, I, P, I, P, I, P, P, I, P, Z, P],
-        "csla_topk_select": [P, P, P, I, I, P, I, I, P, P],
-        "csla_csa_attend": [P, P, P, P, I, P, I, P, I, P, P, P, I, I, P, Z, P],
-        "csla_hca_attend": [P, P, P, P, I, I, P, I, P, P, P, I, I, P, Z, P],
+        "csla_compress_append": [P, P, P, P, I, I, P, P, I, P, P, P],
+        "csla_window_rows": [P, P, P, I, I, P, P, I, P],
+        "csla_indexer_scores": [P, P, P, P, I, P, I, P, I, P, I, P, P, I, P, Z, P],
+        "csla_topk_select": [P, P, P, I, P, I, P, I, I, P, P],
+        "csla_csa_attend": [P, P, P, P, I, P, P, I, P, I, P, P, P, I, I, P, Z, P],
+        "csla_hca_attend": [P, P, P, P, I, P, I, P, I, P, P, P, I, I, P, Z, P],
         "csla_workspace_size": [P, I, I, I],
         "csla_device_error": [P, ctypes.POINTER(ctypes.c_uint32)],
         "csla_strerror": [ctypes.c_int],
         "csla_version": [],
-        "csla_indexer_scores_noalloc": [P, P, P, P, I, I, P, I, P, I, P, P, I, P],
+        "csla_indexer_scores_noalloc": [P, P, P, P, I, P, I, P, I, P, I, P, P, I, P],
     }
     res = {"csla_workspace_size": ctypes.c_size_t, "csla_strerror": ctypes.c_char_p}
     for name, args in sig.items():
@@ -109,47 +136,54 @@ def _ref(s):
     return None if s is None else ctypes.byref(s)
 
 
-def csla_compress_append(cfg, st, cache, slots, B, T, kv_new, kidx_new, kv_dtype, params, stream=None):
+def csla_compress_append(cfg, st, cache, slots, B, T, kv_new, kidx_new, kv_dtype, params, stream=None, tok=None):
+    """tok: optional csla_token_rows receiving every new token's window row."""
     return _check("csla_compress_append", _lib.csla_compress_append(
         _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, T, _ptr(kv_new), _ptr(kidx_new), kv_dtype,
-        _ref(params), _stream(stream)))
+        _ref(params), _ref(tok), _stream(stream)))
+
+
+def csla_window_rows(cfg, st, slots, B, n, rows_out, scales_out, stride, stream=None):
+    return _check("csla_window_rows", _lib.csla_window_rows(
+        _ref(cfg), _ref(st), _ptr(slots), B, n, _ptr(rows_out), _ptr(scales_out), stride, _stream(stream)))
 
 
 def csla_indexer_scores(cfg, st, cache, slots, B, max_len, cq, cq_dtype, W_iq, w_dtype, head_w, scores,
-                        scores_stride, workspace, workspace_bytes, stream=None):
+                        scores_stride, workspace, workspace_bytes, stream=None, qs=None):
+    """qs: optional csla_queries (per-row visible lengths)."""
     return _check("csla_indexer_scores", _lib.csla_indexer_scores(
-        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, max_len, _ptr(cq), cq_dtype, _ptr(W_iq), w_dtype,
+        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, _ref(qs), max_len, _ptr(cq), cq_dtype, _ptr(W_iq), w_dtype,
         _ptr(head_w), _ptr(scores), scores_stride, _ptr(workspace), workspace_bytes, _stream(stream)))
 
 
 def csla_indexer_scores_noalloc(cfg, st, cache, slots, B, max_len, cq, cq_dtype, W_iq, w_dtype, head_w,
-                                scores, scores_stride, stream=None):
+                                scores, scores_stride, stream=None, qs=None):
     """The indexer for callers that cannot allocate device memory: same
     inputs and outputs as csla_indexer_scores, no workspace (the library's
     fixed scratch array is used; see include/csla.h for the limit and the
     rule that overlapping calls race)."""
     return _check("csla_indexer_scores_noalloc", _lib.csla_indexer_scores_noalloc(
-        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, max_len, _ptr(cq), cq_dtype, _ptr(W_iq), w_dtype,
+        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, _ref(qs), max_len, _ptr(cq), cq_dtype, _ptr(W_iq), w_dtype,
         _ptr(head_w), _ptr(scores), scores_stride, _stream(stream)))
 
 
-def csla_topk_select(cfg, st, slots, B, max_len, scores, scores_stride, k, idx, stream=None):
+def csla_topk_select(cfg, st, slots, B, max_len, scores, scores_stride, k, idx, stream=None, qs=None):
     return _check("csla_topk_select", _lib.csla_topk_select(
-        _ref(cfg), _ref(st), _ptr(slots), B, max_len, _ptr(scores), scores_stride, k, _ptr(idx),
+        _ref(cfg), _ref(st), _ptr(slots), B, _ref(qs), max_len, _ptr(scores), scores_stride, k, _ptr(idx),
         _stream(stream)))
 
 
 def csla_csa_attend(cfg, st, cache, slots, B, q, q_dtype, idx, k, sink, gamma_q, out, out_dtype, variant,
-                    workspace, workspace_bytes, stream=None):
+                    workspace, workspace_bytes, stream=None, qs=None):
     return _check("csla_csa_attend", _lib.csla_csa_attend(
-        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, _ptr(q), q_dtype, _ptr(idx), k, _ptr(sink),
+        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, _ref(qs), _ptr(q), q_dtype, _ptr(idx), k, _ptr(sink),
         _ptr(gamma_q), _ptr(out), out_dtype, variant, _ptr(workspace), workspace_bytes, _stream(stream)))
 
 
 def csla_hca_attend(cfg, st, cache, slots, B, max_len, q, q_dtype, sink, gamma_q, out, out_dtype, variant,
-                    workspace, workspace_bytes, stream=None):
+                    workspace, workspace_bytes, stream=None, qs=None):
     return _check("csla_hca_attend", _lib.csla_hca_attend(
-        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, max_len, _ptr(q), q_dtype, _ptr(sink),
+        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, _ref(qs), max_len, _ptr(q), q_dtype, _ptr(sink),
         _ptr(gamma_q), _ptr(out), out_dtype, variant, _ptr(workspace), workspace_bytes, _stream(stream)))
 
 

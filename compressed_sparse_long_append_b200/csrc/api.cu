@@ -79,6 +79,17 @@ int nq_of(int HI) { return (3 * HI + 15) / 16 * 16; }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? CSLA_OK : CSLA_ERR_CUDA; }
 
+int row_bytes_of(const csla_cfg *c) { return (c->D - c->d_rope) + 2 * c->d_rope; }
+
+// Query rows: q_len required; a window source needs its scales and bases.
+int check_queries(const csla_queries *qs) {
+    if (!qs) return CSLA_OK;
+    if (!qs->q_len) return CSLA_ERR_ARG;
+    if (qs->win_rows && (!qs->win_scales || !qs->win_base || qs->n_win_rows < 1 || !aligned16(qs->win_rows)))
+        return CSLA_ERR_ARG;
+    return CSLA_OK;
+}
+
 // Attention workspace: the chunk partials (H*D + 2H floats per chunk).
 size_t attend_ws(const csla_cfg *c, int B, long long max_rows) {
     const size_t per = ((size_t)c->H * c->D + 2 * (size_t)c->H) * sizeof(float);
@@ -153,7 +164,7 @@ int csla_device_error(csla_stream_t stream, uint32_t *bits) {
 
 int csla_compress_append(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
                          int32_t B, int32_t T, const void *kv_new, const void *kidx_new, int32_t kv_dtype,
-                         const csla_compress_params *p, csla_stream_t stream) {
+                         const csla_compress_params *p, const csla_token_rows *tok, csla_stream_t stream) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (!st || !cache || !slots || !kv_new || !p || B < 1 || T < 1 || T > 65535) return CSLA_ERR_ARG;
@@ -164,6 +175,8 @@ int csla_compress_append(const csla_cfg *cfg, const csla_state *st, const csla_c
         return CSLA_ERR_ARG;
     if (!p->gamma_kv || !p->wg || !p->gb) return CSLA_ERR_ARG;
     if (!aligned16(st->tail_kv)) return CSLA_ERR_ARG;
+    if (tok && (!tok->rows || !tok->scales || tok->offset < 0 || (long long)tok->offset + T > tok->stride))
+        return CSLA_ERR_ARG;
     const bool csa = cfg->m == 4;
     if (csa) {
         if (cfg->dI < 4 || cfg->dI > 512 || cfg->dI % 4 || !kidx_new || !cache->kidx || !st->tail_idx || !p->wgi ||
@@ -183,11 +196,29 @@ int csla_compress_append(const csla_cfg *cfg, const csla_state *st, const csla_c
     a.rows = cache->rows; a.scales = cache->scales; a.kidx = csa ? cache->kidx : nullptr;
     a.block_table = cache->block_table; a.bt_stride = cache->bt_stride; a.n_pages = cache->n_pages;
     a.n_slots = st->n_slots;
+    if (tok) {
+        a.tok_rows = tok->rows; a.tok_scales = tok->scales; a.tok_stride = tok->stride; a.tok_offset = tok->offset;
+    }
     return cuda_status(launch_compress_append(a, kv_dtype == CSLA_BF16, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int csla_window_rows(const csla_cfg *cfg, const csla_state *st, const int32_t *slots, int32_t B, int32_t n,
+                     uint8_t *rows_out, float *scales_out, int32_t stride, csla_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (!st || !st->len || !st->win_rows || !st->win_scales || st->n_slots < 1 || !slots || !rows_out ||
+        !scales_out || B < 1 || B > 65535 || n < 1 || n > cfg->n_win || stride < n)
+        return CSLA_ERR_ARG;
+    if (!aligned16(rows_out) || !aligned16(st->win_rows)) return CSLA_ERR_ARG;
+    WindowRowsArgs a{};
+    a.slots = slots; a.len = st->len; a.B = B; a.n = n; a.n_win = cfg->n_win; a.n_slots = st->n_slots;
+    a.row_bytes = row_bytes_of(cfg); a.win_rows = st->win_rows; a.win_scales = st->win_scales;
+    a.out_rows = rows_out; a.out_scales = scales_out; a.stride = stride;
+    return cuda_status(launch_window_rows(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
-                        int32_t B, int32_t max_len, const void *cq, int32_t cq_dtype, const void *W_iq,
+                        int32_t B, const csla_queries *qs, int32_t max_len, const void *cq, int32_t cq_dtype, const void *W_iq,
                         int32_t w_dtype, const float *head_w, float *scores, int32_t scores_stride, void *workspace,
                         size_t workspace_bytes, csla_stream_t stream) {
     int rc = check_cfg(cfg);
@@ -199,7 +230,7 @@ int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_ca
         return CSLA_ERR_ARG;
     if ((cq_dtype != CSLA_F32 && cq_dtype != CSLA_BF16) || (w_dtype != CSLA_F32 && w_dtype != CSLA_BF16))
         return CSLA_ERR_ARG;
-    if (scores_stride < max_len / cfg->m) return CSLA_ERR_ARG;
+    if (scores_stride < max_len / cfg->m || check_queries(qs)) return CSLA_ERR_ARG;
     if (workspace_bytes < csla_workspace_size(cfg, CSLA_OP_INDEXER, B, max_len)) return CSLA_ERR_ARG;
     if (!aligned16(cq) || !aligned16(W_iq) || !aligned16(cache->kidx) || !aligned16(workspace)) return CSLA_ERR_ARG;
     const int NQ = nq_of(cfg->HI);
@@ -217,25 +248,28 @@ int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_ca
     a.max_len = max_len;
     a.cq = cq; a.W = W_iq; a.head_w = head_w; a.scores = scores; a.scores_stride = scores_stride;
     a.q_ws = reinterpret_cast<uint16_t *>(workspace);
+    a.q_len = qs ? qs->q_len : nullptr;
     return cuda_status(launch_indexer(a, cq_dtype == CSLA_BF16, w_dtype == CSLA_BF16, kmap, qmap, num_sms_current(),
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
-int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *slots, int32_t B, int32_t max_len,
+int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *slots, int32_t B,
+                     const csla_queries *qs, int32_t max_len,
                      const float *scores, int32_t scores_stride, int32_t k, int32_t *idx, csla_stream_t stream) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (!st || !st->len || !slots || !scores || !idx || B < 1 || max_len < 0 || k < 1 || k > 2048)
         return CSLA_ERR_ARG;
-    if (scores_stride < max_len / cfg->m) return CSLA_ERR_ARG;
+    if (scores_stride < max_len / cfg->m || check_queries(qs)) return CSLA_ERR_ARG;
     TopkArgs a{};
     a.scores = scores; a.stride = scores_stride; a.slots = slots; a.len = st->len;
     a.m = cfg->m; a.k = k; a.B = B; a.max_n = max_len / cfg->m; a.idx = idx; a.n_slots = st->n_slots;
+    a.q_len = qs ? qs->q_len : nullptr;
     return cuda_status(launch_topk(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 static int attend_common(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
-                         int32_t B, int32_t max_len, const void *q, int32_t q_dtype, const int32_t *idx, int32_t k,
+                         int32_t B, const csla_queries *qs, int32_t max_len, const void *q, int32_t q_dtype, const int32_t *idx, int32_t k,
                          const float *sink, const float *gamma_q, void *out, int32_t out_dtype, int32_t variant,
                          void *workspace, size_t workspace_bytes, csla_stream_t stream) {
     if (!st || !st->len || !st->win_rows || !st->win_scales || !cache || !cache->rows || !cache->scales ||
@@ -243,7 +277,7 @@ static int attend_common(const csla_cfg *cfg, const csla_state *st, const csla_c
         return CSLA_ERR_ARG;
     if ((q_dtype != CSLA_F32 && q_dtype != CSLA_BF16) || (out_dtype != CSLA_F32 && out_dtype != CSLA_BF16))
         return CSLA_ERR_ARG;
-    if (variant < CSLA_VARIANT_AUTO || variant > CSLA_VARIANT_STARVED) return CSLA_ERR_ARG;
+    if (variant < CSLA_VARIANT_AUTO || variant > CSLA_VARIANT_STARVED || check_queries(qs)) return CSLA_ERR_ARG;
     if (!aligned16(q) || !aligned16(cache->rows) || !aligned16(st->win_rows) || !aligned16(workspace))
         return CSLA_ERR_ARG;
     AttendArgs a{};
@@ -259,31 +293,36 @@ static int attend_common(const csla_cfg *cfg, const csla_state *st, const csla_c
     const long long max_rows = idx ? (long long)k + cfg->n_win : (long long)max_len / cfg->m + cfg->n_win;
     a.max_chunks = attend_max_chunks(max_rows);
     a.max_len = max_len;
+    if (qs) {
+        a.q_len = qs->q_len;
+        a.src_rows = qs->win_rows; a.src_scales = qs->win_scales; a.win_base = qs->win_base;
+        a.n_src = qs->n_win_rows;
+    }
     if (workspace_bytes < attend_ws(cfg, B, max_rows)) return CSLA_ERR_ARG;
     return cuda_status(launch_attend(a, q_dtype == CSLA_BF16, out_dtype == CSLA_BF16, variant, num_sms_current(),
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int csla_csa_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
-                    int32_t B, const void *q, int32_t q_dtype, const int32_t *idx, int32_t k, const float *sink,
+                    int32_t B, const csla_queries *qs, const void *q, int32_t q_dtype, const int32_t *idx, int32_t k, const float *sink,
                     const float *gamma_q, void *out, int32_t out_dtype, int32_t variant, void *workspace,
                     size_t workspace_bytes, csla_stream_t stream) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (!idx || k < 1 || k > 2048) return CSLA_ERR_ARG;
     // Without max_len the bound on the context is the int32 range.
-    return attend_common(cfg, st, cache, slots, B, 0x7FFFFFFF, q, q_dtype, idx, k, sink, gamma_q, out, out_dtype,
+    return attend_common(cfg, st, cache, slots, B, qs, 0x7FFFFFFF, q, q_dtype, idx, k, sink, gamma_q, out, out_dtype,
                          variant, workspace, workspace_bytes, stream);
 }
 
 int csla_hca_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
-                    int32_t B, int32_t max_len, const void *q, int32_t q_dtype, const float *sink,
+                    int32_t B, const csla_queries *qs, int32_t max_len, const void *q, int32_t q_dtype, const float *sink,
                     const float *gamma_q, void *out, int32_t out_dtype, int32_t variant, void *workspace,
                     size_t workspace_bytes, csla_stream_t stream) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (max_len < 1) return CSLA_ERR_ARG;
-    return attend_common(cfg, st, cache, slots, B, max_len, q, q_dtype, nullptr, 0, sink, gamma_q, out, out_dtype,
+    return attend_common(cfg, st, cache, slots, B, qs, max_len, q, q_dtype, nullptr, 0, sink, gamma_q, out, out_dtype,
                          variant, workspace, workspace_bytes, stream);
 }
 

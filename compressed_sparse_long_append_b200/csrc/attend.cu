@@ -105,19 +105,28 @@ constexpr int smem_bytes() {
 
 // Request-level facts both variants derive the same way.
 struct Req {
-    int slot, L, nv, n_cmp, win_len, n_rows, chunk, n_chunks;
+    int slot, L, nv, n_cmp, win_len, n_rows, chunk, n_chunks, wbase;
     bool ok;
 };
 __device__ __forceinline__ Req request(const AttendArgs &a, int b) {
     Req r;
     r.slot = __ldg(a.slots + b);
     const bool slot_ok = r.slot >= 0 && r.slot < a.n_slots;
-    r.L = slot_ok ? __ldg(a.len + r.slot) : 0;
+    r.L = slot_ok ? row_visible_len(a.len, a.q_len, r.slot, b) : 0;
     r.ok = slot_ok && r.L >= 1 && r.L <= a.max_len;
     if (!r.ok) r.L = 0;
     r.nv = r.L / a.m;
     r.n_cmp = a.idx ? a.k : r.nv;
     r.win_len = r.L < a.n_win ? r.L : a.n_win;
+    r.wbase = 0;
+    if (r.ok && a.src_rows) {
+        r.wbase = a.win_base[b];
+    } else if (r.ok && a.q_len && r.L - r.win_len < a.len[r.slot] - a.n_win) {
+        // an earlier query's window rows have left the ring
+        if (threadIdx.x == 0) set_dev_err(CSLA_DEVERR_INDEX);
+        r.ok = false;
+        r.L = r.nv = r.n_cmp = r.win_len = 0;
+    }
     r.n_rows = r.ok ? r.n_cmp + r.win_len : 0;
     r.chunk = attend_chunk_rows(r.n_rows);
     r.n_chunks = r.ok ? attend_num_chunks(r.n_rows) : 0;
@@ -293,6 +302,15 @@ __device__ __forceinline__ const uint8_t *row_source(const AttendArgs &a, int b,
     if (r < rq.n_rows) {
         const int w = r - rq.n_cmp;
         const int pos = rq.L - rq.win_len + w;
+        if (a.src_rows) {
+            const long long i = (long long)rq.wbase + pos;
+            if (i < 0 || i >= a.n_src) {
+                set_dev_err(CSLA_DEVERR_INDEX);
+                return nullptr;
+            }
+            *scale = __ldg(a.src_scales + i);
+            return a.src_rows + (size_t)i * rb;
+        }
         const size_t ring = (size_t)rq.slot * a.n_win + (size_t)(pos % a.n_win);
         *scale = __ldg(a.win_scales + ring);
         return a.win_rows + ring * rb;

@@ -37,11 +37,13 @@ __device__ __forceinline__ float load_act<__nv_bfloat16>(const __nv_bfloat16 *p,
     return __bfloat162float(p[i]);
 }
 
-// RMSNorm(v) * gamma, partial RoPE at `pos`, quantise into one cache row.
-// v, gam: smem [D] (v overwritten); red: smem scratch.  The rotation angles
-// are taken first so their latency overlaps the reductions.
+// RMSNorm(v) * gamma, partial RoPE at `pos`, quantise into one cache row
+// (and into a second copy `row2` when given).  v, gam: smem [D] (v
+// overwritten); red: smem scratch.  The rotation angles are taken first so
+// their latency overlaps the reductions.
 __device__ void norm_rope_quantise(float *v, const float *gam, const CompressArgs &a, long long pos, uint8_t *row,
-                                   float *scale_out, float *red) {
+                                   float *scale_out, float *red, uint8_t *row2 = nullptr,
+                                   float *scale2 = nullptr) {
     const int D = a.D, dr = a.d_rope, dn = D - dr;
     float c = 1.f, s = 0.f;
     if (threadIdx.x < dr / 2) rope_cos_sin(pos, a.freq.inv[threadIdx.x], &c, &s);
@@ -62,10 +64,20 @@ __device__ void norm_rope_quantise(float *v, const float *gam, const CompressArg
     for (int d = threadIdx.x; d < dn; d += kThreads) amax = fmaxf(amax, fabsf(v[d]));
     amax = block_max<kWarps>(amax, red);
     const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-    for (int d = threadIdx.x; d < dn; d += kThreads) row[d] = f32_to_e4m3(__fdiv_rn(v[d], scale));
-    uint16_t *rope = reinterpret_cast<uint16_t *>(row + dn);
-    for (int d = threadIdx.x; d < dr; d += kThreads) rope[d] = f32_to_bf16_bits(v[dn + d]);
-    if (threadIdx.x == 0) *scale_out = scale;
+    for (int d = threadIdx.x; d < dn; d += kThreads) {
+        const uint8_t c = f32_to_e4m3(__fdiv_rn(v[d], scale));
+        row[d] = c;
+        if (row2) row2[d] = c;
+    }
+    for (int d = threadIdx.x; d < dr; d += kThreads) {
+        const uint16_t h = f32_to_bf16_bits(v[dn + d]);
+        reinterpret_cast<uint16_t *>(row + dn)[d] = h;
+        if (row2) reinterpret_cast<uint16_t *>(row2 + dn)[d] = h;
+    }
+    if (threadIdx.x == 0) {
+        *scale_out = scale;
+        if (row2) *scale2 = scale;
+    }
 }
 
 // Four consecutive activations (16-byte or 8-byte vector load when `vec`).
@@ -223,12 +235,13 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs 
     // ---- before the wait: only this call's read-only inputs (weights and
     // the new rows), into shared memory and registers
     const bool in_window = token && x >= a.T - a.n_win;   // token stays in the ring
+    const bool emit = token && (in_window || a.tok_rows != nullptr);
     float kreg[kMaxIdxPerThread];
     if (z == 0)
         for (int d = threadIdx.x; d < D; d += kThreads) gam[d] = __ldg(a.gamma_kv + d);
     if (token) {
         const T *kv = reinterpret_cast<const T *>(a.kv_new) + ((size_t)b * a.T + x) * D;
-        if (a.T == 1 || in_window)
+        if (a.T == 1 || emit)
             for (int d = threadIdx.x; d < D; d += kThreads) v[d] = load_act<T>(kv, d);
         if (a.T == 1 && a.kidx != nullptr) {
             const T *ki = reinterpret_cast<const T *>(a.kidx_new) + (size_t)b * a.dI;
@@ -271,9 +284,20 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs 
             }
         }
         CSLA_TL_MARK(1);
-        if (!in_window) return;
-        const size_t ring = (size_t)slot * a.n_win + (size_t)(pos % a.n_win);
-        norm_rope_quantise(v, gam, a, pos, a.win_rows + ring * rb, a.win_scales + ring, red);
+        if (!emit) return;
+        uint8_t *trow = nullptr;
+        float *tscale = nullptr;
+        if (a.tok_rows) {
+            const size_t t = (size_t)b * a.tok_stride + a.tok_offset + x;
+            trow = a.tok_rows + t * rb;
+            tscale = a.tok_scales + t;
+        }
+        if (in_window) {
+            const size_t ring = (size_t)slot * a.n_win + (size_t)(pos % a.n_win);
+            norm_rope_quantise(v, gam, a, pos, a.win_rows + ring * rb, a.win_scales + ring, red, trow, tscale);
+        } else {
+            norm_rope_quantise(v, gam, a, pos, trow, tscale, red);
+        }
         CSLA_TL_MARK(2);
         return;
     }
@@ -346,6 +370,37 @@ __global__ void __launch_bounds__(kThreads) tail_update_kernel(CompressArgs a) {
 }
 
 }  // namespace
+
+// Row i of request b = ring row of position len - n + i (a zero row with
+// scale 0 where that position is negative).  One CTA per row.
+constexpr int kWinThreads = 64;
+__global__ void __launch_bounds__(kWinThreads) window_rows_kernel(WindowRowsArgs a) {
+    pdl_trigger();
+    const int i = blockIdx.x, b = blockIdx.y;
+    const int slot = __ldg(a.slots + b);
+    uint4 *dst = reinterpret_cast<uint4 *>(a.out_rows + ((size_t)b * a.stride + i) * a.row_bytes);
+    float *dscale = a.out_scales + (size_t)b * a.stride + i;
+    const int nq = a.row_bytes / 16;
+    pdl_wait();
+    if (slot < 0 || slot >= a.n_slots) {
+        if (threadIdx.x == 0 && i == 0) set_dev_err(CSLA_DEVERR_INDEX);
+        return;
+    }
+    const long long pos = (long long)a.len[slot] - a.n + i;
+    if (pos < 0) {
+        for (int q = threadIdx.x; q < nq; q += kWinThreads) dst[q] = make_uint4(0u, 0u, 0u, 0u);
+        if (threadIdx.x == 0) *dscale = 0.f;
+        return;
+    }
+    const size_t ring = (size_t)slot * a.n_win + (size_t)(pos % a.n_win);
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.win_rows + ring * a.row_bytes);
+    for (int q = threadIdx.x; q < nq; q += kWinThreads) dst[q] = src[q];
+    if (threadIdx.x == 0) *dscale = a.win_scales[ring];
+}
+
+cudaError_t launch_window_rows(const WindowRowsArgs &a, cudaStream_t stream) {
+    return launch_pdl(window_rows_kernel, dim3(a.n, a.B), dim3(kWinThreads), 0, stream, a);
+}
 
 cudaError_t launch_compress_append(const CompressArgs &a, bool bf16, cudaStream_t stream) {
     const int nb = a.T / a.m + 1;   // blocks one call can complete

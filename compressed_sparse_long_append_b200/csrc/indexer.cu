@@ -267,8 +267,8 @@ __global__ void __launch_bounds__(kIdxThreads)
     pdl_wait();
     CSLA_TL_WAITED();
 
-    const int L = slot_ok ? a.len[slot] : 0;
-    const bool ok = slot_ok && L <= a.max_len;
+    const int L = slot_ok ? row_visible_len(a.len, a.q_len, slot, b) : 0;
+    const bool ok = slot_ok && L >= 0 && L <= a.max_len;
     if (!ok && threadIdx.x == 0 && blockIdx.x == 0) set_dev_err(slot_ok ? CSLA_DEVERR_LEN : CSLA_DEVERR_INDEX);
     const int nv = ok ? L / a.m : 0;
     const int n_tiles = ok ? min(kTPC, (nv + kTileE - 1) / kTileE - t_begin) : 0;

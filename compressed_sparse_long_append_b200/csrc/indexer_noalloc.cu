@@ -51,7 +51,8 @@ void *scratch_address(int *status) {
 }  // namespace
 
 extern "C" int csla_indexer_scores_noalloc(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
-                                           const int32_t *slots, int32_t B, int32_t max_len, const void *cq,
+                                           const int32_t *slots, int32_t B, const csla_queries *qs,
+                                           int32_t max_len, const void *cq,
                                            int32_t cq_dtype, const void *W_iq, int32_t w_dtype,
                                            const float *head_w, float *scores, int32_t scores_stride,
                                            csla_stream_t stream) {
@@ -62,6 +63,6 @@ extern "C" int csla_indexer_scores_noalloc(const csla_cfg *cfg, const csla_state
     int status = CSLA_OK;
     void *ws = scratch_address(&status);
     if (!ws) return status;
-    return csla_indexer_scores(cfg, st, cache, slots, B, max_len, cq, cq_dtype, W_iq, w_dtype, head_w, scores,
+    return csla_indexer_scores(cfg, st, cache, slots, B, qs, max_len, cq, cq_dtype, W_iq, w_dtype, head_w, scores,
                                scores_stride, ws, kScratchBytes, stream);
 }

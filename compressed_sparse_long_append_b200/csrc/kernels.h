@@ -54,8 +54,24 @@ struct CompressArgs {
     uint16_t *kidx;
     const int32_t *block_table;
     int bt_stride, n_pages, n_slots;
+    uint8_t *tok_rows;    // optional: window-format row of every new token
+    float *tok_scales;    //   token i of request b -> row b * tok_stride + tok_offset + i
+    int tok_stride, tok_offset;
 };
 cudaError_t launch_compress_append(const CompressArgs &a, bool bf16, cudaStream_t stream);
+
+// Ring rows of the last n positions of each request, in position order.
+struct WindowRowsArgs {
+    const int32_t *slots;
+    const int32_t *len;
+    int B, n, n_win, n_slots, row_bytes;
+    const uint8_t *win_rows;
+    const float *win_scales;
+    uint8_t *out_rows;
+    float *out_scales;
+    int stride;
+};
+cudaError_t launch_window_rows(const WindowRowsArgs &a, cudaStream_t stream);
 
 // Lightning indexer.  NQ = rows of the bf16 query operand (hi, mid and lo
 // terms of every head, zero padding to a multiple of 16).
@@ -71,6 +87,7 @@ struct IndexerArgs {
     float *scores;
     int scores_stride;
     uint16_t *q_ws;     // [B][NQ][dI] bf16
+    const int32_t *q_len;   // optional per-row visible length (else len[slot])
 };
 cudaError_t launch_indexer(const IndexerArgs &a, bool cq_bf16, bool w_bf16, const CUtensorMap &kmap,
                            const CUtensorMap &qmap, int num_sms, cudaStream_t stream);
@@ -82,6 +99,7 @@ struct TopkArgs {
     const int32_t *len;
     int m, k, B, max_n, n_slots;
     int32_t *idx;
+    const int32_t *q_len;   // optional per-row visible length (else len[slot])
 };
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream);
 
@@ -108,7 +126,21 @@ struct AttendArgs {
     float *part;          // workspace: chunk partials
     int max_chunks;
     int max_len;
+    const int32_t *q_len;         // optional per-row visible length (else len[slot])
+    const uint8_t *src_rows;      // optional window rows by position:
+    const float *src_scales;      //   position p of row b is src row win_base[b] + p
+    const int32_t *win_base;
+    int n_src;
 };
+
+// Visible length of query row b: q_len[b] when given (1 <= q_len[b] <=
+// len[slot]), else len[slot].  Returns -1 for a q_len outside that range.
+__device__ __forceinline__ int row_visible_len(const int32_t *len, const int32_t *q_len, int slot, int b) {
+    const int L = len[slot];
+    if (!q_len) return L;
+    const int lq = q_len[b];
+    return (lq >= 1 && lq <= L) ? lq : -1;
+}
 cudaError_t launch_attend(const AttendArgs &a, bool q_bf16, bool out_bf16, int variant, int num_sms,
                           cudaStream_t stream);
 

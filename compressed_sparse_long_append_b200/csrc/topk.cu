@@ -102,9 +102,9 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
     hist_zero(hist);
     pdl_wait();
     CSLA_TL_WAITED();
-    const int L = slot_ok ? a.len[slot] : 0;
-    int n = L / a.m;
-    if (!slot_ok || L / a.m > a.max_n) {
+    const int L = slot_ok ? row_visible_len(a.len, a.q_len, slot, b) : 0;
+    int n = L < 0 ? 0 : L / a.m;
+    if (!slot_ok || L < 0 || L / a.m > a.max_n) {
         if (threadIdx.x == 0) set_dev_err(CSLA_DEVERR_LEN);
         n = 0;
     }
@@ -391,9 +391,9 @@ __global__ void __launch_bounds__(kRThreads, 1) topk_reg_kernel(TopkArgs a) {
     const bool slot_ok = slot >= 0 && slot < a.n_slots;
     pdl_wait();
     CSLA_TL_WAITED();
-    const int L = slot_ok ? a.len[slot] : 0;
-    int n = L / a.m;
-    if (!slot_ok || L / a.m > a.max_n) {
+    const int L = slot_ok ? row_visible_len(a.len, a.q_len, slot, b) : 0;
+    int n = L < 0 ? 0 : L / a.m;
+    if (!slot_ok || L < 0 || L / a.m > a.max_n) {
         if (threadIdx.x == 0) set_dev_err(CSLA_DEVERR_LEN);
         n = 0;
     }
@@ -607,9 +607,9 @@ __global__ void __cluster_dims__(kG, 1, 1) __launch_bounds__(kRThreads, 1) topk_
     const bool slot_ok = slot >= 0 && slot < a.n_slots;
     pdl_wait();
     CSLA_TL_WAITED();
-    const int L = slot_ok ? a.len[slot] : 0;
-    int n = L / a.m;
-    if (!slot_ok || L / a.m > a.max_n) {
+    const int L = slot_ok ? row_visible_len(a.len, a.q_len, slot, b) : 0;
+    int n = L < 0 ? 0 : L / a.m;
+    if (!slot_ok || L < 0 || L / a.m > a.max_n) {
         if (threadIdx.x == 0 && cr == 0) set_dev_err(CSLA_DEVERR_LEN);
         n = 0;
     }

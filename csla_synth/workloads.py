@@ -40,6 +40,10 @@ CSA_TINY = Workload("csa_decode_tiny_L2048", B=1, L=2048, m=4, H=8, D=128, HI=4,
 CSA_DECODE = Workload("csa_decode_B8_L131072", B=8, L=131072, m=4, H=64, D=512, HI=16, dI=128,
                       dc=1024, k=512, seed=1)
 HCA_DECODE = Workload("hca_decode_B4_L1048576", B=4, L=1048576, m=128, H=64, D=512, seed=2)
+# prefill chunk: T = 4096 new tokens (and queries) after a 262144-token prefix,
+# so the last query sees 66560 compressed entries; B counts queries here
+CSA_PREFILL = Workload("csa_prefill_T4096_L262144", B=4096, L=262144 + 4096, m=4, H=64, D=512, HI=16,
+                       dI=128, dc=1024, k=1024, seed=4)
 
 
 def _act(w: Workload, name, shape, std=1.0, start=0):
@@ -88,4 +92,13 @@ def step_inputs(w: Workload, step):
         out["cq"] = _act(w, "cq/%d" % step, (w.B, w.dc))
         out["head_w"] = normal(w.seed, "head_w/%d" % step, (w.B, w.HI)).astype(np.float32) \
             .astype(np.float64)
+    return out
+
+
+def prefill_inputs(w: Workload, T, tag=0):
+    """Query-side inputs of T prefill queries (one per new token)."""
+    out = {"q": _act(w, "pq/%d" % tag, (T, w.H, w.D))}
+    if w.is_csa:
+        out["cq"] = _act(w, "pcq/%d" % tag, (T, w.dc))
+        out["head_w"] = normal(w.seed, "phw/%d" % tag, (T, w.HI)).astype(np.float32).astype(np.float64)
     return out

@@ -32,7 +32,8 @@
  *     the offending work, records a bit in the library's device error word
  *     and carries on; csla_device_error() reads and clears it.
  *   - A batch is `B` requests given by `slots` (device int32[B], distinct
- *     state-cache slot ids).  Context length of request b after the call is
+ *     state-cache slot ids; query rows passed with a csla_queries may share
+ *     a slot).  Context length of request b after the call is
  *     st->len[slots[b]].  `max_len` (host) is an upper bound on it, used to
  *     size grids.
  *
@@ -136,6 +137,47 @@ typedef struct csla_compress_params {
 } csla_compress_params;
 
 /*
+ * Query rows other than each request's latest token (a prefill chunk's
+ * queries; several recent positions of one request).  Calls that take a
+ * `const csla_queries *qs` treat NULL as plain decode: row b is request
+ * slots[b] at its latest position len-1.  With qs:
+ *   q_len [B] int32 (device): row b's visible length.  Its query sits at
+ *     position q_len[b]-1 and sees what a decode step at that position sees
+ *     (haiqwa §百万 token 怎么切分, causal visibility of compressed blocks:
+ *     entry e is visible iff (e+1)*m <= q_len[b]; window = the last
+ *     min(n_win, q_len[b]) positions before it, inclusive).  Requires
+ *     1 <= q_len[b] <= len[slots[b]]: the cache already holds those tokens.
+ *     A row outside that range sets CSLA_DEVERR_LEN and is skipped.
+ *   win_rows / win_scales / win_base / n_win_rows: where the attention calls
+ *     read window rows.  win_rows NULL: from the ring, so each row's window
+ *     positions must still be there (q_len[b] - min(q_len[b], n_win) >=
+ *     len - n_win, else CSLA_DEVERR_INDEX and the row is skipped).  Else
+ *     position p of row b is row win_base[b] + p of win_rows
+ *     [n_win_rows][row_bytes] (16-byte aligned) with scale win_scales[...];
+ *     a position outside [0, n_win_rows) sets CSLA_DEVERR_INDEX and the row
+ *     is masked.  csla_window_rows and the token-row output of
+ *     csla_compress_append fill such a buffer for a prefill chunk.
+ * The indexer and top-k read q_len only.
+ */
+typedef struct csla_queries {
+    const int32_t *q_len;
+    const uint8_t *win_rows;
+    const float *win_scales;
+    const int32_t *win_base;
+    int32_t n_win_rows;
+} csla_queries;
+
+/* Optional output of csla_compress_append: the window-format row (the one
+ * the ring receives) of every new token, kept for later queries of a prefill
+ * chunk.  New token i of request b goes to row b*stride + offset + i. */
+typedef struct csla_token_rows {
+    uint8_t *rows;       /* [B*stride][row_bytes] */
+    float *scales;       /* [B*stride] */
+    int32_t stride;      /* rows per request, >= offset + T */
+    int32_t offset;      /* row of the call's first new token, >= 0 */
+} csla_token_rows;
+
+/*
  * csla_compress_append -- state-cache and classical-cache update
  * (硅星人 §两大压缩注意力, CSA/HCA compressor and cache paragraphs; haiqwa
  * §Partial RoPE位置编码 sliding window; §RMSNorm归一化).
@@ -155,13 +197,29 @@ typedef struct csla_compress_params {
  * vector loads).  gamma_kv, wg, gb, wgi, gbi are read before the kernel
  * waits on the grid launched before it on the stream (programmatic
  * dependent launch); write them no later than the kernel before that one.
+ * tok: NULL, or where the window-format row of every new token also goes
+ * (csla_token_rows; the ring keeps only the last n_win).
  * Errors: CSLA_ERR_ARG on null/bad sizes or misaligned tails;
  * CSLA_ERR_UNSUPPORTED on shapes.
  */
 int csla_compress_append(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
                          const int32_t *slots, int32_t B, int32_t T, const void *kv_new,
                          const void *kidx_new, int32_t kv_dtype, const csla_compress_params *p,
-                         csla_stream_t stream);
+                         const csla_token_rows *tok, csla_stream_t stream);
+
+/*
+ * csla_window_rows -- copy of the ring rows of each request's last n
+ * positions, in position order: row b*stride + i = the row of position
+ * len - n + i (a zero row with scale 0 where that position is negative).
+ * 1 <= n <= n_win.  With the token-row output of csla_compress_append this
+ * gives a prefill chunk's queries every window row they need: take the
+ * n_win-1 rows before the chunk here, then append the chunk.
+ * rows_out 16-byte aligned.  Errors: CSLA_ERR_ARG; CSLA_DEVERR_INDEX for a
+ * slot outside [0, n_slots).
+ */
+int csla_window_rows(const csla_cfg *cfg, const csla_state *st, const int32_t *slots, int32_t B,
+                     int32_t n, uint8_t *rows_out, float *scales_out, int32_t stride,
+                     csla_stream_t stream);
 
 /*
  * csla_indexer_scores -- lightning indexer (硅星人 §两大压缩注意力, CSA part:
@@ -177,7 +235,7 @@ int csla_compress_append(const csla_cfg *cfg, const csla_state *st, const csla_c
  * workspace: csla_workspace_size(cfg, CSLA_OP_INDEXER, B, max_len) bytes.
  */
 int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
-                        const int32_t *slots, int32_t B, int32_t max_len, const void *cq,
+                        const int32_t *slots, int32_t B, const csla_queries *qs, int32_t max_len, const void *cq,
                         int32_t cq_dtype, const void *W_iq, int32_t w_dtype, const float *head_w,
                         float *scores, int32_t scores_stride, void *workspace,
                         size_t workspace_bytes, csla_stream_t stream);
@@ -190,7 +248,7 @@ int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_ca
  * (-0.0 counts as +0.0).  scores as produced by csla_indexer_scores.
  */
 int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *slots, int32_t B,
-                     int32_t max_len, const float *scores, int32_t scores_stride, int32_t k,
+                     const csla_queries *qs, int32_t max_len, const float *scores, int32_t scores_stride, int32_t k,
                      int32_t *idx, csla_stream_t stream);
 
 /*
@@ -211,7 +269,7 @@ int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *s
  *   max_len here meaning k (the set size is k + n_win).
  */
 int csla_csa_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
-                    const int32_t *slots, int32_t B, const void *q, int32_t q_dtype,
+                    const int32_t *slots, int32_t B, const csla_queries *qs, const void *q, int32_t q_dtype,
                     const int32_t *idx, int32_t k, const float *sink, const float *gamma_q,
                     void *out, int32_t out_dtype, int32_t variant, void *workspace,
                     size_t workspace_bytes, csla_stream_t stream);
@@ -223,7 +281,7 @@ int csla_csa_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache 
  * workspace: csla_workspace_size(cfg, CSLA_OP_HCA_ATTEND, B, max_len).
  */
 int csla_hca_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
-                    const int32_t *slots, int32_t B, int32_t max_len, const void *q,
+                    const int32_t *slots, int32_t B, const csla_queries *qs, int32_t max_len, const void *q,
                     int32_t q_dtype, const float *sink, const float *gamma_q, void *out,
                     int32_t out_dtype, int32_t variant, void *workspace, size_t workspace_bytes,
                     csla_stream_t stream);
@@ -249,7 +307,8 @@ int csla_hca_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache 
  */
 #define CSLA_NOALLOC_INDEXER_SCRATCH_BYTES 786432
 int csla_indexer_scores_noalloc(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
-                                const int32_t *slots, int32_t B, int32_t max_len, const void *cq,
+                                const int32_t *slots, int32_t B, const csla_queries *qs,
+                                int32_t max_len, const void *cq,
                                 int32_t cq_dtype, const void *W_iq, int32_t w_dtype,
                                 const float *head_w, float *scores, int32_t scores_stride,
                                 csla_stream_t stream);

@@ -133,3 +133,27 @@ def assert_bf16_close(got_bits, ref_bits, abs_tol):
     ulp = np.exp2(np.floor(np.log2(np.maximum(mag, 1e-38))) - 7)
     bad = np.nonzero(np.abs(g - r) > ulp + abs_tol)[0]
     assert len(bad) == 0, [(int(i), g[i], r[i]) for i in bad[:8]]
+
+
+MAX_ABS = 1e-2        # attention: the contract's bound for O(1) outputs
+REL_RMS = 2e-2        # attention: derived bound, error / RMS(output) (f16/bf16 q and P operands)
+REL_TOL = 1e-3        # indexer scores, relative to max(|oracle|, 1e-3 * row max)
+
+
+def check_out(got, ref):
+    """Attention output of one request against the oracle's fp64 result."""
+    err = np.abs(got - ref)
+    rms = np.sqrt(np.mean(ref * ref))
+    assert np.all(np.isfinite(got))
+    assert err.max() <= MAX_ABS, err.max()
+    assert err.max() <= REL_RMS * rms, (err.max(), rms)
+    return err.max()
+
+
+def check_scores(got, ref):
+    """Indexer scores of one request against the oracle's fp64 scores."""
+    floor = 1e-3 * max(np.max(np.abs(ref)), 1e-30)
+    err = np.abs(got - ref) / np.maximum(np.abs(ref), floor)
+    assert np.all(np.isfinite(got))
+    assert err.max() <= REL_TOL, err.max()
+    return err.max()

@@ -56,13 +56,24 @@ def test_host_argument_checks():
     L = C._lib
     cfg = _cfg(m=4)
     # null structs / pointers -> CSLA_ERR_ARG, no launch
-    assert L.csla_compress_append(ctypes.byref(cfg), None, None, None, 1, 1, None, None, 0, None, None) == C.CSLA_ERR_ARG
-    assert L.csla_topk_select(ctypes.byref(cfg), None, None, 1, 10, None, 10, 5, None, None) == C.CSLA_ERR_ARG
-    assert L.csla_hca_attend(ctypes.byref(_cfg(m=128)), None, None, None, 1, 100, None, 0, None, None, None, 0,
-                             0, None, 0, None) == C.CSLA_ERR_ARG
+    assert L.csla_compress_append(ctypes.byref(cfg), None, None, None, 1, 1, None, None, 0, None, None,
+                                  None) == C.CSLA_ERR_ARG
+    assert L.csla_topk_select(ctypes.byref(cfg), None, None, 1, None, 10, None, 10, 5, None, None) == C.CSLA_ERR_ARG
+    assert L.csla_hca_attend(ctypes.byref(_cfg(m=128)), None, None, None, 1, None, 100, None, 0, None, None, None,
+                             0, 0, None, 0, None) == C.CSLA_ERR_ARG
+    assert L.csla_window_rows(ctypes.byref(cfg), None, None, 1, 127, None, None, 127, None) == C.CSLA_ERR_ARG
+    # query rows without q_len, or a window source without its bases -> CSLA_ERR_ARG before any launch
+    fake = 1 << 40   # never dereferenced: the host check fails first
+    st = C.csla_state(fake, fake, fake, fake, fake, 4)
+    no_len = C.csla_queries(None, None, None, None, 0)
+    assert L.csla_topk_select(ctypes.byref(cfg), ctypes.byref(st), fake, 1, ctypes.byref(no_len), 10, fake, 10, 5,
+                              fake, None) == C.CSLA_ERR_ARG
+    no_base = C.csla_queries(fake, fake, fake, None, 10)
+    assert L.csla_topk_select(ctypes.byref(cfg), ctypes.byref(st), fake, 1, ctypes.byref(no_base), 10, fake, 10, 5,
+                              fake, None) == C.CSLA_ERR_ARG
     # unsupported shapes
     for bad in (dict(m=8), dict(m=4, D=256), dict(m=4, d_rope=32), dict(m=4, H=65), dict(m=4, n_win=64)):
-        assert L.csla_topk_select(ctypes.byref(_cfg(**bad)), None, None, 1, 10, None, 10, 5, None, None) \
+        assert L.csla_topk_select(ctypes.byref(_cfg(**bad)), None, None, 1, None, 10, None, 10, 5, None, None) \
             == C.CSLA_ERR_UNSUPPORTED, bad
     assert L.csla_strerror(C.CSLA_ERR_DEVICE) == b"device-side input error"
 

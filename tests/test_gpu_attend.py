@@ -11,13 +11,11 @@ import oracle
 from compressed_sparse_long_append_b200 import csla as C
 from compressed_sparse_long_append_b200.layer import LayerBuffers, LayerShape
 from csla_synth.workloads import CSA_DECODE, CSA_TINY, HCA_DECODE, layer_params, step_inputs
-from gpu_helpers import DEV, act_tensor, assert_no_device_error, upload_layer
+from gpu_helpers import DEV, act_tensor, assert_no_device_error, check_out, upload_layer
 from helpers import oracle_cache
 
 pytestmark = pytest.mark.gpu
 
-MAX_ABS = 1e-2        # the contract's bound for O(1) outputs
-REL_RMS = 2e-2        # derived bound: error / RMS(output) (f16/bf16 q and P operands)
 
 
 def attend(w, lb, q, sink, gamma_q, lens, idx=None, variant=C.CSLA_VARIANT_AUTO, slots=None,
@@ -41,15 +39,6 @@ def attend(w, lb, q, sink, gamma_q, lens, idx=None, variant=C.CSLA_VARIANT_AUTO,
         C.csla_hca_attend(cfg, lb.state(), lb.cache(), slots, B, ml, q, qdt, sink, gamma_q, out, odt, variant,
                           ws, wsb)
     return out
-
-
-def check_out(got, ref):
-    err = np.abs(got - ref)
-    rms = np.sqrt(np.mean(ref * ref))
-    assert np.all(np.isfinite(got))
-    assert err.max() <= MAX_ABS, err.max()
-    assert err.max() <= REL_RMS * rms, (err.max(), rms)
-    return err.max()
 
 
 def _dev(x):

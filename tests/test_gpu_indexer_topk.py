@@ -12,12 +12,11 @@ import oracle
 from compressed_sparse_long_append_b200 import csla as C
 from csla_synth import normal, integers
 from csla_synth.workloads import CSA_DECODE, CSA_TINY, layer_params, step_inputs
-from gpu_helpers import DEV, act_tensor, assert_no_device_error, upload_layer
+from gpu_helpers import DEV, act_tensor, assert_no_device_error, check_scores, upload_layer
 from helpers import oracle_cache
 
 pytestmark = pytest.mark.gpu
 
-REL_TOL = 1e-3          # indexer scores, relative
 GAP_TOL = 1e-4          # top-k ambiguity band
 
 
@@ -41,14 +40,6 @@ def oracle_scores(w, cv, s, L, si, p):
     nv = L // w.m
     qI = oracle.index_query(si["cq"][s], p["W_iq"], w.HI, w.dI)
     return oracle.index_scores(qI, si["head_w"][s], cv.gather_keys(s, nv))
-
-
-def check_scores(got, ref):
-    floor = 1e-3 * max(np.max(np.abs(ref)), 1e-30)
-    err = np.abs(got - ref) / np.maximum(np.abs(ref), floor)
-    assert np.all(np.isfinite(got))
-    assert err.max() <= REL_TOL, err.max()
-    return err.max()
 
 
 @pytest.mark.parametrize("w,lens", [

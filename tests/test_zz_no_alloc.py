@@ -73,6 +73,6 @@ def test_noalloc_rejects_batches_beyond_its_scratch():
     dummy = torch.zeros(16, dtype=torch.float32, device=DEV)
     rc = C._lib.csla_indexer_scores_noalloc(
         C.ctypes.byref(lb.cfg()), C.ctypes.byref(lb.state()), C.ctypes.byref(lb.cache()), dummy.data_ptr(),
-        too_many, 600, dummy.data_ptr(), C.CSLA_BF16, dummy.data_ptr(), C.CSLA_BF16, dummy.data_ptr(),
+        too_many, None, 600, dummy.data_ptr(), C.CSLA_BF16, dummy.data_ptr(), C.CSLA_BF16, dummy.data_ptr(),
         dummy.data_ptr(), 150, torch.cuda.current_stream().cuda_stream)
     assert rc == C.CSLA_ERR_ARG
