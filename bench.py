@@ -306,7 +306,7 @@ class PrefillStep:
         self.bufsc = torch.zeros(NW + T, dtype=torch.float32, device=device)
         self.q_len = torch.arange(L0 + 1, L1 + 1, dtype=torch.int32, device=device)
         self.base = torch.full((T,), NW - L0, dtype=torch.int32, device=device)
-        self.qs_rows = C.queries(self.q_len)
+        self.qs_rows = C.queries(self.q_len, one_request=True)
         self.qs_att = C.queries(self.q_len, self.buf, self.bufsc, self.base, NW + T)
         self.tok = C.token_rows(self.buf, self.bufsc, NW + T, NW)
         self.scores = torch.zeros((T, self.stride), dtype=torch.float32, device=device)

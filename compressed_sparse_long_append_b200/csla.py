@@ -51,7 +51,7 @@ class csla_compress_params(ctypes.Structure):
 class csla_queries(ctypes.Structure):
     """Query rows other than each request's latest token (see include/csla.h)."""
     _fields_ = [("q_len", ctypes.c_void_p), ("win_rows", ctypes.c_void_p), ("win_scales", ctypes.c_void_p),
-                ("win_base", ctypes.c_void_p), ("n_win_rows", ctypes.c_int32)]
+                ("win_base", ctypes.c_void_p), ("n_win_rows", ctypes.c_int32), ("one_request", ctypes.c_int32)]
 
 
 class csla_token_rows(ctypes.Structure):
@@ -59,10 +59,11 @@ class csla_token_rows(ctypes.Structure):
                 ("offset", ctypes.c_int32)]
 
 
-def queries(q_len, win_rows=None, win_scales=None, win_base=None, n_win_rows=0):
+def queries(q_len, win_rows=None, win_scales=None, win_base=None, n_win_rows=0, one_request=False):
     """csla_queries from tensors (or device addresses); the struct keeps the
     tensors alive for as long as it lives."""
-    q = csla_queries(_ptr(q_len), _ptr(win_rows), _ptr(win_scales), _ptr(win_base), int(n_win_rows))
+    q = csla_queries(_ptr(q_len), _ptr(win_rows), _ptr(win_scales), _ptr(win_base), int(n_win_rows),
+                     1 if one_request else 0)
     q._keep = (q_len, win_rows, win_scales, win_base)
     return q
 

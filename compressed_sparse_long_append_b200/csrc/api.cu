@@ -237,7 +237,9 @@ int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_ca
     CUtensorMap kmap, qmap;
     if (!encode_bf16_2d(&kmap, cache->kidx, (uint64_t)cfg->dI, (uint64_t)cache->n_pages * 32, 32))
         return CSLA_ERR_CUDA;
-    if (!encode_bf16_2d(&qmap, workspace, (uint64_t)cfg->dI, (uint64_t)B * NQ, (uint32_t)NQ)) return CSLA_ERR_CUDA;
+    const int G = (qs && qs->one_request) ? indexer_rows_per_cta(NQ) : 1;
+    if (!encode_bf16_2d(&qmap, workspace, (uint64_t)cfg->dI, (uint64_t)B * NQ, (uint32_t)(G * NQ)))
+        return CSLA_ERR_CUDA;
     IndexerArgs a{};
     a.m = cfg->m; a.HI = cfg->HI; a.dI = cfg->dI; a.dc = cfg->dc; a.NQ = NQ;
     a.slots = slots; a.len = st->len; a.block_table = cache->block_table; a.bt_stride = cache->bt_stride;
@@ -249,6 +251,7 @@ int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_ca
     a.cq = cq; a.W = W_iq; a.head_w = head_w; a.scores = scores; a.scores_stride = scores_stride;
     a.q_ws = reinterpret_cast<uint16_t *>(workspace);
     a.q_len = qs ? qs->q_len : nullptr;
+    a.rows_per_cta = G;
     return cuda_status(launch_indexer(a, cq_dtype == CSLA_BF16, w_dtype == CSLA_BF16, kmap, qmap, num_sms_current(),
                                       reinterpret_cast<cudaStream_t>(stream)));
 }

@@ -38,9 +38,10 @@ __device__ __forceinline__ float load_act<__nv_bfloat16>(const __nv_bfloat16 *p,
 }
 
 // RMSNorm(v) * gamma, partial RoPE at `pos`, quantise into one cache row
-// (and into a second copy `row2` when given).  v, gam: smem [D] (v
-// overwritten); red: smem scratch.  The rotation angles are taken first so
-// their latency overlaps the reductions.
+// (kTwo: also into a second copy `row2`, when not null).  v, gam: smem [D]
+// (v overwritten); red: smem scratch.  The rotation angles are taken first
+// so their latency overlaps the reductions.
+template <bool kTwo = false>
 __device__ void norm_rope_quantise(float *v, const float *gam, const CompressArgs &a, long long pos, uint8_t *row,
                                    float *scale_out, float *red, uint8_t *row2 = nullptr,
                                    float *scale2 = nullptr) {
@@ -67,16 +68,16 @@ __device__ void norm_rope_quantise(float *v, const float *gam, const CompressArg
     for (int d = threadIdx.x; d < dn; d += kThreads) {
         const uint8_t c = f32_to_e4m3(__fdiv_rn(v[d], scale));
         row[d] = c;
-        if (row2) row2[d] = c;
+        if (kTwo && row2) row2[d] = c;
     }
     for (int d = threadIdx.x; d < dr; d += kThreads) {
         const uint16_t h = f32_to_bf16_bits(v[dn + d]);
         reinterpret_cast<uint16_t *>(row + dn)[d] = h;
-        if (row2) reinterpret_cast<uint16_t *>(row2 + dn)[d] = h;
+        if (kTwo && row2) reinterpret_cast<uint16_t *>(row2 + dn)[d] = h;
     }
     if (threadIdx.x == 0) {
         *scale_out = scale;
-        if (row2) *scale2 = scale;
+        if (kTwo && row2) *scale2 = scale;
     }
 }
 
@@ -208,7 +209,8 @@ __device__ void pool_block(const BlockRows<T> &x, int m, const float *wsm, float
     __syncthreads();
 }
 
-template <typename T>
+// kTok: the call also keeps every new token's window row (CompressArgs::tok_rows).
+template <typename T, bool kTok>
 __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs a) {
     CSLA_TL_SCOPE(kTlCompress);
     extern __shared__ __align__(16) float sm[];
@@ -235,7 +237,7 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs 
     // ---- before the wait: only this call's read-only inputs (weights and
     // the new rows), into shared memory and registers
     const bool in_window = token && x >= a.T - a.n_win;   // token stays in the ring
-    const bool emit = token && (in_window || a.tok_rows != nullptr);
+    const bool emit = token && (in_window || kTok);
     float kreg[kMaxIdxPerThread];
     if (z == 0)
         for (int d = threadIdx.x; d < D; d += kThreads) gam[d] = __ldg(a.gamma_kv + d);
@@ -285,18 +287,18 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs 
         }
         CSLA_TL_MARK(1);
         if (!emit) return;
-        uint8_t *trow = nullptr;
-        float *tscale = nullptr;
-        if (a.tok_rows) {
+        const size_t ring = (size_t)slot * a.n_win + (size_t)(pos % a.n_win);
+        if constexpr (kTok) {
             const size_t t = (size_t)b * a.tok_stride + a.tok_offset + x;
-            trow = a.tok_rows + t * rb;
-            tscale = a.tok_scales + t;
-        }
-        if (in_window) {
-            const size_t ring = (size_t)slot * a.n_win + (size_t)(pos % a.n_win);
-            norm_rope_quantise(v, gam, a, pos, a.win_rows + ring * rb, a.win_scales + ring, red, trow, tscale);
+            uint8_t *trow = a.tok_rows + t * rb;
+            float *tscale = a.tok_scales + t;
+            if (in_window)
+                norm_rope_quantise<true>(v, gam, a, pos, a.win_rows + ring * rb, a.win_scales + ring, red, trow,
+                                         tscale);
+            else
+                norm_rope_quantise(v, gam, a, pos, trow, tscale, red);
         } else {
-            norm_rope_quantise(v, gam, a, pos, trow, tscale, red);
+            norm_rope_quantise(v, gam, a, pos, a.win_rows + ring * rb, a.win_scales + ring, red);
         }
         CSLA_TL_MARK(2);
         return;
@@ -413,17 +415,23 @@ cudaError_t launch_compress_append(const CompressArgs &a, bool bf16, cudaStream_
     if (configured_dev != dev) {
         // largest case: W = 512, m = 128
         const int most = (int)((2 * 512 + 512 + 128 + 4 * kThreads + 32 + kStageRows * 512) * sizeof(float));
-        cudaError_t e = cudaFuncSetAttribute(compress_append_kernel<float>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, most);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(compress_append_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 most);
-        if (e != cudaSuccess) return e;
+        cudaError_t e = cudaSuccess;
+        for (auto fn : {compress_append_kernel<float, false>, compress_append_kernel<float, true>,
+                        compress_append_kernel<__nv_bfloat16, false>, compress_append_kernel<__nv_bfloat16, true>}) {
+            e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+            if (e != cudaSuccess) return e;
+        }
         configured_dev = dev;
     }
     const dim3 grid(a.T + nb, a.B, a.kidx ? 2 : 1);
-    cudaError_t e = bf16 ? launch_pdl(compress_append_kernel<__nv_bfloat16>, grid, dim3(kThreads), smem, stream, a)
-                         : launch_pdl(compress_append_kernel<float>, grid, dim3(kThreads), smem, stream, a);
+    const bool tok = a.tok_rows != nullptr;
+    cudaError_t e;
+    if (bf16)
+        e = tok ? launch_pdl(compress_append_kernel<__nv_bfloat16, true>, grid, dim3(kThreads), smem, stream, a)
+                : launch_pdl(compress_append_kernel<__nv_bfloat16, false>, grid, dim3(kThreads), smem, stream, a);
+    else
+        e = tok ? launch_pdl(compress_append_kernel<float, true>, grid, dim3(kThreads), smem, stream, a)
+                : launch_pdl(compress_append_kernel<float, false>, grid, dim3(kThreads), smem, stream, a);
     if (e != cudaSuccess) return e;
     return bf16 ? launch_pdl(tail_update_kernel<__nv_bfloat16>, dim3(a.B), dim3(kThreads), 0, stream, a)
                 : launch_pdl(tail_update_kernel<float>, dim3(a.B), dim3(kThreads), 0, stream, a);

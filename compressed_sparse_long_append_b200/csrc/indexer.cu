@@ -53,8 +53,9 @@ constexpr int kProjChunkB = 8;                   // requests' cq rows staged in 
 constexpr int kProjKeepB = 128;                  // requests whose results are held before the wait
 
 // One warp per output feature r; lane l covers 8-element chunks l, l+32, ...
-// of the dc inputs.  The W row is read once into registers; the cq rows are
-// staged in shared memory kProjChunkB requests at a time.  The products are
+// of the dc inputs.  The W row is read once into registers; the cq rows of
+// the CTA's kProjKeepB requests (blockIdx.y) are staged in shared memory
+// kProjChunkB requests at a time.  The products are
 // formed before the grid-dependency wait (W and cq are inputs of the call)
 // and held in shared memory; the stores into the workspace follow the wait.
 template <typename TC, typename TW>
@@ -80,9 +81,10 @@ __global__ void __launch_bounds__(kProjThreads, 2) iq_project_kernel(IndexerArgs
             for (int i = 0; i < 8; ++i) wv[q][i] = 0.f;
     }
     bool waited = false;
-    int held0 = 0;   // first request whose results sit in res
-    for (int b0 = 0; b0 < a.B; b0 += kProjChunkB) {
-        const int nb = min(kProjChunkB, a.B - b0);
+    const int b_begin = blockIdx.y * kProjKeepB, b_end = min(a.B, b_begin + kProjKeepB);
+    int held0 = b_begin;   // first request whose results sit in res
+    for (int b0 = b_begin; b0 < b_end; b0 += kProjChunkB) {
+        const int nb = min(kProjChunkB, b_end - b0);
         __syncthreads();   // the previous chunk's cq rows are consumed
         for (int i = threadIdx.x; i < nb * nch; i += kProjThreads) {
             const int u = i / nch, ch = i % nch;
@@ -121,7 +123,7 @@ __global__ void __launch_bounds__(kProjThreads, 2) iq_project_kernel(IndexerArgs
             }
         }
         const int held = b0 + nb - held0;
-        if (held == kProjKeepB || b0 + nb == a.B) {
+        if (held == kProjKeepB || b0 + nb == b_end) {
             __syncthreads();
             if (!waited) {
                 pdl_wait();
@@ -156,7 +158,8 @@ __global__ void __launch_bounds__(kProjThreads) iq_project_wide_kernel(IndexerAr
     const int j = r / a.dI, e = r % a.dI;
     const TW *w = reinterpret_cast<const TW *>(a.W) + (size_t)r * a.dc;
     const int nch = a.dc / 8;
-    for (int b = 0; b < a.B; ++b) {
+    const int b_end = min(a.B, (int)(blockIdx.y + 1) * kProjKeepB);
+    for (int b = blockIdx.y * kProjKeepB; b < b_end; ++b) {
         const TC *c = reinterpret_cast<const TC *>(a.cq) + (size_t)b * a.dc;
         float acc = 0.f;
         for (int ch = lane; ch < nch; ch += 32) {
@@ -183,29 +186,38 @@ constexpr int kStages = 3;
 constexpr int kTileE = 128;          // entries per tile
 constexpr int kPageE = 32;           // CSA entries per 128-token page
 constexpr int kTPC = 8;              // tiles per CTA (consecutive, one request)
-constexpr int kIdxThreads = 192;     // warp 0: TMA, warp 1: MMA, warps 2..5: epilogue
+// warp 0: TMA, warp 1: MMA, then 4 epilogue warps per set of query rows:
+// one set for G = 1, four (rows g, g + 4, ... of the group) for G > 1
+template <int G>
+constexpr int idx_epi_sets() { return G > 1 ? 4 : 1; }
+template <int G>
+constexpr int idx_threads() { return 64 + 128 * idx_epi_sets<G>(); }
 
-template <int DI, int NQ>
+template <int DI, int NQ, int G>
 struct IdxSmem {
     static constexpr int kKeyBytes = kTileE * DI * 2;
-    static constexpr int kQBytes = NQ * DI * 2;
-    static constexpr int kBytes = kStages * kKeyBytes + kQBytes + 1024 /*align*/ + 512 /*barriers, pages*/;
+    static constexpr int kQBytes = G * NQ * DI * 2;
+    static constexpr int kBytes = kStages * kKeyBytes + kQBytes + 1024 /*align*/ + 1024 /*barriers, pages, weights*/;
 };
 
-// Two accumulators of NQ columns, rounded up to a power of two >= 32.
-template <int NQ>
+// Two accumulators of G*NQ columns, rounded up to a power of two >= 32.
+template <int N>
 constexpr uint32_t kTmemCols() {
-    return 2 * NQ <= 32 ? 32 : (2 * NQ <= 64 ? 64 : 128);
+    return 2 * N <= 32 ? 32 : (2 * N <= 64 ? 64 : (2 * N <= 128 ? 128 : (2 * N <= 256 ? 256 : 512)));
 }
 
-// CTA (blockIdx.x, blockIdx.y = request b) scores tiles
-// [blockIdx.x*kTPC, blockIdx.x*kTPC + kTPC) of request b (128 entries each).
-template <int DI, int NQ, int HI>
-__global__ void __launch_bounds__(kIdxThreads)
+// CTA (blockIdx.x, blockIdx.y) scores tiles [blockIdx.x*kTPC, +kTPC) (128
+// entries each) of the query rows r0 = blockIdx.y*G .. r0+G-1, which all
+// read the keys of request slots[r0]: one key tile feeds one MMA of N = G*NQ
+// query columns (decode: G = 1; query rows of one request: G > 1).
+template <int DI, int NQ, int HI, int G>
+__global__ void __launch_bounds__(idx_threads<G>())
     indexer_kernel(IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap qmap) {
     CSLA_TL_SCOPE(kTlIndexer);
-    using S = IdxSmem<DI, NQ>;
+    using S = IdxSmem<DI, NQ, G>;
+    constexpr int N = G * NQ;
+    static_assert(N % 16 == 0 && N <= 256, "UMMA N for M = 128");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t *qbuf = base + kStages * S::kKeyBytes;
@@ -214,11 +226,13 @@ __global__ void __launch_bounds__(kIdxThreads)
     uint64_t *qfull = tempty + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(qfull + 1);
     int *pages = reinterpret_cast<int *>(tmem_holder + 1);      // [kTPC * 4]
+    int *row_nv = pages + kTPC * 4;                              // [G] visible entries per row (-1: skip)
+    float *hw = reinterpret_cast<float *>(row_nv + G);           // [G][HI] head weights
     __shared__ volatile int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int b = blockIdx.y;
-    const int slot = __ldg(a.slots + b);
+    const int r0 = blockIdx.y * G;
+    const int slot = __ldg(a.slots + r0);
     const bool slot_ok = slot >= 0 && slot < a.n_slots;
     const int t_begin = blockIdx.x * kTPC;
 
@@ -231,7 +245,7 @@ __global__ void __launch_bounds__(kIdxThreads)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(tfull + i, 1);
-            mbar_init(tempty + i, 128);
+            mbar_init(tempty + i, 128 * idx_epi_sets<G>());
         }
         mbar_init(qfull, 1);
         fence_mbar_init();
@@ -247,14 +261,12 @@ __global__ void __launch_bounds__(kIdxThreads)
         }
     }
     if (warp == 1) {
-        tmem_alloc(tmem_holder, kTmemCols<NQ>());
+        tmem_alloc(tmem_holder, kTmemCols<N>());
         tmem_relinquish();
     }
-    float wj[HI];
-    if (warp >= 2) {
-        const float *w = a.head_w + (size_t)b * HI;
-#pragma unroll
-        for (int j = 0; j < HI; ++j) wj[j] = __ldg(w + j);
+    for (int i = threadIdx.x; i < G * HI; i += idx_threads<G>()) {
+        const int r = r0 + i / HI;
+        hw[i] = r < a.B ? __ldg(a.head_w + (size_t)r * HI + i % HI) : 0.f;
     }
     tc_fence_before();
     __syncthreads();
@@ -267,18 +279,37 @@ __global__ void __launch_bounds__(kIdxThreads)
     pdl_wait();
     CSLA_TL_WAITED();
 
-    const int L = slot_ok ? row_visible_len(a.len, a.q_len, slot, b) : 0;
-    const bool ok = slot_ok && L >= 0 && L <= a.max_len;
-    if (!ok && threadIdx.x == 0 && blockIdx.x == 0) set_dev_err(slot_ok ? CSLA_DEVERR_LEN : CSLA_DEVERR_INDEX);
-    const int nv = ok ? L / a.m : 0;
-    const int n_tiles = ok ? min(kTPC, (nv + kTileE - 1) / kTileE - t_begin) : 0;
+    // ---- visible entries of each row; the CTA streams the tiles of the longest
+    if (threadIdx.x < G) {
+        const int r = r0 + threadIdx.x;
+        int nv = -1;
+        if (r < a.B) {
+            const int sr = __ldg(a.slots + r);
+            if (!slot_ok || sr != slot) {
+                if (blockIdx.x == 0) set_dev_err(CSLA_DEVERR_INDEX);
+            } else {
+                const int L = row_visible_len(a.len, a.q_len, slot, r);
+                if (L < 0 || L > a.max_len) {
+                    if (blockIdx.x == 0) set_dev_err(CSLA_DEVERR_LEN);
+                } else {
+                    nv = L / a.m;
+                }
+            }
+        }
+        row_nv[threadIdx.x] = nv;
+    }
+    __syncthreads();
+    int nv_max = 0;
+#pragma unroll
+    for (int g = 0; g < G; ++g) nv_max = max(nv_max, row_nv[g]);
+    const int n_tiles = min(kTPC, (nv_max + kTileE - 1) / kTileE - t_begin);
     if (warp == 0 && lane < kTPC * 4) {
         const int e0 = t_begin * kTileE + lane * kPageE;
-        if (e0 < nv && (pg < 0 || pg >= a.n_pages)) {
+        if (e0 < nv_max && (pg < 0 || pg >= a.n_pages)) {
             set_dev_err(CSLA_DEVERR_PAGE);
             pg = -1;
         }
-        pages[lane] = e0 < nv ? pg : -1;
+        pages[lane] = e0 < nv_max ? pg : -1;
     }
     __syncwarp();
 
@@ -288,7 +319,7 @@ __global__ void __launch_bounds__(kIdxThreads)
         if (lane == 0) {
             mbar_arrive_expect_tx(qfull, (uint32_t)S::kQBytes);
 #pragma unroll
-            for (int h = 0; h < DI / 64; ++h) tma_load_2d(qbuf + h * NQ * 128, &qmap, h * 64, b * NQ, qfull);
+            for (int h = 0; h < DI / 64; ++h) tma_load_2d(qbuf + h * N * 128, &qmap, h * 64, r0 * NQ, qfull);
             int n = 0;
             for (int t = 0; t < n_tiles; ++t, ++n) {
                 const int s = n % kStages;
@@ -312,10 +343,11 @@ __global__ void __launch_bounds__(kIdxThreads)
             for (int i = (n > kStages ? n - kStages : 0); i < n; ++i)
                 mbar_wait(full + (i % kStages), (i / kStages) & 1, nullptr);
             mbar_wait(qfull, 0, nullptr);
+            CSLA_TL_MARK_ANY(4);
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(128, NQ, false, false);
+            constexpr uint32_t idesc = idesc_bf16(128, N, false, false);
             int n = 0;
             if (mbar_wait(qfull, 0, &abort_flag)) {
                 const uint32_t qb = smem_u32(qbuf);
@@ -332,8 +364,8 @@ __global__ void __launch_bounds__(kIdxThreads)
                     for (int k = 0; k < DI / 16; ++k) {
                         const uint32_t half = k / 4, ko = (k % 4) * 32;
                         const uint64_t ad = sdesc(kb + half * (kTileE * 128) + ko, 16, 1024);
-                        const uint64_t bd = sdesc(qb + half * (NQ * 128) + ko, 16, 1024);
-                        umma_kind_f16(tmem + acc * NQ, ad, bd, idesc, k > 0 ? 1u : 0u);
+                        const uint64_t bd = sdesc(qb + half * (N * 128) + ko, 16, 1024);
+                        umma_kind_f16(tmem + acc * N, ad, bd, idesc, k > 0 ? 1u : 0u);
                     }
                     umma_commit(empty + s);
                     umma_commit(tfull + acc);
@@ -342,68 +374,95 @@ __global__ void __launch_bounds__(kIdxThreads)
             if (n > 0) mbar_wait(tfull + ((n - 1) & 1), ((n - 1) / 2) & 1, nullptr);
         }
     } else {
+        // TMEM lanes 32*(warp%4).. are this warp's key rows; set `es` takes
+        // the group's rows es, es + sets, ...
+        constexpr int kSets = idx_epi_sets<G>();
         const int lane_base = 32 * (warp & 3);
+        const int es = (warp - 2) / 4;
         const int row = lane_base + lane;
         for (int t = 0, n = 0; t < n_tiles; ++t, ++n) {
             const int acc = n & 1;
             if (!mbar_wait(tfull + acc, (n / 2) & 1, &abort_flag)) break;
             tc_fence_after();
-            uint32_t r[NQ];
-            const uint32_t ta = tmem + ((uint32_t)lane_base << 16) + acc * NQ;
-            if constexpr (NQ == 16) {
-                tmem_ld32x16(ta, r);
-            } else if constexpr (NQ == 32) {
-                tmem_ld32x32(ta, r);
-            } else {
-                static_assert(NQ == 48, "query operand rows");
-                uint32_t (&r0)[32] = *reinterpret_cast<uint32_t (*)[32]>(r);
-                uint32_t (&r1)[16] = *reinterpret_cast<uint32_t (*)[16]>(r + 32);
-                tmem_ld32x32(ta, r0);
-                tmem_ld32x16(ta + 32, r1);
+            const int e = (t_begin + t) * kTileE + row;
+            int last = -1;   // this set's last row with entries in the tile (warp-uniform)
+            for (int g = es; g < G; g += kSets)
+                if (row_nv[g] > (t_begin + t) * kTileE) last = g;
+            if (last < 0) {
+                tc_fence_before();
+                mbar_arrive(tempty + acc);
             }
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(tempty + acc);
+#pragma unroll 1
+            for (int g = es; g <= last; g += kSets) {
+                const int nv = row_nv[g];
+                if (nv <= (t_begin + t) * kTileE) continue;   // the whole tile is past this row (warp-uniform)
+                uint32_t r[NQ];
+                const uint32_t ta = tmem + ((uint32_t)lane_base << 16) + acc * N + g * NQ;
+                if constexpr (NQ == 16) {
+                    tmem_ld32x16(ta, r);
+                } else if constexpr (NQ == 32) {
+                    tmem_ld32x32(ta, r);
+                } else {
+                    static_assert(NQ == 48, "query operand rows");
+                    uint32_t (&r0_)[32] = *reinterpret_cast<uint32_t (*)[32]>(r);
+                    uint32_t (&r1_)[16] = *reinterpret_cast<uint32_t (*)[16]>(r + 32);
+                    tmem_ld32x32(ta, r0_);
+                    tmem_ld32x16(ta + 32, r1_);
+                }
+                tmem_wait_ld();
+                if (g == last) {
+                    // every column this set reads is in registers: the MMA may reuse the accumulator
+                    tc_fence_before();
+                    mbar_arrive(tempty + acc);
+                }
+                if (e < nv) {
+                    float sc = 0.f;
+#pragma unroll
+                    for (int j = 0; j < HI; ++j) {
+                        const float dot = __fadd_rn(__fadd_rn(__uint_as_float(r[j]), __uint_as_float(r[HI + j])),
+                                                    __uint_as_float(r[2 * HI + j]));
+                        sc = __fmaf_rn(hw[g * HI + j], fmaxf(dot, 0.f), sc);
+                    }
+                    a.scores[(size_t)(r0 + g) * a.scores_stride + e] = sc;
+                }
+            }
             if (threadIdx.x == 64 && t == 0) CSLA_TL_MARK_ANY(2);
             if (threadIdx.x == 64 && t == kTPC - 1) CSLA_TL_MARK_ANY(3);
-            const int e = (t_begin + t) * kTileE + row;
-            if (e < nv) {
-                float sc = 0.f;
-#pragma unroll
-                for (int j = 0; j < HI; ++j) {
-                    const float dot = __fadd_rn(__fadd_rn(__uint_as_float(r[j]), __uint_as_float(r[HI + j])),
-                                                __uint_as_float(r[2 * HI + j]));
-                    sc = __fmaf_rn(wj[j], fmaxf(dot, 0.f), sc);
-                }
-                a.scores[(size_t)b * a.scores_stride + e] = sc;
-            }
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols<NQ>());
+        tmem_dealloc(tmem, kTmemCols<N>());
     }
 }
 
-template <int DI, int NQ, int HI>
+template <int DI, int NQ, int HI, int G>
 cudaError_t launch_indexer_t(const IndexerArgs &a, const CUtensorMap &kmap, const CUtensorMap &qmap,
-                             int num_sms, cudaStream_t stream) {
-    using S = IdxSmem<DI, NQ>;
+                             cudaStream_t stream) {
+    using S = IdxSmem<DI, NQ, G>;
     static int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(indexer_kernel<DI, NQ, HI>,
+        cudaError_t e = cudaFuncSetAttribute(indexer_kernel<DI, NQ, HI, G>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
-    (void)num_sms;
     const int groups = (a.tiles_per_req + kTPC - 1) / kTPC;
-    return launch_pdl(indexer_kernel<DI, NQ, HI>, dim3(groups, a.B), dim3(kIdxThreads), S::kBytes, stream, a, kmap,
-                      qmap);
+    return launch_pdl(indexer_kernel<DI, NQ, HI, G>, dim3(groups, (a.B + G - 1) / G), dim3(idx_threads<G>()),
+                      S::kBytes, stream, a, kmap, qmap);
+}
+
+template <int DI, int NQ, int HI>
+cudaError_t launch_indexer_g(const IndexerArgs &a, const CUtensorMap &kmap, const CUtensorMap &qmap,
+                             cudaStream_t stream) {
+    if (a.rows_per_cta == 1) return launch_indexer_t<DI, NQ, HI, 1>(a, kmap, qmap, stream);
+    if (a.rows_per_cta == indexer_rows_per_cta(NQ))
+        return launch_indexer_t<DI, NQ, HI, indexer_rows_per_cta(NQ)>(a, kmap, qmap, stream);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -415,7 +474,7 @@ cudaError_t launch_indexer(const IndexerArgs &a, bool cq_bf16, bool w_bf16, cons
         if (e != cudaSuccess) return e;
     }
     const int pblocks = (a.HI * a.dI + kProjThreads / 32 - 1) / (kProjThreads / 32);
-    const dim3 pg(pblocks), pb(kProjThreads);
+    const dim3 pg(pblocks, (a.B + kProjKeepB - 1) / kProjKeepB), pb(kProjThreads);
     cudaError_t e;
     if (a.dc <= 1024) {
         if (cq_bf16 && w_bf16) e = launch_pdl(iq_project_kernel<__nv_bfloat16, __nv_bfloat16>, pg, pb, 0, stream, a);
@@ -432,16 +491,16 @@ cudaError_t launch_indexer(const IndexerArgs &a, bool cq_bf16, bool w_bf16, cons
     // HI is a template parameter so the epilogue's head loop is unrolled.
     if (a.dI == 128) {
         switch (a.HI) {
-            case 16: return launch_indexer_t<128, 48, 16>(a, kmap, qmap, num_sms, stream);
-            case 8: return launch_indexer_t<128, 32, 8>(a, kmap, qmap, num_sms, stream);
-            case 4: return launch_indexer_t<128, 16, 4>(a, kmap, qmap, num_sms, stream);
+            case 16: return launch_indexer_g<128, 48, 16>(a, kmap, qmap, stream);
+            case 8: return launch_indexer_g<128, 32, 8>(a, kmap, qmap, stream);
+            case 4: return launch_indexer_g<128, 16, 4>(a, kmap, qmap, stream);
             default: break;
         }
     } else if (a.dI == 64) {
         switch (a.HI) {
-            case 16: return launch_indexer_t<64, 48, 16>(a, kmap, qmap, num_sms, stream);
-            case 8: return launch_indexer_t<64, 32, 8>(a, kmap, qmap, num_sms, stream);
-            case 4: return launch_indexer_t<64, 16, 4>(a, kmap, qmap, num_sms, stream);
+            case 16: return launch_indexer_g<64, 48, 16>(a, kmap, qmap, stream);
+            case 8: return launch_indexer_g<64, 32, 8>(a, kmap, qmap, stream);
+            case 4: return launch_indexer_g<64, 16, 4>(a, kmap, qmap, stream);
             default: break;
         }
     }

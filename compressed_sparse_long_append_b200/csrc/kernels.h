@@ -88,7 +88,12 @@ struct IndexerArgs {
     int scores_stride;
     uint16_t *q_ws;     // [B][NQ][dI] bf16
     const int32_t *q_len;   // optional per-row visible length (else len[slot])
+    int rows_per_cta;       // 1, or indexer_rows_per_cta(NQ) when all rows share slots[0]
 };
+
+// Query rows sharing one key tile per MMA when the rows of a call all belong
+// to one request: as many as fit the UMMA N limit of 256 columns.
+__host__ __device__ constexpr int indexer_rows_per_cta(int NQ) { return 256 / NQ; }
 cudaError_t launch_indexer(const IndexerArgs &a, bool cq_bf16, bool w_bf16, const CUtensorMap &kmap,
                            const CUtensorMap &qmap, int num_sms, cudaStream_t stream);
 

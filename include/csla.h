@@ -157,7 +157,11 @@ typedef struct csla_compress_params {
  *     a position outside [0, n_win_rows) sets CSLA_DEVERR_INDEX and the row
  *     is masked.  csla_window_rows and the token-row output of
  *     csla_compress_append fill such a buffer for a prefill chunk.
- * The indexer and top-k read q_len only.
+ *   one_request: nonzero promises slots[b] == slots[0] for every row (the
+ *     queries of one request's prefill chunk); the indexer then scores
+ *     several rows against each key tile it loads.  A row with another slot
+ *     sets CSLA_DEVERR_INDEX and is skipped.
+ * The indexer and top-k read q_len (and one_request) only.
  */
 typedef struct csla_queries {
     const int32_t *q_len;
@@ -165,6 +169,7 @@ typedef struct csla_queries {
     const float *win_scales;
     const int32_t *win_base;
     int32_t n_win_rows;
+    int32_t one_request;
 } csla_queries;
 
 /* Optional output of csla_compress_append: the window-format row (the one

@@ -99,8 +99,11 @@ def _queries(L0, T):
     return np.arange(L0 + 1, L0 + T + 1, dtype=np.int32)
 
 
-def test_indexer_query_rows():
-    w, L0, T = SMALL, 1000, 500
+@pytest.mark.parametrize("L0,T,one", [(1000, 500, False), (1000, 503, True), (37, 44, True)])
+def test_indexer_query_rows(L0, T, one):
+    """one: the rows are flagged as one request's queries, so several rows
+    share each key tile (a group that does not divide T included)."""
+    w = SMALL
     L1 = L0 + T
     cv, p = oracle_cache(w, [L1])
     lb = upload_layer(w, cv, [L1])
@@ -114,7 +117,7 @@ def test_indexer_query_rows():
     ql = _i32(q_len)
     C.csla_indexer_scores(lb.cfg(), lb.state(), lb.cache(), _i32(np.zeros(T)), T, L1, act_tensor(w, pi["cq"]), dt,
                           act_tensor(w, p["W_iq"]), dt, _f32(pi["head_w"]), scores, stride, ws, wsb,
-                          qs=C.queries(ql))
+                          qs=C.queries(ql, one_request=one))
     assert_no_device_error()
     got = scores.cpu().numpy()
     keys = cv.gather_keys(0, L1 // w.m)
@@ -254,3 +257,36 @@ def test_query_row_errors_are_recorded_not_trapped():
     _attend_rows(w, lb, qs, q, p, 2, L1, idx)
     rc, bits = C.csla_device_error()
     assert rc == C.CSLA_ERR_DEVICE and bits & C.CSLA_DEVERR_INDEX
+
+
+def test_indexer_one_request_rows_with_another_slot():
+    """A row flagged as part of one request but naming another slot is
+    skipped (its scores stay untouched) and CSLA_DEVERR_INDEX is recorded;
+    the other rows are scored as usual."""
+    w = SMALL
+    lens = [900, 900]
+    cv, p = oracle_cache(w, lens)
+    lb = upload_layer(w, cv, lens)
+    T = 6
+    pi = prefill_inputs(w, T, tag=5)
+    q_len = np.array([400, 500, 600, 700, 800, 900], np.int32)
+    slots = np.array([0, 0, 1, 0, 0, 0], np.int32)
+    stride = 900 // w.m
+    scores = torch.full((T, stride), float("nan"), dtype=torch.float32, device=DEV)
+    wsb = C.csla_workspace_size(lb.cfg(), C.CSLA_OP_INDEXER, T, 900)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device=DEV)
+    dt = C.CSLA_BF16 if w.act_bf16 else C.CSLA_F32
+    C.csla_indexer_scores(lb.cfg(), lb.state(), lb.cache(), _i32(slots), T, 900, act_tensor(w, pi["cq"]), dt,
+                          act_tensor(w, p["W_iq"]), dt, _f32(pi["head_w"]), scores, stride, ws, wsb,
+                          qs=C.queries(_i32(q_len), one_request=True))
+    rc, bits = C.csla_device_error()
+    assert rc == C.CSLA_ERR_DEVICE and bits == C.CSLA_DEVERR_INDEX
+    got = scores.cpu().numpy()
+    keys = cv.gather_keys(0, 900 // w.m)
+    for i in range(T):
+        if slots[i] != 0:
+            assert np.all(np.isnan(got[i])), i
+            continue
+        nv = int(q_len[i]) // w.m
+        qI = oracle.index_query(pi["cq"][i], p["W_iq"], w.HI, w.dI)
+        check_scores(got[i, :nv].astype(np.float64), oracle.index_scores(qI, pi["head_w"][i], keys[:nv]))
