@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--prefill-only", action="store_true", help="only the CSA prefill-chunk measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", type=int, default=0, help="attention variant: 0 auto, 1 saturated, 2 starved")
+    ap.add_argument("--fused-step", action="store_true",
+                    help="time the CSA step as csla_csa_decode_step instead of the four separate library calls")
     ap.add_argument("--profile", action="store_true",
                     help="only the timed CSA steps, bracketed by cudaProfilerStart/Stop (for ncu "
                          "--profile-from-start off); implies --no-hca --no-cpu-baseline and no e2e leg")
@@ -192,8 +194,12 @@ def step_inputs(shape_kw, n_req, n_steps, seed, rank, device):
 
 
 class CsaStep:
-    """One CSA decode step of one layer copy as four library calls; each call
-    takes the step's input tensors x (dict of device tensors)."""
+    """One CSA decode step of one layer copy: csla_csa_decode_step (or, with
+    fused=False, the four separate library calls); each call takes the step's
+    input tensors x (dict of device tensors).  sep_calls are the four
+    separate calls (per-call timings, the indexer roofline)."""
+
+    fused = False
 
     def __init__(self, lb, cp, params, kw, variant, device):
         import torch
@@ -212,9 +218,20 @@ class CsaStep:
         self.wsa = C.csla_workspace_size(cfg, C.CSLA_OP_CSA_ATTEND, B, kw["k"])
         self.ws_i = torch.zeros(self.wsi, dtype=torch.uint8, device=device)
         self.ws_a = torch.zeros(self.wsa, dtype=torch.uint8, device=device)
+        self.wss = C.csla_workspace_size(cfg, C.CSLA_OP_CSA_DECODE_STEP, B, kw["k"])
+        self.ws_s = torch.zeros(self.wss, dtype=torch.uint8, device=device)
         self.cfg, self.st, self.cache, self.cps = cfg, lb.state(), lb.cache(), cp.struct()
         self.names = ["compress_append", "indexer_scores", "topk_select", "csa_attend"]
-        self.calls = [self._compress, self._indexer, self._topk, self._attend]
+        self.sep_calls = [self._compress, self._indexer, self._topk, self._attend]
+        self.calls = [self._step] if self.fused else self.sep_calls
+
+    def _step(self, x):
+        C = self.C
+        C.csla_csa_decode_step(self.cfg, self.st, self.cache, self.slots, self.B, 1, self.max_len, x["kv"],
+                               x["kidx"], C.CSLA_BF16, self.cps, x["cq"], C.CSLA_BF16, self.p["W_iq"], C.CSLA_BF16,
+                               x["head_w"], self.scores, self.stride, self.kw["k"], self.idx, x["q"], C.CSLA_BF16,
+                               self.p["sink"], self.p["gamma_q"], self.out, C.CSLA_BF16, self.variant, self.ws_i,
+                               self.wsi, self.ws_s, self.wss)
 
     def _compress(self, x):
         C = self.C
@@ -238,17 +255,18 @@ class CsaStep:
                           self.ws_a, self.wsa)
 
     def launches(self):
-        return csa_launches(self.kw, self.variant)
+        return csa_launches(self.kw, self.variant, self.fused)
 
 
-def csa_launches(kw, variant):
+def csa_launches(kw, variant, fused):
     """Kernels of one CSA step: compress (pool + tail/len), iq_project +
     indexer, topk, attend, + combine unless the saturated variant runs
-    (forced, or automatic: one chunk per request or B >= SM count)."""
+    (forced, or automatic: one chunk per request or B >= SM count); the
+    fused step adds the length snapshot and the second indexer launch."""
     rows = kw["k"] + kw["n_win"]
     chunks = -(-rows // (64 * -(-rows // 2048)))
     saturated = variant == 1 or (variant == 0 and (kw["B"] >= 148 or chunks <= 1))
-    return 2 + 2 + 1 + 1 + (0 if saturated else 1)
+    return 2 + 2 + 1 + 1 + (0 if saturated else 1) + (2 if fused else 0)
 
 
 class HcaStep:
@@ -269,6 +287,7 @@ class HcaStep:
         self.cfg, self.st, self.cache, self.cps = cfg, lb.state(), lb.cache(), cp.struct()
         self.names = ["compress_append", "hca_attend"]
         self.calls = [self._compress, self._attend]
+        self.sep_calls = self.calls
 
     def _compress(self, x):
         C = self.C
@@ -514,8 +533,8 @@ def breakdown(steps, inputs, W, K):
     the parts add up to more than the pipelined step)."""
     import torch
     R = len(steps)
-    n = len(steps[0].calls)
-    graphs = [[capture(lambda c=c, x=inputs[W + r]: c(x)) for c in steps[r].calls] for r in range(R)]
+    n = len(steps[0].sep_calls)
+    graphs = [[capture(lambda c=c, x=inputs[W + r]: c(x)) for c in steps[r].sep_calls] for r in range(R)]
     torch.cuda.synchronize()
     segs = []
     for i in range(K):
@@ -539,7 +558,7 @@ def call_time(steps, inputs, W, K, j):
     caches."""
     import torch
     R = len(steps)
-    g = capture(lambda: [steps[i % R].calls[j](inputs[W + i % R]) for i in range(K)])
+    g = capture(lambda: [steps[i % R].sep_calls[j](inputs[W + i % R]) for i in range(K)])
     g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -679,6 +698,7 @@ def main():
     L0s = [kw["L"] - before - (b % m) for b in range(B)]
     lb, cp, params = build_layer(kw, B, L0s, seed, rank, device)
     inputs = step_inputs(kw, B, W + K, seed, rank, device)
+    CsaStep.fused = args.fused_step
     steps = make_copies(CsaStep, lb, cp, params, kw, args.variant, device, R)
     if world > 1:
         dist.barrier()
@@ -758,7 +778,7 @@ def main():
             cpu = {"value": None, "unit": UNIT, "cores": 0, "kind": "oracle", "sample": "failed: %s" % e}
 
     if rank == 0:
-        launches_per_step = csa_launches(kw, args.variant)
+        launches_per_step = csa_launches(kw, args.variant, CsaStep.fused)
         line = {
             "metric": METRIC, "value": B * world / (ms_step * 1e-3), "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -771,8 +791,10 @@ def main():
                        "index_heads": 16, "index_dim": 128, "dc": 1024, "topk": 512, "window": 128,
                        "l2": "inputs larger than L2: %d rotating copies of the layer (caches + W_iq), "
                              "~%d MB touched per rotation vs 126 MB L2" % (R, R * 75),
-                       "launch": "one CUDA graph per step (all four library calls), K graphs replayed back to "
-                                 "back between one event pair",
+                       "launch": ("one CUDA graph per step (csla_csa_decode_step: the append on a side stream "
+                                  "beside the indexer's scoring of the entries already complete)" if CsaStep.fused else
+                                  "one CUDA graph per step (the four library calls)") +
+                                 ", K graphs replayed back to back between one event pair",
                        "parallelism": "dp%d over requests" % world, "variant": args.variant},
             "segments_ms": {"compress_append": seg[0], "indexer_scores": seg[1], "topk_select": seg[2],
                             "csa_attend": seg[3], "note": "one graph launch per call, serialised"},

@@ -14,13 +14,13 @@ LIB_PATH = os.path.join(_HERE, "libcsla.so")
 CSLA_OK, CSLA_ERR_ARG, CSLA_ERR_UNSUPPORTED, CSLA_ERR_CUDA, CSLA_ERR_DEVICE = 0, 1, 2, 3, 4
 CSLA_F32, CSLA_BF16 = 0, 1
 CSLA_VARIANT_AUTO, CSLA_VARIANT_SATURATED, CSLA_VARIANT_STARVED = 0, 1, 2
-CSLA_OP_INDEXER, CSLA_OP_TOPK, CSLA_OP_CSA_ATTEND, CSLA_OP_HCA_ATTEND = 1, 2, 3, 4
+CSLA_OP_INDEXER, CSLA_OP_TOPK, CSLA_OP_CSA_ATTEND, CSLA_OP_HCA_ATTEND, CSLA_OP_CSA_DECODE_STEP = 1, 2, 3, 4, 5
 CSLA_DEVERR_PAGE, CSLA_DEVERR_INDEX, CSLA_DEVERR_LEN, CSLA_DEVERR_TIMEOUT = 1, 2, 4, 8
 CSLA_PAGE_TOKENS = 128
 
 EXPORTS = ("csla_compress_append", "csla_indexer_scores", "csla_topk_select", "csla_csa_attend",
            "csla_hca_attend", "csla_workspace_size", "csla_device_error", "csla_strerror", "csla_version",
-           "csla_indexer_scores_noalloc", "csla_window_rows")
+           "csla_indexer_scores_noalloc", "csla_window_rows", "csla_csa_decode_step")
 CSLA_NOALLOC_INDEXER_SCRATCH_BYTES = 786432
 
 
@@ -100,6 +100,8 @@ def _load():
         "csla_strerror": [ctypes.c_int],
         "csla_version": [],
         "csla_indexer_scores_noalloc": [P, P, P, P, I, P, I, P, I, P, I, P, P, I, P],
+        "csla_csa_decode_step": [P, P, P, P, I, I, I, P, P, I, P, P, I, P, I, P, P, I, I, P, P, I, P, P, P, I, I,
+                                 P, Z, P, Z, P],
     }
     res = {"csla_workspace_size": ctypes.c_size_t, "csla_strerror": ctypes.c_char_p}
     for name, args in sig.items():
@@ -186,6 +188,18 @@ def csla_hca_attend(cfg, st, cache, slots, B, max_len, q, q_dtype, sink, gamma_q
     return _check("csla_hca_attend", _lib.csla_hca_attend(
         _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, _ref(qs), max_len, _ptr(q), q_dtype, _ptr(sink),
         _ptr(gamma_q), _ptr(out), out_dtype, variant, _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def csla_csa_decode_step(cfg, st, cache, slots, B, T, max_len, kv_new, kidx_new, kv_dtype, params, cq, cq_dtype,
+                         W_iq, w_dtype, head_w, scores, scores_stride, k, idx, q, q_dtype, sink, gamma_q, out,
+                         out_dtype, variant, ws_indexer, ws_indexer_bytes, ws_step, ws_step_bytes, stream=None):
+    """compress_append + indexer_scores + topk_select + csa_attend in one call
+    (same results; the indexer overlaps the append, see include/csla.h)."""
+    return _check("csla_csa_decode_step", _lib.csla_csa_decode_step(
+        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, T, max_len, _ptr(kv_new), _ptr(kidx_new), kv_dtype,
+        _ref(params), _ptr(cq), cq_dtype, _ptr(W_iq), w_dtype, _ptr(head_w), _ptr(scores), scores_stride, k,
+        _ptr(idx), _ptr(q), q_dtype, _ptr(sink), _ptr(gamma_q), _ptr(out), out_dtype, variant, _ptr(ws_indexer),
+        ws_indexer_bytes, _ptr(ws_step), ws_step_bytes, _stream(stream)))
 
 
 def csla_workspace_size(cfg, op, B, max_len):

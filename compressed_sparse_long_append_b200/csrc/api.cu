@@ -148,6 +148,8 @@ size_t csla_workspace_size(const csla_cfg *cfg, int32_t op, int32_t B, int32_t m
         case CSLA_OP_TOPK: return 0;
         case CSLA_OP_CSA_ATTEND: return attend_ws(cfg, B, (long long)max_len + cfg->n_win);
         case CSLA_OP_HCA_ATTEND: return attend_ws(cfg, B, (long long)max_len / cfg->m + cfg->n_win);
+        case CSLA_OP_CSA_DECODE_STEP:
+            return attend_ws(cfg, B, (long long)max_len + cfg->n_win) + ((size_t)B * 4 + 15) / 16 * 16;
         default: return 0;
     }
 }
@@ -162,9 +164,9 @@ int csla_device_error(csla_stream_t stream, uint32_t *bits) {
     return v ? CSLA_ERR_DEVICE : CSLA_OK;
 }
 
-int csla_compress_append(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
+static int prep_compress(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
                          int32_t B, int32_t T, const void *kv_new, const void *kidx_new, int32_t kv_dtype,
-                         const csla_compress_params *p, const csla_token_rows *tok, csla_stream_t stream) {
+                         const csla_compress_params *p, const csla_token_rows *tok, CompressArgs *out) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (!st || !cache || !slots || !kv_new || !p || B < 1 || T < 1 || T > 65535) return CSLA_ERR_ARG;
@@ -199,6 +201,16 @@ int csla_compress_append(const csla_cfg *cfg, const csla_state *st, const csla_c
     if (tok) {
         a.tok_rows = tok->rows; a.tok_scales = tok->scales; a.tok_stride = tok->stride; a.tok_offset = tok->offset;
     }
+    *out = a;
+    return CSLA_OK;
+}
+
+int csla_compress_append(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
+                         int32_t B, int32_t T, const void *kv_new, const void *kidx_new, int32_t kv_dtype,
+                         const csla_compress_params *p, const csla_token_rows *tok, csla_stream_t stream) {
+    CompressArgs a;
+    const int rc = prep_compress(cfg, st, cache, slots, B, T, kv_new, kidx_new, kv_dtype, p, tok, &a);
+    if (rc) return rc;
     return cuda_status(launch_compress_append(a, kv_dtype == CSLA_BF16, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -217,10 +229,16 @@ int csla_window_rows(const csla_cfg *cfg, const csla_state *st, const int32_t *s
     return cuda_status(launch_window_rows(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
-                        int32_t B, const csla_queries *qs, int32_t max_len, const void *cq, int32_t cq_dtype, const void *W_iq,
-                        int32_t w_dtype, const float *head_w, float *scores, int32_t scores_stride, void *workspace,
-                        size_t workspace_bytes, csla_stream_t stream) {
+struct IndexerLaunch {
+    IndexerArgs a;
+    CUtensorMap kmap, qmap;
+    bool cq_bf16, w_bf16;
+};
+
+static int prep_indexer(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
+                        int32_t B, const csla_queries *qs, int32_t max_len, const void *cq, int32_t cq_dtype,
+                        const void *W_iq, int32_t w_dtype, const float *head_w, float *scores, int32_t scores_stride,
+                        void *workspace, size_t workspace_bytes, IndexerLaunch *L) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     rc = check_csa_indexer_shape(cfg);
@@ -240,6 +258,10 @@ int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_ca
     const int G = (qs && qs->one_request) ? indexer_rows_per_cta(NQ) : 1;
     if (!encode_bf16_2d(&qmap, workspace, (uint64_t)cfg->dI, (uint64_t)B * NQ, (uint32_t)(G * NQ)))
         return CSLA_ERR_CUDA;
+    L->kmap = kmap;
+    L->qmap = qmap;
+    L->cq_bf16 = cq_dtype == CSLA_BF16;
+    L->w_bf16 = w_dtype == CSLA_BF16;
     IndexerArgs a{};
     a.m = cfg->m; a.HI = cfg->HI; a.dI = cfg->dI; a.dc = cfg->dc; a.NQ = NQ;
     a.slots = slots; a.len = st->len; a.block_table = cache->block_table; a.bt_stride = cache->bt_stride;
@@ -252,13 +274,25 @@ int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_ca
     a.q_ws = reinterpret_cast<uint16_t *>(workspace);
     a.q_len = qs ? qs->q_len : nullptr;
     a.rows_per_cta = G;
-    return cuda_status(launch_indexer(a, cq_dtype == CSLA_BF16, w_dtype == CSLA_BF16, kmap, qmap, num_sms_current(),
+    L->a = a;
+    return CSLA_OK;
+}
+
+int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
+                        int32_t B, const csla_queries *qs, int32_t max_len, const void *cq, int32_t cq_dtype, const void *W_iq,
+                        int32_t w_dtype, const float *head_w, float *scores, int32_t scores_stride, void *workspace,
+                        size_t workspace_bytes, csla_stream_t stream) {
+    IndexerLaunch L;
+    const int rc = prep_indexer(cfg, st, cache, slots, B, qs, max_len, cq, cq_dtype, W_iq, w_dtype, head_w, scores,
+                                scores_stride, workspace, workspace_bytes, &L);
+    if (rc) return rc;
+    return cuda_status(launch_indexer(L.a, L.cq_bf16, L.w_bf16, L.kmap, L.qmap, num_sms_current(),
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
-int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *slots, int32_t B,
+static int prep_topk(const csla_cfg *cfg, const csla_state *st, const int32_t *slots, int32_t B,
                      const csla_queries *qs, int32_t max_len,
-                     const float *scores, int32_t scores_stride, int32_t k, int32_t *idx, csla_stream_t stream) {
+                     const float *scores, int32_t scores_stride, int32_t k, int32_t *idx, TopkArgs *out) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (!st || !st->len || !slots || !scores || !idx || B < 1 || max_len < 0 || k < 1 || k > 2048)
@@ -268,13 +302,24 @@ int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *s
     a.scores = scores; a.stride = scores_stride; a.slots = slots; a.len = st->len;
     a.m = cfg->m; a.k = k; a.B = B; a.max_n = max_len / cfg->m; a.idx = idx; a.n_slots = st->n_slots;
     a.q_len = qs ? qs->q_len : nullptr;
+    *out = a;
+    return CSLA_OK;
+}
+
+int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *slots, int32_t B,
+                     const csla_queries *qs, int32_t max_len, const float *scores, int32_t scores_stride, int32_t k,
+                     int32_t *idx, csla_stream_t stream) {
+    TopkArgs a;
+    const int rc = prep_topk(cfg, st, slots, B, qs, max_len, scores, scores_stride, k, idx, &a);
+    if (rc) return rc;
     return cuda_status(launch_topk(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-static int attend_common(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
-                         int32_t B, const csla_queries *qs, int32_t max_len, const void *q, int32_t q_dtype, const int32_t *idx, int32_t k,
-                         const float *sink, const float *gamma_q, void *out, int32_t out_dtype, int32_t variant,
-                         void *workspace, size_t workspace_bytes, csla_stream_t stream) {
+static int prep_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
+                       int32_t B, const csla_queries *qs, int32_t max_len, const void *q, int32_t q_dtype,
+                       const int32_t *idx, int32_t k, const float *sink, const float *gamma_q, void *out,
+                       int32_t out_dtype, int32_t variant, void *workspace, size_t workspace_bytes,
+                       AttendArgs *res) {
     if (!st || !st->len || !st->win_rows || !st->win_scales || !cache || !cache->rows || !cache->scales ||
         !cache->block_table || !slots || !q || !sink || !gamma_q || !out || !workspace || B < 1)
         return CSLA_ERR_ARG;
@@ -302,6 +347,19 @@ static int attend_common(const csla_cfg *cfg, const csla_state *st, const csla_c
         a.n_src = qs->n_win_rows;
     }
     if (workspace_bytes < attend_ws(cfg, B, max_rows)) return CSLA_ERR_ARG;
+    *res = a;
+    return CSLA_OK;
+}
+
+static int attend_common(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
+                         int32_t B, const csla_queries *qs, int32_t max_len, const void *q, int32_t q_dtype,
+                         const int32_t *idx, int32_t k, const float *sink, const float *gamma_q, void *out,
+                         int32_t out_dtype, int32_t variant, void *workspace, size_t workspace_bytes,
+                         csla_stream_t stream) {
+    AttendArgs a;
+    const int rc = prep_attend(cfg, st, cache, slots, B, qs, max_len, q, q_dtype, idx, k, sink, gamma_q, out, out_dtype,
+                               variant, workspace, workspace_bytes, &a);
+    if (rc) return rc;
     return cuda_status(launch_attend(a, q_dtype == CSLA_BF16, out_dtype == CSLA_BF16, variant, num_sms_current(),
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -327,6 +385,84 @@ int csla_hca_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache 
     if (max_len < 1) return CSLA_ERR_ARG;
     return attend_common(cfg, st, cache, slots, B, qs, max_len, q, q_dtype, nullptr, 0, sink, gamma_q, out, out_dtype,
                          variant, workspace, workspace_bytes, stream);
+}
+
+// Side stream and fork/join events of the calling thread on each device
+// (created on the thread's first decode-step call on that device).
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+static thread_local SideStream tl_side[64];
+
+static int side_stream(SideStream **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CSLA_ERR_CUDA;
+    SideStream &x = tl_side[dev];
+    if (!x.s) {
+        if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) != cudaSuccess)
+            return CSLA_ERR_CUDA;
+    }
+    *out = &x;
+    return CSLA_OK;
+}
+
+int csla_csa_decode_step(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
+                         int32_t B, int32_t T, int32_t max_len, const void *kv_new, const void *kidx_new,
+                         int32_t kv_dtype, const csla_compress_params *p, const void *cq, int32_t cq_dtype,
+                         const void *W_iq, int32_t w_dtype, const float *head_w, float *scores,
+                         int32_t scores_stride, int32_t k, int32_t *idx, const void *q, int32_t q_dtype,
+                         const float *sink, const float *gamma_q, void *out, int32_t out_dtype, int32_t variant,
+                         void *ws_indexer, size_t ws_indexer_bytes, void *ws_step, size_t ws_step_bytes,
+                         csla_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->m != 4) return CSLA_ERR_UNSUPPORTED;
+    if (!idx || k < 1 || k > 2048 || !ws_step || !aligned16(ws_step)) return CSLA_ERR_ARG;
+    CompressArgs ca;
+    IndexerLaunch il;
+    TopkArgs ta;
+    AttendArgs aa;
+    rc = prep_compress(cfg, st, cache, slots, B, T, kv_new, kidx_new, kv_dtype, p, nullptr, &ca);
+    if (rc) return rc;
+    rc = prep_indexer(cfg, st, cache, slots, B, nullptr, max_len, cq, cq_dtype, W_iq, w_dtype, head_w, scores,
+                      scores_stride, ws_indexer, ws_indexer_bytes, &il);
+    if (rc) return rc;
+    rc = prep_topk(cfg, st, slots, B, nullptr, max_len, scores, scores_stride, k, idx, &ta);
+    if (rc) return rc;
+    const size_t att_bytes = attend_ws(cfg, B, (long long)k + cfg->n_win);
+    if (ws_step_bytes < csla_workspace_size(cfg, CSLA_OP_CSA_DECODE_STEP, B, k)) return CSLA_ERR_ARG;
+    rc = prep_attend(cfg, st, cache, slots, B, nullptr, 0x7FFFFFFF, q, q_dtype, idx, k, sink, gamma_q, out,
+                     out_dtype, variant, ws_step, att_bytes, &aa);
+    if (rc) return rc;
+    int32_t *len0 = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(ws_step) + att_bytes);
+    SideStream *side = nullptr;
+    rc = side_stream(&side);
+    if (rc) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // old entries (complete before this append) on the caller's stream while
+    // the append runs on the side stream; then the entries it added
+    IndexerArgs old_a = il.a, new_a = il.a;
+    old_a.range = 1;
+    old_a.len0 = len0;
+    new_a.range = 2;
+    new_a.len0 = len0;
+    new_a.tiles_per_req = ((T / cfg->m + 2) + 127) / 128 + 1;
+    cudaError_t e = launch_len_snapshot(slots, st->len, B, st->n_slots, len0, s);
+    if (e == cudaSuccess) e = cudaEventRecord(side->fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
+    if (e == cudaSuccess) e = launch_compress_append(ca, kv_dtype == CSLA_BF16, side->s);
+    if (e == cudaSuccess) e = cudaEventRecord(side->join, side->s);
+    if (e == cudaSuccess) e = launch_indexer(old_a, il.cq_bf16, il.w_bf16, il.kmap, il.qmap, num_sms_current(), s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, side->join, 0);
+    if (e == cudaSuccess)
+        e = launch_indexer(new_a, il.cq_bf16, il.w_bf16, il.kmap, il.qmap, num_sms_current(), s, false);
+    if (e == cudaSuccess) e = launch_topk(ta, s);
+    if (e == cudaSuccess)
+        e = launch_attend(aa, q_dtype == CSLA_BF16, out_dtype == CSLA_BF16, variant, num_sms_current(), s);
+    return cuda_status(e);
 }
 
 }  // extern "C"

@@ -55,14 +55,18 @@ constexpr int kProjKeepB = 128;                  // requests whose results are h
 // One warp per output feature r; lane l covers 8-element chunks l, l+32, ...
 // of the dc inputs.  The W row is read once into registers; the cq rows of
 // the CTA's kProjKeepB requests (blockIdx.y) are staged in shared memory
-// kProjChunkB requests at a time.  The products are
+// kProjChunkB requests at a time, split into two planes of 4-element halves
+// so that a warp's 16-byte reads are contiguous (no bank conflicts).  Each
+// request's value is one chain of fused multiply-adds over chunks then
+// elements, then the warp's xor tree (the chains of a chunk's requests run
+// interleaved): the same arithmetic whatever the batch.  The products are
 // formed before the grid-dependency wait (W and cq are inputs of the call)
 // and held in shared memory; the stores into the workspace follow the wait.
 template <typename TC, typename TW>
 __global__ void __launch_bounds__(kProjThreads, 2) iq_project_kernel(IndexerArgs a) {
     CSLA_TL_SCOPE(kTlIqProject);
     constexpr int kMaxCh = 4;   // dc <= 32 * 8 * kMaxCh = 1024 on this path
-    __shared__ __align__(16) float cs[kProjChunkB][1024];
+    __shared__ __align__(16) float4 cs[kProjChunkB][2][32 * kMaxCh];
     __shared__ uint16_t res[kProjKeepB][kProjWarps][3];
     pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -90,41 +94,53 @@ __global__ void __launch_bounds__(kProjThreads, 2) iq_project_kernel(IndexerArgs
             const int u = i / nch, ch = i % nch;
             float t[8];
             load8<TC>(reinterpret_cast<const TC *>(a.cq) + (size_t)(b0 + u) * a.dc + ch * 8, t);
-            float4 *dst = reinterpret_cast<float4 *>(&cs[u][ch * 8]);
-            dst[0] = make_float4(t[0], t[1], t[2], t[3]);
-            dst[1] = make_float4(t[4], t[5], t[6], t[7]);
+            cs[u][0][ch] = make_float4(t[0], t[1], t[2], t[3]);
+            cs[u][1][ch] = make_float4(t[4], t[5], t[6], t[7]);
         }
         __syncthreads();
+        if (b0 == b_begin) CSLA_TL_MARK(0);
         if (active) {
-            for (int u = 0; u < nb; ++u) {
-                float acc = 0.f;
+            float acc[kProjChunkB];
 #pragma unroll
-                for (int q = 0; q < kMaxCh; ++q) {
-                    const int ch = lane + 32 * q;
-                    if (ch < nch) {
-                        const float4 c0 = reinterpret_cast<const float4 *>(&cs[u][ch * 8])[0];
-                        const float4 c1 = reinterpret_cast<const float4 *>(&cs[u][ch * 8])[1];
-                        const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            for (int u = 0; u < kProjChunkB; ++u) acc[u] = 0.f;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) acc = __fmaf_rn(wv[q][i], cv[i], acc);
+            for (int q = 0; q < kMaxCh; ++q) {
+                const int ch = lane + 32 * q;
+                if (ch < nch) {
+#pragma unroll
+                    for (int u = 0; u < kProjChunkB; ++u) {
+                        if (u < nb) {
+                            const float4 c0 = cs[u][0][ch], c1 = cs[u][1][ch];
+                            const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) acc[u] = __fmaf_rn(wv[q][i], cv[i], acc[u]);
+                        }
                     }
                 }
-                acc = warp_sum(acc);
-                if (lane == 0) {
-                    const uint16_t hi = f32_to_bf16_bits(acc);
-                    const float r1 = __fsub_rn(acc, bf16_bits_to_f32(hi));
-                    const uint16_t mid = f32_to_bf16_bits(r1);
-                    const uint16_t lo = f32_to_bf16_bits(__fsub_rn(r1, bf16_bits_to_f32(mid)));
-                    uint16_t *o = res[(b0 + u) - held0][warp];
-                    o[0] = hi;
-                    o[1] = mid;
-                    o[2] = lo;
+            }
+#pragma unroll
+            for (int u = 0; u < kProjChunkB; ++u) acc[u] = warp_sum(acc[u]);
+            if (lane == 0) {
+#pragma unroll
+                for (int u = 0; u < kProjChunkB; ++u) {
+                    if (u < nb) {
+                        const uint16_t hi = f32_to_bf16_bits(acc[u]);
+                        const float r1 = __fsub_rn(acc[u], bf16_bits_to_f32(hi));
+                        const uint16_t mid = f32_to_bf16_bits(r1);
+                        const uint16_t lo = f32_to_bf16_bits(__fsub_rn(r1, bf16_bits_to_f32(mid)));
+                        uint16_t *o = res[(b0 + u) - held0][warp];
+                        o[0] = hi;
+                        o[1] = mid;
+                        o[2] = lo;
+                    }
                 }
             }
         }
         const int held = b0 + nb - held0;
+        if (b0 == b_begin) CSLA_TL_MARK(1);
         if (held == kProjKeepB || b0 + nb == b_end) {
             __syncthreads();
+            CSLA_TL_MARK(2);
             if (!waited) {
                 pdl_wait();
                 CSLA_TL_WAITED();
@@ -226,15 +242,16 @@ __global__ void __launch_bounds__(idx_threads<G>())
     uint64_t *qfull = tempty + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(qfull + 1);
     int *pages = reinterpret_cast<int *>(tmem_holder + 1);      // [kTPC * 4]
-    int *row_nv = pages + kTPC * 4;                              // [G] visible entries per row (-1: skip)
-    float *hw = reinterpret_cast<float *>(row_nv + G);           // [G][HI] head weights
+    int *row_nv = pages + kTPC * 4;                              // [G] entries scored below this (-1: skip)
+    int *row_lo = row_nv + G;                                    // [G] first entry scored
+    float *hw = reinterpret_cast<float *>(row_lo + G);           // [G][HI] head weights
     __shared__ volatile int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r0 = blockIdx.y * G;
     const int slot = __ldg(a.slots + r0);
     const bool slot_ok = slot >= 0 && slot < a.n_slots;
-    const int t_begin = blockIdx.x * kTPC;
+    __shared__ int s_t0;   // range 2: first tile of the request's new entries
 
     // ---- before the wait: barriers, TMEM, page ids, head weights
     if (threadIdx.x == 0) {
@@ -252,8 +269,8 @@ __global__ void __launch_bounds__(idx_threads<G>())
     }
     int pg = -1;   // warp 0: page id of this CTA's page `lane`
     if (warp == 0) {
-        const int col = (t_begin * kTileE + lane * kPageE) / kPageE;
-        if (slot_ok && lane < kTPC * 4 && col < a.bt_stride)
+        const int col = (blockIdx.x * kTPC * kTileE + lane * kPageE) / kPageE;
+        if (a.range != 2 && slot_ok && lane < kTPC * 4 && col < a.bt_stride)
             pg = __ldg(a.block_table + (size_t)slot * a.bt_stride + col);
         if (lane == 0) {
             tma_prefetch_desc(&kmap);
@@ -279,30 +296,44 @@ __global__ void __launch_bounds__(idx_threads<G>())
     pdl_wait();
     CSLA_TL_WAITED();
 
-    // ---- visible entries of each row; the CTA streams the tiles of the longest
+    // ---- entries of each row scored here; the CTA streams the tiles of the longest.
+    // range 0: [0, visible); 1: [0, len0/m) (entries complete before an append
+    // that may still be running); 2: [len0/m, visible) (the ones it added).
     if (threadIdx.x < G) {
         const int r = r0 + threadIdx.x;
-        int nv = -1;
+        int nv = -1, lo = 0;
         if (r < a.B) {
             const int sr = __ldg(a.slots + r);
             if (!slot_ok || sr != slot) {
                 if (blockIdx.x == 0) set_dev_err(CSLA_DEVERR_INDEX);
             } else {
-                const int L = row_visible_len(a.len, a.q_len, slot, r);
+                const int L = a.range == 1 ? a.len0[r] : row_visible_len(a.len, a.q_len, slot, r);
                 if (L < 0 || L > a.max_len) {
                     if (blockIdx.x == 0) set_dev_err(CSLA_DEVERR_LEN);
                 } else {
                     nv = L / a.m;
+                    if (a.range == 2) {
+                        lo = a.len0[r] / a.m;
+                        if (lo >= nv) nv = -1;
+                    }
                 }
             }
         }
         row_nv[threadIdx.x] = nv;
+        row_lo[threadIdx.x] = lo;
+        if (threadIdx.x == 0) s_t0 = a.range == 2 ? lo / kTileE : 0;
     }
     __syncthreads();
+    const int t_begin = blockIdx.x * kTPC + s_t0;
     int nv_max = 0;
 #pragma unroll
     for (int g = 0; g < G; ++g) nv_max = max(nv_max, row_nv[g]);
     const int n_tiles = min(kTPC, (nv_max + kTileE - 1) / kTileE - t_begin);
+    if (a.range == 2 && warp == 0) {
+        const int col = (t_begin * kTileE + lane * kPageE) / kPageE;
+        if (slot_ok && lane < kTPC * 4 && col < a.bt_stride)
+            pg = __ldg(a.block_table + (size_t)slot * a.bt_stride + col);
+    }
     if (warp == 0 && lane < kTPC * 4) {
         const int e0 = t_begin * kTileE + lane * kPageE;
         if (e0 < nv_max && (pg < 0 || pg >= a.n_pages)) {
@@ -415,7 +446,7 @@ __global__ void __launch_bounds__(idx_threads<G>())
                     tc_fence_before();
                     mbar_arrive(tempty + acc);
                 }
-                if (e < nv) {
+                if (e < nv && e >= row_lo[g]) {
                     float sc = 0.f;
 #pragma unroll
                     for (int j = 0; j < HI; ++j) {
@@ -465,29 +496,19 @@ cudaError_t launch_indexer_g(const IndexerArgs &a, const CUtensorMap &kmap, cons
     return cudaErrorInvalidValue;
 }
 
-}  // namespace
+// len0[b] = len[slots[b]], read after the grid wait (0 for a bad slot).
+__global__ void __launch_bounds__(256) len_snapshot_kernel(const int32_t *slots, const int32_t *len, int B,
+                                                           int n_slots, int32_t *len0) {
+    pdl_trigger();
+    pdl_wait();
+    const int b = blockIdx.x * 256 + threadIdx.x;
+    if (b >= B) return;
+    const int slot = slots[b];
+    len0[b] = (slot >= 0 && slot < n_slots) ? len[slot] : 0;
+}
 
-cudaError_t launch_indexer(const IndexerArgs &a, bool cq_bf16, bool w_bf16, const CUtensorMap &kmap,
-                           const CUtensorMap &qmap, int num_sms, cudaStream_t stream) {
-    if (a.NQ > 3 * a.HI) {
-        cudaError_t e = cudaMemsetAsync(a.q_ws, 0, (size_t)a.B * a.NQ * a.dI * 2, stream);
-        if (e != cudaSuccess) return e;
-    }
-    const int pblocks = (a.HI * a.dI + kProjThreads / 32 - 1) / (kProjThreads / 32);
-    const dim3 pg(pblocks, (a.B + kProjKeepB - 1) / kProjKeepB), pb(kProjThreads);
-    cudaError_t e;
-    if (a.dc <= 1024) {
-        if (cq_bf16 && w_bf16) e = launch_pdl(iq_project_kernel<__nv_bfloat16, __nv_bfloat16>, pg, pb, 0, stream, a);
-        else if (cq_bf16) e = launch_pdl(iq_project_kernel<__nv_bfloat16, float>, pg, pb, 0, stream, a);
-        else if (w_bf16) e = launch_pdl(iq_project_kernel<float, __nv_bfloat16>, pg, pb, 0, stream, a);
-        else e = launch_pdl(iq_project_kernel<float, float>, pg, pb, 0, stream, a);
-    } else {
-        if (cq_bf16 && w_bf16) e = launch_pdl(iq_project_wide_kernel<__nv_bfloat16, __nv_bfloat16>, pg, pb, 0, stream, a);
-        else if (cq_bf16) e = launch_pdl(iq_project_wide_kernel<__nv_bfloat16, float>, pg, pb, 0, stream, a);
-        else if (w_bf16) e = launch_pdl(iq_project_wide_kernel<float, __nv_bfloat16>, pg, pb, 0, stream, a);
-        else e = launch_pdl(iq_project_wide_kernel<float, float>, pg, pb, 0, stream, a);
-    }
-    if (e != cudaSuccess) return e;
+cudaError_t launch_scoring(const IndexerArgs &a, const CUtensorMap &kmap, const CUtensorMap &qmap,
+                           cudaStream_t stream) {
     // HI is a template parameter so the epilogue's head loop is unrolled.
     if (a.dI == 128) {
         switch (a.HI) {
@@ -505,6 +526,41 @@ cudaError_t launch_indexer(const IndexerArgs &a, bool cq_bf16, bool w_bf16, cons
         }
     }
     return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_indexer(const IndexerArgs &a, bool cq_bf16, bool w_bf16, const CUtensorMap &kmap,
+                           const CUtensorMap &qmap, int num_sms, cudaStream_t stream, bool project) {
+    (void)num_sms;
+    if (project) {
+        if (a.NQ > 3 * a.HI) {
+            cudaError_t e = cudaMemsetAsync(a.q_ws, 0, (size_t)a.B * a.NQ * a.dI * 2, stream);
+            if (e != cudaSuccess) return e;
+        }
+        const int pblocks = (a.HI * a.dI + kProjThreads / 32 - 1) / (kProjThreads / 32);
+        const dim3 pg(pblocks, (a.B + kProjKeepB - 1) / kProjKeepB), pb(kProjThreads);
+        cudaError_t e;
+        if (a.dc <= 1024) {
+            if (cq_bf16 && w_bf16) e = launch_pdl(iq_project_kernel<__nv_bfloat16, __nv_bfloat16>, pg, pb, 0, stream, a);
+            else if (cq_bf16) e = launch_pdl(iq_project_kernel<__nv_bfloat16, float>, pg, pb, 0, stream, a);
+            else if (w_bf16) e = launch_pdl(iq_project_kernel<float, __nv_bfloat16>, pg, pb, 0, stream, a);
+            else e = launch_pdl(iq_project_kernel<float, float>, pg, pb, 0, stream, a);
+        } else {
+            if (cq_bf16 && w_bf16) e = launch_pdl(iq_project_wide_kernel<__nv_bfloat16, __nv_bfloat16>, pg, pb, 0, stream, a);
+            else if (cq_bf16) e = launch_pdl(iq_project_wide_kernel<__nv_bfloat16, float>, pg, pb, 0, stream, a);
+            else if (w_bf16) e = launch_pdl(iq_project_wide_kernel<float, __nv_bfloat16>, pg, pb, 0, stream, a);
+            else e = launch_pdl(iq_project_wide_kernel<float, float>, pg, pb, 0, stream, a);
+        }
+        if (e != cudaSuccess) return e;
+    }
+    return launch_scoring(a, kmap, qmap, stream);
+}
+
+cudaError_t launch_len_snapshot(const int32_t *slots, const int32_t *len, int B, int n_slots, int32_t *len0,
+                                cudaStream_t stream) {
+    return launch_pdl(len_snapshot_kernel, dim3((B + 255) / 256), dim3(256), 0, stream, slots, len, B, n_slots,
+                      len0);
 }
 
 }  // namespace csla

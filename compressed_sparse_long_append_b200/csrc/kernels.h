@@ -89,13 +89,18 @@ struct IndexerArgs {
     uint16_t *q_ws;     // [B][NQ][dI] bf16
     const int32_t *q_len;   // optional per-row visible length (else len[slot])
     int rows_per_cta;       // 1, or indexer_rows_per_cta(NQ) when all rows share slots[0]
+    int range;              // 0: all visible entries; 1: those below len0[b]/m; 2: those from len0[b]/m on
+    const int32_t *len0;    // [B] length of row b's request before the step's append (range 1, 2)
 };
+// len0[b] = len[slots[b]] (0 for a slot outside the pool).
+cudaError_t launch_len_snapshot(const int32_t *slots, const int32_t *len, int B, int n_slots, int32_t *len0,
+                                cudaStream_t stream);
 
 // Query rows sharing one key tile per MMA when the rows of a call all belong
 // to one request: as many as fit the UMMA N limit of 256 columns.
 __host__ __device__ constexpr int indexer_rows_per_cta(int NQ) { return 256 / NQ; }
 cudaError_t launch_indexer(const IndexerArgs &a, bool cq_bf16, bool w_bf16, const CUtensorMap &kmap,
-                           const CUtensorMap &qmap, int num_sms, cudaStream_t stream);
+                           const CUtensorMap &qmap, int num_sms, cudaStream_t stream, bool project = true);
 
 struct TopkArgs {
     const float *scores;

@@ -81,7 +81,13 @@ enum { CSLA_F32 = 0, CSLA_BF16 = 1 };
 
 enum { CSLA_VARIANT_AUTO = 0, CSLA_VARIANT_SATURATED = 1, CSLA_VARIANT_STARVED = 2 };
 
-enum { CSLA_OP_INDEXER = 1, CSLA_OP_TOPK = 2, CSLA_OP_CSA_ATTEND = 3, CSLA_OP_HCA_ATTEND = 4 };
+enum {
+    CSLA_OP_INDEXER = 1,
+    CSLA_OP_TOPK = 2,
+    CSLA_OP_CSA_ATTEND = 3,
+    CSLA_OP_HCA_ATTEND = 4,
+    CSLA_OP_CSA_DECODE_STEP = 5 /* ws_step of csla_csa_decode_step; max_len here means k */
+};
 
 /* device error word bits */
 enum {
@@ -290,6 +296,32 @@ int csla_hca_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache 
                     int32_t q_dtype, const float *sink, const float *gamma_q, void *out,
                     int32_t out_dtype, int32_t variant, void *workspace, size_t workspace_bytes,
                     csla_stream_t stream);
+
+/*
+ * csla_csa_decode_step -- one CSA decode step in one call: the same results,
+ * bit for bit, as csla_compress_append (T new tokens, no token rows), then
+ * csla_indexer_scores, csla_topk_select and csla_csa_attend on `stream`.
+ * It differs only in scheduling: the indexer scores the entries that were
+ * complete before this append on `stream` while the append runs on a side
+ * stream of the calling thread; after the join it scores the entries the
+ * append added, then top-k and attention follow.  (The pages' step order is
+ * kept for every value: an entry's score does not depend on when it is
+ * computed.)  Arguments as in the four calls; ws_indexer as for
+ * csla_indexer_scores, ws_step = csla_workspace_size(cfg,
+ * CSLA_OP_CSA_DECODE_STEP, B, k) bytes (16-byte aligned).  CSA only (m = 4).
+ * The thread's first call on a device creates its side stream and two
+ * events; make it before any stream capture (captured calls then fork and
+ * join the capture like any two-stream work).
+ */
+int csla_csa_decode_step(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
+                         const int32_t *slots, int32_t B, int32_t T, int32_t max_len, const void *kv_new,
+                         const void *kidx_new, int32_t kv_dtype, const csla_compress_params *p,
+                         const void *cq, int32_t cq_dtype, const void *W_iq, int32_t w_dtype,
+                         const float *head_w, float *scores, int32_t scores_stride, int32_t k,
+                         int32_t *idx, const void *q, int32_t q_dtype, const float *sink,
+                         const float *gamma_q, void *out, int32_t out_dtype, int32_t variant,
+                         void *ws_indexer, size_t ws_indexer_bytes, void *ws_step,
+                         size_t ws_step_bytes, csla_stream_t stream);
 
 /*
  * csla_indexer_scores_noalloc -- csla_indexer_scores for callers that cannot

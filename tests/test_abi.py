@@ -90,3 +90,5 @@ def test_workspace_sizes():
     hca = _cfg(m=128)
     assert C.csla_workspace_size(hca, C.CSLA_OP_HCA_ATTEND, 4, 1 << 20) == 4 * 32 * (64 * 512 + 128) * 4
     assert C.csla_workspace_size(_cfg(m=8), C.CSLA_OP_TOPK, 1, 1) == 0
+    # decode step: the attention partials for k, then B int32 lengths (16-byte rounded)
+    assert C.csla_workspace_size(cfg, C.CSLA_OP_CSA_DECODE_STEP, 8, 512) == 8 * 10 * (64 * 512 + 128) * 4 + 32
