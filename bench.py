@@ -381,7 +381,7 @@ class PrefillStep:
         return fi, fa
 
 
-def prefill_leg(W, K, seed, rank, world, device, variant):
+def prefill_leg(W, K, seed, rank, world, device, variant, profile=False):
     """Times the prefill chunk: one CUDA graph of the whole step (five library
     calls and the rewind copies) replayed K times between one event pair."""
     import torch
@@ -405,11 +405,15 @@ def prefill_leg(W, K, seed, rank, world, device, variant):
     g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if profile:
+        torch.cuda.profiler.start()
     e0.record()
     for _ in range(K):
         g.replay()
     e1.record()
     torch.cuda.synchronize()
+    if profile:
+        torch.cuda.profiler.stop()
     ms = dp_max(e0.elapsed_time(e1) / K, world, device)
     del g
     # per-call times: each call its own graph, one event pair around each replay
@@ -682,7 +686,7 @@ def main():
     W, K = max(3, args.warmup), args.steps
     seed = 1
     if args.prefill_only:
-        pre = prefill_leg(W, K, seed + 2, rank, world, device, args.variant)
+        pre = prefill_leg(W, K, seed + 2, rank, world, device, args.variant, profile=args.profile)
         if rank == 0:
             print(json.dumps({"csa_prefill": pre}), flush=True)
         if world > 1:
