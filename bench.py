@@ -264,7 +264,8 @@ def csa_launches(kw, variant, fused):
     (forced, or automatic: one chunk per request or B >= SM count); the
     fused step adds the length snapshot and the second indexer launch."""
     rows = kw["k"] + kw["n_win"]
-    chunks = -(-rows // (64 * -(-rows // 2048)))
+    chunk = 64 * max(-(-rows // 2048), 2 if rows > 1024 else 1)
+    chunks = -(-rows // chunk)
     saturated = variant == 1 or (variant == 0 and (kw["B"] >= 148 or chunks <= 1))
     return 2 + 2 + 1 + 1 + (0 if saturated else 1) + (2 if fused else 0)
 

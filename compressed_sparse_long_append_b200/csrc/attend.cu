@@ -53,6 +53,9 @@ constexpr int kTile = 64;        // rows per tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThresh = 8.0f;
 constexpr int kBarLoad = 1;   // named barrier of the loader warps (0 = __syncthreads)
+// K blocks widened per proxy fence: 1 measured fastest (2 and 8 were 1.4
+// and 2.5 us slower per step: the S products then start later)
+constexpr int kWidenGroup = 1;
 
 template <int D>
 struct Cfg {
@@ -396,26 +399,30 @@ __device__ void loader_role(const AttendArgs &a, int b, const Req &rq, Span sp, 
         if (ok && t > 0) ok = mbar_wait(&ms->x_empty[(t - 1) & 1], ((t - 1) >> 1) & 1, &ms->abort);
         const uint8_t *raw = smem + (buf ? C::kOffRaw1 : C::kOffRaw0);
         uint8_t *xs = smem + C::kOffX;
-        // widen K block by K block; the MMA warp starts on a block as soon
-        // as every loader thread has arrived on its barrier
+        // widen kWidenGroup K blocks at a time (one proxy fence per group);
+        // the MMA warp starts on a block as soon as every loader thread has
+        // arrived on its barrier
 #pragma unroll 1
-        for (int kb = 0; kb < C::kKB; ++kb) {
+        for (int kb0 = 0; kb0 < C::kKB; kb0 += kWidenGroup) {
             if (ok) {
-                // source chunks of this block: 4 fp8 chunks per row (nope) or
-                // 8 bf16 chunks per row (RoPE block)
-                const int cpr = kb < C::kKBN ? 4 : 8;
-                const int ch0 = kb < C::kKBN ? 4 * kb : C::kNopeCH;
+#pragma unroll 1
+                for (int kb = kb0; kb < kb0 + kWidenGroup && kb < C::kKB; ++kb) {
+                    // source chunks of this block: 4 fp8 chunks per row (nope)
+                    // or 8 bf16 chunks per row (RoPE block)
+                    const int cpr = kb < C::kKBN ? 4 : 8;
+                    const int ch0 = kb < C::kKBN ? 4 * kb : C::kNopeCH;
 #pragma unroll 4
-                for (int id = lt; id < kTile * cpr; id += kLoadThreads) {
-                    const int r = id / cpr, ch = ch0 + id % cpr;
-                    const uint4 v = ms->rawvalid[buf][r]
-                                        ? *reinterpret_cast<const uint4 *>(raw + r * C::kRB + ch * 16)
-                                        : make_uint4(0u, 0u, 0u, 0u);
-                    store_chunk<D>(xs, r, ch, v);
+                    for (int id = lt; id < kTile * cpr; id += kLoadThreads) {
+                        const int r = id / cpr, ch = ch0 + id % cpr;
+                        const uint4 v = ms->rawvalid[buf][r]
+                                            ? *reinterpret_cast<const uint4 *>(raw + r * C::kRB + ch * 16)
+                                            : make_uint4(0u, 0u, 0u, 0u);
+                        store_chunk<D>(xs, r, ch, v);
+                    }
                 }
                 fence_proxy_async_smem();
             }
-            mbar_arrive(&ms->kb_full[kb]);
+            for (int kb = kb0; kb < kb0 + kWidenGroup && kb < C::kKB; ++kb) mbar_arrive(&ms->kb_full[kb]);
         }
         if (ok) {
             if (lt < kTile) {
@@ -755,18 +762,58 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int q
     }
     if (!run) return;
     if (kSaturated) {
-        // partials written by this CTA are visible to it after the barrier above
-        __shared__ float wts[kThreads / 32][32];   // per warp: chunk weights
+        // partials written by this CTA are visible to it after the barrier
+        // above.  Every head's chunk weights first (warp-collective per head),
+        // into the staging area the loader no longer uses.
+        float *wall = reinterpret_cast<float *>(smem + C::kOffRaw0);   // [H][33]: w_0..w_31, l
         const int lane = threadIdx.x & 31;
+        const int n = rq.n_chunks;
         for (int hh = warp; hh < a.H; hh += kThreads / 32) {
             float wl, l;
-            fold_weights(a, b, rq.n_chunks, hh, D, &wl, &l);
-            wts[warp][lane] = wl;
-            __syncwarp();
-            for (int d = lane; d < D; d += 32)
-                store_out(a, out_bf16 != 0, ((size_t)b * a.H + hh) * D + d,
-                          fold_dim(a, b, rq.n_chunks, hh, d, D, wts[warp], l));
-            __syncwarp();
+            fold_weights(a, b, n, hh, D, &wl, &l);
+            wall[hh * 33 + lane] = wl;
+            if (lane == 0) wall[hh * 33 + 32] = l;
+        }
+        __syncthreads();
+        if (partial_floats(a.H, D) % 4 == 0) {
+            // (head, 128 dims) per warp, 4 consecutive dims per lane: 16-byte
+            // partial loads, 8 chunks in flight; each dim folded in chunk
+            // order exactly like fold_dim()
+            constexpr int kQ = D / 128;
+            for (int it = warp; it < a.H * kQ; it += kThreads / 32) {
+                const int hh = it / kQ, d = (it % kQ) * 128 + 4 * lane;
+                const float *w = wall + hh * 33;
+                float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+                for (int c0 = 0; c0 < n; c0 += 8) {
+                    float4 v[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        v[j] = *reinterpret_cast<const float4 *>(partial_ptr(a, b, min(c0 + j, n - 1), D) +
+                                                                 (size_t)hh * D + d);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (c0 + j < n) {
+                            const float wc = w[c0 + j];
+                            o0 = __fmaf_rn(v[j].x, wc, o0);
+                            o1 = __fmaf_rn(v[j].y, wc, o1);
+                            o2 = __fmaf_rn(v[j].z, wc, o2);
+                            o3 = __fmaf_rn(v[j].w, wc, o3);
+                        }
+                    }
+                }
+                const float l = w[32];
+                const size_t base = ((size_t)b * a.H + hh) * D + d;
+                store_out(a, out_bf16 != 0, base, __fdiv_rn(o0, l));
+                store_out(a, out_bf16 != 0, base + 1, __fdiv_rn(o1, l));
+                store_out(a, out_bf16 != 0, base + 2, __fdiv_rn(o2, l));
+                store_out(a, out_bf16 != 0, base + 3, __fdiv_rn(o3, l));
+            }
+        } else {
+            // odd head counts: partial records are not 16-byte multiples
+            for (int hh = warp; hh < a.H; hh += kThreads / 32)
+                for (int d = lane; d < D; d += 32)
+                    store_out(a, out_bf16 != 0, ((size_t)b * a.H + hh) * D + d,
+                              fold_dim(a, b, n, hh, d, D, wall + hh * 33, wall[hh * 33 + 32]));
         }
     }
 }

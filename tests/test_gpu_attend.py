@@ -83,6 +83,7 @@ def _oracle_idx(w, cv, s, L, si, p):
 @pytest.mark.parametrize("w,lens", [
     (CSA_SMALL, [2048, 300, 5]),
     (CSA_BIG, [6000, 130]),
+    (dataclasses.replace(CSA_SMALL, H=5, name="att_csa_h5"), [2048, 77]),   # odd head count
 ])
 def test_csa_attend_matches_oracle(w, lens):
     cv, p = oracle_cache(w, lens)
