@@ -198,9 +198,7 @@ __global__ void __launch_bounds__(kProjThreads) iq_project_wide_kernel(IndexerAr
     }
 }
 
-// Key-tile ring depth (5 for grouped query rows measured no faster than 3).
-template <int G>
-constexpr int idx_stages() { return 3; }
+constexpr int kStages = 3;
 constexpr int kTileE = 128;          // entries per tile
 constexpr int kPageE = 32;           // CSA entries per 128-token page
 constexpr int kTPC = 8;              // tiles per CTA (consecutive, one request)
@@ -215,9 +213,7 @@ template <int DI, int NQ, int G>
 struct IdxSmem {
     static constexpr int kKeyBytes = kTileE * DI * 2;
     static constexpr int kQBytes = G * NQ * DI * 2;
-    static constexpr int kStages = idx_stages<G>();
     static constexpr int kBytes = kStages * kKeyBytes + kQBytes + 1024 /*align*/ + 1024 /*barriers, pages, weights*/;
-    static_assert(kBytes <= 232448, "shared memory budget");
 };
 
 // Two accumulators of G*NQ columns, rounded up to a power of two >= 32.
@@ -237,7 +233,6 @@ __global__ void __launch_bounds__(idx_threads<G>())
     CSLA_TL_SCOPE(kTlIndexer);
     using S = IdxSmem<DI, NQ, G>;
     constexpr int N = G * NQ;
-    constexpr int kStages = S::kStages;
     static_assert(N % 16 == 0 && N <= 256, "UMMA N for M = 128");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
