@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--no-hca", action="store_true", help="skip the HCA layer measurement")
     ap.add_argument("--no-prefill", action="store_true", help="skip the CSA prefill-chunk measurement")
     ap.add_argument("--prefill-only", action="store_true", help="only the CSA prefill-chunk measurement")
+    ap.add_argument("--no-invariance", action="store_true",
+                    help="skip the ragged 64-request CSA + HCA decode measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", type=int, default=0, help="attention variant: 0 auto, 1 saturated, 2 starved")
     ap.add_argument("--fused-step", action="store_true",
@@ -447,6 +449,55 @@ def prefill_leg(W, K, seed, rank, world, device, variant, profile=False):
     return out
 
 
+def invariance_leg(W, K, seed, rank, world, device, variant):
+    """The batch-invariance workload as a throughput number: 64 requests
+    with contexts log-uniform in [1K, 1M] tokens (the lengths of the
+    invariance test), one decode step = a CSA layer step (top-k 512) and an
+    HCA layer step for all 64 requests, one CUDA graph per step.  Caches are
+    built by csla_compress_append; they are GBs, far larger than L2."""
+    import math
+    import torch
+    from csla_synth import uniform
+    u = uniform(5, "invariance/len", (64,))
+    lens = [int(math.exp(math.log(1024) + x * math.log(1024))) for x in u]
+    B = len(lens)
+    before = W + K
+    L0s = [L - before for L in lens]
+    ck = dict(CSA, B=B, L=max(lens))
+    hk = dict(HCA, B=B, L=max(lens))
+    clb, ccp, cpar = build_layer(ck, B, L0s, seed, rank, device)
+    hlb, hcp, hpar = build_layer(hk, B, L0s, seed + 1, rank, device)
+    cin = step_inputs(ck, B, W + K, seed, rank, device)
+    hin = step_inputs(hk, B, W + K, seed + 1, rank, device)
+    cs = CsaStep(clb, ccp, cpar, ck, variant, device)
+    hs = HcaStep(hlb, hcp, hpar, hk, variant, device)
+    for i in range(W):
+        for c in cs.calls:
+            c(cin[i])
+        for c in hs.calls:
+            c(hin[i])
+    torch.cuda.synchronize()
+    graphs = []
+    for i in range(W, W + K):
+        graphs.append(capture(lambda: ([c(cin[i]) for c in cs.calls], [c(hin[i]) for c in hs.calls])))
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for g in graphs:
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = dp_max(e0.elapsed_time(e1) / K, world, device)
+    del graphs
+    out = {"workload": "invariance_64req_L1K-1M_csa_hca", "tokens_per_s": B * world / (ms * 1e-3),
+           "ms_per_step": ms, "requests_per_gpu": B, "context_tokens": sum(lens), "context_min": min(lens),
+           "context_max": max(lens), "step": "one CSA layer (top-k 512) + one HCA layer, all requests",
+           "l2": "inputs larger than L2 (CSA index keys alone ~600 MB per step)"}
+    del cs, hs, clb, hlb, cin, hin
+    torch.cuda.empty_cache()
+    return out
+
+
 def clone_layer(lb, params):
     """An independent copy of a layer's device buffers and weights (the
     rotation below walks several such copies, like the layers of a model)."""
@@ -770,6 +821,12 @@ def main():
             del steps, lb
             torch.cuda.empty_cache()
         pre = prefill_leg(W, K, seed + 2, rank, world, device, args.variant)
+    inv = None
+    if not args.no_invariance and not args.profile:
+        if args.no_hca and args.no_prefill:
+            del steps, lb
+            torch.cuda.empty_cache()
+        inv = invariance_leg(W, K, seed + 4, rank, world, device, args.variant)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -814,6 +871,7 @@ def main():
             "clocks": clocks,
             "hca_decode": hca,
             "csa_prefill": pre,
+            "invariance_decode": inv,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
