@@ -71,7 +71,6 @@ struct Cfg {
     static constexpr int kQBytes = kKB * kQKB;
     static constexpr int kPBytes = kHP * kTile * 2;
     static constexpr int kTasks = kTile * kCH;         // 16-byte chunks per tile
-    static constexpr int kTPT = kTasks / kLoadThreads; // chunks widened per loader thread
     static_assert(kTasks % kLoadThreads == 0, "tile split");
     static constexpr int kRawBytes = kTile * kRB;      // one staged tile of raw rows
     // TMEM columns
@@ -134,14 +133,6 @@ __device__ __forceinline__ Req request(const AttendArgs &a, int b) {
     r.chunk = attend_chunk_rows(r.n_rows);
     r.n_chunks = r.ok ? attend_num_chunks(r.n_rows) : 0;
     return r;
-}
-
-__device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
 }
 
 __device__ __forceinline__ void named_sync(int id, int n) {

@@ -217,8 +217,9 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
     CSLA_TL_MARK(6);
 }
 
-// ---------------------------------------------------------------- register variant
-// For n <= kRegMax, one CTA of 512 threads.  Warp w owns the contiguous
+// ---------------------------------------------------------------- selection with scores in registers
+// The steps, as first written for one CTA of 512 threads (the cluster
+// kernel below spreads them over 4 CTAs).  Warp w owns the contiguous
 // range [w*seg, (w+1)*seg), seg = ceil(n / 16); lane l holds the scores
 // w*seg + 32j + l (j < kPer) in registers, so a warp's ballots walk its
 // range in index order.
@@ -380,190 +381,11 @@ __device__ uint32_t radix_select(RegShared &sh, const Each &each, int rank, uint
     return prefix;
 }
 
-__global__ void __launch_bounds__(kRThreads, 1) topk_reg_kernel(TopkArgs a) {
-    CSLA_TL_SCOPE(kTlTopk);
-    extern __shared__ __align__(16) uint8_t dyn_raw[];
-    RegShared &sh = *reinterpret_cast<RegShared *>(dyn_raw);
-    pdl_trigger();
-    const int b = blockIdx.x;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int slot = __ldg(a.slots + b);
-    const bool slot_ok = slot >= 0 && slot < a.n_slots;
-    pdl_wait();
-    CSLA_TL_WAITED();
-    const int L = slot_ok ? row_visible_len(a.len, a.q_len, slot, b) : 0;
-    int n = L < 0 ? 0 : L / a.m;
-    if (!slot_ok || L < 0 || L / a.m > a.max_n) {
-        if (threadIdx.x == 0) set_dev_err(CSLA_DEVERR_LEN);
-        n = 0;
-    }
-    const int k = a.k;
-    int32_t *out = a.idx + (size_t)b * k;
-    if (n <= k) {
-        for (int j = threadIdx.x; j < k; j += kRThreads) out[j] = j < n ? j : -1;
-        return;
-    }
-    const float *sc = a.scores + (size_t)b * a.stride;
-    const int seg = (n + kRWarps - 1) / kRWarps;
-    const int base = warp * seg;
-    float f[kPer];
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-        const int r = 32 * j + lane, i = base + r;
-        f[j] = (r < seg && i < n) ? sc[i] : __int_as_float(-1);   // the NaN whose key is 0: padding
-    }
-    CSLA_TL_MARK(0);
-
-    // ---- 1. threshold: per-warp sorted sample, smallest rw-th largest over warps
-    // lane l samples row js = l * rows / 32 of the warp's range (rows = ceil(seg / 32))
-    const int js = (lane * ((seg + 31) >> 5)) >> 5;
-    uint32_t smp = 0;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j)
-        if (j == js) smp = score_key(f[j]);
-#pragma unroll
-    for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            const uint32_t o = __shfl_xor_sync(0xffffffffu, smp, stride);
-            const bool desc = (lane & size) == 0 || size == 32;
-            const bool lower = (lane & stride) == 0;
-            smp = (lower == desc) ? max(smp, o) : min(smp, o);
-        }
-    }
-    // each warp keeps >= rw samples >= t0, so in expectation >= rw * n / 32 keys are >= t0
-    const int rw = min(32, (int)((48LL * k + n - 1) / n));
-    const uint32_t s_w = __shfl_sync(0xffffffffu, smp, rw - 1);
-    if (lane == 0) sh.tw[warp] = s_w;
-    __syncthreads();
-    uint32_t t0 = lane < kRWarps ? sh.tw[lane] : 0xFFFFFFFFu;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) t0 = min(t0, __shfl_xor_sync(0xffffffffu, t0, o));
-    CSLA_TL_MARK(1);
-
-    // ---- 2. candidates: scores >= the value of t0 (padding, a NaN, never
-    // qualifies; t0 = 0 admits every real score) into this warp's region
-    const float f0 = t0 == 0u ? -INFINITY : key_value(t0);
-    int pos = 0;
-    uint32_t cmax = 0;
-    const unsigned below = (1u << lane) - 1u;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-        const bool q = f[j] >= f0;
-        const unsigned mq = __ballot_sync(0xffffffffu, q);
-        const int at = pos + __popc(mq & below);
-        if (q && at < kRegion) {
-            const uint32_t key = score_key(f[j]);
-            sh.ckey[warp][at] = key;
-            sh.cidx[warp][at] = base + 32 * j + lane;
-            cmax = max(cmax, key);
-        }
-        pos += __popc(mq);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
-    if (lane == 0) {
-        sh.cnt[warp] = pos;
-        sh.tw[warp] = cmax;
-    }
-    __syncthreads();
-    int n_ge;
-    warp_prefix(sh.cnt, warp, &n_ge);
-    bool fits = true;
-#pragma unroll
-    for (int w = 0; w < kRWarps; ++w) fits &= sh.cnt[w] <= kRegion;
-    CSLA_TL_MARK(2);
-
-    int krem;
-    if (fits && n_ge >= k) {
-        const int my_n = sh.cnt[warp];
-        // every candidate lies in [t0, kmax]: they share the top clz(t0 ^ kmax) bits
-        uint32_t kmax = lane < kRWarps ? sh.tw[lane] : 0u;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-        const int bits = 32 - __clz(t0 ^ kmax);
-        const uint32_t T = radix_select(sh, [&](auto fn) {
-            for (int i = lane; i < my_n; i += 32) fn(sh.ckey[warp][i]);
-        }, k, kmax, bits, &krem);
-        CSLA_TL_MARK(3);
-        // ---- 3. output from the regions (index order within and across warps)
-        int gt = 0, eq = 0;
-        for (int i = lane; i < my_n; i += 32) {
-            const uint32_t key = sh.ckey[warp][i];
-            gt += key > T;
-            eq += key == T;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            gt += __shfl_xor_sync(0xffffffffu, gt, o);
-            eq += __shfl_xor_sync(0xffffffffu, eq, o);
-        }
-        if (lane == 0) {
-            sh.warp_a[warp] = gt;
-            sh.warp_b[warp] = eq;
-        }
-        __syncthreads();
-        int tot;
-        const int gt_before = warp_prefix(sh.warp_a, warp, &tot);
-        const int eq_before = warp_prefix(sh.warp_b, warp, &tot);
-        int opos = gt_before + min(eq_before, krem);
-        int eq_seen = eq_before;
-        for (int i0 = 0; i0 < my_n; i0 += 32) {
-            const int i = i0 + lane;
-            const uint32_t key = i < my_n ? sh.ckey[warp][i] : 0u;
-            const bool is_gt = i < my_n && key > T;
-            const bool is_eq = i < my_n && key == T;
-            const unsigned meq = __ballot_sync(0xffffffffu, is_eq);
-            const bool take_eq = is_eq && (eq_seen + __popc(meq & below)) < krem;
-            const unsigned mtake = __ballot_sync(0xffffffffu, is_gt || take_eq);
-            if (is_gt || take_eq) out[opos + __popc(mtake & below)] = sh.cidx[warp][i];
-            opos += __popc(mtake);
-            eq_seen += __popc(meq);
-        }
-    } else {
-        const uint32_t T = radix_select(sh, [&](auto fn) {
-#pragma unroll
-            for (int j = 0; j < kPer; ++j) fn(score_key(f[j]));
-        }, k, 0u, 32, &krem);
-        CSLA_TL_MARK(3);
-        int gt = 0, eq = 0;
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            const uint32_t key = score_key(f[j]);
-            gt += __popc(__ballot_sync(0xffffffffu, key > T));
-            eq += __popc(__ballot_sync(0xffffffffu, key == T));
-        }
-        if (lane == 0) {
-            sh.warp_a[warp] = gt;
-            sh.warp_b[warp] = eq;
-        }
-        __syncthreads();
-        int tot;
-        const int gt_before = warp_prefix(sh.warp_a, warp, &tot);
-        const int eq_before = warp_prefix(sh.warp_b, warp, &tot);
-        int opos = gt_before + min(eq_before, krem);
-        int eq_seen = eq_before;
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            const uint32_t key = score_key(f[j]);
-            const bool is_gt = key > T;
-            const bool is_eq = key == T;
-            const unsigned meq = __ballot_sync(0xffffffffu, is_eq);
-            const bool take_eq = is_eq && (eq_seen + __popc(meq & below)) < krem;
-            const unsigned mtake = __ballot_sync(0xffffffffu, is_gt || take_eq);
-            if (is_gt || take_eq) out[opos + __popc(mtake & below)] = base + 32 * j + lane;
-            opos += __popc(mtake);
-            eq_seen += __popc(meq);
-        }
-    }
-    CSLA_TL_MARK(4);
-}
-
 // ---------------------------------------------------------------- cluster variant
 // For n <= kRegMax: one cluster of kG = 4 CTAs (512 threads each) per
 // request; CTA c owns the c-th quarter of the scores, warp w of it a
 // contiguous range, lane l the scores 32j + l of that range (18 rows) in
-// registers.  The steps of the register variant, spread over the cluster:
+// registers.  The steps above, spread over the cluster:
 //  1. every warp sorts a 32-key sample of its range and publishes its
 //     2nd-largest key; after a cluster barrier every CTA reads all 64 and
 //     takes the j-th largest as the threshold t0 (j = ceil(2048k/n), at
@@ -575,7 +397,7 @@ __global__ void __launch_bounds__(kRThreads, 1) topk_reg_kernel(TopkArgs a) {
 //     their exclusive-prefix offsets (so CTA 0 holds all candidates in
 //     index order);
 //  3. after a third barrier CTA 0 finds the exact k-th key among the
-//     candidates and writes the output, as the register variant does.
+//     candidates and writes the output, as in the steps above.
 // Otherwise (rare: heavy ties, or a sample far off) all four CTAs run the
 // radix select over every key with their four histograms summed through
 // distributed shared memory, and each writes its own picks.
@@ -866,8 +688,6 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
                                              (int)(kHistBytes + kSmemKeysMax * sizeof(uint32_t)));
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kHistBytes);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(topk_reg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RegShared));
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sizeof(ClShared));
