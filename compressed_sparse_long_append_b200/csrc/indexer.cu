@@ -202,10 +202,11 @@ constexpr int kStages = 3;
 constexpr int kTileE = 128;          // entries per tile
 constexpr int kPageE = 32;           // CSA entries per 128-token page
 constexpr int kTPC = 8;              // tiles per CTA (consecutive, one request)
-// warp 0: TMA, warp 1: MMA, then 4 epilogue warps per set of query rows:
-// one set for G = 1, four (rows g, g + 4, ... of the group) for G > 1
+// warp 0: TMA, warp 1: MMA, then 4 epilogue warps per set of query rows
+// (set s takes the group's rows s, s + sets, ...): one set for G = 1, one
+// per row up to 7 rows (balanced: 5 at 16 index heads), else four.
 template <int G>
-constexpr int idx_epi_sets() { return G > 1 ? 4 : 1; }
+constexpr int idx_epi_sets() { return G == 1 ? 1 : (G <= 7 ? G : 4); }
 template <int G>
 constexpr int idx_threads() { return 64 + 128 * idx_epi_sets<G>(); }
 
