@@ -209,6 +209,68 @@ __device__ void pool_block(const BlockRows<T> &x, int m, const float *wsm, float
     __syncthreads();
 }
 
+// pool_block for blocks of at most kSmallM rows (CSA, m = 4), in registers:
+// thread t < width/4 holds columns 4t..4t+3 of every row (one load round
+// trip), its partial gate products go through one block reduction (warp
+// butterfly, then the warps in order), every thread forms the softmax
+// weights itself, and its pooled columns (rows in order) go to out (smem).
+// Two barriers instead of the staged path's ten.
+constexpr int kSmallM = 4;
+template <typename T>
+__device__ void pool_small(const BlockRows<T> &x, int m, const float *wsm, const float *bias, float *red8,
+                           float *out) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nq = x.width >> 2;
+    const bool act = threadIdx.x < nq;
+    float4 xv[kSmallM];
+#pragma unroll
+    for (int i = 0; i < kSmallM; ++i)
+        xv[i] = (act && i < m) ? x.get(i, threadIdx.x) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 w = act ? reinterpret_cast<const float4 *>(wsm)[threadIdx.x] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < kSmallM; ++i) {
+        float p = __fmul_rn(xv[i].x, w.x);
+        p = __fmaf_rn(xv[i].y, w.y, p);
+        p = __fmaf_rn(xv[i].z, w.z, p);
+        p = __fmaf_rn(xv[i].w, w.w, p);
+        p = warp_sum(p);
+        if (lane == 0) red8[warp * kSmallM + i] = p;
+    }
+    __syncthreads();
+    CSLA_TL_MARK(4);
+    float al[kSmallM];
+    float gmax = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kSmallM; ++i) {
+        float g = 0.f;
+#pragma unroll
+        for (int q = 0; q < kWarps; ++q) g = __fadd_rn(g, red8[q * kSmallM + i]);
+        al[i] = __fadd_rn(g, i < m ? bias[i] : 0.f);
+        if (i < m) gmax = fmaxf(gmax, al[i]);
+    }
+    float zs = 0.f;
+#pragma unroll
+    for (int i = 0; i < kSmallM; ++i) {
+        al[i] = i < m ? expf(__fsub_rn(al[i], gmax)) : 0.f;
+        zs = __fadd_rn(zs, al[i]);
+    }
+    if (act) {
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < kSmallM; ++i) {
+            if (i < m) {
+                const float a = __fdiv_rn(al[i], zs);
+                o.x = __fmaf_rn(a, xv[i].x, o.x);
+                o.y = __fmaf_rn(a, xv[i].y, o.y);
+                o.z = __fmaf_rn(a, xv[i].z, o.z);
+                o.w = __fmaf_rn(a, xv[i].w, o.w);
+            }
+        }
+        reinterpret_cast<float4 *>(out)[threadIdx.x] = o;
+    }
+    __syncthreads();
+}
+
 // kTok: the call also keeps every new token's window row (CompressArgs::tok_rows).
 template <typename T, bool kTok>
 __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs a) {
@@ -323,7 +385,8 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs 
         const T *fresh = reinterpret_cast<const T *>(a.kv_new) + ((size_t)b * a.T + f0) * D;
         const BlockRows<T> rows{a.tail_kv + (size_t)slot * m * D, fresh, n_tail, D,
                                 (reinterpret_cast<uintptr_t>(a.kv_new) & vec_mask) == 0};
-        pool_block<T>(rows, m, wsm, alpha, part, xs, v, red);
+        if (m <= kSmallM) pool_small<T>(rows, m, wsm, alpha, part, v);
+        else pool_block<T>(rows, m, wsm, alpha, part, xs, v, red);
         CSLA_TL_MARK(1);
         norm_rope_quantise(v, gam, a, p0, a.rows + ent * rb, a.scales + ent, red);
         CSLA_TL_MARK(2);
@@ -332,7 +395,8 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs 
         const T *fresh = reinterpret_cast<const T *>(a.kidx_new) + ((size_t)b * a.T + f0) * dI;
         const BlockRows<T> rows{a.tail_idx + (size_t)slot * m * dI, fresh, n_tail, dI,
                                 (reinterpret_cast<uintptr_t>(a.kidx_new) & vec_mask) == 0};
-        pool_block<T>(rows, m, wsm, alpha, part, xs, v, red);
+        if (m <= kSmallM) pool_small<T>(rows, m, wsm, alpha, part, v);
+        else pool_block<T>(rows, m, wsm, alpha, part, xs, v, red);
         CSLA_TL_MARK(1);
         for (int e = threadIdx.x; e < dI; e += kThreads) a.kidx[ent * dI + e] = f32_to_bf16_bits(v[e]);
         CSLA_TL_MARK(2);
