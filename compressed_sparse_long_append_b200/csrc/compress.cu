@@ -39,41 +39,65 @@ __device__ __forceinline__ float load_act<__nv_bfloat16>(const __nv_bfloat16 *p,
 
 // RMSNorm(v) * gamma, partial RoPE at `pos`, quantise into one cache row
 // (kTwo: also into a second copy `row2`, when not null).  v, gam: smem [D]
-// (v overwritten); red: smem scratch.  The rotation angles are taken first
-// so their latency overlaps the reductions.
+// (read only); red: smem scratch.  Thread t works on dims t and t + 256 in
+// registers; a RoPE pair (d, d + 1) sits in lanes t, t ^ 1 and is rotated
+// through a shuffle.  The rotation angles are taken first so their latency
+// overlaps the reductions.  Per dim the same operations, in the same order,
+// as the norm, rotation and scaling written out one after the other.
 template <bool kTwo = false>
 __device__ void norm_rope_quantise(float *v, const float *gam, const CompressArgs &a, long long pos, uint8_t *row,
                                    float *scale_out, float *red, uint8_t *row2 = nullptr,
                                    float *scale2 = nullptr) {
+    constexpr int kE = 2;   // dims per thread (D <= 512)
     const int D = a.D, dr = a.d_rope, dn = D - dr;
-    float c = 1.f, s = 0.f;
-    if (threadIdx.x < dr / 2) rope_cos_sin(pos, a.freq.inv[threadIdx.x], &c, &s);
+    float x[kE];
+    bool has[kE], rot[kE];
+    float c[kE], sn[kE];
+#pragma unroll
+    for (int e = 0; e < kE; ++e) {
+        const int d = threadIdx.x + kThreads * e;
+        has[e] = d < D;
+        rot[e] = has[e] && d >= dn;
+        c[e] = 1.f;
+        sn[e] = 0.f;
+        if (rot[e]) rope_cos_sin(pos, a.freq.inv[(d - dn) >> 1], &c[e], &sn[e]);
+        x[e] = has[e] ? v[d] : 0.f;
+    }
     float ss = 0.f;
-    for (int d = threadIdx.x; d < D; d += kThreads) ss = __fmaf_rn(v[d], v[d], ss);
+#pragma unroll
+    for (int e = 0; e < kE; ++e)
+        if (has[e]) ss = __fmaf_rn(x[e], x[e], ss);
     ss = block_sum<kWarps>(ss, red);
     const float r = 1.0f / sqrtf(__fdiv_rn(ss, (float)D) + a.eps);
-    for (int d = threadIdx.x; d < D; d += kThreads) v[d] = __fmul_rn(__fmul_rn(v[d], r), gam[d]);
-    __syncthreads();
-    if (threadIdx.x < dr / 2) {
-        const int i = threadIdx.x;
-        const float x0 = v[dn + 2 * i], x1 = v[dn + 2 * i + 1];
-        v[dn + 2 * i] = __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, s));
-        v[dn + 2 * i + 1] = __fadd_rn(__fmul_rn(x0, s), __fmul_rn(x1, c));
-    }
-    __syncthreads();
     float amax = 0.f;
-    for (int d = threadIdx.x; d < dn; d += kThreads) amax = fmaxf(amax, fabsf(v[d]));
+#pragma unroll
+    for (int e = 0; e < kE; ++e) {
+        const int d = threadIdx.x + kThreads * e;
+        const float y = has[e] ? __fmul_rn(__fmul_rn(x[e], r), gam[d]) : 0.f;
+        const float o = __shfl_xor_sync(0xffffffffu, y, 1);   // the other dim of a RoPE pair
+        if (rot[e]) {
+            x[e] = (d & 1) == 0 ? __fsub_rn(__fmul_rn(y, c[e]), __fmul_rn(o, sn[e]))
+                                : __fadd_rn(__fmul_rn(o, sn[e]), __fmul_rn(y, c[e]));
+        } else {
+            x[e] = y;
+            if (has[e]) amax = fmaxf(amax, fabsf(y));
+        }
+    }
     amax = block_max<kWarps>(amax, red);
     const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-    for (int d = threadIdx.x; d < dn; d += kThreads) {
-        const uint8_t c = f32_to_e4m3(__fdiv_rn(v[d], scale));
-        row[d] = c;
-        if (kTwo && row2) row2[d] = c;
-    }
-    for (int d = threadIdx.x; d < dr; d += kThreads) {
-        const uint16_t h = f32_to_bf16_bits(v[dn + d]);
-        reinterpret_cast<uint16_t *>(row + dn)[d] = h;
-        if (kTwo && row2) reinterpret_cast<uint16_t *>(row2 + dn)[d] = h;
+#pragma unroll
+    for (int e = 0; e < kE; ++e) {
+        const int d = threadIdx.x + kThreads * e;
+        if (!has[e]) continue;
+        if (d < dn) {
+            const uint8_t q = f32_to_e4m3(__fdiv_rn(x[e], scale));
+            row[d] = q;
+            if (kTwo && row2) row2[d] = q;
+        } else {
+            const uint16_t h = f32_to_bf16_bits(x[e]);
+            reinterpret_cast<uint16_t *>(row + dn)[d - dn] = h;
+            if (kTwo && row2) reinterpret_cast<uint16_t *>(row2 + dn)[d - dn] = h;
+        }
     }
     if (threadIdx.x == 0) {
         *scale_out = scale;
