@@ -693,6 +693,75 @@ def cpu_baseline(n_steps=3):
     return times
 
 
+def _filled_cache(m, D, n_entries, L, seed, dI=0):
+    """Oracle cache view of one request whose entries (and window rows) are
+    quantised rows of N(0,1) content through RMSNorm and RoPE at their
+    positions, the distribution the compressor produces; index keys bf16
+    N(0,1).  What a step costs does not depend on how the rows were made."""
+    import numpy as np
+    import oracle
+    from csla_synth import normal, to_bf16_bits
+    epp = 128 // m
+    pages = -(-n_entries // epp)
+    gamma = (1.0 + 0.1 * normal(seed, "cpu/gamma", (D,))).astype(np.float32).astype(np.float64)
+    rb = oracle.row_bytes(D)
+    rows = np.zeros((pages, epp, rb), np.uint8)
+    scales = np.zeros((pages, epp), np.float32)
+    x = normal(seed, "cpu/rows", (n_entries, D))
+    for e in range(n_entries):
+        rows[e // epp, e % epp], scales[e // epp, e % epp] = oracle.window_row(x[e], gamma, e * m)
+    win = np.zeros((1, 128, rb), np.uint8)
+    wsc = np.zeros((1, 128), np.float32)
+    xw = normal(seed, "cpu/win", (128, D))
+    for i, p in enumerate(range(L - 128, L)):
+        win[0, p % 128], wsc[0, p % 128] = oracle.window_row(xw[i], gamma, p)
+    kidx = to_bf16_bits(normal(seed, "cpu/kidx", (pages, epp, dI))) if dI else None
+    bt = np.arange(pages, dtype=np.int32).reshape(1, pages)
+    return oracle.CacheView(m, D, rows, scales, bt, win, wsc, kidx, dI)
+
+
+def cpu_baseline_hca(n_steps=3):
+    """fp64 oracle decode steps of one request of the HCA workload (context
+    2^20 - 64: 8191 entries + 128 window rows per step); seconds per step."""
+    import oracle
+    from csla_synth import normal
+    kw, seed = HCA, 2
+    L = kw["L"] - 64
+    cv = _filled_cache(kw["m"], kw["D"], L // kw["m"], L, seed)
+    sink = normal(seed, "sink", (kw["H"],))
+    gq = 1.0 + 0.1 * normal(seed, "gamma_q", (kw["D"],))
+    times = []
+    for s_ in range(n_steps):
+        q = normal(seed, "cpu/q/%d" % s_, (1, kw["H"], kw["D"]))
+        t0 = time.perf_counter()
+        oracle.hca_decode(cv, [0], [L], q, gq, sink)
+        times.append(time.perf_counter() - t0)
+    return times
+
+
+def cpu_baseline_prefill(n_q=16):
+    """fp64 oracle on a sample of the prefill chunk's queries (n_q of the
+    4096, spread over the chunk; each query = indexer over its ~66K visible
+    entries, top-k 1024, attention over 1152 rows), the oracle's threads
+    across queries.  Returns (seconds for the sample, threads)."""
+    import numpy as np
+    import oracle
+    from csla_synth import normal
+    kw, seed = PREFILL, 4
+    L1 = kw["L0"] + kw["T"]
+    cv = _filled_cache(kw["m"], kw["D"], L1 // kw["m"], L1, seed, dI=kw["dI"])
+    W = normal(seed, "W_iq_cpu", (kw["HI"] * kw["dI"], kw["dc"]), std=1.0 / kw["dc"] ** 0.5)
+    sink = normal(seed, "sink", (kw["H"],))
+    gq = 1.0 + 0.1 * normal(seed, "gamma_q", (kw["D"],))
+    lens = [kw["L0"] + 1 + (i * kw["T"]) // n_q for i in range(n_q)]
+    q = normal(seed, "cpu/pq", (n_q, kw["H"], kw["D"]))
+    cq = normal(seed, "cpu/pcq", (n_q, kw["dc"]))
+    hw = normal(seed, "cpu/phw", (n_q, kw["HI"]))
+    t0 = time.perf_counter()
+    oracle.csa_decode(cv, np.zeros(n_q, np.int32), lens, q, gq, cq, W, hw, sink, kw["HI"], kw["k"])
+    return time.perf_counter() - t0, min(n_q, oracle.num_threads())
+
+
 def run_reference(args):
     t_setup = time.perf_counter()
     times = cpu_baseline(n_steps=args.warmup + args.steps)
@@ -812,6 +881,15 @@ def main():
                "attend_tflops": hflops / (hms_att * 1e-3) / 1e12,
                "attend_tensor_frac_sustained": hflops / (hms_att * 1e-3) / 1e12 / 1395.7,
                "block_closes_in_timed_steps": closes}
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            try:
+                ht = cpu_baseline_hca(3)
+                hca["cpu_baseline"] = {"value": 1.0 / (sum(ht) / len(ht)), "unit": UNIT, "cores": 1, "kind": "oracle",
+                                       "sample": "1 request of this workload (context 2^20 - 64, 8191 entries + "
+                                                 "128 window rows), 3 decode steps, fp64 oracle, single thread"}
+            except Exception as e:  # the baseline never blocks the GPU line
+                hca["cpu_baseline"] = {"value": None, "unit": UNIT, "cores": 0, "kind": "oracle",
+                                       "sample": "failed: %s" % e}
         del hsteps, hlb, hin
         torch.cuda.empty_cache()
 
@@ -821,6 +899,15 @@ def main():
             del steps, lb
             torch.cuda.empty_cache()
         pre = prefill_leg(W, K, seed + 2, rank, world, device, args.variant)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            try:
+                pt, thr = cpu_baseline_prefill(16)
+                pre["cpu_baseline"] = {"value": 16 / pt, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                                       "sample": "16 of the chunk's 4096 queries (spread over it) against a "
+                                                 "cache of the same size, fp64 oracle, threads across queries"}
+            except Exception as e:  # the baseline never blocks the GPU line
+                pre["cpu_baseline"] = {"value": None, "unit": "tokens/s", "cores": 0, "kind": "oracle",
+                                       "sample": "failed: %s" % e}
     inv = None
     if not args.no_invariance and not args.profile:
         if args.no_hca and args.no_prefill:
