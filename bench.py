@@ -548,7 +548,10 @@ def run_steps(steps, inputs, W, K, e2e=False, profile=False):
     K replays are bracketed by one pair of events after a synchronize.
     e2e: every step also copies its inputs from pinned host memory into the
     device buffers the graph reads and copies its output back to pinned
-    host memory, both inside the timed region.  Returns ms per step."""
+    host memory, all inside the timed region; the copies run on a second
+    stream, step i+1's inputs while step i computes (each step has its own
+    input buffers, and an output buffer is reused only R steps later), as a
+    serving loop would.  Returns ms per step."""
     import torch
     R = len(steps)
     for i in range(W):
@@ -565,17 +568,39 @@ def run_steps(steps, inputs, W, K, e2e=False, profile=False):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if profile:
         torch.cuda.profiler.start()
-    e0.record()
-    for j, i in enumerate(range(W, W + K)):
-        if e2e:
-            x = inputs[i]
-            for k, v in x["host"].items():
-                x[k].copy_(v, non_blocking=True)
+    main = torch.cuda.current_stream()
+    e0.record(main)
+    if e2e:
+        cs = torch.cuda.Stream()
+        cs.wait_stream(main)   # every copy after the start event
+        ev_in = [torch.cuda.Event() for _ in range(K)]
+        ev_out = [torch.cuda.Event() for _ in range(K)]
+
+        def h2d(j):
+            x = inputs[W + j]
+            with torch.cuda.stream(cs):
+                for k, v in x["host"].items():
+                    x[k].copy_(v, non_blocking=True)
+                ev_in[j].record(cs)
+
+        def d2h(j):
+            with torch.cuda.stream(cs):
+                cs.wait_event(ev_out[j])
+                outs[j].copy_(steps[(W + j) % R].out, non_blocking=True)
+
+        h2d(0)
+        for j in range(K):
+            if j + 1 < K:
+                h2d(j + 1)
+            main.wait_event(ev_in[j])
             graphs[j].replay()
-            outs[j].copy_(steps[i % R].out, non_blocking=True)
-        else:
+            ev_out[j].record(main)
+            d2h(j)
+        main.wait_stream(cs)   # the last output is on the host
+    else:
+        for j in range(K):
             graphs[j].replay()
-    e1.record()
+    e1.record(main)
     torch.cuda.synchronize()
     if profile:
         torch.cuda.profiler.stop()
