@@ -235,8 +235,8 @@ int csla_window_rows(const csla_cfg *cfg, const csla_state *st, const int32_t *s
 /*
  * csla_indexer_scores -- lightning indexer (硅星人 §两大压缩注意力, CSA part:
  * the query latent dc is up-projected to HI index heads and scored with ReLU
- * against the compressed index keys).  For request b with N_vis = len/m
- * visible entries:
+ * against the compressed index keys).  For row b with N_vis = L/m visible
+ * entries (L = len[slots[b]], or q_len[b] with qs; see csla_queries):
  *   qI = W_iq . cq[b]  ([HI*dI] = [HI*dI][dc] . [dc], fp32 accumulation),
  *   scores[b*scores_stride + s] = sum_j head_w[b][j] * max(0, <qI_j, kidx_s>)
  * for s < N_vis (entries beyond N_vis are not written).  qI enters the tensor
@@ -244,6 +244,10 @@ int csla_window_rows(const csla_cfg *cfg, const csla_state *st, const int32_t *s
  *   cq [B][dc] (cq_dtype), W_iq [HI*dI][dc] (w_dtype), head_w [B][HI] f32,
  *   scores f32 [B][scores_stride], scores_stride >= max_len/m.
  * workspace: csla_workspace_size(cfg, CSLA_OP_INDEXER, B, max_len) bytes.
+ * qs: NULL (decode) or query rows; with qs->one_request several rows share
+ * each key tile.  Errors: CSLA_ERR_ARG (null pointers, stride, workspace,
+ * 16-byte alignment of cq, W_iq, kidx and workspace); CSLA_ERR_UNSUPPORTED
+ * for HI, dI or dc outside the supported set; device bits PAGE, LEN, INDEX.
  */
 int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
                         const int32_t *slots, int32_t B, const csla_queries *qs, int32_t max_len, const void *cq,
@@ -253,10 +257,12 @@ int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_ca
 
 /*
  * csla_topk_select -- top-k selector (硅星人 §两大压缩注意力, CSA part).
- * For request b: the min(k, N_vis) entries of largest score (ties: lower
- * index first), written to idx[b*k ..] in ascending index order, the rest of
- * the row filled with -1.  Exact: integer radix select on the fp32 bits
- * (-0.0 counts as +0.0).  scores as produced by csla_indexer_scores.
+ * For row b (N_vis = L/m as in csla_indexer_scores): the min(k, N_vis)
+ * entries of largest score (ties: lower index first), written to
+ * idx[b*k ..] in ascending index order, the rest of the row filled with -1.
+ * Exact: integer radix select on the fp32 bits (-0.0 counts as +0.0).
+ * scores as produced by csla_indexer_scores.  Errors: CSLA_ERR_ARG (null
+ * pointers, k outside 1..2048, stride); device bit LEN (row skipped).
  */
 int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *slots, int32_t B,
                      const csla_queries *qs, int32_t max_len, const float *scores, int32_t scores_stride, int32_t k,
@@ -265,10 +271,12 @@ int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *s
 /*
  * csla_csa_attend -- core MQA of a CSA layer (硅星人 §两大压缩注意力; haiqwa
  * §RMSNorm归一化, §Partial RoPE位置编码, §让注意力学会"忽略").
- * For request b at position t = len-1 and head h < H:
+ * For row b at position t = L-1 (L = len[slots[b]], or q_len[b] with qs)
+ * and head h < H:
  *   qh = RoPE(RMSNorm(q[b][h]) * gamma_q, t)
  *   set = compressed entries idx[b][0..k) (entries < 0 skipped), then window
- *         tokens max(0, len-n_win) .. len-1, each row decoded as above;
+ *         tokens max(0, L-n_win) .. L-1 (from the ring, or from qs's
+ *         window rows), each row decoded as above;
  *   s_j = <qh, x_j>/sqrt(D);  o = sum_j e^{s_j} x_j / (e^{sink[h]} + sum_j e^{s_j}).
  * One KV head: K = V = the cached row.  Batch invariant: each request's
  * reduction order is fixed by its own set size, identical for every variant.
@@ -278,6 +286,9 @@ int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *s
  *   CSLA_VARIANT_STARVED (one CTA per chunk, then an ordered combine), or AUTO.
  * workspace: csla_workspace_size(cfg, CSLA_OP_CSA_ATTEND, B, max_len) with
  *   max_len here meaning k (the set size is k + n_win).
+ * Errors: CSLA_ERR_ARG (null pointers, k, variant, workspace, 16-byte
+ * alignment of q, rows, window rows, workspace); device bits INDEX (an idx
+ * entry outside the visible range: row masked), PAGE, LEN.
  */
 int csla_csa_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
                     const int32_t *slots, int32_t B, const csla_queries *qs, const void *q, int32_t q_dtype,
