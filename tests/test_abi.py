@@ -92,3 +92,29 @@ def test_workspace_sizes():
     assert C.csla_workspace_size(_cfg(m=8), C.CSLA_OP_TOPK, 1, 1) == 0
     # decode step: the attention partials for k, then B int32 lengths (16-byte rounded)
     assert C.csla_workspace_size(cfg, C.CSLA_OP_CSA_DECODE_STEP, 8, 512) == 8 * 10 * (64 * 512 + 128) * 4 + 32
+
+
+def test_host_checks_of_the_query_row_and_step_calls():
+    """Arguments the host rejects before any launch (no GPU needed)."""
+    from compressed_sparse_long_append_b200 import csla as C
+    L = C._lib
+    fake = 1 << 40   # never dereferenced: every call below fails its host checks first
+    cfg = _cfg(m=4)
+    st = C.csla_state(fake, fake, fake, fake, fake, 4)
+    cache = C.csla_cache(fake, fake, fake, fake, 8, 16)
+    params = C.csla_compress_params(fake, fake, fake, fake, fake)
+    # window snapshot: n outside 1..n_win, stride below n
+    assert L.csla_window_rows(ctypes.byref(cfg), ctypes.byref(st), fake, 1, 129, fake, fake, 200, None) \
+        == C.CSLA_ERR_ARG
+    assert L.csla_window_rows(ctypes.byref(cfg), ctypes.byref(st), fake, 1, 100, fake, fake, 99, None) \
+        == C.CSLA_ERR_ARG
+    # token rows that do not fit the stride
+    tok = C.csla_token_rows(fake, fake, 10, 5)
+    assert L.csla_compress_append(ctypes.byref(cfg), ctypes.byref(st), ctypes.byref(cache), fake, 1, 6, fake, fake,
+                                  C.CSLA_BF16, ctypes.byref(params), ctypes.byref(tok), None) == C.CSLA_ERR_ARG
+    # the fused decode step: CSA only, and it needs a top-k list and its workspace
+    args = [ctypes.byref(st), ctypes.byref(cache), fake, 1, 1, 1024, fake, fake, C.CSLA_BF16, ctypes.byref(params),
+            fake, C.CSLA_BF16, fake, C.CSLA_BF16, fake, fake, 256, 64]
+    tail = [fake, C.CSLA_BF16, fake, fake, fake, C.CSLA_F32, 0, fake, 1 << 20, fake, 1 << 20, None]
+    assert L.csla_csa_decode_step(ctypes.byref(_cfg(m=128)), *args, fake, *tail) == C.CSLA_ERR_UNSUPPORTED
+    assert L.csla_csa_decode_step(ctypes.byref(cfg), *args, None, *tail) == C.CSLA_ERR_ARG
