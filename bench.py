@@ -571,6 +571,10 @@ def run_steps(steps, inputs, W, K, e2e=False, profile=False):
     main = torch.cuda.current_stream()
     e0.record(main)
     if e2e:
+        # step j+1's input copy is queued before step j's output copy on the
+        # copy stream, so step j's output buffer must not be written again by
+        # step j+1: it is reused only R >= 2 steps later
+        assert R >= 2, "the overlapped e2e copies need at least two output buffers"
         cs = torch.cuda.Stream()
         cs.wait_stream(main)   # every copy after the start event
         ev_in = [torch.cuda.Event() for _ in range(K)]

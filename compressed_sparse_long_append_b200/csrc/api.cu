@@ -453,10 +453,16 @@ int csla_csa_decode_step(const csla_cfg *cfg, const csla_state *st, const csla_c
     cudaError_t e = launch_len_snapshot(slots, st->len, B, st->n_slots, len0, s);
     if (e == cudaSuccess) e = cudaEventRecord(side->fork, s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
-    if (e == cudaSuccess) e = launch_compress_append(ca, kv_dtype == CSLA_BF16, side->s);
-    if (e == cudaSuccess) e = cudaEventRecord(side->join, side->s);
-    if (e == cudaSuccess) e = launch_indexer(old_a, il.cq_bf16, il.w_bf16, il.kmap, il.qmap, num_sms_current(), s);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, side->join, 0);
+    if (e == cudaSuccess) {
+        // forked: from here on the side stream is always joined back into the
+        // caller's stream, also when a launch fails (an unjoined fork would
+        // invalidate a stream capture), and the first error is returned
+        e = launch_compress_append(ca, kv_dtype == CSLA_BF16, side->s);
+        cudaError_t ej = cudaEventRecord(side->join, side->s);
+        if (e == cudaSuccess) e = launch_indexer(old_a, il.cq_bf16, il.w_bf16, il.kmap, il.qmap, num_sms_current(), s);
+        if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, side->join, 0);
+        if (e == cudaSuccess) e = ej;
+    }
     if (e == cudaSuccess)
         e = launch_indexer(new_a, il.cq_bf16, il.w_bf16, il.kmap, il.qmap, num_sms_current(), s, false);
     if (e == cudaSuccess) e = launch_topk(ta, s);

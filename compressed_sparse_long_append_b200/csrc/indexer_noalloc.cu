@@ -15,6 +15,8 @@
 // otherwise ordered, are safe.  The array keeps whatever the last call wrote;
 // the padding rows of the operand, which must read as zero, are cleared on
 // every call.
+#include <atomic>
+
 #include "../../include/csla.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -26,7 +28,11 @@ constexpr size_t kScratchBytes = (size_t)CSLA_NOALLOC_INDEXER_SCRATCH_BYTES;
 static __device__ __align__(256) uint8_t g_indexer_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void *g_scratch_ptr[kMaxDevices];
+// Per-device cache of the array's address.  Host threads may make their first
+// call on a device at the same time: each looks the address up and stores the
+// same value, so relaxed atomics suffice.  The cache is never refreshed, so it
+// would be stale after a cudaDeviceReset of that device.
+std::atomic<void *> g_scratch_ptr[kMaxDevices];
 
 // Device address of the array on the current device, looked up once per
 // device.  Returns null if the lookup fails.
@@ -36,16 +42,16 @@ void *scratch_address(int *status) {
         *status = CSLA_ERR_CUDA;
         return nullptr;
     }
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
+    void *p = g_scratch_ptr[dev].load(std::memory_order_relaxed);
+    if (!p) {
         if (cudaGetSymbolAddress(&p, g_indexer_scratch) != cudaSuccess || p == nullptr) {
             *status = CSLA_ERR_CUDA;
             return nullptr;
         }
-        g_scratch_ptr[dev] = p;
+        g_scratch_ptr[dev].store(p, std::memory_order_relaxed);
     }
     *status = CSLA_OK;
-    return g_scratch_ptr[dev];
+    return p;
 }
 
 }  // namespace

@@ -349,7 +349,8 @@ int csla_csa_decode_step(const csla_cfg *cfg, const csla_state *st, const csla_c
  * (64 requests at HI = 16, dI = 128); larger batches return CSLA_ERR_ARG
  * without launching.  The first call on a device looks up the array's device
  * address (cudaGetSymbolAddress, with that device current); make that first
- * call before any stream capture.  Every call shares the array: calls that
+ * call before any stream capture.  The address is cached for the life of the
+ * process and not looked up again after a cudaDeviceReset of that device.  Every call shares the array: calls that
  * overlap on the GPU race on it, calls ordered on one stream do not.  It
  * calls no allocation routine.
  */

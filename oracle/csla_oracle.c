@@ -135,7 +135,7 @@ void csla_orc_rope(double *y, int D, int d_rope, long long pos, double theta)
     }
 }
 
-/* Mixed-precision cache row ([haiqwa] §Partial RoPE位置编码 "混合精度存储";
+/* Mixed-precision cache row ([haiqwa] §Partial RoPE位置编码, the mixed-precision storage paragraph;
  * [silicon] same paragraph: RoPE dims bf16, the other dims fp8).
  * Row bytes: [0, D-dr) = E4M3 codes of dims 0..D-dr-1, then dr little-endian
  * bf16 values of dims D-dr..D-1.  One fp32 scale per row for the fp8 part:
@@ -169,8 +169,8 @@ void csla_orc_dequantize(const uint8_t *row, float scale, int D, int d_rope, dou
         x[dn + d] = csla_orc_bf16_value((unsigned)row[dn + 2 * d] | ((unsigned)row[dn + 2 * d + 1] << 8));
 }
 
-/* Token-level compressor ([haiqwa] §CSA：压缩稀疏注意力 "每 m 个token的KV缓存被压缩成
- * 一个条目"; [silicon] §CSA: Token-Level Compressor, m=4; §HCA: m'=128).
+/* Token-level compressor ([haiqwa] §CSA：压缩稀疏注意力: one cache entry per block
+ * of m tokens; [silicon] §CSA: Token-Level Compressor, m=4; §HCA: m'=128).
  * The pages give no formula.  Reading: one scalar gate per token,
  * g_i = <x_i, wg> + gb[i]; alpha = softmax_i(g); out = sum_i alpha_i x_i. */
 void csla_orc_gate_pool(const double *xs, int m, int width, const double *wg, const double *gb,
@@ -195,7 +195,7 @@ void csla_orc_gate_pool(const double *xs, int m, int width, const double *wg, co
     free(g);
 }
 
-/* Sliding-window row of token `pos` ([haiqwa] §Partial RoPE位置编码 "滑动窗口机制";
+/* Sliding-window row of token `pos` ([haiqwa] §Partial RoPE位置编码, sliding-window paragraph;
  * [silicon] §两大压缩注意力: the last 128 raw tokens kept uncompressed).
  * Reading: the row gets the same RMSNorm (gamma_kv), RoPE at its own position
  * and the same mixed-precision format as a compressed entry. */
@@ -225,8 +225,8 @@ void csla_orc_compressed_row(const double *xs, int m, const double *wg, const do
     free(y);
 }
 
-/* Compressed index key of a CSA block ([silicon] §CSA: the indexer produces
- * "index keys" from the same KV hidden states; "与压缩索引键计较分数").
+/* Compressed index key of a CSA block ([silicon] §CSA: the indexer derives its own
+ * compressed keys from the same KV hidden states and scores queries against them).
  * Reading: its own scalar gate (wgi, gbi), no norm, no RoPE, stored bf16
  * (rounded from fp32). */
 void csla_orc_index_key(const double *xis, int m, const double *wgi, const double *gbi, int dI,
@@ -244,7 +244,8 @@ void csla_orc_index_key(const double *xis, int m, const double *wgi, const doubl
 /* ------------------------------------------------------------------ */
 
 /* Index query: up-projection of the latent cq (dc) to HI heads of dI
- * ([silicon] §CSA "查询端先降维到 dc=1024 ... 再升维到多头索引查询").
+ * ([silicon] §CSA: the query is first reduced to a dc=1024 latent, then
+ * expanded to the index heads).
  * W is [HI*dI][dc] (row r = output feature r).  qI[j*dI+e] = sum_c W[j*dI+e][c] cq[c]. */
 void csla_orc_index_query(const double *cq, const double *W, int HI, int dI, int dc, double *qI)
 {
