@@ -15,12 +15,12 @@ CSLA_OK, CSLA_ERR_ARG, CSLA_ERR_UNSUPPORTED, CSLA_ERR_CUDA, CSLA_ERR_DEVICE = 0,
 CSLA_F32, CSLA_BF16 = 0, 1
 CSLA_VARIANT_AUTO, CSLA_VARIANT_SATURATED, CSLA_VARIANT_STARVED = 0, 1, 2
 CSLA_OP_INDEXER, CSLA_OP_TOPK, CSLA_OP_CSA_ATTEND, CSLA_OP_HCA_ATTEND, CSLA_OP_CSA_DECODE_STEP = 1, 2, 3, 4, 5
-CSLA_DEVERR_PAGE, CSLA_DEVERR_INDEX, CSLA_DEVERR_LEN, CSLA_DEVERR_TIMEOUT = 1, 2, 4, 8
+CSLA_DEVERR_PAGE, CSLA_DEVERR_INDEX, CSLA_DEVERR_LEN, CSLA_DEVERR_TIMEOUT, CSLA_DEVERR_RANGE = 1, 2, 4, 8, 16
 CSLA_PAGE_TOKENS = 128
 
 EXPORTS = ("csla_compress_append", "csla_indexer_scores", "csla_topk_select", "csla_csa_attend",
            "csla_hca_attend", "csla_workspace_size", "csla_device_error", "csla_strerror", "csla_version",
-           "csla_indexer_scores_noalloc", "csla_window_rows", "csla_csa_decode_step")
+           "csla_indexer_scores_noalloc", "csla_window_rows", "csla_csa_decode_step", "csla_check_wait_timeout")
 CSLA_NOALLOC_INDEXER_SCRATCH_BYTES = 786432
 
 
@@ -99,6 +99,7 @@ def _load():
         "csla_device_error": [P, ctypes.POINTER(ctypes.c_uint32)],
         "csla_strerror": [ctypes.c_int],
         "csla_version": [],
+        "csla_check_wait_timeout": [ctypes.c_uint32, P],
         "csla_indexer_scores_noalloc": [P, P, P, P, I, P, I, P, I, P, I, P, P, I, P],
         "csla_csa_decode_step": [P, P, P, P, I, I, I, P, P, I, P, P, I, P, I, P, P, I, I, P, P, I, P, P, P, I, I,
                                  P, Z, P, Z, P],
@@ -215,6 +216,10 @@ def csla_device_error(stream=None):
 
 def csla_strerror(status):
     return _lib.csla_strerror(status).decode()
+
+
+def csla_check_wait_timeout(limit_us, stream=None):
+    return _check("csla_check_wait_timeout", _lib.csla_check_wait_timeout(int(limit_us), _stream(stream)))
 
 
 def csla_version():

@@ -105,9 +105,31 @@ __device__ unsigned int g_timeline_n = 0;
 }  // namespace csla
 #endif
 
+namespace csla {
+namespace {
+// One thread waits, with the library's bounded wait, on an mbarrier that
+// expects one arrival nobody makes; the wait gives up after limit_ns and
+// records CSLA_DEVERR_TIMEOUT.
+__global__ void __launch_bounds__(32) wait_check_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        mbar_wait_limit(&bar, 0, nullptr, limit_ns);
+    }
+}
+}  // namespace
+}  // namespace csla
+
 extern "C" {
 
 int csla_version(void) { return 100; }
+
+int csla_check_wait_timeout(uint32_t limit_us, csla_stream_t stream) {
+    if (limit_us < 1 || limit_us > 2000000) return CSLA_ERR_ARG;
+    csla::wait_check_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>((uint64_t)limit_us * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? CSLA_OK : CSLA_ERR_CUDA;
+}
 
 #ifdef CSLA_TIMELINE
 int csla_timeline_read(void *records, size_t bytes, uint32_t *count) {
@@ -328,6 +350,10 @@ static int prep_attend(const csla_cfg *cfg, const csla_state *st, const csla_cac
     if (variant < CSLA_VARIANT_AUTO || variant > CSLA_VARIANT_STARVED || check_queries(qs)) return CSLA_ERR_ARG;
     if (!aligned16(q) || !aligned16(cache->rows) || !aligned16(st->win_rows) || !aligned16(workspace))
         return CSLA_ERR_ARG;
+    // row locations are 32-bit indices into the cache, the ring and the window-row buffer
+    if ((long long)cache->n_pages * (CSLA_PAGE_TOKENS / cfg->m) > 0xFFFFFFFFll ||
+        (long long)st->n_slots * cfg->n_win > 0xFFFFFFFFll)
+        return CSLA_ERR_UNSUPPORTED;
     AttendArgs a{};
     a.m = cfg->m; a.D = cfg->D; a.d_rope = cfg->d_rope; a.H = cfg->H; a.n_win = cfg->n_win;
     a.theta = cfg->rope_theta; a.eps = cfg->eps;

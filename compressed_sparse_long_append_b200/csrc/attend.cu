@@ -18,25 +18,39 @@
 // same code on the same data, so their outputs are identical bit for bit,
 // and nothing depends on which other requests share the launch.
 //
+// Operands.  A cache row holds fp8 (E4M3) codes c_d with one scale s per row
+// for the first D-64 dims and bf16 values for the 64 RoPE dims.  Every row
+// enters the tensor cores as one f16 vector X' of D dims:
+//   X'_d = e4m3(c_d) / 256            (exact: a move of the code's bits)
+//   X'_d = x_d / (256 s)              (RoPE dims, rounded to f16)
+// so that x_d = 256 s X'_d for every dim.  With Qhat in f16,
+//   s_j = 256 s_j^row * <Qhat, X'_j> / sqrt(D)        (one accumulator),
+//   O  += X'^T . P',   P'_hj = f16(p_hj * 256 s_j^row).
+// A row whose RoPE dims would leave the f16 range this way (|x_d| > 2^15 *
+// 256 s, which needs a row whose fp8 part is ~10^5 times smaller than its
+// RoPE part) takes a larger effective scale on a slow path.  A row whose
+// effective scale exceeds kScaleMax (fp8 dims beyond 448 * 15 = 6720, or
+// RoPE dims beyond ~1.3e8: never a row of a normalised vector) would
+// overflow P'; it is masked and sets CSLA_DEVERR_RANGE.
+//
 // One CTA = three roles over a stream of 64-row tiles:
-//   warps 4-7 (loader)  resolve the 64 row addresses of a tile (one thread
-//                       per row) and fetch the raw cache rows with 1-D bulk
-//                       copies into one of two staging buffers (tiles t+1 and
-//                       t+2 are in flight while tile t is converted); widen
-//                       fp8 codes to f16 (exact; the RoPE dims stay bf16)
-//                       into the SW128 K-major X tile once the previous
-//                       tile's PV product is done;
-//   warp 8 (MMA)        S = Qhat . X^T   tcgen05 M=64 (heads) N=64 (rows),
-//                                        nope and RoPE dims in separate TMEM
-//                                        accumulators: s = scale*S_nope + S_rope
-//                       O^T += X^T . P^T tcgen05 M=128 (dims) N=64 (heads);
-//   warps 0-3 (softmax) build Qhat = RoPE(RMSNorm(q)*gamma_q, t) in smem
-//                       (the norm before the grid-dependency wait, the
-//                       rotation after it); per tile read S, P = 2^(s - m)
-//                       (lanes 0-15 of each warp own one head),
-//                       P_nope = f16(P*scale), P_rope = bf16(P); lazy
-//                       rescale of O^T when a head's max grows by more than 8
-//                       (log2 units); at chunk end read O^T out as the partial.
+//   warps 4-11 (loader)  resolve row addresses eight tiles ahead (a ring of
+//                        16 tiles in shared memory; the three dependent
+//                        lookups -- top-k index, block table, scale -- run
+//                        on separate lane groups for three future tiles
+//                        each step), convert tile t's raw rows from
+//                        registers into X'[t & 1], then load tile t+1
+//                        (bulk-prefetched into L2 a step earlier) and
+//                        prefetch tile t+2;
+//   warp 12 (MMA)        S[t&1] = Qhat . X'^T  tcgen05 M=64 (heads) N=64 (rows)
+//                        O^T   += X'^T . P'^T  tcgen05 M=128 (dims) N=64 (heads),
+//                        issuing S of tile t+1 before PV of tile t;
+//   warps 0-3 (softmax)  build Qhat = RoPE(RMSNorm(q)*gamma_q, t) from a bulk
+//                        copy of q (the norm before the grid-dependency wait,
+//                        the rotation after it); per tile read S, P = 2^(s - m)
+//                        (lanes 0-15 of each warp own one head), lazy rescale
+//                        of O^T when a head's max grows by more than 4 (log2
+//                        units); at chunk end read O^T out as the partial.
 // mbarriers hand tiles between roles; every wait is bounded.
 #include "common.cuh"
 #include "kernels.h"
@@ -44,58 +58,61 @@
 namespace csla {
 namespace {
 
-constexpr int kSoftWarps = 4, kLoadWarps = 4;
-constexpr int kThreads = 32 * (kSoftWarps + kLoadWarps + 1);   // 288
-constexpr int kLoadThreads = 32 * kLoadWarps;
-constexpr int kMmaWarp = kSoftWarps + kLoadWarps;               // warp 8
+constexpr int kSoftWarps = 4, kLoadWarps = 8;
+constexpr int kThreads = 32 * (kSoftWarps + kLoadWarps + 1);   // 416
+constexpr int kMmaWarp = kSoftWarps + kLoadWarps;               // warp 12
 constexpr int kHP = 64;          // heads padded to the UMMA M of the S product
-constexpr int kTile = 64;        // rows per tile
+constexpr int kTile = 32;        // rows per tile
+constexpr int kRowsPerWarp = kTile / kLoadWarps;                // 4 rows of each tile per loader warp
+constexpr int kRing = 16;        // tiles of resolved row addresses
+constexpr int kAhead = 8;        // tiles resolved before the first conversion
+constexpr int kNR = 4;           // raw-row buffers (tiles of bulk copies in flight)
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThresh = 8.0f;
-constexpr int kBarLoad = 1;   // named barrier of the loader warps (0 = __syncthreads)
-// K blocks widened per proxy fence: 1 measured fastest (2 and 8 were 1.4
-// and 2.5 us slower per step: the S products then start later)
-constexpr int kWidenGroup = 1;
+constexpr float kRescaleThresh = 4.0f;
+constexpr float kRopeMax = 32768.0f;   // largest |X'| taken for a RoPE dim at the row's own scale
+// Largest effective row scale: P' = p * 256 * scale stays below the f16
+// maximum for p <= 2^kRescaleThresh.  Rows beyond it are masked and flagged.
+constexpr float kScaleMax = 15.0f;
 
 template <int D>
 struct Cfg {
     static constexpr int kRB = D + 64;                 // row bytes
-    static constexpr int kCH = kRB / 16;               // 16-byte chunks per row
-    static constexpr int kNopeCH = (D - 64) / 16;      // chunks holding fp8 codes
+    static constexpr int kNopeCH = (D - 64) / 16;      // 16-byte chunks of fp8 codes per row
     static constexpr int kKB = D / 64;                 // 64-dim K blocks
-    static constexpr int kKBN = (D - 64) / 64;         // nope K blocks
     static constexpr int kMB = D / 128;                // 128-dim O^T blocks
-    static constexpr int kKBBytes = kTile * 128;       // one K block of X (64 rows x 128 B)
+    static constexpr int kKBBytes = kTile * 128;       // one K block of X' (32 rows x 128 B)
     static constexpr int kXBytes = kKB * kKBBytes;
     static constexpr int kQKB = kHP * 128;             // one K block of Qhat
     static constexpr int kQBytes = kKB * kQKB;
-    static constexpr int kPBytes = kHP * kTile * 2;
-    static constexpr int kTasks = kTile * kCH;         // 16-byte chunks per tile
-    static_assert(kTasks % kLoadThreads == 0, "tile split");
-    static constexpr int kRawBytes = kTile * kRB;      // one staged tile of raw rows
-    // TMEM columns
-    static constexpr int kColSN = 0, kColSR = 64, kColO = 128;
-    static constexpr int kColOR = 128 + 64 * kMB;
-    static constexpr int kTmemCols = (kColOR + 64) <= 256 ? 256 : 512;
-    // smem offsets (from a 1024-aligned base)
+    static constexpr int kPBytes = kHP * 64 * 2;        // P [64 heads][64 cols], cols 0..kTile-1 used
+    static constexpr int kRawBytes = kTile * kRB;       // one raw buffer (bulk-copied cache rows)
+    static constexpr int kNopeIt = (kRowsPerWarp * kNopeCH + 31) / 32;   // fp8 chunk rounds per loader lane
+    static_assert(kRowsPerWarp * 8 == 32, "one RoPE chunk per loader lane");
+    // TMEM columns: two S buffers of kTile columns, then O^T
+    static constexpr int kColS = 0, kColO = 2 * kTile;
+    static constexpr int kTmemCols = (kColO + 64 * kMB) <= 128 ? 128 : ((kColO + 64 * kMB) <= 256 ? 256 : 512);
+    // smem offsets (from a 1024-aligned base); q is staged from X'[0] on at
+    // the start (into the raw buffers too when it is larger than both X')
     static constexpr int kOffQ = 0;
-    static constexpr int kOffX = kOffQ + kQBytes;
-    static constexpr int kOffRaw0 = kOffX + kXBytes;
-    static constexpr int kOffRaw1 = kOffRaw0 + kRawBytes;
-    static constexpr int kOffPn = kOffRaw1 + kRawBytes;
-    static constexpr int kOffPr = kOffPn + kPBytes;
-    static constexpr int kOffMisc = kOffPr + kPBytes;
+    static constexpr int kOffX = kOffQ + kQBytes;      // X'[0], X'[1]
+    static constexpr int kOffRaw = kOffX + 2 * kXBytes;
+    static constexpr int kOffP = kOffRaw + kNR * kRawBytes;
+    static constexpr int kOffMisc = kOffP + kPBytes;
 };
 
+// Kinds of row locations in the loader ring.
+enum : uint8_t { kLocNone = 0, kLocCache = 1, kLocRing = 2, kLocSrc = 3 };
+
 struct Misc {
-    float rawscale[2][kTile];          // loader-private, per staging buffer: fp8 scale of each row
-    int rawvalid[2][kTile];
-    float tscale[2][kTile];            // per tile parity: fp8 scale of each row (0 = masked)
-    int tvalid[2][kTile];
+    float tscale[2][kTile];            // per X' buffer: 256 * effective fp8 scale of each row (0 = masked)
     float fac[2][kHP];                 // per tile parity: O^T column factors (1 = none)
-    uint64_t raw_full[2], x_full[2], x_empty[2], s_full, s_free, p_full, pv_done, o_free, q_ready, fac_ready;
-    uint64_t kb_full[8];               // per K block of X: widened (one phase per tile)
-    int go[2];                         // loader: keep fetching (per tile parity)
+    // loader ring, per tile slot (t % kRing) and row of the tile
+    int ent[kRing][kTile];             // stage 1: compressed entry index (or the set row for window rows)
+    uint32_t loc[kRing][kTile];        // stage 2: row index in its array
+    float scl[kRing][kTile];           // stage 3: fp8 scale (0 = masked)
+    uint8_t kind[kRing][kTile];        // stage 2: kLoc*
+    uint64_t q_staged, q_ready, x_full[2], x_empty[2], s_full[2], s_free[2], p_full, pv_done, o_free, fac_ready,
+        drain, raw_full[kLoadWarps][kNR];   // raw_full[w][j]: warp w's rows of raw buffer j landed
     uint32_t tmem;
     int abort;
 };
@@ -135,205 +152,218 @@ __device__ __forceinline__ Req request(const AttendArgs &a, int b) {
     return r;
 }
 
-__device__ __forceinline__ void named_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
 // Byte offset of 8-element group g (dims 8g..8g+7) of row r in a SW128
 // K-major tile whose K blocks are `kb_bytes` apart.
 __device__ __forceinline__ uint32_t sw128_off(int r, int g, int kb_bytes) {
     return (uint32_t)((g >> 3) * kb_bytes + (r >> 3) * 1024 + (r & 7) * 128 + (((g & 7) ^ (r & 7)) << 4));
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    return (uint32_t)f32_to_bf16_bits(lo) | ((uint32_t)f32_to_bf16_bits(hi) << 16);
-}
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     const __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
+// Two E4M3 codes (bytes kLo and kLo+1 of w) -> f16x2 of their values / 256,
+// exactly: the 7 magnitude bits go under the f16 exponent/mantissa fields,
+// which places E4M3 normals and subnormals alike 8 binades low, and the
+// sign bit moves to bit 15.  (The NaN codes 0x7F/0xFF, which the quantiser
+// never writes, read as 480/256.)
+template <int kLo>
+__device__ __forceinline__ uint32_t e4m3x2_f16x2_div256(uint32_t w) {
+    constexpr uint32_t kSel = kLo == 0 ? 0x1404u : 0x3424u;   // code kLo+1 -> byte 3, code kLo -> byte 1
+    const uint32_t x = __byte_perm(w, 0u, kSel);
+    return (x & 0x80008000u) | ((x >> 1) & 0x3F803F80u);
+}
+
 // ---------------------------------------------------------------- query preparation
 // Qhat = RoPE(RMSNorm(q_h) * gamma_q, t) for the 64 (padded) heads of the
-// request, built in shared memory by the softmax warps in two steps.
+// request, built in shared memory by the softmax warps in two steps from a
+// bulk copy of the request's q rows (`stage`, H*D elements).
 // Before the grid-dependency wait (q and gamma_q are inputs of the call):
-// warp w normalises heads 16w .. 16w+15, lane l owning dims l*D/32 ..; the
-// non-RoPE dims go to the SW128 K-major Qhat image as f16, the RoPE dims
-// stay fp32 in the P area (64 heads x 64 dims x 4 B, unused until the first
-// tile's softmax).  After the wait, when the position t = len - 1 is known,
-// lane i rotates pair i of its warp's 16 heads and writes them as bf16.
+// warp w normalises heads 16w .. 16w+15, one head at a time; lane l owns the
+// 8-dim groups l and l+32 (D = 512) or the 4 dims 4l.. (D = 128), so the
+// staged reads are consecutive per lane (no bank conflicts).  Non-RoPE dims
+// go to the SW128 K-major Qhat image as f16; the RoPE dims are kept in fp32
+// at the start of the head's own staged row (already read).  After the
+// wait, when the position t = len - 1 is known, lane i rotates pair i of its
+// warp's 16 heads and writes them as f16.
 template <int D>
-__device__ void build_q_normed(const AttendArgs &a, int b, uint8_t *smem, int q_bf16) {
+__device__ void build_q_normed(const AttendArgs &a, uint8_t *smem, uint8_t *stage, int q_bf16) {
     using C = Cfg<D>;
-    constexpr int DPL = D / 32;              // dims per lane (16 or 4)
-    constexpr int kBatch = 4;                // heads whose loads are in flight together
+    constexpr int kG = D == 512 ? 2 : 1;       // element groups per lane
+    constexpr int kE = D == 512 ? 8 : 4;       // elements per group
+    constexpr int kStride = D == 512 ? 256 : 0; // dims between a lane's two groups
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float *ropef = reinterpret_cast<float *>(smem + C::kOffPn);   // [64 heads][64 dims]
-    const int d0 = lane * DPL;
-    float gam[DPL];
+    const int rb = D * (q_bf16 ? 2 : 4);       // staged bytes per head
+    float gam[kG][kE];
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) gam[e] = __ldg(a.gamma_q + d0 + e);
-    for (int h0 = 16 * warp; h0 < 16 * warp + 16; h0 += kBatch) {
-        float x[kBatch][DPL];
+    for (int g = 0; g < kG; ++g)
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            // padding heads (h >= H) load head H-1 (in bounds); their values are zeroed below
-            const int h = min(h0 + u, a.H - 1);
-            const size_t off = ((size_t)b * a.H + h) * D + d0;
+        for (int e = 0; e < kE; ++e) gam[g][e] = __ldg(a.gamma_q + g * kStride + kE * lane + e);
+    for (int h = 16 * warp; h < 16 * warp + 16; ++h) {
+        if (h >= a.H) {
+            // padding head: zero Qhat row (the RoPE dims are written zero after the wait)
 #pragma unroll
-            for (int e0 = 0; e0 < DPL; e0 += 8 > DPL ? DPL : 8) {
-                if (q_bf16) {
-                    if constexpr (DPL >= 8) {
-                        const uint4 w4 = __ldg(reinterpret_cast<const uint4 *>(
-                            reinterpret_cast<const __nv_bfloat16 *>(a.q) + off + e0));
-                        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+            for (int g = 0; g < kG; ++g) {
+                const int d = g * kStride + kE * lane;
+                if (d < D - 64) {
+                    if constexpr (kE == 8)
+                        *reinterpret_cast<uint4 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB)) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    else
+                        *reinterpret_cast<uint2 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB) + (d & 7) * 2) =
+                            make_uint2(0u, 0u);
+                }
+            }
+            continue;
+        }
+        const uint8_t *src = stage + h * rb;
+        float x[kG][kE];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            x[u][e0 + 2 * e] = bf16_bits_to_f32(w[e] & 0xFFFFu);
-                            x[u][e0 + 2 * e + 1] = bf16_bits_to_f32(w[e] >> 16);
-                        }
-                    } else {
-                        const uint2 w2 = __ldg(reinterpret_cast<const uint2 *>(
-                            reinterpret_cast<const __nv_bfloat16 *>(a.q) + off + e0));
-                        x[u][e0] = bf16_bits_to_f32(w2.x & 0xFFFFu);
-                        x[u][e0 + 1] = bf16_bits_to_f32(w2.x >> 16);
-                        x[u][e0 + 2] = bf16_bits_to_f32(w2.y & 0xFFFFu);
-                        x[u][e0 + 3] = bf16_bits_to_f32(w2.y >> 16);
+        for (int g = 0; g < kG; ++g) {
+            const int d = g * kStride + kE * lane;
+            if (q_bf16) {
+                if constexpr (kE == 8) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(src + 2 * d);
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        x[g][2 * e] = bf16_bits_to_f32(ww[e] & 0xFFFFu);
+                        x[g][2 * e + 1] = bf16_bits_to_f32(ww[e] >> 16);
                     }
                 } else {
-                    const float4 *p4 = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(a.q) + off + e0);
+                    const uint2 w = *reinterpret_cast<const uint2 *>(src + 2 * d);
+                    x[g][0] = bf16_bits_to_f32(w.x & 0xFFFFu);
+                    x[g][1] = bf16_bits_to_f32(w.x >> 16);
+                    x[g][2] = bf16_bits_to_f32(w.y & 0xFFFFu);
+                    x[g][3] = bf16_bits_to_f32(w.y >> 16);
+                }
+            } else {
 #pragma unroll
-                    for (int e = 0; e < (8 > DPL ? DPL : 8); e += 4) {
-                        const float4 f4 = __ldg(p4 + e / 4);
-                        x[u][e0 + e] = f4.x;
-                        x[u][e0 + e + 1] = f4.y;
-                        x[u][e0 + e + 2] = f4.z;
-                        x[u][e0 + e + 3] = f4.w;
-                    }
+                for (int e0 = 0; e0 < kE; e0 += 4) {
+                    const float4 f4 = *reinterpret_cast<const float4 *>(src + 4 * (d + e0));
+                    x[g][e0] = f4.x;
+                    x[g][e0 + 1] = f4.y;
+                    x[g][e0 + 2] = f4.z;
+                    x[g][e0 + 3] = f4.w;
                 }
             }
         }
+        float ss = 0.f;
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int h = h0 + u;
-            float ss = 0.f;
+        for (int g = 0; g < kG; ++g)
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) ss = __fmaf_rn(x[u][e], x[u][e], ss);
-            ss = warp_sum(ss);
-            const float r = 1.0f / sqrtf(__fdiv_rn(ss, (float)D) + a.eps);
-            float y[DPL];   // padding heads (h >= H) are zero
+            for (int e = 0; e < kE; ++e) ss = __fmaf_rn(x[g][e], x[g][e], ss);
+        ss = warp_sum(ss);   // every lane has read head h's row before anything is written back
+        const float r = 1.0f / sqrtf(__fdiv_rn(ss, (float)D) + a.eps);
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) y[e] = h < a.H ? __fmul_rn(__fmul_rn(x[u][e], r), gam[e]) : 0.f;
-            if (d0 >= D - 64) {
+        for (int g = 0; g < kG; ++g) {
+            const int d = g * kStride + kE * lane;
+            float y[kE];
 #pragma unroll
-                for (int e = 0; e < DPL; ++e) ropef[h * 64 + (d0 - (D - 64)) + e] = y[e];
+            for (int e = 0; e < kE; ++e) y[e] = __fmul_rn(__fmul_rn(x[g][e], r), gam[g][e]);
+            if (d >= D - 64) {
+                float *rf = reinterpret_cast<float *>(stage + h * rb);
+#pragma unroll
+                for (int e = 0; e < kE; ++e) rf[(d - (D - 64)) + e] = y[e];
+            } else if constexpr (kE == 8) {
+                uint4 o;
+                o.x = pack_f16x2(y[0], y[1]);
+                o.y = pack_f16x2(y[2], y[3]);
+                o.z = pack_f16x2(y[4], y[5]);
+                o.w = pack_f16x2(y[6], y[7]);
+                *reinterpret_cast<uint4 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB)) = o;
             } else {
-#pragma unroll
-                for (int e0 = 0; e0 < DPL; e0 += 8 > DPL ? DPL : 8) {
-                    const int d = d0 + e0;
-                    if constexpr (DPL >= 8) {
-                        uint4 o;
-                        o.x = pack_f16x2(y[e0], y[e0 + 1]);
-                        o.y = pack_f16x2(y[e0 + 2], y[e0 + 3]);
-                        o.z = pack_f16x2(y[e0 + 4], y[e0 + 5]);
-                        o.w = pack_f16x2(y[e0 + 6], y[e0 + 7]);
-                        *reinterpret_cast<uint4 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB)) = o;
-                    } else {
-                        uint2 o;
-                        o.x = pack_f16x2(y[e0], y[e0 + 1]);
-                        o.y = pack_f16x2(y[e0 + 2], y[e0 + 3]);
-                        *reinterpret_cast<uint2 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB) + (d & 7) * 2) = o;
-                    }
-                }
+                uint2 o;
+                o.x = pack_f16x2(y[0], y[1]);
+                o.y = pack_f16x2(y[2], y[3]);
+                *reinterpret_cast<uint2 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB) + (d & 7) * 2) = o;
             }
         }
     }
+    __syncwarp();   // the fp32 RoPE dims written by some lanes are read by all in build_q_rope
 }
 
 // After the wait: rotate the RoPE dims by position t and publish Qhat.
 template <int D>
-__device__ void build_q_rope(const AttendArgs &a, long long t, uint8_t *smem, Misc *ms) {
+__device__ void build_q_rope(const AttendArgs &a, long long t, uint8_t *smem, const uint8_t *stage, int q_bf16,
+                             Misc *ms) {
     using C = Cfg<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const float *ropef = reinterpret_cast<const float *>(smem + C::kOffPn);
+    const int rb = D * (q_bf16 ? 2 : 4);
     float c, sn;
     rope_cos_sin(t, a.freq.inv[lane], &c, &sn);
     const int dim = (D - 64) + 2 * lane;
     for (int h = 16 * warp; h < 16 * warp + 16; ++h) {
-        const float y0 = ropef[h * 64 + 2 * lane], y1 = ropef[h * 64 + 2 * lane + 1];
+        float y0 = 0.f, y1 = 0.f;
+        if (h < a.H) {
+            const float *rf = reinterpret_cast<const float *>(stage + h * rb);
+            y0 = rf[2 * lane];
+            y1 = rf[2 * lane + 1];
+        }
         const float r0 = __fsub_rn(__fmul_rn(y0, c), __fmul_rn(y1, sn));
         const float r1 = __fadd_rn(__fmul_rn(y0, sn), __fmul_rn(y1, c));
         *reinterpret_cast<uint32_t *>(smem + C::kOffQ + sw128_off(h, dim >> 3, C::kQKB) + (dim & 7) * 2) =
-            pack_bf16x2(r0, r1);
+            pack_f16x2(r0, r1);
     }
     fence_proxy_async_smem();
-    mbar_arrive(&ms->q_ready);
+    mbar_arrive_warp(&ms->q_ready);
 }
 
-// ---------------------------------------------------------------- loader role helpers
-// Source row (nullptr = masked) and fp8 scale of row r of the request's set.
-__device__ __forceinline__ const uint8_t *row_source(const AttendArgs &a, int b, const Req &rq, int r, int rb,
-                                                     float *scale) {
-    *scale = 0.f;
+// ---------------------------------------------------------------- row resolution (loader)
+// Row r of request b's set: stage 1 -> compressed entry index (a load of the
+// top-k list for CSA); stage 2 -> location (a load of the block table for
+// compressed entries; ring slot or chunk-buffer row for window rows);
+// stage 3 -> fp8 scale.  Bad indices and pages set the device error word and
+// mask the row.
+__device__ __forceinline__ int resolve_s1(const AttendArgs &a, int b, const Req &rq, int r) {
+    if (r < rq.n_cmp && a.idx) return __ldg(a.idx + (size_t)b * a.k + r);
+    return r;
+}
+__device__ __forceinline__ uint8_t resolve_s2(const AttendArgs &a, const Req &rq, int r, int e, uint32_t *loc) {
+    *loc = 0;
+    if (r >= rq.n_rows) return kLocNone;
     if (r < rq.n_cmp) {
-        const int e = a.idx ? __ldg(a.idx + (size_t)b * a.k + r) : r;
-        if (e < 0) return nullptr;
+        if (e < 0) return kLocNone;
         if (e >= rq.nv) {
             set_dev_err(CSLA_DEVERR_INDEX);
-            return nullptr;
+            return kLocNone;
         }
         const int epp = CSLA_PAGE_TOKENS / a.m;
         const int col = e / epp;
         const int pg = col < a.bt_stride ? __ldg(a.block_table + (size_t)rq.slot * a.bt_stride + col) : -1;
         if (pg < 0 || pg >= a.n_pages) {
             set_dev_err(CSLA_DEVERR_PAGE);
-            return nullptr;
+            return kLocNone;
         }
-        const size_t ent = (size_t)pg * epp + (size_t)(e % epp);
-        *scale = __ldg(a.scales + ent);
-        return a.rows + ent * rb;
+        *loc = (uint32_t)pg * (uint32_t)epp + (uint32_t)(e % epp);
+        return kLocCache;
     }
-    if (r < rq.n_rows) {
-        const int w = r - rq.n_cmp;
-        const int pos = rq.L - rq.win_len + w;
-        if (a.src_rows) {
-            const long long i = (long long)rq.wbase + pos;
-            if (i < 0 || i >= a.n_src) {
-                set_dev_err(CSLA_DEVERR_INDEX);
-                return nullptr;
-            }
-            *scale = __ldg(a.src_scales + i);
-            return a.src_rows + (size_t)i * rb;
+    const int w = r - rq.n_cmp;
+    const int pos = rq.L - rq.win_len + w;
+    if (a.src_rows) {
+        const long long i = (long long)rq.wbase + pos;
+        if (i < 0 || i >= a.n_src) {
+            set_dev_err(CSLA_DEVERR_INDEX);
+            return kLocNone;
         }
-        const size_t ring = (size_t)rq.slot * a.n_win + (size_t)(pos % a.n_win);
-        *scale = __ldg(a.win_scales + ring);
-        return a.win_rows + ring * rb;
+        *loc = (uint32_t)i;
+        return kLocSrc;
     }
-    return nullptr;
+    *loc = (uint32_t)rq.slot * (uint32_t)a.n_win + (uint32_t)(pos % a.n_win);
+    return kLocRing;
 }
-
-// Widen one 16-byte chunk of a cache row into the X tile: fp8 codes become
-// f16 (exact), the RoPE dims stay bf16.
-template <int D>
-__device__ __forceinline__ void store_chunk(uint8_t *xs, int r, int c, const uint4 v) {
-    using C = Cfg<D>;
-    if (c < C::kNopeCH) {
-        const int g0 = c * 2;   // 16 codes = two 8-dim groups
-        uint4 lo, hi;
-        lo.x = e4m3x2_to_f16x2(v.x & 0xFFFFu);
-        lo.y = e4m3x2_to_f16x2(v.x >> 16);
-        lo.z = e4m3x2_to_f16x2(v.y & 0xFFFFu);
-        lo.w = e4m3x2_to_f16x2(v.y >> 16);
-        hi.x = e4m3x2_to_f16x2(v.z & 0xFFFFu);
-        hi.y = e4m3x2_to_f16x2(v.z >> 16);
-        hi.z = e4m3x2_to_f16x2(v.w & 0xFFFFu);
-        hi.w = e4m3x2_to_f16x2(v.w >> 16);
-        *reinterpret_cast<uint4 *>(xs + sw128_off(r, g0, C::kKBBytes)) = lo;
-        *reinterpret_cast<uint4 *>(xs + sw128_off(r, g0 + 1, C::kKBBytes)) = hi;
-    } else {
-        const int g = (D - 64) / 8 + (c - C::kNopeCH);
-        *reinterpret_cast<uint4 *>(xs + sw128_off(r, g, C::kKBBytes)) = v;
-    }
+__device__ __forceinline__ float resolve_s3(const AttendArgs &a, uint8_t kind, uint32_t loc) {
+    if (kind == kLocCache) return __ldg(a.scales + loc);
+    if (kind == kLocRing) return __ldg(a.win_scales + loc);
+    if (kind == kLocSrc) return __ldg(a.src_scales + loc);
+    return 0.f;
+}
+__device__ __forceinline__ const uint8_t *row_ptr(const AttendArgs &a, uint8_t kind, uint32_t loc, int rb) {
+    if (kind == kLocCache) return a.rows + (size_t)loc * rb;
+    if (kind == kLocRing) return a.win_rows + (size_t)loc * rb;
+    if (kind == kLocSrc) return a.src_rows + (size_t)loc * rb;
+    return nullptr;
 }
 
 // The chunk range a CTA works on, and where chunk c's partial lives.
@@ -347,154 +377,363 @@ __device__ __forceinline__ float *partial_ptr(const AttendArgs &a, int b, int c,
     return a.part + ((size_t)b * a.max_chunks + c) * partial_floats(a.H, D);
 }
 
-// ---------------------------------------------------------------- the three roles
+// ---------------------------------------------------------------- loader role
+// Loader warp lw owns rows 4*lw .. 4*lw+3 of every tile: it resolves them,
+// bulk-copies them from the cache into its slots of the raw buffers (the
+// copy engine, no registers and no load/store-unit traffic), converts them
+// into X' and re-issues copies into the slots it has just consumed.
+struct LoadCtx {
+    int b, lw, lane, r_begin, r_end, n_tiles;
+};
+
+// Bulk copies of this warp's rows of tile t into raw buffer t % kNR: lanes
+// 0-3 add their row's bytes to the warp's barrier of that buffer and start
+// the copy; lane 0 then arrives on it.  Masked rows copy nothing.
 template <int D>
-__device__ void loader_role(const AttendArgs &a, int b, const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
+__device__ __forceinline__ void issue_rows(const AttendArgs &a, const LoadCtx &L, int t, uint8_t *smem, Misc *ms) {
     using C = Cfg<D>;
-    const int lt = threadIdx.x - 32 * kSoftWarps;
-    // the span's rows, in 64-row tiles (chunk boundaries are tile boundaries)
-    const int r_begin = sp.c0 * rq.chunk;
-    const int r_end = min(rq.n_rows, sp.c1 * rq.chunk);
-    const int n_tiles = (r_end - r_begin + kTile - 1) / kTile;
-    // Bulk-copy tile t's rows into staging buffer t & 1.  Every thread that
-    // issues a copy first adds its bytes to the buffer's transaction count;
-    // one arrival after the loader barrier closes the phase's bookkeeping.
-    // Called uniformly by all loader threads (each reaches the barrier).
-    auto issue = [&](int t) {
-        const int buf = t & 1;
-        if (lt < kTile) {
-            float sc;
-            const int r = r_begin + t * kTile + lt;
-            const uint8_t *p = r < r_end ? row_source(a, b, rq, r, C::kRB, &sc) : nullptr;
-            if (p) {
-                mbar_expect_tx(&ms->raw_full[buf], (uint32_t)C::kRB);
-                bulk_load(smem + (buf ? C::kOffRaw1 : C::kOffRaw0) + lt * C::kRB, p, (uint32_t)C::kRB,
-                          &ms->raw_full[buf]);
-            }
-            ms->rawscale[buf][lt] = p ? sc : 0.f;   // the scale load completes while the copy runs
-            ms->rawvalid[buf][lt] = p ? 1 : 0;
+    uint64_t *bar = &ms->raw_full[L.lw][t % kNR];
+    if (L.lane < kRowsPerWarp) {
+        const int i = kRowsPerWarp * L.lw + L.lane;
+        const uint8_t *p = row_ptr(a, ms->kind[t % kRing][i], ms->loc[t % kRing][i], C::kRB);
+        if (p) {
+            mbar_expect_tx(bar, (uint32_t)C::kRB);
+            bulk_load(smem + C::kOffRaw + (t % kNR) * C::kRawBytes + i * C::kRB, p, (uint32_t)C::kRB, bar);
         }
-        named_sync(kBarLoad, kLoadThreads);
-        if (lt == 0) mbar_arrive(&ms->raw_full[buf]);
-    };
-    int issued = 0, first_fail = n_tiles;
-    if (n_tiles > 0) issue(issued++);
-    if (n_tiles > 1) issue(issued++);
-    CSLA_TL_MARK_ANY(6);
-    for (int t = 0; t < n_tiles; ++t) {
-        const int buf = t & 1;
-        // the staged rows, and the X tile free again (PV of the previous tile done)
-        bool ok = t < issued && mbar_wait(&ms->raw_full[buf], (t >> 1) & 1, &ms->abort);
-        if (lt == 0 && t == 0) CSLA_TL_MARK_ANY(7);
-        if (!ok && t < first_fail) first_fail = t;
-        if (ok && t > 0) ok = mbar_wait(&ms->x_empty[(t - 1) & 1], ((t - 1) >> 1) & 1, &ms->abort);
-        const uint8_t *raw = smem + (buf ? C::kOffRaw1 : C::kOffRaw0);
-        uint8_t *xs = smem + C::kOffX;
-        // widen kWidenGroup K blocks at a time (one proxy fence per group);
-        // the MMA warp starts on a block as soon as every loader thread has
-        // arrived on its barrier
-#pragma unroll 1
-        for (int kb0 = 0; kb0 < C::kKB; kb0 += kWidenGroup) {
-            if (ok) {
-#pragma unroll 1
-                for (int kb = kb0; kb < kb0 + kWidenGroup && kb < C::kKB; ++kb) {
-                    // source chunks of this block: 4 fp8 chunks per row (nope)
-                    // or 8 bf16 chunks per row (RoPE block)
-                    const int cpr = kb < C::kKBN ? 4 : 8;
-                    const int ch0 = kb < C::kKBN ? 4 * kb : C::kNopeCH;
-#pragma unroll 4
-                    for (int id = lt; id < kTile * cpr; id += kLoadThreads) {
-                        const int r = id / cpr, ch = ch0 + id % cpr;
-                        const uint4 v = ms->rawvalid[buf][r]
-                                            ? *reinterpret_cast<const uint4 *>(raw + r * C::kRB + ch * 16)
-                                            : make_uint4(0u, 0u, 0u, 0u);
-                        store_chunk<D>(xs, r, ch, v);
-                    }
-                }
-                fence_proxy_async_smem();
-            }
-            for (int kb = kb0; kb < kb0 + kWidenGroup && kb < C::kKB; ++kb) mbar_arrive(&ms->kb_full[kb]);
-        }
-        if (ok) {
-            if (lt < kTile) {
-                ms->tscale[buf][lt] = ms->rawscale[buf][lt];
-                ms->tvalid[buf][lt] = ms->rawvalid[buf][lt];
-            }
-            if (lt == 0 && t == 0) CSLA_TL_MARK_ANY(4);
-        }
-        mbar_arrive(&ms->x_full[buf]);
-        // staging buffer `buf` is consumed: fetch tile t + 2 into it, unless
-        // the CTA is aborting (one decision for all loader threads)
-        if (lt == 0) ms->go[t & 1] = ms->abort ? 0 : 1;
-        named_sync(kBarLoad, kLoadThreads);
-        if (t + 2 < n_tiles && ms->go[t & 1]) issue(issued++);
     }
-    // copies still in flight after an abort must land before the CTA exits
-    for (int t = first_fail; t < issued; ++t) mbar_wait(&ms->raw_full[t & 1], (t >> 1) & 1, nullptr);
+    __syncwarp();
+    if (L.lane == 0) mbar_arrive(bar);
 }
 
+// Eight bf16 RoPE values (one 16-byte chunk) -> f16 of x * inv; true if one
+// leaves the range the f16 operand takes at this scale.
+__device__ __forceinline__ bool rope_chunk(const uint4 v, float inv, uint4 *o) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[4];
+    float mx = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float y0 = __fmul_rn(bf16_bits_to_f32(w[e] & 0xFFFFu), inv);
+        const float y1 = __fmul_rn(bf16_bits_to_f32(w[e] >> 16), inv);
+        mx = fmaxf(mx, fmaxf(fabsf(y0), fabsf(y1)));
+        out[e] = pack_f16x2(y0, y1);
+    }
+    *o = make_uint4(out[0], out[1], out[2], out[3]);
+    return !(mx <= kRopeMax);
+}
+
+// Rows whose RoPE dims exceed the f16 range at 256 * their own scale (or
+// whose scale is beyond kScaleMax): the warp re-reads each such row from its
+// raw slot and writes it with the effective scale
+// es = max(s, max|x_rope| / (256 * kRopeMax)): fp8 dims e4m3(c) * (s / es) / 256
+// and RoPE dims x / (256 es), both rounded to f16; a row with es beyond
+// kScaleMax is masked and flagged.  Rare (never for rows of normalised
+// vectors); correctness, not speed, matters here.
+template <int D>
+__device__ void wide_rows(const LoadCtx &L, int t, uint32_t rows, const uint8_t *raw, uint8_t *xs, Misc *ms,
+                          int buf) {
+    using C = Cfg<D>;
+    const int slot = t % kRing;
+    while (rows) {
+        const int i4 = __ffs(rows) - 1;
+        rows &= rows - 1;
+        const int i = kRowsPerWarp * L.lw + i4;
+        const uint8_t *p = raw + i * C::kRB;
+        const float s = ms->scl[slot][i];
+        float mx = 0.f;
+        if (L.lane < 8) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(p + 16 * (C::kNopeCH + L.lane));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                mx = fmaxf(mx, fmaxf(fabsf(bf16_bits_to_f32(w[e] & 0xFFFFu)), fabsf(bf16_bits_to_f32(w[e] >> 16))));
+        }
+        mx = warp_max(mx);
+        const float es = fmaxf(s, __fdiv_rn(mx, 256.0f * kRopeMax));
+        const bool masked = !(es <= kScaleMax);
+        const float ratio = masked ? 0.f : __fdiv_rn(s, es);
+        const float inv = masked ? 0.f : __fdiv_rn(1.0f, __fmul_rn(256.0f, es));
+        for (int c = L.lane; c < C::kNopeCH + 8; c += 32) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(p + 16 * c);
+            if (c < C::kNopeCH) {
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                uint32_t o[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t lo = e4m3x2_f16x2_div256<0>(w[e]), hi = e4m3x2_f16x2_div256<2>(w[e]);
+                    const __half2 hl = *reinterpret_cast<const __half2 *>(&lo);
+                    const __half2 hh = *reinterpret_cast<const __half2 *>(&hi);
+                    o[e] = pack_f16x2(__fmul_rn(__low2float(hl), ratio), __fmul_rn(__high2float(hl), ratio));
+                    o[4 + e] = pack_f16x2(__fmul_rn(__low2float(hh), ratio), __fmul_rn(__high2float(hh), ratio));
+                }
+                // o[e] holds dims 4e, 4e+1 of the chunk; o[4+e] dims 4e+2, 4e+3
+                *reinterpret_cast<uint4 *>(xs + sw128_off(i, 2 * c, C::kKBBytes)) = make_uint4(o[0], o[4], o[1], o[5]);
+                *reinterpret_cast<uint4 *>(xs + sw128_off(i, 2 * c + 1, C::kKBBytes)) =
+                    make_uint4(o[2], o[6], o[3], o[7]);
+            } else {
+                uint4 o;
+                rope_chunk(v, inv, &o);
+                *reinterpret_cast<uint4 *>(xs + sw128_off(i, (D - 64) / 8 + (c - C::kNopeCH), C::kKBBytes)) = o;
+            }
+        }
+        if (L.lane == 0) {
+            ms->tscale[buf][i] = masked ? 0.f : __fmul_rn(256.0f, es);
+            if (masked) set_dev_err(CSLA_DEVERR_RANGE);
+        }
+        __syncwarp();
+    }
+}
+
+// Convert this warp's rows of tile t from its raw slots into X'[buf];
+// returns the rows (bit i4 = row 4*lw + i4) that need the wide-range path
+// (warp-uniform).  Masked rows (nothing was copied) become zeros.
+template <int D>
+__device__ __forceinline__ uint32_t convert_rows(const LoadCtx &L, int t, const uint8_t *raw, uint8_t *xs, Misc *ms,
+                                                 int buf) {
+    using C = Cfg<D>;
+    const int slot = t % kRing;
+    constexpr int kNope = kRowsPerWarp * C::kNopeCH;   // this warp's fp8 chunks per tile
+#pragma unroll
+    for (int k = 0; k < C::kNopeIt; ++k) {
+        const int f = L.lane + 32 * k;
+        if (kNope % 32 == 0 || f < kNope) {
+            const int i = kRowsPerWarp * L.lw + f / C::kNopeCH, c = f % C::kNopeCH;
+            const uint4 v = ms->kind[slot][i] != kLocNone ? *reinterpret_cast<const uint4 *>(raw + i * C::kRB + 16 * c)
+                                                          : make_uint4(0u, 0u, 0u, 0u);
+            uint4 lo, hi;
+            lo.x = e4m3x2_f16x2_div256<0>(v.x);
+            lo.y = e4m3x2_f16x2_div256<2>(v.x);
+            lo.z = e4m3x2_f16x2_div256<0>(v.y);
+            lo.w = e4m3x2_f16x2_div256<2>(v.y);
+            hi.x = e4m3x2_f16x2_div256<0>(v.z);
+            hi.y = e4m3x2_f16x2_div256<2>(v.z);
+            hi.z = e4m3x2_f16x2_div256<0>(v.w);
+            hi.w = e4m3x2_f16x2_div256<2>(v.w);
+            *reinterpret_cast<uint4 *>(xs + sw128_off(i, 2 * c, C::kKBBytes)) = lo;
+            *reinterpret_cast<uint4 *>(xs + sw128_off(i, 2 * c + 1, C::kKBBytes)) = hi;
+        }
+    }
+    uint32_t wide = 0;
+    {
+        const int i4 = L.lane >> 3, c = L.lane & 7;
+        const int i = kRowsPerWarp * L.lw + i4;
+        const float s = ms->scl[slot][i];
+        const float inv = s > 0.f ? __fdiv_rn(1.0f, __fmul_rn(256.0f, s)) : 0.f;
+        const uint4 v = ms->kind[slot][i] != kLocNone
+                            ? *reinterpret_cast<const uint4 *>(raw + i * C::kRB + 16 * (C::kNopeCH + c))
+                            : make_uint4(0u, 0u, 0u, 0u);
+        uint4 o;
+        if (rope_chunk(v, inv, &o) || s > kScaleMax) wide = 1u << i4;
+        *reinterpret_cast<uint4 *>(xs + sw128_off(i, (D - 64) / 8 + c, C::kKBBytes)) = o;
+    }
+    if (L.lane < kRowsPerWarp) {
+        const int i = kRowsPerWarp * L.lw + L.lane;
+        ms->tscale[buf][i] = __fmul_rn(256.0f, ms->scl[slot][i]);
+    }
+    // OR of every lane's rows
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wide |= __shfl_xor_sync(0xffffffffu, wide, o);
+    return wide;
+}
+
+// One resolution step for three future tiles on three lane groups: lanes
+// 0-3 stage 3 of tile t3, lanes 4-7 stage 2 of tile t3+1, lanes 8-11 stage
+// 1 of tile t3+2.  Loads are issued now; results are stored by
+// resolve_store at the start of the next step, so their latency overlaps a
+// whole step (each stage reads what the previous step stored).
+struct ResolveRegs {
+    int e;
+    uint32_t loc;
+    uint8_t kind;
+    float s;
+};
+__device__ __forceinline__ ResolveRegs resolve_issue(const AttendArgs &a, const Req &rq, const LoadCtx &L, int t3,
+                                                     const Misc *ms) {
+    ResolveRegs x{0, 0u, kLocNone, 0.f};
+    const int grp = L.lane / kRowsPerWarp, i = kRowsPerWarp * L.lw + L.lane % kRowsPerWarp;
+    const int t = t3 + grp;
+    if (grp > 2 || t >= L.n_tiles) return x;
+    const int r = L.r_begin + t * kTile + i;
+    const int slot = t % kRing;
+    if (grp == 0) {
+        x.kind = ms->kind[slot][i];
+        x.loc = ms->loc[slot][i];
+        x.s = resolve_s3(a, x.kind, x.loc);
+    } else if (grp == 1) {
+        x.kind = r < L.r_end ? resolve_s2(a, rq, r, ms->ent[slot][i], &x.loc) : kLocNone;
+    } else {
+        x.e = r < L.r_end ? resolve_s1(a, L.b, rq, r) : 0;
+    }
+    return x;
+}
+__device__ __forceinline__ void resolve_store(const LoadCtx &L, int t3, const ResolveRegs &x, Misc *ms) {
+    const int grp = L.lane / kRowsPerWarp, i = kRowsPerWarp * L.lw + L.lane % kRowsPerWarp;
+    const int t = t3 + grp;
+    if (grp > 2 || t >= L.n_tiles) return;
+    const int slot = t % kRing;
+    if (grp == 0) {
+        ms->scl[slot][i] = x.s;
+    } else if (grp == 1) {
+        ms->kind[slot][i] = x.kind;
+        ms->loc[slot][i] = x.loc;
+    } else {
+        ms->ent[slot][i] = x.e;
+    }
+}
+
+// Tile t: store the previous step's resolution results and issue this
+// step's; wait for this warp's rows of tile t and for X'[t & 1]; convert
+// them and hand X' over; then copy tile t + kNR into the slots just read.
+// *landed is the last tile whose copies this warp has seen land, *issued the
+// last tile whose copies it has started.
+template <int D>
+__device__ __forceinline__ bool loader_step(const AttendArgs &a, const Req &rq, const LoadCtx &L, int t,
+                                            uint8_t *smem, Misc *ms, ResolveRegs &rr, int *landed, int *issued) {
+    using C = Cfg<D>;
+    if (t > 0) {
+        resolve_store(L, t - 1 + kAhead, rr, ms);
+        __syncwarp();
+    }
+    rr = resolve_issue(a, rq, L, t + kAhead, ms);
+    const int buf = t & 1;
+    if (!warp_all(mbar_wait(&ms->raw_full[L.lw][t % kNR], (t / kNR) & 1, &ms->abort))) return false;
+    *landed = t;
+    if (t >= 2 && !warp_all(mbar_wait(&ms->x_empty[buf], ((t - 2) >> 1) & 1, &ms->abort))) return false;
+    const uint8_t *raw = smem + C::kOffRaw + (t % kNR) * C::kRawBytes;
+    uint8_t *xs = smem + C::kOffX + buf * C::kXBytes;
+    const uint32_t wide = convert_rows<D>(L, t, raw, xs, ms, buf);
+    if (wide) wide_rows<D>(L, t, wide, raw, xs, ms, buf);   // warp-uniform
+    // X' to the tensor cores; the raw slots just read to the copy engine
+    fence_proxy_async_smem();
+    mbar_arrive_warp(&ms->x_full[buf]);
+    if (L.lw == 0 && L.lane == 0 && t < 2) CSLA_TL_MARK_ANY(t == 0 ? 1 : 5);
+    if (t + kNR < L.n_tiles) {
+        issue_rows<D>(a, L, t + kNR, smem, ms);
+        *issued = t + kNR;
+    }
+    return true;
+}
+
+template <int D>
+__device__ void loader_role(const AttendArgs &a, int b, const Req &rq, Span sp, uint8_t *smem, Misc *ms,
+                            bool q_in_raw) {
+    LoadCtx L;
+    L.b = b;
+    L.lw = (threadIdx.x >> 5) - kSoftWarps;
+    L.lane = threadIdx.x & 31;
+    L.r_begin = sp.c0 * rq.chunk;
+    L.r_end = min(rq.n_rows, sp.c1 * rq.chunk);
+    L.n_tiles = (L.r_end - L.r_begin + kTile - 1) / kTile;
+    if (L.n_tiles <= 0) return;
+    // Prologue: tiles 0..kAhead-1 fully resolved (lane l: row l % 4 of tile
+    // l / 4, one independent chain each), and in the same round tile kAhead
+    // through stage 2 (lanes 0-3) and tile kAhead+1 through stage 1 (lanes 4-7).
+    {
+        const int i = kRowsPerWarp * L.lw + L.lane % kRowsPerWarp, j = L.lane / kRowsPerWarp;
+        const int r = L.r_begin + j * kTile + i;
+        int e = 0;
+        uint32_t loc = 0;
+        uint8_t kind = kLocNone;
+        if (j < L.n_tiles && r < L.r_end) {
+            e = resolve_s1(a, b, rq, r);
+            kind = resolve_s2(a, rq, r, e, &loc);
+        }
+        const float s = resolve_s3(a, kind, loc);
+        const int tp = kAhead + j, rp = L.r_begin + tp * kTile + i;
+        int ep = 0;
+        uint32_t locp = 0;
+        uint8_t kindp = kLocNone;
+        if (j < 2 && tp < L.n_tiles && rp < L.r_end) {
+            ep = resolve_s1(a, b, rq, rp);
+            if (j == 0) kindp = resolve_s2(a, rq, rp, ep, &locp);
+        }
+        if (j < L.n_tiles) {
+            ms->kind[j % kRing][i] = kind;
+            ms->loc[j % kRing][i] = loc;
+            ms->scl[j % kRing][i] = s;
+        }
+        if (j < 2 && tp < L.n_tiles) {
+            ms->ent[tp % kRing][i] = ep;
+            if (j == 0) {
+                ms->kind[tp % kRing][i] = kindp;
+                ms->loc[tp % kRing][i] = locp;
+            }
+        }
+        __syncwarp();
+    }
+    // q may be staged in the raw buffers (f32 q): copy rows only once Qhat is built
+    if (q_in_raw && !warp_all(mbar_wait(&ms->q_ready, 0, &ms->abort))) return;
+    int landed = -1, issued = -1;
+    for (int t = 0; t < kNR && t < L.n_tiles; ++t) {
+        issue_rows<D>(a, L, t, smem, ms);
+        issued = t;
+    }
+    // q is staged in the X' buffers: convert only once Qhat is built
+    if (warp_all(mbar_wait(&ms->q_ready, 0, &ms->abort))) {
+        ResolveRegs rr;
+        for (int t = 0; t < L.n_tiles; ++t)
+            if (!loader_step<D>(a, rq, L, t, smem, ms, rr, &landed, &issued)) break;
+    }
+    // copies this warp started but has not seen land (only after an abort)
+    // must land before the CTA exits (each tile's phase has had its arrival)
+    for (int t = landed + 1; t <= issued; ++t) mbar_wait(&ms->raw_full[L.lw][t % kNR], (t / kNR) & 1, nullptr);
+}
+
+// ---------------------------------------------------------------- MMA role
 template <int D>
 __device__ void mma_role(const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
     using C = Cfg<D>;
-    // f16 operands for the fp8-coded dims, bf16 for the RoPE dims.  The PV
-    // blocks are 128 dims tall, so the last non-RoPE block also spans the
-    // RoPE dims (and the RoPE block the last 64 non-RoPE dims) read as the
-    // other type: those O^T rows are never read out.
-    constexpr uint32_t kIdescSN = idesc_f16(64, 64, false, false);
-    constexpr uint32_t kIdescSR = idesc_bf16(64, 64, false, false);
-    constexpr uint32_t kIdescON = idesc_f16(128, 64, true, false);
-    constexpr uint32_t kIdescOR = idesc_bf16(128, 64, true, false);
+    constexpr uint32_t kIdescS = idesc_f16(64, kTile, false, false);
+    constexpr uint32_t kIdescO = idesc_f16(128, 64, true, false);
     const uint32_t tmem = ms->tmem;
     const uint32_t q0 = smem_u32(smem + C::kOffQ);
-    const uint32_t p0n = smem_u32(smem + C::kOffPn), p0r = smem_u32(smem + C::kOffPr);
+    const uint32_t p0 = smem_u32(smem + C::kOffP);
+    const int r_begin = sp.c0 * rq.chunk;
+    const int r_end = min(rq.n_rows, sp.c1 * rq.chunk);
+    const int n_tiles = (r_end - r_begin + kTile - 1) / kTile;
+    const int tpc = rq.chunk / kTile;   // tiles per chunk (chunks are whole tiles)
     if (!mbar_wait(&ms->q_ready, 0, &ms->abort)) return;
-    CSLA_TL_MARK_ANY(5);
-    int g = 0;
-    for (int c = sp.c0; c < sp.c1; ++c) {
-        const int lo = c * rq.chunk;
-        const int hi = min(rq.n_rows, lo + rq.chunk);
-        for (int r0 = lo, ti = 0; r0 < hi; r0 += kTile, ++ti, ++g) {
-            const int buf = g & 1;
-            if (g > 0 && !mbar_wait(&ms->s_free, (g - 1) & 1, &ms->abort)) return;
-            const uint32_t x0 = smem_u32(smem + C::kOffX);
+    CSLA_TL_MARK_ANY(0);
+    for (int g = 0; g <= n_tiles; ++g) {
+        if (g < n_tiles) {
+            // S[g & 1] = Qhat . X'[g & 1]^T
+            const int sb = g & 1;
+            if (!mbar_wait(&ms->x_full[sb], (g >> 1) & 1, &ms->abort)) return;
+            if (g >= 2 && !mbar_wait(&ms->s_free[sb], ((g - 2) >> 1) & 1, &ms->abort)) return;
+            tc_fence_after();
+            const uint32_t x0 = smem_u32(smem + C::kOffX + sb * C::kXBytes);
 #pragma unroll 1
-            for (int kb = 0; kb < C::kKBN; ++kb) {
-                if (!mbar_wait(&ms->kb_full[kb], g & 1, &ms->abort)) return;
-                tc_fence_after();
+            for (int kb = 0; kb < C::kKB; ++kb)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    umma_kind_f16(tmem + C::kColSN, sdesc(q0 + kb * C::kQKB + ks * 32, 16, 1024),
-                                  sdesc(x0 + kb * C::kKBBytes + ks * 32, 16, 1024), kIdescSN, (kb | ks) ? 1u : 0u);
-            }
-            if (!mbar_wait(&ms->kb_full[C::kKBN], g & 1, &ms->abort)) return;
+                    umma_kind_f16(tmem + C::kColS + kTile * sb, sdesc(q0 + kb * C::kQKB + ks * 32, 16, 1024),
+                                  sdesc(x0 + kb * C::kKBBytes + ks * 32, 16, 1024), kIdescS, (kb | ks) ? 1u : 0u);
+            umma_commit(&ms->s_full[sb]);
+            if (g == 0) CSLA_TL_MARK_ANY(4);
+        }
+        if (g >= 1) {
+            // O^T += X'[h & 1]^T . P^T for tile h = g - 1
+            const int h = g - 1, xb = h & 1;
+            const int ti = h % tpc, c = h / tpc;
+            if (!mbar_wait(&ms->p_full, h & 1, &ms->abort)) return;
+            if (ti == 0 && c > 0 && !mbar_wait(&ms->o_free, (c - 1) & 1, &ms->abort)) return;
             tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                umma_kind_f16(tmem + C::kColSR, sdesc(q0 + C::kKBN * C::kQKB + ks * 32, 16, 1024),
-                              sdesc(x0 + C::kKBN * C::kKBBytes + ks * 32, 16, 1024), kIdescSR, ks ? 1u : 0u);
-            if (g == 0) CSLA_TL_MARK_ANY(0);
-            umma_commit(&ms->s_full);
-            if (!mbar_wait(&ms->p_full, g & 1, &ms->abort)) return;
-            if (ti == 0 && c > sp.c0 && !mbar_wait(&ms->o_free, (c - sp.c0 - 1) & 1, &ms->abort)) return;
-            tc_fence_after();
+            const uint32_t x0 = smem_u32(smem + C::kOffX + xb * C::kXBytes);
 #pragma unroll
             for (int mb = 0; mb < C::kMB; ++mb)
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
+                for (int ks = 0; ks < kTile / 16; ++ks)
                     umma_kind_f16(tmem + C::kColO + 64 * mb,
-                              sdesc(x0 + 2 * mb * C::kKBBytes + 2 * ks * 1024, C::kKBBytes, 1024),
-                              sdesc(p0n + ks * 32, 16, 1024), kIdescON, (ti > 0 || ks > 0) ? 1u : 0u);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                umma_kind_f16(tmem + C::kColOR,
-                          sdesc(x0 + 2 * (C::kMB - 1) * C::kKBBytes + 2 * ks * 1024, C::kKBBytes, 1024),
-                          sdesc(p0r + ks * 32, 16, 1024), kIdescOR, (ti > 0 || ks > 0) ? 1u : 0u);
-            umma_commit(&ms->x_empty[buf]);
+                                  sdesc(x0 + 2 * mb * C::kKBBytes + 2 * ks * 1024, C::kKBBytes, 1024),
+                                  sdesc(p0 + ks * 32, 16, 1024), kIdescO, (ti > 0 || ks > 0) ? 1u : 0u);
+            umma_commit(&ms->x_empty[xb]);
             umma_commit(&ms->pv_done);
+            if (g == n_tiles) CSLA_TL_MARK_ANY(7);
         }
     }
 }
 
+// ---------------------------------------------------------------- softmax role
 template <int D>
 __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
     using C = Cfg<D>;
@@ -504,10 +743,7 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
     const bool head_thread = lane < 16;
     const float cscale = kLog2e / sqrtf((float)D);
     const uint32_t tmem = ms->tmem;
-    uint8_t *pn = smem + C::kOffPn;
-    uint8_t *pr = smem + C::kOffPr;
-
-    build_q_rope<D>(a, (long long)rq.L - 1, smem, ms);
+    uint8_t *pp = smem + C::kOffP;
 
     int g = 0, nfac = 0;
     for (int c = sp.c0; c < sp.c1; ++c) {
@@ -515,33 +751,35 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
         const int hi = min(rq.n_rows, lo + rq.chunk);
         float m_run = -INFINITY, l_run = 0.f;
         for (int r0 = lo, ti = 0; r0 < hi; r0 += kTile, ++ti, ++g) {
-            const int buf = g & 1;
-            if (!mbar_wait(&ms->x_full[buf], (g >> 1) & 1, &ms->abort)) return;
-            if (!mbar_wait(&ms->s_full, g & 1, &ms->abort)) return;
-            if (threadIdx.x == 0 && g == 0) CSLA_TL_MARK(1);
+            const int sb = g & 1;
+            if (!warp_all(mbar_wait(&ms->x_full[sb], (g >> 1) & 1, &ms->abort))) return;
+            if (!warp_all(mbar_wait(&ms->s_full[sb], (g >> 1) & 1, &ms->abort))) return;
             tc_fence_after();
+            const float4 *ts4 = reinterpret_cast<const float4 *>(ms->tscale[sb]);
             float s[kTile];
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t rn[32], rr[32];
-                tmem_ld32x32(tmem + lane_base + C::kColSN + 32 * half, rn);
-                tmem_ld32x32(tmem + lane_base + C::kColSR + 32 * half, rr);
+            float mt = -INFINITY;
+            {
+                static_assert(kTile == 32, "one 32-column TMEM load per tile");
+                uint32_t rv[32];
+                tmem_ld32x32(tmem + lane_base + C::kColS + kTile * sb, rv);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int jj = 32 * half + j;
-                    const float v = __fmul_rn(
-                        __fmaf_rn(ms->tscale[buf][jj], __uint_as_float(rn[j]), __uint_as_float(rr[j])), cscale);
-                    s[jj] = ms->tvalid[buf][jj] ? v : -INFINITY;
+                for (int j4 = 0; j4 < kTile / 4; ++j4) {
+                    const float4 t4 = ts4[j4];
+                    const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 4 * j4 + e;
+                        const float v = __uint_as_float(rv[j]);
+                        s[j] = tv[e] > 0.f ? __fmul_rn(__fmul_rn(v, tv[e]), cscale) : -INFINITY;
+                        mt = fmaxf(mt, s[j]);
+                    }
                 }
             }
             tc_fence_before();
-            mbar_arrive(&ms->s_free);        // S may be overwritten by the next tile's MMA
-            float mt = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < kTile; ++j) mt = fmaxf(mt, s[j]);
+            mbar_arrive_warp(&ms->s_free[sb]);   // S[sb] may be overwritten by tile g + 2
             // PV of the previous tile must be done before P and O^T are touched.
-            if (g > 0 && !mbar_wait(&ms->pv_done, (g - 1) & 1, &ms->abort)) return;
+            if (g > 0 && !warp_all(mbar_wait(&ms->pv_done, (g - 1) & 1, &ms->abort))) return;
             tc_fence_after();
             float f = 1.f;
             if (head_thread) {
@@ -556,25 +794,21 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
                 float lsum = 0.f;
 #pragma unroll
                 for (int c8 = 0; c8 < kTile / 8; ++c8) {
+                    const float4 ta = ts4[2 * c8], tb = ts4[2 * c8 + 1];
+                    const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
                     float p[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         p[e] = exp2f(__fsub_rn(s[c8 * 8 + e], muse));
                         lsum = __fadd_rn(lsum, p[e]);
                     }
-                    const float *sc = &ms->tscale[buf][c8 * 8];
-                    uint4 un, ur;
-                    un.x = pack_f16x2(__fmul_rn(p[0], sc[0]), __fmul_rn(p[1], sc[1]));
-                    un.y = pack_f16x2(__fmul_rn(p[2], sc[2]), __fmul_rn(p[3], sc[3]));
-                    un.z = pack_f16x2(__fmul_rn(p[4], sc[4]), __fmul_rn(p[5], sc[5]));
-                    un.w = pack_f16x2(__fmul_rn(p[6], sc[6]), __fmul_rn(p[7], sc[7]));
-                    ur.x = pack_bf16x2(p[0], p[1]);
-                    ur.y = pack_bf16x2(p[2], p[3]);
-                    ur.z = pack_bf16x2(p[4], p[5]);
-                    ur.w = pack_bf16x2(p[6], p[7]);
+                    uint4 u;
+                    u.x = pack_f16x2(__fmul_rn(p[0], tv[0]), __fmul_rn(p[1], tv[1]));
+                    u.y = pack_f16x2(__fmul_rn(p[2], tv[2]), __fmul_rn(p[3], tv[3]));
+                    u.z = pack_f16x2(__fmul_rn(p[4], tv[4]), __fmul_rn(p[5], tv[5]));
+                    u.w = pack_f16x2(__fmul_rn(p[6], tv[6]), __fmul_rn(p[7], tv[7]));
                     const uint32_t off = (uint32_t)((h >> 3) * 1024 + (h & 7) * 128 + ((c8 ^ (h & 7)) << 4));
-                    *reinterpret_cast<uint4 *>(pn + off) = un;
-                    *reinterpret_cast<uint4 *>(pr + off) = ur;
+                    *reinterpret_cast<uint4 *>(pp + off) = u;
                 }
                 l_run = (ti == 0) ? lsum : __fadd_rn(__fmul_rn(l_run, f), lsum);
                 m_run = mnew;
@@ -584,56 +818,61 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
             // row); a chunk's first tile has none (every factor is 1)
             bool any_rescale = false;
             if (ti > 0) {
-                mbar_arrive(&ms->fac_ready);
-                if (!mbar_wait(&ms->fac_ready, nfac & 1, &ms->abort)) return;
+                mbar_arrive_warp(&ms->fac_ready);
+                if (!warp_all(mbar_wait(&ms->fac_ready, nfac & 1, &ms->abort))) return;
                 ++nfac;
-#pragma unroll 8
-                for (int j = 0; j < kHP; ++j) any_rescale |= ms->fac[g & 1][j] != 1.f;
+                const float4 *f4 = reinterpret_cast<const float4 *>(ms->fac[g & 1]);
+#pragma unroll
+                for (int j = 0; j < kHP / 4; ++j) {
+                    const float4 v = f4[j];
+                    any_rescale |= (v.x != 1.f) | (v.y != 1.f) | (v.z != 1.f) | (v.w != 1.f);
+                }
             }
             if (any_rescale) {
-                // O^T columns are heads: every thread scales its own dim lane.
+                // O^T columns are heads: every thread scales its own dim lane,
+                // 16 columns (heads) at a time
 #pragma unroll 1
-                for (int blk = 0; blk <= C::kMB; ++blk) {
+                for (int it = 0; it < 4 * C::kMB; ++it) {
+                    const int blk = it >> 2, q4 = it & 3;
+                    uint32_t v[16];
+                    const uint32_t addr = tmem + lane_base + C::kColO + 64 * blk + 16 * q4;
+                    tmem_ld32x16(addr, v);
+                    tmem_wait_ld();
+                    const float4 *f4 = reinterpret_cast<const float4 *>(&ms->fac[g & 1][16 * q4]);
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        uint32_t v[32];
-                        const uint32_t addr = tmem + lane_base + C::kColO + 64 * blk + 32 * half;
-                        tmem_ld32x32(addr, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            v[j] = __float_as_uint(__fmul_rn(__uint_as_float(v[j]), ms->fac[g & 1][32 * half + j]));
-                        tmem_st32x32(addr, v);
+                    for (int j4 = 0; j4 < 4; ++j4) {
+                        const float4 fv = f4[j4];
+                        v[4 * j4] = __float_as_uint(__fmul_rn(__uint_as_float(v[4 * j4]), fv.x));
+                        v[4 * j4 + 1] = __float_as_uint(__fmul_rn(__uint_as_float(v[4 * j4 + 1]), fv.y));
+                        v[4 * j4 + 2] = __float_as_uint(__fmul_rn(__uint_as_float(v[4 * j4 + 2]), fv.z));
+                        v[4 * j4 + 3] = __float_as_uint(__fmul_rn(__uint_as_float(v[4 * j4 + 3]), fv.w));
                     }
+                    tmem_st32x16(addr, v);
                 }
                 tmem_wait_st();
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&ms->p_full);
+            mbar_arrive_warp(&ms->p_full);
+            if (threadIdx.x == 0 && g < 2) CSLA_TL_MARK_ANY(g == 0 ? 2 : 6);
         }
         // chunk done: drain its last PV and read O^T out as the partial
-        if (!mbar_wait(&ms->pv_done, (g - 1) & 1, &ms->abort)) return;
-        if (threadIdx.x == 0) CSLA_TL_MARK(2);
+        if (!warp_all(mbar_wait(&ms->pv_done, (g - 1) & 1, &ms->abort))) return;
         tc_fence_after();
         float *part = partial_ptr(a, b, c, D);
         float *ml = part + (size_t)a.H * D;
 #pragma unroll 1
-        for (int blk = 0; blk <= C::kMB; ++blk) {
-            const bool rope_blk = blk == C::kMB;
-            const int dim = (rope_blk ? (D - 128) : 128 * blk) + 32 * warp + lane;
-            const bool write = rope_blk ? (dim >= D - 64) : (dim < D - 64);
+        for (int blk = 0; blk < C::kMB; ++blk) {
+            const int dim = 128 * blk + 32 * warp + lane;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t v[32];
                 tmem_ld32x32(tmem + lane_base + C::kColO + 64 * blk + 32 * half, v);
                 tmem_wait_ld();
-                if (write) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int hh = 32 * half + j;
-                        if (hh < a.H) part[(size_t)hh * D + dim] = __uint_as_float(v[j]);
-                    }
+                for (int j = 0; j < 32; ++j) {
+                    const int hh = 32 * half + j;
+                    if (hh < a.H) part[(size_t)hh * D + dim] = __uint_as_float(v[j]);
                 }
             }
         }
@@ -641,9 +880,9 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
             ml[h] = m_run;
             ml[a.H + h] = l_run;
         }
-        if (threadIdx.x == 0) CSLA_TL_MARK(3);
         tc_fence_before();
-        mbar_arrive(&ms->o_free);
+        mbar_arrive_warp(&ms->o_free);
+        if (threadIdx.x == 0 && c == sp.c0) CSLA_TL_MARK_ANY(3);
     }
 }
 
@@ -701,22 +940,30 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int q
     Misc *ms = reinterpret_cast<Misc *>(smem + C::kOffMisc);
     const int b = kSaturated ? blockIdx.x : blockIdx.y;
     const int warp = threadIdx.x >> 5;
+    // q of request b is staged from X'[0] on: in the two X' buffers (bf16 q
+    // of up to 64 heads fills them exactly), reaching into the raw buffers
+    // for f32 q
+    const uint32_t q_bytes = (uint32_t)(a.H * D * (q_bf16 ? 2 : 4));
+    uint8_t *stage = smem + C::kOffX;
+    const bool q_in_raw = q_bytes > (uint32_t)(2 * C::kXBytes);
 
-    // ---- before the wait: barriers and TMEM
+    // ---- before the wait: barriers, TMEM, the q copy
     if (threadIdx.x == 0) {
+        mbar_init(&ms->q_staged, 1);
+        mbar_init(&ms->q_ready, kSoftWarps);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&ms->raw_full[i], 1);
-            mbar_init(&ms->x_full[i], kLoadThreads);
+            mbar_init(&ms->x_full[i], kLoadWarps);
             mbar_init(&ms->x_empty[i], 1);
+            mbar_init(&ms->s_full[i], 1);
+            mbar_init(&ms->s_free[i], kSoftWarps);
         }
-        for (int i = 0; i < C::kKB; ++i) mbar_init(&ms->kb_full[i], kLoadThreads);
-        mbar_init(&ms->s_full, 1);
-        mbar_init(&ms->s_free, 32 * kSoftWarps);
-        mbar_init(&ms->p_full, 32 * kSoftWarps);
+        mbar_init(&ms->p_full, kSoftWarps);
         mbar_init(&ms->pv_done, 1);
-        mbar_init(&ms->o_free, 32 * kSoftWarps);
-        mbar_init(&ms->q_ready, 32 * kSoftWarps);
-        mbar_init(&ms->fac_ready, 32 * kSoftWarps);
+        mbar_init(&ms->o_free, kSoftWarps);
+        mbar_init(&ms->fac_ready, kSoftWarps);
+        mbar_init(&ms->drain, 1);
+        for (int w = 0; w < kLoadWarps; ++w)
+            for (int i = 0; i < kNR; ++i) mbar_init(&ms->raw_full[w][i], 1);
         ms->abort = 0;
         fence_mbar_init();
     }
@@ -728,7 +975,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int q
     __syncthreads();
     tc_fence_after();
     pdl_trigger();   // after the TMEM allocation (see the indexer kernel)
-    if (warp < kSoftWarps) build_q_normed<D>(a, b, smem, q_bf16);
+    if (threadIdx.x == 32 * kMmaWarp) {
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(a.q) + (size_t)b * q_bytes;
+        mbar_arrive_expect_tx(&ms->q_staged, q_bytes);
+        bulk_load(stage, src, q_bytes, &ms->q_staged);
+    }
+    bool q_ok = true;
+    if (warp < kSoftWarps) {
+        q_ok = warp_all(mbar_wait(&ms->q_staged, 0, &ms->abort));
+        if (q_ok) build_q_normed<D>(a, smem, stage, q_bf16);
+    }
     pdl_wait();
     CSLA_TL_WAITED();
 
@@ -739,11 +995,21 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int q
     if (!run) {
         // nothing to do: fall through to the teardown
     } else if (warp < kSoftWarps) {
-        softmax_role<D>(a, b, rq, sp, smem, ms);
+        if (q_ok) {
+            build_q_rope<D>(a, (long long)rq.L - 1, smem, stage, q_bf16, ms);
+            softmax_role<D>(a, b, rq, sp, smem, ms);
+        }
     } else if (warp < kSoftWarps + kLoadWarps) {
-        loader_role<D>(a, b, rq, sp, smem, ms);
+        loader_role<D>(a, b, rq, sp, smem, ms, q_in_raw);
     } else if ((threadIdx.x & 31) == 0) {
         mma_role<D>(rq, sp, smem, ms);
+    }
+    if (threadIdx.x == 32 * kMmaWarp) {
+        // the q copy has landed (it is waited for even when nothing ran), and
+        // every MMA this thread issued has completed, before the CTA tears down
+        mbar_wait(&ms->q_staged, 0, nullptr);
+        umma_commit(&ms->drain);
+        mbar_wait(&ms->drain, 0, nullptr);
     }
     tc_fence_before();
     __syncthreads();
@@ -755,8 +1021,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int q
     if (kSaturated) {
         // partials written by this CTA are visible to it after the barrier
         // above.  Every head's chunk weights first (warp-collective per head),
-        // into the staging area the loader no longer uses.
-        float *wall = reinterpret_cast<float *>(smem + C::kOffRaw0);   // [H][33]: w_0..w_31, l
+        // into the X' area the loader no longer uses.
+        float *wall = reinterpret_cast<float *>(smem + C::kOffX);   // [H][33]: w_0..w_31, l
         const int lane = threadIdx.x & 31;
         const int n = rq.n_chunks;
         for (int hh = warp; hh < a.H; hh += kThreads / 32) {

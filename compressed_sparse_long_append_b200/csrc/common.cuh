@@ -187,22 +187,57 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Wait for phase `parity` of `bar` to complete.  Gives up after kWaitLimitNs,
+// try_wait that lets the hardware suspend the thread until the phase
+// completes or `ns` nanoseconds pass, instead of returning at once: a waiting
+// warp then takes no issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+constexpr uint32_t kWaitSleepNs = 1000000;   // 1 ms: bounds the reaction to an abort
+
+// Wait for phase `parity` of `bar` to complete.  Gives up after limit_ns,
 // records CSLA_DEVERR_TIMEOUT and returns false; also returns false at once
 // when *abort (shared, may be null) is set by another role of the CTA.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
+    const uint32_t sleep = limit_ns < kWaitSleepNs ? (uint32_t)limit_ns : kWaitSleepNs;
     uint64_t t0 = globaltimer_ns();
     for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, sleep)) return true;
         if (abort && *abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             set_dev_err(CSLA_DEVERR_TIMEOUT);
             if (abort) *abort = 1;
             return false;
         }
     }
 }
+// The wait every library kernel uses: limit kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return mbar_wait_limit(bar, parity, abort, kWaitLimitNs);
+}
+
+// One arrival per warp on an mbarrier initialised with a count of warps:
+// every lane's earlier shared-memory (and, after a tcgen05 before-fence,
+// TMEM) work is ordered before lane 0's release by the warp barrier.  All
+// 32 lanes must call it.  (One arrival per thread costs a shared-memory
+// atomic per lane on the same word, which serialises.)
+__device__ __forceinline__ void mbar_arrive_warp(uint64_t *bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+// Warp-uniform outcome of a bounded wait: a lane that gave up makes the whole
+// warp give up, so warp-collective instructions after it never see a split warp.
+__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(idx_threads<G>())
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(tfull + i, 1);
-            mbar_init(tempty + i, 128 * idx_epi_sets<G>());
+            mbar_init(tempty + i, 4 * idx_epi_sets<G>());   // one arrival per epilogue warp
         }
         mbar_init(qfull, 1);
         fence_mbar_init();
@@ -343,7 +343,7 @@ __global__ void __launch_bounds__(idx_threads<G>())
         }
         pages[lane] = e0 < nv_max ? pg : -1;
     }
-    __syncwarp();
+    __syncthreads();   // the epilogue warps read pages[] too (entries of a bad page stay unscored)
 
     if (n_tiles <= 0) {
         // nothing to score: fall through to the teardown
@@ -414,7 +414,7 @@ __global__ void __launch_bounds__(idx_threads<G>())
         const int row = lane_base + lane;
         for (int t = 0, n = 0; t < n_tiles; ++t, ++n) {
             const int acc = n & 1;
-            if (!mbar_wait(tfull + acc, (n / 2) & 1, &abort_flag)) break;
+            if (!warp_all(mbar_wait(tfull + acc, (n / 2) & 1, &abort_flag))) break;
             tc_fence_after();
             const int e = (t_begin + t) * kTileE + row;
             int last = -1;   // this set's last row with entries in the tile (warp-uniform)
@@ -422,7 +422,7 @@ __global__ void __launch_bounds__(idx_threads<G>())
                 if (row_nv[g] > (t_begin + t) * kTileE) last = g;
             if (last < 0) {
                 tc_fence_before();
-                mbar_arrive(tempty + acc);
+                mbar_arrive_warp(tempty + acc);
             }
 #pragma unroll 1
             for (int g = es; g <= last; g += kSets) {
@@ -445,9 +445,10 @@ __global__ void __launch_bounds__(idx_threads<G>())
                 if (g == last) {
                     // every column this set reads is in registers: the MMA may reuse the accumulator
                     tc_fence_before();
-                    mbar_arrive(tempty + acc);
+                    mbar_arrive_warp(tempty + acc);
                 }
-                if (e < nv && e >= row_lo[g]) {
+                // entries of a page outside the pool were not loaded: leave them unscored
+                if (e < nv && e >= row_lo[g] && pages[t * 4 + row / kPageE] >= 0) {
                     float sc = 0.f;
 #pragma unroll
                     for (int j = 0; j < HI; ++j) {

@@ -94,7 +94,8 @@ enum {
     CSLA_DEVERR_PAGE = 1,     /* block-table entry outside [0, n_pages) */
     CSLA_DEVERR_INDEX = 2,    /* top-k index outside [0, visible entries) */
     CSLA_DEVERR_LEN = 4,      /* context length above max_len */
-    CSLA_DEVERR_TIMEOUT = 8   /* a bounded wait inside a kernel gave up */
+    CSLA_DEVERR_TIMEOUT = 8,  /* a bounded wait inside a kernel gave up */
+    CSLA_DEVERR_RANGE = 16    /* a cache row outside the attention operands' range (row masked) */
 };
 
 #define CSLA_PAGE_TOKENS 128
@@ -287,8 +288,15 @@ int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *s
  * workspace: csla_workspace_size(cfg, CSLA_OP_CSA_ATTEND, B, max_len) with
  *   max_len here meaning k (the set size is k + n_win).
  * Errors: CSLA_ERR_ARG (null pointers, k, variant, workspace, 16-byte
- * alignment of q, rows, window rows, workspace); device bits INDEX (an idx
- * entry outside the visible range: row masked), PAGE, LEN.
+ * alignment of q, rows, window rows, workspace); CSLA_ERR_UNSUPPORTED when
+ * n_pages * (128/m) or n_slots * n_win reaches 2^32; device bits INDEX (an
+ * idx entry outside the visible range: row masked), PAGE, LEN, RANGE.
+ * Operand range: the tensor cores take each row in f16 as x / (256 * s_eff)
+ * with P scaled by 256 * s_eff, s_eff = max(fp8 scale, max|RoPE dim| /
+ * 2^23).  A row with s_eff > 15 (fp8 dims above 6720 in magnitude, or RoPE
+ * dims above ~1.3e8; rows of RMSNorm-ed vectors stay far below) is masked
+ * and sets CSLA_DEVERR_RANGE.  RoPE dims below 2^-24 * 256 * s_eff in
+ * magnitude contribute as f16 subnormals or zero.
  */
 int csla_csa_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
                     const int32_t *slots, int32_t B, const csla_queries *qs, const void *q, int32_t q_dtype,
@@ -370,6 +378,20 @@ size_t csla_workspace_size(const csla_cfg *cfg, int32_t op, int32_t B, int32_t m
  * current device.  Returns CSLA_OK, or CSLA_ERR_DEVICE with the CSLA_DEVERR_*
  * bits in *bits (bits may be NULL), or CSLA_ERR_CUDA. */
 int csla_device_error(csla_stream_t stream, uint32_t *bits);
+
+/*
+ * csla_check_wait_timeout -- exercise of the failure path every kernel's
+ * bounded waits share (the pages have no counterpart: an operational check).
+ * Launches one CTA on `stream` whose thread waits, with the library's own
+ * bounded mbarrier wait, on a barrier that nobody arrives at, for at most
+ * limit_us microseconds (1 .. 2000000); the wait gives up, sets
+ * CSLA_DEVERR_TIMEOUT in the device error word and the kernel returns, so
+ * csla_device_error() afterwards reports CSLA_ERR_DEVICE with that bit and
+ * the context stays usable.  (The kernels' own waits give up after 2 s.)
+ * Errors: CSLA_ERR_ARG for a limit outside the range; CSLA_ERR_CUDA if the
+ * launch fails.
+ */
+int csla_check_wait_timeout(uint32_t limit_us, csla_stream_t stream);
 
 /* Static text for a status code. */
 const char *csla_strerror(int status);

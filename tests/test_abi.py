@@ -76,6 +76,16 @@ def test_host_argument_checks():
         assert L.csla_topk_select(ctypes.byref(_cfg(**bad)), None, None, 1, None, 10, None, 10, 5, None, None) \
             == C.CSLA_ERR_UNSUPPORTED, bad
     assert L.csla_strerror(C.CSLA_ERR_DEVICE) == b"device-side input error"
+    # the bounded-wait check takes 1 us .. 2 s
+    assert L.csla_check_wait_timeout(0, None) == C.CSLA_ERR_ARG
+    assert L.csla_check_wait_timeout(2000001, None) == C.CSLA_ERR_ARG
+    # attention: row locations are 32-bit indices
+    big = C.csla_cache(1 << 40, 1 << 40, None, 1 << 40, 1, 1 << 28)   # 2^28 pages x 32 entries = 2^33 rows
+    stq = C.csla_state(1 << 40, 1 << 40, 1 << 40, 1 << 40, 1 << 40, 4)
+    fake = 1 << 40
+    assert L.csla_csa_attend(ctypes.byref(cfg), ctypes.byref(stq), ctypes.byref(big), fake, 1, None, fake,
+                             C.CSLA_BF16, fake, 64, fake, fake, fake, C.CSLA_F32, 0, fake, 1 << 30, None) \
+        == C.CSLA_ERR_UNSUPPORTED
 
 
 def test_workspace_sizes():

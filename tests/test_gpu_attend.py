@@ -47,13 +47,15 @@ def _dev(x):
 
 def test_every_e4m3_code_widens_exactly():
     """Window of one token whose fp8 dims hold every finite E4M3 code with
-    scale 1: with the sink at -1e30 the output is that row, exactly."""
+    scale 1 and whose RoPE dims hold values the f16 operand carries exactly
+    at that scale: with the sink at -1e30 the output is that row, exactly."""
     shape = LayerShape(m=128, D=512, H=8)
     lb = LayerBuffers(shape, 1, 1, 1, DEV)
     codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
     row = np.zeros(576, np.uint8)
     row[:448] = np.resize(codes, 448)
-    rope = np.array([0x3F80, 0xBF80, 0x0080, 0x7F7F] * 16, np.uint16)   # 1, -1, min normal, max
+    # 1, -1, 2^-10, 2992: each / 256 is an f16 value
+    rope = np.array([0x3F80, 0xBF80, 0x3A80, 0x453B] * 16, np.uint16)
     row[448:] = rope.view(np.uint8)
     lb.win_rows[0, 0] = torch.from_numpy(row).to(DEV)
     lb.win_scales[0, 0] = 1.0
@@ -64,9 +66,37 @@ def test_every_e4m3_code_widens_exactly():
                  _dev(np.ones(512)), [1])
     assert_no_device_error()
     want = oracle.dequantize(row, 1.0, 512)
+    assert want[449] == -1.0 and want[450] == 2.0 ** -10 and want[451] == 2992.0
     got = out.cpu().numpy().astype(np.float64)[0]
     for h in range(8):
         assert np.array_equal(got[h], want), np.nonzero(got[h] != want)
+
+
+def test_row_outside_operand_range_is_masked_and_flagged():
+    """A window row whose fp8 scale is beyond the operand range (|x| up to
+    448 * 100) is masked and sets CSLA_DEVERR_RANGE; the output is the
+    attention over the remaining rows, finite."""
+    w = dataclasses.replace(HCA_DECODE, H=8, B=1, L=3, name="range")
+    shape = LayerShape(m=128, D=512, H=8)
+    lb = LayerBuffers(shape, 1, 1, 1, DEV)
+    rng = np.random.default_rng(5)
+    rows = rng.integers(0, 0x7E, size=(3, 576)).astype(np.uint8)
+    rows[:, 448:] = 0
+    scales = np.array([0.01, 100.0, 0.02], np.float32)
+    lb.win_rows[0, :3] = torch.from_numpy(rows).to(DEV)
+    lb.win_scales[0, :3] = torch.from_numpy(scales).to(DEV)
+    lb.len[0] = 3
+    q = torch.zeros((1, 8, 512), dtype=torch.float32, device=DEV)
+    q[..., :8] = 1.0
+    sink = np.zeros(8)
+    out = attend(w, lb, q, _dev(sink), _dev(np.ones(512)), [3])
+    rc, bits = C.csla_device_error()
+    assert rc == C.CSLA_ERR_DEVICE and bits == C.CSLA_DEVERR_RANGE, (rc, bits)
+    kept = np.stack([oracle.dequantize(rows[i], scales[i], 512) for i in (0, 2)])
+    ref, _ = oracle.attend(q.cpu().numpy()[0].astype(np.float64), np.ones(512), 2, kept, sink)
+    got = out.cpu().numpy().astype(np.float64)[0]
+    assert np.all(np.isfinite(got))
+    check_out(got, ref)
 
 
 CSA_SMALL = dataclasses.replace(CSA_TINY, B=3, L=2048, name="att_csa_tiny")
