@@ -23,6 +23,7 @@ class LayerShape:
     d_rope: int = 64
     theta: float = 10000.0
     eps: float = 1e-6
+    key_fmt: int = C.CSLA_KEY_BF16   # CSA index keys: bf16, or E4M3 codes + per-entry power-of-two scale
 
     @property
     def is_csa(self):
@@ -39,7 +40,7 @@ class LayerShape:
     def cfg(self):
         return C.csla_cfg(self.m, self.D, self.d_rope, self.H, self.HI if self.is_csa else 0,
                           self.dI if self.is_csa else 0, self.dc if self.is_csa else 0, self.n_win,
-                          self.theta, self.eps)
+                          self.theta, self.eps, self.key_fmt if self.is_csa else C.CSLA_KEY_BF16)
 
 
 class LayerBuffers:
@@ -52,7 +53,10 @@ class LayerBuffers:
         dev = self.device
         self.rows = torch.zeros((n_pages, s.epp, s.row_bytes), dtype=torch.uint8, device=dev)
         self.scales = torch.zeros((n_pages, s.epp), dtype=torch.float32, device=dev)
-        self.kidx = torch.zeros((n_pages, s.epp, s.dI), dtype=torch.int16, device=dev) if s.is_csa else None
+        fp8_keys = s.is_csa and s.key_fmt == C.CSLA_KEY_E4M3
+        kdt = torch.uint8 if fp8_keys else torch.int16
+        self.kidx = torch.zeros((n_pages, s.epp, s.dI), dtype=kdt, device=dev) if s.is_csa else None
+        self.kscale = torch.zeros((n_pages, s.epp), dtype=torch.float32, device=dev) if fp8_keys else None
         self.block_table = torch.full((n_slots, bt_stride), -1, dtype=torch.int32, device=dev)
         self.win_rows = torch.zeros((n_slots, s.n_win, s.row_bytes), dtype=torch.uint8, device=dev)
         self.win_scales = torch.zeros((n_slots, s.n_win), dtype=torch.float32, device=dev)
@@ -68,7 +72,8 @@ class LayerBuffers:
     def cache(self):
         return C.csla_cache(self.rows.data_ptr(), self.scales.data_ptr(),
                             self.kidx.data_ptr() if self.kidx is not None else None,
-                            self.block_table.data_ptr(), self.bt_stride, self.n_pages)
+                            self.block_table.data_ptr(), self.bt_stride, self.n_pages,
+                            self.kscale.data_ptr() if self.kscale is not None else None)
 
     def state(self):
         return C.csla_state(self.win_rows.data_ptr(), self.win_scales.data_ptr(), self.tail_kv.data_ptr(),
@@ -80,8 +85,10 @@ class LayerBuffers:
         out = {k: getattr(self, k).cpu().numpy() for k in
                ("rows", "scales", "block_table", "win_rows", "win_scales", "tail_kv", "len")}
         if self.kidx is not None:
-            out["kidx"] = self.kidx.cpu().numpy().view("uint16")
+            out["kidx"] = self.kidx.cpu().numpy() if self.kscale is not None else self.kidx.cpu().numpy().view("uint16")
             out["tail_idx"] = self.tail_idx.cpu().numpy()
+        if self.kscale is not None:
+            out["kscale"] = self.kscale.cpu().numpy()
         return out
 
 

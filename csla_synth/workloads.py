@@ -28,6 +28,7 @@ class Workload:
     eps: float = 1e-6
     act_bf16: bool = True   # activations are exact bf16 values
     seed: int = 0
+    key_fmt: int = 0        # CSA index keys: 0 bf16, 1 E4M3 codes + per-entry power-of-two scale
 
     @property
     def is_csa(self):

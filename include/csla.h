@@ -47,7 +47,10 @@
  *   epp = 128/m entries per page (32 for CSA, 1 for HCA):
  *     rows   uint8 [n_pages][epp][row_bytes]
  *     scales f32   [n_pages][epp]
- *     kidx   bf16  [n_pages][epp][dI]         (CSA only: compressed index keys)
+ *     kidx   [n_pages][epp][dI]               (CSA only: compressed index keys),
+ *            bf16 values (key_fmt CSLA_KEY_BF16) or E4M3 codes (CSLA_KEY_E4M3)
+ *     kscale f32   [n_pages][epp]              (CSLA_KEY_E4M3 only) key scale, a power of two:
+ *            key dim e = e4m3(code_e) * kscale
  *     block_table int32 [n_slots][bt_stride]: compressed entry e of slot s is
  *       entry e % epp of page block_table[s][e / epp].
  *   State cache (one layer, per slot):
@@ -80,6 +83,14 @@ enum {
 enum { CSLA_F32 = 0, CSLA_BF16 = 1 };
 
 enum { CSLA_VARIANT_AUTO = 0, CSLA_VARIANT_SATURATED = 1, CSLA_VARIANT_STARVED = 2 };
+
+/* Storage of the CSA compressed index keys (haiqwa §FP4精度加速: the
+ * indexer's key/query path runs in low precision).  E4M3: one byte per dim
+ * plus one power-of-two scale per entry, s = the smallest 2^e (-126 <= e <=
+ * 127) with 448 * s >= max |key dim|, codes = E4M3(key / s) rounded to
+ * nearest even, both decided on the fp32 pooled key; 132 bytes per entry at
+ * dI = 128 instead of 256. */
+enum { CSLA_KEY_BF16 = 0, CSLA_KEY_E4M3 = 1 };
 
 enum {
     CSLA_OP_INDEXER = 1,
@@ -114,15 +125,17 @@ typedef struct csla_cfg {
     int32_t n_win;      /* sliding window, 128 */
     float rope_theta;   /* RoPE base, 10000 */
     float eps;          /* RMSNorm epsilon, 1e-6 */
+    int32_t key_fmt;    /* CSA index-key storage: CSLA_KEY_BF16 (default) or CSLA_KEY_E4M3 */
 } csla_cfg;
 
 typedef struct csla_cache {
     uint8_t *rows;
     float *scales;
-    uint16_t *kidx;            /* CSA only, else NULL */
+    void *kidx;                /* CSA only, else NULL: bf16 values or E4M3 codes (cfg->key_fmt) */
     const int32_t *block_table;
     int32_t bt_stride;
     int32_t n_pages;
+    float *kscale;             /* CSA with CSLA_KEY_E4M3 only, else NULL: per-entry key scale */
 } csla_cache;
 
 typedef struct csla_state {

@@ -51,14 +51,16 @@ def lib():
             "csla_orc_window_row": (None, [dp, dp, I, I, D_, D_, ll, u8p, fp]),
             "csla_orc_compressed_row": (None, [dp, I, dp, dp, dp, I, I, D_, D_, ll, u8p, fp]),
             "csla_orc_index_key": (None, [dp, I, dp, dp, I, u16p]),
+            "csla_orc_key_scale_e4m3": (D_, [D_]),
+            "csla_orc_index_key_e4m3": (None, [dp, I, dp, dp, I, u8p, fp]),
             "csla_orc_index_query": (None, [dp, dp, I, I, I, dp]),
             "csla_orc_index_scores": (None, [dp, dp, I, I, dp, ll, dp]),
             "csla_orc_topk": (None, [dp, I, I, i32p]),
             "csla_orc_attend": (None, [dp, dp, ll, dp, I, dp, I, I, I, D_, D_, dp, dp]),
             "csla_orc_n_visible": (ll, [ll, I]),
             "csla_orc_gather_set": (I, [u8p, fp, i32p, I, u8p, fp, I, I, ll, I, I, I, i32p, I, dp]),
-            "csla_orc_gather_keys": (None, [u16p, i32p, I, I, ll, I, I, dp]),
-            "csla_orc_csa_decode": (None, [u8p, fp, u16p, i32p, I, u8p, fp, I, i32p, i32p, I, I, I,
+            "csla_orc_gather_keys": (None, [ctypes.c_void_p, fp, i32p, I, I, ll, I, I, dp]),
+            "csla_orc_csa_decode": (None, [u8p, fp, ctypes.c_void_p, fp, i32p, I, u8p, fp, I, i32p, i32p, I, I, I,
                                            I, I, I, I, I, I, D_, D_, dp, dp, dp, dp, dp, dp, i32p,
                                            dp]),
             "csla_orc_hca_decode": (None, [u8p, fp, i32p, I, u8p, fp, I, i32p, i32p, I, I, I, I, I,
@@ -188,6 +190,23 @@ def index_key(xis, wgi, gbi):
     return key
 
 
+def key_scale_e4m3(amax):
+    """Smallest 2^e (-126 <= e <= 127) with 448 * 2^e >= amax."""
+    return float(lib().csla_orc_key_scale_e4m3(float(amax)))
+
+
+def index_key_e4m3(xis, wgi, gbi):
+    """E4M3 storage of a CSA block's index key: (codes uint8 [dI], scale)."""
+    xis = _d(xis)
+    m, dI = xis.shape
+    wgi, gbi = _d(wgi), _d(gbi)
+    codes = np.zeros(dI, np.uint8)
+    sc = np.zeros(1, np.float32)
+    lib().csla_orc_index_key_e4m3(_p(xis, ctypes.c_double), m, _p(wgi, ctypes.c_double),
+                                  _p(gbi, ctypes.c_double), dI, _p(codes, ctypes.c_uint8), _p(sc, ctypes.c_float))
+    return codes, float(sc[0])
+
+
 # ---------------------------------------------------------------- indexer / top-k / attention
 def index_query(cq, W, HI, dI):
     cq, W = _d(cq), _d(W)
@@ -240,18 +259,21 @@ class CacheView:
 
       rows   [n_pages, 128//m, row_bytes] uint8      scales [n_pages, 128//m] f32
       kidx   [n_pages, 128//m, dI] uint16 (bf16)     block_table [n_slots, bt_stride] int32
+             or uint8 E4M3 codes with kscale [n_pages, 128//m] f32
       win_rows [n_slots, n_win, row_bytes] uint8     win_scales [n_slots, n_win] f32
     """
 
     def __init__(self, m, D, rows, scales, block_table, win_rows, win_scales, kidx=None, dI=0,
-                 d_rope=64):
+                 d_rope=64, kscale=None):
         self.m, self.D, self.d_rope, self.dI = m, D, d_rope, dI
         self.rows = np.ascontiguousarray(rows, np.uint8)
         self.scales = np.ascontiguousarray(scales, np.float32)
         self.block_table = np.ascontiguousarray(block_table, np.int32)
         self.win_rows = np.ascontiguousarray(win_rows, np.uint8)
         self.win_scales = np.ascontiguousarray(win_scales, np.float32)
-        self.kidx = None if kidx is None else np.ascontiguousarray(kidx, np.uint16)
+        self.kscale = None if kscale is None else np.ascontiguousarray(kscale, np.float32)
+        kdt = np.uint8 if kscale is not None else np.uint16
+        self.kidx = None if kidx is None else np.ascontiguousarray(kidx, kdt)
         self.n_win = self.win_scales.shape[-1]
         self.bt_stride = self.block_table.shape[-1]
 
@@ -271,10 +293,13 @@ class CacheView:
 
     def gather_keys(self, slot, N):
         keys = np.zeros((max(N, 1), self.dI))
-        lib().csla_orc_gather_keys(_p(self.kidx, ctypes.c_uint16), _p(self.block_table, ctypes.c_int32),
+        lib().csla_orc_gather_keys(self.kidx.ctypes.data, self._kscale_p(), _p(self.block_table, ctypes.c_int32),
                                    self.bt_stride, int(slot), int(N), self.m, self.dI,
                                    _p(keys, ctypes.c_double))
         return keys[:N]
+
+    def _kscale_p(self):
+        return None if self.kscale is None else _p(self.kscale, ctypes.c_float)
 
 
 def csa_decode(cv: CacheView, slots, lens, q, gamma_q, cq, W, head_w, sink, HI, k, eps=1e-6,
@@ -288,7 +313,7 @@ def csa_decode(cv: CacheView, slots, lens, q, gamma_q, cq, W, head_w, sink, HI, 
     idx = np.zeros((B, k), np.int32)
     out = np.zeros((B, H, D))
     lib().csla_orc_csa_decode(
-        _p(cv.rows, ctypes.c_uint8), _p(cv.scales, ctypes.c_float), _p(cv.kidx, ctypes.c_uint16),
+        _p(cv.rows, ctypes.c_uint8), _p(cv.scales, ctypes.c_float), cv.kidx.ctypes.data, cv._kscale_p(),
         _p(cv.block_table, ctypes.c_int32), cv.bt_stride, _p(cv.win_rows, ctypes.c_uint8),
         _p(cv.win_scales, ctypes.c_float), cv.n_win, _p(slots, ctypes.c_int32),
         _p(lens, ctypes.c_int32), B, cv.m, H, D, cv.d_rope, HI, cv.dI, dc, k, eps, theta,
@@ -319,13 +344,14 @@ def num_threads():
 
 # ---------------------------------------------------------------- expected state after appends
 def expected_append(raw_kv, raw_idx, L0, L1, m, gamma_kv, wg, gb, wgi=None, gbi=None, eps=1e-6,
-                    theta=10000.0, d_rope=64, window_from=0):
+                    theta=10000.0, d_rope=64, window_from=0, key_e4m3=False):
     """Rows the state and classical caches must hold after tokens L0..L1-1 of a
     request are appended (raw_kv/raw_idx hold the whole token history 0..L1-1).
 
     Returns dict: window {pos: (row, scale)}, entries {b: (row, scale)},
-    keys {b: bf16 key} for every block completed by these tokens.  Window
-    rows are produced for positions >= window_from only.
+    keys {b: bf16 key, or (E4M3 codes, scale) with key_e4m3} for every block
+    completed by these tokens.  Window rows are produced for positions >=
+    window_from only.
     """
     out = {"window": {}, "entries": {}, "keys": {}}
     for p in range(max(L0, window_from), L1):
@@ -336,5 +362,6 @@ def expected_append(raw_kv, raw_idx, L0, L1, m, gamma_kv, wg, gb, wgi=None, gbi=
         xs = raw_kv[b * m:(b + 1) * m]
         out["entries"][b] = compressed_row(xs, wg, gb, gamma_kv, b, eps, theta, d_rope)
         if raw_idx is not None and wgi is not None:
-            out["keys"][b] = index_key(raw_idx[b * m:(b + 1) * m], wgi, gbi)
+            xi = raw_idx[b * m:(b + 1) * m]
+            out["keys"][b] = index_key_e4m3(xi, wgi, gbi) if key_e4m3 else index_key(xi, wgi, gbi)
     return out

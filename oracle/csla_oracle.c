@@ -239,6 +239,38 @@ void csla_orc_index_key(const double *xis, int m, const double *wgi, const doubl
     free(c);
 }
 
+/* E4M3 storage of an index key ([haiqwa] §FP4精度加速: the indexer's key /
+ * query path runs in low precision).  The pages fix neither the format nor
+ * the scale.  Reading: one power-of-two scale per entry, the smallest
+ * s = 2^e (-126 <= e <= 127) with 448 * s >= amax, amax = max |key dim| of
+ * the fp32 key; each dim's code is E4M3(fp32 key / s), round to nearest
+ * even, saturating (the division by a power of two is exact).  The key dim
+ * then reads e4m3(code) * s.  This is the definition written out: e is
+ * found by counting up from -126. */
+double csla_orc_key_scale_e4m3(double amax)
+{
+    int e = -126;
+    while (e < 127 && 448.0 * ldexp(1.0, e) < amax) ++e;
+    return ldexp(1.0, e);
+}
+
+void csla_orc_index_key_e4m3(const double *xis, int m, const double *wgi, const double *gbi, int dI,
+                             uint8_t *codes, float *scale_out)
+{
+    int e;
+    double amax = 0.0, s;
+    double *c = (double *)malloc(sizeof(double) * (size_t)dI);
+    csla_orc_gate_pool(xis, m, dI, wgi, gbi, c, NULL);
+    for (e = 0; e < dI; ++e) {
+        double v = fabs((double)(float)c[e]);
+        if (v > amax) amax = v;
+    }
+    s = csla_orc_key_scale_e4m3(amax);
+    for (e = 0; e < dI; ++e) codes[e] = (uint8_t)csla_orc_e4m3_from_f32((float)((double)(float)c[e] / s));
+    *scale_out = (float)s;
+    free(c);
+}
+
 /* ------------------------------------------------------------------ */
 /* Lightning indexer, top-k, attention                                 */
 /* ------------------------------------------------------------------ */
@@ -422,15 +454,23 @@ int csla_orc_gather_set(const uint8_t *rows, const float *scales, const int32_t 
 }
 
 /* Decoded index keys of the first N compressed entries of a request. */
-void csla_orc_gather_keys(const uint16_t *kidx, const int32_t *block_table, int bt_stride, int slot,
-                          long long N, int m, int dI, double *keys)
+/* Decoded index keys of entries 0..N-1 of `slot`: bf16 values, or (kscale
+ * not NULL) E4M3 codes times the entry's scale. */
+void csla_orc_gather_keys(const void *kidx, const float *kscale, const int32_t *block_table, int bt_stride,
+                          int slot, long long N, int m, int dI, double *keys)
 {
     int epp = ORC_PAGE_TOKENS / m, e;
     long long b;
     for (b = 0; b < N; ++b) {
         long long page = block_table[(size_t)slot * bt_stride + b / epp];
-        const uint16_t *k = kidx + ((size_t)page * epp + (size_t)(b % epp)) * dI;
-        for (e = 0; e < dI; ++e) keys[(size_t)b * dI + e] = csla_orc_bf16_value(k[e]);
+        size_t ent = (size_t)page * epp + (size_t)(b % epp);
+        if (kscale) {
+            const uint8_t *k = (const uint8_t *)kidx + ent * dI;
+            for (e = 0; e < dI; ++e) keys[(size_t)b * dI + e] = csla_orc_e4m3_value(k[e]) * (double)kscale[ent];
+        } else {
+            const uint16_t *k = (const uint16_t *)kidx + ent * dI;
+            for (e = 0; e < dI; ++e) keys[(size_t)b * dI + e] = csla_orc_bf16_value(k[e]);
+        }
     }
 }
 
@@ -438,7 +478,7 @@ void csla_orc_gather_keys(const uint16_t *kidx, const int32_t *block_table, int 
  * B requests, straight from the cache bytes.  Used for sampled parity checks
  * and, timed, as the CPU baseline.  q: [B][H][D]; cq: [B][dc]; W: [HI*dI][dc];
  * head_w: [B][HI]; idx_out: [B][k]; out: [B][H][D].  OpenMP over requests. */
-void csla_orc_csa_decode(const uint8_t *rows, const float *scales, const uint16_t *kidx,
+void csla_orc_csa_decode(const uint8_t *rows, const float *scales, const void *kidx, const float *kscale,
                          const int32_t *block_table, int bt_stride, const uint8_t *win_rows,
                          const float *win_scales, int n_win, const int32_t *slots,
                          const int32_t *lens, int B, int m, int H, int D, int d_rope, int HI, int dI,
@@ -456,7 +496,7 @@ void csla_orc_csa_decode(const uint8_t *rows, const float *scales, const uint16_
         double *set = (double *)malloc(sizeof(double) * (size_t)(k + n_win) * D);
         int n;
         csla_orc_index_query(cq + (size_t)b * dc, W, HI, dI, dc, qI);
-        csla_orc_gather_keys(kidx, block_table, bt_stride, slots[b], nv, m, dI, keys);
+        csla_orc_gather_keys(kidx, kscale, block_table, bt_stride, slots[b], nv, m, dI, keys);
         csla_orc_index_scores(qI, head_w + (size_t)b * HI, HI, dI, keys, nv, sc);
         csla_orc_topk(sc, (int)nv, k, idx_out + (size_t)b * k);
         n = csla_orc_gather_set(rows, scales, block_table, bt_stride, win_rows, win_scales, n_win,

@@ -79,6 +79,22 @@ def index_key(xis, wgi, gbi):
     return c.astype(ml_dtypes.bfloat16).view(np.uint16)
 
 
+def key_scale_e4m3(amax):
+    """2^ceil(log2(amax / 448)), exponent clamped to [-126, 127] (by frexp)."""
+    if amax <= 0:
+        return 2.0 ** -126
+    mant, ex = np.frexp(np.float64(amax) / 448.0)   # amax/448 = mant * 2^ex, mant in [0.5, 1)
+    e = ex - 1 if mant == 0.5 else ex
+    return 2.0 ** int(min(max(e, -126), 127))
+
+
+def index_key_e4m3(xis, wgi, gbi):
+    c = pool(xis, wgi, gbi).astype(np.float32)
+    s = key_scale_e4m3(float(np.max(np.abs(c))))
+    v = np.clip((c.astype(np.float64) / s).astype(np.float32), -448.0, 448.0)
+    return v.astype(ml_dtypes.float8_e4m3fn).view(np.uint8), s
+
+
 def scores(cq, W, w, keys, HI, dI):
     qI = (np.asarray(W, np.float64) @ np.asarray(cq, np.float64)).reshape(HI, dI)
     dots = np.asarray(keys, np.float64) @ qI.T          # [N, HI]

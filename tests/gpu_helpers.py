@@ -15,7 +15,7 @@ DEV = "cuda"
 
 def shape_of(w: Workload):
     return LayerShape(m=w.m, D=w.D, H=w.H, HI=w.HI or 16, dI=w.dI or 128, dc=w.dc or 1024, n_win=w.n_win,
-                      d_rope=w.d_rope, theta=w.theta, eps=w.eps)
+                      d_rope=w.d_rope, theta=w.theta, eps=w.eps, key_fmt=w.key_fmt)
 
 
 def act_tensor(w: Workload, x):
@@ -58,7 +58,10 @@ def upload_layer(w: Workload, cv, lens):
     lb = LayerBuffers(shape, len(lens), n_pages, cv.block_table.shape[1], DEV)
     lb.rows.copy_(torch.from_numpy(cv.rows))
     lb.scales.copy_(torch.from_numpy(cv.scales))
-    if w.is_csa:
+    if w.is_csa and cv.kscale is not None:
+        lb.kidx.copy_(torch.from_numpy(cv.kidx))
+        lb.kscale.copy_(torch.from_numpy(cv.kscale))
+    elif w.is_csa:
         lb.kidx.copy_(torch.from_numpy(cv.kidx.view(np.int16)))
     lb.block_table.copy_(torch.from_numpy(cv.block_table))
     lb.win_rows.copy_(torch.from_numpy(cv.win_rows))
@@ -71,7 +74,7 @@ def upload_layer(w: Workload, cv, lens):
 def cache_view(w: Workload, lb: LayerBuffers):
     h = lb.host_view()
     return oracle.CacheView(w.m, w.D, h["rows"], h["scales"], h["block_table"], h["win_rows"],
-                            h["win_scales"], h.get("kidx"), w.dI, w.d_rope)
+                            h["win_scales"], h.get("kidx"), w.dI, w.d_rope, kscale=h.get("kscale"))
 
 
 def assert_no_device_error():

@@ -35,7 +35,9 @@ def oracle_cache(w: Workload, lens, params=None, with_raw=False, stream_ids=None
     rb = oracle.row_bytes(w.D, w.d_rope)
     rows = np.zeros((n_pages, epp, rb), np.uint8)
     scales = np.zeros((n_pages, epp), np.float32)
-    kidx = np.zeros((n_pages, epp, max(w.dI, 1)), np.uint16) if w.is_csa else None
+    e4m3 = w.is_csa and w.key_fmt == 1
+    kidx = np.zeros((n_pages, epp, max(w.dI, 1)), np.uint8 if e4m3 else np.uint16) if w.is_csa else None
+    kscale = np.zeros((n_pages, epp), np.float32) if e4m3 else None
     win_rows = np.zeros((n_slots, w.n_win, rb), np.uint8)
     win_scales = np.zeros((n_slots, w.n_win), np.float32)
     raws = []
@@ -44,7 +46,7 @@ def oracle_cache(w: Workload, lens, params=None, with_raw=False, stream_ids=None
         raws.append(ts)
         exp = oracle.expected_append(ts["kv"], ts.get("idx"), 0, L, w.m, p["gamma_kv"], p["wg"],
                                      p["gb"], p.get("wgi"), p.get("gbi"), w.eps, w.theta, w.d_rope,
-                                     window_from=L - w.n_win)
+                                     window_from=L - w.n_win, key_e4m3=e4m3)
         for pos, (r, sc) in exp["window"].items():
             if pos >= L - w.n_win:
                 win_rows[s, pos % w.n_win] = r
@@ -53,7 +55,9 @@ def oracle_cache(w: Workload, lens, params=None, with_raw=False, stream_ids=None
             pg = bt[s, b // epp]
             rows[pg, b % epp] = r
             scales[pg, b % epp] = sc
-            if w.is_csa:
+            if e4m3:
+                kidx[pg, b % epp], kscale[pg, b % epp] = exp["keys"][b]
+            elif w.is_csa:
                 kidx[pg, b % epp] = exp["keys"][b]
-    cv = oracle.CacheView(w.m, w.D, rows, scales, bt, win_rows, win_scales, kidx, w.dI, w.d_rope)
+    cv = oracle.CacheView(w.m, w.D, rows, scales, bt, win_rows, win_scales, kidx, w.dI, w.d_rope, kscale=kscale)
     return (cv, raws, p) if with_raw else (cv, p)
