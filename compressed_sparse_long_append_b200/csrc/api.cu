@@ -64,6 +64,7 @@ int check_cfg(const csla_cfg *c) {
         return CSLA_ERR_UNSUPPORTED;
     if (c->H < 1 || c->H > 64) return CSLA_ERR_UNSUPPORTED;
     if (!(c->eps >= 0.f) || !(c->rope_theta > 0.f)) return CSLA_ERR_ARG;
+    if (c->key_fmt != CSLA_KEY_BF16 && c->key_fmt != CSLA_KEY_E4M3) return CSLA_ERR_UNSUPPORTED;
     return CSLA_OK;
 }
 
@@ -207,6 +208,7 @@ static int prep_compress(const csla_cfg *cfg, const csla_state *st, const csla_c
             !p->gbi)
             return CSLA_ERR_ARG;
         if (!aligned16(st->tail_idx)) return CSLA_ERR_ARG;
+        if (cfg->key_fmt == CSLA_KEY_E4M3 && !cache->kscale) return CSLA_ERR_ARG;
     }
     CompressArgs a{};
     a.m = cfg->m; a.D = cfg->D; a.d_rope = cfg->d_rope; a.dI = csa ? cfg->dI : 0; a.n_win = cfg->n_win;
@@ -218,6 +220,8 @@ static int prep_compress(const csla_cfg *cfg, const csla_state *st, const csla_c
     a.win_rows = st->win_rows; a.win_scales = st->win_scales; a.tail_kv = st->tail_kv;
     a.tail_idx = csa ? st->tail_idx : nullptr; a.len = st->len;
     a.rows = cache->rows; a.scales = cache->scales; a.kidx = csa ? cache->kidx : nullptr;
+    a.key_fmt = csa ? cfg->key_fmt : CSLA_KEY_BF16;
+    a.kscale = csa ? cache->kscale : nullptr;
     a.block_table = cache->block_table; a.bt_stride = cache->bt_stride; a.n_pages = cache->n_pages;
     a.n_slots = st->n_slots;
     if (tok) {
@@ -273,9 +277,12 @@ static int prep_indexer(const csla_cfg *cfg, const csla_state *st, const csla_ca
     if (scores_stride < max_len / cfg->m || check_queries(qs)) return CSLA_ERR_ARG;
     if (workspace_bytes < csla_workspace_size(cfg, CSLA_OP_INDEXER, B, max_len)) return CSLA_ERR_ARG;
     if (!aligned16(cq) || !aligned16(W_iq) || !aligned16(cache->kidx) || !aligned16(workspace)) return CSLA_ERR_ARG;
+    const bool e4m3 = cfg->key_fmt == CSLA_KEY_E4M3;
+    if (e4m3 && (!cache->kscale || !aligned16(cache->kscale))) return CSLA_ERR_ARG;
     const int NQ = nq_of(cfg->HI);
     CUtensorMap kmap, qmap;
-    if (!encode_bf16_2d(&kmap, cache->kidx, (uint64_t)cfg->dI, (uint64_t)cache->n_pages * 32, 32))
+    memset(&kmap, 0, sizeof(kmap));   // E4M3 keys arrive by 1-D bulk copies: no key tensor map
+    if (!e4m3 && !encode_bf16_2d(&kmap, cache->kidx, (uint64_t)cfg->dI, (uint64_t)cache->n_pages * 32, 32))
         return CSLA_ERR_CUDA;
     const int G = (qs && qs->one_request) ? indexer_rows_per_cta(NQ) : 1;
     if (!encode_bf16_2d(&qmap, workspace, (uint64_t)cfg->dI, (uint64_t)B * NQ, (uint32_t)(G * NQ)))
@@ -294,6 +301,9 @@ static int prep_indexer(const csla_cfg *cfg, const csla_state *st, const csla_ca
     a.max_len = max_len;
     a.cq = cq; a.W = W_iq; a.head_w = head_w; a.scores = scores; a.scores_stride = scores_stride;
     a.q_ws = reinterpret_cast<uint16_t *>(workspace);
+    a.key_fmt = cfg->key_fmt;
+    a.kidx8 = e4m3 ? reinterpret_cast<const uint8_t *>(cache->kidx) : nullptr;
+    a.kscale = e4m3 ? cache->kscale : nullptr;
     a.q_len = qs ? qs->q_len : nullptr;
     a.rows_per_cta = G;
     L->a = a;

@@ -56,6 +56,19 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two_codes) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Exponent of the E4M3 index-key scale: the smallest e (-126 <= e <= 127)
+// with 448 * 2^e >= amax (amax >= 0, an fp32 value).  With amax = f * 2^k,
+// f in [0.5, 1), 448 * 2^(k-9) = 0.875 * 2^k covers amax iff f <= 0.875,
+// i.e. iff amax's mantissa field is at most 0.75 * 2^23; zero and subnormal
+// amax take the minimum.
+__device__ __forceinline__ int key_exp_e4m3(float amax) {
+    const uint32_t bits = __float_as_uint(amax);
+    const int E = (int)(bits >> 23);
+    if (E == 0) return -126;
+    const int e = (bits & 0x7FFFFFu) <= 0x600000u ? E - 135 : E - 134;
+    return e < -126 ? -126 : (e > 127 ? 127 : e);
+}
+
 // ------------------------------------------------------------ programmatic dependent launch
 // Every libcsla kernel is launched with programmatic stream serialization
 // (programmatic dependent launch) and calls pdl_trigger() first (kernels that

@@ -422,7 +422,21 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs 
         if (m <= kSmallM) pool_small<T>(rows, m, wsm, alpha, part, v);
         else pool_block<T>(rows, m, wsm, alpha, part, xs, v, red);
         CSLA_TL_MARK(1);
-        for (int e = threadIdx.x; e < dI; e += kThreads) a.kidx[ent * dI + e] = f32_to_bf16_bits(v[e]);
+        if (a.key_fmt == CSLA_KEY_E4M3) {
+            // one power-of-two scale per entry: the smallest 2^e with
+            // 448 * 2^e >= max |key dim|, codes E4M3(key / 2^e), on fp32 values
+            float am = 0.f;
+            for (int e = threadIdx.x; e < dI; e += kThreads) am = fmaxf(am, fabsf(v[e]));
+            am = block_max<kThreads / 32>(am, red);
+            const int ex = key_exp_e4m3(am);
+            const float inv = __uint_as_float((uint32_t)(127 - min(ex, 126)) << 23);   // 2^-ex
+            uint8_t *k8 = reinterpret_cast<uint8_t *>(a.kidx) + ent * dI;
+            for (int e = threadIdx.x; e < dI; e += kThreads) k8[e] = f32_to_e4m3(__fmul_rn(v[e], inv));
+            if (threadIdx.x == 0) a.kscale[ent] = __uint_as_float((uint32_t)(ex + 127) << 23);
+        } else {
+            uint16_t *k16 = reinterpret_cast<uint16_t *>(a.kidx) + ent * dI;
+            for (int e = threadIdx.x; e < dI; e += kThreads) k16[e] = f32_to_bf16_bits(v[e]);
+        }
         CSLA_TL_MARK(2);
     }
 }

@@ -198,23 +198,32 @@ __global__ void __launch_bounds__(kProjThreads) iq_project_wide_kernel(IndexerAr
     }
 }
 
-constexpr int kStages = 3;
 constexpr int kTileE = 128;          // entries per tile
 constexpr int kPageE = 32;           // CSA entries per 128-token page
 constexpr int kTPC = 8;              // tiles per CTA (consecutive, one request)
 // warp 0: TMA, warp 1: MMA, then 4 epilogue warps per set of query rows
 // (set s takes the group's rows s, s + sets, ...): one set for G = 1, one
 // per row up to 7 rows (balanced: 5 at 16 index heads), else four.
+// E4M3 keys add four converter warps after the epilogue warps.
 template <int G>
 constexpr int idx_epi_sets() { return G == 1 ? 1 : (G <= 7 ? G : 4); }
-template <int G>
-constexpr int idx_threads() { return 64 + 128 * idx_epi_sets<G>(); }
+constexpr int kConvWarps = 4;
+template <int G, bool kE4M3>
+constexpr int idx_threads() { return 64 + 128 * idx_epi_sets<G>() + (kE4M3 ? 32 * kConvWarps : 0); }
 
-template <int DI, int NQ, int G>
+// bf16 key tiles (what the MMA reads): a 3-stage ring filled by TMA, or with
+// E4M3 keys a 2-stage ring filled by the converter warps from a 3-stage ring
+// of bulk-copied codes and scales.
+template <int DI, int NQ, int G, bool kE4M3>
 struct IdxSmem {
+    static constexpr int kStages = kE4M3 ? 2 : 3;
+    static constexpr int kStages8 = 3;
     static constexpr int kKeyBytes = kTileE * DI * 2;
+    static constexpr int kCodeBytes = kTileE * DI;          // E4M3 codes of a tile
+    static constexpr int kCode8Bytes = kCodeBytes + 1024;   // + the entries' scales (512 B, padded: 1024-aligned stages)
     static constexpr int kQBytes = G * NQ * DI * 2;
-    static constexpr int kBytes = kStages * kKeyBytes + kQBytes + 1024 /*align*/ + 1024 /*barriers, pages, weights*/;
+    static constexpr int kBytes = kStages * kKeyBytes + (kE4M3 ? kStages8 * kCode8Bytes : 0) + kQBytes +
+                                  1024 /*align*/ + 1024 /*barriers, pages, weights*/;
 };
 
 // Two accumulators of G*NQ columns, rounded up to a power of two >= 32.
@@ -227,21 +236,25 @@ constexpr uint32_t kTmemCols() {
 // entries each) of the query rows r0 = blockIdx.y*G .. r0+G-1, which all
 // read the keys of request slots[r0]: one key tile feeds one MMA of N = G*NQ
 // query columns (decode: G = 1; query rows of one request: G > 1).
-template <int DI, int NQ, int HI, int G>
-__global__ void __launch_bounds__(idx_threads<G>())
+template <int DI, int NQ, int HI, int G, bool kE4M3>
+__global__ void __launch_bounds__(idx_threads<G, kE4M3>())
     indexer_kernel(IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap qmap) {
     CSLA_TL_SCOPE(kTlIndexer);
-    using S = IdxSmem<DI, NQ, G>;
+    using S = IdxSmem<DI, NQ, G, kE4M3>;
+    constexpr int kStages = S::kStages;
     constexpr int N = G * NQ;
+    constexpr int kConvWarp0 = 2 + 4 * idx_epi_sets<G>();   // first converter warp (E4M3 keys)
     static_assert(N % 16 == 0 && N <= 256, "UMMA N for M = 128");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t *qbuf = base + kStages * S::kKeyBytes;
+    uint8_t *codes = base + kStages * S::kKeyBytes;                       // E4M3: [kStages8][codes | scales]
+    uint8_t *qbuf = codes + (kE4M3 ? S::kStages8 * S::kCode8Bytes : 0);
     uint64_t *bars = reinterpret_cast<uint64_t *>(qbuf + S::kQBytes);
     uint64_t *full = bars, *empty = bars + kStages, *tfull = bars + 2 * kStages, *tempty = tfull + 2;
     uint64_t *qfull = tempty + 2;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(qfull + 1);
+    uint64_t *full8 = qfull + 1, *empty8 = full8 + S::kStages8;            // E4M3 only
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(empty8 + S::kStages8);
     int *pages = reinterpret_cast<int *>(tmem_holder + 1);      // [kTPC * 4]
     int *row_nv = pages + kTPC * 4;                              // [G] entries scored below this (-1: skip)
     int *row_lo = row_nv + G;                                    // [G] first entry scored
@@ -258,8 +271,12 @@ __global__ void __launch_bounds__(idx_threads<G>())
     if (threadIdx.x == 0) {
         abort_flag = 0;
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(full + s, 1);
+            mbar_init(full + s, kE4M3 ? kConvWarps : 1);   // TMA, or one arrival per converter warp
             mbar_init(empty + s, 1);
+        }
+        for (int s = 0; s < S::kStages8; ++s) {
+            mbar_init(full8 + s, 1);
+            mbar_init(empty8 + s, kConvWarps);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(tfull + i, 1);
@@ -274,7 +291,7 @@ __global__ void __launch_bounds__(idx_threads<G>())
         if (a.range != 2 && slot_ok && lane < kTPC * 4 && col < a.bt_stride)
             pg = __ldg(a.block_table + (size_t)slot * a.bt_stride + col);
         if (lane == 0) {
-            tma_prefetch_desc(&kmap);
+            if (!kE4M3) tma_prefetch_desc(&kmap);
             tma_prefetch_desc(&qmap);
         }
     }
@@ -282,7 +299,7 @@ __global__ void __launch_bounds__(idx_threads<G>())
         tmem_alloc(tmem_holder, kTmemCols<N>());
         tmem_relinquish();
     }
-    for (int i = threadIdx.x; i < G * HI; i += idx_threads<G>()) {
+    for (int i = threadIdx.x; i < G * HI; i += idx_threads<G, kE4M3>()) {
         const int r = r0 + i / HI;
         hw[i] = r < a.B ? __ldg(a.head_w + (size_t)r * HI + i % HI) : 0.f;
     }
@@ -353,27 +370,51 @@ __global__ void __launch_bounds__(idx_threads<G>())
 #pragma unroll
             for (int h = 0; h < DI / 64; ++h) tma_load_2d(qbuf + h * N * 128, &qmap, h * 64, r0 * NQ, qfull);
             int n = 0;
-            for (int t = 0; t < n_tiles; ++t, ++n) {
-                const int s = n % kStages;
-                if (n >= kStages && !mbar_wait(empty + s, ((n / kStages) - 1) & 1, &abort_flag)) break;
-                uint8_t *kb = base + s * S::kKeyBytes;
-                int np = 0;
+            if constexpr (kE4M3) {
+                // codes (32 entries x DI bytes) and scales (32 floats) of each
+                // page: two 1-D bulk copies per page into the code ring
+                constexpr int kS8 = S::kStages8;
+                for (int t = 0; t < n_tiles; ++t, ++n) {
+                    const int s = n % kS8;
+                    if (n >= kS8 && !mbar_wait(empty8 + s, ((n / kS8) - 1) & 1, &abort_flag)) break;
+                    uint8_t *cb = codes + s * S::kCode8Bytes;
+                    int np = 0;
 #pragma unroll
-                for (int p = 0; p < 4; ++p) np += pages[t * 4 + p] >= 0;
-                mbar_arrive_expect_tx(full + s, (uint32_t)(np * kPageE * DI * 2));
+                    for (int p = 0; p < 4; ++p) np += pages[t * 4 + p] >= 0;
+                    mbar_arrive_expect_tx(full8 + s, (uint32_t)(np * kPageE * (DI + 4)));
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const int pg = pages[t * 4 + p];
-                    if (pg < 0) continue;
-#pragma unroll
-                    for (int h = 0; h < DI / 64; ++h)
-                        tma_load_2d(kb + h * (kTileE * 128) + p * (kPageE * 128), &kmap, h * 64, pg * kPageE,
-                                    full + s);
+                    for (int p = 0; p < 4; ++p) {
+                        const int pg = pages[t * 4 + p];
+                        if (pg < 0) continue;
+                        bulk_load(cb + p * kPageE * DI, a.kidx8 + (size_t)pg * kPageE * DI, kPageE * DI, full8 + s);
+                        bulk_load(cb + S::kCodeBytes + p * kPageE * 4, a.kscale + (size_t)pg * kPageE, kPageE * 4,
+                                  full8 + s);
+                    }
                 }
+                for (int i = (n > kS8 ? n - kS8 : 0); i < n; ++i) mbar_wait(full8 + (i % kS8), (i / kS8) & 1, nullptr);
+            } else {
+                for (int t = 0; t < n_tiles; ++t, ++n) {
+                    const int s = n % kStages;
+                    if (n >= kStages && !mbar_wait(empty + s, ((n / kStages) - 1) & 1, &abort_flag)) break;
+                    uint8_t *kb = base + s * S::kKeyBytes;
+                    int np = 0;
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) np += pages[t * 4 + p] >= 0;
+                    mbar_arrive_expect_tx(full + s, (uint32_t)(np * kPageE * DI * 2));
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const int pg = pages[t * 4 + p];
+                        if (pg < 0) continue;
+#pragma unroll
+                        for (int h = 0; h < DI / 64; ++h)
+                            tma_load_2d(kb + h * (kTileE * 128) + p * (kPageE * 128), &kmap, h * 64, pg * kPageE,
+                                        full + s);
+                    }
+                }
+                // every issued copy must land before the CTA may exit
+                for (int i = (n > kStages ? n - kStages : 0); i < n; ++i)
+                    mbar_wait(full + (i % kStages), (i / kStages) & 1, nullptr);
             }
-            // every issued copy must land before the CTA may exit
-            for (int i = (n > kStages ? n - kStages : 0); i < n; ++i)
-                mbar_wait(full + (i % kStages), (i / kStages) & 1, nullptr);
             mbar_wait(qfull, 0, nullptr);
             CSLA_TL_MARK_ANY(4);
         }
@@ -404,6 +445,55 @@ __global__ void __launch_bounds__(idx_threads<G>())
                 }
             }
             if (n > 0) mbar_wait(tfull + ((n - 1) & 1), ((n - 1) / 2) & 1, nullptr);
+        }
+    } else if (kE4M3 && warp >= kConvWarp0) {
+        // converter warps: E4M3 codes * scale -> bf16, exactly (every E4M3
+        // value times a power of two in the normal range is a bf16 value),
+        // into the SW128 K-major key layout the TMA would have produced:
+        // entry r, 8-dim group g at half g/8, row r, 16-byte slot (g%8)^(r%8).
+        // Thread i converts 16-byte code chunks i, i+128, ... (consecutive
+        // threads read consecutive chunks).
+        constexpr int kS8 = S::kStages8;
+        constexpr int kCPR = DI / 16;   // code chunks per entry
+        const int ci = threadIdx.x - 32 * kConvWarp0;
+        int n = 0;
+        for (int t = 0; t < n_tiles; ++t, ++n) {
+            const int s8 = n % kS8, s = n % kStages;
+            if (!warp_all(mbar_wait(full8 + s8, (n / kS8) & 1, &abort_flag))) break;
+            if (n >= kStages && !warp_all(mbar_wait(empty + s, ((n / kStages) - 1) & 1, &abort_flag))) break;
+            const uint8_t *cb = codes + s8 * S::kCode8Bytes;
+            const float *sc = reinterpret_cast<const float *>(cb + S::kCodeBytes);
+            uint8_t *kb = base + s * S::kKeyBytes;
+#pragma unroll
+            for (int k = 0; k < kCPR; ++k) {
+                const int f = ci + 128 * k;
+                const int r = f / kCPR, c = f % kCPR;
+                const uint4 v = *reinterpret_cast<const uint4 *>(cb + r * DI + 16 * c);
+                const float scl = sc[r];
+                const __nv_bfloat162 sv = __floats2bfloat162_rn(scl, scl);   // a power of two: exact
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                uint32_t o[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t lo = e4m3x2_to_bf16x2(w[e] & 0xFFFFu), hi = e4m3x2_to_bf16x2(w[e] >> 16);
+                    __nv_bfloat162 bl = *reinterpret_cast<const __nv_bfloat162 *>(&lo);
+                    __nv_bfloat162 bh = *reinterpret_cast<const __nv_bfloat162 *>(&hi);
+                    bl = __hmul2(bl, sv);
+                    bh = __hmul2(bh, sv);
+                    o[2 * e] = *reinterpret_cast<const uint32_t *>(&bl);
+                    o[2 * e + 1] = *reinterpret_cast<const uint32_t *>(&bh);
+                }
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int g = 2 * c + q;                 // dims 8g .. 8g+7
+                    const int h = g >> 3, j = g & 7;
+                    *reinterpret_cast<uint4 *>(kb + h * (kTileE * 128) + r * 128 + ((j ^ (r & 7)) << 4)) =
+                        make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive_warp(full + s);
+            mbar_arrive_warp(empty8 + s8);
         }
     } else {
         // TMEM lanes 32*(warp%4).. are this warp's key rows; set `es` takes
@@ -471,31 +561,39 @@ __global__ void __launch_bounds__(idx_threads<G>())
     }
 }
 
-template <int DI, int NQ, int HI, int G>
+template <int DI, int NQ, int HI, int G, bool kE4M3>
 cudaError_t launch_indexer_t(const IndexerArgs &a, const CUtensorMap &kmap, const CUtensorMap &qmap,
                              cudaStream_t stream) {
-    using S = IdxSmem<DI, NQ, G>;
+    using S = IdxSmem<DI, NQ, G, kE4M3>;
+    static_assert(S::kBytes <= 232448, "shared memory budget");
     static int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(indexer_kernel<DI, NQ, HI, G>,
+        cudaError_t e = cudaFuncSetAttribute(indexer_kernel<DI, NQ, HI, G, kE4M3>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
     const int groups = (a.tiles_per_req + kTPC - 1) / kTPC;
-    return launch_pdl(indexer_kernel<DI, NQ, HI, G>, dim3(groups, (a.B + G - 1) / G), dim3(idx_threads<G>()),
-                      S::kBytes, stream, a, kmap, qmap);
+    return launch_pdl(indexer_kernel<DI, NQ, HI, G, kE4M3>, dim3(groups, (a.B + G - 1) / G),
+                      dim3(idx_threads<G, kE4M3>()), S::kBytes, stream, a, kmap, qmap);
+}
+
+template <int DI, int NQ, int HI, bool kE4M3>
+cudaError_t launch_indexer_g(const IndexerArgs &a, const CUtensorMap &kmap, const CUtensorMap &qmap,
+                             cudaStream_t stream) {
+    if (a.rows_per_cta == 1) return launch_indexer_t<DI, NQ, HI, 1, kE4M3>(a, kmap, qmap, stream);
+    if (a.rows_per_cta == indexer_rows_per_cta(NQ))
+        return launch_indexer_t<DI, NQ, HI, indexer_rows_per_cta(NQ), kE4M3>(a, kmap, qmap, stream);
+    return cudaErrorInvalidValue;
 }
 
 template <int DI, int NQ, int HI>
-cudaError_t launch_indexer_g(const IndexerArgs &a, const CUtensorMap &kmap, const CUtensorMap &qmap,
+cudaError_t launch_indexer_k(const IndexerArgs &a, const CUtensorMap &kmap, const CUtensorMap &qmap,
                              cudaStream_t stream) {
-    if (a.rows_per_cta == 1) return launch_indexer_t<DI, NQ, HI, 1>(a, kmap, qmap, stream);
-    if (a.rows_per_cta == indexer_rows_per_cta(NQ))
-        return launch_indexer_t<DI, NQ, HI, indexer_rows_per_cta(NQ)>(a, kmap, qmap, stream);
-    return cudaErrorInvalidValue;
+    if (a.key_fmt == CSLA_KEY_E4M3) return launch_indexer_g<DI, NQ, HI, true>(a, kmap, qmap, stream);
+    return launch_indexer_g<DI, NQ, HI, false>(a, kmap, qmap, stream);
 }
 
 // len0[b] = len[slots[b]], read after the grid wait (0 for a bad slot).
@@ -514,16 +612,16 @@ cudaError_t launch_scoring(const IndexerArgs &a, const CUtensorMap &kmap, const 
     // HI is a template parameter so the epilogue's head loop is unrolled.
     if (a.dI == 128) {
         switch (a.HI) {
-            case 16: return launch_indexer_g<128, 48, 16>(a, kmap, qmap, stream);
-            case 8: return launch_indexer_g<128, 32, 8>(a, kmap, qmap, stream);
-            case 4: return launch_indexer_g<128, 16, 4>(a, kmap, qmap, stream);
+            case 16: return launch_indexer_k<128, 48, 16>(a, kmap, qmap, stream);
+            case 8: return launch_indexer_k<128, 32, 8>(a, kmap, qmap, stream);
+            case 4: return launch_indexer_k<128, 16, 4>(a, kmap, qmap, stream);
             default: break;
         }
     } else if (a.dI == 64) {
         switch (a.HI) {
-            case 16: return launch_indexer_g<64, 48, 16>(a, kmap, qmap, stream);
-            case 8: return launch_indexer_g<64, 32, 8>(a, kmap, qmap, stream);
-            case 4: return launch_indexer_g<64, 16, 4>(a, kmap, qmap, stream);
+            case 16: return launch_indexer_k<64, 48, 16>(a, kmap, qmap, stream);
+            case 8: return launch_indexer_k<64, 32, 8>(a, kmap, qmap, stream);
+            case 4: return launch_indexer_k<64, 16, 4>(a, kmap, qmap, stream);
             default: break;
         }
     }

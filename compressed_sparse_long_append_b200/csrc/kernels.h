@@ -51,7 +51,9 @@ struct CompressArgs {
     int32_t *len;
     uint8_t *rows;
     float *scales;
-    uint16_t *kidx;
+    void *kidx;           // bf16 keys, or E4M3 codes (key_fmt)
+    float *kscale;        // E4M3 keys: per-entry power-of-two scale
+    int key_fmt;
     const int32_t *block_table;
     int bt_stride, n_pages, n_slots;
     uint8_t *tok_rows;    // optional: window-format row of every new token
@@ -87,6 +89,9 @@ struct IndexerArgs {
     float *scores;
     int scores_stride;
     uint16_t *q_ws;     // [B][NQ][dI] bf16
+    int key_fmt;                // CSLA_KEY_BF16 (keys by TMA tensor map) or CSLA_KEY_E4M3:
+    const uint8_t *kidx8;       //   E4M3 key codes [n_pages * 32][dI]
+    const float *kscale;        //   and per-entry scales [n_pages * 32]
     const int32_t *q_len;   // optional per-row visible length (else len[slot])
     int rows_per_cta;       // 1, or indexer_rows_per_cta(NQ) when all rows share slots[0]
     int range;              // 0: all visible entries; 1: those below len0[b]/m; 2: those from len0[b]/m on
