@@ -52,6 +52,7 @@ def parse():
     ap.add_argument("--no-hca", action="store_true", help="skip the HCA layer measurement")
     ap.add_argument("--no-prefill", action="store_true", help="skip the CSA prefill-chunk measurement")
     ap.add_argument("--prefill-only", action="store_true", help="only the CSA prefill-chunk measurement")
+    ap.add_argument("--no-e4m3", action="store_true", help="skip the CSA decode leg with E4M3 index keys")
     ap.add_argument("--no-invariance", action="store_true",
                     help="skip the ragged 64-request CSA + HCA decode measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -144,7 +145,8 @@ def build_layer(shape_kw, n_req, L0s, seed, rank, device):
     from csla_synth import torch_gen
 
     sh = LayerShape(m=shape_kw["m"], D=shape_kw["D"], H=shape_kw["H"], HI=shape_kw.get("HI", 16),
-                    dI=shape_kw.get("dI", 128), dc=shape_kw.get("dc", 1024), n_win=shape_kw["n_win"])
+                    dI=shape_kw.get("dI", 128), dc=shape_kw.get("dc", 1024), n_win=shape_kw["n_win"],
+                    key_fmt=shape_kw.get("key_fmt", 0))
     L_cap = shape_kw["L"] + HEADROOM
     pages_per = -(-L_cap // 128)
     n_pages = n_req * pages_per
@@ -445,6 +447,39 @@ def prefill_leg(W, K, seed, rank, world, device, variant, profile=False):
            "l2": "inputs larger than L2 (q 268 MB, fp32 scores 1.09 GB per chunk)",
            "launch": "one CUDA graph per chunk, K replays between one event pair"}
     del st, lb
+    torch.cuda.empty_cache()
+    return out
+
+
+def e4m3_leg(W, K, seed, rank, world, device, variant):
+    """The headline CSA decode workload (8 x 131072, top-k 512) with its index
+    keys stored as E4M3 codes plus one power-of-two scale per entry (132
+    instead of 256 bytes per entry): the same step, timed the same way, and
+    the indexer call's achieved bandwidth on its algorithmic bytes."""
+    import torch
+    kw = dict(CSA, key_fmt=1)
+    R, m, B = CSA_COPIES, kw["m"], kw["B"]
+    before = -(-(W + K) // R)
+    L0s = [kw["L"] - before - (b % m) for b in range(B)]
+    lb, cp, params = build_layer(kw, B, L0s, seed, rank, device)
+    inputs = step_inputs(kw, B, W + K, seed, rank, device)
+    CsaStep.fused = False
+    steps = make_copies(CsaStep, lb, cp, params, kw, variant, device, R)
+    torch.cuda.synchronize()
+    ms = dp_max(run_steps(steps, inputs, W, K), world, device)
+    seg = breakdown(steps, inputs, W, K)
+    ms_idx = call_time(steps, inputs, W, K, 1)
+    nv = sum(int(x) // m for st in steps for x in st.lb.len.tolist()) / R
+    idx_bytes = nv * (kw["dI"] + 4 + 4) + kw["HI"] * kw["dI"] * kw["dc"] * 2
+    peak, peak_kind = peaks()
+    achieved = idx_bytes / (ms_idx * 1e-3) / 1e9
+    out = {"workload": "csa_decode_B8_L131072_e4m3_keys", "tokens_per_s": B * world / (ms * 1e-3),
+           "ms_per_step": ms, "key_bytes_per_entry": kw["dI"] + 4,
+           "segments_ms": {"compress_append": seg[0], "indexer_scores": seg[1], "topk_select": seg[2],
+                           "csa_attend": seg[3]},
+           "indexer": {"call_ms": ms_idx, "algorithmic_bytes": idx_bytes, "achieved_gbs": achieved,
+                       "frac": achieved / peak, "peak": peak, "peak_kind": peak_kind}}
+    del steps, lb, inputs
     torch.cuda.empty_cache()
     return out
 
@@ -937,11 +972,14 @@ def main():
             except Exception as e:  # the baseline never blocks the GPU line
                 pre["cpu_baseline"] = {"value": None, "unit": "tokens/s", "cores": 0, "kind": "oracle",
                                        "sample": "failed: %s" % e}
+    if args.no_hca and args.no_prefill and not args.profile:
+        del steps, lb
+        torch.cuda.empty_cache()
+    e4 = None
+    if not args.no_e4m3 and not args.profile:
+        e4 = e4m3_leg(W, K, seed, rank, world, device, args.variant)
     inv = None
     if not args.no_invariance and not args.profile:
-        if args.no_hca and args.no_prefill:
-            del steps, lb
-            torch.cuda.empty_cache()
         inv = invariance_leg(W, K, seed + 4, rank, world, device, args.variant)
 
     cpu = None
@@ -987,6 +1025,7 @@ def main():
             "clocks": clocks,
             "hca_decode": hca,
             "csa_prefill": pre,
+            "csa_decode_e4m3_keys": e4,
             "invariance_decode": inv,
         }
         print(json.dumps(line), flush=True)

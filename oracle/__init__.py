@@ -52,6 +52,9 @@ def lib():
             "csla_orc_compressed_row": (None, [dp, I, dp, dp, dp, I, I, D_, D_, ll, u8p, fp]),
             "csla_orc_index_key": (None, [dp, I, dp, dp, I, u16p]),
             "csla_orc_key_scale_e4m3": (D_, [D_]),
+            "csla_orc_gate_pool_channel": (None, [dp, I, I, dp, dp, dp]),
+            "csla_orc_key_bf16": (None, [dp, I, u16p]),
+            "csla_orc_key_e4m3": (None, [dp, I, u8p, fp]),
             "csla_orc_index_key_e4m3": (None, [dp, I, dp, dp, I, u8p, fp]),
             "csla_orc_index_query": (None, [dp, dp, I, I, I, dp]),
             "csla_orc_index_scores": (None, [dp, dp, I, I, dp, ll, dp]),
@@ -155,6 +158,40 @@ def gate_pool(xs, wg, gb=None):
                              None if g is None else _p(g, ctypes.c_double), _p(out, ctypes.c_double),
                              _p(alpha, ctypes.c_double))
     return out, alpha
+
+
+def gate_pool_channel(xs, w, b):
+    """Per-channel gated pooling: out_d = sum_i softmax_i(x_id w_d + b_id) x_id."""
+    xs = _d(xs)
+    m, width = xs.shape
+    w, b = _d(w), _d(np.broadcast_to(b, (m, width)))
+    out = np.zeros(width)
+    lib().csla_orc_gate_pool_channel(_p(xs, ctypes.c_double), m, width, _p(w, ctypes.c_double),
+                                     _p(b, ctypes.c_double), _p(out, ctypes.c_double))
+    return out
+
+
+def key_bf16(c):
+    c = _d(c)
+    key = np.zeros(c.shape[-1], np.uint16)
+    lib().csla_orc_key_bf16(_p(c, ctypes.c_double), c.shape[-1], _p(key, ctypes.c_uint16))
+    return key
+
+
+def key_e4m3(c):
+    c = _d(c)
+    codes = np.zeros(c.shape[-1], np.uint8)
+    sc = np.zeros(1, np.float32)
+    lib().csla_orc_key_e4m3(_p(c, ctypes.c_double), c.shape[-1], _p(codes, ctypes.c_uint8), _p(sc, ctypes.c_float))
+    return codes, float(sc[0])
+
+
+def compressed_row_channel(xs, w, b, gamma, bk, eps=1e-6, theta=10000.0, d_rope=64):
+    """Compressed entry of block bk with the per-channel gate: pool, then
+    RMSNorm * gamma, RoPE at position bk * m, quantise (as compressed_row)."""
+    m = np.asarray(xs).shape[0]
+    y = rope(rmsnorm(gate_pool_channel(xs, w, b), gamma, eps), bk * m, theta, d_rope)
+    return quantize(y, d_rope)
 
 
 def window_row(x, gamma, pos, eps=1e-6, theta=10000.0, d_rope=64):
@@ -344,14 +381,15 @@ def num_threads():
 
 # ---------------------------------------------------------------- expected state after appends
 def expected_append(raw_kv, raw_idx, L0, L1, m, gamma_kv, wg, gb, wgi=None, gbi=None, eps=1e-6,
-                    theta=10000.0, d_rope=64, window_from=0, key_e4m3=False):
+                    theta=10000.0, d_rope=64, window_from=0, key_e4m3=False, per_channel=False):
     """Rows the state and classical caches must hold after tokens L0..L1-1 of a
     request are appended (raw_kv/raw_idx hold the whole token history 0..L1-1).
 
     Returns dict: window {pos: (row, scale)}, entries {b: (row, scale)},
     keys {b: bf16 key, or (E4M3 codes, scale) with key_e4m3} for every block
     completed by these tokens.  Window rows are produced for positions >=
-    window_from only.
+    window_from only.  per_channel: the per-channel gate (gb, gbi are
+    [m][width] biases).
     """
     out = {"window": {}, "entries": {}, "keys": {}}
     for p in range(max(L0, window_from), L1):
@@ -360,8 +398,15 @@ def expected_append(raw_kv, raw_idx, L0, L1, m, gamma_kv, wg, gb, wgi=None, gbi=
         if (b + 1) * m <= L0:
             continue
         xs = raw_kv[b * m:(b + 1) * m]
-        out["entries"][b] = compressed_row(xs, wg, gb, gamma_kv, b, eps, theta, d_rope)
+        if per_channel:
+            out["entries"][b] = compressed_row_channel(xs, wg, gb, gamma_kv, b, eps, theta, d_rope)
+        else:
+            out["entries"][b] = compressed_row(xs, wg, gb, gamma_kv, b, eps, theta, d_rope)
         if raw_idx is not None and wgi is not None:
             xi = raw_idx[b * m:(b + 1) * m]
-            out["keys"][b] = index_key_e4m3(xi, wgi, gbi) if key_e4m3 else index_key(xi, wgi, gbi)
+            if per_channel:
+                c = gate_pool_channel(xi, wgi, gbi)
+                out["keys"][b] = key_e4m3(c) if key_e4m3 else key_bf16(c)
+            else:
+                out["keys"][b] = index_key_e4m3(xi, wgi, gbi) if key_e4m3 else index_key(xi, wgi, gbi)
     return out

@@ -195,6 +195,31 @@ void csla_orc_gate_pool(const double *xs, int m, int width, const double *wg, co
     free(g);
 }
 
+/* Per-channel gated pooling (the compressor variant with a gate per
+ * channel; the pages give no compressor formula at all, see gate_pool).
+ * Reading: channel d of token i has the gate g_id = x_id * w_d + b_id
+ * (b is [m][width]); alpha_id = softmax over the m tokens of g_.d, per
+ * channel; out_d = sum_i alpha_id x_id.  With w = 0 and b_id = beta_i for
+ * every d it is gate_pool with wg = 0, gb = beta. */
+void csla_orc_gate_pool_channel(const double *xs, int m, int width, const double *w, const double *b,
+                                double *out)
+{
+    int i, d;
+    for (d = 0; d < width; ++d) {
+        double gmax = -INFINITY, z = 0.0, acc = 0.0;
+        for (i = 0; i < m; ++i) {
+            double g = xs[(size_t)i * width + d] * w[d] + b[(size_t)i * width + d];
+            if (g > gmax) gmax = g;
+        }
+        for (i = 0; i < m; ++i) z += exp(xs[(size_t)i * width + d] * w[d] + b[(size_t)i * width + d] - gmax);
+        for (i = 0; i < m; ++i) {
+            double a = exp(xs[(size_t)i * width + d] * w[d] + b[(size_t)i * width + d] - gmax) / z;
+            acc += a * xs[(size_t)i * width + d];
+        }
+        out[d] = acc;
+    }
+}
+
 /* Sliding-window row of token `pos` ([haiqwa] §Partial RoPE位置编码, sliding-window paragraph;
  * [silicon] §两大压缩注意力: the last 128 raw tokens kept uncompressed).
  * Reading: the row gets the same RMSNorm (gamma_kv), RoPE at its own position
@@ -225,6 +250,8 @@ void csla_orc_compressed_row(const double *xs, int m, const double *wg, const do
     free(y);
 }
 
+void csla_orc_key_bf16(const double *c, int dI, uint16_t *key);
+
 /* Compressed index key of a CSA block ([silicon] §CSA: the indexer derives its own
  * compressed keys from the same KV hidden states and scores queries against them).
  * Reading: its own scalar gate (wgi, gbi), no norm, no RoPE, stored bf16
@@ -235,8 +262,15 @@ void csla_orc_index_key(const double *xis, int m, const double *wgi, const doubl
     int e;
     double *c = (double *)malloc(sizeof(double) * (size_t)dI);
     csla_orc_gate_pool(xis, m, dI, wgi, gbi, c, NULL);
-    for (e = 0; e < dI; ++e) key[e] = (uint16_t)csla_orc_bf16_from_f32((float)c[e]);
+    csla_orc_key_bf16(c, dI, key);
     free(c);
+}
+
+/* Storage of a pooled index key c (dI values): bf16 rounded from fp32. */
+void csla_orc_key_bf16(const double *c, int dI, uint16_t *key)
+{
+    int e;
+    for (e = 0; e < dI; ++e) key[e] = (uint16_t)csla_orc_bf16_from_f32((float)c[e]);
 }
 
 /* E4M3 storage of an index key ([haiqwa] §FP4精度加速: the indexer's key /
@@ -254,13 +288,10 @@ double csla_orc_key_scale_e4m3(double amax)
     return ldexp(1.0, e);
 }
 
-void csla_orc_index_key_e4m3(const double *xis, int m, const double *wgi, const double *gbi, int dI,
-                             uint8_t *codes, float *scale_out)
+void csla_orc_key_e4m3(const double *c, int dI, uint8_t *codes, float *scale_out)
 {
     int e;
     double amax = 0.0, s;
-    double *c = (double *)malloc(sizeof(double) * (size_t)dI);
-    csla_orc_gate_pool(xis, m, dI, wgi, gbi, c, NULL);
     for (e = 0; e < dI; ++e) {
         double v = fabs((double)(float)c[e]);
         if (v > amax) amax = v;
@@ -268,6 +299,14 @@ void csla_orc_index_key_e4m3(const double *xis, int m, const double *wgi, const 
     s = csla_orc_key_scale_e4m3(amax);
     for (e = 0; e < dI; ++e) codes[e] = (uint8_t)csla_orc_e4m3_from_f32((float)((double)(float)c[e] / s));
     *scale_out = (float)s;
+}
+
+void csla_orc_index_key_e4m3(const double *xis, int m, const double *wgi, const double *gbi, int dI,
+                             uint8_t *codes, float *scale_out)
+{
+    double *c = (double *)malloc(sizeof(double) * (size_t)dI);
+    csla_orc_gate_pool(xis, m, dI, wgi, gbi, c, NULL);
+    csla_orc_key_e4m3(c, dI, codes, scale_out);
     free(c);
 }
 

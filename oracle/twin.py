@@ -65,6 +65,15 @@ def pool(xs, wg, gb):
     return a @ xs
 
 
+def pool_channel(xs, w, b):
+    """Per-channel gates: a separate softmax over the block's tokens for every channel."""
+    xs = np.asarray(xs, np.float64)
+    g = xs * np.asarray(w, np.float64)[None, :] + np.broadcast_to(np.asarray(b, np.float64), xs.shape)
+    a = np.exp(g - g.max(axis=0, keepdims=True))
+    a /= a.sum(axis=0, keepdims=True)
+    return (a * xs).sum(axis=0)
+
+
 def window_row(x, gamma, pos, eps=1e-6, theta=10000.0, d_rope=64):
     return quantize(rotate(rms(x, gamma, eps), pos, theta, d_rope), d_rope)
 
