@@ -56,6 +56,21 @@ bool encode_bf16_2d(CUtensorMap *map, const void *ptr, uint64_t cols, uint64_t r
     return r == CUDA_SUCCESS;
 }
 
+// 2-D byte tensor [rows][cols] (cols contiguous, cols <= 128), box = cols x
+// box_rows, 128B swizzle: the E4M3 index keys.
+bool encode_u8_2d(CUtensorMap *map, const void *ptr, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {(cuuint32_t)cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = f(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_cfg(const csla_cfg *c) {
@@ -65,6 +80,7 @@ int check_cfg(const csla_cfg *c) {
     if (c->H < 1 || c->H > 64) return CSLA_ERR_UNSUPPORTED;
     if (!(c->eps >= 0.f) || !(c->rope_theta > 0.f)) return CSLA_ERR_ARG;
     if (c->key_fmt != CSLA_KEY_BF16 && c->key_fmt != CSLA_KEY_E4M3) return CSLA_ERR_UNSUPPORTED;
+    if (c->key_fmt == CSLA_KEY_E4M3 && c->m == 4 && c->dI != 128) return CSLA_ERR_UNSUPPORTED;
     return CSLA_OK;
 }
 
@@ -278,14 +294,20 @@ static int prep_indexer(const csla_cfg *cfg, const csla_state *st, const csla_ca
     if (workspace_bytes < csla_workspace_size(cfg, CSLA_OP_INDEXER, B, max_len)) return CSLA_ERR_ARG;
     if (!aligned16(cq) || !aligned16(W_iq) || !aligned16(cache->kidx) || !aligned16(workspace)) return CSLA_ERR_ARG;
     const bool e4m3 = cfg->key_fmt == CSLA_KEY_E4M3;
-    if (e4m3 && (!cache->kscale || !aligned16(cache->kscale))) return CSLA_ERR_ARG;
+    if (e4m3 && !cache->kscale) return CSLA_ERR_ARG;
     const int NQ = nq_of(cfg->HI);
     CUtensorMap kmap, qmap;
-    memset(&kmap, 0, sizeof(kmap));   // E4M3 keys arrive by 1-D bulk copies: no key tensor map
-    if (!e4m3 && !encode_bf16_2d(&kmap, cache->kidx, (uint64_t)cfg->dI, (uint64_t)cache->n_pages * 32, 32))
+    memset(&qmap, 0, sizeof(qmap));
+    if (e4m3) {
+        // E4M3 keys: one 128-byte box per entry row; the kernel builds its
+        // four-term E4M3 query operand from the projection's bf16 terms
+        if (!encode_u8_2d(&kmap, cache->kidx, (uint64_t)cfg->dI, (uint64_t)cache->n_pages * 32, 32))
+            return CSLA_ERR_CUDA;
+    } else if (!encode_bf16_2d(&kmap, cache->kidx, (uint64_t)cfg->dI, (uint64_t)cache->n_pages * 32, 32)) {
         return CSLA_ERR_CUDA;
-    const int G = (qs && qs->one_request) ? indexer_rows_per_cta(NQ) : 1;
-    if (!encode_bf16_2d(&qmap, workspace, (uint64_t)cfg->dI, (uint64_t)B * NQ, (uint32_t)(G * NQ)))
+    }
+    const int G = (qs && qs->one_request) ? indexer_rows_per_cta(e4m3 ? 4 * cfg->HI : NQ) : 1;
+    if (!e4m3 && !encode_bf16_2d(&qmap, workspace, (uint64_t)cfg->dI, (uint64_t)B * NQ, (uint32_t)(G * NQ)))
         return CSLA_ERR_CUDA;
     L->kmap = kmap;
     L->qmap = qmap;

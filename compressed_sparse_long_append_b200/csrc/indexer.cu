@@ -204,26 +204,24 @@ constexpr int kTPC = 8;              // tiles per CTA (consecutive, one request)
 // warp 0: TMA, warp 1: MMA, then 4 epilogue warps per set of query rows
 // (set s takes the group's rows s, s + sets, ...): one set for G = 1, one
 // per row up to 7 rows (balanced: 5 at 16 index heads), else four.
-// E4M3 keys add four converter warps after the epilogue warps.
 template <int G>
 constexpr int idx_epi_sets() { return G == 1 ? 1 : (G <= 7 ? G : 4); }
-constexpr int kConvWarps = 4;
-template <int G, bool kE4M3>
-constexpr int idx_threads() { return 64 + 128 * idx_epi_sets<G>() + (kE4M3 ? 32 * kConvWarps : 0); }
+template <int G>
+constexpr int idx_threads() { return 64 + 128 * idx_epi_sets<G>(); }
+// Query operand rows per query row: bf16 keys take three bf16 terms of every
+// head (NQ = 3*HI rounded up to 16); E4M3 keys take four E4M3 terms (4*HI).
+template <int HI>
+constexpr int nq_e4m3() { return 4 * HI; }
 
-// bf16 key tiles (what the MMA reads): a 3-stage ring filled by TMA, or with
-// E4M3 keys a 2-stage ring filled by the converter warps from a 3-stage ring
-// of bulk-copied codes and scales.
+// Key tiles arrive by TMA into a 3-stage ring: bf16 (2-D map, 64-dim boxes)
+// or E4M3 codes (2-D map over bytes, one 128-byte box per entry row).
 template <int DI, int NQ, int G, bool kE4M3>
 struct IdxSmem {
-    static constexpr int kStages = kE4M3 ? 2 : 3;
-    static constexpr int kStages8 = 3;
-    static constexpr int kKeyBytes = kTileE * DI * 2;
-    static constexpr int kCodeBytes = kTileE * DI;          // E4M3 codes of a tile
-    static constexpr int kCode8Bytes = kCodeBytes + 1024;   // + the entries' scales (512 B, padded: 1024-aligned stages)
-    static constexpr int kQBytes = G * NQ * DI * 2;
-    static constexpr int kBytes = kStages * kKeyBytes + (kE4M3 ? kStages8 * kCode8Bytes : 0) + kQBytes +
-                                  1024 /*align*/ + 1024 /*barriers, pages, weights*/;
+    static constexpr int kStages = 3;
+    static constexpr int kElt = kE4M3 ? 1 : 2;
+    static constexpr int kKeyBytes = kTileE * DI * kElt;
+    static constexpr int kQBytes = G * NQ * DI * kElt;
+    static constexpr int kBytes = kStages * kKeyBytes + kQBytes + 1024 /*align*/ + 2048 /*barriers, pages, weights, term scales*/;
 };
 
 // Two accumulators of G*NQ columns, rounded up to a power of two >= 32.
@@ -232,33 +230,69 @@ constexpr uint32_t kTmemCols() {
     return 2 * N <= 32 ? 32 : (2 * N <= 64 ? 64 : (2 * N <= 128 ? 128 : (2 * N <= 256 ? 256 : 512)));
 }
 
+// E4M3 query operand of one (row, head): q (the fp32 sum of the projection's
+// three bf16 terms, 4 dims per lane) split into four E4M3 terms with
+// power-of-two scales, q ~ sum_t 2^(e_t) code_t: e_t as for index keys (the
+// smallest 2^e with 448 * 2^e >= max |residual|), codes rounded to nearest
+// even, each residual formed exactly.  After four terms the residual is
+// below ~2^-19 of max |q|.  Warp-collective; lane l writes dims 4l..4l+3 of
+// operand rows n_t = base + t*HI (SW128 K-major, 128 bytes per row) and lane
+// 0 the scales sig[t*HI].
+__device__ __forceinline__ void split_q_e4m3(float (&q)[4], uint8_t *qb, int base, int HI, float *sig) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        float am = fmaxf(fmaxf(fabsf(q[0]), fabsf(q[1])), fmaxf(fabsf(q[2]), fabsf(q[3])));
+        am = warp_max(am);
+        const int ex = key_exp_e4m3(am);
+        const float inv = __uint_as_float((uint32_t)(127 - min(ex, 126)) << 23);
+        const float sc = __uint_as_float((uint32_t)(ex + 127) << 23);
+        uint32_t word = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint8_t c = f32_to_e4m3(__fmul_rn(q[i], inv));
+            const __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E4M3);
+            const float cv = __half2float(__half(h));
+            q[i] = __fsub_rn(q[i], __fmul_rn(cv, sc));   // exact: the rounding residual
+            word |= (uint32_t)c << (8 * i);
+        }
+        const int n = base + t * HI;
+        *reinterpret_cast<uint32_t *>(qb + (n >> 3) * 1024 + (n & 7) * 128 + ((((lane >> 2) ^ (n & 7))) << 4) +
+                                      4 * (lane & 3)) = word;
+        if (lane == 0) sig[t * HI] = sc;
+    }
+}
+
 // CTA (blockIdx.x, blockIdx.y) scores tiles [blockIdx.x*kTPC, +kTPC) (128
 // entries each) of the query rows r0 = blockIdx.y*G .. r0+G-1, which all
 // read the keys of request slots[r0]: one key tile feeds one MMA of N = G*NQ
 // query columns (decode: G = 1; query rows of one request: G > 1).
+// kE4M3: keys are E4M3 codes with a power-of-two scale per entry, scored by
+// kind::f8f6f4 MMAs against the four-term E4M3 query operand that the
+// epilogue warps build before they start (NQ = 4*HI); the epilogue forms
+// each head's dot product from its four terms and applies the entry scale.
 template <int DI, int NQ, int HI, int G, bool kE4M3>
-__global__ void __launch_bounds__(idx_threads<G, kE4M3>())
+__global__ void __launch_bounds__(idx_threads<G>())
     indexer_kernel(IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap qmap) {
     CSLA_TL_SCOPE(kTlIndexer);
     using S = IdxSmem<DI, NQ, G, kE4M3>;
     constexpr int kStages = S::kStages;
     constexpr int N = G * NQ;
-    constexpr int kConvWarp0 = 2 + 4 * idx_epi_sets<G>();   // first converter warp (E4M3 keys)
     static_assert(N % 16 == 0 && N <= 256, "UMMA N for M = 128");
+    static_assert(!kE4M3 || (DI == 128 && NQ == 4 * HI), "E4M3 keys: dI = 128, four query terms");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t *codes = base + kStages * S::kKeyBytes;                       // E4M3: [kStages8][codes | scales]
-    uint8_t *qbuf = codes + (kE4M3 ? S::kStages8 * S::kCode8Bytes : 0);
+    uint8_t *qbuf = base + kStages * S::kKeyBytes;
     uint64_t *bars = reinterpret_cast<uint64_t *>(qbuf + S::kQBytes);
     uint64_t *full = bars, *empty = bars + kStages, *tfull = bars + 2 * kStages, *tempty = tfull + 2;
     uint64_t *qfull = tempty + 2;
-    uint64_t *full8 = qfull + 1, *empty8 = full8 + S::kStages8;            // E4M3 only
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(empty8 + S::kStages8);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(qfull + 1);
     int *pages = reinterpret_cast<int *>(tmem_holder + 1);      // [kTPC * 4]
     int *row_nv = pages + kTPC * 4;                              // [G] entries scored below this (-1: skip)
     int *row_lo = row_nv + G;                                    // [G] first entry scored
     float *hw = reinterpret_cast<float *>(row_lo + G);           // [G][HI] head weights
+    float *sig = hw + G * HI;                                    // [G][NQ] E4M3 query-term scales
     __shared__ volatile int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -271,18 +305,15 @@ __global__ void __launch_bounds__(idx_threads<G, kE4M3>())
     if (threadIdx.x == 0) {
         abort_flag = 0;
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(full + s, kE4M3 ? kConvWarps : 1);   // TMA, or one arrival per converter warp
+            mbar_init(full + s, 1);
             mbar_init(empty + s, 1);
-        }
-        for (int s = 0; s < S::kStages8; ++s) {
-            mbar_init(full8 + s, 1);
-            mbar_init(empty8 + s, kConvWarps);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(tfull + i, 1);
             mbar_init(tempty + i, 4 * idx_epi_sets<G>());   // one arrival per epilogue warp
         }
-        mbar_init(qfull, 1);
+        // the query operand: one TMA (bf16), or one arrival per epilogue warp (E4M3)
+        mbar_init(qfull, kE4M3 ? 4 * idx_epi_sets<G>() : 1);
         fence_mbar_init();
     }
     int pg = -1;   // warp 0: page id of this CTA's page `lane`
@@ -291,15 +322,15 @@ __global__ void __launch_bounds__(idx_threads<G, kE4M3>())
         if (a.range != 2 && slot_ok && lane < kTPC * 4 && col < a.bt_stride)
             pg = __ldg(a.block_table + (size_t)slot * a.bt_stride + col);
         if (lane == 0) {
-            if (!kE4M3) tma_prefetch_desc(&kmap);
-            tma_prefetch_desc(&qmap);
+            tma_prefetch_desc(&kmap);
+            if (!kE4M3) tma_prefetch_desc(&qmap);
         }
     }
     if (warp == 1) {
         tmem_alloc(tmem_holder, kTmemCols<N>());
         tmem_relinquish();
     }
-    for (int i = threadIdx.x; i < G * HI; i += idx_threads<G, kE4M3>()) {
+    for (int i = threadIdx.x; i < G * HI; i += idx_threads<G>()) {
         const int r = r0 + i / HI;
         hw[i] = r < a.B ? __ldg(a.head_w + (size_t)r * HI + i % HI) : 0.f;
     }
@@ -313,6 +344,7 @@ __global__ void __launch_bounds__(idx_threads<G, kE4M3>())
     pdl_trigger();
     pdl_wait();
     CSLA_TL_WAITED();
+
 
     // ---- entries of each row scored here; the CTA streams the tiles of the longest.
     // range 0: [0, visible); 1: [0, len0/m) (entries complete before an append
@@ -366,61 +398,44 @@ __global__ void __launch_bounds__(idx_threads<G, kE4M3>())
         // nothing to score: fall through to the teardown
     } else if (warp == 0) {
         if (lane == 0) {
-            mbar_arrive_expect_tx(qfull, (uint32_t)S::kQBytes);
+            if (!kE4M3) {
+                mbar_arrive_expect_tx(qfull, (uint32_t)S::kQBytes);
 #pragma unroll
-            for (int h = 0; h < DI / 64; ++h) tma_load_2d(qbuf + h * N * 128, &qmap, h * 64, r0 * NQ, qfull);
+                for (int h = 0; h < DI / 64; ++h) tma_load_2d(qbuf + h * N * 128, &qmap, h * 64, r0 * NQ, qfull);
+            }
             int n = 0;
-            if constexpr (kE4M3) {
-                // codes (32 entries x DI bytes) and scales (32 floats) of each
-                // page: two 1-D bulk copies per page into the code ring
-                constexpr int kS8 = S::kStages8;
-                for (int t = 0; t < n_tiles; ++t, ++n) {
-                    const int s = n % kS8;
-                    if (n >= kS8 && !mbar_wait(empty8 + s, ((n / kS8) - 1) & 1, &abort_flag)) break;
-                    uint8_t *cb = codes + s * S::kCode8Bytes;
-                    int np = 0;
+            for (int t = 0; t < n_tiles; ++t, ++n) {
+                const int s = n % kStages;
+                if (n >= kStages && !mbar_wait(empty + s, ((n / kStages) - 1) & 1, &abort_flag)) break;
+                uint8_t *kb = base + s * S::kKeyBytes;
+                int np = 0;
 #pragma unroll
-                    for (int p = 0; p < 4; ++p) np += pages[t * 4 + p] >= 0;
-                    mbar_arrive_expect_tx(full8 + s, (uint32_t)(np * kPageE * (DI + 4)));
+                for (int p = 0; p < 4; ++p) np += pages[t * 4 + p] >= 0;
+                mbar_arrive_expect_tx(full + s, (uint32_t)(np * kPageE * DI * S::kElt));
 #pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        const int pg = pages[t * 4 + p];
-                        if (pg < 0) continue;
-                        bulk_load(cb + p * kPageE * DI, a.kidx8 + (size_t)pg * kPageE * DI, kPageE * DI, full8 + s);
-                        bulk_load(cb + S::kCodeBytes + p * kPageE * 4, a.kscale + (size_t)pg * kPageE, kPageE * 4,
-                                  full8 + s);
-                    }
-                }
-                for (int i = (n > kS8 ? n - kS8 : 0); i < n; ++i) mbar_wait(full8 + (i % kS8), (i / kS8) & 1, nullptr);
-            } else {
-                for (int t = 0; t < n_tiles; ++t, ++n) {
-                    const int s = n % kStages;
-                    if (n >= kStages && !mbar_wait(empty + s, ((n / kStages) - 1) & 1, &abort_flag)) break;
-                    uint8_t *kb = base + s * S::kKeyBytes;
-                    int np = 0;
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) np += pages[t * 4 + p] >= 0;
-                    mbar_arrive_expect_tx(full + s, (uint32_t)(np * kPageE * DI * 2));
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        const int pg = pages[t * 4 + p];
-                        if (pg < 0) continue;
+                for (int p = 0; p < 4; ++p) {
+                    const int pg = pages[t * 4 + p];
+                    if (pg < 0) continue;
+                    if constexpr (kE4M3) {
+                        // one 128-byte box per entry row (the whole E4M3 key)
+                        tma_load_2d(kb + p * (kPageE * 128), &kmap, 0, pg * kPageE, full + s);
+                    } else {
 #pragma unroll
                         for (int h = 0; h < DI / 64; ++h)
                             tma_load_2d(kb + h * (kTileE * 128) + p * (kPageE * 128), &kmap, h * 64, pg * kPageE,
                                         full + s);
                     }
                 }
-                // every issued copy must land before the CTA may exit
-                for (int i = (n > kStages ? n - kStages : 0); i < n; ++i)
-                    mbar_wait(full + (i % kStages), (i / kStages) & 1, nullptr);
             }
+            // every issued copy must land before the CTA may exit
+            for (int i = (n > kStages ? n - kStages : 0); i < n; ++i)
+                mbar_wait(full + (i % kStages), (i / kStages) & 1, nullptr);
             mbar_wait(qfull, 0, nullptr);
             CSLA_TL_MARK_ANY(4);
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(128, N, false, false);
+            constexpr uint32_t idesc = kE4M3 ? idesc_e4m3(128, N) : idesc_bf16(128, N, false, false);
             int n = 0;
             if (mbar_wait(qfull, 0, &abort_flag)) {
                 const uint32_t qb = smem_u32(qbuf);
@@ -433,67 +448,26 @@ __global__ void __launch_bounds__(idx_threads<G, kE4M3>())
                     if (n >= 2 && !mbar_wait(tempty + acc, ((n / 2) - 1) & 1, &abort_flag)) break;
                     tc_fence_after();
                     const uint32_t kb = smem_u32(base + s * S::kKeyBytes);
+                    if constexpr (kE4M3) {
+                        // K = 32 codes (32 bytes) per instruction
 #pragma unroll
-                    for (int k = 0; k < DI / 16; ++k) {
-                        const uint32_t half = k / 4, ko = (k % 4) * 32;
-                        const uint64_t ad = sdesc(kb + half * (kTileE * 128) + ko, 16, 1024);
-                        const uint64_t bd = sdesc(qb + half * (N * 128) + ko, 16, 1024);
-                        umma_kind_f16(tmem + acc * N, ad, bd, idesc, k > 0 ? 1u : 0u);
+                        for (int k = 0; k < DI / 32; ++k)
+                            umma_kind_f8f6f4(tmem + acc * N, sdesc(kb + k * 32, 16, 1024), sdesc(qb + k * 32, 16, 1024),
+                                             idesc, k > 0 ? 1u : 0u);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < DI / 16; ++k) {
+                            const uint32_t half = k / 4, ko = (k % 4) * 32;
+                            const uint64_t ad = sdesc(kb + half * (kTileE * 128) + ko, 16, 1024);
+                            const uint64_t bd = sdesc(qb + half * (N * 128) + ko, 16, 1024);
+                            umma_kind_f16(tmem + acc * N, ad, bd, idesc, k > 0 ? 1u : 0u);
+                        }
                     }
                     umma_commit(empty + s);
                     umma_commit(tfull + acc);
                 }
             }
             if (n > 0) mbar_wait(tfull + ((n - 1) & 1), ((n - 1) / 2) & 1, nullptr);
-        }
-    } else if (kE4M3 && warp >= kConvWarp0) {
-        // converter warps: E4M3 codes * scale -> bf16, exactly (every E4M3
-        // value times a power of two in the normal range is a bf16 value),
-        // into the SW128 K-major key layout the TMA would have produced:
-        // entry r, 8-dim group g at half g/8, row r, 16-byte slot (g%8)^(r%8).
-        // Thread i converts 16-byte code chunks i, i+128, ... (consecutive
-        // threads read consecutive chunks).
-        constexpr int kS8 = S::kStages8;
-        constexpr int kCPR = DI / 16;   // code chunks per entry
-        const int ci = threadIdx.x - 32 * kConvWarp0;
-        int n = 0;
-        for (int t = 0; t < n_tiles; ++t, ++n) {
-            const int s8 = n % kS8, s = n % kStages;
-            if (!warp_all(mbar_wait(full8 + s8, (n / kS8) & 1, &abort_flag))) break;
-            if (n >= kStages && !warp_all(mbar_wait(empty + s, ((n / kStages) - 1) & 1, &abort_flag))) break;
-            const uint8_t *cb = codes + s8 * S::kCode8Bytes;
-            const float *sc = reinterpret_cast<const float *>(cb + S::kCodeBytes);
-            uint8_t *kb = base + s * S::kKeyBytes;
-#pragma unroll
-            for (int k = 0; k < kCPR; ++k) {
-                const int f = ci + 128 * k;
-                const int r = f / kCPR, c = f % kCPR;
-                const uint4 v = *reinterpret_cast<const uint4 *>(cb + r * DI + 16 * c);
-                const float scl = sc[r];
-                const __nv_bfloat162 sv = __floats2bfloat162_rn(scl, scl);   // a power of two: exact
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                uint32_t o[8];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const uint32_t lo = e4m3x2_to_bf16x2(w[e] & 0xFFFFu), hi = e4m3x2_to_bf16x2(w[e] >> 16);
-                    __nv_bfloat162 bl = *reinterpret_cast<const __nv_bfloat162 *>(&lo);
-                    __nv_bfloat162 bh = *reinterpret_cast<const __nv_bfloat162 *>(&hi);
-                    bl = __hmul2(bl, sv);
-                    bh = __hmul2(bh, sv);
-                    o[2 * e] = *reinterpret_cast<const uint32_t *>(&bl);
-                    o[2 * e + 1] = *reinterpret_cast<const uint32_t *>(&bh);
-                }
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int g = 2 * c + q;                 // dims 8g .. 8g+7
-                    const int h = g >> 3, j = g & 7;
-                    *reinterpret_cast<uint4 *>(kb + h * (kTileE * 128) + r * 128 + ((j ^ (r & 7)) << 4)) =
-                        make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-                }
-            }
-            fence_proxy_async_smem();
-            mbar_arrive_warp(full + s);
-            mbar_arrive_warp(empty8 + s8);
         }
     } else {
         // TMEM lanes 32*(warp%4).. are this warp's key rows; set `es` takes
@@ -502,8 +476,39 @@ __global__ void __launch_bounds__(idx_threads<G, kE4M3>())
         const int lane_base = 32 * (warp & 3);
         const int es = (warp - 2) / 4;
         const int row = lane_base + lane;
+        if constexpr (kE4M3) {
+            // the E4M3 query operand: (query row g, head j) per warp task,
+            // from the projection's three bf16 terms (their fp32 sum is q)
+            for (int task = warp - 2; task < G * HI; task += 4 * kSets) {
+                const int g = task / HI, j = task % HI, r = r0 + g;
+                float q[4] = {0.f, 0.f, 0.f, 0.f};
+                if (r < a.B) {
+                    const uint16_t *qw = a.q_ws + (size_t)r * a.NQ * DI + 4 * lane;
+                    const uint2 h = *reinterpret_cast<const uint2 *>(qw + (size_t)j * DI);
+                    const uint2 m = *reinterpret_cast<const uint2 *>(qw + (size_t)(HI + j) * DI);
+                    const uint2 l = *reinterpret_cast<const uint2 *>(qw + (size_t)(2 * HI + j) * DI);
+                    const uint32_t hv[4] = {h.x & 0xFFFFu, h.x >> 16, h.y & 0xFFFFu, h.y >> 16};
+                    const uint32_t mv[4] = {m.x & 0xFFFFu, m.x >> 16, m.y & 0xFFFFu, m.y >> 16};
+                    const uint32_t lv[4] = {l.x & 0xFFFFu, l.x >> 16, l.y & 0xFFFFu, l.y >> 16};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        q[i] = __fadd_rn(__fadd_rn(bf16_bits_to_f32(hv[i]), bf16_bits_to_f32(mv[i])),
+                                         bf16_bits_to_f32(lv[i]));
+                }
+                split_q_e4m3(q, qbuf, g * NQ + j, HI, sig + g * NQ + j);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive_warp(qfull);
+            // the term scales are read by every epilogue warp
+            asm volatile("bar.sync 1, %0;" ::"r"(128 * kSets) : "memory");
+        }
         for (int t = 0, n = 0; t < n_tiles; ++t, ++n) {
             const int acc = n & 1;
+            float ksc = 0.f;   // E4M3: this row's entry scale, loaded before the accumulator wait
+            if constexpr (kE4M3) {
+                const int pgr = pages[t * 4 + row / kPageE];
+                if (pgr >= 0) ksc = __ldg(a.kscale + (size_t)pgr * kPageE + row % kPageE);
+            }
             if (!warp_all(mbar_wait(tfull + acc, (n / 2) & 1, &abort_flag))) break;
             tc_fence_after();
             const int e = (t_begin + t) * kTileE + row;
@@ -524,6 +529,11 @@ __global__ void __launch_bounds__(idx_threads<G, kE4M3>())
                     tmem_ld32x16(ta, r);
                 } else if constexpr (NQ == 32) {
                     tmem_ld32x32(ta, r);
+                } else if constexpr (NQ == 64) {
+                    uint32_t (&r0_)[32] = *reinterpret_cast<uint32_t (*)[32]>(r);
+                    uint32_t (&r1_)[32] = *reinterpret_cast<uint32_t (*)[32]>(r + 32);
+                    tmem_ld32x32(ta, r0_);
+                    tmem_ld32x32(ta + 32, r1_);
                 } else {
                     static_assert(NQ == 48, "query operand rows");
                     uint32_t (&r0_)[32] = *reinterpret_cast<uint32_t (*)[32]>(r);
@@ -540,11 +550,26 @@ __global__ void __launch_bounds__(idx_threads<G, kE4M3>())
                 // entries of a page outside the pool were not loaded: leave them unscored
                 if (e < nv && e >= row_lo[g] && pages[t * 4 + row / kPageE] >= 0) {
                     float sc = 0.f;
+                    if constexpr (kE4M3) {
+                        // head j: sum_t sig_t * acc_t (terms in order), then
+                        // the entry's power-of-two key scale (ReLU commutes with it)
+                        const float *sg = sig + g * NQ;
 #pragma unroll
-                    for (int j = 0; j < HI; ++j) {
-                        const float dot = __fadd_rn(__fadd_rn(__uint_as_float(r[j]), __uint_as_float(r[HI + j])),
-                                                    __uint_as_float(r[2 * HI + j]));
-                        sc = __fmaf_rn(hw[g * HI + j], fmaxf(dot, 0.f), sc);
+                        for (int j = 0; j < HI; ++j) {
+                            float dot = __fmul_rn(sg[j], __uint_as_float(r[j]));
+#pragma unroll
+                            for (int tt = 1; tt < 4; ++tt)
+                                dot = __fmaf_rn(sg[tt * HI + j], __uint_as_float(r[tt * HI + j]), dot);
+                            sc = __fmaf_rn(hw[g * HI + j], fmaxf(dot, 0.f), sc);
+                        }
+                        sc = __fmul_rn(sc, ksc);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < HI; ++j) {
+                            const float dot = __fadd_rn(__fadd_rn(__uint_as_float(r[j]), __uint_as_float(r[HI + j])),
+                                                        __uint_as_float(r[2 * HI + j]));
+                            sc = __fmaf_rn(hw[g * HI + j], fmaxf(dot, 0.f), sc);
+                        }
                     }
                     a.scores[(size_t)(r0 + g) * a.scores_stride + e] = sc;
                 }
@@ -560,6 +585,7 @@ __global__ void __launch_bounds__(idx_threads<G, kE4M3>())
         tmem_dealloc(tmem, kTmemCols<N>());
     }
 }
+
 
 template <int DI, int NQ, int HI, int G, bool kE4M3>
 cudaError_t launch_indexer_t(const IndexerArgs &a, const CUtensorMap &kmap, const CUtensorMap &qmap,
@@ -577,7 +603,7 @@ cudaError_t launch_indexer_t(const IndexerArgs &a, const CUtensorMap &kmap, cons
     }
     const int groups = (a.tiles_per_req + kTPC - 1) / kTPC;
     return launch_pdl(indexer_kernel<DI, NQ, HI, G, kE4M3>, dim3(groups, (a.B + G - 1) / G),
-                      dim3(idx_threads<G, kE4M3>()), S::kBytes, stream, a, kmap, qmap);
+                      dim3(idx_threads<G>()), S::kBytes, stream, a, kmap, qmap);
 }
 
 template <int DI, int NQ, int HI, bool kE4M3>
@@ -589,10 +615,15 @@ cudaError_t launch_indexer_g(const IndexerArgs &a, const CUtensorMap &kmap, cons
     return cudaErrorInvalidValue;
 }
 
+// NQ: rows of the bf16 query operand; E4M3 keys (dI = 128 only) score
+// against four E4M3 terms per head instead.
 template <int DI, int NQ, int HI>
 cudaError_t launch_indexer_k(const IndexerArgs &a, const CUtensorMap &kmap, const CUtensorMap &qmap,
                              cudaStream_t stream) {
-    if (a.key_fmt == CSLA_KEY_E4M3) return launch_indexer_g<DI, NQ, HI, true>(a, kmap, qmap, stream);
+    if (a.key_fmt == CSLA_KEY_E4M3) {
+        if constexpr (DI == 128) return launch_indexer_g<DI, nq_e4m3<HI>(), HI, true>(a, kmap, qmap, stream);
+        return cudaErrorInvalidValue;
+    }
     return launch_indexer_g<DI, NQ, HI, false>(a, kmap, qmap, stream);
 }
 

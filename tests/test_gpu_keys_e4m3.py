@@ -50,7 +50,8 @@ def compare_key_e4m3(codes, scale, key32):
 
 
 KEYS = dataclasses.replace(CSA_DECODE, L=900, key_fmt=1, name="keys_e4m3")
-KEYS_TINY = dataclasses.replace(CSA_TINY, L=700, key_fmt=1, name="keys_e4m3_tiny")
+# E4M3 keys are scored by kind::f8f6f4 MMAs at dI = 128 (the tiny shape with 128-dim keys)
+KEYS_TINY = dataclasses.replace(CSA_TINY, L=700, dI=128, key_fmt=1, name="keys_e4m3_tiny")
 
 
 @pytest.mark.parametrize("w,lens,chunk", [(KEYS, [900, 133], 64), (KEYS_TINY, [700, 9], None), (KEYS, [90], 1)])
@@ -88,7 +89,8 @@ def _scores(w, lb, si, p, slots, max_len, qs=None):
 
 
 @pytest.mark.parametrize("w,lens", [
-    (dataclasses.replace(CSA_TINY, B=3, L=2048, key_fmt=1, name="idx8_tiny"), [2048, 515, 3]),
+    (dataclasses.replace(CSA_TINY, B=3, L=2048, dI=128, key_fmt=1, name="idx8_tiny"), [2048, 515, 3]),
+    (dataclasses.replace(CSA_TINY, B=2, L=2048, dI=128, HI=8, key_fmt=1, name="idx8_hi8"), [2048, 700]),
     (dataclasses.replace(CSA_DECODE, B=2, L=5000, key_fmt=1, name="idx8_big"), [5000, 1113]),
 ])
 def test_indexer_on_e4m3_keys_matches_oracle(w, lens):
@@ -106,10 +108,11 @@ def test_indexer_on_e4m3_keys_matches_oracle(w, lens):
         assert np.all(np.isnan(got[s, nv:]))
 
 
-def test_indexer_query_rows_of_one_request_on_e4m3_keys():
+@pytest.mark.parametrize("HI", [16, 4])
+def test_indexer_query_rows_of_one_request_on_e4m3_keys(HI):
     """Query rows of one request with their own visible lengths: several rows
-    share each key tile (the prefill path)."""
-    w = dataclasses.replace(CSA_DECODE, B=7, L=3000, key_fmt=1, name="idx8_rows")
+    share each key tile (the prefill path: 4 rows at 16 index heads, 16 at 4)."""
+    w = dataclasses.replace(CSA_DECODE, B=7, L=3000, HI=HI, key_fmt=1, name="idx8_rows%d" % HI)
     L = 3000
     cv, p = oracle_cache(w, [L])
     lb = upload_layer(w, cv, [L])
