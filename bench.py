@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--no-e4m3", action="store_true", help="skip the CSA decode leg with E4M3 index keys")
     ap.add_argument("--no-invariance", action="store_true",
                     help="skip the ragged 64-request CSA + HCA decode measurement")
+    ap.add_argument("--no-stack", action="store_true",
+                    help="skip the interleaved CSA/HCA layer stack on one shared block table")
+    ap.add_argument("--stack-layers", type=int, default=8, help="layers of the interleaved stack")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", type=int, default=0, help="attention variant: 0 auto, 1 saturated, 2 starved")
     ap.add_argument("--fused-step", action="store_true",
@@ -135,9 +138,11 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ workload build
-def build_layer(shape_kw, n_req, L0s, seed, rank, device):
+def build_layer(shape_kw, n_req, L0s, seed, rank, device, block_table=None):
     """Caches of n_req requests after appending L0s[r] tokens to request r,
-    through csla_compress_append on raw streams generated on the device."""
+    through csla_compress_append on raw streams generated on the device.
+    block_table: a filled table shared with other layers (else the layer's
+    own, a seeded page permutation)."""
     import torch
     from compressed_sparse_long_append_b200 import csla as C
     from compressed_sparse_long_append_b200.layer import CompressParams, LayerBuffers, LayerShape
@@ -150,9 +155,10 @@ def build_layer(shape_kw, n_req, L0s, seed, rank, device):
     L_cap = shape_kw["L"] + HEADROOM
     pages_per = -(-L_cap // 128)
     n_pages = n_req * pages_per
-    lb = LayerBuffers(sh, n_req, n_pages, pages_per, device)
-    perm = permutation(seed, "pages/%d" % rank, n_pages).astype("int32").reshape(n_req, pages_per)
-    lb.block_table.copy_(torch.from_numpy(perm))
+    lb = LayerBuffers(sh, n_req, n_pages, pages_per, device, block_table=block_table)
+    if block_table is None:
+        perm = permutation(seed, "pages/%d" % rank, n_pages).astype("int32").reshape(n_req, pages_per)
+        lb.block_table.copy_(torch.from_numpy(perm))
     D, dI, m = sh.D, sh.dI, sh.m
     g = lambda name, shp, std=1.0: torch.as_tensor(normal(seed, name, shp, std=std), dtype=torch.float32)
     cp = CompressParams(1.0 + 0.1 * g("gamma_kv", (D,)), g("wg", (D,), 1.0 / D ** 0.5), g("gb", (m,)),
@@ -267,11 +273,16 @@ def csa_launches(kw, variant, fused):
     indexer, topk, attend, + combine unless the saturated variant runs
     (forced, or automatic: one chunk per request or B >= SM count); the
     fused step adds the length snapshot and the second indexer launch."""
-    rows = kw["k"] + kw["n_win"]
+    return 2 + 2 + 1 + attend_launches(kw["k"] + kw["n_win"], kw["B"], variant) + (2 if fused else 0)
+
+
+def attend_launches(rows, B, variant):
+    """Attention kernels of one call over `rows` rows per request: the
+    attention, plus the combine unless the saturated variant runs."""
     chunk = 64 * max(-(-rows // 2048), 2 if rows > 1024 else 1)
     chunks = -(-rows // chunk)
-    saturated = variant == 1 or (variant == 0 and (kw["B"] >= 148 or chunks <= 1))
-    return 2 + 2 + 1 + 1 + (0 if saturated else 1) + (2 if fused else 0)
+    saturated = variant == 1 or (variant == 0 and (B >= 148 or chunks <= 1))
+    return 1 + (0 if saturated else 1)
 
 
 class HcaStep:
@@ -533,13 +544,77 @@ def invariance_leg(W, K, seed, rank, world, device, variant):
     return out
 
 
-def clone_layer(lb, params):
+def stack_leg(W, K, seed, rank, world, device, variant, n_layers):
+    """A model-shaped stack: n_layers attention layers, CSA and HCA
+    interleaved (CSA first), the headline decode batch (8 requests at 131072
+    tokens) going through every layer, all layers paged through ONE block
+    table.  One decode step = every layer's step for every request (CSA:
+    the four library calls; HCA: append + attend), one CUDA graph per step.
+    The layers are independent copies of one built CSA and one built HCA
+    layer (the same bytes, separate memory), so the stack touches n_layers
+    layers' caches per step, far more than L2."""
+    import torch
+    from csla_synth import permutation
+    kc = dict(CSA)
+    kh = dict(HCA, B=kc["B"], L=kc["L"])
+    B, m = kc["B"], kc["m"]
+    L0s = [kc["L"] - (W + K) - (b % m) for b in range(B)]
+    pages_per = -(-(kc["L"] + HEADROOM) // 128)
+    bt = torch.from_numpy(permutation(seed, "stack_pages/%d" % rank, B * pages_per).astype("int32")
+                          .reshape(B, pages_per)).to(device)
+    clb, ccp, cpar = build_layer(kc, B, L0s, seed, rank, device, block_table=bt)
+    hlb, hcp, hpar = build_layer(kh, B, L0s, seed + 1, rank, device, block_table=bt)
+    cin = step_inputs(kc, B, W + K, seed, rank, device)
+    hin = step_inputs(kh, B, W + K, seed + 1, rank, device)
+    CsaStep.fused = False
+    layers = []
+    for i in range(n_layers):
+        csa = i % 2 == 0
+        base, cp, par = (clb, ccp, cpar) if csa else (hlb, hcp, hpar)
+        nb, np_ = (base, par) if i < 2 else clone_layer(base, par, share_block_table=True)
+        layers.append((CsaStep if csa else HcaStep)(nb, cp, np_, kc if csa else kh, variant, device))
+    assert all(st.lb.block_table.data_ptr() == bt.data_ptr() for st in layers)
+    ins = lambda i, j: cin[j] if i % 2 == 0 else hin[j]
+    for j in range(W):
+        for i, st in enumerate(layers):
+            for c in st.calls:
+                c(ins(i, j))
+    torch.cuda.synchronize()
+    graphs = []
+    for j in range(W, W + K):
+        graphs.append(capture(lambda: [c(ins(i, j)) for i, st in enumerate(layers) for c in st.calls]))
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for g in graphs:
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = dp_max(e0.elapsed_time(e1) / K, world, device)
+    del graphs
+    n_csa = (n_layers + 1) // 2
+    hca_launches = 2 + attend_launches(kh["L"] // kh["m"] + kh["n_win"], B, variant)
+    launches = n_csa * csa_launches(kc, variant, False) + (n_layers - n_csa) * hca_launches
+    out = {"workload": "stack%d_csa_hca_B8_L131072" % n_layers, "layers": n_layers,
+           "layer_order": "CSA, HCA, CSA, ... (interleaved)", "tokens_per_s": B * world / (ms * 1e-3),
+           "ms_per_step": ms, "us_per_layer": ms * 1e3 / n_layers, "launches_per_step": launches,
+           "block_table": "one [8, %d] int32 table shared by all layers" % pages_per,
+           "l2": "inputs larger than L2 (%d layers' caches touched per step)" % n_layers}
+    del layers, clb, hlb, cin, hin
+    torch.cuda.empty_cache()
+    return out
+
+
+def clone_layer(lb, params, share_block_table=False):
     """An independent copy of a layer's device buffers and weights (the
     rotation below walks several such copies, like the layers of a model)."""
     from compressed_sparse_long_append_b200.layer import LayerBuffers
     nb = object.__new__(LayerBuffers)
     nb.__dict__.update(lb.__dict__)
-    for k in ("rows", "scales", "kidx", "block_table", "win_rows", "win_scales", "tail_kv", "tail_idx", "len"):
+    for k in ("rows", "scales", "kidx", "kscale", "block_table", "win_rows", "win_scales", "tail_kv", "tail_idx",
+              "len"):
+        if k == "block_table" and share_block_table:
+            continue
         v = getattr(lb, k)
         setattr(nb, k, None if v is None else v.clone())
     return nb, {k: v.clone() for k, v in params.items()}
@@ -981,6 +1056,9 @@ def main():
     inv = None
     if not args.no_invariance and not args.profile:
         inv = invariance_leg(W, K, seed + 4, rank, world, device, args.variant)
+    stk = None
+    if not args.no_stack and not args.profile:
+        stk = stack_leg(W, K, seed + 6, rank, world, device, args.variant, args.stack_layers)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -1027,6 +1105,7 @@ def main():
             "csa_prefill": pre,
             "csa_decode_e4m3_keys": e4,
             "invariance_decode": inv,
+            "stack_decode": stk,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -15,6 +15,7 @@ CSLA_OK, CSLA_ERR_ARG, CSLA_ERR_UNSUPPORTED, CSLA_ERR_CUDA, CSLA_ERR_DEVICE = 0,
 CSLA_F32, CSLA_BF16 = 0, 1
 CSLA_VARIANT_AUTO, CSLA_VARIANT_SATURATED, CSLA_VARIANT_STARVED = 0, 1, 2
 CSLA_KEY_BF16, CSLA_KEY_E4M3 = 0, 1
+CSLA_GATE_TOKEN, CSLA_GATE_CHANNEL = 0, 1
 CSLA_OP_INDEXER, CSLA_OP_TOPK, CSLA_OP_CSA_ATTEND, CSLA_OP_HCA_ATTEND, CSLA_OP_CSA_DECODE_STEP = 1, 2, 3, 4, 5
 CSLA_DEVERR_PAGE, CSLA_DEVERR_INDEX, CSLA_DEVERR_LEN, CSLA_DEVERR_TIMEOUT, CSLA_DEVERR_RANGE = 1, 2, 4, 8, 16
 CSLA_PAGE_TOKENS = 128
@@ -29,7 +30,7 @@ class csla_cfg(ctypes.Structure):
     _fields_ = [("m", ctypes.c_int32), ("D", ctypes.c_int32), ("d_rope", ctypes.c_int32),
                 ("H", ctypes.c_int32), ("HI", ctypes.c_int32), ("dI", ctypes.c_int32),
                 ("dc", ctypes.c_int32), ("n_win", ctypes.c_int32), ("rope_theta", ctypes.c_float),
-                ("eps", ctypes.c_float), ("key_fmt", ctypes.c_int32)]
+                ("eps", ctypes.c_float), ("key_fmt", ctypes.c_int32), ("gate", ctypes.c_int32)]
 
 
 class csla_cache(ctypes.Structure):

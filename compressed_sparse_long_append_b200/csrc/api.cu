@@ -81,6 +81,7 @@ int check_cfg(const csla_cfg *c) {
     if (!(c->eps >= 0.f) || !(c->rope_theta > 0.f)) return CSLA_ERR_ARG;
     if (c->key_fmt != CSLA_KEY_BF16 && c->key_fmt != CSLA_KEY_E4M3) return CSLA_ERR_UNSUPPORTED;
     if (c->key_fmt == CSLA_KEY_E4M3 && c->m == 4 && c->dI != 128) return CSLA_ERR_UNSUPPORTED;
+    if (c->gate != CSLA_GATE_TOKEN && c->gate != CSLA_GATE_CHANNEL) return CSLA_ERR_UNSUPPORTED;
     return CSLA_OK;
 }
 
@@ -215,6 +216,8 @@ static int prep_compress(const csla_cfg *cfg, const csla_state *st, const csla_c
         !cache->block_table || cache->bt_stride < 1 || cache->n_pages < 1)
         return CSLA_ERR_ARG;
     if (!p->gamma_kv || !p->wg || !p->gb) return CSLA_ERR_ARG;
+    const bool per_channel = cfg->gate == CSLA_GATE_CHANNEL;
+    if (per_channel && (!aligned16(p->gb) || (p->gbi && !aligned16(p->gbi)))) return CSLA_ERR_ARG;
     if (!aligned16(st->tail_kv)) return CSLA_ERR_ARG;
     if (tok && (!tok->rows || !tok->scales || tok->offset < 0 || (long long)tok->offset + T > tok->stride))
         return CSLA_ERR_ARG;
@@ -237,6 +240,7 @@ static int prep_compress(const csla_cfg *cfg, const csla_state *st, const csla_c
     a.tail_idx = csa ? st->tail_idx : nullptr; a.len = st->len;
     a.rows = cache->rows; a.scales = cache->scales; a.kidx = csa ? cache->kidx : nullptr;
     a.key_fmt = csa ? cfg->key_fmt : CSLA_KEY_BF16;
+    a.gate = cfg->gate;
     a.kscale = csa ? cache->kscale : nullptr;
     a.block_table = cache->block_table; a.bt_stride = cache->bt_stride; a.n_pages = cache->n_pages;
     a.n_slots = st->n_slots;

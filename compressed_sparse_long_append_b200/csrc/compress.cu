@@ -295,6 +295,118 @@ __device__ void pool_small(const BlockRows<T> &x, int m, const float *wsm, const
     __syncthreads();
 }
 
+// Per-channel gate: channel d of row i has the gate x_id * w_d + b_id, and
+// every channel takes its own softmax over the block's rows.  Thread t <
+// width/4 owns columns 4t..4t+3; the rows it sees are folded in order into a
+// running (max, sum of weights, weighted sum) that is rescaled whenever the
+// max rises.  pool_small_channel: one group of rows (m <= kSmallM, every
+// row in registers, max first).  pool_block_channel: G = 256 / (width / 4)
+// row groups, group g folds rows g, g + G, ...; the groups' states meet in
+// shared memory (st, 12 * kThreads floats) and are merged in group order.
+// The pooled row (width floats) goes to out (smem).
+struct ChanState {
+    float4 mx, z, acc;
+};
+__device__ __forceinline__ void chan_fold1(float &mx, float &z, float &acc, float g, float xv) {
+    if (g > mx) {
+        const float r = expf(__fsub_rn(mx, g));   // 0 on the first row (mx = -inf)
+        z = __fmaf_rn(z, r, 1.f);
+        acc = __fmaf_rn(acc, r, xv);
+        mx = g;
+    } else {
+        const float e = g == -INFINITY ? 0.f : expf(__fsub_rn(g, mx));   // a -inf gate weighs 0
+        z = __fadd_rn(z, e);
+        acc = __fmaf_rn(e, xv, acc);
+    }
+}
+__device__ __forceinline__ void chan_fold(ChanState &s, float4 x, float4 w, float4 b) {
+    chan_fold1(s.mx.x, s.z.x, s.acc.x, __fmaf_rn(x.x, w.x, b.x), x.x);
+    chan_fold1(s.mx.y, s.z.y, s.acc.y, __fmaf_rn(x.y, w.y, b.y), x.y);
+    chan_fold1(s.mx.z, s.z.z, s.acc.z, __fmaf_rn(x.z, w.z, b.z), x.z);
+    chan_fold1(s.mx.w, s.z.w, s.acc.w, __fmaf_rn(x.w, w.w, b.w), x.w);
+}
+// Merge state o into s (o's rows come after s's).
+__device__ __forceinline__ void chan_merge1(float &mx, float &z, float &acc, float omx, float oz, float oacc) {
+    const float M = fmaxf(mx, omx);
+    if (M == -INFINITY) return;
+    const float rs = expf(__fsub_rn(mx, M)), ro = expf(__fsub_rn(omx, M));
+    z = __fmaf_rn(oz, ro, __fmul_rn(z, rs));
+    acc = __fmaf_rn(oacc, ro, __fmul_rn(acc, rs));
+    mx = M;
+}
+
+template <typename T>
+__device__ void pool_small_channel(const BlockRows<T> &x, int m, const float *wsm, const float *bias, float *out) {
+    const int nq = x.width >> 2;
+    if (threadIdx.x < nq) {
+        const float4 w = reinterpret_cast<const float4 *>(wsm)[threadIdx.x];
+        ChanState s{make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY), make_float4(0.f, 0.f, 0.f, 0.f),
+                    make_float4(0.f, 0.f, 0.f, 0.f)};
+#pragma unroll
+        for (int i = 0; i < kSmallM; ++i) {
+            if (i < m) {
+                const float4 b = __ldg(reinterpret_cast<const float4 *>(bias + (size_t)i * x.width) + threadIdx.x);
+                chan_fold(s, x.get(i, threadIdx.x), w, b);
+            }
+        }
+        reinterpret_cast<float4 *>(out)[threadIdx.x] =
+            make_float4(__fdiv_rn(s.acc.x, s.z.x), __fdiv_rn(s.acc.y, s.z.y), __fdiv_rn(s.acc.z, s.z.z),
+                        __fdiv_rn(s.acc.w, s.z.w));
+    }
+    __syncthreads();
+}
+
+template <typename T>
+__device__ void pool_block_channel(const BlockRows<T> &x, int m, const float *wsm, const float *bias, float *st,
+                                   float *out) {
+    const int nq = x.width >> 2;
+    const int G = kThreads / nq;   // nq <= 128, so G >= 2
+    const int g = threadIdx.x / nq, c4 = threadIdx.x % nq;
+    float4 *st4 = reinterpret_cast<float4 *>(st);
+    if (g < G) {
+        const float4 w = reinterpret_cast<const float4 *>(wsm)[c4];
+        ChanState s{make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY), make_float4(0.f, 0.f, 0.f, 0.f),
+                    make_float4(0.f, 0.f, 0.f, 0.f)};
+#pragma unroll 4
+        for (int i = g; i < m; i += G) {
+            const float4 b = __ldg(reinterpret_cast<const float4 *>(bias + (size_t)i * x.width) + c4);
+            chan_fold(s, x.get(i, c4), w, b);
+        }
+        st4[(0 * G + g) * nq + c4] = s.mx;
+        st4[(1 * G + g) * nq + c4] = s.z;
+        st4[(2 * G + g) * nq + c4] = s.acc;
+    }
+    __syncthreads();
+    if (threadIdx.x < nq) {
+        ChanState s{st4[threadIdx.x], st4[G * nq + threadIdx.x], st4[2 * G * nq + threadIdx.x]};
+        for (int q = 1; q < G; ++q) {
+            const float4 omx = st4[q * nq + threadIdx.x], oz = st4[(G + q) * nq + threadIdx.x],
+                         oa = st4[(2 * G + q) * nq + threadIdx.x];
+            chan_merge1(s.mx.x, s.z.x, s.acc.x, omx.x, oz.x, oa.x);
+            chan_merge1(s.mx.y, s.z.y, s.acc.y, omx.y, oz.y, oa.y);
+            chan_merge1(s.mx.z, s.z.z, s.acc.z, omx.z, oz.z, oa.z);
+            chan_merge1(s.mx.w, s.z.w, s.acc.w, omx.w, oz.w, oa.w);
+        }
+        reinterpret_cast<float4 *>(out)[threadIdx.x] =
+            make_float4(__fdiv_rn(s.acc.x, s.z.x), __fdiv_rn(s.acc.y, s.z.y), __fdiv_rn(s.acc.z, s.z.z),
+                        __fdiv_rn(s.acc.w, s.z.w));
+    }
+    __syncthreads();
+}
+
+template <typename T>
+__device__ __forceinline__ void pool_any(const BlockRows<T> &x, int m, int gate, const float *wsm, float *alpha,
+                                         const float *bias, float *part, float *xs, float *out, float *red) {
+    if (gate == CSLA_GATE_CHANNEL) {
+        if (m <= kSmallM) pool_small_channel<T>(x, m, wsm, bias, out);
+        else pool_block_channel<T>(x, m, wsm, bias, xs, out);
+    } else if (m <= kSmallM) {
+        pool_small<T>(x, m, wsm, alpha, part, out);
+    } else {
+        pool_block<T>(x, m, wsm, alpha, part, xs, out, red);
+    }
+}
+
 // kTok: the call also keeps every new token's window row (CompressArgs::tok_rows).
 template <typename T, bool kTok>
 __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs a) {
@@ -344,7 +456,8 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs 
         const float *w = z == 0 ? a.wg : a.wgi;
         const float *gb = z == 0 ? a.gb : a.gbi;
         for (int d = threadIdx.x; d < width; d += kThreads) wsm[d] = __ldg(w + d);
-        for (int i = threadIdx.x; i < m; i += kThreads) alpha[i] = __ldg(gb + i);
+        if (a.gate != CSLA_GATE_CHANNEL)
+            for (int i = threadIdx.x; i < m; i += kThreads) alpha[i] = __ldg(gb + i);
     }
     pdl_wait();
     CSLA_TL_WAITED();
@@ -409,8 +522,7 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs 
         const T *fresh = reinterpret_cast<const T *>(a.kv_new) + ((size_t)b * a.T + f0) * D;
         const BlockRows<T> rows{a.tail_kv + (size_t)slot * m * D, fresh, n_tail, D,
                                 (reinterpret_cast<uintptr_t>(a.kv_new) & vec_mask) == 0};
-        if (m <= kSmallM) pool_small<T>(rows, m, wsm, alpha, part, v);
-        else pool_block<T>(rows, m, wsm, alpha, part, xs, v, red);
+        pool_any<T>(rows, m, a.gate, wsm, alpha, a.gb, part, xs, v, red);
         CSLA_TL_MARK(1);
         norm_rope_quantise(v, gam, a, p0, a.rows + ent * rb, a.scales + ent, red);
         CSLA_TL_MARK(2);
@@ -419,8 +531,7 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs 
         const T *fresh = reinterpret_cast<const T *>(a.kidx_new) + ((size_t)b * a.T + f0) * dI;
         const BlockRows<T> rows{a.tail_idx + (size_t)slot * m * dI, fresh, n_tail, dI,
                                 (reinterpret_cast<uintptr_t>(a.kidx_new) & vec_mask) == 0};
-        if (m <= kSmallM) pool_small<T>(rows, m, wsm, alpha, part, v);
-        else pool_block<T>(rows, m, wsm, alpha, part, xs, v, red);
+        pool_any<T>(rows, m, a.gate, wsm, alpha, a.gbi, part, xs, v, red);
         CSLA_TL_MARK(1);
         if (a.key_fmt == CSLA_KEY_E4M3) {
             // one power-of-two scale per entry: the smallest 2^e with

@@ -54,6 +54,7 @@ struct CompressArgs {
     void *kidx;           // bf16 keys, or E4M3 codes (key_fmt)
     float *kscale;        // E4M3 keys: per-entry power-of-two scale
     int key_fmt;
+    int gate;             // CSLA_GATE_TOKEN or CSLA_GATE_CHANNEL (gb, gbi [m][width])
     const int32_t *block_table;
     int bt_stride, n_pages, n_slots;
     uint8_t *tok_rows;    // optional: window-format row of every new token

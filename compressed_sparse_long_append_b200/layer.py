@@ -24,6 +24,7 @@ class LayerShape:
     theta: float = 10000.0
     eps: float = 1e-6
     key_fmt: int = C.CSLA_KEY_BF16   # CSA index keys: bf16, or E4M3 codes + per-entry power-of-two scale
+    gate: int = C.CSLA_GATE_TOKEN    # compressor gate: one per token, or one per token and channel
 
     @property
     def is_csa(self):
@@ -40,13 +41,16 @@ class LayerShape:
     def cfg(self):
         return C.csla_cfg(self.m, self.D, self.d_rope, self.H, self.HI if self.is_csa else 0,
                           self.dI if self.is_csa else 0, self.dc if self.is_csa else 0, self.n_win,
-                          self.theta, self.eps, self.key_fmt if self.is_csa else C.CSLA_KEY_BF16)
+                          self.theta, self.eps, self.key_fmt if self.is_csa else C.CSLA_KEY_BF16, self.gate)
 
 
 class LayerBuffers:
-    """Classical cache pages + block table + state cache for `n_slots` requests."""
+    """Classical cache pages + block table + state cache for `n_slots` requests.
+    `block_table` ([n_slots, bt_stride] int32 on the device) is used as given
+    instead of a table of the layer's own (layers of one model share one)."""
 
-    def __init__(self, shape: LayerShape, n_slots: int, n_pages: int, bt_stride: int, device="cuda"):
+    def __init__(self, shape: LayerShape, n_slots: int, n_pages: int, bt_stride: int, device="cuda",
+                 block_table=None):
         s = shape
         self.shape = s
         self.device = torch.device(device)
@@ -57,7 +61,12 @@ class LayerBuffers:
         kdt = torch.uint8 if fp8_keys else torch.int16
         self.kidx = torch.zeros((n_pages, s.epp, s.dI), dtype=kdt, device=dev) if s.is_csa else None
         self.kscale = torch.zeros((n_pages, s.epp), dtype=torch.float32, device=dev) if fp8_keys else None
-        self.block_table = torch.full((n_slots, bt_stride), -1, dtype=torch.int32, device=dev)
+        if block_table is None:
+            block_table = torch.full((n_slots, bt_stride), -1, dtype=torch.int32, device=dev)
+        elif (block_table.dtype != torch.int32 or tuple(block_table.shape) != (n_slots, bt_stride)
+              or not block_table.is_contiguous() or block_table.device != dev):
+            raise ValueError("block_table must be a contiguous [n_slots, bt_stride] int32 tensor on %s" % dev)
+        self.block_table = block_table
         self.win_rows = torch.zeros((n_slots, s.n_win, s.row_bytes), dtype=torch.uint8, device=dev)
         self.win_scales = torch.zeros((n_slots, s.n_win), dtype=torch.float32, device=dev)
         self.tail_kv = torch.zeros((n_slots, s.m, s.D), dtype=torch.float32, device=dev)
@@ -90,6 +99,29 @@ class LayerBuffers:
         if self.kscale is not None:
             out["kscale"] = self.kscale.cpu().numpy()
         return out
+
+
+class LayerStack:
+    """The attention layers of one model over one block table.  A page is
+    128 raw tokens of a request in every layer (32 CSA entries or 1 HCA
+    entry), so page id p of a request names page p of each layer's own
+    pool: one allocation covers the whole stack.  Every layer keeps its own
+    pools, window ring, tail and length (each layer appends its own
+    compressed KV).  `shapes[i]` is layer i's shape, e.g. CSA and HCA
+    layers interleaved."""
+
+    def __init__(self, shapes, n_slots: int, n_pages: int, bt_stride: int, device="cuda"):
+        self.device = torch.device(device)
+        self.block_table = torch.full((n_slots, bt_stride), -1, dtype=torch.int32, device=self.device)
+        self.layers = [LayerBuffers(s, n_slots, n_pages, bt_stride, device, block_table=self.block_table)
+                       for s in shapes]
+        self.n_slots, self.n_pages, self.bt_stride = n_slots, n_pages, bt_stride
+
+    def __len__(self):
+        return len(self.layers)
+
+    def __getitem__(self, i):
+        return self.layers[i]
 
 
 class CompressParams:

@@ -29,6 +29,7 @@ class Workload:
     act_bf16: bool = True   # activations are exact bf16 values
     seed: int = 0
     key_fmt: int = 0        # CSA index keys: 0 bf16, 1 E4M3 codes + per-entry power-of-two scale
+    gate: int = 0           # compressor gate: 0 one per token, 1 one per token and channel
 
     @property
     def is_csa(self):
@@ -68,6 +69,15 @@ def layer_params(w: Workload):
     if w.is_csa:
         p["wgi"] = normal(w.seed, "wgi", (w.dI,), std=1.0 / np.sqrt(w.dI))
         p["gbi"] = normal(w.seed, "gbi", (w.m,))
+    if w.gate == 1:
+        # per-channel gate x_id * w_d + b_id: an O(1) weight per channel and
+        # a bias per position and channel
+        p["wg"] = normal(w.seed, "wg_ch", (w.D,))
+        p["gb"] = normal(w.seed, "gb_ch", (w.m, w.D))
+        if w.is_csa:
+            p["wgi"] = normal(w.seed, "wgi_ch", (w.dI,))
+            p["gbi"] = normal(w.seed, "gbi_ch", (w.m, w.dI))
+    if w.is_csa:
         p["W_iq"] = _act(w, "W_iq", (w.HI * w.dI, w.dc), std=1.0 / np.sqrt(w.dc))
     # fp32 parameters: round once so both sides see the same fp32 values
     return {k: v.astype(np.float32).astype(np.float64) for k, v in p.items()}

@@ -92,6 +92,15 @@ enum { CSLA_VARIANT_AUTO = 0, CSLA_VARIANT_SATURATED = 1, CSLA_VARIANT_STARVED =
  * dI = 128 instead of 256. */
 enum { CSLA_KEY_BF16 = 0, CSLA_KEY_E4M3 = 1 };
 
+/* Gate of the token-level compressor (硅星人 §两大压缩注意力: a token-level
+ * compressor turns each block of m tokens into one entry; the pages give no
+ * formula).  TOKEN: one scalar gate per token, g_i = <x_i, wg> + gb[i],
+ * softmax over the block's tokens, entry = sum_i alpha_i x_i.  CHANNEL: one
+ * gate per token and channel, g_id = x_id * wg[d] + gb[i][d], a separate
+ * softmax over the block's tokens for every channel d, entry_d =
+ * sum_i alpha_id x_id (gb, gbi are then [m][D], [m][dI]). */
+enum { CSLA_GATE_TOKEN = 0, CSLA_GATE_CHANNEL = 1 };
+
 enum {
     CSLA_OP_INDEXER = 1,
     CSLA_OP_TOPK = 2,
@@ -125,7 +134,8 @@ typedef struct csla_cfg {
     int32_t n_win;      /* sliding window, 128 */
     float rope_theta;   /* RoPE base, 10000 */
     float eps;          /* RMSNorm epsilon, 1e-6 */
-    int32_t key_fmt;    /* CSA index-key storage: CSLA_KEY_BF16 (default) or CSLA_KEY_E4M3 */
+    int32_t key_fmt;    /* CSA index-key storage: CSLA_KEY_BF16 (default) or CSLA_KEY_E4M3 (dI = 128) */
+    int32_t gate;       /* compressor gate: CSLA_GATE_TOKEN (default) or CSLA_GATE_CHANNEL */
 } csla_cfg;
 
 typedef struct csla_cache {
@@ -147,13 +157,15 @@ typedef struct csla_state {
     int32_t n_slots;
 } csla_state;
 
-/* Compressor parameters, device f32 arrays. */
+/* Compressor parameters, device f32 arrays (shapes for CSLA_GATE_TOKEN;
+ * with CSLA_GATE_CHANNEL the biases have one value per position and channel
+ * and must be 16-byte aligned). */
 typedef struct csla_compress_params {
     const float *gamma_kv;     /* [D]  RMSNorm weight of the KV head */
     const float *wg;           /* [D]  gate weight of the KV compressor */
-    const float *gb;           /* [m]  gate bias per position in the block */
+    const float *gb;           /* [m]  gate bias per position in the block ([m][D] per channel) */
     const float *wgi;          /* [dI] gate weight of the index-key compressor (CSA) */
-    const float *gbi;          /* [m]  gate bias of the index-key compressor (CSA) */
+    const float *gbi;          /* [m]  gate bias of the index-key compressor (CSA; [m][dI] per channel) */
 } csla_compress_params;
 
 /*

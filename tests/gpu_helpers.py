@@ -15,7 +15,7 @@ DEV = "cuda"
 
 def shape_of(w: Workload):
     return LayerShape(m=w.m, D=w.D, H=w.H, HI=w.HI or 16, dI=w.dI or 128, dc=w.dc or 1024, n_win=w.n_win,
-                      d_rope=w.d_rope, theta=w.theta, eps=w.eps, key_fmt=w.key_fmt)
+                      d_rope=w.d_rope, theta=w.theta, eps=w.eps, key_fmt=w.key_fmt, gate=w.gate)
 
 
 def act_tensor(w: Workload, x):
@@ -53,9 +53,15 @@ def append(w, lb, cp, slot, ts, start, stop, chunk=None):
 def upload_layer(w: Workload, cv, lens):
     """Device copy of a cache the oracle built (tests/helpers.oracle_cache):
     the GPU steps then read exactly the bytes the oracle decodes."""
-    shape = shape_of(w)
     n_pages = cv.rows.shape[0]
-    lb = LayerBuffers(shape, len(lens), n_pages, cv.block_table.shape[1], DEV)
+    lb = LayerBuffers(shape_of(w), len(lens), n_pages, cv.block_table.shape[1], DEV)
+    fill_layer(lb, w, cv, lens)
+    return lb
+
+
+def fill_layer(lb: LayerBuffers, w: Workload, cv, lens):
+    """Copy an oracle-built cache into existing layer buffers (the block
+    table too: with a table shared by several layers it must be the same)."""
     lb.rows.copy_(torch.from_numpy(cv.rows))
     lb.scales.copy_(torch.from_numpy(cv.scales))
     if w.is_csa and cv.kscale is not None:
@@ -68,7 +74,6 @@ def upload_layer(w: Workload, cv, lens):
     lb.win_scales.copy_(torch.from_numpy(cv.win_scales))
     lb.len.copy_(torch.tensor(list(lens), dtype=torch.int32))
     torch.cuda.synchronize()
-    return lb
 
 
 def cache_view(w: Workload, lb: LayerBuffers):
@@ -160,3 +165,29 @@ def check_scores(got, ref):
     assert np.all(np.isfinite(got))
     assert err.max() <= REL_TOL, err.max()
     return err.max()
+
+
+def check_csa_step(w: Workload, cv, p, si, lens, gidx, gout):
+    """One CSA decode step of len(lens) requests on the GPU (top-k lists
+    gidx, outputs gout) against the oracle on the cache cv: every entry
+    scoring clearly above the k-th oracle score is selected, none clearly
+    below; the output matches the oracle's step, or, where a tie inside the
+    band picked another set, the oracle's attention over the GPU's set."""
+    B = len(lens)
+    oidx, oout = oracle.csa_decode(cv, np.arange(B), lens, si["q"][:B], p["gamma_q"], si["cq"][:B], p["W_iq"],
+                                   si["head_w"][:B], p["sink"], w.HI, w.k, w.eps, w.theta)
+    for s, L in enumerate(lens):
+        nv = L // w.m
+        sel = set(int(x) for x in gidx[s] if x >= 0)
+        if nv > 0:
+            qI = oracle.index_query(si["cq"][s], p["W_iq"], w.HI, w.dI)
+            ref = oracle.index_scores(qI, si["head_w"][s], cv.gather_keys(s, nv))
+            kth = np.sort(ref)[::-1][min(w.k, nv) - 1]
+            assert set(np.nonzero(ref > kth + 1e-4)[0].tolist()) <= sel, s
+            assert not (sel & set(np.nonzero(ref < kth - 1e-4)[0].tolist())), s
+        if set(oidx[s][oidx[s] >= 0].tolist()) == sel:
+            check_out(gout[s], oout[s])
+        else:
+            rows = cv.gather_set(s, L, gidx[s])
+            r2, _ = oracle.attend(si["q"][s], p["gamma_q"], L - 1, rows, p["sink"], w.eps, w.theta, w.d_rope)
+            check_out(gout[s], r2)

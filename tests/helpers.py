@@ -24,13 +24,17 @@ def block_table(w: Workload, lens, n_slots, seed_name="bt"):
     return bt, max(total, 1)
 
 
-def oracle_cache(w: Workload, lens, params=None, with_raw=False, stream_ids=None):
+def oracle_cache(w: Workload, lens, params=None, with_raw=False, stream_ids=None, bt=None):
     """Expected cache of len(lens) requests (slot i = request i, whose token
     stream is stream_ids[i], default i) after their whole token streams
-    0..L_i-1 were appended, computed by the oracle."""
+    0..L_i-1 were appended, computed by the oracle.  bt: a given block table
+    (pages 0..max id), else a seeded one of the layer's own."""
     p = params or layer_params(w)
     n_slots = len(lens)
-    bt, n_pages = block_table(w, lens, n_slots)
+    if bt is None:
+        bt, n_pages = block_table(w, lens, n_slots)
+    else:
+        n_pages = int(bt.max()) + 1
     epp = PAGE // w.m
     rb = oracle.row_bytes(w.D, w.d_rope)
     rows = np.zeros((n_pages, epp, rb), np.uint8)
@@ -46,7 +50,8 @@ def oracle_cache(w: Workload, lens, params=None, with_raw=False, stream_ids=None
         raws.append(ts)
         exp = oracle.expected_append(ts["kv"], ts.get("idx"), 0, L, w.m, p["gamma_kv"], p["wg"],
                                      p["gb"], p.get("wgi"), p.get("gbi"), w.eps, w.theta, w.d_rope,
-                                     window_from=L - w.n_win, key_e4m3=e4m3)
+                                     window_from=L - w.n_win, key_e4m3=e4m3,
+                                     per_channel=w.gate == 1)
         for pos, (r, sc) in exp["window"].items():
             if pos >= L - w.n_win:
                 win_rows[s, pos % w.n_win] = r

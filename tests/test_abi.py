@@ -75,6 +75,15 @@ def test_host_argument_checks():
     for bad in (dict(m=8), dict(m=4, D=256), dict(m=4, d_rope=32), dict(m=4, H=65), dict(m=4, n_win=64)):
         assert L.csla_topk_select(ctypes.byref(_cfg(**bad)), None, None, 1, None, 10, None, 10, 5, None, None) \
             == C.CSLA_ERR_UNSUPPORTED, bad
+    assert L.csla_topk_select(ctypes.byref(_cfg(m=4, gate=2)), None, None, 1, None, 10, None, 10, 5, None, None) \
+        == C.CSLA_ERR_UNSUPPORTED
+    # per-channel gate biases must be 16-byte aligned
+    cst = C.csla_state(fake, fake, fake, fake, fake, 4)
+    cch = C.csla_cache(fake, fake, fake, fake, 8, 16)
+    odd = C.csla_compress_params(fake, fake, fake + 4, fake, fake)
+    assert L.csla_compress_append(ctypes.byref(_cfg(m=4, gate=C.CSLA_GATE_CHANNEL)), ctypes.byref(cst),
+                                  ctypes.byref(cch), fake, 1, 1, fake, fake, C.CSLA_BF16, ctypes.byref(odd), None,
+                                  None) == C.CSLA_ERR_ARG
     assert L.csla_strerror(C.CSLA_ERR_DEVICE) == b"device-side input error"
     # the bounded-wait check takes 1 us .. 2 s
     assert L.csla_check_wait_timeout(0, None) == C.CSLA_ERR_ARG

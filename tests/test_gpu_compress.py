@@ -31,14 +31,20 @@ def _check_layer(w, lb, p, lens):
         # compressed entries
         for b in range(L // w.m):
             xs = ts["kv"][b * w.m:(b + 1) * w.m]
-            c, _ = oracle.gate_pool(xs, p["wg"], p["gb"])
+            if w.gate == 1:
+                c = oracle.gate_pool_channel(xs, p["wg"], p["gb"])
+            else:
+                c, _ = oracle.gate_pool(xs, p["wg"], p["gb"])
             y = oracle.rope(oracle.rmsnorm(c, p["gamma_kv"], w.eps), b * w.m, w.theta, w.d_rope)
             pg = h["block_table"][s, b // epp]
             tolerated += compare_rows(h["rows"][pg, b % epp], h["scales"][pg, b % epp], y, w.D, w.d_rope)
             checked += 1
             if w.is_csa:
                 xi = ts["idx"][b * w.m:(b + 1) * w.m]
-                ref = oracle.index_key(xi, p["wgi"], p["gbi"])
+                if w.gate == 1:
+                    ref = oracle.key_bf16(oracle.gate_pool_channel(xi, p["wgi"], p["gbi"]))
+                else:
+                    ref = oracle.index_key(xi, p["wgi"], p["gbi"])
                 got = h["kidx"][pg, b % epp]
                 # fp32 gates and pooled sum: error well under 1e-5 of the largest input
                 assert_bf16_close(got, ref, 1e-5 * float(np.max(np.abs(xi))))
@@ -60,6 +66,10 @@ CSA_BIG = dataclasses.replace(CSA_DECODE, L=600, name="compress_csa512")
     (CSA_BIG, [600, 77], 64),
     (HCA_SMALL, [1000, 128, 255], 200),
     (HCA_SMALL, [300], 1),                # decode: one token per call
+    (dataclasses.replace(TINY, gate=1), [700, 3, 129], None),      # per-channel gate
+    (dataclasses.replace(CSA_BIG, gate=1), [600, 77], 1),
+    (dataclasses.replace(HCA_SMALL, gate=1), [1000, 128, 255], 200),
+    (dataclasses.replace(HCA_SMALL, gate=1), [300], 1),
 ])
 def test_compress_append_matches_oracle(w, lens, chunk):
     lb, cp, p = build_layer(w, lens, chunk=chunk)
