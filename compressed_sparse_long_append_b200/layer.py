@@ -64,7 +64,7 @@ class LayerBuffers:
         if block_table is None:
             block_table = torch.full((n_slots, bt_stride), -1, dtype=torch.int32, device=dev)
         elif (block_table.dtype != torch.int32 or tuple(block_table.shape) != (n_slots, bt_stride)
-              or not block_table.is_contiguous() or block_table.device != dev):
+              or not block_table.is_contiguous() or block_table.device.type != dev.type):
             raise ValueError("block_table must be a contiguous [n_slots, bt_stride] int32 tensor on %s" % dev)
         self.block_table = block_table
         self.win_rows = torch.zeros((n_slots, s.n_win, s.row_bytes), dtype=torch.uint8, device=dev)
