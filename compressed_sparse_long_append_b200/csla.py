@@ -22,7 +22,9 @@ CSLA_PAGE_TOKENS = 128
 
 EXPORTS = ("csla_compress_append", "csla_indexer_scores", "csla_topk_select", "csla_csa_attend",
            "csla_hca_attend", "csla_workspace_size", "csla_device_error", "csla_strerror", "csla_version",
-           "csla_indexer_scores_noalloc", "csla_window_rows", "csla_csa_decode_step", "csla_check_wait_timeout")
+           "csla_indexer_scores_noalloc", "csla_window_rows", "csla_csa_decode_step", "csla_check_wait_timeout",
+           "csla_cp_record_bytes", "csla_cp_select", "csla_cp_place")
+CSLA_CP_MAX_RANKS = 64
 CSLA_NOALLOC_INDEXER_SCRATCH_BYTES = 786432
 
 
@@ -102,11 +104,15 @@ def _load():
         "csla_strerror": [ctypes.c_int],
         "csla_version": [],
         "csla_check_wait_timeout": [ctypes.c_uint32, P],
+        "csla_cp_record_bytes": [P],
+        "csla_cp_select": [P, P, P, I, I, I, I, P, P],
+        "csla_cp_place": [P, P, P, I, P, I, I, P, P, P],
         "csla_indexer_scores_noalloc": [P, P, P, P, I, P, I, P, I, P, I, P, P, I, P],
         "csla_csa_decode_step": [P, P, P, P, I, I, I, P, P, I, P, P, I, P, I, P, P, I, I, P, P, I, P, P, P, I, I,
                                  P, Z, P, Z, P],
     }
-    res = {"csla_workspace_size": ctypes.c_size_t, "csla_strerror": ctypes.c_char_p}
+    res = {"csla_workspace_size": ctypes.c_size_t, "csla_strerror": ctypes.c_char_p,
+           "csla_cp_record_bytes": ctypes.c_int32}
     for name, args in sig.items():
         f = getattr(L, name)
         f.argtypes = args
@@ -218,6 +224,23 @@ def csla_device_error(stream=None):
 
 def csla_strerror(status):
     return _lib.csla_strerror(status).decode()
+
+
+def csla_cp_record_bytes(cfg):
+    return int(_lib.csla_cp_record_bytes(_ref(cfg)))
+
+
+def csla_cp_select(cfg, st, cache, slot, b_lo, n, E_max, recs, stream=None):
+    return _check("csla_cp_select", _lib.csla_cp_select(_ref(cfg), _ref(st), _ref(cache), slot, b_lo, n, E_max,
+                                                        _ptr(recs), _stream(stream)))
+
+
+def csla_cp_place(cfg, st, cache, slot, recs, E_max, b_lo, n, stream=None):
+    """b_lo, n: sequences of R ints (host)."""
+    R = len(b_lo)
+    arr = ctypes.c_int32 * max(R, 1)
+    return _check("csla_cp_place", _lib.csla_cp_place(_ref(cfg), _ref(st), _ref(cache), slot, _ptr(recs), R,
+                                                      E_max, arr(*b_lo), arr(*n), _stream(stream)))
 
 
 def csla_check_wait_timeout(limit_us, stream=None):

@@ -533,4 +533,65 @@ int csla_csa_decode_step(const csla_cfg *cfg, const csla_state *st, const csla_c
     return cuda_status(e);
 }
 
+// ---- context-parallel entry records
+
+static int cp_key_bytes(const csla_cfg *cfg) {
+    if (cfg->m != 4) return 0;
+    return cfg->key_fmt == CSLA_KEY_E4M3 ? cfg->dI : 2 * cfg->dI;
+}
+
+int32_t csla_cp_record_bytes(const csla_cfg *cfg) {
+    if (check_cfg(cfg) != CSLA_OK) return 0;
+    return (row_bytes_of(cfg) + cp_key_bytes(cfg) + 8 + 15) / 16 * 16;
+}
+
+static int prep_cp(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, int32_t slot,
+                   const void *recs, int32_t E_max, CpArgs *a) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (!st || slot >= st->n_slots) return CSLA_ERR_ARG;
+    if (!cache || !cache->rows || !cache->scales || !cache->block_table || cache->bt_stride < 1 ||
+        cache->n_pages < 1 || !recs || slot < 0 || E_max < 0)
+        return CSLA_ERR_ARG;
+    const bool csa = cfg->m == 4;
+    if (csa && (!cache->kidx || (cfg->key_fmt == CSLA_KEY_E4M3 && !cache->kscale))) return CSLA_ERR_ARG;
+    if (!aligned16(recs) || !aligned16(cache->rows) || (csa && !aligned16(cache->kidx))) return CSLA_ERR_ARG;
+    *a = CpArgs{};
+    a->slot = slot; a->epp = CSLA_PAGE_TOKENS / cfg->m; a->bt_stride = cache->bt_stride; a->n_pages = cache->n_pages;
+    a->block_table = cache->block_table; a->rows = cache->rows; a->scales = cache->scales;
+    a->kidx = csa ? static_cast<uint8_t *>(cache->kidx) : nullptr;
+    a->kscale = csa && cfg->key_fmt == CSLA_KEY_E4M3 ? cache->kscale : nullptr;
+    a->row_bytes = row_bytes_of(cfg); a->key_bytes = cp_key_bytes(cfg); a->rec_bytes = csla_cp_record_bytes(cfg);
+    a->E_max = E_max;
+    return CSLA_OK;
+}
+
+int csla_cp_select(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, int32_t slot,
+                   int32_t b_lo, int32_t n, int32_t E_max, uint8_t *recs, csla_stream_t stream) {
+    CpArgs a;
+    int rc = prep_cp(cfg, st, cache, slot, recs, E_max, &a);
+    if (rc) return rc;
+    if (b_lo < 0 || n < 0 || n > E_max) return CSLA_ERR_ARG;
+    a.place = 0; a.R = 1; a.b_lo[0] = b_lo; a.n[0] = n;
+    a.recs = recs;
+    return cuda_status(launch_cp_move(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int csla_cp_place(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, int32_t slot,
+                  const uint8_t *recs, int32_t R, int32_t E_max, const int32_t *b_lo, const int32_t *n,
+                  csla_stream_t stream) {
+    CpArgs a;
+    int rc = prep_cp(cfg, st, cache, slot, recs, E_max, &a);
+    if (rc) return rc;
+    if (R < 1 || R > CSLA_CP_MAX_RANKS || !b_lo || !n) return CSLA_ERR_ARG;
+    for (int r = 0; r < R; ++r) {
+        if (b_lo[r] < 0 || n[r] < 0 || n[r] > E_max) return CSLA_ERR_ARG;
+        a.b_lo[r] = b_lo[r];
+        a.n[r] = n[r];
+    }
+    a.place = 1; a.R = R;
+    a.recs = const_cast<uint8_t *>(recs);
+    return cuda_status(launch_cp_move(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

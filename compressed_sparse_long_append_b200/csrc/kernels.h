@@ -76,6 +76,23 @@ struct WindowRowsArgs {
 };
 cudaError_t launch_window_rows(const WindowRowsArgs &a, cudaStream_t stream);
 
+// Context-parallel entry records (csla_cp_select / csla_cp_place).
+struct CpArgs {
+    int place;                   // 0: cache -> records (select), 1: records -> cache (place)
+    int slot, epp, bt_stride, n_pages;
+    const int32_t *block_table;
+    uint8_t *rows;
+    float *scales;
+    uint8_t *kidx;               // CSA keys (bf16 or E4M3 bytes), else null
+    float *kscale;               // E4M3 key scales, else null
+    int row_bytes, key_bytes, rec_bytes;
+    uint8_t *recs;               // [R][E_max][rec_bytes]
+    int R, E_max;
+    int b_lo[CSLA_CP_MAX_RANKS];  // first block of rank r's run
+    int n[CSLA_CP_MAX_RANKS];     // valid records of rank r
+};
+cudaError_t launch_cp_move(const CpArgs &a, cudaStream_t stream);
+
 // Lightning indexer.  NQ = rows of the bf16 query operand (hi, mid and lo
 // terms of every head, zero padding to a multiple of 16).
 struct IndexerArgs {

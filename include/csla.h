@@ -418,6 +418,40 @@ int csla_device_error(csla_stream_t stream, uint32_t *bits);
  */
 int csla_check_wait_timeout(uint32_t limit_us, csla_stream_t stream);
 
+/*
+ * Context-parallel prefill (haiqwa "DeepSeek-V4" blog, §百万 token
+ * 怎么切分到多张卡: the compressed KV of one long request is built by R ranks,
+ * each compressing the blocks that close inside its own token range, then
+ * exchanged by one all-gather and reassembled by a select-and-pad step).
+ * Every rank holds a full copy of the request's paged cache (same block
+ * table shape; page ids may differ per rank).  These two calls are the
+ * data movement on either side of the all-gather; the exchange itself is
+ * the caller's collective (NCCL all-gather of equal-sized buffers).
+ *
+ * Entry record (csla_cp_record_bytes(cfg) bytes, a multiple of 16):
+ *   [row_bytes: the entry's row][key: dI*2 bytes bf16 or dI bytes E4M3, CSA
+ *   only][f32 row scale][f32 key scale, 0 for bf16 keys][zero pad].
+ *
+ * csla_cp_select: records 0..n-1 of `recs` = entries b_lo..b_lo+n-1 of
+ *   request `slot` (in block order); records n..E_max-1 are zero (padding).
+ *   recs [E_max][record] device, 16-byte aligned; 0 <= n <= E_max.
+ * csla_cp_place: for every rank r < R and j < n[r], record r*E_max + j of
+ *   `recs` becomes entry b_lo[r] + j of request `slot`; padding records are
+ *   skipped.  b_lo, n: HOST arrays of R int32 (copied at the call);
+ *   1 <= R <= CSLA_CP_MAX_RANKS.
+ * slot: the request's row of the block table (0 <= slot < st->n_slots;
+ * only st->n_slots is read).  A block whose page the block table does not
+ * map sets CSLA_DEVERR_PAGE and is skipped.  Errors: CSLA_ERR_ARG on null/bad sizes or misalignment;
+ * CSLA_ERR_UNSUPPORTED on shapes.
+ */
+#define CSLA_CP_MAX_RANKS 64
+int32_t csla_cp_record_bytes(const csla_cfg *cfg);
+int csla_cp_select(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, int32_t slot,
+                   int32_t b_lo, int32_t n, int32_t E_max, uint8_t *recs, csla_stream_t stream);
+int csla_cp_place(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, int32_t slot,
+                  const uint8_t *recs, int32_t R, int32_t E_max, const int32_t *b_lo, const int32_t *n,
+                  csla_stream_t stream);
+
 /* Static text for a status code. */
 const char *csla_strerror(int status);
 

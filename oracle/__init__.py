@@ -380,6 +380,9 @@ def num_threads():
 
 
 # ---------------------------------------------------------------- expected state after appends
+_encode_key_e4m3 = key_e4m3   # the flag argument below shadows the name
+
+
 def expected_append(raw_kv, raw_idx, L0, L1, m, gamma_kv, wg, gb, wgi=None, gbi=None, eps=1e-6,
                     theta=10000.0, d_rope=64, window_from=0, key_e4m3=False, per_channel=False):
     """Rows the state and classical caches must hold after tokens L0..L1-1 of a
@@ -406,7 +409,7 @@ def expected_append(raw_kv, raw_idx, L0, L1, m, gamma_kv, wg, gb, wgi=None, gbi=
             xi = raw_idx[b * m:(b + 1) * m]
             if per_channel:
                 c = gate_pool_channel(xi, wgi, gbi)
-                out["keys"][b] = key_e4m3(c) if key_e4m3 else key_bf16(c)
+                out["keys"][b] = _encode_key_e4m3(c) if key_e4m3 else key_bf16(c)
             else:
                 out["keys"][b] = index_key_e4m3(xi, wgi, gbi) if key_e4m3 else index_key(xi, wgi, gbi)
     return out

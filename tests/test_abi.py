@@ -137,3 +137,31 @@ def test_host_checks_of_the_query_row_and_step_calls():
     tail = [fake, C.CSLA_BF16, fake, fake, fake, C.CSLA_F32, 0, fake, 1 << 20, fake, 1 << 20, None]
     assert L.csla_csa_decode_step(ctypes.byref(_cfg(m=128)), *args, fake, *tail) == C.CSLA_ERR_UNSUPPORTED
     assert L.csla_csa_decode_step(ctypes.byref(cfg), *args, None, *tail) == C.CSLA_ERR_ARG
+
+
+def test_cp_record_size_and_host_checks():
+    """Context-parallel entry records: size per the header's layout, and the
+    arguments the host rejects before any launch."""
+    from compressed_sparse_long_append_b200 import csla as C
+    L = C._lib
+    fake = 1 << 40
+    # row 576 + bf16 key 256 + 8 -> 848; HCA row 576 + 8 -> 592; E4M3 key 128 -> 720
+    assert C.csla_cp_record_bytes(_cfg(m=4)) == 848
+    assert C.csla_cp_record_bytes(_cfg(m=128)) == 592
+    assert C.csla_cp_record_bytes(_cfg(m=4, key_fmt=C.CSLA_KEY_E4M3)) == 720
+    assert C.csla_cp_record_bytes(_cfg(m=4, D=128, dI=64)) == 192 + 128 + 16
+    cfg = _cfg(m=4)
+    st = C.csla_state(fake, fake, fake, fake, fake, 4)
+    cache = C.csla_cache(fake, fake, fake, fake, 8, 16)
+    arr = ctypes.c_int32 * 2
+    sel = lambda slot, n, e, recs: L.csla_cp_select(ctypes.byref(cfg), ctypes.byref(st), ctypes.byref(cache), slot,
+                                                    0, n, e, recs, None)
+    assert sel(4, 1, 1, fake) == C.CSLA_ERR_ARG          # slot beyond the state's slots
+    assert sel(0, 2, 1, fake) == C.CSLA_ERR_ARG          # more records than the run holds
+    assert sel(0, 1, 1, fake + 8) == C.CSLA_ERR_ARG      # misaligned records
+    place = lambda R, b, n: L.csla_cp_place(ctypes.byref(cfg), ctypes.byref(st), ctypes.byref(cache), 0, fake, R,
+                                            4, b, n, None)
+    assert place(C.CSLA_CP_MAX_RANKS + 1, arr(0, 0), arr(1, 1)) == C.CSLA_ERR_ARG
+    assert place(2, arr(0, -1), arr(1, 1)) == C.CSLA_ERR_ARG
+    assert place(2, arr(0, 4), arr(1, 5)) == C.CSLA_ERR_ARG
+    assert place(2, None, arr(1, 1)) == C.CSLA_ERR_ARG
