@@ -59,9 +59,11 @@ def upload_layer(w: Workload, cv, lens):
     return lb
 
 
-def fill_layer(lb: LayerBuffers, w: Workload, cv, lens):
+def fill_layer(lb: LayerBuffers, w: Workload, cv, lens, stream_ids=None):
     """Copy an oracle-built cache into existing layer buffers (the block
-    table too: with a table shared by several layers it must be the same)."""
+    table too: with a table shared by several layers it must be the same),
+    and put the raw rows of every request's open block into the tail, so
+    that the next appends close blocks from the right rows."""
     lb.rows.copy_(torch.from_numpy(cv.rows))
     lb.scales.copy_(torch.from_numpy(cv.scales))
     if w.is_csa and cv.kscale is not None:
@@ -73,6 +75,13 @@ def fill_layer(lb: LayerBuffers, w: Workload, cv, lens):
     lb.win_rows.copy_(torch.from_numpy(cv.win_rows))
     lb.win_scales.copy_(torch.from_numpy(cv.win_scales))
     lb.len.copy_(torch.tensor(list(lens), dtype=torch.int32))
+    for slot, L in enumerate(lens):
+        n = int(L) % w.m
+        if n:
+            ts = token_stream(w, slot if stream_ids is None else stream_ids[slot], int(L) - n, int(L))
+            lb.tail_kv[slot, :n] = torch.from_numpy(ts["kv"].astype(np.float32))
+            if w.is_csa:
+                lb.tail_idx[slot, :n] = torch.from_numpy(ts["idx"].astype(np.float32))
     torch.cuda.synchronize()
 
 

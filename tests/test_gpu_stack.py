@@ -100,12 +100,15 @@ def test_interleaved_stack_on_one_block_table():
             cv, p = oracle_cache(w, lens, bt=bt)
             got = st["out"].cpu().numpy().astype(np.float64)
             assert np.all(np.isfinite(got)), (step, i)
-            if w.is_csa:
-                check_csa_step(w, cv, p, si, lens, st["idx"].cpu().numpy(), got)
-            else:
-                ref = oracle.hca_decode(cv, np.arange(B), lens, si["q"][:B], p["gamma_q"], p["sink"], w.eps,
-                                        w.theta)
-                for s in range(B):
-                    check_out(got[s], ref[s])
+            try:
+                if w.is_csa:
+                    check_csa_step(w, cv, p, si, lens, st["idx"].cpu().numpy(), got)
+                else:
+                    ref = oracle.hca_decode(cv, np.arange(B), lens, si["q"][:B], p["gamma_q"], p["sink"], w.eps,
+                                            w.theta)
+                    for s in range(B):
+                        check_out(got[s], ref[s])
+            except AssertionError as e:
+                raise AssertionError("step %d layer %d (%s): %s" % (step, i, w.name, e)) from None
     # the table itself is only read
     assert np.array_equal(stack.block_table.cpu().numpy(), bt)
