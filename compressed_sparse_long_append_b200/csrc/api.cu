@@ -278,6 +278,8 @@ int csla_window_rows(const csla_cfg *cfg, const csla_state *st, const int32_t *s
 struct IndexerLaunch {
     IndexerArgs a;
     CUtensorMap kmap, qmap;
+    ProjMaps pm;
+    bool gemm;   // the projection runs on the tensor cores (bf16 cq and W_iq)
     bool cq_bf16, w_bf16;
 };
 
@@ -317,6 +319,10 @@ static int prep_indexer(const csla_cfg *cfg, const csla_state *st, const csla_ca
     L->qmap = qmap;
     L->cq_bf16 = cq_dtype == CSLA_BF16;
     L->w_bf16 = w_dtype == CSLA_BF16;
+    L->gemm = L->cq_bf16 && L->w_bf16;
+    if (L->gemm && (!encode_bf16_2d(&L->pm.cq, cq, (uint64_t)cfg->dc, (uint64_t)B, 128) ||
+                    !encode_bf16_2d(&L->pm.w, W_iq, (uint64_t)cfg->dc, (uint64_t)cfg->HI * cfg->dI, 64)))
+        return CSLA_ERR_CUDA;
     IndexerArgs a{};
     a.m = cfg->m; a.HI = cfg->HI; a.dI = cfg->dI; a.dc = cfg->dc; a.NQ = NQ;
     a.slots = slots; a.len = st->len; a.block_table = cache->block_table; a.bt_stride = cache->bt_stride;
@@ -345,7 +351,7 @@ int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_ca
                                 scores_stride, workspace, workspace_bytes, &L);
     if (rc) return rc;
     return cuda_status(launch_indexer(L.a, L.cq_bf16, L.w_bf16, L.kmap, L.qmap, num_sms_current(),
-                                      reinterpret_cast<cudaStream_t>(stream)));
+                                      reinterpret_cast<cudaStream_t>(stream), true, L.gemm ? &L.pm : nullptr));
 }
 
 static int prep_topk(const csla_cfg *cfg, const csla_state *st, const int32_t *slots, int32_t B,
@@ -521,7 +527,8 @@ int csla_csa_decode_step(const csla_cfg *cfg, const csla_state *st, const csla_c
         // invalidate a stream capture), and the first error is returned
         e = launch_compress_append(ca, kv_dtype == CSLA_BF16, side->s);
         cudaError_t ej = cudaEventRecord(side->join, side->s);
-        if (e == cudaSuccess) e = launch_indexer(old_a, il.cq_bf16, il.w_bf16, il.kmap, il.qmap, num_sms_current(), s);
+        if (e == cudaSuccess) e = launch_indexer(old_a, il.cq_bf16, il.w_bf16, il.kmap, il.qmap, num_sms_current(), s, true,
+                                                 il.gemm ? &il.pm : nullptr);
         if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, side->join, 0);
         if (e == cudaSuccess) e = ej;
     }

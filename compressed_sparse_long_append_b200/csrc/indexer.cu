@@ -638,6 +638,157 @@ __global__ void __launch_bounds__(256) len_snapshot_kernel(const int32_t *slots,
     len0[b] = (slot >= 0 && slot < n_slots) ? len[slot] : 0;
 }
 
+// ---- index-query projection on the tensor cores (bf16 cq and W_iq)
+//
+// q_I = cq . W_iq^T as a tcgen05 GEMM: a CTA owns 128 query rows x 64
+// output features; warp 0 streams 64-column (128-byte) slabs of both
+// operands by TMA into a 4-stage ring (128-byte swizzle, K-major), warp 1
+// issues one M=128 N=64 K=16 bf16 MMA per 32 bytes of a slab into a 64-column
+// fp32 TMEM accumulator, warps 2-5 read it back (one row per thread) and
+// store each value as its three bf16 terms (hi, mid, lo: their fp32 sum is
+// the value) in the workspace.  Every output is one accumulation over the
+// slabs in order: the same arithmetic whatever the batch.  Slabs past dc
+// and rows past B read as zeros (TMA fill).  The loads and products come
+// before the grid-dependency wait (cq and W_iq are inputs of the call);
+// the stores follow it.
+constexpr int kGemmBM = 128, kGemmBN = 64, kGemmStages = 4, kGemmThreads = 192;
+constexpr int kGemmABytes = kGemmBM * 128, kGemmBBytes = kGemmBN * 128;
+constexpr int kGemmSmem = 1024 + kGemmStages * (kGemmABytes + kGemmBBytes) + 256;
+
+__global__ void __launch_bounds__(kGemmThreads) iq_gemm_kernel(IndexerArgs a, const __grid_constant__ CUtensorMap cqmap,
+                                                                const __grid_constant__ CUtensorMap wmap) {
+    CSLA_TL_SCOPE(kTlIqProject);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *As = base;
+    uint8_t *Bs = base + kGemmStages * kGemmABytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(Bs + kGemmStages * kGemmBBytes);
+    uint64_t *empty = full + kGemmStages, *done = empty + kGemmStages;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(done + 1);
+    __shared__ volatile int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * kGemmBM, n0 = blockIdx.y * kGemmBN;
+    const int nk = (a.dc + 63) / 64;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        for (int s = 0; s < kGemmStages; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        mbar_init(done, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&cqmap);
+        tma_prefetch_desc(&wmap);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, 64);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    pdl_trigger();   // after the TMEM allocation (see indexer_kernel)
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int k = 0;
+            for (; k < nk; ++k) {
+                const int s = k % kGemmStages;
+                if (k >= kGemmStages && !mbar_wait(empty + s, ((k / kGemmStages) - 1) & 1, &abort_flag)) break;
+                mbar_arrive_expect_tx(full + s, (uint32_t)(kGemmABytes + kGemmBBytes));
+                tma_load_2d(As + s * kGemmABytes, &cqmap, k * 64, m0, full + s);
+                tma_load_2d(Bs + s * kGemmBBytes, &wmap, k * 64, n0, full + s);
+            }
+            // every issued copy must land before the CTA may exit
+            for (int i = (k > kGemmStages ? k - kGemmStages : 0); i < k; ++i)
+                mbar_wait(full + (i % kGemmStages), (i / kGemmStages) & 1, nullptr);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(kGemmBM, kGemmBN, false, false);
+            int k = 0;
+            for (; k < nk; ++k) {
+                const int s = k % kGemmStages;
+                if (!mbar_wait(full + s, (k / kGemmStages) & 1, &abort_flag)) break;
+                tc_fence_after();
+                const uint32_t ab = smem_u32(As + s * kGemmABytes), bb = smem_u32(Bs + s * kGemmBBytes);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_kind_f16(tmem, sdesc(ab + kk * 32, 16, 1024), sdesc(bb + kk * 32, 16, 1024), idesc,
+                                  (k | kk) > 0 ? 1u : 0u);
+                umma_commit(empty + s);
+            }
+            if (k == nk) umma_commit(done);
+            else abort_flag = 1;
+        }
+    } else {
+        const int lane_base = 32 * (warp & 3);
+        const int row = m0 + lane_base + lane;
+        const bool ok = warp_all(mbar_wait(done, 0, &abort_flag));
+        pdl_wait();
+        CSLA_TL_WAITED();
+        if (ok) {
+            tc_fence_after();
+            const int j = n0 / a.dI, e0 = n0 % a.dI;
+            uint16_t *dst = a.q_ws + (size_t)(row < a.B ? row : 0) * a.NQ * a.dI + (size_t)j * a.dI + e0;
+            const size_t tstride = (size_t)a.HI * a.dI;   // hi, mid, lo term rows are HI rows apart
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                uint32_t r[32];
+                tmem_ld32x32(tmem + ((uint32_t)lane_base << 16) + 32 * half, r);
+                tmem_wait_ld();
+                if (row < a.B) {
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        uint32_t h[4], md[4], lo[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            uint32_t hh[2], mm[2], ll[2];
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const float v = __uint_as_float(r[c8 * 8 + 2 * i + u]);
+                                const uint16_t vh = f32_to_bf16_bits(v);
+                                const float rem = __fsub_rn(v, bf16_bits_to_f32(vh));
+                                const uint16_t vm = f32_to_bf16_bits(rem);
+                                hh[u] = vh;
+                                mm[u] = vm;
+                                ll[u] = f32_to_bf16_bits(__fsub_rn(rem, bf16_bits_to_f32(vm)));
+                            }
+                            h[i] = hh[0] | (hh[1] << 16);
+                            md[i] = mm[0] | (mm[1] << 16);
+                            lo[i] = ll[0] | (ll[1] << 16);
+                        }
+                        uint16_t *o = dst + 32 * half + c8 * 8;
+                        *reinterpret_cast<uint4 *>(o) = make_uint4(h[0], h[1], h[2], h[3]);
+                        *reinterpret_cast<uint4 *>(o + tstride) = make_uint4(md[0], md[1], md[2], md[3]);
+                        *reinterpret_cast<uint4 *>(o + 2 * tstride) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 64);
+    }
+}
+
+cudaError_t launch_iq_gemm(const IndexerArgs &a, const ProjMaps &pm, cudaStream_t stream) {
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        cudaError_t e = cudaFuncSetAttribute(iq_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+        if (e != cudaSuccess) return e;
+        configured_dev = dev;
+    }
+    const dim3 grid((a.B + kGemmBM - 1) / kGemmBM, (a.HI * a.dI) / kGemmBN);
+    return launch_pdl(iq_gemm_kernel, grid, dim3(kGemmThreads), (size_t)kGemmSmem, stream, a, pm.cq, pm.w);
+}
+
 cudaError_t launch_scoring(const IndexerArgs &a, const CUtensorMap &kmap, const CUtensorMap &qmap,
                            cudaStream_t stream) {
     // HI is a template parameter so the epilogue's head loop is unrolled.
@@ -662,12 +813,18 @@ cudaError_t launch_scoring(const IndexerArgs &a, const CUtensorMap &kmap, const 
 }  // namespace
 
 cudaError_t launch_indexer(const IndexerArgs &a, bool cq_bf16, bool w_bf16, const CUtensorMap &kmap,
-                           const CUtensorMap &qmap, int num_sms, cudaStream_t stream, bool project) {
+                           const CUtensorMap &qmap, int num_sms, cudaStream_t stream, bool project,
+                           const ProjMaps *pm) {
     (void)num_sms;
     if (project) {
         if (a.NQ > 3 * a.HI) {
             cudaError_t e = cudaMemsetAsync(a.q_ws, 0, (size_t)a.B * a.NQ * a.dI * 2, stream);
             if (e != cudaSuccess) return e;
+        }
+        if (pm != nullptr && cq_bf16 && w_bf16) {
+            cudaError_t e = launch_iq_gemm(a, *pm, stream);
+            if (e != cudaSuccess) return e;
+            return launch_scoring(a, kmap, qmap, stream);
         }
         const int pblocks = (a.HI * a.dI + kProjThreads / 32 - 1) / (kProjThreads / 32);
         const dim3 pg(pblocks, (a.B + kProjKeepB - 1) / kProjKeepB), pb(kProjThreads);

@@ -122,8 +122,15 @@ cudaError_t launch_len_snapshot(const int32_t *slots, const int32_t *len, int B,
 // Query rows sharing one key tile per MMA when the rows of a call all belong
 // to one request: as many as fit the UMMA N limit of 256 columns.
 __host__ __device__ constexpr int indexer_rows_per_cta(int NQ) { return 256 / NQ; }
+// Tensor maps of the index-query projection on the tensor cores (bf16 cq
+// and W_iq): cq [B][dc] in 128-row boxes, W_iq [HI*dI][dc] in 64-row boxes,
+// 64 columns (128 bytes) per box, 128-byte swizzle.
+struct ProjMaps {
+    CUtensorMap cq, w;
+};
 cudaError_t launch_indexer(const IndexerArgs &a, bool cq_bf16, bool w_bf16, const CUtensorMap &kmap,
-                           const CUtensorMap &qmap, int num_sms, cudaStream_t stream, bool project = true);
+                           const CUtensorMap &qmap, int num_sms, cudaStream_t stream, bool project = true,
+                           const ProjMaps *pm = nullptr);
 
 struct TopkArgs {
     const float *scores;
