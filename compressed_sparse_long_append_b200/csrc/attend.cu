@@ -66,7 +66,12 @@ constexpr int kTile = 32;        // rows per tile
 constexpr int kRowsPerWarp = kTile / kLoadWarps;                // 4 rows of each tile per loader warp
 constexpr int kRing = 16;        // tiles of resolved row addresses
 constexpr int kAhead = 8;        // tiles resolved before the first conversion
-constexpr int kNR = 4;           // raw-row buffers (tiles of bulk copies in flight)
+constexpr int kNR = 2;           // raw-row buffers (tiles of bulk copies in flight)
+// X' buffers.  Converting tile t needs X'[t % kNX] back from the PV of tile
+// t - kNX; with two buffers that PV is issued only after S of tile t - 1, so
+// every conversion waited on the tensor cores and softmax of the tile before
+// (half of a loader's time); with three the conversions run back to back.
+constexpr int kNX = 3;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThresh = 4.0f;
 constexpr float kRopeMax = 32768.0f;   // largest |X'| taken for a RoPE dim at the row's own scale
@@ -92,10 +97,10 @@ struct Cfg {
     static constexpr int kColS = 0, kColO = 2 * kTile;
     static constexpr int kTmemCols = (kColO + 64 * kMB) <= 128 ? 128 : ((kColO + 64 * kMB) <= 256 ? 256 : 512);
     // smem offsets (from a 1024-aligned base); q is staged from X'[0] on at
-    // the start (into the raw buffers too when it is larger than both X')
+    // the start (into the raw buffers too when it is larger than the X' buffers)
     static constexpr int kOffQ = 0;
-    static constexpr int kOffX = kOffQ + kQBytes;      // X'[0], X'[1]
-    static constexpr int kOffRaw = kOffX + 2 * kXBytes;
+    static constexpr int kOffX = kOffQ + kQBytes;      // X'[0 .. kNX)
+    static constexpr int kOffRaw = kOffX + kNX * kXBytes;
     static constexpr int kOffP = kOffRaw + kNR * kRawBytes;
     static constexpr int kOffMisc = kOffP + kPBytes;
 };
@@ -104,14 +109,14 @@ struct Cfg {
 enum : uint8_t { kLocNone = 0, kLocCache = 1, kLocRing = 2, kLocSrc = 3 };
 
 struct Misc {
-    float tscale[2][kTile];            // per X' buffer: 256 * effective fp8 scale of each row (0 = masked)
+    float tscale[kNX][kTile];          // per X' buffer: 256 * effective fp8 scale of each row (0 = masked)
     float fac[2][kHP];                 // per tile parity: O^T column factors (1 = none)
     // loader ring, per tile slot (t % kRing) and row of the tile
     int ent[kRing][kTile];             // stage 1: compressed entry index (or the set row for window rows)
     uint32_t loc[kRing][kTile];        // stage 2: row index in its array
     float scl[kRing][kTile];           // stage 3: fp8 scale (0 = masked)
     uint8_t kind[kRing][kTile];        // stage 2: kLoc*
-    uint64_t q_staged, q_ready, x_full[2], x_empty[2], s_full[2], s_free[2], p_full, pv_done, o_free, fac_ready,
+    uint64_t q_staged, q_ready, x_full[kNX], x_empty[kNX], s_full[2], s_free[2], p_full, pv_done, o_free, fac_ready,
         drain, raw_full[kLoadWarps][kNR];   // raw_full[w][j]: warp w's rows of raw buffer j landed
     uint32_t tmem;
     int abort;
@@ -595,10 +600,10 @@ __device__ __forceinline__ bool loader_step(const AttendArgs &a, const Req &rq, 
         __syncwarp();
     }
     rr = resolve_issue(a, rq, L, t + kAhead, ms);
-    const int buf = t & 1;
+    const int buf = t % kNX;
     if (!warp_all(mbar_wait(&ms->raw_full[L.lw][t % kNR], (t / kNR) & 1, &ms->abort))) return false;
     *landed = t;
-    if (t >= 2 && !warp_all(mbar_wait(&ms->x_empty[buf], ((t - 2) >> 1) & 1, &ms->abort))) return false;
+    if (t >= kNX && !warp_all(mbar_wait(&ms->x_empty[buf], ((t - kNX) / kNX) & 1, &ms->abort))) return false;
     const uint8_t *raw = smem + C::kOffRaw + (t % kNR) * C::kRawBytes;
     uint8_t *xs = smem + C::kOffX + buf * C::kXBytes;
     const uint32_t wide = convert_rows<D>(L, t, raw, xs, ms, buf);
@@ -697,11 +702,11 @@ __device__ void mma_role(const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
     for (int g = 0; g <= n_tiles; ++g) {
         if (g < n_tiles) {
             // S[g & 1] = Qhat . X'[g & 1]^T
-            const int sb = g & 1;
-            if (!mbar_wait(&ms->x_full[sb], (g >> 1) & 1, &ms->abort)) return;
+            const int sb = g & 1, xg = g % kNX;
+            if (!mbar_wait(&ms->x_full[xg], (g / kNX) & 1, &ms->abort)) return;
             if (g >= 2 && !mbar_wait(&ms->s_free[sb], ((g - 2) >> 1) & 1, &ms->abort)) return;
             tc_fence_after();
-            const uint32_t x0 = smem_u32(smem + C::kOffX + sb * C::kXBytes);
+            const uint32_t x0 = smem_u32(smem + C::kOffX + xg * C::kXBytes);
 #pragma unroll 1
             for (int kb = 0; kb < C::kKB; ++kb)
 #pragma unroll
@@ -713,7 +718,7 @@ __device__ void mma_role(const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
         }
         if (g >= 1) {
             // O^T += X'[h & 1]^T . P^T for tile h = g - 1
-            const int h = g - 1, xb = h & 1;
+            const int h = g - 1, xb = h % kNX;
             const int ti = h % tpc, c = h / tpc;
             if (!mbar_wait(&ms->p_full, h & 1, &ms->abort)) return;
             if (ti == 0 && c > 0 && !mbar_wait(&ms->o_free, (c - 1) & 1, &ms->abort)) return;
@@ -751,11 +756,11 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
         const int hi = min(rq.n_rows, lo + rq.chunk);
         float m_run = -INFINITY, l_run = 0.f;
         for (int r0 = lo, ti = 0; r0 < hi; r0 += kTile, ++ti, ++g) {
-            const int sb = g & 1;
-            if (!warp_all(mbar_wait(&ms->x_full[sb], (g >> 1) & 1, &ms->abort))) return;
+            const int sb = g & 1, xg = g % kNX;
+            if (!warp_all(mbar_wait(&ms->x_full[xg], (g / kNX) & 1, &ms->abort))) return;
             if (!warp_all(mbar_wait(&ms->s_full[sb], (g >> 1) & 1, &ms->abort))) return;
             tc_fence_after();
-            const float4 *ts4 = reinterpret_cast<const float4 *>(ms->tscale[sb]);
+            const float4 *ts4 = reinterpret_cast<const float4 *>(ms->tscale[xg]);
             float s[kTile];
             float mt = -INFINITY;
             {
@@ -940,20 +945,22 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int q
     Misc *ms = reinterpret_cast<Misc *>(smem + C::kOffMisc);
     const int b = kSaturated ? blockIdx.x : blockIdx.y;
     const int warp = threadIdx.x >> 5;
-    // q of request b is staged from X'[0] on: in the two X' buffers (bf16 q
-    // of up to 64 heads fills them exactly), reaching into the raw buffers
-    // for f32 q
+    // q of request b is staged from X'[0] on: in the X' buffers (bf16 q of
+    // up to 64 heads fills two of them), reaching into the raw buffers for
+    // f32 q
     const uint32_t q_bytes = (uint32_t)(a.H * D * (q_bf16 ? 2 : 4));
     uint8_t *stage = smem + C::kOffX;
-    const bool q_in_raw = q_bytes > (uint32_t)(2 * C::kXBytes);
+    const bool q_in_raw = q_bytes > (uint32_t)(kNX * C::kXBytes);
 
     // ---- before the wait: barriers, TMEM, the q copy
     if (threadIdx.x == 0) {
         mbar_init(&ms->q_staged, 1);
         mbar_init(&ms->q_ready, kSoftWarps);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kNX; ++i) {
             mbar_init(&ms->x_full[i], kLoadWarps);
             mbar_init(&ms->x_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&ms->s_full[i], 1);
             mbar_init(&ms->s_free[i], kSoftWarps);
         }
