@@ -72,6 +72,10 @@ constexpr int kNR = 2;           // raw-row buffers (tiles of bulk copies in fli
 // every conversion waited on the tensor cores and softmax of the tile before
 // (half of a loader's time); with three the conversions run back to back.
 constexpr int kNX = 3;
+// X' buffer of tile t.  q is staged from X'[0] on, so tile 0 goes to the last
+// buffer: when q fits in the first two, tile 0 is converted while Qhat is
+// still being built.
+__device__ __forceinline__ int xbuf(int t) { return (t + kNX - 1) % kNX; }
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThresh = 4.0f;
 constexpr float kRopeMax = 32768.0f;   // largest |X'| taken for a RoPE dim at the row's own scale
@@ -600,7 +604,7 @@ __device__ __forceinline__ bool loader_step(const AttendArgs &a, const Req &rq, 
         __syncwarp();
     }
     rr = resolve_issue(a, rq, L, t + kAhead, ms);
-    const int buf = t % kNX;
+    const int buf = xbuf(t);
     if (!warp_all(mbar_wait(&ms->raw_full[L.lw][t % kNR], (t / kNR) & 1, &ms->abort))) return false;
     *landed = t;
     if (t >= kNX && !warp_all(mbar_wait(&ms->x_empty[buf], ((t - kNX) / kNX) & 1, &ms->abort))) return false;
@@ -619,9 +623,12 @@ __device__ __forceinline__ bool loader_step(const AttendArgs &a, const Req &rq, 
     return true;
 }
 
+// q_in_raw: q is staged into the raw buffers too (copies wait for Qhat);
+// q_in_two: q fits in X'[0] and X'[1], so tile 0 (X'[kNX-1]) may be
+// converted before Qhat is built.
 template <int D>
 __device__ void loader_role(const AttendArgs &a, int b, const Req &rq, Span sp, uint8_t *smem, Misc *ms,
-                            bool q_in_raw) {
+                            bool q_in_raw, bool q_in_two) {
     LoadCtx L;
     L.b = b;
     L.lw = (threadIdx.x >> 5) - kSoftWarps;
@@ -673,10 +680,13 @@ __device__ void loader_role(const AttendArgs &a, int b, const Req &rq, Span sp, 
         issue_rows<D>(a, L, t, smem, ms);
         issued = t;
     }
-    // q is staged in the X' buffers: convert only once Qhat is built
-    if (warp_all(mbar_wait(&ms->q_ready, 0, &ms->abort))) {
-        ResolveRegs rr;
-        for (int t = 0; t < L.n_tiles; ++t)
+    // q is staged in the X' buffers: convert into them only once Qhat is built
+    ResolveRegs rr;
+    int t = 0;
+    bool ok = true;
+    if (q_in_two && !q_in_raw) ok = loader_step<D>(a, rq, L, t++, smem, ms, rr, &landed, &issued);
+    if (ok && warp_all(mbar_wait(&ms->q_ready, 0, &ms->abort))) {
+        for (; t < L.n_tiles; ++t)
             if (!loader_step<D>(a, rq, L, t, smem, ms, rr, &landed, &issued)) break;
     }
     // copies this warp started but has not seen land (only after an abort)
@@ -702,7 +712,7 @@ __device__ void mma_role(const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
     for (int g = 0; g <= n_tiles; ++g) {
         if (g < n_tiles) {
             // S[g & 1] = Qhat . X'[g & 1]^T
-            const int sb = g & 1, xg = g % kNX;
+            const int sb = g & 1, xg = xbuf(g);
             if (!mbar_wait(&ms->x_full[xg], (g / kNX) & 1, &ms->abort)) return;
             if (g >= 2 && !mbar_wait(&ms->s_free[sb], ((g - 2) >> 1) & 1, &ms->abort)) return;
             tc_fence_after();
@@ -718,7 +728,7 @@ __device__ void mma_role(const Req &rq, Span sp, uint8_t *smem, Misc *ms) {
         }
         if (g >= 1) {
             // O^T += X'[h & 1]^T . P^T for tile h = g - 1
-            const int h = g - 1, xb = h % kNX;
+            const int h = g - 1, xb = xbuf(h);
             const int ti = h % tpc, c = h / tpc;
             if (!mbar_wait(&ms->p_full, h & 1, &ms->abort)) return;
             if (ti == 0 && c > 0 && !mbar_wait(&ms->o_free, (c - 1) & 1, &ms->abort)) return;
@@ -756,7 +766,7 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
         const int hi = min(rq.n_rows, lo + rq.chunk);
         float m_run = -INFINITY, l_run = 0.f;
         for (int r0 = lo, ti = 0; r0 < hi; r0 += kTile, ++ti, ++g) {
-            const int sb = g & 1, xg = g % kNX;
+            const int sb = g & 1, xg = xbuf(g);
             if (!warp_all(mbar_wait(&ms->x_full[xg], (g / kNX) & 1, &ms->abort))) return;
             if (!warp_all(mbar_wait(&ms->s_full[sb], (g >> 1) & 1, &ms->abort))) return;
             tc_fence_after();
@@ -1007,7 +1017,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int q
             softmax_role<D>(a, b, rq, sp, smem, ms);
         }
     } else if (warp < kSoftWarps + kLoadWarps) {
-        loader_role<D>(a, b, rq, sp, smem, ms, q_in_raw);
+        loader_role<D>(a, b, rq, sp, smem, ms, q_in_raw, q_bytes <= (uint32_t)(2 * C::kXBytes));
     } else if ((threadIdx.x & 31) == 0) {
         mma_role<D>(rq, sp, smem, ms);
     }

@@ -186,12 +186,14 @@ cudaError_t launch_attend(const AttendArgs &a, bool q_bf16, bool out_bf16, int v
 
 // Canonical chunk length for a set of n rows (a function of n only):
 // 64 * ceil(n / 2048) rows, so a request never has more than 32 chunks, and
-// at least 128 rows once n > 1024 (top-k 1024 + window: 9 chunks, not 18 —
-// every chunk costs an H*D fp32 partial written and read back).
+// 320 rows for 1024 < n <= 4096 (top-k 1024 + window: 4 chunks, not 18 --
+// every chunk costs an H*D fp32 partial written and read back, which is
+// most of a query row's time when thousands of rows fill the GPU; decode at
+// top-k 512 keeps 64-row chunks, which spread few requests over the SMs).
 __host__ __device__ inline int attend_chunk_rows(long long n) {
     long long c = (n + 2047) / 2048;
     if (c < 1) c = 1;
-    if (n > 1024 && c < 2) c = 2;
+    if (n > 1024 && n <= 4096) c = 5;
     return (int)(64 * c);
 }
 __host__ __device__ inline int attend_num_chunks(long long n) {

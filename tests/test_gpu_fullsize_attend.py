@@ -136,9 +136,8 @@ def test_hca_full_size_matches_oracle():
 def test_csa_query_rows_full_topk_match_oracle(k):
     """Query rows of one request with per-row visible lengths, top-k lists of
     k entries (seeded subsets of each row's visible entries) and window rows
-    from a buffer indexed by position: k + 128 rows per set (chunks of at
-    least 128 rows), both variants bit-identical, every row against the
-    oracle."""
+    from a buffer indexed by position: k + 128 rows per set (320-row
+    chunks), both variants bit-identical, every row against the oracle."""
     seed = 4
     L1 = 4 * k + 3000
     cv, lb = _filled(4, [L1], seed)
