@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true", help="skip the CSA prefill-chunk measurement")
     ap.add_argument("--prefill-only", action="store_true", help="only the CSA prefill-chunk measurement")
     ap.add_argument("--no-e4m3", action="store_true", help="skip the CSA decode leg with E4M3 index keys")
+    ap.add_argument("--hca-only", action="store_true", help="only the HCA decode measurement")
+    ap.add_argument("--e4m3-only", action="store_true", help="only the CSA decode leg with E4M3 index keys")
     ap.add_argument("--no-invariance", action="store_true",
                     help="skip the ragged 64-request CSA + HCA decode measurement")
     ap.add_argument("--no-stack", action="store_true",
@@ -63,8 +65,10 @@ def parse():
     ap.add_argument("--fused-step", action="store_true",
                     help="time the CSA step as csla_csa_decode_step instead of the four separate library calls")
     ap.add_argument("--profile", action="store_true",
-                    help="only the timed CSA steps, bracketed by cudaProfilerStart/Stop (for ncu "
-                         "--profile-from-start off); implies --no-hca --no-cpu-baseline and no e2e leg")
+                    help="only the timed steps of the first leg run (CSA decode; the prefill chunk with "
+                         "--prefill-only; the HCA step with --hca-only; the E4M3-key CSA step with --e4m3-only), "
+                         "bracketed by cudaProfilerStart/Stop (for ncu --profile-from-start off); implies "
+                         "--no-hca --no-cpu-baseline and no e2e leg")
     return ap.parse_args()
 
 
@@ -462,7 +466,37 @@ def prefill_leg(W, K, seed, rank, world, device, variant, profile=False):
     return out
 
 
-def e4m3_leg(W, K, seed, rank, world, device, variant):
+def hca_leg(W, K, seed, rank, world, device, variant, peak, profile=False):
+    """The HCA layer decode step: 4 requests at 2^20 tokens."""
+    import torch
+    hk = dict(HCA)
+    HR, hm, hB = HCA_COPIES, hk["m"], hk["B"]
+    # requests staggered 16 tokens apart inside one block, clear of its end:
+    # with fewer than ~78 appends per copy no block closes during the run
+    # (in steady decode one closes every 128 steps per request)
+    hL0s = [hk["L"] - 127 + 16 * b for b in range(hB)]
+    closes = sum(1 for i in range(W, W + K) for b in range(hB) if (hL0s[b] + i // HR + 1) % hm == 0)
+    hlb, hcp, hparams = build_layer(hk, hB, hL0s, seed, rank, device)
+    hin = step_inputs(hk, hB, W + K, seed, rank, device)
+    hsteps = make_copies(HcaStep, hlb, hcp, hparams, hk, variant, device, HR)
+    hms = dp_max(run_steps(hsteps, hin, W, K, profile=profile), world, device)
+    out = {"workload": "hca_decode_B4_L1048576", "tokens_per_s": hB * world / (hms * 1e-3), "ms_per_step": hms,
+           "block_closes_in_timed_steps": closes}
+    if not profile:
+        hms_att = dp_max(call_time(hsteps, hin, W, K, 1), world, device)
+        rows = sum(int(x) // hm for x in hsteps[0].lb.len.tolist()) / hB + hk["n_win"]
+        hbytes = hB * (rows * (hk["D"] + 64 + 4) + 2 * hk["H"] * hk["D"] * 2)
+        hflops = hB * rows * hk["H"] * hk["D"] * 4
+        out.update({"attend_ms": hms_att, "attend_hbm_gbs": hbytes / (hms_att * 1e-3) / 1e9,
+                    "attend_hbm_frac": hbytes / (hms_att * 1e-3) / 1e9 / peak,
+                    "attend_tflops": hflops / (hms_att * 1e-3) / 1e12,
+                    "attend_tensor_frac_sustained": hflops / (hms_att * 1e-3) / 1e12 / 1395.7})
+    del hsteps, hlb, hin
+    torch.cuda.empty_cache()
+    return out
+
+
+def e4m3_leg(W, K, seed, rank, world, device, variant, profile=False):
     """The headline CSA decode workload (8 x 131072, top-k 512) with its index
     keys stored as E4M3 codes plus one power-of-two scale per entry (132
     instead of 256 bytes per entry): the same step, timed the same way, and
@@ -477,7 +511,10 @@ def e4m3_leg(W, K, seed, rank, world, device, variant):
     CsaStep.fused = False
     steps = make_copies(CsaStep, lb, cp, params, kw, variant, device, R)
     torch.cuda.synchronize()
-    ms = dp_max(run_steps(steps, inputs, W, K), world, device)
+    ms = dp_max(run_steps(steps, inputs, W, K, profile=profile), world, device)
+    if profile:
+        return {"workload": "csa_decode_B8_L131072_e4m3_keys", "tokens_per_s": B * world / (ms * 1e-3),
+                "ms_per_step": ms}
     seg = breakdown(steps, inputs, W, K)
     ms_idx = call_time(steps, inputs, W, K, 1)
     nv = sum(int(x) // m for st in steps for x in st.lb.len.tolist()) / R
@@ -783,9 +820,12 @@ def indexer_traffic():
 
 # ------------------------------------------------------------------ CPU oracle baseline
 def cpu_baseline(n_steps=3):
-    """fp64 oracle on one request of the CSA workload (bounded sample): the
-    oracle builds that request's cache from the seeded raw stream, then runs
-    whole decode steps (indexer -> top-k -> attention) on it."""
+    """fp64 oracle on the CSA workload (bounded sample): the oracle builds
+    one request's cache from the seeded raw stream, then runs whole decode
+    steps (indexer -> top-k -> attention) for as many requests as the host
+    has oracle threads (every request reads that one cache, each with its
+    own query inputs; the oracle runs requests in parallel).  Returns
+    (seconds per step, requests per step)."""
     import numpy as np
     import oracle
     import torch
@@ -817,19 +857,21 @@ def cpu_baseline(n_steps=3):
     wsc = np.zeros((1, 128), np.float32)
     for p in range(L - 128, L):
         win[0, p % 128], wsc[0, p % 128] = oracle.window_row(kv[p], gamma_kv, p)
-    cv = oracle.CacheView(m, D, rows, scales, bt, win, wsc, kidx, dI)
+    nreq = max(1, oracle.num_threads())
+    cv = oracle.CacheView(m, D, rows, scales, np.repeat(bt, nreq, axis=0), np.repeat(win, nreq, axis=0),
+                          np.repeat(wsc, nreq, axis=0), kidx, dI)
     W = normal(seed, "W_iq_cpu", (kw["HI"] * dI, kw["dc"]), std=1.0 / kw["dc"] ** 0.5)
     sink = normal(seed, "sink", (kw["H"],))
     gq = 1.0 + 0.1 * normal(seed, "gamma_q", (D,))
     times = []
     for s in range(n_steps):
-        q = normal(seed, "cpu/q/%d" % s, (1, kw["H"], D))
-        cq = normal(seed, "cpu/cq/%d" % s, (1, kw["dc"]))
-        hw = normal(seed, "cpu/hw/%d" % s, (1, kw["HI"]))
+        q = normal(seed, "cpu/q/%d" % s, (nreq, kw["H"], D))
+        cq = normal(seed, "cpu/cq/%d" % s, (nreq, kw["dc"]))
+        hw = normal(seed, "cpu/hw/%d" % s, (nreq, kw["HI"]))
         t0 = time.perf_counter()
-        oracle.csa_decode(cv, [0], [L], q, gq, cq, W, hw, sink, kw["HI"], kw["k"])
+        oracle.csa_decode(cv, list(range(nreq)), [L] * nreq, q, gq, cq, W, hw, sink, kw["HI"], kw["k"])
         times.append(time.perf_counter() - t0)
-    return times
+    return times, nreq
 
 
 def _filled_cache(m, D, n_entries, L, seed, dI=0):
@@ -860,22 +902,27 @@ def _filled_cache(m, D, n_entries, L, seed, dI=0):
 
 
 def cpu_baseline_hca(n_steps=3):
-    """fp64 oracle decode steps of one request of the HCA workload (context
-    2^20 - 64: 8191 entries + 128 window rows per step); seconds per step."""
+    """fp64 oracle decode steps of the HCA workload (context 2^20 - 64: 8191
+    entries + 128 window rows per request and step), one request per oracle
+    thread, all reading one cache; (seconds per step, requests per step)."""
     import oracle
     from csla_synth import normal
     kw, seed = HCA, 2
     L = kw["L"] - 64
+    import numpy as np
     cv = _filled_cache(kw["m"], kw["D"], L // kw["m"], L, seed)
+    nreq = max(1, oracle.num_threads())
+    cv = oracle.CacheView(cv.m, cv.D, cv.rows, cv.scales, np.repeat(cv.block_table, nreq, axis=0),
+                          np.repeat(cv.win_rows, nreq, axis=0), np.repeat(cv.win_scales, nreq, axis=0), None, 0)
     sink = normal(seed, "sink", (kw["H"],))
     gq = 1.0 + 0.1 * normal(seed, "gamma_q", (kw["D"],))
     times = []
     for s_ in range(n_steps):
-        q = normal(seed, "cpu/q/%d" % s_, (1, kw["H"], kw["D"]))
+        q = normal(seed, "cpu/q/%d" % s_, (nreq, kw["H"], kw["D"]))
         t0 = time.perf_counter()
-        oracle.hca_decode(cv, [0], [L], q, gq, sink)
+        oracle.hca_decode(cv, list(range(nreq)), [L] * nreq, q, gq, sink)
         times.append(time.perf_counter() - t0)
-    return times
+    return times, nreq
 
 
 def cpu_baseline_prefill(n_q=16):
@@ -903,17 +950,18 @@ def cpu_baseline_prefill(n_q=16):
 
 def run_reference(args):
     t_setup = time.perf_counter()
-    times = cpu_baseline(n_steps=args.warmup + args.steps)
+    times, nreq = cpu_baseline(n_steps=args.warmup + args.steps)
     timed = times[args.warmup:]
     per_step = sum(timed) / len(timed)
-    value = 1.0 / per_step
-    sample = "1 request of the CSA workload (context 131072, 32768 entries, k=512), fp64 oracle"
+    value = nreq / per_step
+    sample = ("%d requests of the CSA workload per step (context 131072, 32768 entries, k=512; one oracle-built "
+              "cache read by all), fp64 oracle, one host thread per request" % nreq)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded splitmix64 / Box-Muller)",
-            "config": {"workload": "csa_decode_B8_L131072", "sample": "1 of 8 requests per step"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "config": {"workload": "csa_decode_B8_L131072", "sample": "%d requests per step" % nreq},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": nreq, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "setup_s": time.perf_counter() - t_setup}
     print(json.dumps(line), flush=True)
@@ -945,10 +993,18 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
     W, K = max(3, args.warmup), args.steps
     seed = 1
-    if args.prefill_only:
-        pre = prefill_leg(W, K, seed + 2, rank, world, device, args.variant, profile=args.profile)
+    if args.prefill_only or args.hca_only or args.e4m3_only:
+        if args.prefill_only:
+            key, res = "csa_prefill", prefill_leg(W, K, seed + 2, rank, world, device, args.variant,
+                                                  profile=args.profile)
+        elif args.hca_only:
+            key, res = "hca_decode", hca_leg(W, K, seed + 1, rank, world, device, args.variant, peaks()[0],
+                                             profile=args.profile)
+        else:
+            key, res = "csa_decode_e4m3_keys", e4m3_leg(W, K, seed, rank, world, device, args.variant,
+                                                        profile=args.profile)
         if rank == 0:
-            print(json.dumps({"csa_prefill": pre}), flush=True)
+            print(json.dumps({key: res}), flush=True)
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()
@@ -998,39 +1054,18 @@ def main():
     if not args.no_hca:
         del steps, lb
         torch.cuda.empty_cache()
-        hk = dict(HCA)
-        HR, hm, hB = HCA_COPIES, hk["m"], hk["B"]
-        # requests staggered 16 tokens apart inside one block, clear of its end:
-        # with fewer than ~78 appends per copy no block closes during the run
-        # (in steady decode one closes every 128 steps per request)
-        hL0s = [hk["L"] - 127 + 16 * b for b in range(hB)]
-        closes = sum(1 for i in range(W, W + K) for b in range(hB) if (hL0s[b] + i // HR + 1) % hm == 0)
-        hlb, hcp, hparams = build_layer(hk, hB, hL0s, seed + 1, rank, device)
-        hin = step_inputs(hk, hB, W + K, seed + 1, rank, device)
-        hsteps = make_copies(HcaStep, hlb, hcp, hparams, hk, args.variant, device, HR)
-        hms = run_steps(hsteps, hin, W, K)
-        hms_att = call_time(hsteps, hin, W, K, 1)
-        rows = sum(int(x) // hm for x in hsteps[0].lb.len.tolist()) / hB + hk["n_win"]
-        hbytes = hB * (rows * (hk["D"] + 64 + 4) + 2 * hk["H"] * hk["D"] * 2)
-        hflops = hB * rows * hk["H"] * hk["D"] * 4
-        hca = {"workload": "hca_decode_B4_L1048576", "tokens_per_s": hB / (hms * 1e-3),
-               "ms_per_step": hms, "attend_ms": hms_att,
-               "attend_hbm_gbs": hbytes / (hms_att * 1e-3) / 1e9,
-               "attend_hbm_frac": hbytes / (hms_att * 1e-3) / 1e9 / peak,
-               "attend_tflops": hflops / (hms_att * 1e-3) / 1e12,
-               "attend_tensor_frac_sustained": hflops / (hms_att * 1e-3) / 1e12 / 1395.7,
-               "block_closes_in_timed_steps": closes}
+        hca = hca_leg(W, K, seed + 1, rank, world, device, args.variant, peak)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             try:
-                ht = cpu_baseline_hca(3)
-                hca["cpu_baseline"] = {"value": 1.0 / (sum(ht) / len(ht)), "unit": UNIT, "cores": 1, "kind": "oracle",
-                                       "sample": "1 request of this workload (context 2^20 - 64, 8191 entries + "
-                                                 "128 window rows), 3 decode steps, fp64 oracle, single thread"}
+                ht, nreq = cpu_baseline_hca(3)
+                hca["cpu_baseline"] = {"value": nreq / (sum(ht) / len(ht)), "unit": UNIT, "cores": nreq,
+                                       "kind": "oracle",
+                                       "sample": "%d requests of this workload (context 2^20 - 64, 8191 entries + "
+                                                 "128 window rows; one cache read by all), 3 decode steps, fp64 "
+                                                 "oracle, one thread per request" % nreq}
             except Exception as e:  # the baseline never blocks the GPU line
                 hca["cpu_baseline"] = {"value": None, "unit": UNIT, "cores": 0, "kind": "oracle",
                                        "sample": "failed: %s" % e}
-        del hsteps, hlb, hin
-        torch.cuda.empty_cache()
 
     pre = None
     if not args.no_prefill and not args.profile:
@@ -1063,11 +1098,11 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         try:
-            ct = cpu_baseline(n_steps=3)
-            v = 1.0 / (sum(ct) / len(ct))
-            cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
-                   "sample": "1 request of this workload (context 131072, k=512), 3 decode steps, fp64 oracle, "
-                             "single thread"}
+            ct, nreq = cpu_baseline(n_steps=3)
+            v = nreq / (sum(ct) / len(ct))
+            cpu = {"value": v, "unit": UNIT, "cores": nreq, "kind": "oracle",
+                   "sample": "%d requests of this workload (context 131072, k=512; one oracle-built cache read "
+                             "by all), 3 decode steps, fp64 oracle, one thread per request" % nreq}
         except Exception as e:  # the baseline never blocks the GPU line
             cpu = {"value": None, "unit": UNIT, "cores": 0, "kind": "oracle", "sample": "failed: %s" % e}
 
