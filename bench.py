@@ -526,7 +526,8 @@ def e4m3_leg(W, K, seed, rank, world, device, variant, profile=False):
            "segments_ms": {"compress_append": seg[0], "indexer_scores": seg[1], "topk_select": seg[2],
                            "csa_attend": seg[3]},
            "indexer": {"call_ms": ms_idx, "algorithmic_bytes": idx_bytes, "achieved_gbs": achieved,
-                       "frac": achieved / peak, "peak": peak, "peak_kind": peak_kind}}
+                       "frac": achieved / peak, "peak": peak, "peak_kind": peak_kind,
+                       "traffic": indexer_traffic("csla_indexer_scores_e4m3")}}
     del steps, lb, inputs
     torch.cuda.empty_cache()
     return out
@@ -802,13 +803,13 @@ def call_time(steps, inputs, W, K, j):
     return e0.elapsed_time(e1) / K
 
 
-def indexer_traffic():
-    """DRAM bytes per indexer launch from the committed ncu summary, if it
-    was taken on the current kernel source (else None)."""
+def indexer_traffic(key="csla_indexer_scores"):
+    """DRAM bytes per indexer call from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            t = json.load(f)["csla_indexer_scores"]
+            t = json.load(f)[key]
         h = hashlib.sha256()
         for name in t["sources"]:
             with open(os.path.join(ROOT, name), "rb") as f:
