@@ -3,19 +3,17 @@
 //   硅星人 "DeepSeek V4 ... 让token大降价" §两大压缩注意力, CSA part: of all
 //   compressed blocks only the k most relevant (512; 1024 for Pro) are kept.
 //
-// One CTA of 1024 threads per request.  Scores become order-preserving
-// uint32 keys (-0.0 folded onto +0.0), staged in shared memory when the
-// request's visible entries fit (else re-read from global memory each pass).
-// The exact k-th largest key T is found by a radix select over 11/11/10 key
-// bits: each pass builds a histogram of the keys matching the prefix so far
-// (kCopies private copies, one per group of four warps, so that the
-// shared-memory atomics of different groups never contend: scores crowd
-// into few bins), sums the copies and picks the bin holding the remaining
-// rank.  The first pass's histogram is built while the keys are staged.  The
-// output pass keeps every key > T and the lowest-index keys == T: each warp
-// owns a contiguous range, per-warp counts give its first slot and ballots
-// place the picks, so indices come out ascending.  All counts are integers:
-// the selection is exact and independent of thread timing and batch.
+// Scores become order-preserving uint32 keys (-0.0 folded onto +0.0).  The
+// output is every key > T and the lowest-index keys == T, T the exact k-th
+// largest key, indices ascending: each warp owns a contiguous range (or the
+// candidates of one), per-warp counts give its first slot and ballots place
+// the picks.  All counts are integers: the selection is exact and
+// independent of thread timing and batch.  Two kernels: a cluster of four
+// CTAs per request with the scores in registers (up to 36864 visible
+// entries: decode), and one CTA per row streaming its scores (longer rows:
+// query rows of a long prefill).  Both find T among the candidates above a
+// sampled threshold, with a radix select over every key as the fallback.
+
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -26,195 +24,12 @@ namespace cg = cooperative_groups;
 namespace csla {
 namespace {
 
-constexpr int kThreads = 1024;
-constexpr int kWarps = kThreads / 32;
-constexpr int kCopies = 8;                    // histogram copies (4 warps each)
 constexpr int kBins = 2048;
-constexpr int kSmemKeysMax = 36864;           // keys per request staged in shared memory
-constexpr int kBatch = 16;                    // score loads a thread keeps in flight
-constexpr size_t kHistBytes = (size_t)kBins * kCopies * sizeof(int);
 
 __device__ __forceinline__ uint32_t score_key(float f) {
     uint32_t u = __float_as_uint(f);
     if (u == 0x80000000u) u = 0u;
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-struct Shared {
-    int hsum[kBins];           // summed histogram of the current pass
-    int warp_a[kWarps], warp_b[kWarps];
-    int sel_bin, sel_krem;
-};
-
-// Find the bin holding the krem-th largest key of hist[0..nb) (counted from
-// the top).  Result in sh->sel_bin / sh->sel_krem.  All threads call it.
-__device__ void pick_bin(Shared *sh, const int *hist, int nb, int krem) {
-    const int per = nb / kThreads;   // bins per thread, highest first
-    int c = 0;
-    for (int q = 0; q < per; ++q) c += hist[nb - 1 - (threadIdx.x * per + q)];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int v = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += t;
-    }
-    if (lane == 31) sh->warp_a[warp] = v;
-    __syncthreads();
-    int before = 0;
-    for (int w = 0; w < warp; ++w) before += sh->warp_a[w];
-    const int incl = v + before;
-    const int excl = incl - c;
-    if (excl < krem && krem <= incl) {
-        int run = excl;
-        for (int q = 0; q < per; ++q) {
-            const int bin = nb - 1 - (threadIdx.x * per + q);
-            const int h = hist[bin];
-            if (run + h >= krem) {
-                sh->sel_bin = bin;
-                sh->sel_krem = krem - run;
-                break;
-            }
-            run += h;
-        }
-    }
-    __syncthreads();
-}
-
-__device__ __forceinline__ void hist_zero(int *hist) {
-    int4 *p = reinterpret_cast<int4 *>(hist);
-    for (int i = threadIdx.x; i < kBins * kCopies / 4; i += kThreads) p[i] = make_int4(0, 0, 0, 0);
-}
-
-template <bool kSmemKeys>
-__global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
-    CSLA_TL_SCOPE(kTlTopk);
-    extern __shared__ __align__(16) int dyn[];
-    int *hist = dyn;                                                     // [kBins][kCopies]
-    uint32_t *keys_s = reinterpret_cast<uint32_t *>(dyn + kBins * kCopies);   // [n] when staged
-    __shared__ Shared sh;
-    pdl_trigger();
-    const int b = blockIdx.x;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int copy = warp & (kCopies - 1);
-    const int slot = __ldg(a.slots + b);
-    const bool slot_ok = slot >= 0 && slot < a.n_slots;
-    hist_zero(hist);
-    pdl_wait();
-    CSLA_TL_WAITED();
-    const int L = slot_ok ? row_visible_len(a.len, a.q_len, slot, b) : 0;
-    int n = L < 0 ? 0 : L / a.m;
-    if (!slot_ok || L < 0 || L / a.m > a.max_n) {
-        if (threadIdx.x == 0) set_dev_err(CSLA_DEVERR_LEN);
-        n = 0;
-    }
-    const int k = a.k;
-    int32_t *out = a.idx + (size_t)b * k;
-    const float *sc = a.scores + (size_t)b * a.stride;
-    if (n <= k) {
-        for (int j = threadIdx.x; j < k; j += kThreads) out[j] = j < n ? j : -1;
-        return;
-    }
-    auto key_at = [&](int i) -> uint32_t { return kSmemKeys ? keys_s[i] : score_key(__ldg(sc + i)); };
-    __syncthreads();   // zeroed histogram
-    if (kSmemKeys) {
-        // stage the keys (kBatch loads in flight per thread) and build the
-        // first pass's histogram (top 11 key bits) on the way
-        for (int i0 = 0; i0 < n; i0 += kThreads * kBatch) {
-            float f[kBatch];
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                const int i = i0 + u * kThreads + threadIdx.x;
-                f[u] = i < n ? sc[i] : 0.f;
-            }
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                const int i = i0 + u * kThreads + threadIdx.x;
-                if (i < n) {
-                    const uint32_t key = score_key(f[u]);
-                    keys_s[i] = key;
-                    atomicAdd(&hist[(key >> 21) * kCopies + copy], 1);
-                }
-            }
-            if (i0 == 0) CSLA_TL_MARK(5);
-        }
-    }
-    CSLA_TL_MARK(0);
-
-    uint32_t prefix = 0, pmask = 0;
-    int krem = k;
-    const int shifts[3] = {21, 10, 0};
-    const int widths[3] = {11, 11, 10};
-    for (int pass = 0; pass < 3; ++pass) {
-        const int shb = shifts[pass], nb = 1 << widths[pass];
-        if (pass > 0 || !kSmemKeys) {
-            if (pass > 0) {
-                hist_zero(hist);
-                __syncthreads();
-            }
-            for (int i = threadIdx.x; i < n; i += kThreads) {
-                const uint32_t key = key_at(i);
-                if ((key & pmask) == prefix) atomicAdd(&hist[((key >> shb) & (uint32_t)(nb - 1)) * kCopies + copy], 1);
-            }
-        }
-        __syncthreads();
-        for (int bin = threadIdx.x; bin < nb; bin += kThreads) {
-            const int4 *h4 = reinterpret_cast<const int4 *>(hist + bin * kCopies);
-            int t = 0;
-#pragma unroll
-            for (int j = 0; j < kCopies / 4; ++j) {
-                const int4 v = h4[j];
-                t += v.x + v.y + v.z + v.w;
-            }
-            sh.hsum[bin] = t;
-        }
-        __syncthreads();
-        pick_bin(&sh, sh.hsum, nb, krem);
-        prefix |= (uint32_t)sh.sel_bin << shb;
-        pmask |= (uint32_t)(nb - 1) << shb;
-        krem = sh.sel_krem;
-        CSLA_TL_MARK(1 + pass);
-    }
-    // prefix is now the k-th largest key T; krem = how many keys == T to keep.
-    const uint32_t T = prefix;
-
-    // ---- output: warp w owns a contiguous part of the request's range
-    const int seg = (n + kWarps - 1) / kWarps;
-    const int wlo = min(n, warp * seg), whi = min(n, wlo + seg);
-    int gt = 0, eq = 0;
-    for (int i0 = wlo; i0 < whi; i0 += 32) {
-        const int i = i0 + lane;
-        const uint32_t key = i < whi ? key_at(i) : 0u;
-        gt += __popc(__ballot_sync(0xffffffffu, i < whi && key > T));
-        eq += __popc(__ballot_sync(0xffffffffu, i < whi && key == T));
-    }
-    if (lane == 0) {
-        sh.warp_a[warp] = gt;
-        sh.warp_b[warp] = eq;
-    }
-    __syncthreads();
-    CSLA_TL_MARK(4);
-    int gt_before = 0, eq_before = 0;
-    for (int w = 0; w < warp; ++w) {
-        gt_before += sh.warp_a[w];
-        eq_before += sh.warp_b[w];
-    }
-    int pos = gt_before + min(eq_before, krem);
-    int eq_seen = eq_before;
-    for (int i0 = wlo; i0 < whi; i0 += 32) {
-        const int i = i0 + lane;
-        const uint32_t key = i < whi ? key_at(i) : 0u;
-        const bool is_gt = i < whi && key > T;
-        const bool is_eq = i < whi && key == T;
-        const unsigned meq = __ballot_sync(0xffffffffu, is_eq);
-        const unsigned below = (1u << lane) - 1u;
-        const bool take_eq = is_eq && (eq_seen + __popc(meq & below)) < krem;
-        const unsigned mtake = __ballot_sync(0xffffffffu, is_gt || take_eq);
-        if (is_gt || take_eq) out[pos + __popc(mtake & below)] = i;
-        pos += __popc(mtake);
-        eq_seen += __popc(meq);
-    }
-    CSLA_TL_MARK(6);
 }
 
 // ---------------------------------------------------------------- selection with scores in registers
@@ -332,6 +147,11 @@ __device__ uint32_t radix_select(RegShared &sh, const Each &each, int rank, uint
         const int shb = left - width;
         const int nb = 1 << width;
         left = shb;
+        // every thread has read the previous digit's hist[sel] (the small-bin
+        // test below) before any thread clears it: without this barrier a
+        // fast thread's clearing can flip a slow thread's test, the threads
+        // then take different paths through the barriers that follow
+        __syncthreads();
         for (int i = threadIdx.x; i < kBins; i += kRThreads) sh.hist[i] = 0;
         __syncthreads();
         each([&](uint32_t key) {
@@ -349,7 +169,10 @@ __device__ uint32_t radix_select(RegShared &sh, const Each &each, int rank, uint
             if (threadIdx.x == 0) sh.small_n = 0;
             __syncthreads();
             each([&](uint32_t key) {
-                if (key != 0u && (key & pmask) == prefix) sh.small[atomicAdd(&sh.small_n, 1)] = key;
+                if (key != 0u && (key & pmask) == prefix) {
+                    const int at = atomicAdd(&sh.small_n, 1);
+                    if (at < 32) sh.small[at] = key;
+                }
             });
             __syncthreads();
             if (warp == 0) {
@@ -677,6 +500,208 @@ __global__ void __cluster_dims__(kG, 1, 1) __launch_bounds__(kRThreads, 1) topk_
     cl.sync();   // no CTA leaves while another may still read its counts
 }
 
+// ---------------------------------------------------------------- streaming variant
+// For n > kRegMax (query rows of a long prefill): one CTA of 512 threads per
+// row, the row's scores read from global memory once on the fast path.
+// Warp w owns the contiguous range [w*seg, (w+1)*seg), seg = ceil(n / 16).
+//  1. Threshold from a sample: every warp sorts 32 keys spread over its
+//     range and takes its rw-th largest, rw = ceil(48k / n); t0 is the
+//     smallest of these, so about 1.5k or more keys lie at or above it.
+//  2. One streaming sweep (8 loads in flight per lane) compacts the keys
+//     >= t0, with their indices, into the warp's region, in index order.
+//  3. When every region fitted and there are at least k candidates, the
+//     exact k-th largest key T is found among them (every key >= T is one)
+//     and the output is written from the regions; otherwise (heavy ties, a
+//     sample far off) a radix select over all keys re-reads the row, and
+//     the output pass walks it once more.  Either way the output is the
+//     keys > T and the lowest-index keys == T, ascending.
+constexpr int kSBatch = 8;   // score loads a lane keeps in flight in the sweep
+
+__global__ void __launch_bounds__(kRThreads, 2) topk_stream_kernel(TopkArgs a) {
+    CSLA_TL_SCOPE(kTlTopk);
+    extern __shared__ __align__(16) uint8_t dyn_st[];
+    RegShared &sh = *reinterpret_cast<RegShared *>(dyn_st);
+    pdl_trigger();
+    const int b = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const unsigned below = (1u << lane) - 1u;
+    const int slot = __ldg(a.slots + b);
+    const bool slot_ok = slot >= 0 && slot < a.n_slots;
+    pdl_wait();
+    CSLA_TL_WAITED();
+    const int L = slot_ok ? row_visible_len(a.len, a.q_len, slot, b) : 0;
+    int n = L < 0 ? 0 : L / a.m;
+    if (!slot_ok || L < 0 || L / a.m > a.max_n) {
+        if (threadIdx.x == 0) set_dev_err(CSLA_DEVERR_LEN);
+        n = 0;
+    }
+    const int k = a.k;
+    int32_t *out = a.idx + (size_t)b * k;
+    if (n <= k) {
+        for (int j = threadIdx.x; j < k; j += kRThreads) out[j] = j < n ? j : -1;
+        return;
+    }
+    const float *sc = a.scores + (size_t)b * a.stride;
+    const int seg = (n + kRWarps - 1) / kRWarps;
+    const int wlo = min(n, warp * seg), whi = min(n, wlo + seg);
+
+    // ---- 1. threshold from a per-warp sample
+    const int ns = whi - wlo;
+    uint32_t smp = 0;
+    if (ns > 0) smp = score_key(__ldg(sc + wlo + (int)(((long long)lane * ns) >> 5)));
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const uint32_t o = __shfl_xor_sync(0xffffffffu, smp, stride);
+            const bool desc = (lane & size) == 0 || size == 32;
+            const bool lower = (lane & stride) == 0;
+            smp = (lower == desc) ? max(smp, o) : min(smp, o);
+        }
+    }
+    const int rw = min(32, max(1, (int)((48LL * k + n - 1) / n)));
+    const uint32_t s_w = __shfl_sync(0xffffffffu, smp, rw - 1);
+    if (lane == 0) sh.tw[warp] = ns > 0 ? s_w : 0xFFFFFFFFu;   // an empty range imposes nothing
+    __syncthreads();
+    uint32_t t0 = lane < kRWarps ? sh.tw[lane] : 0xFFFFFFFFu;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t0 = min(t0, __shfl_xor_sync(0xffffffffu, t0, o));
+    CSLA_TL_MARK(0);
+
+    // ---- 2. this warp's keys >= t0 into its region, in index order
+    int pos = 0;
+    uint32_t cmax = 0;
+    for (int i0 = wlo; i0 < whi; i0 += 32 * kSBatch) {
+        float f[kSBatch];
+#pragma unroll
+        for (int u = 0; u < kSBatch; ++u) {
+            const int i = i0 + 32 * u + lane;
+            f[u] = i < whi ? __ldg(sc + i) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kSBatch; ++u) {
+            const int i = i0 + 32 * u + lane;
+            const uint32_t key = score_key(f[u]);
+            const bool q = i < whi && key >= t0;
+            const unsigned mq = __ballot_sync(0xffffffffu, q);
+            const int at = pos + __popc(mq & below);
+            if (q && at < kRegion) {
+                sh.ckey[warp][at] = key;
+                sh.cidx[warp][at] = i;
+            }
+            if (q) cmax = max(cmax, key);
+            pos += __popc(mq);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+    if (lane == 0) {
+        sh.cnt[warp] = pos;
+        sh.warp_b[warp] = (int)cmax;
+    }
+    __syncthreads();
+    const int cn = lane < kRWarps ? sh.cnt[lane] : 0;
+    const bool fits = __all_sync(0xffffffffu, cn <= kRegion);
+    int n_ge = cn;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n_ge += __shfl_xor_sync(0xffffffffu, n_ge, o);
+    uint32_t kmax = lane < kRWarps ? (uint32_t)sh.warp_b[lane] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    CSLA_TL_MARK(1);
+    __syncthreads();   // warp_b is reused below
+
+    if (fits && n_ge >= k) {
+        // ---- 3. the exact k-th key among the candidates, output from the regions
+        const int my_n = sh.cnt[warp];
+        int krem;
+        const int bits = 32 - __clz(t0 ^ kmax);
+        const uint32_t T = radix_select(sh, [&](auto fn) {
+            for (int i = lane; i < my_n; i += 32) fn(sh.ckey[warp][i]);
+        }, k, kmax, bits, &krem);
+        CSLA_TL_MARK(2);
+        int gt = 0, eq = 0;
+        for (int i = lane; i < my_n; i += 32) {
+            const uint32_t key = sh.ckey[warp][i];
+            gt += key > T;
+            eq += key == T;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            gt += __shfl_xor_sync(0xffffffffu, gt, o);
+            eq += __shfl_xor_sync(0xffffffffu, eq, o);
+        }
+        if (lane == 0) {
+            sh.warp_a[warp] = gt;
+            sh.warp_b[warp] = eq;
+        }
+        __syncthreads();
+        int tot;
+        const int gt_before = warp_prefix(sh.warp_a, warp, &tot);
+        const int eq_before = warp_prefix(sh.warp_b, warp, &tot);
+        int opos = gt_before + min(eq_before, krem);
+        int eq_seen = eq_before;
+        for (int i0 = 0; i0 < my_n; i0 += 32) {
+            const int i = i0 + lane;
+            const uint32_t key = i < my_n ? sh.ckey[warp][i] : 0u;
+            const bool is_gt = i < my_n && key > T;
+            const bool is_eq = i < my_n && key == T;
+            const unsigned meq = __ballot_sync(0xffffffffu, is_eq);
+            const bool take_eq = is_eq && (eq_seen + __popc(meq & below)) < krem;
+            const unsigned mtake = __ballot_sync(0xffffffffu, is_gt || take_eq);
+            if (is_gt || take_eq) {
+                const int p = opos + __popc(mtake & below);
+                if (p >= 0 && p < k) out[p] = sh.cidx[warp][i];
+                else set_dev_err(CSLA_DEVERR_INDEX);   // never for a correct selection
+            }
+            opos += __popc(mtake);
+            eq_seen += __popc(meq);
+        }
+        CSLA_TL_MARK(3);
+        return;
+    }
+
+    // ---- fallback: radix select over every key, re-read from global memory
+    int krem;
+    const uint32_t T = radix_select(sh, [&](auto fn) {
+        for (int i = wlo + lane; i < whi; i += 32) fn(score_key(__ldg(sc + i)));
+    }, k, 0u, 32, &krem);
+    int gt = 0, eq = 0;
+    for (int i0 = wlo; i0 < whi; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t key = i < whi ? score_key(__ldg(sc + i)) : 0u;
+        gt += __popc(__ballot_sync(0xffffffffu, i < whi && key > T));
+        eq += __popc(__ballot_sync(0xffffffffu, i < whi && key == T));
+    }
+    if (lane == 0) {
+        sh.warp_a[warp] = gt;
+        sh.warp_b[warp] = eq;
+    }
+    __syncthreads();
+    int tot;
+    const int gt_before = warp_prefix(sh.warp_a, warp, &tot);
+    const int eq_before = warp_prefix(sh.warp_b, warp, &tot);
+    int opos = gt_before + min(eq_before, krem);
+    int eq_seen = eq_before;
+    for (int i0 = wlo; i0 < whi; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t key = i < whi ? score_key(__ldg(sc + i)) : 0u;
+        const bool is_gt = i < whi && key > T;
+        const bool is_eq = i < whi && key == T;
+        const unsigned meq = __ballot_sync(0xffffffffu, is_eq);
+        const bool take_eq = is_eq && (eq_seen + __popc(meq & below)) < krem;
+        const unsigned mtake = __ballot_sync(0xffffffffu, is_gt || take_eq);
+        if (is_gt || take_eq) {
+            const int p = opos + __popc(mtake & below);
+            if (p >= 0 && p < k) out[p] = i;
+            else set_dev_err(CSLA_DEVERR_INDEX);   // never for a correct selection
+        }
+        opos += __popc(mtake);
+        eq_seen += __popc(meq);
+    }
+    CSLA_TL_MARK(4);
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
@@ -684,23 +709,17 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)(kHistBytes + kSmemKeysMax * sizeof(uint32_t)));
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kHistBytes);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sizeof(ClShared));
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(topk_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(RegShared));
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
     if (a.max_n <= kRegMax)
         return launch_pdl(topk_cluster_kernel, dim3(a.B * kG), dim3(kRThreads), sizeof(ClShared), stream, a);
-    if (a.max_n <= kSmemKeysMax) {
-        const size_t smem = kHistBytes + (size_t)(a.max_n > 0 ? a.max_n : 1) * sizeof(uint32_t);
-        return launch_pdl(topk_kernel<true>, dim3(a.B), dim3(kThreads), smem, stream, a);
-    }
-    return launch_pdl(topk_kernel<false>, dim3(a.B), dim3(kThreads), kHistBytes, stream, a);
+    return launch_pdl(topk_stream_kernel, dim3(a.B), dim3(kRThreads), sizeof(RegShared), stream, a);
 }
 
 }  // namespace csla
