@@ -321,7 +321,8 @@ static int prep_indexer(const csla_cfg *cfg, const csla_state *st, const csla_ca
     L->w_bf16 = w_dtype == CSLA_BF16;
     L->gemm = L->cq_bf16 && L->w_bf16;
     if (L->gemm && (!encode_bf16_2d(&L->pm.cq, cq, (uint64_t)cfg->dc, (uint64_t)B, 128) ||
-                    !encode_bf16_2d(&L->pm.w, W_iq, (uint64_t)cfg->dc, (uint64_t)cfg->HI * cfg->dI, 64)))
+                    !encode_bf16_2d(&L->pm.w, W_iq, (uint64_t)cfg->dc, (uint64_t)cfg->HI * cfg->dI,
+                                    (uint32_t)iq_gemm_bn(B))))
         return CSLA_ERR_CUDA;
     IndexerArgs a{};
     a.m = cfg->m; a.HI = cfg->HI; a.dI = cfg->dI; a.dc = cfg->dc; a.NQ = NQ;

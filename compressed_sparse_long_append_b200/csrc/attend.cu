@@ -684,7 +684,9 @@ __device__ void loader_role(const AttendArgs &a, int b, const Req &rq, Span sp, 
     ResolveRegs rr;
     int t = 0;
     bool ok = true;
-    if (q_in_two && !q_in_raw) ok = loader_step<D>(a, rq, L, t++, smem, ms, rr, &landed, &issued);
+    // (with few tiles the conversion would only slow the Qhat build, which
+    // is then on the critical path)
+    if (q_in_two && !q_in_raw && L.n_tiles >= 4) ok = loader_step<D>(a, rq, L, t++, smem, ms, rr, &landed, &issued);
     if (ok && warp_all(mbar_wait(&ms->q_ready, 0, &ms->abort))) {
         for (; t < L.n_tiles; ++t)
             if (!loader_step<D>(a, rq, L, t, smem, ms, rr, &landed, &issued)) break;

@@ -394,10 +394,10 @@ __device__ void pool_block_channel(const BlockRows<T> &x, int m, const float *ws
     __syncthreads();
 }
 
-template <typename T>
-__device__ __forceinline__ void pool_any(const BlockRows<T> &x, int m, int gate, const float *wsm, float *alpha,
+template <typename T, bool kChannel>
+__device__ __forceinline__ void pool_any(const BlockRows<T> &x, int m, const float *wsm, float *alpha,
                                          const float *bias, float *part, float *xs, float *out, float *red) {
-    if (gate == CSLA_GATE_CHANNEL) {
+    if constexpr (kChannel) {
         if (m <= kSmallM) pool_small_channel<T>(x, m, wsm, bias, out);
         else pool_block_channel<T>(x, m, wsm, bias, xs, out);
     } else if (m <= kSmallM) {
@@ -408,7 +408,9 @@ __device__ __forceinline__ void pool_any(const BlockRows<T> &x, int m, int gate,
 }
 
 // kTok: the call also keeps every new token's window row (CompressArgs::tok_rows).
-template <typename T, bool kTok>
+// kChannel: the per-channel gate (a separate instantiation, so that the
+// per-token path carries none of its code).
+template <typename T, bool kTok, bool kChannel>
 __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs a) {
     CSLA_TL_SCOPE(kTlCompress);
     extern __shared__ __align__(16) float sm[];
@@ -456,7 +458,7 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs 
         const float *w = z == 0 ? a.wg : a.wgi;
         const float *gb = z == 0 ? a.gb : a.gbi;
         for (int d = threadIdx.x; d < width; d += kThreads) wsm[d] = __ldg(w + d);
-        if (a.gate != CSLA_GATE_CHANNEL)
+        if (!kChannel)
             for (int i = threadIdx.x; i < m; i += kThreads) alpha[i] = __ldg(gb + i);
     }
     pdl_wait();
@@ -522,7 +524,7 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs 
         const T *fresh = reinterpret_cast<const T *>(a.kv_new) + ((size_t)b * a.T + f0) * D;
         const BlockRows<T> rows{a.tail_kv + (size_t)slot * m * D, fresh, n_tail, D,
                                 (reinterpret_cast<uintptr_t>(a.kv_new) & vec_mask) == 0};
-        pool_any<T>(rows, m, a.gate, wsm, alpha, a.gb, part, xs, v, red);
+        pool_any<T, kChannel>(rows, m, wsm, alpha, a.gb, part, xs, v, red);
         CSLA_TL_MARK(1);
         norm_rope_quantise(v, gam, a, p0, a.rows + ent * rb, a.scales + ent, red);
         CSLA_TL_MARK(2);
@@ -531,7 +533,7 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs 
         const T *fresh = reinterpret_cast<const T *>(a.kidx_new) + ((size_t)b * a.T + f0) * dI;
         const BlockRows<T> rows{a.tail_idx + (size_t)slot * m * dI, fresh, n_tail, dI,
                                 (reinterpret_cast<uintptr_t>(a.kidx_new) & vec_mask) == 0};
-        pool_any<T>(rows, m, a.gate, wsm, alpha, a.gbi, part, xs, v, red);
+        pool_any<T, kChannel>(rows, m, wsm, alpha, a.gbi, part, xs, v, red);
         CSLA_TL_MARK(1);
         if (a.key_fmt == CSLA_KEY_E4M3) {
             // one power-of-two scale per entry: the smallest 2^e with
@@ -629,8 +631,12 @@ cudaError_t launch_compress_append(const CompressArgs &a, bool bf16, cudaStream_
         // largest case: W = 512, m = 128
         const int most = (int)((2 * 512 + 512 + 128 + 4 * kThreads + 32 + kStageRows * 512) * sizeof(float));
         cudaError_t e = cudaSuccess;
-        for (auto fn : {compress_append_kernel<float, false>, compress_append_kernel<float, true>,
-                        compress_append_kernel<__nv_bfloat16, false>, compress_append_kernel<__nv_bfloat16, true>}) {
+        for (auto fn : {compress_append_kernel<float, false, false>, compress_append_kernel<float, true, false>,
+                        compress_append_kernel<__nv_bfloat16, false, false>,
+                        compress_append_kernel<__nv_bfloat16, true, false>,
+                        compress_append_kernel<float, false, true>, compress_append_kernel<float, true, true>,
+                        compress_append_kernel<__nv_bfloat16, false, true>,
+                        compress_append_kernel<__nv_bfloat16, true, true>}) {
             e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
             if (e != cudaSuccess) return e;
         }
@@ -638,13 +644,16 @@ cudaError_t launch_compress_append(const CompressArgs &a, bool bf16, cudaStream_
     }
     const dim3 grid(a.T + nb, a.B, a.kidx ? 2 : 1);
     const bool tok = a.tok_rows != nullptr;
-    cudaError_t e;
+    const bool ch = a.gate == CSLA_GATE_CHANNEL;
+    void (*fn)(CompressArgs);
     if (bf16)
-        e = tok ? launch_pdl(compress_append_kernel<__nv_bfloat16, true>, grid, dim3(kThreads), smem, stream, a)
-                : launch_pdl(compress_append_kernel<__nv_bfloat16, false>, grid, dim3(kThreads), smem, stream, a);
+        fn = ch ? (tok ? compress_append_kernel<__nv_bfloat16, true, true> : compress_append_kernel<__nv_bfloat16, false, true>)
+                : (tok ? compress_append_kernel<__nv_bfloat16, true, false>
+                       : compress_append_kernel<__nv_bfloat16, false, false>);
     else
-        e = tok ? launch_pdl(compress_append_kernel<float, true>, grid, dim3(kThreads), smem, stream, a)
-                : launch_pdl(compress_append_kernel<float, false>, grid, dim3(kThreads), smem, stream, a);
+        fn = ch ? (tok ? compress_append_kernel<float, true, true> : compress_append_kernel<float, false, true>)
+                : (tok ? compress_append_kernel<float, true, false> : compress_append_kernel<float, false, false>);
+    cudaError_t e = launch_pdl(fn, grid, dim3(kThreads), smem, stream, a);
     if (e != cudaSuccess) return e;
     return bf16 ? launch_pdl(tail_update_kernel<__nv_bfloat16>, dim3(a.B), dim3(kThreads), 0, stream, a)
                 : launch_pdl(tail_update_kernel<float>, dim3(a.B), dim3(kThreads), 0, stream, a);

@@ -651,10 +651,15 @@ __global__ void __launch_bounds__(256) len_snapshot_kernel(const int32_t *slots,
 // and rows past B read as zeros (TMA fill).  The loads and products come
 // before the grid-dependency wait (cq and W_iq are inputs of the call);
 // the stores follow it.
-constexpr int kGemmBM = 128, kGemmBN = 64, kGemmStages = 4, kGemmThreads = 192;
-constexpr int kGemmABytes = kGemmBM * 128, kGemmBBytes = kGemmBN * 128;
-constexpr int kGemmSmem = 1024 + kGemmStages * (kGemmABytes + kGemmBBytes) + 256;
+constexpr int kGemmBM = 128, kGemmStages = 4, kGemmThreads = 192;
+constexpr int kGemmABytes = kGemmBM * 128;
+template <int BN>
+constexpr int gemm_smem() { return 1024 + kGemmStages * (kGemmABytes + BN * 128) + 256; }
 
+// BN: output features per CTA (iq_gemm_bn).  An output's value does not
+// depend on it, nor on the output's tile or lane: each is its own dot
+// product over the K slabs, in order.
+template <int BN>
 __global__ void __launch_bounds__(kGemmThreads) iq_gemm_kernel(IndexerArgs a, const __grid_constant__ CUtensorMap cqmap,
                                                                 const __grid_constant__ CUtensorMap wmap) {
     CSLA_TL_SCOPE(kTlIqProject);
@@ -662,12 +667,12 @@ __global__ void __launch_bounds__(kGemmThreads) iq_gemm_kernel(IndexerArgs a, co
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t *As = base;
     uint8_t *Bs = base + kGemmStages * kGemmABytes;
-    uint64_t *full = reinterpret_cast<uint64_t *>(Bs + kGemmStages * kGemmBBytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(Bs + kGemmStages * (BN * 128));
     uint64_t *empty = full + kGemmStages, *done = empty + kGemmStages;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(done + 1);
     __shared__ volatile int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * kGemmBM, n0 = blockIdx.y * kGemmBN;
+    const int m0 = blockIdx.x * kGemmBM, n0 = blockIdx.y * BN;
     const int nk = (a.dc + 63) / 64;
     if (threadIdx.x == 0) {
         abort_flag = 0;
@@ -696,9 +701,9 @@ __global__ void __launch_bounds__(kGemmThreads) iq_gemm_kernel(IndexerArgs a, co
             for (; k < nk; ++k) {
                 const int s = k % kGemmStages;
                 if (k >= kGemmStages && !mbar_wait(empty + s, ((k / kGemmStages) - 1) & 1, &abort_flag)) break;
-                mbar_arrive_expect_tx(full + s, (uint32_t)(kGemmABytes + kGemmBBytes));
+                mbar_arrive_expect_tx(full + s, (uint32_t)(kGemmABytes + (BN * 128)));
                 tma_load_2d(As + s * kGemmABytes, &cqmap, k * 64, m0, full + s);
-                tma_load_2d(Bs + s * kGemmBBytes, &wmap, k * 64, n0, full + s);
+                tma_load_2d(Bs + s * (BN * 128), &wmap, k * 64, n0, full + s);
             }
             // every issued copy must land before the CTA may exit
             for (int i = (k > kGemmStages ? k - kGemmStages : 0); i < k; ++i)
@@ -706,13 +711,13 @@ __global__ void __launch_bounds__(kGemmThreads) iq_gemm_kernel(IndexerArgs a, co
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(kGemmBM, kGemmBN, false, false);
+            constexpr uint32_t idesc = idesc_bf16(kGemmBM, BN, false, false);
             int k = 0;
             for (; k < nk; ++k) {
                 const int s = k % kGemmStages;
                 if (!mbar_wait(full + s, (k / kGemmStages) & 1, &abort_flag)) break;
                 tc_fence_after();
-                const uint32_t ab = smem_u32(As + s * kGemmABytes), bb = smem_u32(Bs + s * kGemmBBytes);
+                const uint32_t ab = smem_u32(As + s * kGemmABytes), bb = smem_u32(Bs + s * (BN * 128));
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_kind_f16(tmem, sdesc(ab + kk * 32, 16, 1024), sdesc(bb + kk * 32, 16, 1024), idesc,
@@ -734,13 +739,13 @@ __global__ void __launch_bounds__(kGemmThreads) iq_gemm_kernel(IndexerArgs a, co
             uint16_t *dst = a.q_ws + (size_t)(row < a.B ? row : 0) * a.NQ * a.dI + (size_t)j * a.dI + e0;
             const size_t tstride = (size_t)a.HI * a.dI;   // hi, mid, lo term rows are HI rows apart
 #pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r[32];
-                tmem_ld32x32(tmem + ((uint32_t)lane_base << 16) + 32 * half, r);
+            for (int c16 = 0; c16 < BN / 16; ++c16) {
+                uint32_t r[16];
+                tmem_ld32x16(tmem + ((uint32_t)lane_base << 16) + 16 * c16, r);
                 tmem_wait_ld();
                 if (row < a.B) {
 #pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
+                    for (int c8 = 0; c8 < 2; ++c8) {
                         uint32_t h[4], md[4], lo[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
@@ -759,7 +764,7 @@ __global__ void __launch_bounds__(kGemmThreads) iq_gemm_kernel(IndexerArgs a, co
                             md[i] = mm[0] | (mm[1] << 16);
                             lo[i] = ll[0] | (ll[1] << 16);
                         }
-                        uint16_t *o = dst + 32 * half + c8 * 8;
+                        uint16_t *o = dst + 16 * c16 + c8 * 8;
                         *reinterpret_cast<uint4 *>(o) = make_uint4(h[0], h[1], h[2], h[3]);
                         *reinterpret_cast<uint4 *>(o + tstride) = make_uint4(md[0], md[1], md[2], md[3]);
                         *reinterpret_cast<uint4 *>(o + 2 * tstride) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
@@ -781,12 +786,14 @@ cudaError_t launch_iq_gemm(const IndexerArgs &a, const ProjMaps &pm, cudaStream_
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(iq_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+        cudaError_t e = cudaFuncSetAttribute(iq_gemm_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             gemm_smem<64>());
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
-    const dim3 grid((a.B + kGemmBM - 1) / kGemmBM, (a.HI * a.dI) / kGemmBN);
-    return launch_pdl(iq_gemm_kernel, grid, dim3(kGemmThreads), (size_t)kGemmSmem, stream, a, pm.cq, pm.w);
+    if (iq_gemm_bn(a.B) != 64) return cudaErrorInvalidValue;
+    const dim3 grid((a.B + kGemmBM - 1) / kGemmBM, (a.HI * a.dI) / 64);
+    return launch_pdl(iq_gemm_kernel<64>, grid, dim3(kGemmThreads), (size_t)gemm_smem<64>(), stream, a, pm.cq, pm.w);
 }
 
 cudaError_t launch_scoring(const IndexerArgs &a, const CUtensorMap &kmap, const CUtensorMap &qmap,

@@ -123,11 +123,18 @@ cudaError_t launch_len_snapshot(const int32_t *slots, const int32_t *len, int B,
 // to one request: as many as fit the UMMA N limit of 256 columns.
 __host__ __device__ constexpr int indexer_rows_per_cta(int NQ) { return 256 / NQ; }
 // Tensor maps of the index-query projection on the tensor cores (bf16 cq
-// and W_iq): cq [B][dc] in 128-row boxes, W_iq [HI*dI][dc] in 64-row boxes,
-// 64 columns (128 bytes) per box, 128-byte swizzle.
+// and W_iq): cq [B][dc] in 128-row boxes, W_iq [HI*dI][dc] in boxes of
+// iq_gemm_bn(B) rows, 64 columns (128 bytes) per box, 128-byte swizzle.
 struct ProjMaps {
     CUtensorMap cq, w;
 };
+// Output features per CTA of that projection (the W_iq box height).
+// (16 for small batches measured slower at decode: 24.5 against 17.6 us per
+// indexer call, the extra CTAs each filling a whole 128-row cq tile.)
+inline int iq_gemm_bn(int B) {
+    (void)B;
+    return 64;
+}
 cudaError_t launch_indexer(const IndexerArgs &a, bool cq_bf16, bool w_bf16, const CUtensorMap &kmap,
                            const CUtensorMap &qmap, int num_sms, cudaStream_t stream, bool project = true,
                            const ProjMaps *pm = nullptr);

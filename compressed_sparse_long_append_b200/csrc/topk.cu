@@ -504,9 +504,13 @@ __global__ void __cluster_dims__(kG, 1, 1) __launch_bounds__(kRThreads, 1) topk_
 // For n > kRegMax (query rows of a long prefill): one CTA of 512 threads per
 // row, the row's scores read from global memory once on the fast path.
 // Warp w owns the contiguous range [w*seg, (w+1)*seg), seg = ceil(n / 16).
-//  1. Threshold from a sample: every warp sorts 32 keys spread over its
-//     range and takes its rw-th largest, rw = ceil(48k / n); t0 is the
-//     smallest of these, so about 1.5k or more keys lie at or above it.
+//  1. Threshold from a sample: every lane takes the largest of S keys
+//     spread over its warp's range (S = ceil(n / 6k), at most 64), every
+//     warp sorts its 32 and takes the rw-th largest, rw = ceil(48kS / n)
+//     (about 8); t0 is the smallest of these, so about 1.5k or more keys
+//     lie at or above it whatever the row length, and the warps' regions
+//     rarely overflow (a larger sample keeps the smallest of the 16
+//     estimates close to the others).
 //  2. One streaming sweep (8 loads in flight per lane) compacts the keys
 //     >= t0, with their indices, into the warp's region, in index order.
 //  3. When every region fitted and there are at least k candidates, the
@@ -545,10 +549,16 @@ __global__ void __launch_bounds__(kRThreads, 2) topk_stream_kernel(TopkArgs a) {
     const int seg = (n + kRWarps - 1) / kRWarps;
     const int wlo = min(n, warp * seg), whi = min(n, wlo + seg);
 
-    // ---- 1. threshold from a per-warp sample
+    // ---- 1. threshold from a per-warp sample: lane l keeps the largest of
+    // its S keys spread over the warp's range
     const int ns = whi - wlo;
+    const int S = min(64, max(1, (int)(((long long)n + 6LL * k - 1) / (6LL * k))));
     uint32_t smp = 0;
-    if (ns > 0) smp = score_key(__ldg(sc + wlo + (int)(((long long)lane * ns) >> 5)));
+    if (ns > 0) {
+        const long long span = 32LL * S;
+        for (int u = 0; u < S; ++u)
+            smp = max(smp, score_key(__ldg(sc + wlo + (int)(((long long)(lane * S + u) * ns) / span))));
+    }
 #pragma unroll
     for (int size = 2; size <= 32; size <<= 1) {
 #pragma unroll
@@ -559,7 +569,7 @@ __global__ void __launch_bounds__(kRThreads, 2) topk_stream_kernel(TopkArgs a) {
             smp = (lower == desc) ? max(smp, o) : min(smp, o);
         }
     }
-    const int rw = min(32, max(1, (int)((48LL * k + n - 1) / n)));
+    const int rw = min(32, max(1, (int)((48LL * k * S + n - 1) / n)));
     const uint32_t s_w = __shfl_sync(0xffffffffu, smp, rw - 1);
     if (lane == 0) sh.tw[warp] = ns > 0 ? s_w : 0xFFFFFFFFu;   // an empty range imposes nothing
     __syncthreads();

@@ -130,3 +130,34 @@ def test_pipeline_topk_set_within_ambiguity_band():
         gs = set(g.tolist())
         assert must <= gs and not (gs & never)
         assert len(gs ^ set(ref[ref >= 0].tolist())) <= 2 * len(np.nonzero(np.abs(ref_scores - kth) <= GAP_TOL)[0])
+
+
+@pytest.mark.parametrize("key_fmt", [0, 1])
+def test_indexer_scores_do_not_depend_on_the_batch(key_fmt):
+    """One request's scores bit-identical whether it is scored alone or as
+    one of 200 rows: the batch changes the projection's tiling (the request
+    lands in another 128-row tile and TMEM lane of the tensor-core GEMM) and
+    the indexer's grid, never a row's arithmetic."""
+    w = dataclasses.replace(CSA_DECODE, B=1, L=3000, key_fmt=key_fmt, name="idx_inv")
+    cv, p = oracle_cache(w, [3000])
+    lb = upload_layer(w, cv, [3000])
+    nb = 200
+    # 200 slots that all read the one request's pages
+    from compressed_sparse_long_append_b200.layer import LayerBuffers
+    from gpu_helpers import fill_layer, shape_of
+    big = LayerBuffers(shape_of(w), nb, lb.n_pages, lb.bt_stride, DEV)
+    fill_layer(big, w, cv, [3000])
+    big.block_table.copy_(lb.block_table.expand(nb, -1))
+    big.len.fill_(3000)
+    big.win_rows.copy_(lb.win_rows.expand(nb, -1, -1))
+    big.win_scales.copy_(lb.win_scales.expand(nb, -1))
+    si = step_inputs(dataclasses.replace(w, B=nb), 11)
+    rows = [0, 37, 131, 199]
+    cq_all = np.stack([si["cq"][r] for r in range(nb)])
+    hw_all = np.stack([si["head_w"][r] for r in range(nb)])
+    s_big, _ = run_indexer(w, big, {"cq": cq_all, "head_w": hw_all}, p, nb, 3000)
+    for r in rows:
+        s_one, _ = run_indexer(w, lb, {"cq": cq_all[r:r + 1], "head_w": hw_all[r:r + 1]}, p, 1, 3000)
+        nv = 3000 // w.m
+        assert torch.equal(s_one[0, :nv].view(torch.int32), s_big[r, :nv].view(torch.int32)), r
+    assert_no_device_error()
