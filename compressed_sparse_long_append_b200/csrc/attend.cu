@@ -502,38 +502,51 @@ __device__ __forceinline__ uint32_t convert_rows(const LoadCtx &L, int t, const 
     using C = Cfg<D>;
     const int slot = t % kRing;
     constexpr int kNope = kRowsPerWarp * C::kNopeCH;   // this warp's fp8 chunks per tile
+    // every shared-memory read first (the row kinds of this warp's 4 rows in
+    // one word, then all raw chunks), so that the loads overlap instead of
+    // each waiting behind the previous chunk's stores
+    static_assert(kRowsPerWarp == 4, "one 32-bit word of row kinds per warp");
+    const uint32_t kinds = *reinterpret_cast<const uint32_t *>(&ms->kind[slot][kRowsPerWarp * L.lw]);
+    uint4 v[C::kNopeIt];
+#pragma unroll
+    for (int k = 0; k < C::kNopeIt; ++k) {
+        const int f = L.lane + 32 * k;
+        const int r = f / C::kNopeCH, c = f % C::kNopeCH;
+        const bool live = (kNope % 32 == 0 || f < kNope) && ((kinds >> (8 * (r & 3))) & 0xFFu) != kLocNone;
+        v[k] = live ? *reinterpret_cast<const uint4 *>(raw + (kRowsPerWarp * L.lw + r) * C::kRB + 16 * c)
+                    : make_uint4(0u, 0u, 0u, 0u);
+    }
+    const int i4 = L.lane >> 3, cr = L.lane & 7;
+    const int ir = kRowsPerWarp * L.lw + i4;
+    const float s = ms->scl[slot][ir];
+    const uint4 vr = ((kinds >> (8 * i4)) & 0xFFu) != kLocNone
+                         ? *reinterpret_cast<const uint4 *>(raw + ir * C::kRB + 16 * (C::kNopeCH + cr))
+                         : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
     for (int k = 0; k < C::kNopeIt; ++k) {
         const int f = L.lane + 32 * k;
         if (kNope % 32 == 0 || f < kNope) {
             const int i = kRowsPerWarp * L.lw + f / C::kNopeCH, c = f % C::kNopeCH;
-            const uint4 v = ms->kind[slot][i] != kLocNone ? *reinterpret_cast<const uint4 *>(raw + i * C::kRB + 16 * c)
-                                                          : make_uint4(0u, 0u, 0u, 0u);
             uint4 lo, hi;
-            lo.x = e4m3x2_f16x2_div256<0>(v.x);
-            lo.y = e4m3x2_f16x2_div256<2>(v.x);
-            lo.z = e4m3x2_f16x2_div256<0>(v.y);
-            lo.w = e4m3x2_f16x2_div256<2>(v.y);
-            hi.x = e4m3x2_f16x2_div256<0>(v.z);
-            hi.y = e4m3x2_f16x2_div256<2>(v.z);
-            hi.z = e4m3x2_f16x2_div256<0>(v.w);
-            hi.w = e4m3x2_f16x2_div256<2>(v.w);
+            lo.x = e4m3x2_f16x2_div256<0>(v[k].x);
+            lo.y = e4m3x2_f16x2_div256<2>(v[k].x);
+            lo.z = e4m3x2_f16x2_div256<0>(v[k].y);
+            lo.w = e4m3x2_f16x2_div256<2>(v[k].y);
+            hi.x = e4m3x2_f16x2_div256<0>(v[k].z);
+            hi.y = e4m3x2_f16x2_div256<2>(v[k].z);
+            hi.z = e4m3x2_f16x2_div256<0>(v[k].w);
+            hi.w = e4m3x2_f16x2_div256<2>(v[k].w);
             *reinterpret_cast<uint4 *>(xs + sw128_off(i, 2 * c, C::kKBBytes)) = lo;
             *reinterpret_cast<uint4 *>(xs + sw128_off(i, 2 * c + 1, C::kKBBytes)) = hi;
         }
     }
     uint32_t wide = 0;
     {
-        const int i4 = L.lane >> 3, c = L.lane & 7;
-        const int i = kRowsPerWarp * L.lw + i4;
-        const float s = ms->scl[slot][i];
-        const float inv = s > 0.f ? __fdiv_rn(1.0f, __fmul_rn(256.0f, s)) : 0.f;
-        const uint4 v = ms->kind[slot][i] != kLocNone
-                            ? *reinterpret_cast<const uint4 *>(raw + i * C::kRB + 16 * (C::kNopeCH + c))
-                            : make_uint4(0u, 0u, 0u, 0u);
+        // 1 / (256 s), correctly rounded (the same value as a division)
+        const float inv = s > 0.f ? __frcp_rn(__fmul_rn(256.0f, s)) : 0.f;
         uint4 o;
-        if (rope_chunk(v, inv, &o) || s > kScaleMax) wide = 1u << i4;
-        *reinterpret_cast<uint4 *>(xs + sw128_off(i, (D - 64) / 8 + c, C::kKBBytes)) = o;
+        if (rope_chunk(vr, inv, &o) || s > kScaleMax) wide = 1u << i4;
+        *reinterpret_cast<uint4 *>(xs + sw128_off(ir, (D - 64) / 8 + cr, C::kKBBytes)) = o;
     }
     if (L.lane < kRowsPerWarp) {
         const int i = kRowsPerWarp * L.lw + L.lane;
