@@ -189,7 +189,9 @@ __device__ __forceinline__ uint32_t e4m3x2_f16x2_div256(uint32_t w) {
 // request, built in shared memory by the softmax warps in two steps from a
 // bulk copy of the request's q rows (`stage`, H*D elements).
 // Before the grid-dependency wait (q and gamma_q are inputs of the call):
-// warp w normalises heads 16w .. 16w+15, one head at a time; lane l owns the
+// gamma_q is loaded while the copy is in flight, then warp w normalises heads
+// 16w .. 16w+15, two heads at a time (false if the copy's wait gave up);
+// lane l owns the
 // 8-dim groups l and l+32 (D = 512) or the 4 dims 4l.. (D = 128), so the
 // staged reads are consecutive per lane (no bank conflicts).  Non-RoPE dims
 // go to the SW128 K-major Qhat image as f16; the RoPE dims are kept in fp32
@@ -197,7 +199,7 @@ __device__ __forceinline__ uint32_t e4m3x2_f16x2_div256(uint32_t w) {
 // wait, when the position t = len - 1 is known, lane i rotates pair i of its
 // warp's 16 heads and writes them as f16.
 template <int D>
-__device__ void build_q_normed(const AttendArgs &a, uint8_t *smem, uint8_t *stage, int q_bf16) {
+__device__ bool build_q_normed(const AttendArgs &a, uint8_t *smem, uint8_t *stage, int q_bf16, Misc *ms) {
     using C = Cfg<D>;
     constexpr int kG = D == 512 ? 2 : 1;       // element groups per lane
     constexpr int kE = D == 512 ? 8 : 4;       // elements per group
@@ -209,88 +211,109 @@ __device__ void build_q_normed(const AttendArgs &a, uint8_t *smem, uint8_t *stag
     for (int g = 0; g < kG; ++g)
 #pragma unroll
         for (int e = 0; e < kE; ++e) gam[g][e] = __ldg(a.gamma_q + g * kStride + kE * lane + e);
-    for (int h = 16 * warp; h < 16 * warp + 16; ++h) {
-        if (h >= a.H) {
-            // padding head: zero Qhat row (the RoPE dims are written zero after the wait)
+    // gamma_q is in registers before q's rows are waited for
+    if (!warp_all(mbar_wait(&ms->q_staged, 0, &ms->abort))) return false;
+    // two heads at a time: their loads, reductions and square roots are
+    // independent chains that overlap
+    constexpr int kHB = 2;
+    for (int h0 = 16 * warp; h0 < 16 * warp + 16; h0 += kHB) {
+        float x[kHB][kG][kE];
+#pragma unroll
+        for (int u = 0; u < kHB; ++u) {
+            const int h = h0 + u;
+            const uint8_t *src = stage + h * rb;
 #pragma unroll
             for (int g = 0; g < kG; ++g) {
                 const int d = g * kStride + kE * lane;
-                if (d < D - 64) {
-                    if constexpr (kE == 8)
-                        *reinterpret_cast<uint4 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB)) =
-                            make_uint4(0u, 0u, 0u, 0u);
-                    else
-                        *reinterpret_cast<uint2 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB) + (d & 7) * 2) =
-                            make_uint2(0u, 0u);
-                }
-            }
-            continue;
-        }
-        const uint8_t *src = stage + h * rb;
-        float x[kG][kE];
+                if (h >= a.H) {
 #pragma unroll
-        for (int g = 0; g < kG; ++g) {
-            const int d = g * kStride + kE * lane;
-            if (q_bf16) {
-                if constexpr (kE == 8) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(src + 2 * d);
-                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                    for (int e = 0; e < kE; ++e) x[u][g][e] = 0.f;
+                } else if (q_bf16) {
+                    if constexpr (kE == 8) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(src + 2 * d);
+                        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        x[g][2 * e] = bf16_bits_to_f32(ww[e] & 0xFFFFu);
-                        x[g][2 * e + 1] = bf16_bits_to_f32(ww[e] >> 16);
+                        for (int e = 0; e < 4; ++e) {
+                            x[u][g][2 * e] = bf16_bits_to_f32(ww[e] & 0xFFFFu);
+                            x[u][g][2 * e + 1] = bf16_bits_to_f32(ww[e] >> 16);
+                        }
+                    } else {
+                        const uint2 w = *reinterpret_cast<const uint2 *>(src + 2 * d);
+                        x[u][g][0] = bf16_bits_to_f32(w.x & 0xFFFFu);
+                        x[u][g][1] = bf16_bits_to_f32(w.x >> 16);
+                        x[u][g][2] = bf16_bits_to_f32(w.y & 0xFFFFu);
+                        x[u][g][3] = bf16_bits_to_f32(w.y >> 16);
                     }
                 } else {
-                    const uint2 w = *reinterpret_cast<const uint2 *>(src + 2 * d);
-                    x[g][0] = bf16_bits_to_f32(w.x & 0xFFFFu);
-                    x[g][1] = bf16_bits_to_f32(w.x >> 16);
-                    x[g][2] = bf16_bits_to_f32(w.y & 0xFFFFu);
-                    x[g][3] = bf16_bits_to_f32(w.y >> 16);
-                }
-            } else {
 #pragma unroll
-                for (int e0 = 0; e0 < kE; e0 += 4) {
-                    const float4 f4 = *reinterpret_cast<const float4 *>(src + 4 * (d + e0));
-                    x[g][e0] = f4.x;
-                    x[g][e0 + 1] = f4.y;
-                    x[g][e0 + 2] = f4.z;
-                    x[g][e0 + 3] = f4.w;
+                    for (int e0 = 0; e0 < kE; e0 += 4) {
+                        const float4 f4 = *reinterpret_cast<const float4 *>(src + 4 * (d + e0));
+                        x[u][g][e0] = f4.x;
+                        x[u][g][e0 + 1] = f4.y;
+                        x[u][g][e0 + 2] = f4.z;
+                        x[u][g][e0 + 3] = f4.w;
+                    }
                 }
             }
         }
-        float ss = 0.f;
+        float r[kHB];
 #pragma unroll
-        for (int g = 0; g < kG; ++g)
+        for (int u = 0; u < kHB; ++u) {
+            float ss = 0.f;
 #pragma unroll
-            for (int e = 0; e < kE; ++e) ss = __fmaf_rn(x[g][e], x[g][e], ss);
-        ss = warp_sum(ss);   // every lane has read head h's row before anything is written back
-        const float r = 1.0f / sqrtf(__fdiv_rn(ss, (float)D) + a.eps);
+            for (int g = 0; g < kG; ++g)
 #pragma unroll
-        for (int g = 0; g < kG; ++g) {
-            const int d = g * kStride + kE * lane;
-            float y[kE];
+                for (int e = 0; e < kE; ++e) ss = __fmaf_rn(x[u][g][e], x[u][g][e], ss);
+            r[u] = ss;
+        }
+        // every lane has read both heads' rows before anything is written back
 #pragma unroll
-            for (int e = 0; e < kE; ++e) y[e] = __fmul_rn(__fmul_rn(x[g][e], r), gam[g][e]);
-            if (d >= D - 64) {
-                float *rf = reinterpret_cast<float *>(stage + h * rb);
+        for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-                for (int e = 0; e < kE; ++e) rf[(d - (D - 64)) + e] = y[e];
-            } else if constexpr (kE == 8) {
-                uint4 o;
-                o.x = pack_f16x2(y[0], y[1]);
-                o.y = pack_f16x2(y[2], y[3]);
-                o.z = pack_f16x2(y[4], y[5]);
-                o.w = pack_f16x2(y[6], y[7]);
-                *reinterpret_cast<uint4 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB)) = o;
-            } else {
-                uint2 o;
-                o.x = pack_f16x2(y[0], y[1]);
-                o.y = pack_f16x2(y[2], y[3]);
-                *reinterpret_cast<uint2 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB) + (d & 7) * 2) = o;
+            for (int u = 0; u < kHB; ++u) r[u] += __shfl_xor_sync(0xffffffffu, r[u], o);
+#pragma unroll
+        for (int u = 0; u < kHB; ++u) r[u] = 1.0f / sqrtf(__fdiv_rn(r[u], (float)D) + a.eps);
+#pragma unroll
+        for (int u = 0; u < kHB; ++u) {
+            const int h = h0 + u;
+#pragma unroll
+            for (int g = 0; g < kG; ++g) {
+                const int d = g * kStride + kE * lane;
+                float y[kE];
+#pragma unroll
+                for (int e = 0; e < kE; ++e) y[e] = __fmul_rn(__fmul_rn(x[u][g][e], r[u]), gam[g][e]);
+                if (h >= a.H) {
+                    // padding head: zero Qhat row (the RoPE dims are written zero after the wait)
+                    if (d < D - 64) {
+                        if constexpr (kE == 8)
+                            *reinterpret_cast<uint4 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB)) =
+                                make_uint4(0u, 0u, 0u, 0u);
+                        else
+                            *reinterpret_cast<uint2 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB) + (d & 7) * 2) =
+                                make_uint2(0u, 0u);
+                    }
+                } else if (d >= D - 64) {
+                    float *rf = reinterpret_cast<float *>(stage + h * rb);
+#pragma unroll
+                    for (int e = 0; e < kE; ++e) rf[(d - (D - 64)) + e] = y[e];
+                } else if constexpr (kE == 8) {
+                    uint4 o;
+                    o.x = pack_f16x2(y[0], y[1]);
+                    o.y = pack_f16x2(y[2], y[3]);
+                    o.z = pack_f16x2(y[4], y[5]);
+                    o.w = pack_f16x2(y[6], y[7]);
+                    *reinterpret_cast<uint4 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB)) = o;
+                } else {
+                    uint2 o;
+                    o.x = pack_f16x2(y[0], y[1]);
+                    o.y = pack_f16x2(y[2], y[3]);
+                    *reinterpret_cast<uint2 *>(smem + C::kOffQ + sw128_off(h, d >> 3, C::kQKB) + (d & 7) * 2) = o;
+                }
             }
         }
     }
     __syncwarp();   // the fp32 RoPE dims written by some lanes are read by all in build_q_rope
+    return true;
 }
 
 // After the wait: rotate the RoPE dims by position t and publish Qhat.
@@ -1014,8 +1037,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttendArgs a, int q
     }
     bool q_ok = true;
     if (warp < kSoftWarps) {
-        q_ok = warp_all(mbar_wait(&ms->q_staged, 0, &ms->abort));
-        if (q_ok) build_q_normed<D>(a, smem, stage, q_bf16);
+        q_ok = build_q_normed<D>(a, smem, stage, q_bf16, ms);
     }
     pdl_wait();
     CSLA_TL_WAITED();
