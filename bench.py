@@ -491,9 +491,53 @@ def hca_leg(W, K, seed, rank, world, device, variant, peak, profile=False):
                     "attend_hbm_frac": hbytes / (hms_att * 1e-3) / 1e9 / peak,
                     "attend_tflops": hflops / (hms_att * 1e-3) / 1e12,
                     "attend_tensor_frac_sustained": hflops / (hms_att * 1e-3) / 1e12 / 1395.7})
+        out["block_close"] = hca_block_close(K, seed, rank, world, device, hk, hcp)
     del hsteps, hlb, hin
     torch.cuda.empty_cache()
     return out
+
+
+def hca_block_close(K, seed, rank, world, device, hk, hcp):
+    """What closing a 128-token HCA block adds to a step: the append of one
+    token to 4 requests whose next token closes a block (the block is pooled
+    from its 128 raw rows, normed, rotated and quantised) against one whose
+    next token does not, each replayed K times with the length put back
+    after every append.  One request closes a block every 128 steps, so the
+    amortised cost per step is the difference / 128."""
+    import torch
+    from compressed_sparse_long_append_b200 import csla as C
+    from compressed_sparse_long_append_b200.layer import LayerBuffers, LayerShape
+    from csla_synth import torch_gen
+    B = hk["B"]
+    res = {}
+    for name, L0 in (("close", 1023), ("open", 1024)):
+        kw = dict(hk, B=B, L=2048)
+        lb, _, _ = build_layer(kw, B, [L0] * B, seed + 7, rank, device)
+        kv = torch_gen.normal(seed + 7, "bc/%d" % rank, (B, 1, hk["D"]), device=device).to(torch.bfloat16)
+        slots = torch.arange(B, dtype=torch.int32, device=device)
+        len0 = lb.len.clone()
+        cfg, st, cache, cps = lb.cfg(), lb.state(), lb.cache(), hcp.struct()
+
+        def step():
+            C.csla_compress_append(cfg, st, cache, slots, B, 1, kv, None, C.CSLA_BF16, cps)
+            lb.len.copy_(len0)
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        g = capture(lambda: [step() for _ in range(K)])
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        res[name] = dp_max(e0.elapsed_time(e1) / K, world, device) * 1e3
+        del g, lb
+    extra = res["close"] - res["open"]
+    return {"append_us_all_4_close": res["close"], "append_us_none_close": res["open"],
+            "extra_us_when_all_close": extra, "amortised_us_per_step": extra / 128,
+            "note": "each request closes one block per 128 steps"}
 
 
 def e4m3_leg(W, K, seed, rank, world, device, variant, profile=False):

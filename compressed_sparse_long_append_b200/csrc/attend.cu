@@ -792,7 +792,11 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
     using C = Cfg<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    const int h = 16 * warp + lane;       // head owned by lanes 0..15 (M=64 TMEM layout)
+    // The M = 64 TMEM layout puts head 16w + l in lane l < 16 of warp w; lane
+    // l + 16 takes the second half of that head's columns of each tile
+    // (handed over by shuffles), so all 32 lanes share the exponentials.
+    const int h = 16 * warp + (lane & 15);
+    const int half = lane >> 4;
     const bool head_thread = lane < 16;
     const float cscale = kLog2e / sqrtf((float)D);
     const uint32_t tmem = ms->tmem;
@@ -829,13 +833,21 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
                     }
                 }
             }
+            // lanes 16..31: columns 16..31 of head h (and its tile maximum) from lane l - 16
+#pragma unroll
+            for (int j = 0; j < kTile / 2; ++j) {
+                const float t = __shfl_up_sync(0xffffffffu, s[kTile / 2 + j], 16);
+                if (half) s[j] = t;
+            }
+            mt = __shfl_sync(0xffffffffu, mt, lane & 15);
             tc_fence_before();
             mbar_arrive_warp(&ms->s_free[sb]);   // S[sb] may be overwritten by tile g + 2
             // PV of the previous tile must be done before P and O^T are touched.
             if (g > 0 && !warp_all(mbar_wait(&ms->pv_done, (g - 1) & 1, &ms->abort))) return;
             tc_fence_after();
             float f = 1.f;
-            if (head_thread) {
+            {
+                // both lanes of head h take the same decisions (same mt, m_run, l_run)
                 float mnew = m_run;
                 if (ti == 0) {
                     mnew = mt;
@@ -846,13 +858,14 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
                 const float muse = mnew == -INFINITY ? 0.f : mnew;
                 float lsum = 0.f;
 #pragma unroll
-                for (int c8 = 0; c8 < kTile / 8; ++c8) {
+                for (int c8l = 0; c8l < kTile / 16; ++c8l) {
+                    const int c8 = 2 * half + c8l;   // this lane's 8-column groups
                     const float4 ta = ts4[2 * c8], tb = ts4[2 * c8 + 1];
                     const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
                     float p[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        p[e] = exp2f(__fsub_rn(s[c8 * 8 + e], muse));
+                        p[e] = exp2f(__fsub_rn(s[c8l * 8 + e], muse));
                         lsum = __fadd_rn(lsum, p[e]);
                     }
                     uint4 u;
@@ -863,9 +876,11 @@ __device__ void softmax_role(const AttendArgs &a, int b, const Req &rq, Span sp,
                     const uint32_t off = (uint32_t)((h >> 3) * 1024 + (h & 7) * 128 + ((c8 ^ (h & 7)) << 4));
                     *reinterpret_cast<uint4 *>(pp + off) = u;
                 }
+                // the tile's sum: columns 0..15 plus columns 16..31 (the same on both lanes)
+                lsum = __fadd_rn(lsum, __shfl_xor_sync(0xffffffffu, lsum, 16));
                 l_run = (ti == 0) ? lsum : __fadd_rn(__fmul_rn(l_run, f), lsum);
                 m_run = mnew;
-                ms->fac[g & 1][h] = f;
+                if (head_thread) ms->fac[g & 1][h] = f;
             }
             // every head's factor is needed by every thread (each owns one O^T
             // row); a chunk's first tile has none (every factor is 1)

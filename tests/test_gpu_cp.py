@@ -86,6 +86,8 @@ def _run(w, plan, kv, ki, pin, p, seed_name):
     (CSA_CP, 3, [0, 400, 1001, 1500]),
     (CSA_CP8, 2, [0, 733, 1500]),
     (HCA_CP, 3, [0, 300, 811, 1300]),
+    (dataclasses.replace(CSA_CP, L=10000, name="cp_csa10k"), 4, [0, 2501, 4999, 7777, 10000]),
+    (dataclasses.replace(HCA_CP, L=6000, name="cp_hca6k"), 4, None),
 ])
 def test_cp_prefill_equals_one_piece(w, R, starts):
     N = w.L
