@@ -192,16 +192,20 @@ cudaError_t launch_attend(const AttendArgs &a, bool q_bf16, bool out_bf16, int v
                           cudaStream_t stream);
 
 // Canonical chunk length for a set of n rows (a function of n only):
-// 64 * ceil(n / 2048) rows, so a request never has more than 32 chunks, and
-// 320 rows for 1024 < n <= 4096 (top-k 1024 + window: 4 chunks, not 18 --
-// every chunk costs an H*D fp32 partial written and read back, which is
-// most of a query row's time when thousands of rows fill the GPU; decode at
-// top-k 512 keeps 64-row chunks, which spread few requests over the SMs).
+//   n <= 1024:         64 rows (decode at top-k 512: 10 chunks spread a few
+//                      requests over the SMs);
+//   1024 < n <= 4096:  320 rows (top-k 1024 + window: 4 chunks, not 18 --
+//                      every chunk costs an H*D fp32 partial written and
+//                      read back, most of a query row's time when thousands
+//                      of rows fill the GPU);
+//   n > 4096:          32 * ceil(n / 1024) rows, whole tiles, so that a long
+//                      HCA set has close to 32 chunks (8320 rows: 29 chunks
+//                      of 288, against 26 of 320 at 64-row granularity).
+// A request never has more than 32 chunks.
 __host__ __device__ inline int attend_chunk_rows(long long n) {
-    long long c = (n + 2047) / 2048;
-    if (c < 1) c = 1;
-    if (n > 1024 && n <= 4096) c = 5;
-    return (int)(64 * c);
+    if (n <= 1024) return 64;
+    if (n <= 4096) return 320;
+    return (int)(32 * ((n + 1023) / 1024));
 }
 __host__ __device__ inline int attend_num_chunks(long long n) {
     const int c = attend_chunk_rows(n);
