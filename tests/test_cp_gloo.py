@@ -167,6 +167,8 @@ def _rank_main(rank, world, port, kind, starts, ret):
     ("csa_e4m3_channel", 2, [0, 733, 1500]),       # E4M3 keys, per-channel gate
     ("hca", 2, [0, 645, 1300]),                    # HCA: a 128-token block across the boundary
     ("hca", 3, [0, 300, 811, 1300]),
+    ("csa", 4, [0, 300, 640, 1003, 1500]),        # boundary exactly at a page start (640)
+    ("hca", 4, [0, 256, 512, 1024, 1300]),         # boundaries at block starts: no open block to send
 ])
 def test_cp_prefill_on_gloo_ranks(kind, world, starts):
     port = _free_port()
