@@ -739,11 +739,15 @@ def run_steps(steps, inputs, W, K, e2e=False, profile=False):
     graph holding all of the step's library calls, captured beforehand; the
     K replays are bracketed by one pair of events after a synchronize.
     e2e: every step also copies its inputs from pinned host memory into the
-    device buffers the graph reads and copies its output back to pinned
-    host memory, all inside the timed region; the copies run on a second
-    stream, step i+1's inputs while step i computes (each step has its own
-    input buffers, and an output buffer is reused only R steps later), as a
-    serving loop would.  Returns ms per step."""
+    device buffers its calls read and copies its output back to pinned host
+    memory, all inside the timed region, as a serving loop would: step j's
+    graph holds, beside its library calls, a branch on a second stream that
+    copies step j+1's inputs in and step j-1's output out (each step has its
+    own input buffers, and an output buffer is reused only R steps later), so
+    the copies overlap the compute and one graph launch drives a whole step.
+    The first step's inputs are copied before the first replay and the last
+    output after the last, both inside the timed region.  Returns ms per
+    step."""
     import torch
     R = len(steps)
     for i in range(W):
@@ -752,10 +756,40 @@ def run_steps(steps, inputs, W, K, e2e=False, profile=False):
             c(inputs[i])
     torch.cuda.synchronize()
     graphs = []
-    for i in range(W, W + K):
-        st, x = steps[i % R], inputs[i]
-        graphs.append(capture(lambda: [c(x) for c in st.calls]))
-    outs = [torch.empty_like(steps[i % R].out, device="cpu").pin_memory() for i in range(W, W + K)] if e2e else None
+    outs = None
+    if e2e:
+        # step j-1's output is copied out while step j computes into another
+        # copy's output buffer: at least two output buffers
+        assert R >= 2, "the overlapped e2e copies need at least two output buffers"
+        outs = [torch.empty_like(steps[i % R].out, device="cpu").pin_memory() for i in range(W, W + K)]
+        cs = torch.cuda.Stream()
+        for j in range(K):
+            i = W + j
+            st, x = steps[i % R], inputs[i]
+            nxt = inputs[i + 1] if j + 1 < K else None
+            prev = (outs[j - 1], steps[(i - 1) % R].out) if j >= 1 else None
+
+            def body(st=st, x=x, nxt=nxt, prev=prev):
+                cur = torch.cuda.current_stream()
+                fork = torch.cuda.Event()
+                fork.record(cur)
+                cs.wait_event(fork)
+                with torch.cuda.stream(cs):
+                    if nxt is not None:
+                        for k, v in nxt["host"].items():
+                            nxt[k].copy_(v, non_blocking=True)
+                    if prev is not None:
+                        prev[0].copy_(prev[1], non_blocking=True)
+                for c in st.calls:
+                    c(x)
+                join = torch.cuda.Event()
+                join.record(cs)
+                cur.wait_event(join)
+            graphs.append(capture(body))
+    else:
+        for i in range(W, W + K):
+            st, x = steps[i % R], inputs[i]
+            graphs.append(capture(lambda: [c(x) for c in st.calls]))
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if profile:
@@ -763,36 +797,12 @@ def run_steps(steps, inputs, W, K, e2e=False, profile=False):
     main = torch.cuda.current_stream()
     e0.record(main)
     if e2e:
-        # step j+1's input copy is queued before step j's output copy on the
-        # copy stream, so step j's output buffer must not be written again by
-        # step j+1: it is reused only R >= 2 steps later
-        assert R >= 2, "the overlapped e2e copies need at least two output buffers"
-        cs = torch.cuda.Stream()
-        cs.wait_stream(main)   # every copy after the start event
-        ev_in = [torch.cuda.Event() for _ in range(K)]
-        ev_out = [torch.cuda.Event() for _ in range(K)]
-
-        def h2d(j):
-            x = inputs[W + j]
-            with torch.cuda.stream(cs):
-                for k, v in x["host"].items():
-                    x[k].copy_(v, non_blocking=True)
-                ev_in[j].record(cs)
-
-        def d2h(j):
-            with torch.cuda.stream(cs):
-                cs.wait_event(ev_out[j])
-                outs[j].copy_(steps[(W + j) % R].out, non_blocking=True)
-
-        h2d(0)
+        x0 = inputs[W]
+        for k, v in x0["host"].items():
+            x0[k].copy_(v, non_blocking=True)
         for j in range(K):
-            if j + 1 < K:
-                h2d(j + 1)
-            main.wait_event(ev_in[j])
             graphs[j].replay()
-            ev_out[j].record(main)
-            d2h(j)
-        main.wait_stream(cs)   # the last output is on the host
+        outs[K - 1].copy_(steps[(W + K - 1) % R].out, non_blocking=True)
     else:
         for j in range(K):
             graphs[j].replay()
