@@ -325,8 +325,9 @@ class PrefillStep:
     """One CSA prefill chunk of one request: the ring snapshot of the NW
     positions before the chunk, the chunk's append (T tokens, every token's
     window row kept), then the T queries (query i at position L0+i) through
-    the indexer, top-k and attention with per-row visible lengths and the
-    window rows from the chunk buffer.  A last pair of device copies puts the
+    the indexer and top-k (one csla_indexer_topk call: the rows' scores are
+    not stored) and attention with per-row visible lengths and the window
+    rows from the chunk buffer.  A last pair of device copies puts the
     request's length and ring back to their pre-chunk state, so that every
     step does the same work (the appended entries are rewritten with the same
     bytes)."""
@@ -352,14 +353,33 @@ class PrefillStep:
         self.idx = torch.zeros((T, k), dtype=torch.int32, device=device)
         self.out = torch.zeros((T, kw["H"], kw["D"]), dtype=torch.bfloat16, device=device)
         cfg = lb.cfg()
-        self.wsi = C.csla_workspace_size(cfg, C.CSLA_OP_INDEXER, T, self.max_len)
+        self.wsi = C.csla_workspace_size(cfg, C.CSLA_OP_INDEXER_TOPK, T, self.max_len)
         self.wsa = C.csla_workspace_size(cfg, C.CSLA_OP_CSA_ATTEND, T, k)
         self.ws_i = torch.zeros(self.wsi, dtype=torch.uint8, device=device)
         self.ws_a = torch.zeros(self.wsa, dtype=torch.uint8, device=device)
         self.len0, self.win0, self.wsc0 = lb.len.clone(), lb.win_rows.clone(), lb.win_scales.clone()
         self.cfg, self.st, self.cache, self.cps = cfg, lb.state(), lb.cache(), cp.struct()
-        self.names = ["window_rows", "compress_append", "indexer_scores", "topk_select", "csa_attend", "rewind"]
-        self.calls = [self._snapshot, self._compress, self._indexer, self._topk, self._attend, self._rewind]
+        self.names = ["window_rows", "compress_append", "indexer_topk", "csa_attend", "rewind"]
+        self.calls = [self._snapshot, self._compress, self._indexer_topk, self._attend, self._rewind]
+        # the same selection as two calls (scores stored, then read), timed beside it
+        self.two_call_names = ["indexer_scores", "topk_select"]
+        self.two_calls = [self._indexer, self._topk]
+
+    def selection_stats(self):
+        """Rows that fell back to stored scores, and the candidate counts of
+        the others (read from the csla_indexer_topk workspace: query terms,
+        sample scores, thresholds, four counts per row, flags)."""
+        import numpy as np
+        import torch
+        up16 = lambda x: (x + 15) // 16 * 16
+        T, kw = self.T, self.kw
+        nq = (3 * kw["HI"] + 15) // 16 * 16
+        o_cnt = up16(T * nq * kw["dI"] * 2) + up16(T * 1024 * 4) + up16(T * 4)
+        o_flag = o_cnt + up16(T * 16)
+        cnt = self.ws_i[o_cnt:o_cnt + 16 * T].view(torch.int32).cpu().numpy().reshape(T, 4).sum(axis=1)
+        flag = self.ws_i[o_flag:o_flag + 4 * T].view(torch.int32).cpu().numpy()
+        ok = flag == 0
+        return int((~ok).sum()), float(np.mean(cnt[ok])) if ok.any() else 0.0, int(cnt.max())
 
     def _snapshot(self, x):
         self.C.csla_window_rows(self.cfg, self.st, self.slot, 1, NW, self.buf, self.bufsc, NW + self.T)
@@ -374,6 +394,12 @@ class PrefillStep:
         C.csla_indexer_scores(self.cfg, self.st, self.cache, self.rows_slots, self.T, self.max_len, x["cq"],
                               C.CSLA_BF16, self.p["W_iq"], C.CSLA_BF16, x["head_w"], self.scores, self.stride,
                               self.ws_i, self.wsi, qs=self.qs_rows)
+
+    def _indexer_topk(self, x):
+        C = self.C
+        C.csla_indexer_topk(self.cfg, self.st, self.cache, self.rows_slots, self.T, self.max_len, x["cq"],
+                            C.CSLA_BF16, self.p["W_iq"], C.CSLA_BF16, x["head_w"], self.kw["k"], self.idx,
+                            self.scores, self.stride, self.ws_i, self.wsi, qs=self.qs_rows)
 
     def _topk(self, x):
         self.C.csla_topk_select(self.cfg, self.st, self.rows_slots, self.T, self.max_len, self.scores, self.stride,
@@ -436,8 +462,13 @@ def prefill_leg(W, K, seed, rank, world, device, variant, profile=False):
         torch.cuda.profiler.stop()
     ms = dp_max(e0.elapsed_time(e1) / K, world, device)
     del g
-    # per-call times: each call its own graph, one event pair around each replay
-    gs = [capture(lambda c=c: c(x)) for c in st.calls]
+    fb_rows, cand_mean, cand_max = st.selection_stats()
+    # per-call times: each call its own graph, one event pair around each
+    # replay; the two-call selection, for comparison, right after the fused
+    # call (before the rewind, which leaves the queries past the length)
+    order = st.calls[:3] + st.two_calls + st.calls[3:]
+    order_names = st.names[:3] + st.two_call_names + st.names[3:]
+    gs = [capture(lambda c=c: c(x)) for c in order]
     seg = [0.0] * len(gs)
     for _ in range(max(1, K // 2)):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(gs) + 1)]
@@ -452,14 +483,17 @@ def prefill_leg(W, K, seed, rank, world, device, variant, profile=False):
     fi, fa = st.flops()
     tpk, tkind = tensor_peak()
     tf = (fi + fa) / (ms * 1e-3) / 1e12
+    sg = dict(zip(order_names, seg))
     out = {"workload": "csa_prefill_T4096_L262144", "tokens_per_s": T * world / (ms * 1e-3), "ms_per_chunk": ms,
            "queries": T, "prefix": L0, "topk": kw["k"],
-           "segments_ms": dict(zip(st.names, seg)),
+           "segments_ms": {n: sg[n] for n in st.names},
+           "two_call_selection_ms": {n: sg[n] for n in st.two_call_names},
+           "selection": {"fallback_rows": fb_rows, "mean_candidates": cand_mean, "max_candidates": cand_max},
            "algorithmic_tflop": (fi + fa) / 1e12, "indexer_tflop": fi / 1e12, "attend_tflop": fa / 1e12,
            "tensor_tflops": tf, "tensor_peak": tpk, "tensor_peak_kind": tkind, "tensor_frac": tf / tpk,
-           "indexer_tensor_frac": fi / (seg[2] * 1e-3) / 1e12 / tpk,
-           "attend_tensor_frac": fa / (seg[4] * 1e-3) / 1e12 / tpk,
-           "l2": "inputs larger than L2 (q 268 MB, fp32 scores 1.09 GB per chunk)",
+           "indexer_topk_tensor_frac": fi / (sg["indexer_topk"] * 1e-3) / 1e12 / tpk,
+           "attend_tensor_frac": fa / (sg["csa_attend"] * 1e-3) / 1e12 / tpk,
+           "l2": "inputs larger than L2 (q 268 MB; the rows' scores are not stored)",
            "launch": "one CUDA graph per chunk, K replays between one event pair"}
     del st, lb
     torch.cuda.empty_cache()

@@ -17,13 +17,14 @@ CSLA_VARIANT_AUTO, CSLA_VARIANT_SATURATED, CSLA_VARIANT_STARVED = 0, 1, 2
 CSLA_KEY_BF16, CSLA_KEY_E4M3 = 0, 1
 CSLA_GATE_TOKEN, CSLA_GATE_CHANNEL = 0, 1
 CSLA_OP_INDEXER, CSLA_OP_TOPK, CSLA_OP_CSA_ATTEND, CSLA_OP_HCA_ATTEND, CSLA_OP_CSA_DECODE_STEP = 1, 2, 3, 4, 5
+CSLA_OP_INDEXER_TOPK = 6
 CSLA_DEVERR_PAGE, CSLA_DEVERR_INDEX, CSLA_DEVERR_LEN, CSLA_DEVERR_TIMEOUT, CSLA_DEVERR_RANGE = 1, 2, 4, 8, 16
 CSLA_PAGE_TOKENS = 128
 
 EXPORTS = ("csla_compress_append", "csla_indexer_scores", "csla_topk_select", "csla_csa_attend",
            "csla_hca_attend", "csla_workspace_size", "csla_device_error", "csla_strerror", "csla_version",
            "csla_indexer_scores_noalloc", "csla_window_rows", "csla_csa_decode_step", "csla_check_wait_timeout",
-           "csla_cp_record_bytes", "csla_cp_select", "csla_cp_place")
+           "csla_cp_record_bytes", "csla_cp_select", "csla_cp_place", "csla_indexer_topk")
 CSLA_CP_MAX_RANKS = 64
 CSLA_NOALLOC_INDEXER_SCRATCH_BYTES = 786432
 
@@ -97,6 +98,7 @@ def _load():
         "csla_window_rows": [P, P, P, I, I, P, P, I, P],
         "csla_indexer_scores": [P, P, P, P, I, P, I, P, I, P, I, P, P, I, P, Z, P],
         "csla_topk_select": [P, P, P, I, P, I, P, I, I, P, P],
+        "csla_indexer_topk": [P, P, P, P, I, P, I, P, I, P, I, P, I, P, P, I, P, Z, P],
         "csla_csa_attend": [P, P, P, P, I, P, P, I, P, I, P, P, P, I, I, P, Z, P],
         "csla_hca_attend": [P, P, P, P, I, P, I, P, I, P, P, P, I, I, P, Z, P],
         "csla_workspace_size": [P, I, I, I],
@@ -183,6 +185,16 @@ def csla_topk_select(cfg, st, slots, B, max_len, scores, scores_stride, k, idx, 
     return _check("csla_topk_select", _lib.csla_topk_select(
         _ref(cfg), _ref(st), _ptr(slots), B, _ref(qs), max_len, _ptr(scores), scores_stride, k, _ptr(idx),
         _stream(stream)))
+
+
+def csla_indexer_topk(cfg, st, cache, slots, B, max_len, cq, cq_dtype, W_iq, w_dtype, head_w, k, idx, scores,
+                      scores_stride, workspace, workspace_bytes, stream=None, qs=None):
+    """csla_indexer_scores + csla_topk_select in one call (same idx); the
+    scores of long rows are not stored (`scores` is scratch for rows that
+    fall back to the two-step path)."""
+    return _check("csla_indexer_topk", _lib.csla_indexer_topk(
+        _ref(cfg), _ref(st), _ref(cache), _ptr(slots), B, _ref(qs), max_len, _ptr(cq), cq_dtype, _ptr(W_iq), w_dtype,
+        _ptr(head_w), k, _ptr(idx), _ptr(scores), scores_stride, _ptr(workspace), workspace_bytes, _stream(stream)))
 
 
 def csla_csa_attend(cfg, st, cache, slots, B, q, q_dtype, idx, k, sink, gamma_q, out, out_dtype, variant,

@@ -179,6 +179,25 @@ const char *csla_strerror(int s) {
     }
 }
 
+// csla_indexer_topk workspace: the indexer's query terms, then sample
+// scores [B][kSampleCols], thresholds [B], candidate counts [B][kCandSub],
+// row flags [B] and candidates [B][kCandCap] (key, entry), each part
+// 16-byte aligned.
+struct ItkLayout {
+    size_t sample, t0, cnt, flag, cand, total;
+};
+static size_t up16(size_t x) { return (x + 15) / 16 * 16; }
+static ItkLayout itk_layout(int B, int NQ, int dI) {
+    ItkLayout l;
+    l.sample = up16((size_t)B * NQ * dI * 2);
+    l.t0 = l.sample + up16((size_t)B * kSampleCols * 4);
+    l.cnt = l.t0 + up16((size_t)B * 4);
+    l.flag = l.cnt + up16((size_t)B * kCandSub * 4);
+    l.cand = l.flag + up16((size_t)B * 4);
+    l.total = l.cand + (size_t)B * kCandCap * 8;
+    return l;
+}
+
 size_t csla_workspace_size(const csla_cfg *cfg, int32_t op, int32_t B, int32_t max_len) {
     if (check_cfg(cfg) != CSLA_OK || B < 1 || max_len < 0) return 0;
     switch (op) {
@@ -190,6 +209,9 @@ size_t csla_workspace_size(const csla_cfg *cfg, int32_t op, int32_t B, int32_t m
         case CSLA_OP_HCA_ATTEND: return attend_ws(cfg, B, (long long)max_len / cfg->m + cfg->n_win);
         case CSLA_OP_CSA_DECODE_STEP:
             return attend_ws(cfg, B, (long long)max_len + cfg->n_win) + ((size_t)B * 4 + 15) / 16 * 16;
+        case CSLA_OP_INDEXER_TOPK:
+            if (check_csa_indexer_shape(cfg) != CSLA_OK) return 0;
+            return itk_layout(B, nq_of(cfg->HI), cfg->dI).total;
         default: return 0;
     }
 }
@@ -378,6 +400,60 @@ int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *s
     const int rc = prep_topk(cfg, st, slots, B, qs, max_len, scores, scores_stride, k, idx, &a);
     if (rc) return rc;
     return cuda_status(launch_topk(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int csla_indexer_topk(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,
+                      int32_t B, const csla_queries *qs, int32_t max_len, const void *cq, int32_t cq_dtype,
+                      const void *W_iq, int32_t w_dtype, const float *head_w, int32_t k, int32_t *idx,
+                      float *scores, int32_t scores_stride, void *workspace, size_t workspace_bytes,
+                      csla_stream_t stream) {
+    if (k < 1 || k > 2048) return CSLA_ERR_ARG;
+    if (workspace_bytes < csla_workspace_size(cfg, CSLA_OP_INDEXER_TOPK, B, max_len)) return CSLA_ERR_ARG;
+    TopkArgs t;
+    int rc = prep_topk(cfg, st, slots, B, qs, max_len, scores, scores_stride, k, idx, &t);
+    if (rc) return rc;
+    IndexerLaunch L;
+    rc = prep_indexer(cfg, st, cache, slots, B, qs, max_len, cq, cq_dtype, W_iq, w_dtype, head_w, scores,
+                      scores_stride, workspace, workspace_bytes, &L);
+    if (rc) return rc;
+    const ItkLayout l = itk_layout(B, L.a.NQ, cfg->dI);
+    uint8_t *w = reinterpret_cast<uint8_t *>(workspace);
+    CandArgs c{};
+    c.sample = reinterpret_cast<const float *>(w + l.sample);
+    c.page_step = (L.a.tiles_per_req * 4 + 31) / 32;   // 32 sample pages spread over the longest row
+    if (c.page_step < 1) c.page_step = 1;
+    c.cand_t0 = reinterpret_cast<uint32_t *>(w + l.t0);
+    c.cand_cnt = reinterpret_cast<int32_t *>(w + l.cnt);
+    c.row_flag = reinterpret_cast<int32_t *>(w + l.flag);
+    c.cand = reinterpret_cast<const uint2 *>(w + l.cand);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int nsm = num_sms_current();
+    // 1. projection, then the sample pass (scores of the sample tiles only)
+    IndexerArgs as = L.a;
+    as.page_step = c.page_step;
+    as.scores = reinterpret_cast<float *>(w + l.sample);
+    as.scores_stride = kSampleCols;
+    cudaError_t e = launch_indexer(as, L.cq_bf16, L.w_bf16, L.kmap, L.qmap, nsm, s, true, L.gemm ? &L.pm : nullptr);
+    // 2. thresholds; 3. candidate pass; 4. selection among the candidates
+    if (e == cudaSuccess) e = launch_cand_threshold(t, c, s);
+    IndexerArgs ac = L.a;
+    ac.cand_t0 = c.cand_t0;
+    ac.cand = reinterpret_cast<uint2 *>(w + l.cand);
+    ac.cand_cnt = c.cand_cnt;
+    ac.cand_cap = kCandCap / kCandSub;
+    if (e == cudaSuccess) e = launch_indexer(ac, L.cq_bf16, L.w_bf16, L.kmap, L.qmap, nsm, s, false);
+    if (e == cudaSuccess) e = launch_cand_select(t, c, s);
+    // 5. flagged rows: scores stored (kPersistSlices CTAs per row group,
+    //    each a run of tiles; groups without a flagged row exit at once),
+    //    then the top-k on them
+    IndexerArgs af = L.a;
+    af.persist = kPersistSlices;
+    af.row_flag = c.row_flag;
+    if (e == cudaSuccess) e = launch_indexer(af, L.cq_bf16, L.w_bf16, L.kmap, L.qmap, nsm, s, false);
+    TopkArgs tf = t;
+    tf.row_flag = c.row_flag;
+    if (e == cudaSuccess) e = launch_topk(tf, s);
+    return cuda_status(e);
 }
 
 static int prep_attend(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache, const int32_t *slots,

@@ -25,6 +25,20 @@ extern __device__ unsigned int g_dev_err;
 __device__ __forceinline__ void set_dev_err(unsigned bits) { atomicOr(&g_dev_err, bits); }
 
 // ------------------------------------------------------------ number formats
+// Order-preserving unsigned key of an fp32 score (-0.0 folded onto +0.0):
+// a > b as floats exactly when score_key(a) > score_key(b).  The top-k
+// selector and the indexer's candidate output compare scores through it.
+__device__ __forceinline__ uint32_t score_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+// The score whose key is `key` (key 0, below every score's key: -inf).
+__device__ __forceinline__ float key_score(uint32_t key) {
+    if (key == 0u) return -__int_as_float(0x7f800000);
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
 
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {

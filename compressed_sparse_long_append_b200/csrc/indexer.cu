@@ -263,6 +263,15 @@ __device__ __forceinline__ void split_q_e4m3(float (&q)[4], uint8_t *qb, int bas
     }
 }
 
+// A warp's candidates of one (row, tile) whose list places are still to be
+// read from the row counter (lane 0's `at`).
+struct Pending {
+    unsigned mq = 0u;
+    bool q = false;
+    uint32_t key = 0u;
+    int e = 0, row = 0, at = 0;
+};
+
 // CTA (blockIdx.x, blockIdx.y) scores tiles [blockIdx.x*kTPC, +kTPC) (128
 // entries each) of the query rows r0 = blockIdx.y*G .. r0+G-1, which all
 // read the keys of request slots[r0]: one key tile feeds one MMA of N = G*NQ
@@ -293,10 +302,19 @@ __global__ void __launch_bounds__(idx_threads<G>())
     int *row_lo = row_nv + G;                                    // [G] first entry scored
     float *hw = reinterpret_cast<float *>(row_lo + G);           // [G][HI] head weights
     float *sig = hw + G * HI;                                    // [G][NQ] E4M3 query-term scales
+    float *row_t0 = sig + G * NQ;                                // [G] candidate thresholds (scores)
     __shared__ volatile int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r0 = blockIdx.y * G;
+    if (a.persist && a.row_flag) {
+        // the fallback of a streaming selection: most row groups have no
+        // flagged row, so look before taking barriers and TMEM
+        pdl_wait();
+        int any = 0;
+        if (threadIdx.x < G && r0 + threadIdx.x < a.B) any = a.row_flag[r0 + threadIdx.x] != 0;
+        if (!__syncthreads_or(any)) return;
+    }
     const int slot = __ldg(a.slots + r0);
     const bool slot_ok = slot >= 0 && slot < a.n_slots;
     __shared__ int s_t0;   // range 2: first tile of the request's new entries
@@ -316,10 +334,12 @@ __global__ void __launch_bounds__(idx_threads<G>())
         mbar_init(qfull, kE4M3 ? 4 * idx_epi_sets<G>() : 1);
         fence_mbar_init();
     }
+    // page j of this CTA (j < 4*kTPC) is page (4*kTPC*x + j)*Z of the request
+    const int Z = a.page_step > 1 ? a.page_step : 1;
     int pg = -1;   // warp 0: page id of this CTA's page `lane`
     if (warp == 0) {
-        const int col = (blockIdx.x * kTPC * kTileE + lane * kPageE) / kPageE;
-        if (a.range != 2 && slot_ok && lane < kTPC * 4 && col < a.bt_stride)
+        const int col = (blockIdx.x * kTPC * 4 + lane) * Z;
+        if (!a.persist && a.range != 2 && slot_ok && lane < kTPC * 4 && col < a.bt_stride)
             pg = __ldg(a.block_table + (size_t)slot * a.bt_stride + col);
         if (lane == 0) {
             tma_prefetch_desc(&kmap);
@@ -366,26 +386,32 @@ __global__ void __launch_bounds__(idx_threads<G>())
                         lo = a.len0[r] / a.m;
                         if (lo >= nv) nv = -1;
                     }
+                    if (a.row_flag && a.row_flag[r] == 0) nv = -1;
                 }
             }
         }
         row_nv[threadIdx.x] = nv;
         row_lo[threadIdx.x] = lo;
+        row_t0[threadIdx.x] = key_score((a.cand_t0 && r < a.B) ? a.cand_t0[r] : 0u);
         if (threadIdx.x == 0) s_t0 = a.range == 2 ? lo / kTileE : 0;
     }
     __syncthreads();
-    const int t_begin = blockIdx.x * kTPC + s_t0;
+    // persist: CTA x walks tiles [x*run, (x+1)*run) of the request
+    const int run = a.persist ? (a.tiles_per_req + a.persist - 1) / a.persist : kTPC;
+    const int t_begin = a.persist ? blockIdx.x * run : blockIdx.x * kTPC + s_t0;
     int nv_max = 0;
 #pragma unroll
     for (int g = 0; g < G; ++g) nv_max = max(nv_max, row_nv[g]);
-    const int n_tiles = min(kTPC, (nv_max + kTileE - 1) / kTileE - t_begin);
+    const int pages_row = (nv_max + kPageE - 1) / kPageE;
+    // tiles with an entry to score: of 4 consecutive pages, or (sample) of 4 pages Z apart
+    const int n_tiles = min(run, ((pages_row + Z - 1) / Z + 3) / 4 - t_begin);
     if (a.range == 2 && warp == 0) {
         const int col = (t_begin * kTileE + lane * kPageE) / kPageE;
         if (slot_ok && lane < kTPC * 4 && col < a.bt_stride)
             pg = __ldg(a.block_table + (size_t)slot * a.bt_stride + col);
     }
-    if (warp == 0 && lane < kTPC * 4) {
-        const int e0 = t_begin * kTileE + lane * kPageE;
+    if (!a.persist && warp == 0 && lane < kTPC * 4) {
+        const int e0 = ((t_begin * 4 + lane) * Z) * kPageE;
         if (e0 < nv_max && (pg < 0 || pg >= a.n_pages)) {
             set_dev_err(CSLA_DEVERR_PAGE);
             pg = -1;
@@ -393,6 +419,22 @@ __global__ void __launch_bounds__(idx_threads<G>())
         pages[lane] = e0 < nv_max ? pg : -1;
     }
     __syncthreads();   // the epilogue warps read pages[] too (entries of a bad page stay unscored)
+    // Page id of page p (< 4) of this CTA's tile t, -1 when it holds no
+    // entry to score or lies outside the pool: from pages[] for the kTPC
+    // tiles of a CTA, read from the block table per tile when a CTA walks a
+    // longer run (persist: Z = 1).
+    auto page_id = [&](int t, int p, bool report) -> int {
+        if (!a.persist) return pages[t * 4 + p];
+        const int e0 = (t_begin + t) * kTileE + p * kPageE;
+        if (e0 >= nv_max) return -1;
+        const int col = e0 / kPageE;
+        const int q = col < a.bt_stride ? __ldg(a.block_table + (size_t)slot * a.bt_stride + col) : -1;
+        if (q < 0 || q >= a.n_pages) {
+            if (report) set_dev_err(CSLA_DEVERR_PAGE);
+            return -1;
+        }
+        return q;
+    };
 
     if (n_tiles <= 0) {
         // nothing to score: fall through to the teardown
@@ -408,13 +450,16 @@ __global__ void __launch_bounds__(idx_threads<G>())
                 const int s = n % kStages;
                 if (n >= kStages && !mbar_wait(empty + s, ((n / kStages) - 1) & 1, &abort_flag)) break;
                 uint8_t *kb = base + s * S::kKeyBytes;
-                int np = 0;
+                int tp[4], np = 0;
 #pragma unroll
-                for (int p = 0; p < 4; ++p) np += pages[t * 4 + p] >= 0;
+                for (int p = 0; p < 4; ++p) {
+                    tp[p] = page_id(t, p, true);
+                    np += tp[p] >= 0;
+                }
                 mbar_arrive_expect_tx(full + s, (uint32_t)(np * kPageE * DI * S::kElt));
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
-                    const int pg = pages[t * 4 + p];
+                    const int pg = tp[p];
                     if (pg < 0) continue;
                     if constexpr (kE4M3) {
                         // one 128-byte box per entry row (the whole E4M3 key)
@@ -502,19 +547,38 @@ __global__ void __launch_bounds__(idx_threads<G>())
             // the term scales are read by every epilogue warp
             asm volatile("bar.sync 1, %0;" ::"r"(128 * kSets) : "memory");
         }
+        // Candidate output: a warp's candidates of one (row, tile) take
+        // their places in the row's sub-list of this warp's entries
+        // ((entry/32) % 4 = warp % 4: four counters per row share the
+        // updates) from one counter update.  When a set scores one row per
+        // tile, the update of a tile is issued and its places used at the
+        // next tile (or after the last), so that the counter's round trip
+        // overlaps a tile of work.
+        constexpr bool kDefer = kSets >= G;
+        Pending pend;
+        auto flush = [&]() {
+            if (pend.mq) {
+                const int at = __shfl_sync(0xffffffffu, pend.at, 0) + __popc(pend.mq & ((1u << lane) - 1u));
+                if (pend.q && at < a.cand_cap)
+                    a.cand[(size_t)pend.row * a.cand_cap + at] = make_uint2(pend.key, (uint32_t)pend.e);
+                pend.mq = 0u;
+            }
+        };
         for (int t = 0, n = 0; t < n_tiles; ++t, ++n) {
             const int acc = n & 1;
             float ksc = 0.f;   // E4M3: this row's entry scale, loaded before the accumulator wait
+            const int pgr = page_id(t, row / kPageE, false);
             if constexpr (kE4M3) {
-                const int pgr = pages[t * 4 + row / kPageE];
                 if (pgr >= 0) ksc = __ldg(a.kscale + (size_t)pgr * kPageE + row % kPageE);
             }
             if (!warp_all(mbar_wait(tfull + acc, (n / 2) & 1, &abort_flag))) break;
             tc_fence_after();
-            const int e = (t_begin + t) * kTileE + row;
+            const int tile_e0 = (t_begin + t) * 4 * Z * kPageE;          // the tile's first entry
+            const int e = (((t_begin + t) * 4 + row / kPageE) * Z) * kPageE + row % kPageE;
+            const int col_out = (t_begin + t) * kTileE + row;            // its score column (e unless sampling)
             int last = -1;   // this set's last row with entries in the tile (warp-uniform)
             for (int g = es; g < G; g += kSets)
-                if (row_nv[g] > (t_begin + t) * kTileE) last = g;
+                if (row_nv[g] > tile_e0) last = g;
             if (last < 0) {
                 tc_fence_before();
                 mbar_arrive_warp(tempty + acc);
@@ -522,7 +586,7 @@ __global__ void __launch_bounds__(idx_threads<G>())
 #pragma unroll 1
             for (int g = es; g <= last; g += kSets) {
                 const int nv = row_nv[g];
-                if (nv <= (t_begin + t) * kTileE) continue;   // the whole tile is past this row (warp-uniform)
+                if (nv <= tile_e0) continue;   // the whole tile is past this row (warp-uniform)
                 uint32_t r[NQ];
                 const uint32_t ta = tmem + ((uint32_t)lane_base << 16) + acc * N + g * NQ;
                 if constexpr (NQ == 16) {
@@ -548,8 +612,9 @@ __global__ void __launch_bounds__(idx_threads<G>())
                     mbar_arrive_warp(tempty + acc);
                 }
                 // entries of a page outside the pool were not loaded: leave them unscored
-                if (e < nv && e >= row_lo[g] && pages[t * 4 + row / kPageE] >= 0) {
-                    float sc = 0.f;
+                const bool valid = e < nv && e >= row_lo[g] && pgr >= 0;
+                float sc = 0.f;
+                if (valid) {
                     if constexpr (kE4M3) {
                         // head j: sum_t sig_t * acc_t (terms in order), then
                         // the entry's power-of-two key scale (ReLU commutes with it)
@@ -571,12 +636,28 @@ __global__ void __launch_bounds__(idx_threads<G>())
                             sc = __fmaf_rn(hw[g * HI + j], fmaxf(dot, 0.f), sc);
                         }
                     }
-                    a.scores[(size_t)(r0 + g) * a.scores_stride + e] = sc;
+                }
+                if (a.cand_t0) {
+                    // the entries at or above the row's threshold (warp-uniform
+                    // mask; the float order is the key order, -0 == +0)
+                    const bool q = valid && sc >= row_t0[g];
+                    const unsigned mq = __ballot_sync(0xffffffffu, q);
+                    if constexpr (kDefer) flush();
+                    pend.mq = mq;
+                    pend.q = q;
+                    pend.key = score_key(sc);
+                    pend.e = e;
+                    pend.row = (r0 + g) * kCandSub + (warp & 3);
+                    if (mq && lane == 0) pend.at = atomicAdd(a.cand_cnt + pend.row, __popc(mq));
+                    if constexpr (!kDefer) flush();
+                } else if (valid) {
+                    a.scores[(size_t)(r0 + g) * a.scores_stride + col_out] = sc;
                 }
             }
             if (threadIdx.x == 64 && t == 0) CSLA_TL_MARK_ANY(2);
             if (threadIdx.x == 64 && t == kTPC - 1) CSLA_TL_MARK_ANY(3);
         }
+        flush();
     }
     tc_fence_before();
     __syncthreads();
@@ -601,7 +682,10 @@ cudaError_t launch_indexer_t(const IndexerArgs &a, const CUtensorMap &kmap, cons
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
-    const int groups = (a.tiles_per_req + kTPC - 1) / kTPC;
+    // tiles a row group walks: all of the request's, or (sample) tiles of 4
+    // pages page_step apart; persist: `persist` CTAs per row group
+    const int Z = a.page_step > 1 ? a.page_step : 1;
+    const int groups = a.persist ? a.persist : (((a.tiles_per_req * 4 + Z - 1) / Z + 3) / 4 + kTPC - 1) / kTPC;
     return launch_pdl(indexer_kernel<DI, NQ, HI, G, kE4M3>, dim3(groups, (a.B + G - 1) / G),
                       dim3(idx_threads<G>()), S::kBytes, stream, a, kmap, qmap);
 }

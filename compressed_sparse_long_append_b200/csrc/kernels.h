@@ -114,6 +114,18 @@ struct IndexerArgs {
     int rows_per_cta;       // 1, or indexer_rows_per_cta(NQ) when all rows share slots[0]
     int range;              // 0: all visible entries; 1: those below len0[b]/m; 2: those from len0[b]/m on
     const int32_t *len0;    // [B] length of row b's request before the step's append (range 1, 2)
+    // Streaming selection (csla_indexer_topk); all zero/null for a plain call.
+    int page_step;          // > 1 (range 0, sample): the CTA's pages are the request's pages
+                            //   (32x + j)*page_step, j < 32, in 8 tiles of 4; entry i of its j-th
+                            //   page goes to score column 32*(32x + j) + i
+    int persist;            // > 0 (range 0): `persist` CTAs per row group (grid.x) each walk a
+                            //   contiguous run of tiles, page ids read per tile; a CTA whose rows
+                            //   are all unflagged (row_flag) exits before it sets anything up
+    const uint32_t *cand_t0;   // candidate output: entries whose score_key >= cand_t0[b] are appended,
+    uint2 *cand;               //   as (key, entry), to sub-list j = (entry/32) % 4 of row b:
+    int32_t *cand_cnt;         //   cand[(4b + j) * cand_cap + ..] (any order), cand_cnt[4b + j] counting
+    int cand_cap;              //   them all, also past cand_cap (per sub-list); nothing goes to `scores`
+    const int32_t *row_flag;   // rows with row_flag[b] == 0 are not scored
 };
 // len0[b] = len[slots[b]] (0 for a slot outside the pool).
 cudaError_t launch_len_snapshot(const int32_t *slots, const int32_t *len, int B, int n_slots, int32_t *len0,
@@ -147,8 +159,30 @@ struct TopkArgs {
     int m, k, B, max_n, n_slots;
     int32_t *idx;
     const int32_t *q_len;   // optional per-row visible length (else len[slot])
+    const int32_t *row_flag;   // rows with row_flag[b] == 0 are left alone (their idx untouched)
 };
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream);
+
+// Streaming selection (csla_indexer_topk), around the indexer's sample and
+// candidate passes.  Per row b of a TopkArgs `t`:
+//  threshold: cand_t0[b] from the sample scores (32 pages of 32 entries,
+//    page_step apart: 1024 columns per row), cand_cnt[b] = 0;
+//  select: the top-k from the cand_cnt[b] candidates when k <= cand_cnt[b]
+//    <= cand_cap (row_flag[b] = 0), else row_flag[b] = 1 and idx untouched.
+constexpr int kCandCap = 8192;        // candidates kept per row (4 sub-lists of 2048)
+constexpr int kCandSub = 4;
+constexpr int kSampleCols = 1024;     // sample scores per row (32 pages)
+constexpr int kPersistSlices = 4;     // CTAs per row group in the stored-score fallback
+struct CandArgs {
+    const float *sample;
+    int page_step;
+    uint32_t *cand_t0;
+    const uint2 *cand;
+    int32_t *cand_cnt;
+    int32_t *row_flag;
+};
+cudaError_t launch_cand_threshold(const TopkArgs &t, const CandArgs &c, cudaStream_t stream);
+cudaError_t launch_cand_select(const TopkArgs &t, const CandArgs &c, cudaStream_t stream);
 
 // Attention over the canonical row set of each request: compressed entries
 // (top-k list or all visible) then the window, reduced in fixed chunks.

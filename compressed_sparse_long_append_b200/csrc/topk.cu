@@ -15,6 +15,7 @@
 // sampled threshold, with a radix select over every key as the fallback.
 
 #include <cooperative_groups.h>
+#include <cstddef>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -25,12 +26,6 @@ namespace csla {
 namespace {
 
 constexpr int kBins = 2048;
-
-__device__ __forceinline__ uint32_t score_key(float f) {
-    uint32_t u = __float_as_uint(f);
-    if (u == 0x80000000u) u = 0u;
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 // ---------------------------------------------------------------- selection with scores in registers
 // The steps, as first written for one CTA of 512 threads (the cluster
@@ -93,7 +88,8 @@ __device__ __forceinline__ int warp_prefix(const int *v, int warp, int *total) {
 
 // The bin of sh.hist[0..nb) holding the krem-th largest key (counted from
 // the top): sh.sel_bin, and the rank within it: sh.sel_krem.  All threads.
-__device__ void pick_bin_r(RegShared &sh, int nb, int krem) {
+template <typename SH>
+__device__ void pick_bin_r(SH &sh, int nb, int krem) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // thread t covers bins nb-1-t*per .. (highest first); per = 0 for t beyond nb
     const int per = (nb + kRThreads - 1) / kRThreads;
@@ -134,8 +130,8 @@ __device__ void pick_bin_r(RegShared &sh, int nb, int krem) {
 // share their top 32 - bits bits with `prefix`; *krem_out = how many keys
 // equal to the result are within that rank.  Digits of up to 11 bits, from
 // the top of the `bits` low bits down.
-template <typename Each>
-__device__ uint32_t radix_select(RegShared &sh, const Each &each, int rank, uint32_t prefix, int bits,
+template <typename SH, typename Each>
+__device__ uint32_t radix_select(SH &sh, const Each &each, int rank, uint32_t prefix, int bits,
                                  int *krem_out) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t pmask = bits >= 32 ? 0u : ~((1u << bits) - 1u);
@@ -260,6 +256,7 @@ __global__ void __cluster_dims__(kG, 1, 1) __launch_bounds__(kRThreads, 1) topk_
     }
     const int k = a.k;
     int32_t *out = a.idx + (size_t)b * k;
+    if (a.row_flag && a.row_flag[b] == 0) return;   // the same decision in every CTA of the cluster
     if (n <= k) {   // the same decision in every CTA of the cluster
         if (cr == 0)
             for (int j = threadIdx.x; j < k; j += kRThreads) out[j] = j < n ? j : -1;
@@ -541,6 +538,7 @@ __global__ void __launch_bounds__(kRThreads, 2) topk_stream_kernel(TopkArgs a) {
     }
     const int k = a.k;
     int32_t *out = a.idx + (size_t)b * k;
+    if (a.row_flag && a.row_flag[b] == 0) return;
     if (n <= k) {
         for (int j = threadIdx.x; j < k; j += kRThreads) out[j] = j < n ? j : -1;
         return;
@@ -712,6 +710,200 @@ __global__ void __launch_bounds__(kRThreads, 2) topk_stream_kernel(TopkArgs a) {
     CSLA_TL_MARK(4);
 }
 
+// ---------------------------------------------------------------- streaming selection (csla_indexer_topk)
+// The indexer scores the long rows without storing their scores.  A sample
+// pass scores 32 pages (32 entries each) of each row, spread evenly
+// (page_step apart); the threshold kernel takes as t0 the key that about
+// cand_target(k) of the row's keys reach (the r-th largest of the valid
+// sample keys, r the target scaled by sample size over row length); the
+// candidate pass appends every (key, entry) at or above t0; the select
+// kernel finds the exact top-k among them when there are at least k and at
+// most kCandCap, and otherwise flags the row for the plain path (scores
+// stored, then the streaming top-k).  The output never depends on t0: when
+// at least k keys reach it, every key at or above the k-th largest is a
+// candidate.
+struct SelShared {
+    int hist[kBins];
+    int warp_a[kRWarps];
+    int sel_bin, sel_krem;
+    uint32_t small[32];
+    int small_n;
+    uint32_t small_t;
+};
+
+// Candidates aimed for per row: 3k, at least 2048 and at most half of
+// kCandCap, so that a sample of ~1000 keys rarely lands outside [k, kCandCap].
+__device__ __forceinline__ int cand_target(int k) { return min(kCandCap / 2, max(2048, 3 * k)); }
+
+// Entries of row b: n = L/m, 0 (and the LEN bit) for a bad slot or length.
+__device__ __forceinline__ int cand_row_n(const TopkArgs &a, int b, int slot, bool report) {
+    const bool slot_ok = slot >= 0 && slot < a.n_slots;
+    const int L = slot_ok ? row_visible_len(a.len, a.q_len, slot, b) : 0;
+    if (!slot_ok || L < 0 || L / a.m > a.max_n) {
+        if (report && threadIdx.x == 0) set_dev_err(CSLA_DEVERR_LEN);
+        return 0;
+    }
+    return L / a.m;
+}
+
+__global__ void __launch_bounds__(kRThreads) cand_threshold_kernel(TopkArgs a, CandArgs c) {
+    __shared__ SelShared sh;
+    pdl_trigger();
+    const int b = blockIdx.x;
+    const int slot = __ldg(a.slots + b);
+    pdl_wait();
+    const int n = cand_row_n(a, b, slot, false);
+    uint32_t t0 = 0u;   // rows of at most kCandCap entries: every entry is a candidate
+    if (n > kCandCap && n > a.k) {
+        // sample column 32*j + i holds entry 32*j*Z + i (when below n)
+        const int Z = c.page_step;
+        int ns = 0;
+        for (int j = 0; j < kSampleCols / 32; ++j) ns += max(0, min(32, n - j * Z * 32));
+        const float *sp = c.sample + (size_t)b * kSampleCols;
+        if (ns > 0) {
+            const int r = (int)min((long long)ns, max(1LL, ((long long)cand_target(a.k) * ns + n - 1) / n));
+            int krem;
+            t0 = radix_select(sh, [&](auto fn) {
+                for (int i = threadIdx.x; i < kSampleCols; i += kRThreads)
+                    if ((i / 32) * Z * 32 + (i % 32) < n) fn(score_key(sp[i]));
+            }, r, 0u, 32, &krem);
+        }
+    }
+    if (threadIdx.x == 0) c.cand_t0[b] = t0;
+    if (threadIdx.x < kCandSub) c.cand_cnt[b * kCandSub + threadIdx.x] = 0;
+}
+
+struct CandShared {
+    SelShared s;
+    uint32_t key[kCandCap];
+    int ent[kCandCap];
+    uint32_t wmax[kRWarps];
+    int neq;
+    uint32_t bm[1];   // [bm_words]: bitmap of the picked entries (dynamic size)
+};
+constexpr int kCandFixed = (int)offsetof(CandShared, bm);
+constexpr int kCandBmMax = (232448 - kCandFixed) / 4;   // bitmap words that fit the shared memory
+
+// One CTA per row: the exact top-k among the row's candidates (the keys >
+// T, then of the keys == T those of lowest entry), marked in a bitmap over
+// the row's entries and written in entry order.
+__global__ void __launch_bounds__(kRThreads) cand_select_kernel(TopkArgs a, CandArgs c, int bm_words) {
+    CSLA_TL_SCOPE(kTlTopk);
+    extern __shared__ __align__(16) uint8_t dyn_cs[];
+    CandShared &sh = *reinterpret_cast<CandShared *>(dyn_cs);
+    pdl_trigger();
+    const int b = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int slot = __ldg(a.slots + b);
+    pdl_wait();
+    CSLA_TL_WAITED();
+    const int n = cand_row_n(a, b, slot, true);
+    const int k = a.k;
+    int32_t *out = a.idx + (size_t)b * k;
+    if (n <= k) {
+        for (int j = threadIdx.x; j < k; j += kRThreads) out[j] = j < n ? j : -1;
+        if (threadIdx.x == 0) c.row_flag[b] = 0;
+        return;
+    }
+    // the row's four sub-lists (entries with (entry/32) % 4 = j), each of
+    // at most kCandCap/4, taken one after another
+    constexpr int kSubCap = kCandCap / kCandSub;
+    int sub[kCandSub], cnt = 0;
+    bool fits = true;
+#pragma unroll
+    for (int j = 0; j < kCandSub; ++j) {
+        sub[j] = c.cand_cnt[b * kCandSub + j];
+        fits = fits && sub[j] <= kSubCap;
+        cnt += sub[j];
+    }
+    const int W = (n + 31) / 32;
+    if (cnt < k || !fits || W > bm_words) {
+        if (threadIdx.x == 0) c.row_flag[b] = 1;   // the plain path takes this row
+        return;
+    }
+    if (threadIdx.x == 0) {
+        c.row_flag[b] = 0;
+        sh.neq = 0;
+    }
+    uint32_t mx = 0u;
+    for (int j = 0, at = 0; j < kCandSub; at += sub[j], ++j) {
+        const uint2 *cp = c.cand + ((size_t)b * kCandSub + j) * kSubCap;
+        for (int i = threadIdx.x; i < sub[j]; i += kRThreads) {
+            const uint2 v = cp[i];
+            sh.key[at + i] = v.x;
+            sh.ent[at + i] = (int)v.y;
+            mx = max(mx, v.x);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) sh.wmax[warp] = mx;
+    for (int w = threadIdx.x; w < W; w += kRThreads) sh.bm[w] = 0u;
+    __syncthreads();
+    uint32_t kmax = lane < kRWarps ? sh.wmax[lane] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    // every candidate lies in [t0, kmax]: the digits above their highest
+    // differing bit are already known
+    const uint32_t t0 = c.cand_t0[b];
+    const int bits = (t0 ^ kmax) ? 32 - __clz(t0 ^ kmax) : 0;
+    int krem;
+    const uint32_t T = radix_select(sh.s, [&](auto fn) {
+        for (int i = threadIdx.x; i < cnt; i += kRThreads) fn(sh.key[i]);
+    }, k, kmax, bits, &krem);
+    CSLA_TL_MARK(0);
+    for (int i = threadIdx.x; i < cnt; i += kRThreads) {
+        const uint32_t key = sh.key[i];
+        const int e = sh.ent[i];
+        if (key > T && e < n) atomicOr(&sh.bm[e >> 5], 1u << (e & 31));
+        else if (key == T) atomicAdd(&sh.neq, 1);
+    }
+    __syncthreads();
+    // of the keys == T, the krem of lowest entry: the entries up to the
+    // krem-th smallest (found as the krem-th largest of ~entry)
+    uint32_t emax = 0xFFFFFFFFu;
+    if (sh.neq > krem) {
+        int kr2;
+        emax = ~radix_select(sh.s, [&](auto fn) {
+            for (int i = threadIdx.x; i < cnt; i += kRThreads)
+                if (sh.key[i] == T) fn(~(uint32_t)sh.ent[i]);
+        }, krem, 0u, 32, &kr2);
+    }
+    for (int i = threadIdx.x; i < cnt; i += kRThreads) {
+        const int e = sh.ent[i];
+        if (sh.key[i] == T && (uint32_t)e <= emax && e < n) atomicOr(&sh.bm[e >> 5], 1u << (e & 31));
+    }
+    __syncthreads();
+    // thread t writes the picks of bitmap words [t*per, (t+1)*per), after
+    // those of the threads before it
+    const int per = (W + kRThreads - 1) / kRThreads;
+    const int w0 = min(W, threadIdx.x * per), w1 = min(W, w0 + per);
+    int my = 0;
+    for (int w = w0; w < w1; ++w) my += __popc(sh.bm[w]);
+    int incl = my;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) sh.s.warp_a[warp] = incl;
+    __syncthreads();
+    int total;
+    int pos = warp_prefix(sh.s.warp_a, warp, &total) + incl - my;
+    if (total != k) {   // never for a correct selection
+        if (threadIdx.x == 0) set_dev_err(CSLA_DEVERR_INDEX);
+        return;
+    }
+    for (int w = w0; w < w1; ++w) {
+        uint32_t m = sh.bm[w];
+        while (m) {
+            out[pos++] = 32 * w + (__ffs(m) - 1);
+            m &= m - 1u;
+        }
+    }
+    CSLA_TL_MARK(1);
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
@@ -730,6 +922,29 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
     if (a.max_n <= kRegMax)
         return launch_pdl(topk_cluster_kernel, dim3(a.B * kG), dim3(kRThreads), sizeof(ClShared), stream, a);
     return launch_pdl(topk_stream_kernel, dim3(a.B), dim3(kRThreads), sizeof(RegShared), stream, a);
+}
+
+cudaError_t launch_cand_threshold(const TopkArgs &t, const CandArgs &c, cudaStream_t stream) {
+    return launch_pdl(cand_threshold_kernel, dim3(t.B), dim3(kRThreads), 0, stream, t, c);
+}
+
+cudaError_t launch_cand_select(const TopkArgs &t, const CandArgs &c, cudaStream_t stream) {
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        cudaError_t e = cudaFuncSetAttribute(cand_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kCandFixed + 4 * kCandBmMax);
+        if (e != cudaSuccess) return e;
+        configured_dev = dev;
+    }
+    // a bitmap word per 32 entries of the longest row (rows beyond what
+    // fits take the plain path)
+    long long words = ((long long)t.max_n + 31) / 32;
+    if (words < 1) words = 1;
+    if (words > kCandBmMax) words = kCandBmMax;
+    return launch_pdl(cand_select_kernel, dim3(t.B), dim3(kRThreads), (size_t)kCandFixed + 4 * (size_t)words, stream,
+                      t, c, (int)words);
 }
 
 }  // namespace csla

@@ -106,7 +106,8 @@ enum {
     CSLA_OP_TOPK = 2,
     CSLA_OP_CSA_ATTEND = 3,
     CSLA_OP_HCA_ATTEND = 4,
-    CSLA_OP_CSA_DECODE_STEP = 5 /* ws_step of csla_csa_decode_step; max_len here means k */
+    CSLA_OP_CSA_DECODE_STEP = 5, /* ws_step of csla_csa_decode_step; max_len here means k */
+    CSLA_OP_INDEXER_TOPK = 6     /* csla_indexer_topk */
 };
 
 /* device error word bits */
@@ -293,6 +294,34 @@ int csla_indexer_scores(const csla_cfg *cfg, const csla_state *st, const csla_ca
 int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *slots, int32_t B,
                      const csla_queries *qs, int32_t max_len, const float *scores, int32_t scores_stride, int32_t k,
                      int32_t *idx, csla_stream_t stream);
+
+/*
+ * csla_indexer_topk -- csla_indexer_scores then csla_topk_select in one
+ * call, without storing the scores of rows that are long (硅星人
+ * §两大压缩注意力, CSA part: score every compressed block, keep the k best;
+ * "DeepSeek-V4深度拆解" §2: the prefill's KV-cache traffic).  The result,
+ * idx [B][k], is bit for bit the one of the two calls.  Steps, all on
+ * `stream`: a sample pass scores 32 evenly spaced 32-entry pages of every
+ * row; a threshold t0 per row is taken from the sample so that about 3k of
+ * the row's scores should reach it; a candidate pass scores every entry and
+ * keeps (score, entry) for those >= t0 only; the exact top-k is selected
+ * among the candidates when there are at least k and at most 8192 of them
+ * (every score >= the k-th largest is then a candidate).  A row outside that
+ * range (heavy ties, a sample far from the row's distribution) is scored
+ * again into `scores` and selected there, as by the two calls.  Rows of at
+ * most 8192 entries keep every entry as a candidate.
+ *   Arguments as for csla_indexer_scores and csla_topk_select; `scores`
+ *   [B][scores_stride] f32 is scratch (written only for rows taken by the
+ *   fallback; its contents are unspecified afterwards).  workspace:
+ *   csla_workspace_size(cfg, CSLA_OP_INDEXER_TOPK, B, max_len) bytes,
+ *   16-byte aligned.  Errors: those of the two calls.
+ */
+int csla_indexer_topk(const csla_cfg *cfg, const csla_state *st, const csla_cache *cache,
+                      const int32_t *slots, int32_t B, const csla_queries *qs, int32_t max_len,
+                      const void *cq, int32_t cq_dtype, const void *W_iq, int32_t w_dtype,
+                      const float *head_w, int32_t k, int32_t *idx, float *scores,
+                      int32_t scores_stride, void *workspace, size_t workspace_bytes,
+                      csla_stream_t stream);
 
 /*
  * csla_csa_attend -- core MQA of a CSA layer (硅星人 §两大压缩注意力; haiqwa

@@ -111,6 +111,12 @@ def test_workspace_sizes():
     assert C.csla_workspace_size(_cfg(m=8), C.CSLA_OP_TOPK, 1, 1) == 0
     # decode step: the attention partials for k, then B int32 lengths (16-byte rounded)
     assert C.csla_workspace_size(cfg, C.CSLA_OP_CSA_DECODE_STEP, 8, 512) == 8 * 10 * (64 * 512 + 128) * 4 + 32
+    # indexer + top-k: the indexer's query terms, 1024 sample scores, a
+    # threshold, four counts and a flag per row (int32, each part 16-byte
+    # rounded), 8192 (key, entry) candidates per row
+    assert C.csla_workspace_size(cfg, C.CSLA_OP_INDEXER_TOPK, 8, 131072) == \
+        8 * 48 * 128 * 2 + 8 * 1024 * 4 + 32 + 128 + 32 + 8 * 8192 * 8
+    assert C.csla_workspace_size(_cfg(m=128), C.CSLA_OP_INDEXER_TOPK, 8, 131072) == 0
 
 
 def test_host_checks_of_the_query_row_and_step_calls():
@@ -137,6 +143,15 @@ def test_host_checks_of_the_query_row_and_step_calls():
     tail = [fake, C.CSLA_BF16, fake, fake, fake, C.CSLA_F32, 0, fake, 1 << 20, fake, 1 << 20, None]
     assert L.csla_csa_decode_step(ctypes.byref(_cfg(m=128)), *args, fake, *tail) == C.CSLA_ERR_UNSUPPORTED
     assert L.csla_csa_decode_step(ctypes.byref(cfg), *args, None, *tail) == C.CSLA_ERR_ARG
+    # indexer + top-k: k outside 1..2048, a workspace below its size, no scratch scores
+    itk = [ctypes.byref(cfg), ctypes.byref(st), ctypes.byref(cache), fake, 8, None, 131072, fake, C.CSLA_BF16,
+           fake, C.CSLA_BF16, fake]
+    need = C.csla_workspace_size(cfg, C.CSLA_OP_INDEXER_TOPK, 8, 131072)
+    assert L.csla_indexer_topk(*itk, 0, fake, fake, 32768, fake, need, None) == C.CSLA_ERR_ARG
+    assert L.csla_indexer_topk(*itk, 2049, fake, fake, 32768, fake, need, None) == C.CSLA_ERR_ARG
+    assert L.csla_indexer_topk(*itk, 1024, fake, fake, 32768, fake, need - 1, None) == C.CSLA_ERR_ARG
+    assert L.csla_indexer_topk(*itk, 1024, fake, None, 32768, fake, need, None) == C.CSLA_ERR_ARG
+    assert L.csla_indexer_topk(*itk, 1024, fake, fake, 1000, fake, need, None) == C.CSLA_ERR_ARG
 
 
 def test_cp_record_size_and_host_checks():
