@@ -172,7 +172,8 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream);
 constexpr int kCandCap = 8192;        // candidates kept per row (4 sub-lists of 2048)
 constexpr int kCandSub = 4;
 constexpr int kSampleCols = 1024;     // sample scores per row (32 pages)
-constexpr int kPersistSlices = 4;     // CTAs per row group in the stored-score fallback
+constexpr int kPersistSlices = 2;     // CTAs per row group in the stored-score fallback (few: most
+                                      // groups have no flagged row and exit at once)
 struct CandArgs {
     const float *sample;
     int page_step;
