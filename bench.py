@@ -10,7 +10,7 @@ RoPE dims), dc=1024 -> 16 index heads of 128, top-k 512, window 128.
 An HCA layer (4 requests at 1,048,576 tokens, m'=128) is measured after it
 and reported in the same JSON line under "hca_decode", then a CSA prefill
 chunk (4096 new tokens and their queries after a 262144-token prefix, top-k
-1024) under "csa_prefill".
+1024; indexer and top-k as one csla_indexer_topk call) under "csa_prefill".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
