@@ -101,10 +101,10 @@ def check(w, lb, slots, B, max_len, k, tag, qs=None, zero_weights=False, n_rows=
     g, e = got.cpu().numpy(), want.cpu().numpy()
     for b in range(B):
         assert np.array_equal(g[b], e[b]), (b, int(np.sum(g[b] != e[b])))
-    sc = scores.cpu().numpy()
     for b in oracle_rows:
-        n = n_rows[b]
-        assert np.array_equal(g[b], oracle.topk(sc[b, :n].astype(np.float64), k)), b
+        n = int(n_rows[b])
+        sc = scores[b, :n].cpu().numpy().astype(np.float64)
+        assert np.array_equal(g[b], oracle.topk(sc, k)), b
     return flags
 
 
@@ -170,3 +170,17 @@ def test_ties_on_query_rows_fall_back():
     flags = check(W16, lb, _i32(np.zeros(T)), T, L0 + T, k, "itk_f", qs=C.queries(_i32(q_len), one_request=True),
                   zero_weights=True, n_rows=q_len // 4, oracle_rows=(3,))
     assert list(flags) == [1] * T, flags
+
+
+def test_full_size_prefill_chunk():
+    """The bench's prefill chunk shape: 4096 query rows of one request after
+    a 262144-token prefix (~66 K entries per row), k = 1024, in the launch
+    configuration the bench times (5 rows per key tile, runs of tiles per
+    CTA).  idx equal to the two calls' for every row; a few rows against
+    the oracle's top-k of the stored scores."""
+    L0, T, k = 262144, 4096, 1024
+    lb = random_layer(W16, [L0 + T], "itk_full")
+    q_len = np.arange(L0 + 1, L0 + T + 1)
+    flags = check(W16, lb, _i32(np.zeros(T)), T, L0 + T, k, "itk_full",
+                  qs=C.queries(_i32(q_len), one_request=True), n_rows=q_len // 4, oracle_rows=(0, 1777, T - 1))
+    assert (flags == 0).sum() >= T - 8, int((flags != 0).sum())
