@@ -288,7 +288,8 @@ struct Pending {
 // epilogue warps build before they start (NQ = 4*HI); the epilogue forms
 // each head's dot product from its four terms and applies the entry scale.
 template <int DI, int NQ, int HI, int G, bool kE4M3>
-__global__ void __launch_bounds__(idx_threads<G>())
+// decode rows (G = 1): two CTAs per SM (registers for 2 x 192 threads)
+__global__ void __launch_bounds__(idx_threads<G>(), G == 1 ? 2 : 1)
     indexer_kernel(IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap qmap) {
     CSLA_TL_SCOPE(kTlIndexer);
