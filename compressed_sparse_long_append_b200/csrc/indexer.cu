@@ -287,7 +287,7 @@ struct Pending {
 // kind::f8f6f4 MMAs against the four-term E4M3 query operand that the
 // epilogue warps build before they start (NQ = 4*HI); the epilogue forms
 // each head's dot product from its four terms and applies the entry scale.
-template <int DI, int NQ, int HI, int G, bool kE4M3>
+template <int DI, int NQ, int HI, int G, bool kE4M3, bool kSel>
 // decode rows (G = 1): two CTAs per SM (registers for 2 x 192 threads)
 __global__ void __launch_bounds__(idx_threads<G>(), G == 1 ? 2 : 1)
     indexer_kernel(IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
@@ -316,12 +316,18 @@ __global__ void __launch_bounds__(idx_threads<G>(), G == 1 ? 2 : 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r0 = blockIdx.y * G;
-    if (a.persist && a.row_flag) {
+    // the streaming-selection modes (sample, candidates, row flags) exist in
+    // the kSel instantiations only; runs of tiles also for grouped rows
+    const int persist = (kSel || G > 1) ? a.persist : 0;
+    const int page_step = kSel ? a.page_step : 0;
+    const int32_t *row_flag = kSel ? a.row_flag : nullptr;
+    const uint32_t *cand_t0 = kSel ? a.cand_t0 : nullptr;
+    if (persist && row_flag) {
         // the fallback of a streaming selection: most row groups have no
         // flagged row, so look before taking barriers and TMEM
         pdl_wait();
         int any = 0;
-        if (threadIdx.x < G && r0 + threadIdx.x < a.B) any = a.row_flag[r0 + threadIdx.x] != 0;
+        if (threadIdx.x < G && r0 + threadIdx.x < a.B) any = row_flag[r0 + threadIdx.x] != 0;
         if (!__syncthreads_or(any)) return;
     }
     const int slot = __ldg(a.slots + r0);
@@ -344,11 +350,11 @@ __global__ void __launch_bounds__(idx_threads<G>(), G == 1 ? 2 : 1)
         fence_mbar_init();
     }
     // page j of this CTA (j < 4*kTPC) is page (4*kTPC*x + j)*Z of the request
-    const int Z = a.page_step > 1 ? a.page_step : 1;
+    const int Z = page_step > 1 ? page_step : 1;
     int pg = -1;   // warp 0: page id of this CTA's page `lane`
     if (warp == 0) {
         const int col = (blockIdx.x * kTPC * 4 + lane) * Z;
-        if (!a.persist && a.range != 2 && slot_ok && lane < kTPC * 4 && col < a.bt_stride)
+        if (!persist && a.range != 2 && slot_ok && lane < kTPC * 4 && col < a.bt_stride)
             pg = __ldg(a.block_table + (size_t)slot * a.bt_stride + col);
         if (lane == 0) {
             tma_prefetch_desc(&kmap);
@@ -395,19 +401,19 @@ __global__ void __launch_bounds__(idx_threads<G>(), G == 1 ? 2 : 1)
                         lo = a.len0[r] / a.m;
                         if (lo >= nv) nv = -1;
                     }
-                    if (a.row_flag && a.row_flag[r] == 0) nv = -1;
+                    if (row_flag && row_flag[r] == 0) nv = -1;
                 }
             }
         }
         row_nv[threadIdx.x] = nv;
         row_lo[threadIdx.x] = lo;
-        row_t0[threadIdx.x] = key_score((a.cand_t0 && r < a.B) ? a.cand_t0[r] : 0u);
+        row_t0[threadIdx.x] = key_score((cand_t0 && r < a.B) ? cand_t0[r] : 0u);
         if (threadIdx.x == 0) s_t0 = a.range == 2 ? lo / kTileE : 0;
     }
     __syncthreads();
     // persist: CTA x walks tiles [x*run, (x+1)*run) of the request
-    const int run = a.persist ? (a.tiles_per_req + a.persist - 1) / a.persist : kTPC;
-    const int t_begin = a.persist ? blockIdx.x * run : blockIdx.x * kTPC + s_t0;
+    const int run = persist ? (a.tiles_per_req + persist - 1) / persist : kTPC;
+    const int t_begin = persist ? blockIdx.x * run : blockIdx.x * kTPC + s_t0;
     int nv_max = 0;
 #pragma unroll
     for (int g = 0; g < G; ++g) nv_max = max(nv_max, row_nv[g]);
@@ -419,7 +425,7 @@ __global__ void __launch_bounds__(idx_threads<G>(), G == 1 ? 2 : 1)
         if (slot_ok && lane < kTPC * 4 && col < a.bt_stride)
             pg = __ldg(a.block_table + (size_t)slot * a.bt_stride + col);
     }
-    if (!a.persist && warp == 0 && lane < kTPC * 4) {
+    if (!persist && warp == 0 && lane < kTPC * 4) {
         const int e0 = ((t_begin * 4 + lane) * Z) * kPageE;
         if (e0 < nv_max && (pg < 0 || pg >= a.n_pages)) {
             set_dev_err(CSLA_DEVERR_PAGE);
@@ -433,7 +439,7 @@ __global__ void __launch_bounds__(idx_threads<G>(), G == 1 ? 2 : 1)
     // tiles of a CTA, read from the block table per tile when a CTA walks a
     // longer run (persist: Z = 1).
     auto page_id = [&](int t, int p, bool report) -> int {
-        if (!a.persist) return pages[t * 4 + p];
+        if (!persist) return pages[t * 4 + p];
         const int e0 = (t_begin + t) * kTileE + p * kPageE;
         if (e0 >= nv_max) return -1;
         const int col = e0 / kPageE;
@@ -563,7 +569,7 @@ __global__ void __launch_bounds__(idx_threads<G>(), G == 1 ? 2 : 1)
         // and moves them out once more than 32 are staged, and after its
         // last tile: one counter update per ~32 candidates.  Otherwise each
         // (row, tile) takes its places from one counter update.
-        constexpr bool kStaged = kSets >= G && G > 1;
+        constexpr bool kStaged = kSel && kSets >= G && G > 1;
         uint2 *stage = stage_all + (warp - 2) * kStageCands;
         int staged = 0;
         int stage_row = 0;
@@ -661,7 +667,7 @@ __global__ void __launch_bounds__(idx_threads<G>(), G == 1 ? 2 : 1)
                         }
                     }
                 }
-                if (a.cand_t0) {
+                if (cand_t0) {
                     // the entries at or above the row's threshold (warp-uniform
                     // mask; the float order is the key order, -0 == +0)
                     const bool q = valid && sc >= row_t0[g];
@@ -700,7 +706,7 @@ __global__ void __launch_bounds__(idx_threads<G>(), G == 1 ? 2 : 1)
 }
 
 
-template <int DI, int NQ, int HI, int G, bool kE4M3>
+template <int DI, int NQ, int HI, int G, bool kE4M3, bool kSel>
 cudaError_t launch_indexer_t(const IndexerArgs &a, const CUtensorMap &kmap, const CUtensorMap &qmap,
                              cudaStream_t stream) {
     using S = IdxSmem<DI, NQ, G, kE4M3>;
@@ -709,25 +715,32 @@ cudaError_t launch_indexer_t(const IndexerArgs &a, const CUtensorMap &kmap, cons
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(indexer_kernel<DI, NQ, HI, G, kE4M3>,
+        cudaError_t e = cudaFuncSetAttribute(indexer_kernel<DI, NQ, HI, G, kE4M3, kSel>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
     // tiles a row group walks: all of the request's, or (sample) tiles of 4
     // pages page_step apart; persist: `persist` CTAs per row group
-    const int Z = a.page_step > 1 ? a.page_step : 1;
-    const int groups = a.persist ? a.persist : (((a.tiles_per_req * 4 + Z - 1) / Z + 3) / 4 + kTPC - 1) / kTPC;
-    return launch_pdl(indexer_kernel<DI, NQ, HI, G, kE4M3>, dim3(groups, (a.B + G - 1) / G),
+    const int Z = kSel && a.page_step > 1 ? a.page_step : 1;
+    const int persist = (kSel || G > 1) ? a.persist : 0;   // as the kernel reads it
+    const int groups = persist ? persist : (((a.tiles_per_req * 4 + Z - 1) / Z + 3) / 4 + kTPC - 1) / kTPC;
+    return launch_pdl(indexer_kernel<DI, NQ, HI, G, kE4M3, kSel>, dim3(groups, (a.B + G - 1) / G),
                       dim3(idx_threads<G>()), S::kBytes, stream, a, kmap, qmap);
 }
 
 template <int DI, int NQ, int HI, bool kE4M3>
 cudaError_t launch_indexer_g(const IndexerArgs &a, const CUtensorMap &kmap, const CUtensorMap &qmap,
                              cudaStream_t stream) {
-    if (a.rows_per_cta == 1) return launch_indexer_t<DI, NQ, HI, 1, kE4M3>(a, kmap, qmap, stream);
-    if (a.rows_per_cta == indexer_rows_per_cta(NQ))
-        return launch_indexer_t<DI, NQ, HI, indexer_rows_per_cta(NQ), kE4M3>(a, kmap, qmap, stream);
+    // the plain scoring kernels carry none of the streaming-selection code
+    const bool sel = a.page_step > 1 || a.cand_t0 != nullptr || a.row_flag != nullptr;
+    constexpr int GR = indexer_rows_per_cta(NQ);
+    if (a.rows_per_cta == 1)
+        return sel ? launch_indexer_t<DI, NQ, HI, 1, kE4M3, true>(a, kmap, qmap, stream)
+                   : launch_indexer_t<DI, NQ, HI, 1, kE4M3, false>(a, kmap, qmap, stream);
+    if (a.rows_per_cta == GR)
+        return sel ? launch_indexer_t<DI, NQ, HI, GR, kE4M3, true>(a, kmap, qmap, stream)
+                   : launch_indexer_t<DI, NQ, HI, GR, kE4M3, false>(a, kmap, qmap, stream);
     return cudaErrorInvalidValue;
 }
 
