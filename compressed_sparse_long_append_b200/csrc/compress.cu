@@ -140,36 +140,51 @@ struct BlockRows {
 };
 
 constexpr int kMaxIdxPerThread = 2;   // index-key inputs (dI <= 512) per thread
-constexpr int kChanStateFloats = 12 * kThreads;   // per-channel pooling: (max, sum, acc) float4 per thread
+constexpr int kStageRows = 32;    // block rows staged in shared memory at a time
+
+// Rows c0 .. c0+R-1 of the block into xs[R][width] (shared memory), one
+// float4 per thread and iteration.
+template <typename T>
+__device__ __forceinline__ void stage_rows(const BlockRows<T> &x, int c0, int R, float *xs) {
+    const int nq = x.width >> 2, total = R * nq;
+    for (int idx = threadIdx.x; idx < total; idx += kThreads)
+        reinterpret_cast<float4 *>(xs)[idx] = x.get(c0 + idx / nq, idx % nq);
+}
 
 // Pool the block with softmax weights of the scalar gates g_i = <x_i, w> +
 // bias_i.  On entry alpha[i] = bias_i and wsm = w (smem); the pooled row
-// (width floats) goes to out (smem).  The rows are read straight from the
-// tail (fp32) and the new rows, twice (they are L2-resident; staging them
-// through shared memory 32 rows at a time made every stage a full load
-// round trip).  Gates: one warp per row, lane l sums columns 4(l + 32j) ..
-// +3 in order of j, then a butterfly over the lanes.  Pooled sum: G = 256 /
-// (width / 4) row groups; group g sums rows g, g + G, ... in order, and the
-// groups are added in order.
+// (width floats) goes to out (smem).  The rows pass through shared memory
+// (xs) kStageRows at a time; a block of at most kStageRows rows is staged
+// once for both passes.  Gates: one warp per row, lane l sums columns
+// 4(l + 32j) .. +3 in order of j, then a butterfly over the lanes.  Pooled
+// sum: G = 256 / (width / 4) row groups; group g sums rows g, g + G, ... in
+// order, and the groups are added in order.
 template <typename T>
-__device__ void pool_block(const BlockRows<T> &x, int m, const float *wsm, float *alpha, float *part, float *out,
-                           float *red) {
+__device__ void pool_block(const BlockRows<T> &x, int m, const float *wsm, float *alpha, float *part, float *xs,
+                           float *out, float *red) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int width = x.width, nq = width >> 2;
+    const float4 *xs4 = reinterpret_cast<const float4 *>(xs);
     const float4 *w4 = reinterpret_cast<const float4 *>(wsm);
-    CSLA_TL_MARK(3);
-#pragma unroll 4
-    for (int r = warp; r < m; r += kWarps) {
-        float acc = 0.f;
-        for (int c4 = lane; c4 < nq; c4 += 32) {
-            const float4 xv = x.get(r, c4), wv = w4[c4];
-            acc = __fmaf_rn(xv.x, wv.x, acc);
-            acc = __fmaf_rn(xv.y, wv.y, acc);
-            acc = __fmaf_rn(xv.z, wv.z, acc);
-            acc = __fmaf_rn(xv.w, wv.w, acc);
+    const bool staged_once = m <= kStageRows;
+    for (int c0 = 0; c0 < m; c0 += kStageRows) {
+        const int R = min(kStageRows, m - c0);
+        __syncthreads();   // the previous chunk is consumed
+        stage_rows(x, c0, R, xs);
+        __syncthreads();
+        if (c0 == 0) CSLA_TL_MARK(3);
+        for (int r = warp; r < R; r += kWarps) {
+            float acc = 0.f;
+            for (int c4 = lane; c4 < nq; c4 += 32) {
+                const float4 xv = xs4[r * nq + c4], wv = w4[c4];
+                acc = __fmaf_rn(xv.x, wv.x, acc);
+                acc = __fmaf_rn(xv.y, wv.y, acc);
+                acc = __fmaf_rn(xv.z, wv.z, acc);
+                acc = __fmaf_rn(xv.w, wv.w, acc);
+            }
+            acc = warp_sum(acc);
+            if (lane == 0) alpha[c0 + r] = __fadd_rn(acc, alpha[c0 + r]);
         }
-        acc = warp_sum(acc);
-        if (lane == 0) alpha[r] = __fadd_rn(acc, alpha[r]);
     }
     __syncthreads();
     CSLA_TL_MARK(4);
@@ -189,18 +204,25 @@ __device__ void pool_block(const BlockRows<T> &x, int m, const float *wsm, float
     const int G = kThreads / nq;   // nq <= 128, so G >= 2
     const int g = threadIdx.x / nq, c4 = threadIdx.x % nq;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (g < G) {
-#pragma unroll 8
-        for (int r = g; r < m; r += G) {
-            const float al = alpha[r];
-            const float4 xv = x.get(r, c4);
-            acc.x = __fmaf_rn(al, xv.x, acc.x);
-            acc.y = __fmaf_rn(al, xv.y, acc.y);
-            acc.z = __fmaf_rn(al, xv.z, acc.z);
-            acc.w = __fmaf_rn(al, xv.w, acc.w);
+    for (int c0 = 0; c0 < m; c0 += kStageRows) {
+        const int R = min(kStageRows, m - c0);
+        if (!staged_once) {
+            __syncthreads();
+            stage_rows(x, c0, R, xs);
+            __syncthreads();
         }
-        reinterpret_cast<float4 *>(part)[g * nq + c4] = acc;
+        if (g < G) {
+            for (int r = g; r < R; r += G) {
+                const float al = alpha[c0 + r];
+                const float4 xv = xs4[r * nq + c4];
+                acc.x = __fmaf_rn(al, xv.x, acc.x);
+                acc.y = __fmaf_rn(al, xv.y, acc.y);
+                acc.z = __fmaf_rn(al, xv.z, acc.z);
+                acc.w = __fmaf_rn(al, xv.w, acc.w);
+            }
+        }
     }
+    if (g < G) reinterpret_cast<float4 *>(part)[g * nq + c4] = acc;
     __syncthreads();
     CSLA_TL_MARK(6);
     for (int d = threadIdx.x; d < width; d += kThreads) {
@@ -216,7 +238,7 @@ __device__ void pool_block(const BlockRows<T> &x, int m, const float *wsm, float
 // trip), its partial gate products go through one block reduction (warp
 // butterfly, then the warps in order), every thread forms the softmax
 // weights itself, and its pooled columns (rows in order) go to out (smem).
-// Two barriers instead of the 128-row path's five.
+// Two barriers instead of the staged path's ten.
 constexpr int kSmallM = 4;
 template <typename T>
 __device__ void pool_small(const BlockRows<T> &x, int m, const float *wsm, const float *bias, float *red8,
@@ -381,7 +403,7 @@ __device__ __forceinline__ void pool_any(const BlockRows<T> &x, int m, const flo
     } else if (m <= kSmallM) {
         pool_small<T>(x, m, wsm, alpha, part, out);
     } else {
-        pool_block<T>(x, m, wsm, alpha, part, out, red);
+        pool_block<T>(x, m, wsm, alpha, part, xs, out, red);
     }
 }
 
@@ -400,7 +422,7 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(CompressArgs 
     float *alpha = wsm + W;             // [m]   gate bias, then weights
     float *part = alpha + m;            // [4 * kThreads]
     float *red = part + 4 * kThreads;   // [32]
-    float *xs = red + 32;               // [kChanStateFloats]  per-channel pooling states
+    float *xs = red + 32;               // [min(m, kStageRows)][W]  staged block rows
     __shared__ int s_old_len;
     pdl_trigger();
     const int x = blockIdx.x, b = blockIdx.y, z = blockIdx.z;
@@ -600,13 +622,14 @@ cudaError_t launch_window_rows(const WindowRowsArgs &a, cudaStream_t stream) {
 cudaError_t launch_compress_append(const CompressArgs &a, bool bf16, cudaStream_t stream) {
     const int nb = a.T / a.m + 1;   // blocks one call can complete
     const size_t W = (size_t)(a.D > a.dI ? a.D : a.dI);
-    const size_t smem = (2 * W + (size_t)a.D + (size_t)a.m + 4 * kThreads + 32 + kChanStateFloats) * sizeof(float);
+    const size_t R = (size_t)(a.m < kStageRows ? a.m : kStageRows);
+    const size_t smem = (2 * W + (size_t)a.D + (size_t)a.m + 4 * kThreads + 32 + R * W) * sizeof(float);
     static int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {
         // largest case: W = 512, m = 128
-        const int most = (int)((2 * 512 + 512 + 128 + 4 * kThreads + 32 + kChanStateFloats) * sizeof(float));
+        const int most = (int)((2 * 512 + 512 + 128 + 4 * kThreads + 32 + kStageRows * 512) * sizeof(float));
         cudaError_t e = cudaSuccess;
         for (auto fn : {compress_append_kernel<float, false, false>, compress_append_kernel<float, true, false>,
                         compress_append_kernel<__nv_bfloat16, false, false>,
