@@ -718,7 +718,7 @@ __global__ void __launch_bounds__(kRThreads, 2) topk_stream_kernel(TopkArgs a) {
 // sample keys, r the target scaled by sample size over row length); the
 // candidate pass appends every (key, entry) at or above t0; the select
 // kernel finds the exact top-k among them when there are at least k and at
-// most kCandCap, and otherwise flags the row for the plain path (scores
+// most kSelCap, and otherwise flags the row for the plain path (scores
 // stored, then the streaming top-k).  The output never depends on t0: when
 // at least k keys reach it, every key at or above the k-th largest is a
 // candidate.
@@ -731,8 +731,12 @@ struct SelShared {
     uint32_t small_t;
 };
 
+// Candidates a select CTA holds: 6144 of the kCandCap a row may keep (three
+// CTAs per SM fit; more than 6144 candidates send the row to the fallback).
+constexpr int kSelCap = 6144;
+
 // Candidates aimed for per row: 3k, at least 2048 and at most half of
-// kCandCap, so that a sample of ~1000 keys rarely lands outside [k, kCandCap].
+// kCandCap, so that a sample of ~1000 keys rarely lands outside [k, kSelCap].
 __device__ __forceinline__ int cand_target(int k) { return min(kCandCap / 2, max(2048, 3 * k)); }
 
 // Entries of row b: n = L/m, 0 (and the LEN bit) for a bad slot or length.
@@ -753,8 +757,8 @@ __global__ void __launch_bounds__(kRThreads) cand_threshold_kernel(TopkArgs a, C
     const int slot = __ldg(a.slots + b);
     pdl_wait();
     const int n = cand_row_n(a, b, slot, false);
-    uint32_t t0 = 0u;   // rows of at most kCandCap entries: every entry is a candidate
-    if (n > kCandCap && n > a.k) {
+    uint32_t t0 = 0u;   // rows of at most kSelCap entries: every entry is a candidate
+    if (n > kSelCap && n > a.k) {
         // sample column 32*j + i holds entry 32*j*Z + i (when below n)
         const int Z = c.page_step;
         int ns = 0;
@@ -775,8 +779,8 @@ __global__ void __launch_bounds__(kRThreads) cand_threshold_kernel(TopkArgs a, C
 
 struct CandShared {
     SelShared s;
-    uint32_t key[kCandCap];
-    int ent[kCandCap];
+    uint32_t key[kSelCap];
+    int ent[kSelCap];
     uint32_t wmax[kRWarps];
     int neq;
     uint32_t bm[1];   // [bm_words]: bitmap of the picked entries (dynamic size)
@@ -817,7 +821,7 @@ __global__ void __launch_bounds__(kRThreads) cand_select_kernel(TopkArgs a, Cand
         cnt += sub[j];
     }
     const int W = (n + 31) / 32;
-    if (cnt < k || !fits || W > bm_words) {
+    if (cnt < k || cnt > kSelCap || !fits || W > bm_words) {
         if (threadIdx.x == 0) c.row_flag[b] = 1;   // the plain path takes this row
         return;
     }

@@ -305,11 +305,11 @@ int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *s
  * row; a threshold t0 per row is taken from the sample so that about 3k of
  * the row's scores should reach it; a candidate pass scores every entry and
  * keeps (score, entry) for those >= t0 only; the exact top-k is selected
- * among the candidates when there are at least k and at most 8192 of them
+ * among the candidates when there are at least k and at most 6144 of them
  * (every score >= the k-th largest is then a candidate).  A row outside that
  * range (heavy ties, a sample far from the row's distribution) is scored
  * again into `scores` and selected there, as by the two calls.  Rows of at
- * most 8192 entries keep every entry as a candidate.
+ * most 6144 entries keep every entry as a candidate.
  *   Arguments as for csla_indexer_scores and csla_topk_select; `scores`
  *   [B][scores_stride] f32 is scratch (written only for rows taken by the
  *   fallback; its contents are unspecified afterwards).  workspace:

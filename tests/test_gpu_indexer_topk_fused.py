@@ -5,7 +5,7 @@ by csla_topk_select on the same inputs: idx equal, element for element.
 The index keys are seeded random values written straight into a scattered
 page pool (no compressor run): the selection is what is compared.  The cases
 reach every path of the fused call: rows of at most k entries, rows of at
-most 8192 entries (every entry a candidate), long rows through the sample
+most 6144 entries (every entry a candidate), long rows through the sample
 threshold, and rows that fall back to the stored-score path (all scores
 equal: more candidates than the call keeps), with bf16 and E4M3 keys, query
 rows of one request (several rows per key tile) and decode rows of several
@@ -29,7 +29,7 @@ pytestmark = pytest.mark.gpu
 
 W16 = dataclasses.replace(CSA_PREFILL, name="itk_bf16")
 W8 = dataclasses.replace(CSA_PREFILL, key_fmt=C.CSLA_KEY_E4M3, name="itk_e4m3")
-CAND_CAP, SAMPLE_COLS = 8192, 1024
+SAMPLE_COLS = 1024
 
 
 def _i32(x):
@@ -139,7 +139,7 @@ def test_e4m3_keys_query_rows():
 
 
 def test_decode_rows_of_several_requests():
-    """One row per request: no entries, k < n <= 8192 (every entry a
+    """One row per request: no entries, k < n <= 6144 (every entry a
     candidate), and long rows (sample threshold)."""
     lens = [3, 5000, 40000, 100000, 33000, 64004]
     lb = random_layer(W16, lens, "itk_d")
@@ -151,7 +151,7 @@ def test_decode_rows_of_several_requests():
 
 @pytest.mark.parametrize("w", [W16, W8])
 def test_ties_fall_back_or_break_by_entry(w):
-    """Every score 0.  Rows of more than 8192 entries keep too many
+    """Every score 0.  Rows of more than 6144 entries keep too many
     candidates and take the stored-score path (a few CTAs per row group,
     each walking a run of tiles); rows of fewer keep them all and break the
     tie by entry."""
