@@ -22,7 +22,7 @@ from compressed_sparse_long_append_b200 import csla as C
 from compressed_sparse_long_append_b200.layer import LayerBuffers
 from csla_synth import torch_gen as TG
 from csla_synth.workloads import CSA_PREFILL, layer_params
-from gpu_helpers import DEV, act_tensor, assert_no_device_error, shape_of
+from gpu_helpers import DEV, act_tensor, assert_no_device_error, cache_view, check_scores, shape_of
 from helpers import block_table
 
 pytestmark = pytest.mark.gpu
@@ -92,7 +92,10 @@ def fused(w, lb, slots, B, max_len, cq, W, hw, k, qs):
     return idx, flags
 
 
-def check(w, lb, slots, B, max_len, k, tag, qs=None, zero_weights=False, n_rows=None, oracle_rows=()):
+def check(w, lb, slots, B, max_len, k, tag, qs=None, zero_weights=False, n_rows=None, oracle_rows=(),
+          score_rows=()):
+    """score_rows: rows whose stored scores (the two-call path's) are also
+    checked against the oracle's index scores (one request in slot 0)."""
     cq, W, hw = inputs(w, B, tag, zero_weights)
     want, scores = two_calls(w, lb, slots, B, max_len, cq, W, hw, k, qs)
     got, flags = fused(w, lb, slots, B, max_len, cq, W, hw, k, qs)
@@ -105,6 +108,13 @@ def check(w, lb, slots, B, max_len, k, tag, qs=None, zero_weights=False, n_rows=
         n = int(n_rows[b])
         sc = scores[b, :n].cpu().numpy().astype(np.float64)
         assert np.array_equal(g[b], oracle.topk(sc, k)), b
+    if score_rows:
+        keys = cache_view(w, lb).gather_keys(0, int(max(n_rows[b] for b in score_rows)))
+        cqh, Wh, hwh = (t.to(torch.float64).cpu().numpy() for t in (cq, W, hw))
+        for b in score_rows:
+            n = int(n_rows[b])
+            qI = oracle.index_query(cqh[b], Wh, w.HI, w.dI)
+            check_scores(scores[b, :n].cpu().numpy().astype(np.float64), oracle.index_scores(qI, hwh[b], keys[:n]))
     return flags
 
 
@@ -184,3 +194,22 @@ def test_full_size_prefill_chunk():
     flags = check(W16, lb, _i32(np.zeros(T)), T, L0 + T, k, "itk_full",
                   qs=C.queries(_i32(q_len), one_request=True), n_rows=q_len // 4, oracle_rows=(0, 1777, T - 1))
     assert (flags == 0).sum() >= T - 8, int((flags != 0).sum())
+
+
+@pytest.mark.parametrize("HI,dI,zero", [(4, 64, False), (8, 128, False), (4, 64, True)])
+def test_query_rows_with_several_rows_per_epilogue_set(HI, dI, zero):
+    """Fewer index heads: 16 (HI = 4) or 8 (HI = 8) query rows share a key
+    tile and each epilogue warp set scores several of them, so the
+    candidates take their places per (row, tile) from the row counters
+    instead of a shared-memory stage; with zero head weights every row
+    falls back to stored scores."""
+    w = dataclasses.replace(W16, HI=HI, dI=dI, dc=256, name="itk_h%d" % HI)
+    L0, T, k = 50000, 37, 512
+    lb = random_layer(w, [L0 + T], "itk_g%d" % HI)
+    q_len = np.arange(L0 + 1, L0 + T + 1)
+    flags = check(w, lb, _i32(np.zeros(T)), T, L0 + T, k, "itk_g%d" % HI, qs=C.queries(_i32(q_len), one_request=True),
+                  zero_weights=zero, n_rows=q_len // 4, oracle_rows=(0, T - 1), score_rows=(0, 17, T - 1))
+    if zero:
+        assert list(flags) == [1] * T, flags
+    else:
+        assert (flags == 0).sum() >= T - 1, flags
