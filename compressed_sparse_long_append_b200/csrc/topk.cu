@@ -750,10 +750,17 @@ __device__ __forceinline__ int cand_row_n(const TopkArgs &a, int b, int slot, bo
     return L / a.m;
 }
 
-__global__ void __launch_bounds__(kRThreads) cand_threshold_kernel(TopkArgs a, CandArgs c) {
-    __shared__ SelShared sh;
+// One warp per row: the r-th largest valid sample key, exactly, by a radix
+// select over 8-bit digits (a 256-bin histogram per warp in shared memory,
+// four passes).  Lane l holds sample column 32j + l (page j, entry l of the
+// page) for every j.
+constexpr int kThrWarps = 8;
+__global__ void __launch_bounds__(32 * kThrWarps) cand_threshold_kernel(TopkArgs a, CandArgs c) {
+    __shared__ int hist_all[kThrWarps][256];
     pdl_trigger();
-    const int b = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.x * kThrWarps + warp;
+    if (b >= a.B) return;   // warp-uniform; the warps never wait on one another
     const int slot = __ldg(a.slots + b);
     pdl_wait();
     const int n = cand_row_n(a, b, slot, false);
@@ -761,20 +768,64 @@ __global__ void __launch_bounds__(kRThreads) cand_threshold_kernel(TopkArgs a, C
     if (n > kSelCap && n > a.k) {
         // sample column 32*j + i holds entry 32*j*Z + i (when below n)
         const int Z = c.page_step;
-        int ns = 0;
-        for (int j = 0; j < kSampleCols / 32; ++j) ns += max(0, min(32, n - j * Z * 32));
         const float *sp = c.sample + (size_t)b * kSampleCols;
+        uint32_t key[kSampleCols / 32];
+        int ns = 0;
+#pragma unroll
+        for (int j = 0; j < kSampleCols / 32; ++j) {
+            key[j] = j * Z * 32 + lane < n ? score_key(sp[32 * j + lane]) : 0u;
+            ns += max(0, min(32, n - j * Z * 32));
+        }
         if (ns > 0) {
-            const int r = (int)min((long long)ns, max(1LL, ((long long)cand_target(a.k) * ns + n - 1) / n));
-            int krem;
-            t0 = radix_select(sh, [&](auto fn) {
-                for (int i = threadIdx.x; i < kSampleCols; i += kRThreads)
-                    if ((i / 32) * Z * 32 + (i % 32) < n) fn(score_key(sp[i]));
-            }, r, 0u, 32, &krem);
+            int r = (int)min((long long)ns, max(1LL, ((long long)cand_target(a.k) * ns + n - 1) / n));
+            int *hist = hist_all[warp];
+            uint32_t prefix = 0u, pmask = 0u;
+            for (int shift = 24; shift >= 0; shift -= 8) {
+                for (int i = lane; i < 256; i += 32) hist[i] = 0;
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < kSampleCols / 32; ++j)
+                    if (key[j] != 0u && (key[j] & pmask) == prefix) atomicAdd(&hist[(key[j] >> shift) & 255u], 1);
+                __syncwarp();
+                // lane l counts bins 255 - 8l .. 248 - 8l (from the top)
+                int cnt[8], sum = 0;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    cnt[q] = hist[255 - 8 * lane - q];
+                    sum += cnt[q];
+                }
+                int incl = sum;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                const int excl = incl - sum;
+                const bool mine = excl < r && r <= incl;
+                const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+                int sel = 0, rem = 0;
+                if (mine) {
+                    int run = excl;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        if (sel == 0 && rem == 0 && run + cnt[q] >= r) {
+                            sel = 255 - 8 * lane - q;
+                            rem = r - run;
+                        }
+                        run += cnt[q];
+                    }
+                }
+                sel = __shfl_sync(0xffffffffu, sel, src);
+                r = __shfl_sync(0xffffffffu, rem, src);
+                prefix |= (uint32_t)sel << shift;
+                pmask |= 0xFFu << shift;
+                __syncwarp();
+            }
+            t0 = prefix;
         }
     }
-    if (threadIdx.x == 0) c.cand_t0[b] = t0;
-    if (threadIdx.x < kCandSub) c.cand_cnt[b * kCandSub + threadIdx.x] = 0;
+    if (lane == 0) c.cand_t0[b] = t0;
+    if (lane < kCandSub) c.cand_cnt[b * kCandSub + lane] = 0;
 }
 
 struct CandShared {
@@ -929,7 +980,8 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
 }
 
 cudaError_t launch_cand_threshold(const TopkArgs &t, const CandArgs &c, cudaStream_t stream) {
-    return launch_pdl(cand_threshold_kernel, dim3(t.B), dim3(kRThreads), 0, stream, t, c);
+    return launch_pdl(cand_threshold_kernel, dim3((t.B + kThrWarps - 1) / kThrWarps), dim3(32 * kThrWarps), 0,
+                      stream, t, c);
 }
 
 cudaError_t launch_cand_select(const TopkArgs &t, const CandArgs &c, cudaStream_t stream) {
