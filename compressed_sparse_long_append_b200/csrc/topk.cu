@@ -518,18 +518,13 @@ __global__ void __cluster_dims__(kG, 1, 1) __launch_bounds__(kRThreads, 1) topk_
 //     keys > T and the lowest-index keys == T, ascending.
 constexpr int kSBatch = 8;   // score loads a lane keeps in flight in the sweep
 
-__global__ void __launch_bounds__(kRThreads, 2) topk_stream_kernel(TopkArgs a) {
-    CSLA_TL_SCOPE(kTlTopk);
-    extern __shared__ __align__(16) uint8_t dyn_st[];
-    RegShared &sh = *reinterpret_cast<RegShared *>(dyn_st);
-    pdl_trigger();
-    const int b = blockIdx.x;
+// Row b of the streaming top-k: every thread of the CTA runs it, and every
+// barrier inside is taken by all of them or by none.
+__device__ void stream_row(const TopkArgs &a, RegShared &sh, int b) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const unsigned below = (1u << lane) - 1u;
     const int slot = __ldg(a.slots + b);
     const bool slot_ok = slot >= 0 && slot < a.n_slots;
-    pdl_wait();
-    CSLA_TL_WAITED();
     const int L = slot_ok ? row_visible_len(a.len, a.q_len, slot, b) : 0;
     int n = L < 0 ? 0 : L / a.m;
     if (!slot_ok || L < 0 || L / a.m > a.max_n) {
@@ -538,7 +533,6 @@ __global__ void __launch_bounds__(kRThreads, 2) topk_stream_kernel(TopkArgs a) {
     }
     const int k = a.k;
     int32_t *out = a.idx + (size_t)b * k;
-    if (a.row_flag && a.row_flag[b] == 0) return;
     if (n <= k) {
         for (int j = threadIdx.x; j < k; j += kRThreads) out[j] = j < n ? j : -1;
         return;
@@ -708,6 +702,23 @@ __global__ void __launch_bounds__(kRThreads, 2) topk_stream_kernel(TopkArgs a) {
         eq_seen += __popc(meq);
     }
     CSLA_TL_MARK(4);
+}
+
+// One row per CTA; with row flags (the fallback of the fused indexer +
+// top-k: most rows unflagged) a grid of two CTAs per SM walks the rows and
+// skips the unflagged ones.
+__global__ void __launch_bounds__(kRThreads, 2) topk_stream_kernel(TopkArgs a) {
+    CSLA_TL_SCOPE(kTlTopk);
+    extern __shared__ __align__(16) uint8_t dyn_st[];
+    RegShared &sh = *reinterpret_cast<RegShared *>(dyn_st);
+    pdl_trigger();
+    pdl_wait();
+    CSLA_TL_WAITED();
+    for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
+        if (a.row_flag && a.row_flag[b] == 0) continue;   // the same for every thread
+        stream_row(a, sh, b);
+        __syncthreads();   // the next row reuses the shared memory
+    }
 }
 
 // ---------------------------------------------------------------- streaming selection (csla_indexer_topk)
@@ -976,7 +987,13 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
     }
     if (a.max_n <= kRegMax)
         return launch_pdl(topk_cluster_kernel, dim3(a.B * kG), dim3(kRThreads), sizeof(ClShared), stream, a);
-    return launch_pdl(topk_stream_kernel, dim3(a.B), dim3(kRThreads), sizeof(RegShared), stream, a);
+    int grid = a.B;
+    if (a.row_flag) {
+        int sms = 148;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (grid > 2 * sms) grid = 2 * sms;
+    }
+    return launch_pdl(topk_stream_kernel, dim3(grid), dim3(kRThreads), sizeof(RegShared), stream, a);
 }
 
 cudaError_t launch_cand_threshold(const TopkArgs &t, const CandArgs &c, cudaStream_t stream) {

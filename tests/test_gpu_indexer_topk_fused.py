@@ -213,3 +213,15 @@ def test_query_rows_with_several_rows_per_epilogue_set(HI, dI, zero):
         assert list(flags) == [1] * T, flags
     else:
         assert (flags == 0).sum() >= T - 1, flags
+
+
+def test_fallback_through_the_streaming_top_k():
+    """Rows longer than the cluster top-k holds (> 36864 entries) that fall
+    back: the stored-score top-k is the streaming kernel, which skips the
+    rows that were not flagged (the short row here)."""
+    lens = [160000, 3000, 150001]
+    lb = random_layer(W16, lens, "itk_s")
+    B = len(lens)
+    flags = check(W16, lb, torch.arange(B, dtype=torch.int32, device=DEV), B, max(lens), 1024, "itk_s",
+                  zero_weights=True, n_rows=[L // 4 for L in lens], oracle_rows=(0, 2))
+    assert list(flags) == [1, 0, 1], flags
