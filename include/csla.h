@@ -302,15 +302,18 @@ int csla_topk_select(const csla_cfg *cfg, const csla_state *st, const int32_t *s
  * "DeepSeek-V4深度拆解" §2: the prefill's KV-cache traffic).  The result,
  * idx [B][k], is bit for bit the one of the two calls.  Steps, all on
  * `stream`: a sample pass scores 32 evenly spaced 32-entry pages of every
- * row; a threshold t0 per row is taken from the sample so that about 3k of
- * the row's scores should reach it; a candidate pass scores every entry and
+ * row; a threshold t0 per row is taken from the sample so that about
+ * min(4096, max(2048, 3k)) of the row's scores should reach it (the r-th
+ * largest sample score, r scaled from the row to the sample); a candidate
+ * pass scores every entry and
  * keeps (score, entry) for those >= t0 only; the exact top-k is selected
  * among the candidates when there are at least k and at most 6144 of them
  * (every score >= the k-th largest is then a candidate).  A row outside that
  * range (heavy ties, a sample far from the row's distribution) is scored
  * again into `scores` and selected there, as by the two calls.  Rows of at
  * most 6144 entries keep every entry as a candidate.
- *   Arguments as for csla_indexer_scores and csla_topk_select; `scores`
+ *   Arguments as for csla_indexer_scores and csla_topk_select (device
+ *   pointers owned by the caller; the call keeps none of them); `scores`
  *   [B][scores_stride] f32 is scratch (written only for rows taken by the
  *   fallback; its contents are unspecified afterwards).  workspace:
  *   csla_workspace_size(cfg, CSLA_OP_INDEXER_TOPK, B, max_len) bytes,
