@@ -225,3 +225,26 @@ def test_fallback_through_the_streaming_top_k():
     flags = check(W16, lb, torch.arange(B, dtype=torch.int32, device=DEV), B, max(lens), 1024, "itk_s",
                   zero_weights=True, n_rows=[L // 4 for L in lens], oracle_rows=(0, 2))
     assert list(flags) == [1, 0, 1], flags
+
+
+def test_scores_rising_with_position():
+    """Keys scaled up with their entry index, so that the top-k crowd into
+    the last part of every row: the candidates come from a few tiles (the
+    warps there stage and move out many of them), the sample still sees
+    the whole row."""
+    L0, T, k = 120000, 13, 1024
+    lens = [L0 + T]
+    lb = random_layer(W16, lens, "itk_p")
+    bt = lb.block_table.cpu().numpy()[0]
+    n = (L0 + T) // 4
+    scale = torch.ones((lb.n_pages, 32), dtype=torch.float64)
+    for c, pg in enumerate(bt):
+        if pg >= 0:
+            e = 32 * c + torch.arange(32, dtype=torch.float64)
+            scale[int(pg)] = 1.0 + 3.0 * (e / n) ** 4
+    keys = lb.kidx.view(torch.bfloat16).to(torch.float64) * scale.to(DEV)[:, :, None]
+    lb.kidx.copy_(keys.to(torch.bfloat16).view(torch.int16))
+    q_len = np.arange(L0 + 1, L0 + T + 1)
+    flags = check(W16, lb, _i32(np.zeros(T)), T, L0 + T, k, "itk_p", qs=C.queries(_i32(q_len), one_request=True),
+                  n_rows=q_len // 4, oracle_rows=(0, T - 1))
+    assert (flags == 0).sum() >= T - 1, flags
