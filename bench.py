@@ -283,9 +283,9 @@ def csa_launches(kw, variant, fused):
 def attend_launches(rows, B, variant):
     """Attention kernels of one call over `rows` rows per request: the
     attention, plus the combine unless the saturated variant runs."""
-    chunk = 64 * max(-(-rows // 2048), 2 if rows > 1024 else 1)
-    chunks = -(-rows // chunk)
-    saturated = variant == 1 or (variant == 0 and (B >= 148 or chunks <= 1))
+    # the library's bound on a call's chunk count (the starved grid's width)
+    max_chunks = min(32, max(1, -(-rows // 64)))
+    saturated = variant == 1 or (variant == 0 and (B >= 148 or max_chunks <= 1))
     return 1 + (0 if saturated else 1)
 
 
