@@ -371,11 +371,9 @@ class PrefillStep:
         sample scores, thresholds, four counts per row, flags)."""
         import numpy as np
         import torch
-        up16 = lambda x: (x + 15) // 16 * 16
         T, kw = self.T, self.kw
-        nq = (3 * kw["HI"] + 15) // 16 * 16
-        o_cnt = up16(T * nq * kw["dI"] * 2) + up16(T * 1024 * 4) + up16(T * 4)
-        o_flag = o_cnt + up16(T * 16)
+        lay = self.C.indexer_topk_layout(T, kw["HI"], kw["dI"])
+        o_cnt, o_flag = lay["counts"], lay["flags"]
         cnt = self.ws_i[o_cnt:o_cnt + 16 * T].view(torch.int32).cpu().numpy().reshape(T, 4).sum(axis=1)
         flag = self.ws_i[o_flag:o_flag + 4 * T].view(torch.int32).cpu().numpy()
         ok = flag == 0

@@ -227,6 +227,24 @@ def csla_workspace_size(cfg, op, B, max_len):
     return int(_lib.csla_workspace_size(_ref(cfg), op, B, max_len))
 
 
+def indexer_topk_layout(B, HI, dI):
+    """Byte offsets of the parts of a csla_indexer_topk workspace, for
+    reading its per-row diagnostics after a call: query terms, sample
+    scores [B][1024] f32, thresholds [B], candidate counts [B][4] and row
+    flags [B] (int32; 1 = the row took the stored-score path), candidates
+    [B][4][2048] (key, entry); each part 16-byte aligned.  "total" equals
+    csla_workspace_size(cfg, CSLA_OP_INDEXER_TOPK, B, .)."""
+    up16 = lambda x: (x + 15) // 16 * 16
+    nq = (3 * HI + 15) // 16 * 16
+    lay = {"sample": up16(B * nq * dI * 2)}
+    lay["t0"] = lay["sample"] + up16(B * 1024 * 4)
+    lay["counts"] = lay["t0"] + up16(B * 4)
+    lay["flags"] = lay["counts"] + up16(B * 16)
+    lay["cand"] = lay["flags"] + up16(B * 4)
+    lay["total"] = lay["cand"] + B * 8192 * 8
+    return lay
+
+
 def csla_device_error(stream=None):
     """Synchronise the stream; return (status, bits) of the device error word (cleared)."""
     bits = ctypes.c_uint32(0)

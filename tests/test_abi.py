@@ -117,6 +117,11 @@ def test_workspace_sizes():
     assert C.csla_workspace_size(cfg, C.CSLA_OP_INDEXER_TOPK, 8, 131072) == \
         8 * 48 * 128 * 2 + 8 * 1024 * 4 + 32 + 128 + 32 + 8 * 8192 * 8
     assert C.csla_workspace_size(_cfg(m=128), C.CSLA_OP_INDEXER_TOPK, 8, 131072) == 0
+    # the binding's view of its parts agrees with the library's size
+    for B, HI, dI in ((8, 16, 128), (37, 4, 64), (4096, 8, 128)):
+        lay = C.indexer_topk_layout(B, HI, dI)
+        assert lay["total"] == C.csla_workspace_size(_cfg(m=4, HI=HI, dI=dI), C.CSLA_OP_INDEXER_TOPK, B, 1 << 18)
+        assert all(lay[k] % 16 == 0 for k in ("sample", "t0", "counts", "flags", "cand"))
 
 
 def test_host_checks_of_the_query_row_and_step_calls():

@@ -29,7 +29,6 @@ pytestmark = pytest.mark.gpu
 
 W16 = dataclasses.replace(CSA_PREFILL, name="itk_bf16")
 W8 = dataclasses.replace(CSA_PREFILL, key_fmt=C.CSLA_KEY_E4M3, name="itk_e4m3")
-SAMPLE_COLS = 1024
 
 
 def _i32(x):
@@ -85,9 +84,7 @@ def fused(w, lb, slots, B, max_len, cq, W, hw, k, qs):
     idx = torch.full((B, k), -7, dtype=torch.int32, device=DEV)
     C.csla_indexer_topk(lb.cfg(), lb.state(), lb.cache(), slots, B, max_len, cq, C.CSLA_BF16, W, C.CSLA_BF16, hw,
                         k, idx, scores, stride, ws, wsb, qs=qs)
-    up16 = lambda x: (x + 15) // 16 * 16
-    nq = (3 * w.HI + 15) // 16 * 16
-    off = up16(B * nq * w.dI * 2) + up16(B * SAMPLE_COLS * 4) + up16(B * 4) + up16(B * 16)
+    off = C.indexer_topk_layout(B, w.HI, w.dI)["flags"]
     flags = ws[off:off + 4 * B].view(torch.int32).cpu().numpy()
     return idx, flags
 
