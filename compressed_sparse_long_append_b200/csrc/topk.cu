@@ -1,4 +1,6 @@
-// topk.cu -- top-k selector (csla_topk_select).
+// topk.cu -- top-k selector (csla_topk_select) and the selection side of
+// csla_indexer_topk (thresholds from a score sample, select among the
+// candidates the indexer kept).
 //
 //   硅星人 "DeepSeek V4 ... 让token大降价" §两大压缩注意力, CSA part: of all
 //   compressed blocks only the k most relevant (512; 1024 for Pro) are kept.
@@ -13,6 +15,8 @@
 // entries: decode), and one CTA per row streaming its scores (longer rows:
 // query rows of a long prefill).  Both find T among the candidates above a
 // sampled threshold, with a radix select over every key as the fallback.
+// The fused call's select kernel applies the same rule to candidates that
+// arrive in any order (the picks are marked in a bitmap over the entries).
 
 #include <cooperative_groups.h>
 #include <cstddef>
