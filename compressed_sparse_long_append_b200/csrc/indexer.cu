@@ -20,6 +20,13 @@
 //     accumulator (one entry per thread) and reduce
 //       score = sum_j w_j * relu((acc[j] + acc[HI + j]) + acc[2HI + j])
 //     in head order.  Every score depends only on its own entry and request.
+//     Query rows of one request: G rows share each key tile, and a few CTAs
+//     per row group each walk a run of tiles (page ids read per tile).
+//     For csla_indexer_topk (separate instantiations): a sample mode (32
+//     spread pages per row, scores into a small buffer), a candidate mode
+//     (only the entries at or above a per-row threshold leave the kernel,
+//     as (key, entry) pairs) and a row-flag mode for the rows that fall
+//     back to stored scores.
 #include "common.cuh"
 #include "kernels.h"
 
